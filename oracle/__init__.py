@@ -1,0 +1,169 @@
+"""Float64 CPU oracle for the Gated DeltaNet-2 recurrence.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. It shares no code
+with the CUDA library (``delta_rule_linear_gdn_b200``) and neither imports the
+other.
+
+Functions and the passages they follow:
+
+* :func:`gdn2_forward` -- the token-by-token recurrence of
+  "Resumo Técnico: Gated DeltaNet-2", Metodologia §1 "Regra Delta Portão-2":
+  ``S_t = (I - k_t (b_t ⊙ k_t)^T) Diag(α_t) S_{t-1} + k_t (w_t ⊙ v_t)^T``,
+  read after the write as ``o_t = s · S_t^T q_t`` (C++ loop in
+  ``gdn2_oracle.cpp``).
+* :func:`expand_tied_gates` -- the reductions of the same section: tying
+  ``b_t`` and ``w_t`` to one scalar ``β_t`` gives KDA; tying ``α_t`` to a
+  scalar as well gives Gated DeltaNet.
+* :func:`causal_conv4` -- depthwise causal convolution with kernel 4
+  ("Gated DeltaNet: o mixer em 48 das 64 camadas", Conceito).
+* :func:`l2norm` -- row-wise L2 normalisation of queries and keys (the pages
+  assume normalised keys: "Uma análise das variantes de atenção linear da
+  família DeltaNet", Notação e ordem da derivação).
+* :func:`preprocess` -- conv then L2 norm, in that order.
+
+Pins: every function above is checked in ``tests/test_oracle_pins.py`` against
+closed forms, special cases and brute force (no function is parity-unpinned).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn2_oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+L2NORM_EPS = 1e-6
+
+
+def build(force: bool = False) -> str:
+    """Compile the C++ oracle with g++ (plain -O2, IEEE double)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", _SRC, "-o", _LIB_PATH]
+        subprocess.run(cmd, check=True)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_gdn2_forward.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [dp] * 9 + [ctypes.c_int]
+        lib.oracle_gdn2_forward.restype = ctypes.c_int
+        lib.oracle_causal_conv4.argtypes = [ctypes.c_int] * 3 + [dp] * 3
+        lib.oracle_causal_conv4.restype = ctypes.c_int
+        lib.oracle_l2norm.argtypes = [ctypes.c_longlong, ctypes.c_int, ctypes.c_double, dp, dp]
+        lib.oracle_l2norm.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def gdn2_forward(q, k, v, alpha, b, w, S0=None, scale: float = 1.0, threads: int = 0):
+    """Run the recurrence. Shapes: q,k [B,T,Hqk,dk]; v [B,T,Hv,dv];
+    alpha,b [B,T,Hv,dk]; w [B,T,Hv,dv]; S0 [B,Hv,dk,dv] or None.
+    Returns (o [B,T,Hv,dv], S_T [B,Hv,dk,dv]) in float64."""
+    q, k, v, alpha, b, w = (_f64(x) for x in (q, k, v, alpha, b, w))
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    assert k.shape == q.shape and v.shape[:2] == (B, T)
+    assert alpha.shape == (B, T, Hv, dk) and b.shape == (B, T, Hv, dk) and w.shape == (B, T, Hv, dv)
+    if S0 is not None:
+        S0 = _f64(S0)
+        assert S0.shape == (B, Hv, dk, dv)
+    o = np.zeros((B, T, Hv, dv), dtype=np.float64)
+    ST = np.zeros((B, Hv, dk, dv), dtype=np.float64)
+    rc = _load().oracle_gdn2_forward(B, T, Hqk, Hv, dk, dv, float(scale), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o), _ptr(ST),
+                                     int(threads))
+    if rc != 0:
+        raise ValueError("oracle_gdn2_forward rejected its arguments")
+    return o, ST
+
+
+def expand_tied_gates(mode: str, alpha, beta, d_k: int, d_v: int):
+    """Per-channel gates of a tied variant.
+
+    mode "kda": alpha [...,dk] per channel, beta [...] scalar -> b = beta·1_dk, w = beta·1_dv.
+    mode "gdn": alpha [...] scalar and beta [...] scalar -> alpha·1_dk as well.
+    Returns (alpha [..., dk], b [..., dk], w [..., dv]) in float64.
+    """
+    beta = _f64(beta)
+    b = np.repeat(beta[..., None], d_k, axis=-1)
+    w = np.repeat(beta[..., None], d_v, axis=-1)
+    alpha = _f64(alpha)
+    if mode == "gdn":
+        alpha = np.repeat(alpha[..., None], d_k, axis=-1)
+    elif mode != "kda":
+        raise ValueError(mode)
+    return alpha, b, w
+
+
+def causal_conv4(x, W):
+    """x [B,T,C], W [C,4] -> y [B,T,C] (depthwise causal conv, zero history)."""
+    x = _f64(x)
+    W = _f64(W)
+    B, T, C = x.shape
+    assert W.shape == (C, 4)
+    y = np.zeros_like(x)
+    if _load().oracle_causal_conv4(B, T, C, _ptr(x), _ptr(W), _ptr(y)) != 0:
+        raise ValueError("oracle_causal_conv4 rejected its arguments")
+    return y
+
+
+def l2norm(x, eps: float = L2NORM_EPS):
+    """Normalise the last axis: x · (Σx² + eps)^(-1/2)."""
+    x = _f64(x)
+    d = x.shape[-1]
+    n = x.size // d if d else 0
+    y = np.zeros_like(x)
+    if _load().oracle_l2norm(n, d, float(eps), _ptr(x), _ptr(y)) != 0:
+        raise ValueError("oracle_l2norm rejected its arguments")
+    return y
+
+
+def preprocess(q, k, v, conv_w=None, l2norm_qk: bool = False):
+    """Optional depthwise causal conv on q, k, v (weights [Hqk·dk + Hqk·dk + Hv·dv, 4],
+    rows ordered q | k | v), then optional L2 normalisation of q and k."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if conv_w is not None:
+        W = _f64(conv_w)
+        nq = Hqk * dk
+        assert W.shape == (2 * nq + Hv * dv, 4)
+        q = causal_conv4(q.reshape(B, T, nq), W[:nq]).reshape(q.shape)
+        k = causal_conv4(k.reshape(B, T, nq), W[nq:2 * nq]).reshape(k.shape)
+        v = causal_conv4(v.reshape(B, T, Hv * dv), W[2 * nq:]).reshape(v.shape)
+    if l2norm_qk:
+        q = l2norm(q)
+        k = l2norm(k)
+    return q, k, v
+
+
+def rel_err(got, ref) -> float:
+    """max |got - ref| / RMS(ref): the parity metric for every floating output."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    if ref.size == 0:
+        return 0.0
+    err = float(np.max(np.abs(got - ref)))
+    return err / rms if rms > 0 else err
