@@ -1,0 +1,385 @@
+"""Benchmark of the GDN-2 recurrence on B200.
+
+One step = one chunked prefill (gdn2_chunk_fwd) of the 48-V-head, d=128 layer
+over T=32768 tokens of one sequence (bf16 q,k,v, fp32 per-channel gates,
+chunk 64), inputs resident in HBM. The decode workload (B=256 sequences, one
+token per step, fp32 states [256,48,128,128]) is timed in the same run and
+reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own sequence
+(independent problems, no data-path collective); value = tokens of all ranks /
+max-over-ranks time ("weak" scaling).
+
+--impl reference times the float64 CPU oracle (the only other code path that
+computes the recurrence) on the host cores, on a bounded sample of the same
+workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s (48 Vheads x 128^2, T=32K) + % tensor peak; decode HBM GB/s"
+PREFILL = "prefill_t32768"
+DECODE = "decode_b256"
+L2_BYTES = 126 * 2**20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ accounting
+
+def prefill_bytes(w, gate_mode="full", o_bytes=2, s0=False):
+    """Algorithmic HBM bytes of one chunk_fwd call: every input read once, every
+    output written once."""
+    tok = w.B * w.T
+    qkb = 2 if w.qkv_dtype == "bf16" else 4
+    n = tok * w.H_qk * w.d * qkb * 2 + tok * w.H_v * w.d * qkb
+    if gate_mode == "full":
+        n += tok * w.H_v * w.d * 4 * 3
+    elif gate_mode == "kda":
+        n += tok * w.H_v * (w.d + 1) * 4
+    else:
+        n += tok * w.H_v * 2 * 4
+    n += tok * w.H_v * w.d * o_bytes
+    n += w.B * w.H_v * w.d * w.d * 4 * (2 if s0 else 1)
+    if w.conv:
+        n += (2 * w.H_qk * w.d + w.H_v * w.d) * 16
+    return n
+
+
+def prefill_flops(w):
+    """Algorithmic FLOPs per call: 6d² + 5Cd per token per value head (state
+    products Q̄S, ĒS, K_endᵀU; T and A_qk Gram triangles; A_qk·U; the solve)."""
+    return w.B * w.T * w.H_v * (6 * w.d * w.d + 5 * w.chunk * w.d)
+
+
+def decode_bytes(w, o_bytes=2):
+    B, d = w.B, w.d
+    state = B * w.H_v * d * d * 4 * 2
+    io = B * w.H_qk * d * 2 * 2 + B * w.H_v * d * 2 + B * w.H_v * d * 4 * 3 + B * w.H_v * d * o_bytes
+    return state + io
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self._t is not None:
+                self._t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ reference arm
+
+def cpu_oracle_rate(w, heads, tokens, threads=0, seed=2):
+    """Run the float64 oracle on `heads` value heads x `tokens` tokens of workload
+    w; return (layer tokens/s, seconds, threads used)."""
+    import numpy as np
+    import torch
+    import oracle
+    from dataclasses import replace
+    from delta_rule_linear_gdn_b200.inputs import make_inputs
+
+    sub = replace(w, T=tokens, H_v=heads, H_qk=max(1, heads * w.H_qk // w.H_v))
+    inp = make_inputs(sub, seed=seed)
+    f = lambda t: None if t is None else t.to(torch.float64).numpy()
+    args = [f(inp[k]) for k in ("q", "k", "v", "alpha", "b", "w")]
+    nthreads = threads or os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.gdn2_forward(*args, f(inp["S0"]), threads=nthreads)
+    dt = time.perf_counter() - t0
+    layer_tokens = tokens * heads / w.H_v
+    return layer_tokens / dt, dt, min(nthreads, heads)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from delta_rule_linear_gdn_b200.inputs import workload
+    w = workload(PREFILL)
+    heads, tokens = w.H_v, 512
+    rates = []
+    for i in range(args.warmup + args.steps):
+        r, dt, used = cpu_oracle_rate(w, heads, tokens)
+        if i >= args.warmup:
+            rates.append((r, dt))
+    total_tok = sum(tokens for _ in rates)
+    total_t = sum(dt for _, dt in rates)
+    value = total_tok / total_t
+    sample = f"{heads} V heads x {tokens} tokens per step of the T=32768 layer (layer tokens = tokens x heads/48)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / max(1, len(rates)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    return {"workload": f"{w.name}: B={w.B} T={w.T} H_qk={w.H_qk} H_v={w.H_v} d={w.d} chunk={w.chunk} "
+                        f"{w.qkv_dtype} q,k,v, fp32 per-channel gates, S0=0",
+            "global_batch": w.B, "seq_len": w.T, "parallelism": "independent sequences per GPU",
+            "l2": "no flush: each step reads ~3.5 GB of inputs, > 126 MB L2"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from delta_rule_linear_gdn_b200 import gdn2
+    from delta_rule_linear_gdn_b200.inputs import make_decode_pool, make_inputs, workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk = peaks()
+    w = workload(PREFILL)
+    stream = torch.cuda.Stream(device=dev)
+    inp = make_inputs(w, seed=2 + 1000 * rank, device=dev)
+    o = torch.empty((w.B, w.T, w.H_v, w.d), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((w.B, w.H_v, w.d, w.d), dtype=torch.float32, device=dev)
+    p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk)
+    ws_bytes = gdn2.chunk_fwd_workspace(p)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    launches_per_call = 1
+
+    def prefill_call():
+        gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None, chunk=w.chunk,
+                       o=o, S_T=S_T, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            prefill_call()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                prefill_call()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = max_over_ranks(ms)
+    tokens_per_step = w.B * w.T * world
+    value = tokens_per_step / (ms_max * 1e-3)
+
+    nbytes = prefill_bytes(w)
+    flops = prefill_flops(w)
+    kernel_s = ms * 1e-3  # one launch per call
+    achieved_gbs = nbytes / kernel_s / 1e9
+    tflops = flops / kernel_s / 1e12
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / pk["hbm_gbs"], "traffic": None,
+                "peak_source": pk["source"],
+                "kernel": "gdn2 chunk_fwd", "alg_bytes_per_launch": nbytes, "alg_flops_per_launch": flops,
+                "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"]}
+
+    # ---------------------------------------------------------------- decode
+    dw = workload(DECODE)
+    pool = make_decode_pool(dw, pool=16, device=dev)
+    S = pool["S0"].clone()
+    od = torch.empty((dw.B, dw.H_v, dw.d), dtype=torch.bfloat16, device=dev)
+
+    def decode_call(i):
+        gdn2.decode_step(pool["q"][i], pool["k"][i], pool["v"][i], pool["alpha"][i], pool["b"][i], pool["w"][i],
+                         S, o=od, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(5):
+            decode_call(i % 16)
+    torch.cuda.synchronize()
+    barrier()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.decode_steps):
+            decode_call(i % 16)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    dms = max_over_ranks(d0.elapsed_time(d1) / args.decode_steps)
+    dbytes = decode_bytes(dw)
+    decode = {"workload": f"{dw.name}: B={dw.B} sequences, one token per step, H_qk={dw.H_qk} H_v={dw.H_v} "
+                          f"d={dw.d}, fp32 state, bf16 q,k,v,o, {args.decode_steps} consecutive steps",
+              "us_per_step": dms * 1e3, "gbs": dbytes / (dms * 1e-3) / 1e9 * world,
+              "roofline": {"bound": "hbm", "achieved": dbytes / (dms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                           "unit": "GB/s", "frac": dbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                           "traffic": None, "alg_bytes_per_launch": dbytes},
+              "tokens_per_s": dw.B * world / (dms * 1e-3)}
+
+    # ---------------------------------------------------------------- end to end
+    host = {k: inp[k].cpu().pin_memory() for k in ("q", "k", "v", "alpha", "b", "w")}
+    dev_in = {k: torch.empty_like(inp[k]) for k in host}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_host = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
+
+    def e2e_call():
+        for k_ in host:
+            dev_in[k_].copy_(host[k_], non_blocking=True)
+        gdn2.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["b"], dev_in["w"], None,
+                       chunk=w.chunk, o=o, S_T=S_T, workspace=ws, stream=stream)
+        o_host.copy_(o, non_blocking=True)
+        S_host.copy_(S_T, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_call()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.e2e_steps):
+            e2e_call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ems = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
+    e2e = {"value": tokens_per_step / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+
+    # ---------------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        heads, tokens = w.H_v, 2048
+        rate, dt, used = cpu_oracle_rate(w, heads, tokens)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
+               "sample": f"{heads} V heads x {tokens} tokens of the T=32768 layer workload "
+                         f"({dt:.1f} s, layer tokens = tokens x heads/48)"}
+
+    clocks = clk.summary()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,185 @@
+// C ABI entry points: argument validation on the host, then one launch on the
+// caller's stream. See include/gdn2.h for the contract of each call.
+
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+
+using namespace gdn2;
+
+namespace {
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// Byte range [p, p + n) overlaps [q, q + m)?
+bool overlaps(const void* p, size_t n, const void* q, size_t m) {
+  if (!p || !q || n == 0 || m == 0) return false;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+  return a < b + m && b < a + n;
+}
+
+size_t dsize(int dtype) { return dtype == GDN2_BF16 ? 2 : 4; }
+
+// Shared shape/enum checks. tokens = B*T (chunk) or B (decode).
+gdn2_status check_common(const gdn2_params* p, bool decode) {
+  if (!p) return GDN2_ERR_INVALID_ARG;
+  if (p->B < 0 || (!decode && p->T < 0) || p->H_qk <= 0 || p->H_v <= 0) return GDN2_ERR_INVALID_ARG;
+  if (p->H_v % p->H_qk != 0) return GDN2_ERR_INVALID_ARG;
+  if (p->d_k <= 0 || p->d_v <= 0) return GDN2_ERR_INVALID_ARG;
+  if (p->qkv_dtype != GDN2_F32 && p->qkv_dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
+  if (p->o_dtype != GDN2_F32 && p->o_dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
+  if (p->gate_mode < GDN2_GATES_FULL || p->gate_mode > GDN2_GATES_GDN) return GDN2_ERR_INVALID_ARG;
+  if (p->precision != GDN2_PREC_DEFAULT && p->precision != GDN2_PREC_FP32) return GDN2_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return GDN2_ERR_INVALID_ARG;
+  if (p->d_k != p->d_v || !supported_dim(p->d_k)) return GDN2_ERR_UNSUPPORTED;
+  // Element counts must fit comfortably in 63 bits and grid sizes in 31.
+  const double elems = (double)p->B * (decode ? 1.0 : (double)p->T) * p->H_v * p->d_k;
+  if (elems > 9.0e15) return GDN2_ERR_INVALID_ARG;
+  if ((double)p->B * p->H_v * (p->d_k / 16) > 2.0e9) return GDN2_ERR_INVALID_ARG;
+  return GDN2_OK;
+}
+
+struct Sizes {
+  size_t qk, v, ga, gb, gw, st;  // bytes of q (= k), v, alpha, b, w, state
+};
+
+Sizes sizes(const gdn2_params* p, size_t tokens) {
+  Sizes s;
+  const size_t dk = p->d_k, dv = p->d_v;
+  s.qk = tokens * p->H_qk * dk * dsize(p->qkv_dtype);
+  s.v = tokens * p->H_v * dv * dsize(p->qkv_dtype);
+  s.ga = tokens * p->H_v * (p->gate_mode == GDN2_GATES_GDN ? 1 : dk) * 4;
+  s.gb = tokens * p->H_v * (p->gate_mode == GDN2_GATES_FULL ? dk : 1) * 4;
+  s.gw = p->gate_mode == GDN2_GATES_FULL ? tokens * p->H_v * dv * 4 : 0;
+  s.st = (size_t)p->B * p->H_v * dk * dv * 4;
+  return s;
+}
+
+gdn2_status check_gate_ptrs(const gdn2_params* p, const float* alpha, const float* b, const float* w) {
+  if (!alpha || !b) return GDN2_ERR_INVALID_ARG;
+  if (p->gate_mode == GDN2_GATES_FULL ? (w == nullptr) : (w != nullptr)) return GDN2_ERR_INVALID_ARG;
+  return GDN2_OK;
+}
+
+ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* b, const float* w, const float* S0, void* o,
+                          float* S_T, void* ws, size_t ws_bytes) {
+  ChunkArgs a;
+  a.B = p->B; a.T = p->T; a.Hqk = p->H_qk; a.Hv = p->H_v; a.dk = p->d_k; a.dv = p->d_v;
+  a.chunk = p->chunk; a.scale = p->scale; a.gate_mode = p->gate_mode; a.l2norm = p->l2norm_qk != 0;
+  a.conv_w = p->conv_w;
+  a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S0 = S0; a.o = o; a.ST = S_T;
+  a.workspace = ws; a.ws_bytes = ws_bytes;
+  return a;
+}
+
+bool use_tc(const gdn2_params* p, const ChunkArgs& a) {
+  return p->precision == GDN2_PREC_DEFAULT && p->T > 0 && p->B > 0 &&
+         chunk_tc_supported(a, p->qkv_dtype == GDN2_BF16);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn2_status_str(gdn2_status s) {
+  switch (s) {
+    case GDN2_OK: return "GDN2_OK";
+    case GDN2_ERR_INVALID_ARG: return "GDN2_ERR_INVALID_ARG: invalid argument (pointer, shape, alignment or aliasing)";
+    case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED: no kernel for this configuration";
+    case GDN2_ERR_WORKSPACE: return "GDN2_ERR_WORKSPACE: workspace missing or too small";
+    case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA: CUDA launch or runtime error";
+    case GDN2_ERR_TIMEOUT: return "GDN2_ERR_TIMEOUT: a device-side wait gave up";
+  }
+  return "GDN2: unknown status";
+}
+
+int gdn2_version(void) { return 100; }
+
+size_t gdn2_chunk_fwd_workspace(const gdn2_params* p) {
+  if (check_common(p, false) != GDN2_OK) return 0;
+  ChunkArgs a = make_chunk_args(p, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                nullptr, nullptr, 0);
+  return use_tc(p, a) ? chunk_tc_workspace(a) : 0;
+}
+
+gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* b, const float* w, const float* S0, void* o,
+                           float* S_T, void* workspace, size_t ws_bytes, void* stream) {
+  gdn2_status st = check_common(p, false);
+  if (st != GDN2_OK) return st;
+  if (p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return GDN2_ERR_UNSUPPORTED;
+  const size_t tokens = (size_t)p->B * p->T;
+  if (tokens > 0) {
+    if (!q || !k || !v || !o) return GDN2_ERR_INVALID_ARG;
+    if ((st = check_gate_ptrs(p, alpha, b, w)) != GDN2_OK) return st;
+  }
+  const void* ptrs[] = {q, k, v, alpha, b, w, S0, o, S_T, p->conv_w, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return GDN2_ERR_INVALID_ARG;
+  const Sizes sz = sizes(p, tokens);
+  const size_t o_bytes = tokens * p->H_v * p->d_v * dsize(p->o_dtype);
+  const size_t conv_bytes = ((size_t)2 * p->H_qk * p->d_k + (size_t)p->H_v * p->d_v) * 4 * sizeof(float);
+  struct R { const void* p; size_t n; } ins[] = {{q, sz.qk}, {k, sz.qk}, {v, sz.v}, {alpha, sz.ga},
+                                                  {b, sz.gb}, {w, sz.gw}, {S0, sz.st}, {p->conv_w, conv_bytes}};
+  for (const R& r : ins) {
+    if (overlaps(o, o_bytes, r.p, r.n)) return GDN2_ERR_INVALID_ARG;
+    if (r.p != S0 && overlaps(S_T, sz.st, r.p, r.n)) return GDN2_ERR_INVALID_ARG;
+  }
+  if (S0 && S_T && S0 != S_T && overlaps(S0, sz.st, S_T, sz.st)) return GDN2_ERR_INVALID_ARG;
+  if (overlaps(o, o_bytes, S_T, sz.st)) return GDN2_ERR_INVALID_ARG;
+
+  ChunkArgs a = make_chunk_args(p, q, k, v, alpha, b, w, S0, o, S_T, workspace, ws_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (use_tc(p, a)) {
+    const size_t need = chunk_tc_workspace(a);
+    if (need > 0 && (workspace == nullptr || ws_bytes < need)) return GDN2_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GDN2_ERR_INVALID_ARG;
+    if (need > 0 && (overlaps(workspace, need, o, o_bytes) || overlaps(workspace, need, S_T, sz.st)))
+      return GDN2_ERR_INVALID_ARG;
+    e = launch_chunk_tc(a, p->o_dtype == GDN2_BF16, s);
+  } else {
+    e = launch_chunk_simt(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16, s);
+  }
+  return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k, const void* v,
+                             const float* alpha, const float* b, const float* w, float* S, void* o,
+                             void* stream) {
+  gdn2_status st = check_common(p, true);
+  if (st != GDN2_OK) return st;
+  if (p->conv_w != nullptr) return GDN2_ERR_UNSUPPORTED;
+  const size_t tokens = (size_t)p->B;
+  if (tokens > 0) {
+    if (!q || !k || !v || !o || !S) return GDN2_ERR_INVALID_ARG;
+    if ((st = check_gate_ptrs(p, alpha, b, w)) != GDN2_OK) return st;
+  }
+  const void* ptrs[] = {q, k, v, alpha, b, w, S, o};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return GDN2_ERR_INVALID_ARG;
+  const Sizes sz = sizes(p, tokens);
+  const size_t o_bytes = tokens * p->H_v * p->d_v * dsize(p->o_dtype);
+  struct R { const void* p; size_t n; } ins[] = {{q, sz.qk}, {k, sz.qk}, {v, sz.v}, {alpha, sz.ga},
+                                                  {b, sz.gb}, {w, sz.gw}};
+  for (const R& r : ins) {
+    if (overlaps(o, o_bytes, r.p, r.n)) return GDN2_ERR_INVALID_ARG;
+    if (overlaps(S, sz.st, r.p, r.n)) return GDN2_ERR_INVALID_ARG;
+  }
+  if (overlaps(o, o_bytes, S, sz.st)) return GDN2_ERR_INVALID_ARG;
+  if (tokens == 0) return GDN2_OK;
+
+  DecodeArgs a;
+  a.B = p->B; a.Hqk = p->H_qk; a.Hv = p->H_v; a.d = p->d_k; a.scale = p->scale;
+  a.gate_mode = p->gate_mode; a.l2norm = p->l2norm_qk != 0;
+  a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S = S; a.o = o;
+  cudaError_t e = launch_decode(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16,
+                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// Internal declarations shared by the CUDA translation units of libgdn2.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn2.h"
+
+namespace gdn2 {
+
+// Conversions between the I/O dtypes and fp32.
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// The epsilon of the fused L2 normalisation: x · (Σx² + eps)^(−1/2).
+constexpr float kL2Eps = 1e-6f;
+
+// Arguments of one launch, already validated by the host entry points.
+struct ChunkArgs {
+  int B, T, Hqk, Hv, dk, dv, chunk;
+  float scale;
+  int gate_mode;
+  int l2norm;
+  const float* conv_w;
+  const void *q, *k, *v;
+  const float *alpha, *b, *w, *S0;
+  void* o;
+  float* ST;
+  void* workspace;
+  size_t ws_bytes;
+};
+
+struct DecodeArgs {
+  int B, Hqk, Hv, d;
+  float scale;
+  int gate_mode;
+  int l2norm;
+  const void *q, *k, *v;
+  const float *alpha, *b, *w;
+  float* S;
+  void* o;
+};
+
+// Launchers (return cudaSuccess or the launch error).
+cudaError_t launch_decode(const DecodeArgs& a, int qkv_bf16, int o_bf16, cudaStream_t s);
+cudaError_t launch_chunk_simt(const ChunkArgs& a, int qkv_bf16, int o_bf16, cudaStream_t s);
+bool chunk_tc_supported(const ChunkArgs& a, int qkv_bf16);
+size_t chunk_tc_workspace(const ChunkArgs& a);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s);
+
+}  // namespace gdn2

@@ -1,0 +1,191 @@
+// Fused recurrent decode step of the Gated DeltaNet-2 recurrence (one token).
+//
+// Per (sequence, value head) — "Resumo Técnico: Gated DeltaNet-2", Metodologia
+// §1, and the fused recurrent schedule of "Uma análise das variantes de
+// atenção linear da família DeltaNet", section "Kernel Triton recorrente
+// fundido para decode":
+//     S̄ = Diag(α) S                 (decay)
+//     r = S̄ᵀ e,  p = S̄ᵀ q            (key-read and query-read reductions)
+//     u = z − r                     (residual)
+//     S ← S̄ + k uᵀ                  (outer-product write)
+//     o = s (p + (kᵀq) u)           (= s·Sᵀq after the write)
+// with e = b ⊙ k, z = w ⊙ v. Both reductions run on the decayed state in the
+// same register pass, so the state is read from HBM once and written once.
+//
+// Work split: one CTA per (sequence, value head, tile of COLS value columns).
+// Thread (cg, rg) owns 4 consecutive columns (one float4) of rows
+// rg, rg+16, rg+32, ...: a warp instruction covers whole 4·COLS-byte row
+// segments, so every state access is a coalesced 128-bit load/store. The
+// state is streamed (evict-first) because it is far larger than L2.
+
+#include "common.cuh"
+
+namespace gdn2 {
+namespace {
+
+constexpr int kRowGroups = 16;
+
+template <int D, int COLS, typename TIn, typename TOut>
+__global__ void __launch_bounds__((COLS / 4) * kRowGroups)
+decode_kernel(DecodeArgs a) {
+  constexpr int CG = COLS / 4;            // column groups (float4 each)
+  constexpr int NT = CG * kRowGroups;     // threads
+  constexpr int RPT = D / kRowGroups;     // rows per thread
+  constexpr int NW = NT / 32;             // warps
+  constexpr int TILES = D / COLS;
+  static_assert(NT % 32 == 0 && RPT >= 1, "bad decode tiling");
+
+  const int tile = blockIdx.x % TILES;
+  const int bh = blockIdx.x / TILES;      // b * Hv + h
+  const int h = bh % a.Hv;
+  const int bi = bh / a.Hv;
+  const int hq = h / (a.Hv / a.Hqk);
+  const int tid = threadIdx.x;
+  const int cg = tid % CG;
+  const int rg = tid / CG;
+  const int col0 = tile * COLS;
+
+  __shared__ float s_q[D], s_k[D], s_a[D], s_e[D];
+  __shared__ float s_z[COLS];
+  __shared__ float s_red[2][NW][COLS];
+  __shared__ float s_u[COLS];
+  __shared__ float s_scalar[4];           // |q|⁻¹, |k|⁻¹, kᵀq
+
+  // Issue the state loads first: they are the only HBM-heavy traffic.
+  float4* Sg = reinterpret_cast<float4*>(a.S + (size_t)bh * D * D + col0) + cg;
+  float4 st[RPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) st[i] = __ldcs(Sg + (size_t)(rg + kRowGroups * i) * (D / 4));
+
+  // Per-token vectors into shared memory (fp32).
+  const TIn* qg = static_cast<const TIn*>(a.q) + ((size_t)bi * a.Hqk + hq) * D;
+  const TIn* kg = static_cast<const TIn*>(a.k) + ((size_t)bi * a.Hqk + hq) * D;
+  const TIn* vg = static_cast<const TIn*>(a.v) + (size_t)bh * D + col0;
+  for (int i = tid; i < D; i += NT) {
+    s_q[i] = to_f32(qg[i]);
+    s_k[i] = to_f32(kg[i]);
+    s_a[i] = (a.gate_mode == GDN2_GATES_GDN) ? a.alpha[bh] : a.alpha[(size_t)bh * D + i];
+  }
+  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : a.b[bh];
+  for (int j = tid; j < COLS; j += NT) {
+    const float wj = (a.gate_mode == GDN2_GATES_FULL) ? a.w[(size_t)bh * D + col0 + j] : beta;
+    s_z[j] = wj * to_f32(vg[j]);
+  }
+  __syncthreads();
+  if (tid < 32) {
+    float sq = 0.f, sk = 0.f, kq = 0.f;
+    for (int i = tid; i < D; i += 32) {
+      sq += s_q[i] * s_q[i];
+      sk += s_k[i] * s_k[i];
+      kq += s_k[i] * s_q[i];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      sk += __shfl_xor_sync(0xffffffffu, sk, off);
+      kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    }
+    if (tid == 0) {
+      float iq = 1.f, ik = 1.f;
+      if (a.l2norm) {
+        iq = rsqrtf(sq + kL2Eps);
+        ik = rsqrtf(sk + kL2Eps);
+      }
+      s_scalar[0] = iq;
+      s_scalar[1] = ik;
+      s_scalar[2] = kq * iq * ik;
+    }
+  }
+  __syncthreads();
+  const float iq = s_scalar[0], ik = s_scalar[1], kq = s_scalar[2];
+  for (int i = tid; i < D; i += NT) {
+    const float kk = s_k[i] * ik;
+    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? a.b[(size_t)bh * D + i] : beta;
+    s_e[i] = bb * kk;
+  }
+  __syncthreads();
+
+  // Decay and both reductions over the thread's rows.
+  float r[4] = {0.f, 0.f, 0.f, 0.f}, p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int row = rg + kRowGroups * i;
+    const float al = s_a[row];
+    st[i].x *= al; st[i].y *= al; st[i].z *= al; st[i].w *= al;
+    const float er = s_e[row], qr = s_q[row] * iq;
+    r[0] += st[i].x * er; r[1] += st[i].y * er; r[2] += st[i].z * er; r[3] += st[i].w * er;
+    p[0] += st[i].x * qr; p[1] += st[i].y * qr; p[2] += st[i].z * qr; p[3] += st[i].w * qr;
+  }
+  // Reduce across the row groups that share a warp (lanes cg + CG·m).
+#pragma unroll
+  for (int off = CG; off < 32; off <<= 1) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      r[c] += __shfl_xor_sync(0xffffffffu, r[c], off);
+      p[c] += __shfl_xor_sync(0xffffffffu, p[c], off);
+    }
+  }
+  const int lane = tid & 31, warp = tid >> 5;
+  if (lane < CG) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      s_red[0][warp][cg * 4 + c] = r[c];
+      s_red[1][warp][cg * 4 + c] = p[c];
+    }
+  }
+  __syncthreads();
+  if (tid < COLS) {
+    float rr = 0.f, pp = 0.f;
+#pragma unroll
+    for (int w_ = 0; w_ < NW; ++w_) {
+      rr += s_red[0][w_][tid];
+      pp += s_red[1][w_][tid];
+    }
+    const float u = s_z[tid] - rr;
+    s_u[tid] = u;
+    TOut* og = static_cast<TOut*>(a.o) + (size_t)bh * D + col0;
+    og[tid] = from_f32<TOut>(a.scale * (pp + kq * u));
+  }
+  __syncthreads();
+
+  // Write S ← S̄ + k uᵀ.
+  const float u0 = s_u[cg * 4 + 0], u1 = s_u[cg * 4 + 1], u2 = s_u[cg * 4 + 2], u3 = s_u[cg * 4 + 3];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int row = rg + kRowGroups * i;
+    const float kr = s_k[row] * ik;
+    float4 x = st[i];
+    x.x += kr * u0; x.y += kr * u1; x.z += kr * u2; x.w += kr * u3;
+    __stcs(Sg + (size_t)row * (D / 4), x);
+  }
+}
+
+template <int D, int COLS, typename TIn, typename TOut>
+cudaError_t launch_t(const DecodeArgs& a, cudaStream_t s) {
+  const int grid = a.B * a.Hv * (D / COLS);
+  if (grid == 0) return cudaSuccess;
+  decode_kernel<D, COLS, TIn, TOut><<<grid, (COLS / 4) * kRowGroups, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename TIn, typename TOut>
+cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
+  switch (a.d) {
+    case 16: return launch_t<16, 16, TIn, TOut>(a, s);
+    case 32: return launch_t<32, 32, TIn, TOut>(a, s);
+    case 64: return launch_t<64, 64, TIn, TOut>(a, s);
+    case 128: return launch_t<128, 64, TIn, TOut>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a, int qkv_bf16, int o_bf16, cudaStream_t s) {
+  if (qkv_bf16) {
+    return o_bf16 ? launch_d<__nv_bfloat16, __nv_bfloat16>(a, s) : launch_d<__nv_bfloat16, float>(a, s);
+  }
+  return o_bf16 ? launch_d<float, __nv_bfloat16>(a, s) : launch_d<float, float>(a, s);
+}
+
+}  // namespace gdn2

@@ -1,0 +1,185 @@
+"""ctypes binding of libgdn2 (declared in include/gdn2.h).
+
+Argument marshalling only: shapes are read from the tensors, outputs are
+allocated with PyTorch (device memory), and every step of the recurrence runs
+in the CUDA library. There is no CPU or PyTorch fallback: if the library is
+missing or fails to load, every call raises.
+
+Entry points mirror the C ABI:
+
+* :func:`chunk_fwd` -> ``gdn2_chunk_fwd`` (chunked prefill)
+* :func:`chunk_fwd_workspace` -> ``gdn2_chunk_fwd_workspace``
+* :func:`decode_step` -> ``gdn2_decode_step`` (one recurrent step, state in place)
+* :func:`status_str`, :func:`version`
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn2.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+F32, BF16 = 0, 1
+GATES = {"full": 0, "kda": 1, "gdn": 2}
+PRECISION = {"default": 0, "fp32": 1}
+
+EXPORTS = ("gdn2_status_str", "gdn2_version", "gdn2_chunk_fwd_workspace", "gdn2_chunk_fwd",
+           "gdn2_decode_step")
+
+
+class Params(ctypes.Structure):
+    """Mirror of ``gdn2_params``."""
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("H_qk", ctypes.c_int), ("H_v", ctypes.c_int),
+        ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("chunk", ctypes.c_int),
+        ("scale", ctypes.c_float), ("qkv_dtype", ctypes.c_int), ("o_dtype", ctypes.c_int),
+        ("gate_mode", ctypes.c_int), ("precision", ctypes.c_int), ("l2norm_qk", ctypes.c_int),
+        ("conv_w", ctypes.c_void_p),
+    ]
+
+
+class GDN2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)}")
+
+
+_lib = None
+
+
+def lib():
+    """Load libgdn2.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m delta_rule_linear_gdn_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp = ctypes.c_void_p
+        pp = ctypes.POINTER(Params)
+        L.gdn2_status_str.argtypes = [ctypes.c_int]
+        L.gdn2_status_str.restype = ctypes.c_char_p
+        L.gdn2_version.argtypes = []
+        L.gdn2_version.restype = ctypes.c_int
+        L.gdn2_chunk_fwd_workspace.argtypes = [pp]
+        L.gdn2_chunk_fwd_workspace.restype = ctypes.c_size_t
+        L.gdn2_chunk_fwd.argtypes = [pp] + [vp] * 10 + [ctypes.c_size_t, vp]
+        L.gdn2_chunk_fwd.restype = ctypes.c_int
+        L.gdn2_decode_step.argtypes = [pp] + [vp] * 9
+        L.gdn2_decode_step.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().gdn2_status_str(int(status)).decode()
+
+
+def version() -> int:
+    return lib().gdn2_version()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dtype_code(dt) -> int:
+    if dt == torch.bfloat16:
+        return BF16
+    if dt == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {dt} (bf16 or fp32)")
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def make_params(B, T, H_qk, H_v, d_k, d_v, *, chunk=64, scale=1.0, qkv_dtype=BF16, o_dtype=BF16,
+                gate_mode="full", precision="default", l2norm_qk=False, conv_w=None) -> Params:
+    return Params(int(B), int(T), int(H_qk), int(H_v), int(d_k), int(d_v), int(chunk), float(scale),
+                  int(qkv_dtype), int(o_dtype), GATES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode),
+                  PRECISION[precision] if isinstance(precision, str) else int(precision),
+                  1 if l2norm_qk else 0, _ptr(conv_w))
+
+
+def _check(t, name, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def chunk_fwd_workspace(params: Params) -> int:
+    return int(lib().gdn2_chunk_fwd_workspace(ctypes.byref(params)))
+
+
+def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_mode="full",
+              precision="default", l2norm_qk=False, conv_w=None, o_dtype=None, o=None, S_T=None,
+              workspace=None, stream=None, want_state=True):
+    """Chunked prefill. q,k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; gates fp32 per
+    ``gate_mode``; S0 [B,H_v,d_k,d_v] fp32 or None. Returns (o, S_T)."""
+    B, T, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    o_dtype = q.dtype if o_dtype is None else o_dtype
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, q.dtype)
+    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S0", S0), ("conv_w", conv_w)):
+        _check(t, name, torch.float32)
+    p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
+                    o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, precision=precision,
+                    l2norm_qk=l2norm_qk, conv_w=conv_w)
+    if o is None:
+        o = torch.empty((B, T, H_v, d_v), dtype=o_dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H_v, d_k, d_v), dtype=torch.float32, device=q.device)
+    _check(o, "o", o_dtype)
+    _check(S_T, "S_T", torch.float32)
+    need = chunk_fwd_workspace(p)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdn2_chunk_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
+                              _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
+                              _stream_handle(stream))
+    if st != OK:
+        raise GDN2Error(st, "gdn2_chunk_fwd")
+    return o, S_T
+
+
+def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_qk=False, o_dtype=None,
+                o=None, stream=None):
+    """One decode step. q,k [B,H_qk,d_k]; v [B,H_v,d_v]; gates fp32 without the
+    T axis; S [B,H_v,d_k,d_v] fp32 updated in place. Returns o [B,H_v,d_v]."""
+    B, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[1], v.shape[2]
+    o_dtype = q.dtype if o_dtype is None else o_dtype
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, q.dtype)
+    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S", S)):
+        _check(t, name, torch.float32)
+    p = make_params(B, 1, H_qk, H_v, d_k, d_v, scale=scale, qkv_dtype=_dtype_code(q.dtype),
+                    o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk)
+    if o is None:
+        o = torch.empty((B, H_v, d_v), dtype=o_dtype, device=q.device)
+    _check(o, "o", o_dtype)
+    st = lib().gdn2_decode_step(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
+                                _ptr(S), _ptr(o), _stream_handle(stream))
+    if st != OK:
+        raise GDN2Error(st, "gdn2_decode_step")
+    return o

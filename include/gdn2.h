@@ -1,0 +1,163 @@
+/*
+ * gdn2.h — C ABI of the B200 (sm_100a) Gated DeltaNet-2 recurrence library.
+ *
+ * The operation ("Resumo Técnico: Gated DeltaNet-2", Metodologia, §1 "Regra
+ * Delta Portão-2", the state update equation), per value head, with state
+ * S ∈ R^{d_k × d_v}:
+ *
+ *     e_t = b_t ⊙ k_t                 erase gate b_t ∈ [0,1]^{d_k}, key axis
+ *     z_t = w_t ⊙ v_t                 write gate w_t ∈ [0,1]^{d_v}, value axis
+ *     S_t = (I − k_t e_tᵀ) Diag(α_t) S_{t−1} + k_t z_tᵀ
+ *     o_t = s · S_tᵀ q_t              read after the write, scale s (default 1)
+ *
+ * Tied gates (same section): b_t = w_t = β_t·1 gives KDA; α_t scalar as well
+ * gives Gated DeltaNet; α_t = 1 gives DeltaNet.
+ *
+ * Grouped heads ("Gated DeltaNet: o mixer em 48 das 64 camadas", Conceito):
+ * H_qk query/key heads serve H_v value heads; value head h reads query/key
+ * head h / (H_v / H_qk) (contiguous groups).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays
+ *    owned by the caller. The library allocates nothing, keeps no state
+ *    between calls and never synchronises: all work is enqueued on `stream`
+ *    (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *  - q, k, v, o are bf16 or fp32 (see gdn2_params); gates, S0/S_T/S, conv
+ *    weights are always fp32.
+ *  - Every pointer must be 16-byte aligned.
+ *  - Arguments are validated on the host before any launch. A rejected call
+ *    enqueues nothing and returns GDN2_ERR_INVALID_ARG (bad pointer, shape,
+ *    alignment) or GDN2_ERR_UNSUPPORTED (a valid request this build has no
+ *    kernel for). A launch failure returns GDN2_ERR_CUDA. Nothing is thrown
+ *    across the ABI.
+ *  - Preconditions NOT checked on the device: gates finite with α ∈ (0,1]
+ *    for gdn2_chunk_fwd (α ∈ [0,1] for gdn2_decode_step), b, w ∈ [0,1];
+ *    q, k of unit length unless l2norm_qk is set.
+ *  - Output buffers must not alias inputs, except S0 == S_T (in place).
+ */
+#ifndef GDN2_H_
+#define GDN2_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDN2_API __attribute__((visibility("default")))
+#else
+#define GDN2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN2_OK = 0,
+  GDN2_ERR_INVALID_ARG = 1,
+  GDN2_ERR_UNSUPPORTED = 2,
+  GDN2_ERR_WORKSPACE = 3,
+  GDN2_ERR_CUDA = 4,
+  GDN2_ERR_TIMEOUT = 5 /* reserved: no kernel here waits on another block */
+} gdn2_status;
+
+typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
+
+/* Gate layouts ([B,T,...] for gdn2_chunk_fwd; drop T for gdn2_decode_step):
+ *   GDN2_GATES_FULL  alpha [B,T,H_v,d_k], b [B,T,H_v,d_k], w [B,T,H_v,d_v]
+ *   GDN2_GATES_KDA   alpha [B,T,H_v,d_k], b = beta [B,T,H_v], w = NULL
+ *   GDN2_GATES_GDN   alpha [B,T,H_v],     b = beta [B,T,H_v], w = NULL      */
+typedef enum { GDN2_GATES_FULL = 0, GDN2_GATES_KDA = 1, GDN2_GATES_GDN = 2 } gdn2_gate_mode;
+
+/* Arithmetic of gdn2_chunk_fwd:
+ *   GDN2_PREC_DEFAULT  bf16 q,k,v with d_k = d_v = 128 and chunk 64 run on the
+ *                      tcgen05 tensor-core kernel (bf16 operands, fp32
+ *                      accumulate, fp32 state); everything else runs the fp32
+ *                      SIMT chunk kernel.
+ *   GDN2_PREC_FP32     always the fp32 SIMT chunk kernel (fp32 arithmetic
+ *                      throughout, any input dtype).                          */
+typedef enum { GDN2_PREC_DEFAULT = 0, GDN2_PREC_FP32 = 1 } gdn2_precision;
+
+typedef struct {
+  int B;          /* sequences                                                */
+  int T;          /* tokens per sequence (gdn2_decode_step: ignored, one step)*/
+  int H_qk;       /* query/key heads                                          */
+  int H_v;        /* value heads; H_v % H_qk == 0                             */
+  int d_k;        /* key head dim: 16, 32, 64 or 128                          */
+  int d_v;        /* value head dim: equal to d_k in this build               */
+  int chunk;      /* chunk length C for gdn2_chunk_fwd: 16, 32 or 64          */
+  float scale;    /* readout scale s                                          */
+  int qkv_dtype;  /* gdn2_dtype of q, k, v                                    */
+  int o_dtype;    /* gdn2_dtype of o                                          */
+  int gate_mode;  /* gdn2_gate_mode                                           */
+  int precision;  /* gdn2_precision                                           */
+  int l2norm_qk;  /* nonzero: normalise q and k (after the conv) inside the
+                     kernel: x · (Σx² + 1e-6)^(-1/2)                          */
+  const float* conv_w; /* NULL, or device weights [2·H_qk·d_k + H_v·d_v, 4] of
+                     the depthwise causal conv (kernel 4, no bias, zero
+                     history) applied to q | k | v channels before the
+                     recurrence ("Gated DeltaNet: o mixer em 48 das 64
+                     camadas", Conceito). Tap 3 weights the current token.
+                     gdn2_chunk_fwd only.                                     */
+} gdn2_params;
+
+/* Human-readable name of a status code (static string, never NULL). */
+GDN2_API const char* gdn2_status_str(gdn2_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+GDN2_API int gdn2_version(void);
+
+/* Bytes of device workspace gdn2_chunk_fwd needs for `p` (0 if none). Returns
+ * 0 for invalid parameters as well; gdn2_chunk_fwd reports those. */
+GDN2_API size_t gdn2_chunk_fwd_workspace(const gdn2_params* p);
+
+/* Chunked prefill: runs the recurrence over T tokens of B sequences.
+ *
+ * Schedule ("Uma análise das variantes de atenção linear da família
+ * DeltaNet", sections "Chunkwise KDA" and "Pipeline Triton da versão por
+ * chunks"; generalised to decoupled gates as in "Resumo Técnico: Gated
+ * DeltaNet-2", Metodologia §3 "Treinamento Paralelo Eficiente por Blocos"):
+ * per chunk of C tokens the cumulative per-channel log decay is absorbed into
+ * the erase (Ē) and write (Z) factors, the intra-chunk dependencies are
+ * resolved by a unit-lower-triangular solve (I + T)⁻¹, and the state is
+ * carried serially across chunks. The result equals the token loop up to
+ * rounding.
+ *
+ *   q, k   [B,T,H_qk,d_k]   qkv_dtype
+ *   v      [B,T,H_v,d_v]    qkv_dtype
+ *   alpha, b, w             fp32, layout by gate_mode (above)
+ *   S0     [B,H_v,d_k,d_v]  fp32 initial state, or NULL for zeros
+ *   o      [B,T,H_v,d_v]    o_dtype, written
+ *   S_T    [B,H_v,d_k,d_v]  fp32 final state, written; may be NULL; may equal S0
+ *   workspace               device scratch of at least
+ *                           gdn2_chunk_fwd_workspace(p) bytes (NULL if 0),
+ *                           256-byte aligned; contents need not be preserved
+ *                           between calls; calls sharing a workspace must
+ *                           not overlap on the device.
+ * T == 0 or B == 0 is valid: S_T = S0 (or zeros) and nothing else is written.
+ * Returns GDN2_ERR_WORKSPACE if ws_bytes is too small.                        */
+GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* b, const float* w,
+                           const float* S0, void* o, float* S_T,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* One recurrent decode step for B sequences (one token each), state in place.
+ *
+ * The fused recurrent schedule ("Uma análise das variantes de atenção linear
+ * da família DeltaNet", section "Kernel Triton recorrente fundido para
+ * decode": decay, key-read reduction, residual, outer-product write,
+ * query-read reduction), with the GDN-2 gates. Each state is read once from
+ * HBM and written once.
+ *
+ *   q, k   [B,H_qk,d_k]     qkv_dtype (l2norm_qk honoured; conv_w must be NULL)
+ *   v      [B,H_v,d_v]      qkv_dtype
+ *   alpha, b, w             fp32, gate_mode layouts without the T axis
+ *   S      [B,H_v,d_k,d_v]  fp32, read and overwritten with the new state
+ *   o      [B,H_v,d_v]      o_dtype, written                                  */
+GDN2_API gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k, const void* v,
+                             const float* alpha, const float* b, const float* w,
+                             float* S, void* o, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H_ */

@@ -1,0 +1,62 @@
+"""Helpers shared by the GPU parity tests: run the oracle on the same inputs the
+CUDA path sees and compare with the max|err|/RMS(ref) metric."""
+
+import numpy as np
+import torch
+
+import oracle
+
+TOL_FP32 = 1e-4   # fp32 path
+TOL_BF16 = 2e-2   # bf16 operands, fp32 accumulate
+
+
+def np64(t):
+    return None if t is None else t.detach().to(torch.float64).cpu().numpy()
+
+
+def oracle_gates(mode, alpha, b, w, d_k, d_v):
+    """Per-channel float64 gates for the oracle from the tensors the kernel gets."""
+    if mode == "full":
+        return np64(alpha), np64(b), np64(w)
+    return oracle.expand_tied_gates(mode, np64(alpha), np64(b), d_k, d_v)
+
+
+def oracle_chunk(inp, gate_mode="full", scale=1.0, l2norm_qk=False, S0=None, threads=0,
+                 heads=None):
+    """Oracle (o, S_T) for a chunk_fwd input dict. ``heads`` optionally restricts
+    to a list of (sequence, value head) pairs; returns dict keyed by pair then."""
+    q, k, v = np64(inp["q"]), np64(inp["k"]), np64(inp["v"])
+    d_k, d_v = q.shape[-1], v.shape[-1]
+    conv_w = np64(inp.get("conv_w"))
+    S0 = np64(inp.get("S0")) if S0 is None else np64(S0)
+    alpha, b, w = oracle_gates(gate_mode, inp["alpha"], inp["b"], inp.get("w"), d_k, d_v)
+    if heads is None:
+        qp, kp, vp = oracle.preprocess(q, k, v, conv_w, l2norm_qk)
+        return oracle.gdn2_forward(qp, kp, vp, alpha, b, w, S0, scale=scale, threads=threads)
+    Hqk, Hv = q.shape[2], v.shape[2]
+    g = Hv // Hqk
+    out = {}
+    for (bi, h) in heads:
+        hq = h // g
+        qh, kh = q[bi:bi + 1, :, hq:hq + 1], k[bi:bi + 1, :, hq:hq + 1]
+        vh = v[bi:bi + 1, :, h:h + 1]
+        cw = None
+        if conv_w is not None:
+            n = Hqk * d_k
+            cw = np.concatenate([conv_w[hq * d_k:(hq + 1) * d_k], conv_w[n + hq * d_k:n + (hq + 1) * d_k],
+                                 conv_w[2 * n + h * d_v:2 * n + (h + 1) * d_v]])
+        qp, kp, vp = oracle.preprocess(qh, kh, vh, cw, l2norm_qk)
+        s0 = None if S0 is None else S0[bi:bi + 1, h:h + 1]
+        out[(bi, h)] = oracle.gdn2_forward(qp, kp, vp, alpha[bi:bi + 1, :, h:h + 1], b[bi:bi + 1, :, h:h + 1],
+                                           w[bi:bi + 1, :, h:h + 1], s0, scale=scale, threads=threads)
+    return out
+
+
+def to_cuda(inp):
+    return {k_: (None if t is None else t.cuda()) for k_, t in inp.items()}
+
+
+def assert_close(got, ref, tol, what):
+    err = oracle.rel_err(np64(got) if torch.is_tensor(got) else got, ref)
+    assert np.isfinite(err) and err <= tol, f"{what}: max|err|/RMS(ref) = {err:.3e} > {tol:.1e}"
+    return err

@@ -1,0 +1,115 @@
+"""The C ABI library loads and exports every symbol include/gdn2.h declares, and
+host-side validation rejects bad arguments before any CUDA call (so these run
+without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from delta_rule_linear_gdn_b200 import gdn2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn2.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(gdn2.LIB_PATH):
+        from delta_rule_linear_gdn_b200 import build
+        build.build()
+    return gdn2.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN2_API\s+[\w\s\*]+?\b(gdn2_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    assert set(gdn2.EXPORTS) <= set(syms), syms
+    assert "gdn2_chunk_fwd" in syms and "gdn2_decode_step" in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version(L):
+    for s in range(6):
+        assert gdn2.status_str(s).startswith("GDN2_")
+    assert "unknown" in gdn2.status_str(99)
+    assert gdn2.version() >= 100
+
+
+def _params(**kw):
+    base = dict(B=1, T=64, H_qk=1, H_v=1, d_k=16, d_v=16, chunk=16, qkv_dtype=gdn2.F32, o_dtype=gdn2.F32)
+    base.update(kw)
+    return gdn2.make_params(**base)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _call_chunk(L, p, **ptrs):
+    names = ["q", "k", "v", "alpha", "b", "w", "S0", "o", "S_T", "ws"]
+    vals = {n: FAKE * (i + 1) for i, n in enumerate(names)}
+    vals["ws"] = None
+    vals.update(ptrs)
+    return L.gdn2_chunk_fwd(ctypes.byref(p), *[vals[n] for n in names], 0, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=-1), gdn2.ERR_INVALID_ARG),
+    (dict(T=-5), gdn2.ERR_INVALID_ARG),
+    (dict(H_qk=2, H_v=3), gdn2.ERR_INVALID_ARG),
+    (dict(H_qk=0), gdn2.ERR_INVALID_ARG),
+    (dict(d_k=24, d_v=24), gdn2.ERR_UNSUPPORTED),
+    (dict(d_k=16, d_v=32), gdn2.ERR_UNSUPPORTED),
+    (dict(chunk=48), gdn2.ERR_UNSUPPORTED),
+    (dict(qkv_dtype=7), gdn2.ERR_INVALID_ARG),
+    (dict(gate_mode=5), gdn2.ERR_INVALID_ARG),
+    (dict(precision=3), gdn2.ERR_INVALID_ARG),
+    (dict(scale=float("nan")), gdn2.ERR_INVALID_ARG),
+])
+def test_chunk_rejects_bad_params(L, kw, expect):
+    assert _call_chunk(L, _params(**kw)) == expect
+
+
+def test_chunk_rejects_null_and_misaligned_pointers(L):
+    p = _params()
+    assert _call_chunk(L, p, q=None) == gdn2.ERR_INVALID_ARG
+    assert _call_chunk(L, p, o=None) == gdn2.ERR_INVALID_ARG
+    assert _call_chunk(L, p, alpha=None) == gdn2.ERR_INVALID_ARG
+    assert _call_chunk(L, p, k=FAKE * 2 + 4) == gdn2.ERR_INVALID_ARG
+    # full gates need w; tied gates forbid it
+    assert _call_chunk(L, p, w=None) == gdn2.ERR_INVALID_ARG
+    assert _call_chunk(L, _params(gate_mode=1)) == gdn2.ERR_INVALID_ARG
+
+
+def test_chunk_rejects_aliased_output(L):
+    p = _params()
+    # o on top of q
+    assert _call_chunk(L, p, o=FAKE) == gdn2.ERR_INVALID_ARG
+    # S_T overlapping o
+    assert _call_chunk(L, p, S_T=FAKE * 8 + 64) == gdn2.ERR_INVALID_ARG
+
+
+def test_decode_rejects_conv_and_bad_args(L):
+    p = _params(conv_w=FAKE * 20)
+    args = [FAKE * (i + 1) for i in range(8)]
+    assert L.gdn2_decode_step(ctypes.byref(p), *args, None) == gdn2.ERR_UNSUPPORTED
+    p = _params()
+    args[6] = None  # S
+    assert L.gdn2_decode_step(ctypes.byref(p), *args, None) == gdn2.ERR_INVALID_ARG
+    assert L.gdn2_decode_step(None, *[FAKE] * 8, None) == gdn2.ERR_INVALID_ARG
+
+
+def test_workspace_query_is_host_only(L):
+    assert L.gdn2_chunk_fwd_workspace(None) == 0
+    assert gdn2.chunk_fwd_workspace(_params(B=-1)) == 0
+    # the precise path needs no workspace
+    assert gdn2.chunk_fwd_workspace(_params(precision=1)) == 0

@@ -1,0 +1,192 @@
+"""Chunked prefill (gdn2_chunk_fwd) against the float64 oracle, element by
+element, on seeded inputs; plus schedule-equivalence properties."""
+
+from dataclasses import replace
+
+import pytest
+import torch
+
+from delta_rule_linear_gdn_b200 import gdn2
+from delta_rule_linear_gdn_b200.inputs import make_inputs, workload
+from tests.gpu_util import TOL_BF16, TOL_FP32, assert_close, oracle_chunk, to_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def run(inp, **kw):
+    c = to_cuda(inp)
+    o, S = gdn2.chunk_fwd(c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], c["S0"],
+                          conv_w=c["conv_w"], **kw)
+    torch.cuda.synchronize()
+    return o, S
+
+
+def small(T=64, B=1, H_qk=1, H_v=1, d=16, chunk=16, qkv="f32", s0="zeros", conv=False, **kw):
+    return replace(workload(0), T=T, B=B, H_qk=H_qk, H_v=H_v, d=d, chunk=chunk, qkv_dtype=qkv, s0=s0,
+                   conv=conv, **kw)
+
+
+def test_oracle_scale_workload_fp32():
+    """d=16, T=64, chunk 16, fp32: the 1e-4 bar."""
+    w = workload("oracle_d16_t64")
+    inp = make_inputs(w, seed=0)
+    o, S = run(inp, chunk=w.chunk)
+    o_ref, S_ref = oracle_chunk(inp)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(S, S_ref, TOL_FP32, "S_T")
+
+
+@pytest.mark.parametrize("T", [1, 15, 17, 61, 130])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_ragged_lengths(T, chunk):
+    inp = make_inputs(small(T=T, s0="normal"), seed=T)
+    o, S = run(inp, chunk=chunk)
+    o_ref, S_ref = oracle_chunk(inp)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(S, S_ref, TOL_FP32, "S_T")
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("gate_mode", ["full", "kda", "gdn"])
+def test_grouped_heads_all_dims_and_gate_modes(d, gate_mode):
+    w = small(T=100, B=2, H_qk=2, H_v=6, d=d, chunk=32, s0="normal")
+    inp = make_inputs(w, seed=d, gate_mode=gate_mode)
+    o, S = run(inp, chunk=32, gate_mode=gate_mode, precision="fp32")
+    o_ref, S_ref = oracle_chunk(inp, gate_mode=gate_mode)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(S, S_ref, TOL_FP32, "S_T")
+
+
+def test_conv_and_l2norm_fused():
+    w = small(T=77, B=2, H_qk=2, H_v=4, d=32, chunk=16, s0="normal", conv=True)
+    inp = make_inputs(w, seed=5)
+    o, S = run(inp, chunk=16, l2norm_qk=True)
+    o_ref, S_ref = oracle_chunk(inp, l2norm_qk=True)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(S, S_ref, TOL_FP32, "S_T")
+
+
+def test_scale_and_fp32_out_from_bf16_in():
+    w = small(T=90, B=1, H_qk=1, H_v=3, d=64, chunk=64, qkv="bf16", s0="normal")
+    inp = make_inputs(w, seed=6)
+    s = 64 ** -0.5
+    o, S = run(inp, chunk=64, scale=s, o_dtype=torch.float32, precision="fp32")
+    o_ref, S_ref = oracle_chunk(inp, scale=s)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(S, S_ref, TOL_FP32, "S_T")
+
+
+@pytest.mark.parametrize("gate_mode", ["full", "kda", "gdn"])
+def test_bf16_d128_chunk64(gate_mode):
+    """The layer shape (bf16 in/out, d=128, chunk 64) on a short sequence with a
+    ragged tail, through the default dispatch."""
+    w = small(T=200, B=1, H_qk=2, H_v=6, d=128, chunk=64, qkv="bf16", s0="normal")
+    inp = make_inputs(w, seed=7, gate_mode=gate_mode)
+    o, S = run(inp, chunk=64, gate_mode=gate_mode)
+    o_ref, S_ref = oracle_chunk(inp, gate_mode=gate_mode)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(S, S_ref, TOL_BF16, "S_T")
+
+
+def test_empty_sequence_copies_state():
+    inp = make_inputs(small(T=0, s0="normal"), seed=8)
+    o, S = run(inp, chunk=16)
+    assert o.shape[1] == 0
+    torch.testing.assert_close(S.cpu(), inp["S0"], rtol=0, atol=0)
+    inp0 = make_inputs(small(T=0), seed=8)
+    _, S0z = run(inp0, chunk=16)
+    assert torch.count_nonzero(S0z) == 0
+
+
+def test_in_place_state():
+    inp = make_inputs(small(T=40, B=2, H_qk=1, H_v=2, d=32, s0="normal"), seed=9)
+    c = to_cuda(inp)
+    S = c["S0"].clone()
+    o, S_out = gdn2.chunk_fwd(c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], S, chunk=16, S_T=S)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle_chunk(inp)
+    assert S_out.data_ptr() == S.data_ptr()
+    assert_close(S, S_ref, TOL_FP32, "S_T in place")
+    assert_close(o, o_ref, TOL_FP32, "o")
+
+
+def test_chunk_size_invariance_and_split_sequence():
+    """Schedules of the same recurrence agree: chunk 16/32/64, and [0,T) vs
+    [0,t) then [t,T) carrying the state."""
+    w = small(T=150, B=1, H_qk=1, H_v=2, d=64, s0="normal")
+    inp = make_inputs(w, seed=10)
+    outs = [run(inp, chunk=c) for c in (16, 32, 64)]
+    for o, S in outs[1:]:
+        torch.testing.assert_close(o, outs[0][0], rtol=1e-5, atol=1e-5)
+        torch.testing.assert_close(S, outs[0][1], rtol=1e-5, atol=1e-5)
+    c = to_cuda(inp)
+    t = 70
+    sl = lambda x: x[:, :t].contiguous()
+    sr = lambda x: x[:, t:].contiguous()
+    oa, Sa = gdn2.chunk_fwd(sl(c["q"]), sl(c["k"]), sl(c["v"]), sl(c["alpha"]), sl(c["b"]), sl(c["w"]),
+                            c["S0"], chunk=32)
+    ob, Sb = gdn2.chunk_fwd(sr(c["q"]), sr(c["k"]), sr(c["v"]), sr(c["alpha"]), sr(c["b"]), sr(c["w"]),
+                            Sa, chunk=32)
+    torch.testing.assert_close(torch.cat([oa, ob], 1), outs[1][0], rtol=1e-5, atol=1e-5)
+    torch.testing.assert_close(Sb, outs[1][1], rtol=1e-5, atol=1e-5)
+
+
+def test_decode_steps_equal_chunked_prefill():
+    w = small(T=48, B=2, H_qk=2, H_v=4, d=32, s0="normal")
+    inp = make_inputs(w, seed=11)
+    o_ref, S_ref = run(inp, chunk=16)
+    c = to_cuda(inp)
+    S = c["S0"].clone()
+    outs = []
+    for t in range(w.T):
+        outs.append(gdn2.decode_step(c["q"][:, t].contiguous(), c["k"][:, t].contiguous(),
+                                     c["v"][:, t].contiguous(), c["alpha"][:, t].contiguous(),
+                                     c["b"][:, t].contiguous(), c["w"][:, t].contiguous(), S))
+    torch.cuda.synchronize()
+    torch.testing.assert_close(torch.stack(outs, 1), o_ref, rtol=1e-4, atol=1e-5)
+    torch.testing.assert_close(S, S_ref, rtol=1e-4, atol=1e-5)
+
+
+def test_outputs_have_no_nan_and_no_stray_writes():
+    """Canary: o and S_T sit inside larger buffers whose margins must stay untouched."""
+    w = small(T=33, B=1, H_qk=1, H_v=2, d=32, s0="normal")
+    inp = make_inputs(w, seed=12)
+    c = to_cuda(inp)
+    pad = 256
+    o_buf = torch.full((pad * 2 + 33 * 2 * 32,), 7.0, device="cuda")
+    s_buf = torch.full((pad * 2 + 2 * 32 * 32,), 7.0, device="cuda")
+    o = o_buf[pad:pad + 33 * 2 * 32].view(1, 33, 2, 32)
+    S = s_buf[pad:pad + 2 * 32 * 32].view(1, 2, 32, 32)
+    gdn2.chunk_fwd(c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], c["S0"], chunk=16, o=o, S_T=S)
+    torch.cuda.synchronize()
+    for buf, n in ((o_buf, o.numel()), (s_buf, S.numel())):
+        assert torch.all(buf[:pad] == 7.0) and torch.all(buf[pad + n:] == 7.0)
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+
+
+# ------------------------------------------------------------ full-size workloads
+
+def _sampled(name, heads, gate_mode="full", **kw):
+    w = workload(name)
+    inp = make_inputs(w, device="cuda", gate_mode=gate_mode)
+    o, S = gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"],
+                          chunk=w.chunk, gate_mode=gate_mode, conv_w=inp["conv_w"], l2norm_qk=w.conv, **kw)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    ref = oracle_chunk(inp, gate_mode=gate_mode, l2norm_qk=w.conv, heads=heads)
+    for (bi, h), (o_ref, S_ref) in ref.items():
+        assert_close(o[bi:bi + 1, :, h:h + 1], o_ref, TOL_BF16, f"{name} o[{bi},{h}]")
+        assert_close(S[bi:bi + 1, h:h + 1], S_ref, TOL_BF16, f"{name} S_T[{bi},{h}]")
+
+
+def test_full_size_prefill_t4096_sampled():
+    _sampled("prefill_t4096", [(0, 0), (0, 1), (0, 2), (0, 47)])
+
+
+@pytest.mark.parametrize("gate_mode", ["full", "kda", "gdn"])
+def test_full_size_prefill_t32768_sampled(gate_mode):
+    _sampled("prefill_t32768", [(0, 5), (0, 46)], gate_mode=gate_mode)
+
+
+def test_full_size_conv_prefill_b8_sampled():
+    _sampled("conv_prefill_b8_t8192", [(0, 0), (3, 17), (7, 47)])
