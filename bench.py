@@ -360,7 +360,7 @@ def main():
     # ---------------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        heads, tokens = w.H_v, 2048
+        heads, tokens = w.H_v, 8192
         rate, dt, used = cpu_oracle_rate(w, heads, tokens)
         cpu = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
                "sample": f"{heads} V heads x {tokens} tokens of the T=32768 layer workload "

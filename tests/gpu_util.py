@@ -56,6 +56,17 @@ def to_cuda(inp):
     return {k_: (None if t is None else t.cuda()) for k_, t in inp.items()}
 
 
+def assert_bf16_rounding(o_bf16, o_f32, what):
+    """A bf16 output must be the fp32 result rounded to nearest bf16 (1 ulp slack):
+    the tolerance bar applies to the kernel's arithmetic, and rounding the output
+    to bf16 adds at most 2^-9 relative per element on top of it."""
+    assert o_bf16.dtype == torch.bfloat16 and o_f32.dtype == torch.float32
+    diff = (o_bf16.float() - o_f32.to(torch.bfloat16).float()).abs()
+    ulp = o_f32.abs() * 2.0 ** -7 + 1e-30
+    bad = int((diff > ulp).sum())
+    assert bad == 0, f"{what}: {bad} bf16 outputs are not the rounded fp32 result"
+
+
 def assert_close(got, ref, tol, what):
     err = oracle.rel_err(np64(got) if torch.is_tensor(got) else got, ref)
     assert np.isfinite(err) and err <= tol, f"{what}: max|err|/RMS(ref) = {err:.3e} > {tol:.1e}"

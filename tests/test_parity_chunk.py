@@ -8,7 +8,7 @@ import torch
 
 from delta_rule_linear_gdn_b200 import gdn2
 from delta_rule_linear_gdn_b200.inputs import make_inputs, workload
-from tests.gpu_util import TOL_BF16, TOL_FP32, assert_close, oracle_chunk, to_cuda
+from tests.gpu_util import TOL_BF16, TOL_FP32, assert_bf16_rounding, assert_close, oracle_chunk, to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -82,10 +82,13 @@ def test_bf16_d128_chunk64(gate_mode):
     ragged tail, through the default dispatch."""
     w = small(T=200, B=1, H_qk=2, H_v=6, d=128, chunk=64, qkv="bf16", s0="normal")
     inp = make_inputs(w, seed=7, gate_mode=gate_mode)
-    o, S = run(inp, chunk=64, gate_mode=gate_mode)
+    o, S = run(inp, chunk=64, gate_mode=gate_mode, o_dtype=torch.float32)
     o_ref, S_ref = oracle_chunk(inp, gate_mode=gate_mode)
     assert_close(o, o_ref, TOL_BF16, "o")
     assert_close(S, S_ref, TOL_BF16, "S_T")
+    o16, S16 = run(inp, chunk=64, gate_mode=gate_mode)
+    assert_bf16_rounding(o16, o, "o bf16")
+    torch.testing.assert_close(S16, S, rtol=0, atol=0)
 
 
 def test_empty_sequence_copies_state():
@@ -167,12 +170,20 @@ def test_outputs_have_no_nan_and_no_stray_writes():
 # ------------------------------------------------------------ full-size workloads
 
 def _sampled(name, heads, gate_mode="full", **kw):
+    """Full-size workload in the bench's launch configuration (bf16 o), plus the
+    same launch with an fp32 o that the tolerance is applied to."""
     w = workload(name)
     inp = make_inputs(w, device="cuda", gate_mode=gate_mode)
-    o, S = gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"],
-                          chunk=w.chunk, gate_mode=gate_mode, conv_w=inp["conv_w"], l2norm_qk=w.conv, **kw)
+    call = lambda od: gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"],
+                                     inp["S0"], chunk=w.chunk, gate_mode=gate_mode, conv_w=inp["conv_w"],
+                                     l2norm_qk=w.conv, o_dtype=od, **kw)
+    o16, S16 = call(torch.bfloat16)
+    o, S = call(torch.float32)
     torch.cuda.synchronize()
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    assert_bf16_rounding(o16, o, f"{name} o bf16")
+    torch.testing.assert_close(S16, S, rtol=0, atol=0)
+    del o16, S16
     ref = oracle_chunk(inp, gate_mode=gate_mode, l2norm_qk=w.conv, heads=heads)
     for (bi, h), (o_ref, S_ref) in ref.items():
         assert_close(o[bi:bi + 1, :, h:h + 1], o_ref, TOL_BF16, f"{name} o[{bi},{h}]")

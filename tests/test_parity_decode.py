@@ -9,7 +9,7 @@ import torch
 import oracle
 from delta_rule_linear_gdn_b200 import gdn2
 from delta_rule_linear_gdn_b200.inputs import make_decode_pool, make_inputs, workload
-from tests.gpu_util import TOL_BF16, TOL_FP32, assert_close, np64, oracle_gates
+from tests.gpu_util import TOL_BF16, TOL_FP32, assert_bf16_rounding, assert_close, np64, oracle_gates
 
 pytestmark = pytest.mark.gpu
 
@@ -47,14 +47,18 @@ def test_decode_l2norm_and_scale_bf16_out():
     outs = []
     for t in range(w.T):
         st = {k: (None if v is None else v.cuda()) for k, v in _step_inputs(inp, t).items()}
+        S16 = S.clone()
+        o16 = gdn2.decode_step(st["q"], st["k"], st["v"], st["alpha"], st["b"], st["w"], S16,
+                               scale=s, l2norm_qk=True)
         outs.append(gdn2.decode_step(st["q"], st["k"], st["v"], st["alpha"], st["b"], st["w"], S,
-                                     scale=s, l2norm_qk=True))
-    torch.cuda.synchronize()
+                                     scale=s, l2norm_qk=True, o_dtype=torch.float32))
+        torch.cuda.synchronize()
+        assert_bf16_rounding(o16, outs[-1], f"o bf16 step {t}")
+        torch.testing.assert_close(S16, S, rtol=0, atol=0)
     q, k, v = oracle.preprocess(np64(inp["q"]), np64(inp["k"]), np64(inp["v"]), None, True)
     o_ref, S_ref = oracle.gdn2_forward(q, k, v, np64(inp["alpha"]), np64(inp["b"]), np64(inp["w"]),
                                        np64(inp["S0"]), scale=s)
-    assert outs[0].dtype == torch.bfloat16
-    assert_close(torch.stack(outs, 1), o_ref, TOL_BF16, "o")
+    assert_close(torch.stack(outs, 1), o_ref, TOL_FP32, "o")
     assert_close(S, S_ref, TOL_FP32, "S")
 
 
@@ -80,11 +84,19 @@ def test_full_size_decode_b256():
     outs = []
     for t in range(steps):
         i = t % 16
+        if t == 0:
+            # the bench's launch (bf16 o) and the same step with fp32 o, from the same state
+            S_copy = S.clone()
+            o16 = gdn2.decode_step(pool["q"][i], pool["k"][i], pool["v"][i], pool["alpha"][i],
+                                   pool["b"][i], pool["w"][i], S_copy)
         outs.append(gdn2.decode_step(pool["q"][i], pool["k"][i], pool["v"][i], pool["alpha"][i],
-                                     pool["b"][i], pool["w"][i], S).float())
+                                     pool["b"][i], pool["w"][i], S, o_dtype=torch.float32))
         if t == 0:
             torch.cuda.synchronize()
             S1 = np64(S)
+            assert_bf16_rounding(o16, outs[0], "o bf16 step 1")
+            torch.testing.assert_close(S_copy, S, rtol=0, atol=0)
+            del S_copy
     torch.cuda.synchronize()
     # step 1 on the whole tensor
     x = {k: np64(pool[k][0])[:, None] for k in ("q", "k", "v", "alpha", "b", "w")}
