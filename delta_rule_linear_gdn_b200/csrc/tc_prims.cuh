@@ -1,0 +1,186 @@
+// sm_100a primitives: tcgen05 tensor-core MMA with TMEM accumulators, TMEM
+// loads/stores, shared-memory matrix descriptors and mbarriers (inline PTX).
+//
+// Operand tiles in shared memory use the non-swizzled ("interleaved")
+// canonical layout: the matrix is cut into core matrices of 8 rows × 16 bytes
+// (8 × 8 bf16), each stored as 128 contiguous bytes (row r of the core at byte
+// 16·r). A tile X[R][C] (logical row-major, bf16) is stored core-row-major:
+// core (rb, cb) at byte (rb·C/8 + cb)·128. The same storage serves as
+//   * a K-major operand (rows = M or N, columns = K):
+//       leading byte offset (LBO, between K core matrices)   = 128
+//       stride byte offset  (SBO, between 8-row groups)      = C/8 · 128
+//   * an MN-major operand (rows = K, columns = M or N):
+//       LBO (between K groups of 8 rows)                     = C/8 · 128
+//       SBO (between MN groups of 8 columns)                 = 128
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace gdn2 {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Byte offset of element (r, c) of a tiled bf16 matrix with C columns.
+__host__ __device__ __forceinline__ uint32_t tile_off(int r, int c, int C) {
+  return (uint32_t)(((r >> 3) * (C >> 3) + (c >> 3)) * 128 + (r & 7) * 16 + (c & 7) * 2);
+}
+
+// Shared-memory matrix descriptor, no swizzle, Blackwell version field = 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // version
+  // base offset 0, LBO mode 0, layout type 0 (no swizzle)
+  return d;
+}
+
+// Descriptors for a tiled X[R][C] used as a K-major or MN-major operand.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, int C) { return sdesc(saddr, 128, (C / 8) * 128); }
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr, int C) { return sdesc(saddr, (C / 8) * 128, 128); }
+
+// Instruction descriptor of kind::f16 with an fp32 accumulator. A and B
+// share one 16-bit type: `bf16` selects bf16, otherwise fp16.
+__host__ __device__ constexpr uint32_t idesc_16(int M, int N, bool a_mn, bool b_mn, bool bf16) {
+  return (1u << 4)                          // D format f32
+         | ((bf16 ? 1u : 0u) << 7)          // A format (0 = f16, 1 = bf16)
+         | ((bf16 ? 1u : 0u) << 10)         // B format
+         | ((a_mn ? 1u : 0u) << 15)         // A major (0 = K)
+         | ((b_mn ? 1u : 0u) << 16)         // B major
+         | ((uint32_t)(N >> 3) << 17)       // N / 8
+         | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_16(M, N, a_mn, b_mn, true);
+}
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_16(M, N, a_mn, b_mn, false);
+}
+
+// D[tmem] (+)= A · B for one K=16 step. Issued by a single thread.
+__device__ __forceinline__ void mma16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+      :
+      : "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on an mbarrier once every tcgen05 operation issued so far by this
+// thread has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                   smem_u32(mbar))
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// Make generic-proxy shared-memory writes visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+// TMEM allocation (one full warp executes these).
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes
+// 32·(w%4) .. +31; taddr carries that lane base in bits 31:16).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// mbarriers.
+__device__ __forceinline__ void mbar_init(uint64_t* mbar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* mbar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(mbar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false if the phase did not complete within the limit
+// (each try_wait itself suspends for a hardware-defined interval).
+__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint32_t limit = (1u << 24)) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(mbar, parity)) return true;
+  return false;
+}
+
+// Pack 8 floats to 8 bf16 (16 bytes), round to nearest even.
+__device__ __forceinline__ uint4 pack8_bf16(const float* x) {
+  uint4 u;
+  __nv_bfloat162 h;
+  h = __floats2bfloat162_rn(x[0], x[1]); u.x = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2bfloat162_rn(x[2], x[3]); u.y = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2bfloat162_rn(x[4], x[5]); u.z = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2bfloat162_rn(x[6], x[7]); u.w = *reinterpret_cast<uint32_t*>(&h);
+  return u;
+}
+
+// Pack 8 floats to 8 fp16 (16 bytes), round to nearest even.
+__device__ __forceinline__ uint4 pack8_f16(const float* x) {
+  uint4 u;
+  __half2 h;
+  h = __floats2half2_rn(x[0], x[1]); u.x = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2half2_rn(x[2], x[3]); u.y = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2half2_rn(x[4], x[5]); u.z = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2half2_rn(x[6], x[7]); u.w = *reinterpret_cast<uint32_t*>(&h);
+  return u;
+}
+__device__ __forceinline__ uint4 pack8(const float* x, bool bf16) { return bf16 ? pack8_bf16(x) : pack8_f16(x); }
+
+}  // namespace tc
+}  // namespace gdn2
