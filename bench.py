@@ -195,6 +195,29 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ rank plumbing
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's own sequence (independent problems per GPU)."""
+    return 2 + 1000 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
 def config_dict(w):
     return {"workload": f"{w.name}: B={w.B} T={w.T} H_qk={w.H_qk} H_v={w.H_v} d={w.d} chunk={w.chunk} "
                         f"{w.qkv_dtype} q,k,v, fp32 per-channel gates, S0=0",
@@ -238,17 +261,10 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     pk = peaks()
     w = workload(PREFILL)
     stream = torch.cuda.Stream(device=dev)
-    inp = make_inputs(w, seed=2 + 1000 * rank, device=dev)
+    inp = make_inputs(w, seed=rank_seed(rank), device=dev)
     o = torch.empty((w.B, w.T, w.H_v, w.d), dtype=torch.bfloat16, device=dev)
     S_T = torch.empty((w.B, w.H_v, w.d, w.d), dtype=torch.float32, device=dev)
     p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk)
@@ -277,9 +293,9 @@ def main():
     barrier()
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1) / args.steps
-    ms_max = max_over_ranks(ms)
+    ms_max = max_over_ranks(ms, dev)
     tokens_per_step = w.B * w.T * world
-    value = tokens_per_step / (ms_max * 1e-3)
+    value = weak_value(w.B * w.T, world, ms_max)
 
     nbytes = prefill_bytes(w)
     flops = prefill_flops(w)
@@ -315,7 +331,7 @@ def main():
     d1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    dms = max_over_ranks(d0.elapsed_time(d1) / args.decode_steps)
+    dms = max_over_ranks(d0.elapsed_time(d1) / args.decode_steps, dev)
     dbytes = decode_bytes(dw)
     decode = {"workload": f"{dw.name}: B={dw.B} sequences, one token per step, H_qk={dw.H_qk} H_v={dw.H_v} "
                           f"d={dw.d}, fp32 state, bf16 q,k,v,o, {args.decode_steps} consecutive steps",
@@ -353,7 +369,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ems = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
+    ems = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
     e2e = {"value": tokens_per_step / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
