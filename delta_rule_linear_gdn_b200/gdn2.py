@@ -10,6 +10,8 @@ Entry points mirror the C ABI:
 * :func:`chunk_fwd` -> ``gdn2_chunk_fwd`` (chunked prefill)
 * :func:`chunk_fwd_workspace` -> ``gdn2_chunk_fwd_workspace``
 * :func:`decode_step` -> ``gdn2_decode_step`` (one recurrent step, state in place)
+* :func:`chunk_fwd_noalloc` -> ``gdn2_chunk_fwd_noalloc`` (prefill with the library's
+  own fixed scratch, for callers that cannot allocate device memory)
 * :func:`status_str`, :func:`version`
 """
 
@@ -183,3 +185,29 @@ def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_
     if st != OK:
         raise GDN2Error(st, "gdn2_decode_step")
     return o
+
+
+def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T, chunk=64, scale=1.0, gate_mode="full",
+                      stream=None):
+    """Chunked prefill through ``gdn2_chunk_fwd_noalloc``: the library takes the
+    kernel's scratch from its own fixed device array, so nothing is allocated
+    for the call. ``o`` and ``S_T`` are caller-provided outputs (the caller
+    owns all device memory). Returns (o, S_T)."""
+    L = lib()
+    fn = L.gdn2_chunk_fwd_noalloc
+    fn.argtypes = [ctypes.POINTER(Params)] + [ctypes.c_void_p] * 10
+    fn.restype = ctypes.c_int
+    B, T, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, q.dtype)
+    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S0", S0), ("S_T", S_T)):
+        _check(t, name, torch.float32)
+    _check(o, "o")
+    p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
+                    o_dtype=_dtype_code(o.dtype), gate_mode=gate_mode)
+    st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+            _ptr(S_T), _stream_handle(stream))
+    if st != OK:
+        raise GDN2Error(st, "gdn2_chunk_fwd_noalloc")
+    return o, S_T
