@@ -83,32 +83,10 @@ bool use_tc(const gdn2_params* p, const ChunkArgs& a) {
 
 }  // namespace
 
-extern "C" {
-
-const char* gdn2_status_str(gdn2_status s) {
-  switch (s) {
-    case GDN2_OK: return "GDN2_OK";
-    case GDN2_ERR_INVALID_ARG: return "GDN2_ERR_INVALID_ARG: invalid argument (pointer, shape, alignment or aliasing)";
-    case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED: no kernel for this configuration";
-    case GDN2_ERR_WORKSPACE: return "GDN2_ERR_WORKSPACE: workspace missing or too small";
-    case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA: CUDA launch or runtime error";
-    case GDN2_ERR_TIMEOUT: return "GDN2_ERR_TIMEOUT: a device-side wait gave up";
-  }
-  return "GDN2: unknown status";
-}
-
-int gdn2_version(void) { return 100; }
-
-size_t gdn2_chunk_fwd_workspace(const gdn2_params* p) {
-  if (check_common(p, false) != GDN2_OK) return 0;
-  ChunkArgs a = make_chunk_args(p, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                nullptr, nullptr, 0);
-  return use_tc(p, a) ? chunk_tc_workspace(a) : 0;
-}
-
-gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const void* k, const void* v,
-                           const float* alpha, const float* b, const float* w, const float* S0, void* o,
-                           float* S_T, void* workspace, size_t ws_bytes, void* stream) {
+gdn2_status gdn2::chunk_fwd_checked(const gdn2_params* p, const void* q, const void* k, const void* v,
+                                     const float* alpha, const float* b, const float* w, const float* S0,
+                                     void* o, float* S_T, void* workspace, size_t ws_bytes, void* stream,
+                                     bool segmented_ok) {
   gdn2_status st = check_common(p, false);
   if (st != GDN2_OK) return st;
   if (p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return GDN2_ERR_UNSUPPORTED;
@@ -136,16 +114,46 @@ gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const void* k, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (use_tc(p, a)) {
-    const size_t need = chunk_tc_workspace(a);
+    const size_t need = segmented_ok ? chunk_tc_min_workspace(a, S_T == nullptr) : chunk_tc_workspace(a);
     if (need > 0 && (workspace == nullptr || ws_bytes < need)) return GDN2_ERR_WORKSPACE;
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GDN2_ERR_INVALID_ARG;
-    if (need > 0 && (overlaps(workspace, need, o, o_bytes) || overlaps(workspace, need, S_T, sz.st)))
+    if (need > 0 && (overlaps(workspace, ws_bytes, o, o_bytes) || overlaps(workspace, ws_bytes, S_T, sz.st)))
       return GDN2_ERR_INVALID_ARG;
+    a.ws_bytes = segmented_ok ? ws_bytes : chunk_tc_workspace(a);
     e = launch_chunk_tc(a, p->o_dtype == GDN2_BF16, s);
   } else {
     e = launch_chunk_simt(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16, s);
   }
   return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+extern "C" {
+
+const char* gdn2_status_str(gdn2_status s) {
+  switch (s) {
+    case GDN2_OK: return "GDN2_OK";
+    case GDN2_ERR_INVALID_ARG: return "GDN2_ERR_INVALID_ARG: invalid argument (pointer, shape, alignment or aliasing)";
+    case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED: no kernel for this configuration";
+    case GDN2_ERR_WORKSPACE: return "GDN2_ERR_WORKSPACE: workspace missing or too small";
+    case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA: CUDA launch or runtime error";
+    case GDN2_ERR_TIMEOUT: return "GDN2_ERR_TIMEOUT: a device-side wait gave up";
+  }
+  return "GDN2: unknown status";
+}
+
+int gdn2_version(void) { return 100; }
+
+size_t gdn2_chunk_fwd_workspace(const gdn2_params* p) {
+  if (check_common(p, false) != GDN2_OK) return 0;
+  ChunkArgs a = make_chunk_args(p, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                nullptr, nullptr, 0);
+  return use_tc(p, a) ? chunk_tc_workspace(a) : 0;
+}
+
+gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* b, const float* w, const float* S0, void* o,
+                           float* S_T, void* workspace, size_t ws_bytes, void* stream) {
+  return gdn2::chunk_fwd_checked(p, q, k, v, alpha, b, w, S0, o, S_T, workspace, ws_bytes, stream, false);
 }
 
 gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k, const void* v,

@@ -16,16 +16,26 @@
 //     O = s (Q̄ S + Aqk U),        Q̄_i = γ_i ⊙ q_i
 //     S ← Diag(γ_C) S + K_endᵀ U,  K_end,j = k_j ⊙ Π_{j<s≤C} α_s
 //
-// Everything is computed transposed so that the MMA's M dimension is always
-// 128 (d_v or d_k or a stacked pair of 64-token operands):
-//     (Y S)ᵀ = Sᵀ Yᵀ,  Oᵀ = Sᵀ Q̄ᵀ + Uᵀ Aqkᵀ,  Sᵀ ← Sᵀ Γ + Uᵀ K_end,
-//     Yᵀ = Ēᵀ Aᵀ,  U_wᵀ = Zᵀ Aᵀ,  [T; Aqk] = [Ē'; Q̄'] K̃'ᵀ.
-// Sᵀ lives in TMEM in fp32 for the whole sequence; an fp16 copy in shared
-// memory feeds the next chunk's MMAs.
+// Two kernels, following the pages' split between the parallel intra-chunk
+// work and the single inter-chunk sweep ("Pipeline Triton da versão por
+// chunks"):
+//   * prep: one CTA per (chunk, sequence, value head), all in parallel. It
+//     builds T and Aqk (tensor cores), inverts I + T (fp32), forms Yᵀ and U_wᵀ
+//     (tensor cores) and writes the chunk's scan operands — Yᵀ, U_wᵀ, Q̄, K_end,
+//     Aqk as fp16 tiles already in the MMA shared-memory layout, and γ_C — to
+//     one 73 KB workspace slot.
+//   * scan: one CTA per (sequence, value head) walks the chunks in order. It
+//     streams the slots into shared memory with bulk copies (double-buffered,
+//     chunk c+1 in flight while c computes) and runs
+//         (Y S)ᵀ = Sᵀ Yᵀ,  Oᵀ = Sᵀ Q̄ᵀ,  Uᵀ = U_wᵀ − (Y S)ᵀ,
+//         Sᵀ ← Sᵀ Γ + Uᵀ K_end,  Oᵀ += Uᵀ Aqkᵀ,
+//     with the fp32 state Sᵀ resident in TMEM and an fp16 copy in shared
+//     memory feeding the next chunk's MMAs.
+// Everything is computed transposed so that every MMA has M = 128.
 //
 // Decay factors of the Gram matrices. Π_{j<s≤i} α is split into two factors
 // about a reference token so that one factor multiplies row i and the other
-// row j (and each GEMM stays a GEMM):
+// row j (each product stays a GEMM):
 //   * i, j in the same 32-token half: reference at the boundary of the half's
 //     two 16-token quarters (factors are products over at most 16 tokens);
 //   * i in the second half, j in the first: reference at the half boundary
@@ -36,12 +46,14 @@
 // SIMT kernel has no such restriction.
 //
 // Operand precision. Every operand after the Gram step (Ē, Z, Q̄, K_end, A,
-// Aqk, Y, U and the copy of S) is bounded in magnitude and is stored as fp16
-// (11-bit significand), which is eight times finer than bf16 at the same
-// tensor-core rate; this is what keeps the chunked result within 2e-2 of the
-// float64 token loop. The Gram factors contain reciprocals of decay products
-// and use fp16 only when the chunk's largest factor is below 2^14, bf16
-// (fp32 range) otherwise. The fp16 operands require |S| and |v| below 6e4.
+// Aqk, Y, U_w, U and the copy of S) is bounded in magnitude and is stored as
+// fp16 (11-bit significand), eight times finer than bf16 at the same
+// tensor-core rate; this keeps the chunked result within 2e-2 of the float64
+// token loop. The Gram factors contain reciprocals of decay products and use
+// fp16 when every quarter product of α exceeds 2^-14, bf16 (fp32 range)
+// otherwise, chosen per chunk. The fp16 operands require |S| and |v| < 6e4.
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "tc_prims.cuh"
@@ -53,48 +65,62 @@ using namespace tc;
 
 constexpr int D = 128;            // d_k = d_v
 constexpr int C = 64;             // chunk
-constexpr int NT = 256;           // threads (8 warps)
+constexpr int NT = 256;           // threads per CTA (8 warps)
 
-// Shared-memory map (bytes). Region G holds the Gram operands and is reused
-// after the Gram MMAs for the solve, the inverse and the scan's U and Y tiles.
-constexpr int OFF_GB = 0;                      // [Ē_bnd ; Q̄_bnd] 128 × 128 (rows 32..63, 96..127 used)
-constexpr int OFF_GM = OFF_GB + 128 * D * 2;   // [Ē_mid ; Q̄_mid] 128 × 128
-constexpr int OFF_KM = OFF_GM + 128 * D * 2;   // K̃_mid 64 × 128
-constexpr int OFF_KB = OFF_KM + C * D * 2;     // K̃_bnd 32 × 128
-constexpr int G_END = OFF_KB + 32 * D * 2;     // 90112
-// reuse of region G after the Gram MMAs
-constexpr int OFF_AINV = 0;                    // A = (I+T)⁻¹ fp16 64 × 64
-constexpr int OFF_AQK = OFF_AINV + C * C * 2;  // Aqk fp16 64 × 64
-constexpr int TP = C + 1;                      // padded fp32 row stride
-constexpr int OFF_T = OFF_AQK + C * C * 2;     // T fp32 [64][65]
-constexpr int OFF_INV = OFF_T + C * TP * 4;    // inverse fp32 [64][65]
-constexpr int OFF_TMP = OFF_INV + C * TP * 4;  // temp fp32 [64][65]
-constexpr int OFF_YT = OFF_T;                  // Yᵀ fp16 128 × 64 (after the inverse is packed)
-constexpr int OFF_UT = OFF_YT + D * C * 2;     // Uᵀ fp16 128 × 64
-static_assert(OFF_TMP + C * TP * 4 <= G_END, "region G overflow");
-static_assert(OFF_UT + D * C * 2 <= G_END, "region G overflow");
-// persistent tiles
-constexpr int OFF_EB = G_END;                  // Ē   [64 tok][128 key]
-constexpr int OFF_Z = OFF_EB + C * D * 2;      // Z   [64 tok][128 dv]
-constexpr int OFF_QB = OFF_Z + C * D * 2;      // Q̄   [64 tok][128 key]
-constexpr int OFF_KE = OFF_QB + C * D * 2;     // K_end [64 tok][128 key]
-constexpr int OFF_ST = OFF_KE + C * D * 2;     // Sᵀ fp16 [128 dv][128 key]
-constexpr int OFF_GC = OFF_ST + D * D * 2;     // γ_C fp32 [128]
-constexpr int OFF_BAR = OFF_GC + D * 4;        // mbarrier
-constexpr int OFF_TMEMP = OFF_BAR + 16;        // TMEM base address
-constexpr int OFF_FLAG = OFF_TMEMP + 16;       // error flag
-constexpr int OFF_RED = OFF_FLAG + 16;         // per-warp reduction slots [8]
-constexpr int SMEM_BYTES = OFF_RED + 32;
+// ------------------------------------------------------------------ workspace
+// Word 0 of the workspace is the device status (nonzero: a wait gave up).
+// Slots follow, one per (sequence, value head, chunk of the segment).
+constexpr size_t WS_HEAD = 256;
+constexpr int SL_YT = 0;              // Yᵀ   fp16 [128 key][64 tok]
+constexpr int SL_UW = 16384;          // U_wᵀ fp16 [128 dv][64 tok]
+constexpr int SL_QB = 32768;          // Q̄    fp16 [64 tok][128 key]
+constexpr int SL_KE = 49152;          // K_end fp16 [64 tok][128 key]
+constexpr int SL_AQ = 65536;          // Aqk  fp16 [64 i][64 j]
+constexpr int SL_GC = 73728;          // γ_C  fp32 [128]
+constexpr int SLOT_USED = 74240;      // bytes copied per chunk
+constexpr int SLOT = 74752;           // slot stride (1 KB multiple)
 
-// TMEM columns (fp32, 128 lanes).
-constexpr uint32_t TM_S = 0;        // Sᵀ [dv lanes][128 key]
-constexpr uint32_t TM_GM = 128;     // Gram mid [128][64]
-constexpr uint32_t TM_GB = 192;     // Gram bnd [128][32]
-constexpr uint32_t TM_YT = 224;     // Yᵀ [key lanes][64 tok]
-constexpr uint32_t TM_UW = 288;     // U_wᵀ [dv][64]
-constexpr uint32_t TM_YS = 352;     // (Y S)ᵀ [dv][64]
-constexpr uint32_t TM_O = 416;      // Oᵀ [dv][64]
-constexpr uint32_t TM_COLS = 512;
+// ------------------------------------------------------------------ prep smem
+// [0, 32K): Gram "boundary" operand [Ē_bnd ; Q̄_bnd] as a 128-row tile whose
+// rows 32..63 and 96..127 are used; its unused row groups hold K̃_bnd
+// (rows 0..31 → [0, 8K)) and the quarter products and reduction slots
+// ([16K, 24K)); the MMA reads those rows as don't-care. After the Gram MMAs,
+// [8K, 16K) holds A = (I+T)⁻¹ (fp16 64 × 64). 112 KB in all, so two CTAs
+// share an SM.
+constexpr int P_GB = 0;
+constexpr int P_KB = 0;               // K̃_bnd [32 tok][128] (C = 128 tile, rows 0..31)
+constexpr int P_AINV = 8192;          // A fp16 [64][64]
+constexpr int P_GM = 32768;           // [Ē_mid ; Q̄_mid] 128 × 128
+constexpr int P_KM = 65536;           // K̃_mid [64][128]
+constexpr int P_EB = 81920;           // Ē [64 tok][128 key]
+constexpr int P_Z = 98304;            // Z [64 tok][128 dv]
+constexpr int P_END = 114688;
+// fp32 work arrays of the inverse reuse [P_GM, P_EB) after the Gram MMAs
+constexpr int TS = 68;                // row stride (floats), 16-byte aligned rows
+constexpr int P_T = P_GM;             // T   [64][68]
+constexpr int P_I = P_T + C * TS * 4; // inv [64][68]
+constexpr int P_X = P_I + C * TS * 4; // tmp [32][36]
+static_assert(P_X + 32 * 36 * 4 <= P_EB, "prep smem overlap");
+constexpr int P_PQ = 16384;           // quarter products [4][128] fp32
+constexpr int P_RED = P_PQ + 4 * D * 4;
+static_assert(P_RED + 64 <= 24576, "quarter products must stay in the unused Gram rows");
+constexpr int P_BAR = P_END;
+constexpr int P_TMEMP = P_BAR + 16;
+constexpr int P_FLAG = P_TMEMP + 16;
+constexpr int P_SMEM = P_FLAG + 16;
+// prep TMEM columns
+constexpr uint32_t PT_GM = 0, PT_GB = 64, PT_YT = 128, PT_UW = 192, PT_COLS = 256;
+
+// ------------------------------------------------------------------ scan smem
+constexpr int S_STAGE0 = 0;
+constexpr int S_STAGE1 = SLOT;
+constexpr int S_ST = 2 * SLOT;        // Sᵀ fp16 [128 dv][128 key]
+constexpr int S_UT = S_ST + D * D * 2;// Uᵀ fp16 [128 dv][64 tok]
+constexpr int S_BAR = S_UT + D * C * 2;   // full[2], mma
+constexpr int S_TMEMP = S_BAR + 32;
+constexpr int S_FLAG = S_TMEMP + 16;
+constexpr int S_SMEM = S_FLAG + 16;
+constexpr uint32_t ST_S = 0, ST_YS = 128, ST_O = 192, ST_COLS = 256;
 
 __device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
   *reinterpret_cast<uint4*>(base + off) = v;
@@ -115,33 +141,53 @@ __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float* x) {
     x[2 * i + 1] = f.y;
   }
 }
+__device__ __forceinline__ void unpack8_f16(uint4 u, float* x) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
 
-// Wait for the tensor core to finish the MMAs committed to `bar`; all threads
-// take part. On a timeout the CTA's error flag is raised (uniformly read after
-// the barrier that follows).
 __device__ __forceinline__ void wait_mma(uint64_t* bar, uint32_t& phase, int* sflag) {
   if (!mbar_wait(bar, phase)) atomicOr(sflag, 1);
   phase ^= 1u;
   fence_after_sync();
 }
 
-template <typename TOut>
-__global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(ChunkArgs a) {
+__device__ __forceinline__ void sync_for_mma() {
+  fence_async_smem();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+}
+
+// =============================================================================
+// prep kernel: one CTA per (chunk of the segment, sequence, value head)
+// =============================================================================
+__global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + OFF_TMEMP);
-  int* sflag = reinterpret_cast<int*>(smem + OFF_FLAG);
-  float* sgC = reinterpret_cast<float*>(smem + OFF_GC);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + P_BAR);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + P_TMEMP);
+  int* sflag = reinterpret_cast<int*>(smem + P_FLAG);
+  float* sPq = reinterpret_cast<float*>(smem + P_PQ);
+  float* sred = reinterpret_cast<float*>(smem + P_RED);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;
+  // CTA order: value head fastest, so the value heads sharing a query/key head
+  // run together and share its q, k lines in L2.
+  const int work = blockIdx.x;
+  const int bh = work % (a.B * a.Hv);
+  const int cl = work / (a.B * a.Hv);          // chunk within the segment
+  const int ck = c_begin + cl;
   const int h = bh % a.Hv, bi = bh / a.Hv;
   const int hq = h / (a.Hv / a.Hqk);
   const int mode = a.gate_mode;
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
-  TOut* og = static_cast<TOut*>(a.o);
+  const int t0 = ck * C;
+  const int Lc = min(C, a.T - t0);
+  uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)bh * n_seg + cl) * SLOT;
 
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -149,425 +195,480 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(ChunkArgs a) {
     *sflag = 0;
   }
   if (warp == 0) {
-    tmem_alloc(tmem_ptr, TM_COLS);
+    tmem_alloc(tmem_ptr, PT_COLS);
+    tmem_relinquish();
+  }
+
+  // Element mapping: lane r16 = token within a 16-token quarter, 8 channels.
+  const int r16 = lane & 15;
+  const int cg = 2 * warp + (lane >> 4);
+  const int ch0 = cg * 8;
+
+  // -------- pass 1: α per quarter, quarter products Π over 16 tokens
+  float al[4][8];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int i = 16 * m + r16;
+    if (i < Lc) {
+      const size_t gt = ((size_t)bi * a.T + t0 + i) * a.Hv + h;
+      if (mode == GDN2_GATES_GDN) {
+        const float s = __ldg(a.alpha + gt);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) al[m][c] = s;
+      } else {
+        load8_f32(a.alpha + gt * D + ch0, al[m]);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) al[m][c] = 1.f;
+    }
+  }
+  float mn = 1.f;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float x = al[m][c];
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) x *= __shfl_xor_sync(0xffffffffu, x, off);
+      mn = fminf(mn, x);
+      if (r16 == 0) sPq[m * D + ch0 + c] = x;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+  if (lane == 0) sred[warp] = mn;
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_ptr;
+  bool gram_bf16;
+  {
+    float mall = sred[0];
+#pragma unroll
+    for (int w_ = 1; w_ < 8; ++w_) mall = fminf(mall, sred[w_]);
+    // every in-quarter forward/backward product is ≥ the quarter product
+    gram_bf16 = !(mall > 6.103515625e-05f);   // 2^-14
+  }
+  if (tid < D) {
+    const float g = sPq[tid] * sPq[D + tid] * sPq[2 * D + tid] * sPq[3 * D + tid];
+    reinterpret_cast<float*>(slot + SL_GC)[tid] = g;
+  }
+
+  // -------- pass 2: operand tiles
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int i = 16 * m + r16;
+    float kx[8], qx[8], ex[8], zx[8];
+    if (i < Lc) {
+      const size_t tq = ((size_t)bi * a.T + t0 + i) * a.Hqk + hq;
+      const size_t gt = ((size_t)bi * a.T + t0 + i) * a.Hv + h;
+      float bx[8], wx[8], vx[8];
+      load8_bf16(static_cast<const __nv_bfloat16*>(a.k) + tq * D + ch0, kx);
+      load8_bf16(static_cast<const __nv_bfloat16*>(a.q) + tq * D + ch0, qx);
+      load8_bf16(static_cast<const __nv_bfloat16*>(a.v) + gt * D + ch0, vx);
+      if (mode == GDN2_GATES_FULL) {
+        load8_f32(a.b + gt * D + ch0, bx);
+        load8_f32(a.w + gt * D + ch0, wx);
+      } else {
+        const float beta = __ldg(a.b + gt);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) { bx[c] = beta; wx[c] = beta; }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        ex[c] = bx[c] * kx[c];
+        zx[c] = wx[c] * vx[c];
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) { kx[c] = 0.f; qx[c] = 0.f; ex[c] = 0.f; zx[c] = 0.f; }
+    }
+    float o_eb[8], o_qb[8], o_ke[8], o_em[8], o_qm[8], o_km[8], o_x1[8], o_x2[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      // in-quarter forward inclusive (fw) and backward exclusive (bw) products
+      float fw = al[m][c];
+#pragma unroll
+      for (int dd = 1; dd < 16; dd <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, fw, dd, 16);
+        if (r16 >= dd) fw *= y;
+      }
+      float bi_ = al[m][c];
+#pragma unroll
+      for (int dd = 1; dd < 16; dd <<= 1) {
+        const float y = __shfl_down_sync(0xffffffffu, bi_, dd, 16);
+        if (r16 + dd < 16) bi_ *= y;
+      }
+      float bw = __shfl_down_sync(0xffffffffu, bi_, 1, 16);
+      if (r16 == 15) bw = 1.f;
+      float pre = 1.f, suf = 1.f;
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        if (mm < m) pre *= sPq[mm * D + ch0 + c];
+        if (mm > m) suf *= sPq[mm * D + ch0 + c];
+      }
+      const float g = pre * fw;          // γ_i
+      const float bk = bw * suf;         // Π_{i<s≤63} α
+      o_eb[c] = ex[c] * g;
+      o_qb[c] = qx[c] * g;
+      o_ke[c] = kx[c] * bk;
+      float fe, fk;
+      if ((m & 1) == 0) {
+        fe = __fdividef(1.f, bw);
+        fk = bw;
+      } else {
+        fe = fw;
+        fk = __fdividef(1.f, fw);
+      }
+      o_em[c] = ex[c] * fe;
+      o_qm[c] = qx[c] * fe;
+      o_km[c] = kx[c] * fk;
+      if (m >= 2) {
+        const float fq = (m == 3 ? sPq[2 * D + ch0 + c] : 1.f) * fw;
+        o_x1[c] = ex[c] * fq;
+        o_x2[c] = qx[c] * fq;
+      } else {
+        const float fb = bw * (m == 0 ? sPq[D + ch0 + c] : 1.f);
+        o_x1[c] = kx[c] * fb;
+        o_x2[c] = 0.f;
+      }
+    }
+    *reinterpret_cast<uint4*>(slot + SL_QB + tile_off(i, ch0, D)) = pack8_f16(o_qb);
+    *reinterpret_cast<uint4*>(slot + SL_KE + tile_off(i, ch0, D)) = pack8_f16(o_ke);
+    st16(smem + P_EB, tile_off(i, ch0, D), pack8_f16(o_eb));
+    st16(smem + P_Z, tile_off(i, ch0, D), pack8_f16(zx));
+    st16(smem + P_GM, tile_off(i, ch0, D), pack8(o_em, gram_bf16));
+    st16(smem + P_GM, tile_off(64 + i, ch0, D), pack8(o_qm, gram_bf16));
+    st16(smem + P_KM, tile_off(i, ch0, D), pack8(o_km, gram_bf16));
+    if (m >= 2) {
+      st16(smem + P_GB, tile_off(i, ch0, D), pack8(o_x1, gram_bf16));
+      st16(smem + P_GB, tile_off(64 + i, ch0, D), pack8(o_x2, gram_bf16));
+    } else {
+      st16(smem + P_KB, tile_off(i, ch0, D), pack8(o_x1, gram_bf16));
+    }
+  }
+  sync_for_mma();
+
+  // -------- Gram MMAs: [T; Aqk] candidates
+  uint32_t phase = 0;
+  if (tid == 0) {
+    const uint32_t gm = smem_u32(smem + P_GM), km = smem_u32(smem + P_KM);
+    const uint32_t gb = smem_u32(smem + P_GB), kb = smem_u32(smem + P_KB);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      mma16(tmem + PT_GM, desc_kmajor(gm + ks * 256, D), desc_kmajor(km + ks * 256, D),
+            idesc_16(128, 64, false, false, gram_bf16), ks > 0);
+      mma16(tmem + PT_GB, desc_kmajor(gb + ks * 256, D), desc_kmajor(kb + ks * 256, D),
+            idesc_16(128, 32, false, false, gram_bf16), ks > 0);
+    }
+    mma_commit(bar);
+  }
+  __syncwarp();
+  wait_mma(bar, phase, sflag);
+
+  // -------- T (fp32, shared) and Aqk (fp16, workspace) from TMEM
+  float* sT = reinterpret_cast<float*>(smem + P_T);
+  float* sI = reinterpret_cast<float*>(smem + P_I);
+  float* sX = reinterpret_cast<float*>(smem + P_X);
+  const int lq = warp & 3;
+  const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
+  const int row = lq * 32 + lane;
+  const bool lo = warp < 4;
+  {
+    // lanes 0..63: rows of T; lanes 64..127: rows of Aqk. Warps 0-3 take
+    // columns 0..31, warps 4-7 columns 32..63.
+    const bool is_t = row < 64;
+    const int i = row & 63;
+    const int j0 = lo ? 0 : 32;
+#pragma unroll
+    for (int jb = 0; jb < 32; jb += 16) {
+      float dm[16], db[16];
+      tmem_ld16(t_lane + PT_GM + j0 + jb, dm);
+      tmem_ld16(t_lane + PT_GB + jb, db);
+      tmem_wait_ld();
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int j = j0 + jb + u;
+        const bool keep = is_t ? (j < i) : (j <= i);
+        const bool same = (j >> 5) == (i >> 5);
+        const float x = same ? dm[u] : (j0 == 0 ? db[u] : 0.f);
+        v[u] = keep ? x : 0.f;
+      }
+      if (is_t) {
+#pragma unroll
+        for (int u = 0; u < 16; u += 4)
+          *reinterpret_cast<float4*>(sT + i * TS + j0 + jb + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+      } else {
+        *reinterpret_cast<uint4*>(slot + SL_AQ + tile_off(i, j0 + jb, C)) = pack8_f16(v);
+        *reinterpret_cast<uint4*>(slot + SL_AQ + tile_off(i, j0 + jb + 8, C)) = pack8_f16(v + 8);
+      }
+    }
+  }
+  __syncthreads();
+
+  // -------- A = (I + T)⁻¹, blocked
+  // level 0: the four 16 × 16 diagonal blocks by forward substitution, one
+  // column per thread; the other threads zero the two upper-right 16 × 16
+  // blocks of the 32-halves (read by the level-2 products).
+  if (tid < 64) {
+    const int blk = tid >> 4, j = tid & 15, base = blk * 16;
+    float x[16];
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) {
+      float acc = (ii == j) ? 1.f : 0.f;
+#pragma unroll
+      for (int l = 0; l < ii; ++l)
+        if (l >= j) acc -= sT[(base + ii) * TS + base + l] * x[l];
+      x[ii] = (ii >= j) ? acc : 0.f;
+    }
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) sI[(base + ii) * TS + base + j] = x[ii];
+  } else {
+    for (int o = tid - 64; o < 512; o += NT - 64) {
+      const int hf = o >> 8, ii = (o >> 4) & 15, jj = o & 15;
+      sI[(hf * 32 + ii) * TS + hf * 32 + 16 + jj] = 0.f;
+    }
+  }
+  __syncthreads();
+  // level 1: X21 = −I22 T21 I11 in each 32-half (thread: 4 columns)
+  if (tid < 128) {
+    const int hf = tid >> 6, ii = (tid >> 2) & 15, jq = (tid & 3) * 4;
+    const int r0 = hf * 32 + 16, c0 = hf * 32;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int l = 0; l < 16; ++l) {
+      const float t = sT[(r0 + ii) * TS + c0 + l];
+      const float4 iv = *reinterpret_cast<const float4*>(sI + (c0 + l) * TS + c0 + jq);
+      acc[0] += t * iv.x; acc[1] += t * iv.y; acc[2] += t * iv.z; acc[3] += t * iv.w;
+    }
+    *reinterpret_cast<float4*>(sX + (hf * 16 + ii) * 36 + jq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
+  __syncthreads();
+  if (tid < 128) {
+    const int hf = tid >> 6, ii = (tid >> 2) & 15, jq = (tid & 3) * 4;
+    const int r0 = hf * 32 + 16, c0 = hf * 32;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int l = 0; l < 16; ++l) {
+      const float t = sI[(r0 + ii) * TS + r0 + l];
+      const float4 xv = *reinterpret_cast<const float4*>(sX + (hf * 16 + l) * 36 + jq);
+      acc[0] += t * xv.x; acc[1] += t * xv.y; acc[2] += t * xv.z; acc[3] += t * xv.w;
+    }
+    *reinterpret_cast<float4*>(sI + (r0 + ii) * TS + c0 + jq) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+  }
+  __syncthreads();
+  // level 2: X_QP = −I_QQ T_QP I_PP (thread: row ii, 4 columns)
+  {
+    const int ii = tid >> 3, jq = (tid & 7) * 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int l = 0; l < 32; ++l) {
+      const float t = sT[(32 + ii) * TS + l];
+      const float4 iv = *reinterpret_cast<const float4*>(sI + l * TS + jq);
+      acc[0] += t * iv.x; acc[1] += t * iv.y; acc[2] += t * iv.z; acc[3] += t * iv.w;
+    }
+    *reinterpret_cast<float4*>(sX + ii * 36 + jq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
+  __syncthreads();
+  {
+    const int ii = tid >> 3, jq = (tid & 7) * 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int l = 0; l < 32; ++l) {
+      const float t = sI[(32 + ii) * TS + 32 + l];
+      const float4 xv = *reinterpret_cast<const float4*>(sX + l * 36 + jq);
+      acc[0] += t * xv.x; acc[1] += t * xv.y; acc[2] += t * xv.z; acc[3] += t * xv.w;
+    }
+    *reinterpret_cast<float4*>(sI + (32 + ii) * TS + jq) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+  }
+  __syncthreads();
+  // pack A (lower triangle; zeros above the diagonal)
+  for (int o = tid; o < C * 8; o += NT) {
+    const int i = o >> 3, j0 = (o & 7) * 8;
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = (j0 + u <= i) ? sI[i * TS + j0 + u] : 0.f;
+    st16(smem + P_AINV, tile_off(i, j0, C), pack8_f16(x));
+  }
+  sync_for_mma();
+
+  // -------- Yᵀ = Ēᵀ Aᵀ, U_wᵀ = Zᵀ Aᵀ
+  if (tid == 0) {
+    const uint32_t eb = smem_u32(smem + P_EB), z = smem_u32(smem + P_Z);
+    const uint32_t ai = smem_u32(smem + P_AINV);
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      const uint64_t bdesc = desc_kmajor(ai + ks * 256, C);
+      mma16(tmem + PT_YT, desc_mnmajor(eb + ks * 2 * (D / 8) * 128, D), bdesc, idesc_f16(128, 64, true, false),
+            ks > 0);
+      mma16(tmem + PT_UW, desc_mnmajor(z + ks * 2 * (D / 8) * 128, D), bdesc, idesc_f16(128, 64, true, false),
+            ks > 0);
+    }
+    mma_commit(bar);
+  }
+  __syncwarp();
+  wait_mma(bar, phase, sflag);
+  {
+    // warps 0-3: Yᵀ rows (key lanes); warps 4-7: U_wᵀ rows (dv lanes)
+    const uint32_t col = lo ? PT_YT : PT_UW;
+    uint8_t* dst = slot + (lo ? SL_YT : SL_UW);
+#pragma unroll
+    for (int cb = 0; cb < C; cb += 16) {
+      float v[16];
+      tmem_ld16(t_lane + col + cb, v);
+      tmem_wait_ld();
+      *reinterpret_cast<uint4*>(dst + tile_off(row, cb, C)) = pack8_f16(v);
+      *reinterpret_cast<uint4*>(dst + tile_off(row, cb + 8, C)) = pack8_f16(v + 8);
+    }
+  }
+  if (*sflag && tid == 0) atomicOr(static_cast<int*>(a.workspace), 1);
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, PT_COLS);
+}
+
+// =============================================================================
+// scan kernel: one CTA per (sequence, value head), chunks of the segment in order
+// =============================================================================
+template <typename TOut>
+__global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, const float* S_in,
+                                                           float* S_out) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S_BAR);
+  uint64_t* mbar = full + 2;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + S_TMEMP);
+  int* sflag = reinterpret_cast<int*>(smem + S_FLAG);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  const int h = bh % a.Hv, bi = bh / a.Hv;
+  const uint8_t* slots = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + (size_t)bh * n_seg * SLOT;
+  TOut* og = static_cast<TOut*>(a.o);
+
+  if (tid == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_init(mbar, 1);
+    fence_mbar_init();
+    *sflag = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_ptr, ST_COLS);
     tmem_relinquish();
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_ptr;
-  uint32_t phase = 0;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&full[0], SLOT_USED);
+    bulk_g2s(smem + S_STAGE0, slots, SLOT_USED, &full[0]);
+  }
 
-  // TMEM lane quarter of this warp and the row this thread owns there.
   const int lq = warp & 3;
   const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
-  const int row = lq * 32 + lane;          // dv index (or key / token-row index)
-  const bool lo = warp < 4;                // warps 0-3: first column half; 4-7: second
+  const int row = lq * 32 + lane;       // dv index j of Sᵀ[j][*]
+  const bool lo = warp < 4;
 
-  // ---------------------------------------------------------------- entry state
+  // entry state: Sᵀ[j][c] = S[c][j]
   {
-    // Thread (row = dv j) owns Sᵀ[j][*] = S[*][j]; each warp pair splits the 128 key columns.
     const int c0 = lo ? 0 : 64;
-    const float* S0 = a.S0 ? a.S0 + (size_t)bh * D * D : nullptr;
+    const float* S0 = S_in ? S_in + (size_t)bh * D * D : nullptr;
     for (int cb = c0; cb < c0 + 64; cb += 16) {
       float v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) v[u] = S0 ? __ldg(S0 + (size_t)(cb + u) * D + row) : 0.f;
-      tmem_st16(t_lane + TM_S + cb, v);
-      st16(smem + OFF_ST, tile_off(row, cb, D), pack8_f16(v));
-      st16(smem + OFF_ST, tile_off(row, cb + 8, D), pack8_f16(v + 8));
+      tmem_st16(t_lane + ST_S + cb, v);
+      st16(smem + S_ST, tile_off(row, cb, D), pack8_f16(v));
+      st16(smem + S_ST, tile_off(row, cb + 8, D), pack8_f16(v + 8));
     }
     tmem_wait_st();
   }
+  sync_for_mma();
 
-  const int nchunks = (a.T + C - 1) / C;
-  // Element mapping of the load/elementwise passes: lane r = token within a
-  // 16-token quarter, 8 channels per thread.
-  const int r16 = lane & 15;
-  const int cg = 2 * warp + (lane >> 4);
-  const int ch0 = cg * 8;
-
-  for (int ck = 0; ck < nchunks; ++ck) {
-    const int t0 = ck * C;
+  uint32_t mphase = 0;
+  int issued = 1;                       // bulk copies issued (for the error path)
+  int waited = 0;
+  for (int cl = 0; cl < n_seg; ++cl) {
+    const int s = cl & 1;
+    uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
+    const int t0 = (c_begin + cl) * C;
     const int Lc = min(C, a.T - t0);
-
-    // ------------------------------------------------ pass 1: α quarter products
-    float fw[4][8], bw[4][8], Pq[4][8];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int i = 16 * m + r16;
-      const int t = t0 + i;
-      float al[8];
-      if (i < Lc) {
-        const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
-        if (mode == GDN2_GATES_GDN) {
-          const float s = __ldg(a.alpha + gt);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) al[c] = s;
-        } else {
-          load8_f32(a.alpha + gt * D + ch0, al);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) al[c] = 1.f;
+    if (!mbar_wait(&full[s], (cl >> 1) & 1)) atomicOr(sflag, 1);
+    ++waited;
+    // prefetch the next chunk into the other stage (free: its MMAs and reads
+    // finished before the barrier that closed the previous iteration)
+    if (cl + 1 < n_seg) {
+      if (tid == 0) {
+        uint8_t* nstg = smem + (s ? S_STAGE0 : S_STAGE1);
+        mbar_arrive_expect_tx(&full[s ^ 1], SLOT_USED);
+        bulk_g2s(nstg, slots + (size_t)(cl + 1) * SLOT, SLOT_USED, &full[s ^ 1]);
       }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float x = al[c];   // forward inclusive product within the quarter
-#pragma unroll
-        for (int dd = 1; dd < 16; dd <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, x, dd, 16);
-          if (r16 >= dd) x *= y;
-        }
-        fw[m][c] = x;
-        Pq[m][c] = __shfl_sync(0xffffffffu, x, 15, 16);
-        float z = al[c];   // backward inclusive product within the quarter
-#pragma unroll
-        for (int dd = 1; dd < 16; dd <<= 1) {
-          const float y = __shfl_down_sync(0xffffffffu, z, dd, 16);
-          if (r16 + dd < 16) z *= y;
-        }
-        const float zn = __shfl_down_sync(0xffffffffu, z, 1, 16);
-        bw[m][c] = (r16 == 15) ? 1.f : zn;   // exclusive: Π_{s>i} within the quarter
-      }
+      ++issued;
     }
-    if (r16 == 0) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) sgC[ch0 + c] = Pq[0][c] * Pq[1][c] * Pq[2][c] * Pq[3][c];
-    }
-    // Smallest decay product whose reciprocal enters a Gram factor: fp16 Gram
-    // operands when every factor stays below 2^14.
-    bool gram_bf16;
-    {
-      float mn = 1.f;
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mn = fminf(mn, (m & 1) ? fw[m][c] : bw[m][c]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-      float* sred = reinterpret_cast<float*>(smem + OFF_RED);
-      if (lane == 0) sred[warp] = mn;
-      __syncthreads();
-      float mall = sred[0];
-#pragma unroll
-      for (int w_ = 1; w_ < 8; ++w_) mall = fminf(mall, sred[w_]);
-      gram_bf16 = !(mall > 6.103515625e-05f);   // 2^-14
-    }
-
-    // ------------------------------------------------ pass 2: operand tiles
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int i = 16 * m + r16;
-      const int t = t0 + i;
-      float kx[8], qx[8], ex[8], zx[8];
-      if (i < Lc) {
-        const size_t tq = ((size_t)bi * a.T + t) * a.Hqk + hq;
-        const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
-        load8_bf16(kg + tq * D + ch0, kx);
-        load8_bf16(qg + tq * D + ch0, qx);
-        float bx[8], wx[8], vx[8];
-        load8_bf16(vg + gt * D + ch0, vx);
-        if (mode == GDN2_GATES_FULL) {
-          load8_f32(a.b + gt * D + ch0, bx);
-          load8_f32(a.w + gt * D + ch0, wx);
-        } else {
-          const float beta = __ldg(a.b + gt);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) { bx[c] = beta; wx[c] = beta; }
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          ex[c] = bx[c] * kx[c];
-          zx[c] = wx[c] * vx[c];
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) { kx[c] = 0.f; qx[c] = 0.f; ex[c] = 0.f; zx[c] = 0.f; }
-      }
-      float o_eb[8], o_qb[8], o_ke[8], o_em[8], o_qm[8], o_km[8], o_x1[8], o_x2[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float pre = 1.f, suf = 1.f;
-#pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-          if (mm < m) pre *= Pq[mm][c];
-          if (mm > m) suf *= Pq[mm][c];
-        }
-        const float g = pre * fw[m][c];          // γ_i
-        const float bk = bw[m][c] * suf;          // Π_{i<s≤63} α
-        o_eb[c] = ex[c] * g;
-        o_qb[c] = qx[c] * g;
-        o_ke[c] = kx[c] * bk;
-        // reference at the quarter boundary inside the half
-        float fe, fk;
-        if ((m & 1) == 0) {
-          fe = __fdividef(1.f, bw[m][c]);
-          fk = bw[m][c];
-        } else {
-          fe = fw[m][c];
-          fk = __fdividef(1.f, fw[m][c]);
-        }
-        o_em[c] = ex[c] * fe;
-        o_qm[c] = qx[c] * fe;
-        o_km[c] = kx[c] * fk;
-        // reference at the half boundary (token 31 | 32)
-        if (m >= 2) {
-          const float fq = (m == 3 ? Pq[2][c] : 1.f) * fw[m][c];
-          o_x1[c] = ex[c] * fq;   // Ē_bnd
-          o_x2[c] = qx[c] * fq;   // Q̄_bnd
-        } else {
-          const float fb = bw[m][c] * (m == 0 ? Pq[1][c] : 1.f);
-          o_x1[c] = kx[c] * fb;   // K̃_bnd
-          o_x2[c] = 0.f;
-        }
-      }
-      st16(smem + OFF_EB, tile_off(i, ch0, D), pack8_f16(o_eb));
-      st16(smem + OFF_QB, tile_off(i, ch0, D), pack8_f16(o_qb));
-      st16(smem + OFF_KE, tile_off(i, ch0, D), pack8_f16(o_ke));
-      st16(smem + OFF_Z, tile_off(i, ch0, D), pack8_f16(zx));
-      st16(smem + OFF_GM, tile_off(i, ch0, D), pack8(o_em, gram_bf16));
-      st16(smem + OFF_GM, tile_off(64 + i, ch0, D), pack8(o_qm, gram_bf16));
-      st16(smem + OFF_KM, tile_off(i, ch0, D), pack8(o_km, gram_bf16));
-      if (m >= 2) {
-        st16(smem + OFF_GB, tile_off(i, ch0, D), pack8(o_x1, gram_bf16));
-        st16(smem + OFF_GB, tile_off(64 + i, ch0, D), pack8(o_x2, gram_bf16));
-      } else {
-        st16(smem + OFF_KB, tile_off(i, ch0, D), pack8(o_x1, gram_bf16));
-      }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-
-    // ------------------------------------------------ Gram MMAs
+    // (Y S)ᵀ = Sᵀ Yᵀ and Oᵀ = Sᵀ Q̄ᵀ
     if (tid == 0) {
-      const uint32_t gm = smem_u32(smem + OFF_GM), km = smem_u32(smem + OFF_KM);
-      const uint32_t gb = smem_u32(smem + OFF_GB), kb = smem_u32(smem + OFF_KB);
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        mma16(tmem + TM_GM, desc_kmajor(gm + ks * 256, D), desc_kmajor(km + ks * 256, D),
-              idesc_16(128, 64, false, false, gram_bf16), ks > 0);
-        mma16(tmem + TM_GB, desc_kmajor(gb + ks * 256, D), desc_kmajor(kb + ks * 256, D),
-              idesc_16(128, 32, false, false, gram_bf16), ks > 0);
-      }
-      mma_commit(bar);
-    }
-    __syncwarp();
-    wait_mma(bar, phase, sflag);
-
-    // ------------------------------------------------ T and Aqk from TMEM
-    float* sT = reinterpret_cast<float*>(smem + OFF_T);
-    if (warp < 4) {
-      // lanes 0..63: T rows; lanes 64..127: Aqk rows
-      const bool is_t = row < 64;
-      const int i = row & 63;
-      float dm[64], db[32];
-#pragma unroll
-      for (int cb = 0; cb < 64; cb += 16) tmem_ld16(t_lane + TM_GM + cb, dm + cb);
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) tmem_ld16(t_lane + TM_GB + cb, db + cb);
-      tmem_wait_ld();
-      float val[64];
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const bool keep = is_t ? (j < i) : (j <= i);
-        const bool same = (j >> 5) == (i >> 5);
-        float x = same ? dm[j] : (j < 32 ? db[j & 31] : 0.f);
-        val[j] = keep ? x : 0.f;
-      }
-      if (is_t) {
-#pragma unroll
-        for (int j = 0; j < 64; ++j) sT[i * TP + j] = val[j];
-      } else {
-#pragma unroll
-        for (int j = 0; j < 64; j += 8) st16(smem + OFF_AQK, tile_off(i, j, C), pack8_f16(val + j));
-      }
-    }
-    __syncthreads();
-
-    // ------------------------------------------------ A = (I + T)⁻¹, blocked
-    float* sI = reinterpret_cast<float*>(smem + OFF_INV);
-    float* sX = reinterpret_cast<float*>(smem + OFF_TMP);
-    // zero the strict upper triangle region we never write otherwise
-    for (int idx = tid; idx < C * C; idx += NT) {
-      const int i = idx >> 6, j = idx & 63;
-      if (j > i) sI[i * TP + j] = 0.f;
-    }
-    // level 0: 16 × 16 diagonal blocks by forward substitution, one column per thread
-    if (tid < 64) {
-      const int blk = tid >> 4, j = tid & 15, base = blk * 16;
-      float x[16];
-#pragma unroll
-      for (int ii = 0; ii < 16; ++ii) {
-        float acc = (ii == j) ? 1.f : 0.f;
-        if (ii > j) {
-#pragma unroll
-          for (int l = 0; l < 16; ++l)
-            if (l >= j && l < ii) acc -= sT[(base + ii) * TP + base + l] * x[l];
-        }
-        x[ii] = (ii >= j) ? acc : 0.f;
-      }
-#pragma unroll
-      for (int ii = 0; ii < 16; ++ii) sI[(base + ii) * TP + base + j] = x[ii];
-    }
-    __syncthreads();
-    // level 1: off-diagonal 16 × 16 block of each 32-half: X = −I22 T21 I11
-    {
-      // tmp = T21 · I11 for both halves: 2 × 256 outputs
-      for (int o = tid; o < 512; o += NT) {
-        const int hf = o >> 8, ii = (o >> 4) & 15, jj = o & 15;
-        const int r0 = hf * 32 + 16, c0 = hf * 32;
-        float acc = 0.f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l) acc += sT[(r0 + ii) * TP + c0 + l] * sI[(c0 + l) * TP + c0 + jj];
-        sX[(r0 + ii) * TP + c0 + jj] = acc;
-      }
-      __syncthreads();
-      for (int o = tid; o < 512; o += NT) {
-        const int hf = o >> 8, ii = (o >> 4) & 15, jj = o & 15;
-        const int r0 = hf * 32 + 16, c0 = hf * 32;
-        float acc = 0.f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l) acc += sI[(r0 + ii) * TP + r0 + l] * sX[(r0 + l) * TP + c0 + jj];
-        sI[(r0 + ii) * TP + c0 + jj] = -acc;
-      }
-      __syncthreads();
-    }
-    // level 2: lower-left 32 × 32 block: X = −I_QQ T_QP I_PP
-    {
-      for (int o = tid; o < 1024; o += NT) {
-        const int ii = o >> 5, jj = o & 31;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) acc += sT[(32 + ii) * TP + l] * sI[l * TP + jj];
-        sX[(32 + ii) * TP + jj] = acc;
-      }
-      __syncthreads();
-      for (int o = tid; o < 1024; o += NT) {
-        const int ii = o >> 5, jj = o & 31;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int l = 0; l < 32; ++l) acc += sI[(32 + ii) * TP + 32 + l] * sX[(32 + l) * TP + jj];
-        sI[(32 + ii) * TP + jj] = -acc;
-      }
-      __syncthreads();
-    }
-    // pack A (fp16, [i][j], 64 columns)
-    for (int o = tid; o < C * 8; o += NT) {
-      const int i = o >> 3, j0 = (o & 7) * 8;
-      float x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = sI[i * TP + j0 + u];
-      st16(smem + OFF_AINV, tile_off(i, j0, C), pack8_f16(x));
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-
-    // ------------------------------------------------ Yᵀ = Ēᵀ Aᵀ, U_wᵀ = Zᵀ Aᵀ
-    if (tid == 0) {
-      const uint32_t eb = smem_u32(smem + OFF_EB), z = smem_u32(smem + OFF_Z);
-      const uint32_t ai = smem_u32(smem + OFF_AINV);
-#pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks) {
-        const uint64_t bdesc = desc_kmajor(ai + ks * 256, C);
-        mma16(tmem + TM_YT, desc_mnmajor(eb + ks * 2 * (D / 8) * 128, D), bdesc,
-                 idesc_f16(128, 64, true, false), ks > 0);
-        mma16(tmem + TM_UW, desc_mnmajor(z + ks * 2 * (D / 8) * 128, D), bdesc,
-                 idesc_f16(128, 64, true, false), ks > 0);
-      }
-      mma_commit(bar);
-    }
-    __syncwarp();
-    wait_mma(bar, phase, sflag);
-
-    // Yᵀ (TMEM, key lanes) → fp16 tile [key][tok] (an MN-major B operand)
-    {
-      const int c0 = lo ? 0 : 32;
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        float v[16];
-        tmem_ld16(t_lane + TM_YT + c0 + cb, v);
-        tmem_wait_ld();
-        st16(smem + OFF_YT, tile_off(row, c0 + cb, C), pack8_f16(v));
-        st16(smem + OFF_YT, tile_off(row, c0 + cb + 8, C), pack8_f16(v + 8));
-      }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-
-    // ------------------------------------------------ (Y S)ᵀ = Sᵀ Yᵀ, Oᵀ = Sᵀ Q̄ᵀ
-    if (tid == 0) {
-      const uint32_t st = smem_u32(smem + OFF_ST), yt = smem_u32(smem + OFF_YT);
-      const uint32_t qb = smem_u32(smem + OFF_QB);
+      const uint32_t st = smem_u32(smem + S_ST);
+      const uint32_t yt = smem_u32(stg + SL_YT), qb = smem_u32(stg + SL_QB);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint64_t adesc = desc_kmajor(st + ks * 256, D);
-        mma16(tmem + TM_YS, adesc, desc_mnmajor(yt + ks * 2 * (C / 8) * 128, C),
-                 idesc_f16(128, 64, false, true), ks > 0);
-        mma16(tmem + TM_O, adesc, desc_kmajor(qb + ks * 256, D), idesc_f16(128, 64, false, false), ks > 0);
+        mma16(tmem + ST_YS, adesc, desc_mnmajor(yt + ks * 2 * (C / 8) * 128, C), idesc_f16(128, 64, false, true),
+              ks > 0);
+        mma16(tmem + ST_O, adesc, desc_kmajor(qb + ks * 256, D), idesc_f16(128, 64, false, false), ks > 0);
       }
-      mma_commit(bar);
+      mma_commit(mbar);
     }
-    // meanwhile: Sᵀ ← Sᵀ Γ in TMEM (column c scaled by γ_C[c]); the running MMAs
-    // read only the fp16 copy.
+    // meanwhile Sᵀ ← Sᵀ Γ in TMEM (column c scaled by γ_C[c])
     {
+      const float* gC = reinterpret_cast<const float*>(stg + SL_GC);
       const int c0 = lo ? 0 : 64;
       for (int cb = c0; cb < c0 + 64; cb += 16) {
         float v[16];
-        tmem_ld16(t_lane + TM_S + cb, v);
+        tmem_ld16(t_lane + ST_S + cb, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] *= sgC[cb + u];
-        tmem_st16(t_lane + TM_S + cb, v);
+        for (int u = 0; u < 16; ++u) v[u] *= gC[cb + u];
+        tmem_st16(t_lane + ST_S + cb, v);
       }
       tmem_wait_st();
     }
     __syncwarp();
-    wait_mma(bar, phase, sflag);
-
-    // Uᵀ = U_wᵀ − (Y S)ᵀ → fp16 tile [dv][tok] (K-major A operand)
+    wait_mma(mbar, mphase, sflag);
+    // Uᵀ = U_wᵀ − (Y S)ᵀ
     {
       const int c0 = lo ? 0 : 32;
 #pragma unroll
       for (int cb = 0; cb < 32; cb += 16) {
-        float uw[16], ys[16];
-        tmem_ld16(t_lane + TM_UW + c0 + cb, uw);
-        tmem_ld16(t_lane + TM_YS + c0 + cb, ys);
+        float ys[16], uw[16];
+        tmem_ld16(t_lane + ST_YS + c0 + cb, ys);
+        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + tile_off(row, c0 + cb, C)), uw);
+        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + tile_off(row, c0 + cb + 8, C)), uw + 8);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u) uw[u] -= ys[u];
-        st16(smem + OFF_UT, tile_off(row, c0 + cb, C), pack8_f16(uw));
-        st16(smem + OFF_UT, tile_off(row, c0 + cb + 8, C), pack8_f16(uw + 8));
+        st16(smem + S_UT, tile_off(row, c0 + cb, C), pack8_f16(uw));
+        st16(smem + S_UT, tile_off(row, c0 + cb + 8, C), pack8_f16(uw + 8));
       }
     }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-
-    // ------------------------------------------------ Sᵀ += Uᵀ K_end, Oᵀ += Uᵀ Aqkᵀ
+    sync_for_mma();
+    // Sᵀ += Uᵀ K_end, Oᵀ += Uᵀ Aqkᵀ
     if (tid == 0) {
-      const uint32_t ut = smem_u32(smem + OFF_UT), ke = smem_u32(smem + OFF_KE);
-      const uint32_t aq = smem_u32(smem + OFF_AQK);
+      const uint32_t ut = smem_u32(smem + S_UT);
+      const uint32_t ke = smem_u32(stg + SL_KE), aq = smem_u32(stg + SL_AQ);
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks) {
         const uint64_t adesc = desc_kmajor(ut + ks * 256, C);
-        mma16(tmem + TM_S, adesc, desc_mnmajor(ke + ks * 2 * (D / 8) * 128, D),
-                 idesc_f16(128, 128, false, true), 1);
-        mma16(tmem + TM_O, adesc, desc_kmajor(aq + ks * 256, C), idesc_f16(128, 64, false, false), 1);
+        mma16(tmem + ST_S, adesc, desc_mnmajor(ke + ks * 2 * (D / 8) * 128, D), idesc_f16(128, 128, false, true), 1);
+        mma16(tmem + ST_O, adesc, desc_kmajor(aq + ks * 256, C), idesc_f16(128, 64, false, false), 1);
       }
-      mma_commit(bar);
+      mma_commit(mbar);
     }
     __syncwarp();
-    wait_mma(bar, phase, sflag);
-
-    // outputs: thread (dv j) writes o[t0 + i][h][j]
+    wait_mma(mbar, mphase, sflag);
+    // outputs o[t0 + i][h][j]
     {
       const int c0 = lo ? 0 : 32;
       TOut* orow = og + (((size_t)bi * a.T + t0) * a.Hv + h) * D + row;
@@ -575,7 +676,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(ChunkArgs a) {
 #pragma unroll
       for (int cb = 0; cb < 32; cb += 16) {
         float v[16];
-        tmem_ld16(t_lane + TM_O + c0 + cb, v);
+        tmem_ld16(t_lane + ST_O + c0 + cb, v);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
@@ -589,36 +690,39 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(ChunkArgs a) {
       const int c0 = lo ? 0 : 64;
       for (int cb = c0; cb < c0 + 64; cb += 16) {
         float v[16];
-        tmem_ld16(t_lane + TM_S + cb, v);
+        tmem_ld16(t_lane + ST_S + cb, v);
         tmem_wait_ld();
-        st16(smem + OFF_ST, tile_off(row, cb, D), pack8_f16(v));
-        st16(smem + OFF_ST, tile_off(row, cb + 8, D), pack8_f16(v + 8));
+        st16(smem + S_ST, tile_off(row, cb, D), pack8_f16(v));
+        st16(smem + S_ST, tile_off(row, cb + 8, D), pack8_f16(v + 8));
       }
     }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
+    sync_for_mma();
     if (*sflag) break;
   }
 
-  // ---------------------------------------------------------------- final state
-  if (a.ST && !*sflag) {
+  if (S_out && !*sflag) {
     const int c0 = lo ? 0 : 64;
-    float* ST = a.ST + (size_t)bh * D * D;
+    float* ST = S_out + (size_t)bh * D * D;
     for (int cb = c0; cb < c0 + 64; cb += 16) {
       float v[16];
-      tmem_ld16(t_lane + TM_S + cb, v);
+      tmem_ld16(t_lane + ST_S + cb, v);
       tmem_wait_ld();
 #pragma unroll
       for (int u = 0; u < 16; ++u) ST[(size_t)(cb + u) * D + row] = v[u];
     }
   }
-  if (*sflag && tid == 0 && a.workspace) atomicOr(static_cast<int*>(a.workspace), 1);
+  if (*sflag && tid == 0) {
+    atomicOr(static_cast<int*>(a.workspace), 1);
+    // after an early exit a prefetched bulk copy may still be in flight:
+    // wait for it (bounded) before this CTA's shared memory is released
+    if (issued > waited) mbar_wait(&full[waited & 1], (waited >> 1) & 1, 1u << 16);
+  }
   fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+  if (warp == 0) tmem_dealloc(tmem, ST_COLS);
 }
+
+size_t state_bytes(const ChunkArgs& a) { return (size_t)a.B * a.Hv * D * D * sizeof(float); }
 
 }  // namespace
 
@@ -626,24 +730,53 @@ bool chunk_tc_supported(const ChunkArgs& a, int qkv_bf16) {
   return qkv_bf16 && a.dk == D && a.dv == D && a.chunk == C && a.conv_w == nullptr && !a.l2norm;
 }
 
-size_t chunk_tc_workspace(const ChunkArgs&) { return 256; }
+// Workspace for the whole sequence in one segment.
+size_t chunk_tc_workspace(const ChunkArgs& a) {
+  const size_t nchunks = (a.T + C - 1) / C;
+  return WS_HEAD + (size_t)a.B * a.Hv * nchunks * SLOT;
+}
 
+size_t chunk_tc_min_workspace(const ChunkArgs& a, bool carry_state) {
+  return WS_HEAD + (size_t)a.B * a.Hv * SLOT + (carry_state ? state_bytes(a) : 0);
+}
+
+// Runs the chunks in segments when the workspace holds fewer chunk slots than
+// the sequence has; the state is carried between segments through S_T (or,
+// when S_T is NULL, through the end of the workspace).
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
-  const int grid = a.B * a.Hv;
+  const int BH = a.B * a.Hv;
+  const int nchunks = (a.T + C - 1) / C;
+  if (a.ws_bytes < WS_HEAD) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(a.workspace, 0, sizeof(int), s);
-  if (e != cudaSuccess || grid == 0) return e;
-  if (o_bf16) {
-    auto k = chunk_tc_kernel<__nv_bfloat16>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    k<<<grid, NT, SMEM_BYTES, s>>>(a);
-  } else {
-    auto k = chunk_tc_kernel<float>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    k<<<grid, NT, SMEM_BYTES, s>>>(a);
+  if (e != cudaSuccess || BH == 0 || nchunks == 0) return e;
+  size_t slot_bytes = a.ws_bytes - WS_HEAD;
+  int seg = (int)std::min<size_t>(nchunks, slot_bytes / ((size_t)BH * SLOT));
+  float* carry = a.ST;
+  if (seg < nchunks && carry == nullptr) {
+    const size_t sb = state_bytes(a);
+    slot_bytes = slot_bytes > sb ? slot_bytes - sb : 0;
+    seg = (int)std::min<size_t>(nchunks, slot_bytes / ((size_t)BH * SLOT));
+    carry = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + WS_HEAD + (size_t)BH * seg * SLOT);
   }
-  return cudaGetLastError();
+  if (seg < 1) return cudaErrorInvalidValue;
+
+  if ((e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) !=
+      cudaSuccess)
+    return e;
+  auto scan = o_bf16 ? chunk_scan_kernel<__nv_bfloat16> : chunk_scan_kernel<float>;
+  if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM)) != cudaSuccess) return e;
+
+  const float* s_in = a.S0;
+  for (int c0 = 0; c0 < nchunks; c0 += seg) {
+    const int n = std::min(seg, nchunks - c0);
+    const bool last = c0 + n >= nchunks;
+    float* s_out = last ? a.ST : carry;
+    chunk_prep_kernel<<<BH * n, NT, P_SMEM, s>>>(a, c0, n);
+    scan<<<BH, NT, S_SMEM, s>>>(a, c0, n, s_in, s_out);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    s_in = carry;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace gdn2

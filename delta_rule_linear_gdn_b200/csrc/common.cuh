@@ -51,7 +51,17 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, int qkv_bf16, int o_bf16, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, int qkv_bf16, int o_bf16, cudaStream_t s);
 bool chunk_tc_supported(const ChunkArgs& a, int qkv_bf16);
+// Workspace of the tensor-core path for the whole sequence at once, and the
+// least it can run with (one chunk slot per sequence-head, plus the carried
+// state when S_T is NULL); in between, it runs the sequence in segments.
 size_t chunk_tc_workspace(const ChunkArgs& a);
+size_t chunk_tc_min_workspace(const ChunkArgs& a, bool carry_state);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s);
+
+// gdn2_chunk_fwd after argument checks; `segmented_ok` accepts a workspace
+// between the minimum and the full size.
+gdn2_status chunk_fwd_checked(const gdn2_params* p, const void* q, const void* k, const void* v,
+                              const float* alpha, const float* b, const float* w, const float* S0, void* o,
+                              float* S_T, void* workspace, size_t ws_bytes, void* stream, bool segmented_ok);
 
 }  // namespace gdn2

@@ -14,8 +14,8 @@
 
 namespace {
 
-// Stated maximum scratch of the allocation-free call.
-constexpr size_t kNoAllocScratchBytes = 4096;
+// Stated maximum scratch of the allocation-free call: 32 MiB per GPU.
+constexpr size_t kNoAllocScratchBytes = 32u << 20;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -51,10 +51,12 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_params* p, con
   // Only the tensor-core prefill uses scratch; it is the configuration this
   // call serves (every other configuration runs without scratch through
   // gdn2_chunk_fwd).
-  const size_t need = gdn2_chunk_fwd_workspace(p);
-  if (need == 0) return GDN2_ERR_UNSUPPORTED;
-  if (need > kNoAllocScratchBytes) return GDN2_ERR_WORKSPACE;
+  if (gdn2_chunk_fwd_workspace(p) == 0) return GDN2_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return GDN2_ERR_CUDA;
-  return gdn2_chunk_fwd(p, q, k, v, alpha, b, w, S0, o, S_T, scratch, kNoAllocScratchBytes, stream);
+  // The array holds as many chunks per (sequence, value head) as fit; the
+  // sequence runs in segments of that many chunks. A problem whose single
+  // chunk slot per sequence-head exceeds the array gets GDN2_ERR_WORKSPACE.
+  return gdn2::chunk_fwd_checked(p, q, k, v, alpha, b, w, S0, o, S_T, scratch, kNoAllocScratchBytes, stream,
+                                 /*segmented_ok=*/true);
 }

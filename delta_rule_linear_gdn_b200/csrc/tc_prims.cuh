@@ -159,6 +159,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint3
   return false;
 }
 
+// Arrive on an mbarrier and add `bytes` to the transaction count it waits for.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(bytes)
+               : "memory");
+}
+
+// Bulk (non-tensor) asynchronous copy global → shared of `bytes` (multiple of
+// 16, both addresses 16-byte aligned), completing on `mbar` as transactions.
+// No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_u32(mbar))
+      : "memory");
+}
+
 // Pack 8 floats to 8 bf16 (16 bytes), round to nearest even.
 __device__ __forceinline__ uint4 pack8_bf16(const float* x) {
   uint4 u;

@@ -187,12 +187,12 @@ def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_
     return o
 
 
-def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T, chunk=64, scale=1.0, gate_mode="full",
-                      stream=None):
+def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=64, scale=1.0,
+                      gate_mode="full", stream=None):
     """Chunked prefill through ``gdn2_chunk_fwd_noalloc``: the library takes the
     kernel's scratch from its own fixed device array, so nothing is allocated
-    for the call. ``o`` and ``S_T`` are caller-provided outputs (the caller
-    owns all device memory). Returns (o, S_T)."""
+    for the call. ``o`` and ``S_T`` (or None) are caller-provided outputs (the
+    caller owns all device memory). Returns (o, S_T)."""
     L = lib()
     fn = L.gdn2_chunk_fwd_noalloc
     fn.argtypes = [ctypes.POINTER(Params)] + [ctypes.c_void_p] * 10

@@ -160,7 +160,7 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const
  * gdn2_chunk_fwd for the configurations that run the tensor-core kernel
  * (bf16 q,k,v, d_k = d_v = 128, chunk 64, no conv, no fused L2 norm,
  * GDN2_PREC_DEFAULT), with the kernel's device scratch taken from a fixed
- * 4 KiB array compiled into the library instead of a caller-provided
+ * 32 MiB array compiled into the library instead of a caller-provided
  * workspace. The pages have no counterpart of this call.
  *
  * It exists for callers that cannot hand the library device memory at call
@@ -172,18 +172,23 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const
  *
  *   Arguments: as gdn2_chunk_fwd, without workspace and ws_bytes.
  *   Scratch:   one array per GPU, held from library load until process exit.
- *              The first call on each device looks up the array's device
- *              address (with that device current); make that first call
- *              before any stream capture. Each call clears the status word
- *              it uses before its launch.
+ *              The sequence is processed in segments of as many 64-token
+ *              chunks as the array holds for all B·H_v sequence-heads (73 KB
+ *              per chunk and sequence-head; 9 chunks for B·H_v = 48), so long
+ *              sequences take more launches than gdn2_chunk_fwd. The first
+ *              call on each device looks up the array's device address (with
+ *              that device current); make that first call before any stream
+ *              capture. Each call clears the status word it uses before its
+ *              launches; nothing else in the array needs to start at zero.
  *   Sharing:   every call on a device uses the same array, so calls whose
  *              work overlaps on the GPU (different streams, no ordering
  *              between them) race; order them on one stream or by events.
  *   Errors:    GDN2_ERR_UNSUPPORTED for configurations that do not run the
  *              tensor-core kernel (call gdn2_chunk_fwd: they need no
- *              scratch); GDN2_ERR_WORKSPACE if the problem would need more
- *              than the 4 KiB array; GDN2_ERR_CUDA if the address lookup
- *              fails; otherwise exactly the statuses of gdn2_chunk_fwd.     */
+ *              scratch); GDN2_ERR_WORKSPACE if even one chunk per
+ *              sequence-head does not fit (B·H_v above about 440);
+ *              GDN2_ERR_CUDA if the address lookup fails; otherwise exactly
+ *              the statuses of gdn2_chunk_fwd.                              */
 GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_params* p, const void* q, const void* k,
                                             const void* v, const float* alpha, const float* b,
                                             const float* w, const float* S0, void* o, float* S_T,

@@ -38,6 +38,26 @@ def test_noalloc_matches_regular_entry_point_twice():
         assert torch.equal(o, o_ref) and torch.equal(S, S_ref)
 
 
+@pytest.mark.parametrize("with_state", [True, False])
+def test_noalloc_long_sequence_runs_in_segments(with_state):
+    """48 sequence-heads and 19 chunks: more than the fixed array holds at once,
+    so the call runs in segments (carrying the state through S_T, or through
+    the array itself when S_T is NULL)."""
+    w = replace(workload("prefill_t4096"), T=1200, s0="normal")
+    inp = make_inputs(w, seed=23, device="cuda")
+    args = (inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"])
+    o_ref, S_ref = gdn2.chunk_fwd(*args, chunk=64, o_dtype=torch.float32)
+    o = torch.full_like(o_ref, float("nan"))
+    S = torch.full_like(S_ref, float("nan")) if with_state else None
+    gdn2.chunk_fwd_noalloc(*args, o=o, S_T=S, chunk=64)
+    torch.cuda.synchronize()
+    assert_close(o, np64(o_ref), TOL_BF16, "o")
+    if with_state:
+        assert_close(S, np64(S_ref), TOL_BF16, "S_T")
+        assert torch.equal(S, S_ref)
+    assert torch.equal(o, o_ref)
+
+
 def test_noalloc_rejects_configurations_without_scratch():
     w = replace(workload("prefill_t4096"), T=64, H_qk=1, H_v=1, d=64)
     inp = make_inputs(w, seed=22, device="cuda")
