@@ -141,6 +141,46 @@ __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float* x) {
     x[2 * i + 1] = f.y;
   }
 }
+__device__ __forceinline__ void unpack8_bf16(uint4 u, float* x) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
+// Pass-2 inputs of one token and 8 channels, kept packed while in flight.
+struct QuarterIn {
+  uint4 k, q, v;           // bf16 × 8
+  float4 b0, b1, w0, w1;   // fp32 × 8 (tied gates: β broadcast)
+};
+
+// Inputs of token t0 + r16 (zeros when r16 >= valid).
+__device__ __forceinline__ void load_quarter(const ChunkArgs& a, int bi, int t0, int h, int hq, int ch0, int r16,
+                                             int valid, QuarterIn& r) {
+  if (r16 < valid) {
+    const size_t tq = ((size_t)bi * a.T + t0 + r16) * a.Hqk + hq;
+    const size_t gt = ((size_t)bi * a.T + t0 + r16) * a.Hv + h;
+    r.k = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + tq * D + ch0));
+    r.q = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + tq * D + ch0));
+    r.v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + gt * D + ch0));
+    if (a.gate_mode == GDN2_GATES_FULL) {
+      const float4* bp = reinterpret_cast<const float4*>(a.b + gt * D + ch0);
+      const float4* wp = reinterpret_cast<const float4*>(a.w + gt * D + ch0);
+      r.b0 = __ldg(bp); r.b1 = __ldg(bp + 1);
+      r.w0 = __ldg(wp); r.w1 = __ldg(wp + 1);
+    } else {
+      const float beta = __ldg(a.b + gt);
+      r.b0 = r.b1 = r.w0 = r.w1 = make_float4(beta, beta, beta, beta);
+    }
+  } else {
+    r.k = r.q = r.v = make_uint4(0, 0, 0, 0);
+    r.b0 = r.b1 = r.w0 = r.w1 = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
 __device__ __forceinline__ void unpack8_f16(uint4 u, float* x) {
   const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
@@ -204,35 +244,44 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   const int cg = 2 * warp + (lane >> 4);
   const int ch0 = cg * 8;
 
-  // -------- pass 1: α per quarter, quarter products Π over 16 tokens
-  float al[4][8];
+  // -------- pass 1: α, forward products within each 16-token quarter and
+  // the quarter products P (the last forward product). The pass-2 inputs of
+  // quarter 0 are requested at the same time.
+  float fw[4][8];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const int i = 16 * m + r16;
     if (i < Lc) {
       const size_t gt = ((size_t)bi * a.T + t0 + i) * a.Hv + h;
       if (mode == GDN2_GATES_GDN) {
-        const float s = __ldg(a.alpha + gt);
+        const float sa = __ldg(a.alpha + gt);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) al[m][c] = s;
+        for (int c = 0; c < 8; ++c) fw[m][c] = sa;
       } else {
-        load8_f32(a.alpha + gt * D + ch0, al[m]);
+        load8_f32(a.alpha + gt * D + ch0, fw[m]);
       }
     } else {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) al[m][c] = 1.f;
+      for (int c = 0; c < 8; ++c) fw[m][c] = 1.f;
     }
   }
+  QuarterIn cur;
+  load_quarter(a, bi, t0, h, hq, ch0, r16, Lc, cur);
   float mn = 1.f;
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      float x = al[m][c];
+      float x = fw[m][c];
 #pragma unroll
-      for (int off = 1; off < 16; off <<= 1) x *= __shfl_xor_sync(0xffffffffu, x, off);
-      mn = fminf(mn, x);
-      if (r16 == 0) sPq[m * D + ch0 + c] = x;
+      for (int dd = 1; dd < 16; dd <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, dd, 16);
+        if (r16 >= dd) x *= y;
+      }
+      fw[m][c] = x;
+      const float P = __shfl_sync(0xffffffffu, x, 15, 16);
+      mn = fminf(mn, P);
+      if (r16 == 0) sPq[m * D + ch0 + c] = P;
     }
   }
 #pragma unroll
@@ -255,81 +304,65 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     reinterpret_cast<float*>(slot + SL_GC)[tid] = g;
   }
 
-  // -------- pass 2: operand tiles
+  // -------- pass 2: operand tiles; the next quarter's inputs are in flight
+  // while this one is computed
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const int i = 16 * m + r16;
+    QuarterIn nxt;
+    if (m < 3) load_quarter(a, bi, t0 + 16 * (m + 1), h, hq, ch0, r16, Lc - 16 * (m + 1), nxt);
     float kx[8], qx[8], ex[8], zx[8];
-    if (i < Lc) {
-      const size_t tq = ((size_t)bi * a.T + t0 + i) * a.Hqk + hq;
-      const size_t gt = ((size_t)bi * a.T + t0 + i) * a.Hv + h;
-      float bx[8], wx[8], vx[8];
-      load8_bf16(static_cast<const __nv_bfloat16*>(a.k) + tq * D + ch0, kx);
-      load8_bf16(static_cast<const __nv_bfloat16*>(a.q) + tq * D + ch0, qx);
-      load8_bf16(static_cast<const __nv_bfloat16*>(a.v) + gt * D + ch0, vx);
-      if (mode == GDN2_GATES_FULL) {
-        load8_f32(a.b + gt * D + ch0, bx);
-        load8_f32(a.w + gt * D + ch0, wx);
-      } else {
-        const float beta = __ldg(a.b + gt);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) { bx[c] = beta; wx[c] = beta; }
-      }
+    {
+      float vx[8], bx[8], wx[8];
+      unpack8_bf16(cur.k, kx);
+      unpack8_bf16(cur.q, qx);
+      unpack8_bf16(cur.v, vx);
+      bx[0] = cur.b0.x; bx[1] = cur.b0.y; bx[2] = cur.b0.z; bx[3] = cur.b0.w;
+      bx[4] = cur.b1.x; bx[5] = cur.b1.y; bx[6] = cur.b1.z; bx[7] = cur.b1.w;
+      wx[0] = cur.w0.x; wx[1] = cur.w0.y; wx[2] = cur.w0.z; wx[3] = cur.w0.w;
+      wx[4] = cur.w1.x; wx[5] = cur.w1.y; wx[6] = cur.w1.z; wx[7] = cur.w1.w;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         ex[c] = bx[c] * kx[c];
         zx[c] = wx[c] * vx[c];
       }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) { kx[c] = 0.f; qx[c] = 0.f; ex[c] = 0.f; zx[c] = 0.f; }
     }
     float o_eb[8], o_qb[8], o_ke[8], o_em[8], o_qm[8], o_km[8], o_x1[8], o_x2[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      // in-quarter forward inclusive (fw) and backward exclusive (bw) products
-      float fw = al[m][c];
-#pragma unroll
-      for (int dd = 1; dd < 16; dd <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, fw, dd, 16);
-        if (r16 >= dd) fw *= y;
-      }
-      float bi_ = al[m][c];
-#pragma unroll
-      for (int dd = 1; dd < 16; dd <<= 1) {
-        const float y = __shfl_down_sync(0xffffffffu, bi_, dd, 16);
-        if (r16 + dd < 16) bi_ *= y;
-      }
-      float bw = __shfl_down_sync(0xffffffffu, bi_, 1, 16);
-      if (r16 == 15) bw = 1.f;
+      const float* pq = sPq + ch0 + c;
+      const float P = pq[m * D];
       float pre = 1.f, suf = 1.f;
 #pragma unroll
       for (int mm = 0; mm < 4; ++mm) {
-        if (mm < m) pre *= sPq[mm * D + ch0 + c];
-        if (mm > m) suf *= sPq[mm * D + ch0 + c];
+        if (mm < m) pre *= pq[mm * D];
+        if (mm > m) suf *= pq[mm * D];
       }
-      const float g = pre * fw;          // γ_i
-      const float bk = bw * suf;         // Π_{i<s≤63} α
+      const float f = fw[m][c];               // Π_{quarter start ≤ s ≤ i} α
+      const float rf = __fdividef(1.f, f);
+      const float bw = P * rf;                // Π_{i < s ≤ quarter end} α
+      const float g = pre * f;                // γ_i
+      const float bk = bw * suf;              // Π_{i < s ≤ 63} α
       o_eb[c] = ex[c] * g;
       o_qb[c] = qx[c] * g;
       o_ke[c] = kx[c] * bk;
       float fe, fk;
       if ((m & 1) == 0) {
-        fe = __fdividef(1.f, bw);
+        fe = f * __fdividef(1.f, P);          // 1 / bw
         fk = bw;
       } else {
-        fe = fw;
-        fk = __fdividef(1.f, fw);
+        fe = f;
+        fk = rf;
       }
       o_em[c] = ex[c] * fe;
       o_qm[c] = qx[c] * fe;
       o_km[c] = kx[c] * fk;
       if (m >= 2) {
-        const float fq = (m == 3 ? sPq[2 * D + ch0 + c] : 1.f) * fw;
+        const float fq = (m == 3 ? pq[2 * D] : 1.f) * f;
         o_x1[c] = ex[c] * fq;
         o_x2[c] = qx[c] * fq;
       } else {
-        const float fb = bw * (m == 0 ? sPq[D + ch0 + c] : 1.f);
+        const float fb = bw * (m == 0 ? pq[D] : 1.f);
         o_x1[c] = kx[c] * fb;
         o_x2[c] = 0.f;
       }
@@ -347,6 +380,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     } else {
       st16(smem + P_KB, tile_off(i, ch0, D), pack8(o_x1, gram_bf16));
     }
+    if (m < 3) cur = nxt;
   }
   sync_for_mma();
 
@@ -572,37 +606,44 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   const int row = lq * 32 + lane;       // dv index j of Sᵀ[j][*]
   const bool lo = warp < 4;
 
-  // entry state: Sᵀ[j][c] = S[c][j]
+  // Entry state: Sᵀ[j][c] = S[c][j]. The fp16 copy (operand of the first
+  // chunk's MMAs) is the state itself; TMEM holds it already multiplied by the
+  // first chunk's decay Γ, ready for the first update Sᵀ ← Sᵀ Γ + Uᵀ K_end.
+  if (!mbar_wait(&full[0], 0)) atomicOr(sflag, 1);
   {
+    const float* gC = reinterpret_cast<const float*>(smem + S_STAGE0 + SL_GC);
     const int c0 = lo ? 0 : 64;
     const float* S0 = S_in ? S_in + (size_t)bh * D * D : nullptr;
     for (int cb = c0; cb < c0 + 64; cb += 16) {
       float v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) v[u] = S0 ? __ldg(S0 + (size_t)(cb + u) * D + row) : 0.f;
-      tmem_st16(t_lane + ST_S + cb, v);
       st16(smem + S_ST, tile_off(row, cb, D), pack8_f16(v));
       st16(smem + S_ST, tile_off(row, cb + 8, D), pack8_f16(v + 8));
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] *= gC[cb + u];
+      tmem_st16(t_lane + ST_S + cb, v);
     }
     tmem_wait_st();
   }
   sync_for_mma();
 
+  // O staging: [rows][128] of TOut in the 16 KB U tile, which is free once the
+  // chunk's second MMA group has completed.
+  constexpr int O_ROWS = 16384 / (D * (int)sizeof(TOut));   // 64 (bf16) or 32 (fp32)
   uint32_t mphase = 0;
   int issued = 1;                       // bulk copies issued (for the error path)
-  int waited = 0;
+  int waited = 1;
   for (int cl = 0; cl < n_seg; ++cl) {
     const int s = cl & 1;
     uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
+    uint8_t* nstg = smem + (s ? S_STAGE0 : S_STAGE1);
     const int t0 = (c_begin + cl) * C;
     const int Lc = min(C, a.T - t0);
-    if (!mbar_wait(&full[s], (cl >> 1) & 1)) atomicOr(sflag, 1);
-    ++waited;
     // prefetch the next chunk into the other stage (free: its MMAs and reads
     // finished before the barrier that closed the previous iteration)
     if (cl + 1 < n_seg) {
       if (tid == 0) {
-        uint8_t* nstg = smem + (s ? S_STAGE0 : S_STAGE1);
         mbar_arrive_expect_tx(&full[s ^ 1], SLOT_USED);
         bulk_g2s(nstg, slots + (size_t)(cl + 1) * SLOT, SLOT_USED, &full[s ^ 1]);
       }
@@ -621,37 +662,22 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       }
       mma_commit(mbar);
     }
-    // meanwhile Sᵀ ← Sᵀ Γ in TMEM (column c scaled by γ_C[c])
-    {
-      const float* gC = reinterpret_cast<const float*>(stg + SL_GC);
-      const int c0 = lo ? 0 : 64;
-      for (int cb = c0; cb < c0 + 64; cb += 16) {
-        float v[16];
-        tmem_ld16(t_lane + ST_S + cb, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] *= gC[cb + u];
-        tmem_st16(t_lane + ST_S + cb, v);
-      }
-      tmem_wait_st();
-    }
     __syncwarp();
     wait_mma(mbar, mphase, sflag);
     // Uᵀ = U_wᵀ − (Y S)ᵀ
     {
       const int c0 = lo ? 0 : 32;
+      float ys[32], uw[32];
+      tmem_ld16(t_lane + ST_YS + c0, ys);
+      tmem_ld16(t_lane + ST_YS + c0 + 16, ys + 16);
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        float ys[16], uw[16];
-        tmem_ld16(t_lane + ST_YS + c0 + cb, ys);
-        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + tile_off(row, c0 + cb, C)), uw);
-        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + tile_off(row, c0 + cb + 8, C)), uw + 8);
-        tmem_wait_ld();
+      for (int cb = 0; cb < 32; cb += 8)
+        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + tile_off(row, c0 + cb, C)), uw + cb);
+      tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 16; ++u) uw[u] -= ys[u];
-        st16(smem + S_UT, tile_off(row, c0 + cb, C), pack8_f16(uw));
-        st16(smem + S_UT, tile_off(row, c0 + cb + 8, C), pack8_f16(uw + 8));
-      }
+      for (int u = 0; u < 32; ++u) uw[u] -= ys[u];
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 8) st16(smem + S_UT, tile_off(row, c0 + cb, C), pack8_f16(uw + cb));
     }
     sync_for_mma();
     // Sᵀ += Uᵀ K_end, Oᵀ += Uᵀ Aqkᵀ
@@ -668,32 +694,58 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
     }
     __syncwarp();
     wait_mma(mbar, mphase, sflag);
-    // outputs o[t0 + i][h][j]
+    // Next chunk's fp16 Sᵀ operand, then Sᵀ ← Sᵀ Γ_next in TMEM (the next
+    // slot's γ_C; its copy was issued at the top of this iteration).
+    const bool more = cl + 1 < n_seg;
+    if (more) {
+      if (!mbar_wait(&full[s ^ 1], ((cl + 1) >> 1) & 1)) atomicOr(sflag, 1);
+      ++waited;
+    }
     {
-      const int c0 = lo ? 0 : 32;
-      TOut* orow = og + (((size_t)bi * a.T + t0) * a.Hv + h) * D + row;
-      const size_t tstride = (size_t)a.Hv * D;
+      const float* gN = reinterpret_cast<const float*>(nstg + SL_GC);
+      const int c0 = lo ? 0 : 64;
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        float v[16];
-        tmem_ld16(t_lane + ST_O + c0 + cb, v);
+      for (int half = 0; half < 2; ++half) {
+        float v[32];
+        tmem_ld16(t_lane + ST_S + c0 + half * 32, v);
+        tmem_ld16(t_lane + ST_S + c0 + half * 32 + 16, v + 16);
         tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = c0 + cb + u;
-          if (i < Lc) orow[(size_t)i * tstride] = from_f32<TOut>(a.scale * v[u]);
+        for (int cb = 0; cb < 32; cb += 8) st16(smem + S_ST, tile_off(row, c0 + half * 32 + cb, D), pack8_f16(v + cb));
+        if (more) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] *= gN[c0 + half * 32 + u];
+          tmem_st16(t_lane + ST_S + c0 + half * 32, v);
+          tmem_st16(t_lane + ST_S + c0 + half * 32 + 16, v + 16);
         }
       }
+      if (more) tmem_wait_st();
     }
-    // next chunk's fp16 Sᵀ operand
+    // Outputs o[t0 + i][h][:] through the staging tile, O_ROWS tokens at a time,
+    // written as contiguous 16-byte vectors.
     {
-      const int c0 = lo ? 0 : 64;
-      for (int cb = c0; cb < c0 + 64; cb += 16) {
-        float v[16];
-        tmem_ld16(t_lane + ST_S + cb, v);
-        tmem_wait_ld();
-        st16(smem + S_ST, tile_off(row, cb, D), pack8_f16(v));
-        st16(smem + S_ST, tile_off(row, cb + 8, D), pack8_f16(v + 8));
+      TOut* so = reinterpret_cast<TOut*>(smem + S_UT);
+      const int c0 = lo ? 0 : 32;
+      float v[32];
+      tmem_ld16(t_lane + ST_O + c0, v);
+      tmem_ld16(t_lane + ST_O + c0 + 16, v + 16);
+      tmem_wait_ld();
+      constexpr int VEC = 16 / (int)sizeof(TOut);             // elements per 16 bytes
+      for (int r0 = 0; r0 < C; r0 += O_ROWS) {
+        __syncthreads();
+        if (c0 >= r0 && c0 < r0 + O_ROWS) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) so[(c0 - r0 + u) * D + row] = from_f32<TOut>(a.scale * v[u]);
+        }
+        __syncthreads();
+        const int nvec = O_ROWS * D / VEC;
+        for (int e = tid; e < nvec; e += NT) {
+          const int rr = e / (D / VEC), cc = (e % (D / VEC)) * VEC;
+          const int i = r0 + rr;
+          if (i < Lc)
+            *reinterpret_cast<uint4*>(og + (((size_t)bi * a.T + t0 + i) * a.Hv + h) * D + cc) =
+                *reinterpret_cast<const uint4*>(so + rr * D + cc);
+        }
       }
     }
     sync_for_mma();
