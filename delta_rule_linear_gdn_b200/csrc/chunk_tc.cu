@@ -31,7 +31,9 @@
 //         Sᵀ ← Sᵀ Γ + Uᵀ K_end,  Oᵀ += Uᵀ Aqkᵀ,
 //     with the fp32 state Sᵀ resident in TMEM and an fp16 copy in shared
 //     memory feeding the next chunk's MMAs.
-// Everything is computed transposed so that every MMA has M = 128.
+// Everything is computed transposed so that every MMA has M = 128. All MMA
+// operand tiles use the 128-byte-swizzled layout (see tc_prims.cuh), so that
+// a warp writing or reading whole rows is free of bank conflicts.
 //
 // Decay factors of the Gram matrices. Π_{j<s≤i} α is split into two factors
 // about a reference token so that one factor multiplies row i and the other
@@ -69,41 +71,50 @@ constexpr int NT = 256;           // threads per CTA (8 warps)
 
 // ------------------------------------------------------------------ workspace
 // Word 0 of the workspace is the device status (nonzero: a wait gave up).
-// Slots follow, one per (sequence, value head, chunk of the segment).
+// Slots follow, one per (sequence, value head, chunk of the segment). Tiles
+// are swizzled; "BS" is the byte stride between 64-column blocks.
 constexpr size_t WS_HEAD = 256;
-constexpr int SL_YT = 0;              // Yᵀ   fp16 [128 key][64 tok]
+constexpr int SL_YT = 0;              // Yᵀ   fp16 [128 key][64 tok]   (MN-major B of (YS)ᵀ)
 constexpr int SL_UW = 16384;          // U_wᵀ fp16 [128 dv][64 tok]
-constexpr int SL_QB = 32768;          // Q̄    fp16 [64 tok][128 key]
-constexpr int SL_KE = 49152;          // K_end fp16 [64 tok][128 key]
-constexpr int SL_AQ = 65536;          // Aqk  fp16 [64 i][64 j]
+constexpr int SL_QB = 32768;          // Q̄    fp16 [64 tok][128 key]  BS 8192 (K-major B of Oᵀ)
+constexpr int SL_KE = 49152;          // K_end fp16 [64 tok][128 key] BS 8192 (MN-major B of Sᵀ)
+constexpr int SL_AQ = 65536;          // Aqk  fp16 [64 i][64 j]        (K-major B of Oᵀ)
 constexpr int SL_GC = 73728;          // γ_C  fp32 [128]
 constexpr int SLOT_USED = 74240;      // bytes copied per chunk
 constexpr int SLOT = 74752;           // slot stride (1 KB multiple)
+constexpr int BS_ROW128 = 16384;      // block stride of a 128-row tile
+constexpr int BS_ROW64 = 8192;        // block stride of a 64-row tile
 
 // ------------------------------------------------------------------ prep smem
-// [0, 32K): Gram "boundary" operand [Ē_bnd ; Q̄_bnd] as a 128-row tile whose
-// rows 32..63 and 96..127 are used; its unused row groups hold K̃_bnd
-// (rows 0..31 → [0, 8K)) and the quarter products and reduction slots
-// ([16K, 24K)); the MMA reads those rows as don't-care. After the Gram MMAs,
-// [8K, 16K) holds A = (I+T)⁻¹ (fp16 64 × 64). 112 KB in all, so two CTAs
-// share an SM.
+// [0, 32K)   Gb: Gram boundary operand [Ē_bnd ; Q̄_bnd], 128 rows (32..63 and
+//            96..127 used), BS 16K. Its rows 0..31 hold K̃_bnd (the Kb tile,
+//            BS 16K) and its block-0 rows 64..95 ([8K, 12K)) hold the quarter
+//            products; the MMA reads those rows as don't-care.
+// [32K, 64K) Gm: [Ē_mid ; Q̄_mid], 128 rows, BS 16K
+// [64K, 80K) Km: K̃_mid, 64 rows, BS 8K
+// [80K, 96K) Ē (64 tok × 128 key, BS 8K)   [96K, 112K) Z (64 tok × 128 dv)
+// Before pass 2, [32K, 66K) stages α for the cumulative products; after the
+// Gram MMAs, [32K, 71K) holds the fp32 arrays of the inverse and [0, 8K) the
+// fp16 A = (I+T)⁻¹ (64 × 64).
 constexpr int P_GB = 0;
-constexpr int P_KB = 0;               // K̃_bnd [32 tok][128] (C = 128 tile, rows 0..31)
-constexpr int P_AINV = 8192;          // A fp16 [64][64]
-constexpr int P_GM = 32768;           // [Ē_mid ; Q̄_mid] 128 × 128
-constexpr int P_KM = 65536;           // K̃_mid [64][128]
-constexpr int P_EB = 81920;           // Ē [64 tok][128 key]
-constexpr int P_Z = 98304;            // Z [64 tok][128 dv]
+constexpr int P_KB = 0;
+constexpr int P_PQ = 8192;            // quarter products [4][128] fp32
+constexpr int P_RED = P_PQ + 4 * D * 4;
+static_assert(P_RED + 64 <= 12288, "quarter products must stay in the unused Gram rows");
+constexpr int P_GM = 32768;
+constexpr int P_KM = 65536;
+constexpr int P_EB = 81920;
+constexpr int P_Z = 98304;
 constexpr int P_END = 114688;
-// fp32 work arrays of the inverse reuse [P_GM, P_EB) after the Gram MMAs
-constexpr int TS = 68;                // row stride (floats), 16-byte aligned rows
+constexpr int SS = 132;               // α staging row stride (floats)
+constexpr int P_STG = P_GM;
+static_assert(P_STG + C * SS * 4 <= P_EB, "staging overlap");
+constexpr int P_AINV = 0;
+constexpr int TS = 68;                // fp32 row stride of T and its inverse
 constexpr int P_T = P_GM;             // T   [64][68]
 constexpr int P_I = P_T + C * TS * 4; // inv [64][68]
 constexpr int P_X = P_I + C * TS * 4; // tmp [32][36]
 static_assert(P_X + 32 * 36 * 4 <= P_EB, "prep smem overlap");
-constexpr int P_PQ = 16384;           // quarter products [4][128] fp32
-constexpr int P_RED = P_PQ + 4 * D * 4;
-static_assert(P_RED + 64 <= 24576, "quarter products must stay in the unused Gram rows");
 constexpr int P_BAR = P_END;
 constexpr int P_TMEMP = P_BAR + 16;
 constexpr int P_FLAG = P_TMEMP + 16;
@@ -114,8 +125,8 @@ constexpr uint32_t PT_GM = 0, PT_GB = 64, PT_YT = 128, PT_UW = 192, PT_COLS = 25
 // ------------------------------------------------------------------ scan smem
 constexpr int S_STAGE0 = 0;
 constexpr int S_STAGE1 = SLOT;
-constexpr int S_ST = 2 * SLOT;        // Sᵀ fp16 [128 dv][128 key]
-constexpr int S_UT = S_ST + D * D * 2;// Uᵀ fp16 [128 dv][64 tok]
+constexpr int S_ST = 2 * SLOT;        // Sᵀ fp16 [128 dv][128 key], BS 16K
+constexpr int S_UT = S_ST + D * D * 2;// Uᵀ fp16 [128 dv][64 tok]; output staging afterwards
 constexpr int S_BAR = S_UT + D * C * 2;   // full[2], mma
 constexpr int S_TMEMP = S_BAR + 32;
 constexpr int S_FLAG = S_TMEMP + 16;
@@ -125,62 +136,15 @@ constexpr uint32_t ST_S = 0, ST_YS = 128, ST_O = 192, ST_COLS = 256;
 __device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
   *reinterpret_cast<uint4*>(base + off) = v;
 }
-
-__device__ __forceinline__ void load8_f32(const float* p, float* x) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+__device__ __forceinline__ void st8(uint8_t* base, uint32_t off, uint2 v) {
+  *reinterpret_cast<uint2*>(base + off) = v;
 }
-__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float* x) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+
+__device__ __forceinline__ void unpack4_bf16(uint2 u, float* x) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    x[2 * i] = f.x;
-    x[2 * i + 1] = f.y;
-  }
+  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
 }
-__device__ __forceinline__ void unpack8_bf16(uint4 u, float* x) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    x[2 * i] = f.x;
-    x[2 * i + 1] = f.y;
-  }
-}
-
-// Pass-2 inputs of one token and 8 channels, kept packed while in flight.
-struct QuarterIn {
-  uint4 k, q, v;           // bf16 × 8
-  float4 b0, b1, w0, w1;   // fp32 × 8 (tied gates: β broadcast)
-};
-
-// Inputs of token t0 + r16 (zeros when r16 >= valid).
-__device__ __forceinline__ void load_quarter(const ChunkArgs& a, int bi, int t0, int h, int hq, int ch0, int r16,
-                                             int valid, QuarterIn& r) {
-  if (r16 < valid) {
-    const size_t tq = ((size_t)bi * a.T + t0 + r16) * a.Hqk + hq;
-    const size_t gt = ((size_t)bi * a.T + t0 + r16) * a.Hv + h;
-    r.k = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + tq * D + ch0));
-    r.q = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + tq * D + ch0));
-    r.v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + gt * D + ch0));
-    if (a.gate_mode == GDN2_GATES_FULL) {
-      const float4* bp = reinterpret_cast<const float4*>(a.b + gt * D + ch0);
-      const float4* wp = reinterpret_cast<const float4*>(a.w + gt * D + ch0);
-      r.b0 = __ldg(bp); r.b1 = __ldg(bp + 1);
-      r.w0 = __ldg(wp); r.w1 = __ldg(wp + 1);
-    } else {
-      const float beta = __ldg(a.b + gt);
-      r.b0 = r.b1 = r.w0 = r.w1 = make_float4(beta, beta, beta, beta);
-    }
-  } else {
-    r.k = r.q = r.v = make_uint4(0, 0, 0, 0);
-    r.b0 = r.b1 = r.w0 = r.w1 = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
 __device__ __forceinline__ void unpack8_f16(uint4 u, float* x) {
   const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
@@ -188,6 +152,36 @@ __device__ __forceinline__ void unpack8_f16(uint4 u, float* x) {
     const float2 f = __half22float2(h[i]);
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
+  }
+}
+
+// Key-side inputs of one token for 4 channels (coalesced: a warp reads whole
+// rows), and the pointers and sizes needed to load them, passed by value.
+struct KeyIn {
+  uint2 k, q;              // bf16 × 4
+  float4 b;                // fp32 × 4 (tied gates: β broadcast)
+};
+struct RowSrc {
+  const __nv_bfloat16 *k, *q;
+  const float* b;
+  int T, Hqk, Hv, full_gates;
+};
+
+__device__ __forceinline__ void load_key_row(RowSrc r_, int bi, int t, int h, int hq, int c4, bool valid, KeyIn& r) {
+  if (valid) {
+    const size_t tq = ((size_t)bi * r_.T + t) * r_.Hqk + hq;
+    const size_t gt = ((size_t)bi * r_.T + t) * r_.Hv + h;
+    r.k = __ldg(reinterpret_cast<const uint2*>(r_.k + tq * D + c4));
+    r.q = __ldg(reinterpret_cast<const uint2*>(r_.q + tq * D + c4));
+    if (r_.full_gates) {
+      r.b = __ldg(reinterpret_cast<const float4*>(r_.b + gt * D + c4));
+    } else {
+      const float beta = __ldg(r_.b + gt);
+      r.b = make_float4(beta, beta, beta, beta);
+    }
+  } else {
+    r.k = r.q = make_uint2(0, 0);
+    r.b = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -214,6 +208,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   int* sflag = reinterpret_cast<int*>(smem + P_FLAG);
   float* sPq = reinterpret_cast<float*>(smem + P_PQ);
   float* sred = reinterpret_cast<float*>(smem + P_RED);
+  float* stage = reinterpret_cast<float*>(smem + P_STG);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // CTA order: value head fastest, so the value heads sharing a query/key head
@@ -224,7 +219,6 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   const int ck = c_begin + cl;
   const int h = bh % a.Hv, bi = bh / a.Hv;
   const int hq = h / (a.Hv / a.Hqk);
-  const int mode = a.gate_mode;
   const int t0 = ck * C;
   const int Lc = min(C, a.T - t0);
   uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)bh * n_seg + cl) * SLOT;
@@ -239,58 +233,74 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     tmem_relinquish();
   }
 
-  // Element mapping: lane r16 = token within a 16-token quarter, 8 channels.
-  const int r16 = lane & 15;
-  const int cg = 2 * warp + (lane >> 4);
-  const int ch0 = cg * 8;
+  // Element mapping: lane → 4 channels (a warp covers a whole 128-channel
+  // row), warp → tokens warp, warp + 8, ..., so token j·8 + warp lies in
+  // quarter j/2.
+  const int c4 = lane * 4;
 
-  // -------- pass 1: α, forward products within each 16-token quarter and
-  // the quarter products P (the last forward product). The pass-2 inputs of
-  // quarter 0 are requested at the same time.
-  float fw[4][8];
+  // -------- pass 1: α rows into the staging tile; the write side Z = w ⊙ v
+  // (which needs no decay) goes straight to its tile
+  {
+    float4 al[8], wv[8];
+    uint2 vv[8];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int i = 16 * m + r16;
-    if (i < Lc) {
-      const size_t gt = ((size_t)bi * a.T + t0 + i) * a.Hv + h;
-      if (mode == GDN2_GATES_GDN) {
-        const float sa = __ldg(a.alpha + gt);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) fw[m][c] = sa;
-      } else {
-        load8_f32(a.alpha + gt * D + ch0, fw[m]);
+    for (int j = 0; j < 8; ++j) {
+      const int i = warp + 8 * j;
+      al[j] = make_float4(1.f, 1.f, 1.f, 1.f);
+      wv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      vv[j] = make_uint2(0, 0);
+      if (i < Lc) {
+        const size_t gt = ((size_t)bi * a.T + t0 + i) * a.Hv + h;
+        if (a.gate_mode == GDN2_GATES_GDN) {
+          const float sa = __ldg(a.alpha + gt);
+          al[j] = make_float4(sa, sa, sa, sa);
+        } else {
+          al[j] = __ldg(reinterpret_cast<const float4*>(a.alpha + gt * D + c4));
+        }
+        if (a.gate_mode == GDN2_GATES_FULL) {
+          wv[j] = __ldg(reinterpret_cast<const float4*>(a.w + gt * D + c4));
+        } else {
+          const float beta = __ldg(a.b + gt);
+          wv[j] = make_float4(beta, beta, beta, beta);
+        }
+        vv[j] = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.v) + gt * D + c4));
       }
-    } else {
+    }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) fw[m][c] = 1.f;
+    for (int j = 0; j < 8; ++j) {
+      const int i = warp + 8 * j;
+      *reinterpret_cast<float4*>(stage + i * SS + c4) = al[j];
+      float vx[4];
+      unpack4_bf16(vv[j], vx);
+      st8(smem, P_Z + sw_off(i, c4, BS_ROW64),
+          pack4_f16(wv[j].x * vx[0], wv[j].y * vx[1], wv[j].z * vx[2], wv[j].w * vx[3]));
     }
   }
-  QuarterIn cur;
-  load_quarter(a, bi, t0, h, hq, ch0, r16, Lc, cur);
-  float mn = 1.f;
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float x = fw[m][c];
-#pragma unroll
-      for (int dd = 1; dd < 16; dd <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, dd, 16);
-        if (r16 >= dd) x *= y;
-      }
-      fw[m][c] = x;
-      const float P = __shfl_sync(0xffffffffu, x, 15, 16);
-      mn = fminf(mn, P);
-      if (r16 == 0) sPq[m * D + ch0 + c] = P;
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-  if (lane == 0) sred[warp] = mn;
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_ptr;
+  // forward cumulative products down each channel within each quarter
+  {
+    const int c = tid & 127;
+    float mn = 1.f;
+#pragma unroll
+    for (int q = tid >> 7; q < 4; q += 2) {
+      float acc = 1.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) {
+        float* p = stage + (16 * q + s) * SS + c;
+        acc *= *p;
+        *p = acc;
+      }
+      sPq[q * D + c] = acc;
+      mn = fminf(mn, acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    if (lane == 0) sred[warp] = mn;
+  }
+  __syncthreads();
   bool gram_bf16;
   {
     float mall = sred[0];
@@ -303,84 +313,95 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     const float g = sPq[tid] * sPq[D + tid] * sPq[2 * D + tid] * sPq[3 * D + tid];
     reinterpret_cast<float*>(slot + SL_GC)[tid] = g;
   }
+  float fw[8][4], Pq[4][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 v = *reinterpret_cast<const float4*>(stage + (warp + 8 * j) * SS + c4);
+    fw[j][0] = v.x; fw[j][1] = v.y; fw[j][2] = v.z; fw[j][3] = v.w;
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 v = *reinterpret_cast<const float4*>(sPq + q * D + c4);
+    Pq[q][0] = v.x; Pq[q][1] = v.y; Pq[q][2] = v.z; Pq[q][3] = v.w;
+  }
+  __syncthreads();   // the staging tile is free from here on
 
-  // -------- pass 2: operand tiles; the next quarter's inputs are in flight
-  // while this one is computed
+  // -------- pass 2: key-side operand tiles, PB tokens in flight at a time
+  constexpr int PB = 4;
+  const RowSrc src{static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.q), a.b, a.T, a.Hqk,
+                   a.Hv, a.gate_mode == GDN2_GATES_FULL};
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int i = 16 * m + r16;
-    QuarterIn nxt;
-    if (m < 3) load_quarter(a, bi, t0 + 16 * (m + 1), h, hq, ch0, r16, Lc - 16 * (m + 1), nxt);
-    float kx[8], qx[8], ex[8], zx[8];
-    {
-      float vx[8], bx[8], wx[8];
-      unpack8_bf16(cur.k, kx);
-      unpack8_bf16(cur.q, qx);
-      unpack8_bf16(cur.v, vx);
-      bx[0] = cur.b0.x; bx[1] = cur.b0.y; bx[2] = cur.b0.z; bx[3] = cur.b0.w;
-      bx[4] = cur.b1.x; bx[5] = cur.b1.y; bx[6] = cur.b1.z; bx[7] = cur.b1.w;
-      wx[0] = cur.w0.x; wx[1] = cur.w0.y; wx[2] = cur.w0.z; wx[3] = cur.w0.w;
-      wx[4] = cur.w1.x; wx[5] = cur.w1.y; wx[6] = cur.w1.z; wx[7] = cur.w1.w;
+  for (int bt = 0; bt < 8 / PB; ++bt) {
+    KeyIn in[PB];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        ex[c] = bx[c] * kx[c];
-        zx[c] = wx[c] * vx[c];
-      }
+    for (int jj = 0; jj < PB; ++jj) {
+      const int i = warp + 8 * (PB * bt + jj);
+      load_key_row(src, bi, t0 + i, h, hq, c4, i < Lc, in[jj]);
     }
-    float o_eb[8], o_qb[8], o_ke[8], o_em[8], o_qm[8], o_km[8], o_x1[8], o_x2[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float* pq = sPq + ch0 + c;
-      const float P = pq[m * D];
-      float pre = 1.f, suf = 1.f;
+    for (int jj = 0; jj < PB; ++jj) {
+      const int j = PB * bt + jj;
+      const int m = j >> 1;               // quarter of token i
+      const int i = warp + 8 * j;
+      float kx[4], qx[4], ex[4];
+      unpack4_bf16(in[jj].k, kx);
+      unpack4_bf16(in[jj].q, qx);
+      ex[0] = in[jj].b.x * kx[0]; ex[1] = in[jj].b.y * kx[1]; ex[2] = in[jj].b.z * kx[2]; ex[3] = in[jj].b.w * kx[3];
+      float o_eb[4], o_qb[4], o_ke[4], o_em[4], o_qm[4], o_km[4], o_x1[4], o_x2[4];
 #pragma unroll
-      for (int mm = 0; mm < 4; ++mm) {
-        if (mm < m) pre *= pq[mm * D];
-        if (mm > m) suf *= pq[mm * D];
+      for (int c = 0; c < 4; ++c) {
+        const float P = Pq[m][c];
+        float pre = 1.f, suf = 1.f;
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          if (mm < m) pre *= Pq[mm][c];
+          if (mm > m) suf *= Pq[mm][c];
+        }
+        const float f = fw[j][c];               // Π_{quarter start ≤ s ≤ i} α
+        const float rf = __fdividef(1.f, f);
+        const float bw = P * rf;                // Π_{i < s ≤ quarter end} α
+        const float g = pre * f;                // γ_i
+        const float bk = bw * suf;              // Π_{i < s ≤ 63} α
+        o_eb[c] = ex[c] * g;
+        o_qb[c] = qx[c] * g;
+        o_ke[c] = kx[c] * bk;
+        float fe, fk;
+        if ((m & 1) == 0) {
+          fe = f * __fdividef(1.f, P);          // 1 / bw
+          fk = bw;
+        } else {
+          fe = f;
+          fk = rf;
+        }
+        o_em[c] = ex[c] * fe;
+        o_qm[c] = qx[c] * fe;
+        o_km[c] = kx[c] * fk;
+        if (m >= 2) {
+          const float fq = (m == 3 ? Pq[2][c] : 1.f) * f;
+          o_x1[c] = ex[c] * fq;
+          o_x2[c] = qx[c] * fq;
+        } else {
+          const float fb = bw * (m == 0 ? Pq[1][c] : 1.f);
+          o_x1[c] = kx[c] * fb;
+          o_x2[c] = 0.f;
+        }
       }
-      const float f = fw[m][c];               // Π_{quarter start ≤ s ≤ i} α
-      const float rf = __fdividef(1.f, f);
-      const float bw = P * rf;                // Π_{i < s ≤ quarter end} α
-      const float g = pre * f;                // γ_i
-      const float bk = bw * suf;              // Π_{i < s ≤ 63} α
-      o_eb[c] = ex[c] * g;
-      o_qb[c] = qx[c] * g;
-      o_ke[c] = kx[c] * bk;
-      float fe, fk;
-      if ((m & 1) == 0) {
-        fe = f * __fdividef(1.f, P);          // 1 / bw
-        fk = bw;
-      } else {
-        fe = f;
-        fk = rf;
-      }
-      o_em[c] = ex[c] * fe;
-      o_qm[c] = qx[c] * fe;
-      o_km[c] = kx[c] * fk;
+      st8(slot, SL_QB + sw_off(i, c4, BS_ROW64), pack4(o_qb, false));
+      st8(slot, SL_KE + sw_off(i, c4, BS_ROW64), pack4(o_ke, false));
+      st8(smem, P_EB + sw_off(i, c4, BS_ROW64), pack4(o_eb, false));
+      st8(smem, P_GM + sw_off(i, c4, BS_ROW128), pack4(o_em, gram_bf16));
+      st8(smem, P_GM + sw_off(64 + i, c4, BS_ROW128), pack4(o_qm, gram_bf16));
+      st8(smem, P_KM + sw_off(i, c4, BS_ROW64), pack4(o_km, gram_bf16));
       if (m >= 2) {
-        const float fq = (m == 3 ? pq[2 * D] : 1.f) * f;
-        o_x1[c] = ex[c] * fq;
-        o_x2[c] = qx[c] * fq;
+        st8(smem, P_GB + sw_off(i, c4, BS_ROW128), pack4(o_x1, gram_bf16));
+        st8(smem, P_GB + sw_off(64 + i, c4, BS_ROW128), pack4(o_x2, gram_bf16));
       } else {
-        const float fb = bw * (m == 0 ? pq[D] : 1.f);
-        o_x1[c] = kx[c] * fb;
-        o_x2[c] = 0.f;
+        st8(smem, P_KB + sw_off(i, c4, BS_ROW128), pack4(o_x1, gram_bf16));
       }
     }
-    *reinterpret_cast<uint4*>(slot + SL_QB + tile_off(i, ch0, D)) = pack8_f16(o_qb);
-    *reinterpret_cast<uint4*>(slot + SL_KE + tile_off(i, ch0, D)) = pack8_f16(o_ke);
-    st16(smem + P_EB, tile_off(i, ch0, D), pack8_f16(o_eb));
-    st16(smem + P_Z, tile_off(i, ch0, D), pack8_f16(zx));
-    st16(smem + P_GM, tile_off(i, ch0, D), pack8(o_em, gram_bf16));
-    st16(smem + P_GM, tile_off(64 + i, ch0, D), pack8(o_qm, gram_bf16));
-    st16(smem + P_KM, tile_off(i, ch0, D), pack8(o_km, gram_bf16));
-    if (m >= 2) {
-      st16(smem + P_GB, tile_off(i, ch0, D), pack8(o_x1, gram_bf16));
-      st16(smem + P_GB, tile_off(64 + i, ch0, D), pack8(o_x2, gram_bf16));
-    } else {
-      st16(smem + P_KB, tile_off(i, ch0, D), pack8(o_x1, gram_bf16));
-    }
-    if (m < 3) cur = nxt;
+    // keep the next batch's loads from being hoisted above this one (register
+    // pressure): one batch of rows in flight at a time
+    asm volatile("" ::: "memory");
   }
   sync_for_mma();
 
@@ -391,9 +412,9 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     const uint32_t gb = smem_u32(smem + P_GB), kb = smem_u32(smem + P_KB);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      mma16(tmem + PT_GM, desc_kmajor(gm + ks * 256, D), desc_kmajor(km + ks * 256, D),
+      mma16(tmem + PT_GM, desc_k_sw(gm, ks, BS_ROW128), desc_k_sw(km, ks, BS_ROW64),
             idesc_16(128, 64, false, false, gram_bf16), ks > 0);
-      mma16(tmem + PT_GB, desc_kmajor(gb + ks * 256, D), desc_kmajor(kb + ks * 256, D),
+      mma16(tmem + PT_GB, desc_k_sw(gb, ks, BS_ROW128), desc_k_sw(kb, ks, BS_ROW128),
             idesc_16(128, 32, false, false, gram_bf16), ks > 0);
     }
     mma_commit(bar);
@@ -435,8 +456,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
         for (int u = 0; u < 16; u += 4)
           *reinterpret_cast<float4*>(sT + i * TS + j0 + jb + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
       } else {
-        *reinterpret_cast<uint4*>(slot + SL_AQ + tile_off(i, j0 + jb, C)) = pack8_f16(v);
-        *reinterpret_cast<uint4*>(slot + SL_AQ + tile_off(i, j0 + jb + 8, C)) = pack8_f16(v + 8);
+        st16(slot, SL_AQ + sw_off(i, j0 + jb, BS_ROW64), pack8_f16(v));
+        st16(slot, SL_AQ + sw_off(i, j0 + jb + 8, BS_ROW64), pack8_f16(v + 8));
       }
     }
   }
@@ -524,7 +545,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     float x[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) x[u] = (j0 + u <= i) ? sI[i * TS + j0 + u] : 0.f;
-    st16(smem + P_AINV, tile_off(i, j0, C), pack8_f16(x));
+    st16(smem, P_AINV + sw_off(i, j0, BS_ROW64), pack8_f16(x));
   }
   sync_for_mma();
 
@@ -534,11 +555,9 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     const uint32_t ai = smem_u32(smem + P_AINV);
 #pragma unroll
     for (int ks = 0; ks < C / 16; ++ks) {
-      const uint64_t bdesc = desc_kmajor(ai + ks * 256, C);
-      mma16(tmem + PT_YT, desc_mnmajor(eb + ks * 2 * (D / 8) * 128, D), bdesc, idesc_f16(128, 64, true, false),
-            ks > 0);
-      mma16(tmem + PT_UW, desc_mnmajor(z + ks * 2 * (D / 8) * 128, D), bdesc, idesc_f16(128, 64, true, false),
-            ks > 0);
+      const uint64_t bdesc = desc_k_sw(ai, ks, BS_ROW64);
+      mma16(tmem + PT_YT, desc_mn_sw(eb, ks, BS_ROW64), bdesc, idesc_f16(128, 64, true, false), ks > 0);
+      mma16(tmem + PT_UW, desc_mn_sw(z, ks, BS_ROW64), bdesc, idesc_f16(128, 64, true, false), ks > 0);
     }
     mma_commit(bar);
   }
@@ -547,14 +566,14 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   {
     // warps 0-3: Yᵀ rows (key lanes); warps 4-7: U_wᵀ rows (dv lanes)
     const uint32_t col = lo ? PT_YT : PT_UW;
-    uint8_t* dst = slot + (lo ? SL_YT : SL_UW);
+    const int dst = lo ? SL_YT : SL_UW;
 #pragma unroll
     for (int cb = 0; cb < C; cb += 16) {
       float v[16];
       tmem_ld16(t_lane + col + cb, v);
       tmem_wait_ld();
-      *reinterpret_cast<uint4*>(dst + tile_off(row, cb, C)) = pack8_f16(v);
-      *reinterpret_cast<uint4*>(dst + tile_off(row, cb + 8, C)) = pack8_f16(v + 8);
+      st16(slot, dst + sw_off(row, cb, BS_ROW128), pack8_f16(v));
+      st16(slot, dst + sw_off(row, cb + 8, BS_ROW128), pack8_f16(v + 8));
     }
   }
   if (*sflag && tid == 0) atomicOr(static_cast<int*>(a.workspace), 1);
@@ -618,8 +637,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       float v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) v[u] = S0 ? __ldg(S0 + (size_t)(cb + u) * D + row) : 0.f;
-      st16(smem + S_ST, tile_off(row, cb, D), pack8_f16(v));
-      st16(smem + S_ST, tile_off(row, cb + 8, D), pack8_f16(v + 8));
+      st16(smem, S_ST + sw_off(row, cb, BS_ROW128), pack8_f16(v));
+      st16(smem, S_ST + sw_off(row, cb + 8, BS_ROW128), pack8_f16(v + 8));
 #pragma unroll
       for (int u = 0; u < 16; ++u) v[u] *= gC[cb + u];
       tmem_st16(t_lane + ST_S + cb, v);
@@ -655,10 +674,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       const uint32_t yt = smem_u32(stg + SL_YT), qb = smem_u32(stg + SL_QB);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        const uint64_t adesc = desc_kmajor(st + ks * 256, D);
-        mma16(tmem + ST_YS, adesc, desc_mnmajor(yt + ks * 2 * (C / 8) * 128, C), idesc_f16(128, 64, false, true),
-              ks > 0);
-        mma16(tmem + ST_O, adesc, desc_kmajor(qb + ks * 256, D), idesc_f16(128, 64, false, false), ks > 0);
+        const uint64_t adesc = desc_k_sw(st, ks, BS_ROW128);
+        mma16(tmem + ST_YS, adesc, desc_mn_sw(yt, ks, BS_ROW128), idesc_f16(128, 64, false, true), ks > 0);
+        mma16(tmem + ST_O, adesc, desc_k_sw(qb, ks, BS_ROW64), idesc_f16(128, 64, false, false), ks > 0);
       }
       mma_commit(mbar);
     }
@@ -672,12 +690,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       tmem_ld16(t_lane + ST_YS + c0 + 16, ys + 16);
 #pragma unroll
       for (int cb = 0; cb < 32; cb += 8)
-        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + tile_off(row, c0 + cb, C)), uw + cb);
+        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + sw_off(row, c0 + cb, BS_ROW128)), uw + cb);
       tmem_wait_ld();
 #pragma unroll
       for (int u = 0; u < 32; ++u) uw[u] -= ys[u];
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) st16(smem + S_UT, tile_off(row, c0 + cb, C), pack8_f16(uw + cb));
+      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_UT + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(uw + cb));
     }
     sync_for_mma();
     // Sᵀ += Uᵀ K_end, Oᵀ += Uᵀ Aqkᵀ
@@ -686,9 +704,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       const uint32_t ke = smem_u32(stg + SL_KE), aq = smem_u32(stg + SL_AQ);
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks) {
-        const uint64_t adesc = desc_kmajor(ut + ks * 256, C);
-        mma16(tmem + ST_S, adesc, desc_mnmajor(ke + ks * 2 * (D / 8) * 128, D), idesc_f16(128, 128, false, true), 1);
-        mma16(tmem + ST_O, adesc, desc_kmajor(aq + ks * 256, C), idesc_f16(128, 64, false, false), 1);
+        const uint64_t adesc = desc_k_sw(ut, ks, BS_ROW128);
+        mma16(tmem + ST_S, adesc, desc_mn_sw(ke, ks, BS_ROW64), idesc_f16(128, 128, false, true), 1);
+        mma16(tmem + ST_O, adesc, desc_k_sw(aq, ks, BS_ROW64), idesc_f16(128, 64, false, false), 1);
       }
       mma_commit(mbar);
     }
@@ -711,7 +729,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         tmem_ld16(t_lane + ST_S + c0 + half * 32 + 16, v + 16);
         tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(smem + S_ST, tile_off(row, c0 + half * 32 + cb, D), pack8_f16(v + cb));
+        for (int cb = 0; cb < 32; cb += 8)
+          st16(smem, S_ST + sw_off(row, c0 + half * 32 + cb, BS_ROW128), pack8_f16(v + cb));
         if (more) {
 #pragma unroll
           for (int u = 0; u < 32; ++u) v[u] *= gN[c0 + half * 32 + u];

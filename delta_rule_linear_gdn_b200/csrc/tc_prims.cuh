@@ -30,6 +30,19 @@ __host__ __device__ __forceinline__ uint32_t tile_off(int r, int c, int C) {
   return (uint32_t)(((r >> 3) * (C >> 3) + (c >> 3)) * 128 + (r & 7) * 16 + (c & 7) * 2);
 }
 
+// 128-byte-swizzled tiles. A tile X[R][C] (16-bit, C a multiple of 64) is
+// stored as 64-column blocks, block b at byte b·BS (BS ≥ R·128, 1024-aligned);
+// row r of a block occupies bytes [r·128, r·128 + 128) and its 16-byte chunk j
+// sits at chunk position j XOR (r mod 8). A warp writing or reading whole rows
+// touches every bank once, and the tensor core reads the tile with
+//   K-major  (rows = M/N, columns = K): SBO = 1024 (8-row groups); a K=16 step
+//            moves the start by 32 bytes inside a block and by BS across blocks;
+//   MN-major (rows = K, columns = M/N): SBO = 1024 (8 K-rows), LBO = BS (next
+//            64 columns of M/N); a K=16 step moves the start by 2048 bytes.
+__host__ __device__ __forceinline__ uint32_t sw_off(int r, int c, int BS) {
+  return (uint32_t)((c >> 6) * BS + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+}
+
 // Shared-memory matrix descriptor, no swizzle, Blackwell version field = 1.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
@@ -39,6 +52,17 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   d |= (uint64_t)1 << 46;  // version
   // base offset 0, LBO mode 0, layout type 0 (no swizzle)
   return d;
+}
+
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return sdesc(saddr, lbo, sbo) | ((uint64_t)2 << 61);   // layout type 2: 128-byte swizzle
+}
+// Descriptor of K step `ks` (16 elements) of a swizzled tile.
+__device__ __forceinline__ uint64_t desc_k_sw(uint32_t base, int ks, int BS) {
+  return sdesc_sw128(base + (uint32_t)((ks >> 2) * BS + (ks & 3) * 32), 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_mn_sw(uint32_t base, int ks, int BS) {
+  return sdesc_sw128(base + (uint32_t)(ks * 2048), (uint32_t)BS, 1024);
 }
 
 // Descriptors for a tiled X[R][C] used as a K-major or MN-major operand.
@@ -198,6 +222,25 @@ __device__ __forceinline__ uint4 pack8_f16(const float* x) {
   return u;
 }
 __device__ __forceinline__ uint4 pack8(const float* x, bool bf16) { return bf16 ? pack8_bf16(x) : pack8_f16(x); }
+
+// Pack 4 floats to 4 16-bit values (8 bytes).
+__device__ __forceinline__ uint2 pack4_f16(float a, float b, float c, float d) {
+  uint2 u;
+  __half2 h;
+  h = __floats2half2_rn(a, b); u.x = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2half2_rn(c, d); u.y = *reinterpret_cast<uint32_t*>(&h);
+  return u;
+}
+__device__ __forceinline__ uint2 pack4_bf16(float a, float b, float c, float d) {
+  uint2 u;
+  __nv_bfloat162 h;
+  h = __floats2bfloat162_rn(a, b); u.x = *reinterpret_cast<uint32_t*>(&h);
+  h = __floats2bfloat162_rn(c, d); u.y = *reinterpret_cast<uint32_t*>(&h);
+  return u;
+}
+__device__ __forceinline__ uint2 pack4(const float* x, bool bf16) {
+  return bf16 ? pack4_bf16(x[0], x[1], x[2], x[3]) : pack4_f16(x[0], x[1], x[2], x[3]);
+}
 
 }  // namespace tc
 }  // namespace gdn2
