@@ -126,12 +126,13 @@ constexpr uint32_t PT_GM = 0, PT_GB = 64, PT_YT = 128, PT_UW = 192, PT_COLS = 25
 constexpr int S_STAGE0 = 0;
 constexpr int S_STAGE1 = SLOT;
 constexpr int S_ST = 2 * SLOT;        // Sᵀ fp16 [128 dv][128 key], BS 16K
-constexpr int S_UT = S_ST + D * D * 2;// Uᵀ fp16 [128 dv][64 tok]; output staging afterwards
-constexpr int S_BAR = S_UT + D * C * 2;   // full[2], mma
-constexpr int S_TMEMP = S_BAR + 32;
+constexpr int S_UT = S_ST + D * D * 2;// Uᵀ fp16 [128 dv][64 tok]
+constexpr int S_OS = S_UT + D * C * 2;// output staging, 16 KB of [rows][128] TOut
+constexpr int S_BAR = S_OS + 16384;   // full[2], ys, st, o
+constexpr int S_TMEMP = S_BAR + 48;
 constexpr int S_FLAG = S_TMEMP + 16;
 constexpr int S_SMEM = S_FLAG + 16;
-constexpr uint32_t ST_S = 0, ST_YS = 128, ST_O = 192, ST_COLS = 256;
+constexpr uint32_t ST_S = 0, ST_YS = 128, ST_O = 192, ST_COLS = 512;   // Oᵀ double-buffered: 192, 256
 
 __device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
   *reinterpret_cast<uint4*>(base + off) = v;
@@ -590,7 +591,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
                                                            float* S_out) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S_BAR);
-  uint64_t* mbar = full + 2;
+  uint64_t* bar_ys = full + 2;          // (Y S)ᵀ done
+  uint64_t* bar_st = full + 3;          // state update done
+  uint64_t* bar_o = full + 4;           // all MMAs of the chunk done
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + S_TMEMP);
   int* sflag = reinterpret_cast<int*>(smem + S_FLAG);
 
@@ -603,7 +606,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   if (tid == 0) {
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
-    mbar_init(mbar, 1);
+    mbar_init(bar_ys, 1);
+    mbar_init(bar_st, 1);
+    mbar_init(bar_o, 1);
     fence_mbar_init();
     *sflag = 0;
   }
@@ -647,18 +652,47 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   }
   sync_for_mma();
 
-  // O staging: [rows][128] of TOut in the 16 KB U tile, which is free once the
-  // chunk's second MMA group has completed.
+  // Output epilogue of a chunk: Oᵀ (TMEM buffer `ob`) → staging tile
+  // [rows][128] of TOut → contiguous 16-byte stores to o, O_ROWS tokens at a
+  // time. It runs while the next chunk's first MMAs execute.
   constexpr int O_ROWS = 16384 / (D * (int)sizeof(TOut));   // 64 (bf16) or 32 (fp32)
+  auto out_epilogue = [&](uint32_t ob, int t0o, int Lco) {
+    TOut* so = reinterpret_cast<TOut*>(smem + S_OS);
+    const int c0 = lo ? 0 : 32;
+    float v[32];
+    tmem_ld16(t_lane + ob + c0, v);
+    tmem_ld16(t_lane + ob + c0 + 16, v + 16);
+    tmem_wait_ld();
+    constexpr int VEC = 16 / (int)sizeof(TOut);             // elements per 16 bytes
+    for (int r0 = 0; r0 < C; r0 += O_ROWS) {
+      if (r0 > 0) __syncthreads();
+      if (c0 >= r0 && c0 < r0 + O_ROWS) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) so[(c0 - r0 + u) * D + row] = from_f32<TOut>(a.scale * v[u]);
+      }
+      __syncthreads();
+      const int nvec = O_ROWS * D / VEC;
+      for (int e = tid; e < nvec; e += NT) {
+        const int rr = e / (D / VEC), cc = (e % (D / VEC)) * VEC;
+        const int i = r0 + rr;
+        if (i < Lco)
+          *reinterpret_cast<uint4*>(og + (((size_t)bi * a.T + t0o + i) * a.Hv + h) * D + cc) =
+              *reinterpret_cast<const uint4*>(so + rr * D + cc);
+      }
+    }
+  };
+
   uint32_t mphase = 0;
   int issued = 1;                       // bulk copies issued (for the error path)
   int waited = 1;
+  int prev_t0 = 0, prev_L = 0;          // chunk whose outputs are still in TMEM
   for (int cl = 0; cl < n_seg; ++cl) {
     const int s = cl & 1;
     uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
     uint8_t* nstg = smem + (s ? S_STAGE0 : S_STAGE1);
     const int t0 = (c_begin + cl) * C;
     const int Lc = min(C, a.T - t0);
+    const uint32_t ob = ST_O + 64u * (uint32_t)s;           // this chunk's Oᵀ buffer
     // prefetch the next chunk into the other stage (free: its MMAs and reads
     // finished before the barrier that closed the previous iteration)
     if (cl + 1 < n_seg) {
@@ -668,20 +702,29 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       }
       ++issued;
     }
-    // (Y S)ᵀ = Sᵀ Yᵀ and Oᵀ = Sᵀ Q̄ᵀ
+    // (Y S)ᵀ = Sᵀ Yᵀ (waited for right away), then Oᵀ = Sᵀ Q̄ᵀ
     if (tid == 0) {
-      const uint32_t st = smem_u32(smem + S_ST);
-      const uint32_t yt = smem_u32(stg + SL_YT), qb = smem_u32(stg + SL_QB);
+      const uint64_t a0 = desc_k_sw(smem_u32(smem + S_ST), 0, BS_ROW128);
+      const uint64_t y0 = desc_mn_sw(smem_u32(stg + SL_YT), 0, BS_ROW128);
+      const uint64_t q0 = desc_k_sw(smem_u32(stg + SL_QB), 0, BS_ROW64);
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint64_t adesc = desc_k_sw(st, ks, BS_ROW128);
-        mma16(tmem + ST_YS, adesc, desc_mn_sw(yt, ks, BS_ROW128), idesc_f16(128, 64, false, true), ks > 0);
-        mma16(tmem + ST_O, adesc, desc_k_sw(qb, ks, BS_ROW64), idesc_f16(128, 64, false, false), ks > 0);
-      }
-      mma_commit(mbar);
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma16(tmem + ST_YS, a0 + k_step_sw(ks, BS_ROW128), y0 + mn_step_sw(ks), idesc_f16(128, 64, false, true),
+              ks > 0);
+      mma_commit(bar_ys);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma16(tmem + ob, a0 + k_step_sw(ks, BS_ROW128), q0 + k_step_sw(ks, BS_ROW64),
+              idesc_f16(128, 64, false, false), ks > 0);
     }
+    // meanwhile: the previous chunk's outputs (its MMAs completed before the
+    // barrier that closed the previous iteration)
+    if (cl > 0) out_epilogue(ST_O + 64u * (uint32_t)(s ^ 1), prev_t0, prev_L);
     __syncwarp();
-    wait_mma(mbar, mphase, sflag);
+    {
+      uint32_t ph = mphase;
+      wait_mma(bar_ys, ph, sflag);
+    }
     // Uᵀ = U_wᵀ − (Y S)ᵀ
     {
       const int c0 = lo ? 0 : 32;
@@ -698,20 +741,26 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       for (int cb = 0; cb < 32; cb += 8) st16(smem, S_UT + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(uw + cb));
     }
     sync_for_mma();
-    // Sᵀ += Uᵀ K_end, Oᵀ += Uᵀ Aqkᵀ
+    // Sᵀ += Uᵀ K_end (waited for by the state copy), then Oᵀ += Uᵀ Aqkᵀ
     if (tid == 0) {
-      const uint32_t ut = smem_u32(smem + S_UT);
-      const uint32_t ke = smem_u32(stg + SL_KE), aq = smem_u32(stg + SL_AQ);
+      const uint64_t u0 = desc_k_sw(smem_u32(smem + S_UT), 0, BS_ROW128);
+      const uint64_t k0 = desc_mn_sw(smem_u32(stg + SL_KE), 0, BS_ROW64);
+      const uint64_t q0 = desc_k_sw(smem_u32(stg + SL_AQ), 0, BS_ROW64);
 #pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks) {
-        const uint64_t adesc = desc_k_sw(ut, ks, BS_ROW128);
-        mma16(tmem + ST_S, adesc, desc_mn_sw(ke, ks, BS_ROW64), idesc_f16(128, 128, false, true), 1);
-        mma16(tmem + ST_O, adesc, desc_k_sw(aq, ks, BS_ROW64), idesc_f16(128, 64, false, false), 1);
-      }
-      mma_commit(mbar);
+      for (int ks = 0; ks < C / 16; ++ks)
+        mma16(tmem + ST_S, u0 + k_step_sw(ks, BS_ROW128), k0 + mn_step_sw(ks), idesc_f16(128, 128, false, true), 1);
+      mma_commit(bar_st);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks)
+        mma16(tmem + ob, u0 + k_step_sw(ks, BS_ROW128), q0 + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, false, false),
+              1);
+      mma_commit(bar_o);
     }
     __syncwarp();
-    wait_mma(mbar, mphase, sflag);
+    {
+      uint32_t ph = mphase;
+      wait_mma(bar_st, ph, sflag);
+    }
     // Next chunk's fp16 Sᵀ operand, then Sᵀ ← Sᵀ Γ_next in TMEM (the next
     // slot's γ_C; its copy was issued at the top of this iteration).
     const bool more = cl + 1 < n_seg;
@@ -740,36 +789,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       }
       if (more) tmem_wait_st();
     }
-    // Outputs o[t0 + i][h][:] through the staging tile, O_ROWS tokens at a time,
-    // written as contiguous 16-byte vectors.
     {
-      TOut* so = reinterpret_cast<TOut*>(smem + S_UT);
-      const int c0 = lo ? 0 : 32;
-      float v[32];
-      tmem_ld16(t_lane + ST_O + c0, v);
-      tmem_ld16(t_lane + ST_O + c0 + 16, v + 16);
-      tmem_wait_ld();
-      constexpr int VEC = 16 / (int)sizeof(TOut);             // elements per 16 bytes
-      for (int r0 = 0; r0 < C; r0 += O_ROWS) {
-        __syncthreads();
-        if (c0 >= r0 && c0 < r0 + O_ROWS) {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) so[(c0 - r0 + u) * D + row] = from_f32<TOut>(a.scale * v[u]);
-        }
-        __syncthreads();
-        const int nvec = O_ROWS * D / VEC;
-        for (int e = tid; e < nvec; e += NT) {
-          const int rr = e / (D / VEC), cc = (e % (D / VEC)) * VEC;
-          const int i = r0 + rr;
-          if (i < Lc)
-            *reinterpret_cast<uint4*>(og + (((size_t)bi * a.T + t0 + i) * a.Hv + h) * D + cc) =
-                *reinterpret_cast<const uint4*>(so + rr * D + cc);
-        }
-      }
+      uint32_t ph = mphase;
+      wait_mma(bar_o, ph, sflag);
+      mphase ^= 1u;                   // the three MMA barriers advance together
     }
+    prev_t0 = t0;
+    prev_L = Lc;
     sync_for_mma();
     if (*sflag) break;
   }
+  // the last chunk's outputs
+  if (!*sflag && n_seg > 0) out_epilogue(ST_O + 64u * (uint32_t)((n_seg - 1) & 1), prev_t0, prev_L);
 
   if (S_out && !*sflag) {
     const int c0 = lo ? 0 : 64;

@@ -65,6 +65,14 @@ __device__ __forceinline__ uint64_t desc_mn_sw(uint32_t base, int ks, int BS) {
   return sdesc_sw128(base + (uint32_t)(ks * 2048), (uint32_t)BS, 1024);
 }
 
+// Increments to add to the descriptor of K step 0 to reach K step `ks` (the
+// start-address field counts 16-byte units; shared addresses stay < 256 KB,
+// so the addition never carries out of the field).
+__host__ __device__ constexpr uint64_t k_step_sw(int ks, int BS) {
+  return (uint64_t)(((ks >> 2) * BS + (ks & 3) * 32) >> 4);
+}
+__host__ __device__ constexpr uint64_t mn_step_sw(int ks) { return (uint64_t)((ks * 2048) >> 4); }
+
 // Descriptors for a tiled X[R][C] used as a K-major or MN-major operand.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, int C) { return sdesc(saddr, 128, (C / 8) * 128); }
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr, int C) { return sdesc(saddr, (C / 8) * 128, 128); }
