@@ -200,9 +200,69 @@ __device__ __forceinline__ void sync_for_mma() {
 }
 
 // =============================================================================
-// prep kernel: one CTA per (chunk of the segment, sequence, value head)
+// prep kernel: persistent, one 512-thread CTA per SM looping over the work
+// items (chunk of the segment, sequence, value head). Each item's inputs are
+// loaded in one round into registers; the next item's loads are issued as
+// soon as the current item's elementwise pass has consumed its registers, so
+// they arrive while the Gram, inverse and Yᵀ/U_wᵀ phases run.
 // =============================================================================
-__global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg) {
+constexpr int NP = 512;               // prep threads (16 warps)
+
+// Inputs of one token for 4 channels (a warp reads whole rows).
+struct TokIn {
+  float4 al, b, w;
+  uint2 k, q, v;
+};
+struct PrepSrc {
+  const float *alpha, *b, *w;
+  const __nv_bfloat16 *k, *q, *v;
+  int T, Hqk, Hv, mode;
+};
+
+__device__ __forceinline__ void load_token(const PrepSrc& p, int bi, int t, int h, int hq, int c4, bool valid,
+                                           TokIn& r) {
+  if (valid) {
+    const size_t gt = ((size_t)bi * p.T + t) * p.Hv + h;
+    const size_t tq = ((size_t)bi * p.T + t) * p.Hqk + hq;
+    if (p.mode == GDN2_GATES_GDN) {
+      const float sa = __ldg(p.alpha + gt);
+      r.al = make_float4(sa, sa, sa, sa);
+    } else {
+      r.al = __ldg(reinterpret_cast<const float4*>(p.alpha + gt * D + c4));
+    }
+    if (p.mode == GDN2_GATES_FULL) {
+      r.b = __ldg(reinterpret_cast<const float4*>(p.b + gt * D + c4));
+      r.w = __ldg(reinterpret_cast<const float4*>(p.w + gt * D + c4));
+    } else {
+      const float beta = __ldg(p.b + gt);
+      r.b = r.w = make_float4(beta, beta, beta, beta);
+    }
+    r.k = __ldg(reinterpret_cast<const uint2*>(p.k + tq * D + c4));
+    r.q = __ldg(reinterpret_cast<const uint2*>(p.q + tq * D + c4));
+    r.v = __ldg(reinterpret_cast<const uint2*>(p.v + gt * D + c4));
+  } else {
+    r.al = make_float4(1.f, 1.f, 1.f, 1.f);
+    r.b = r.w = make_float4(0.f, 0.f, 0.f, 0.f);
+    r.k = r.q = r.v = make_uint2(0, 0);
+  }
+}
+
+struct Item {
+  int bh, cl, h, bi, hq, t0, Lc;
+};
+__device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int item) {
+  Item it;
+  it.bh = item % (a.B * a.Hv);      // value head fastest: heads sharing q, k run together
+  it.cl = item / (a.B * a.Hv);
+  it.h = it.bh % a.Hv;
+  it.bi = it.bh / a.Hv;
+  it.hq = it.h / (a.Hv / a.Hqk);
+  it.t0 = (c_begin + it.cl) * C;
+  it.Lc = min(C, a.T - it.t0);
+  return it;
+}
+
+__global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + P_BAR);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + P_TMEMP);
@@ -210,20 +270,12 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   float* sPq = reinterpret_cast<float*>(smem + P_PQ);
   float* sred = reinterpret_cast<float*>(smem + P_RED);
   float* stage = reinterpret_cast<float*>(smem + P_STG);
+  float* sT = reinterpret_cast<float*>(smem + P_T);
+  float* sI = reinterpret_cast<float*>(smem + P_I);
+  float* sX = reinterpret_cast<float*>(smem + P_X);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // CTA order: value head fastest, so the value heads sharing a query/key head
-  // run together and share its q, k lines in L2.
-  const int work = blockIdx.x;
-  const int bh = work % (a.B * a.Hv);
-  const int cl = work / (a.B * a.Hv);          // chunk within the segment
-  const int ck = c_begin + cl;
-  const int h = bh % a.Hv, bi = bh / a.Hv;
-  const int hq = h / (a.Hv / a.Hqk);
-  const int t0 = ck * C;
-  const int Lc = min(C, a.T - t0);
-  uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)bh * n_seg + cl) * SLOT;
-
+  const int n_items = a.B * a.Hv * n_seg;
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
@@ -233,121 +285,99 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     tmem_alloc(tmem_ptr, PT_COLS);
     tmem_relinquish();
   }
-
-  // Element mapping: lane → 4 channels (a warp covers a whole 128-channel
-  // row), warp → tokens warp, warp + 8, ..., so token j·8 + warp lies in
-  // quarter j/2.
-  const int c4 = lane * 4;
-
-  // -------- pass 1: α rows into the staging tile; the write side Z = w ⊙ v
-  // (which needs no decay) goes straight to its tile
-  {
-    float4 al[8], wv[8];
-    uint2 vv[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = warp + 8 * j;
-      al[j] = make_float4(1.f, 1.f, 1.f, 1.f);
-      wv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      vv[j] = make_uint2(0, 0);
-      if (i < Lc) {
-        const size_t gt = ((size_t)bi * a.T + t0 + i) * a.Hv + h;
-        if (a.gate_mode == GDN2_GATES_GDN) {
-          const float sa = __ldg(a.alpha + gt);
-          al[j] = make_float4(sa, sa, sa, sa);
-        } else {
-          al[j] = __ldg(reinterpret_cast<const float4*>(a.alpha + gt * D + c4));
-        }
-        if (a.gate_mode == GDN2_GATES_FULL) {
-          wv[j] = __ldg(reinterpret_cast<const float4*>(a.w + gt * D + c4));
-        } else {
-          const float beta = __ldg(a.b + gt);
-          wv[j] = make_float4(beta, beta, beta, beta);
-        }
-        vv[j] = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.v) + gt * D + c4));
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = warp + 8 * j;
-      *reinterpret_cast<float4*>(stage + i * SS + c4) = al[j];
-      float vx[4];
-      unpack4_bf16(vv[j], vx);
-      st8(smem, P_Z + sw_off(i, c4, BS_ROW64),
-          pack4_f16(wv[j].x * vx[0], wv[j].y * vx[1], wv[j].z * vx[2], wv[j].w * vx[3]));
-    }
-  }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_ptr;
-  // forward cumulative products down each channel within each quarter
-  {
-    const int c = tid & 127;
-    float mn = 1.f;
+  const int lq = warp & 3;                       // TMEM lane quarter of this warp
+  const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
+  const int row = lq * 32 + lane;
+  const int cgp = warp >> 2;                     // column group (0..3) among warps of a lane quarter
+
+  // Element mapping: lane → 4 channels c4..c4+3 (a warp covers a whole row),
+  // warp w → token w + 16 j of quarter j (j = 0..3).
+  const int c4 = lane * 4;
+  // Swizzled offsets of this thread's 4-channel piece: every token it handles
+  // has row ≡ warp (mod 8), so only a multiple of 128 bytes depends on the row.
+  const uint32_t col64 = sw_off(warp & 7, c4, BS_ROW64) - (uint32_t)((warp & 7) * 128);
+  const uint32_t col128 = sw_off(warp & 7, c4, BS_ROW128) - (uint32_t)((warp & 7) * 128);
+  const PrepSrc src{a.alpha, a.b, a.w, static_cast<const __nv_bfloat16*>(a.k),
+                    static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.v),
+                    a.T, a.Hqk, a.Hv, a.gate_mode};
+  TokIn in[4];
+  int item = blockIdx.x;
+  if (item < n_items) {
+    const Item it = decode_item(a, c_begin, item);
 #pragma unroll
-    for (int q = tid >> 7; q < 4; q += 2) {
+    for (int j = 0; j < 4; ++j) {
+      const int i = warp + 16 * j;
+      load_token(src, it.bi, it.t0 + i, it.h, it.hq, c4, i < it.Lc, in[j]);
+    }
+  }
+  uint32_t phase = 0;
+  for (; item < n_items; item += gridDim.x) {
+    const Item it = decode_item(a, c_begin, item);
+    uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)it.bh * n_seg + it.cl) * SLOT;
+
+    // -------- pass 1: α rows into the staging tile; the write side Z = w ⊙ v
+    // (which needs no decay) goes straight to its tile
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = warp + 16 * j;
+      *reinterpret_cast<float4*>(stage + i * SS + c4) = in[j].al;
+      float vx[4];
+      unpack4_bf16(in[j].v, vx);
+      st8(smem, P_Z + col64 + i * 128,
+          pack4_f16(in[j].w.x * vx[0], in[j].w.y * vx[1], in[j].w.z * vx[2], in[j].w.w * vx[3]));
+    }
+    __syncthreads();
+    // forward cumulative products down each channel within each quarter
+    {
+      const int c = tid & 127, q = tid >> 7;
       float acc = 1.f;
 #pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        float* p = stage + (16 * q + s) * SS + c;
-        acc *= *p;
-        *p = acc;
+      for (int s_ = 0; s_ < 16; ++s_) {
+        float* pp = stage + (16 * q + s_) * SS + c;
+        acc *= *pp;
+        *pp = acc;
       }
       sPq[q * D + c] = acc;
-      mn = fminf(mn, acc);
+      float mn = acc;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      if (lane == 0) sred[warp] = mn;
     }
+    __syncthreads();
+    bool gram_bf16;
+    {
+      float mall = sred[0];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    if (lane == 0) sred[warp] = mn;
-  }
-  __syncthreads();
-  bool gram_bf16;
-  {
-    float mall = sred[0];
+      for (int w_ = 1; w_ < NP / 32; ++w_) mall = fminf(mall, sred[w_]);
+      // every in-quarter forward/backward product is ≥ the quarter product
+      gram_bf16 = !(mall > 6.103515625e-05f);   // 2^-14
+    }
+    if (tid < D) {
+      const float g = sPq[tid] * sPq[D + tid] * sPq[2 * D + tid] * sPq[3 * D + tid];
+      reinterpret_cast<float*>(slot + SL_GC)[tid] = g;
+    }
+    float fw[4][4], Pq[4][4];
 #pragma unroll
-    for (int w_ = 1; w_ < 8; ++w_) mall = fminf(mall, sred[w_]);
-    // every in-quarter forward/backward product is ≥ the quarter product
-    gram_bf16 = !(mall > 6.103515625e-05f);   // 2^-14
-  }
-  if (tid < D) {
-    const float g = sPq[tid] * sPq[D + tid] * sPq[2 * D + tid] * sPq[3 * D + tid];
-    reinterpret_cast<float*>(slot + SL_GC)[tid] = g;
-  }
-  float fw[8][4], Pq[4][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float4 v = *reinterpret_cast<const float4*>(stage + (warp + 8 * j) * SS + c4);
-    fw[j][0] = v.x; fw[j][1] = v.y; fw[j][2] = v.z; fw[j][3] = v.w;
-  }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 v = *reinterpret_cast<const float4*>(sPq + q * D + c4);
-    Pq[q][0] = v.x; Pq[q][1] = v.y; Pq[q][2] = v.z; Pq[q][3] = v.w;
-  }
-  __syncthreads();   // the staging tile is free from here on
+    for (int j = 0; j < 4; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(stage + (warp + 16 * j) * SS + c4);
+      fw[j][0] = v.x; fw[j][1] = v.y; fw[j][2] = v.z; fw[j][3] = v.w;
+      const float4 pq = *reinterpret_cast<const float4*>(sPq + j * D + c4);
+      Pq[j][0] = pq.x; Pq[j][1] = pq.y; Pq[j][2] = pq.z; Pq[j][3] = pq.w;
+    }
+    __syncthreads();   // the staging tile is free from here on
 
-  // -------- pass 2: key-side operand tiles, PB tokens in flight at a time
-  constexpr int PB = 4;
-  const RowSrc src{static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.q), a.b, a.T, a.Hqk,
-                   a.Hv, a.gate_mode == GDN2_GATES_FULL};
+    // -------- pass 2: key-side operand tiles (token i = warp + 16 m is in quarter m)
 #pragma unroll
-  for (int bt = 0; bt < 8 / PB; ++bt) {
-    KeyIn in[PB];
-#pragma unroll
-    for (int jj = 0; jj < PB; ++jj) {
-      const int i = warp + 8 * (PB * bt + jj);
-      load_key_row(src, bi, t0 + i, h, hq, c4, i < Lc, in[jj]);
-    }
-#pragma unroll
-    for (int jj = 0; jj < PB; ++jj) {
-      const int j = PB * bt + jj;
-      const int m = j >> 1;               // quarter of token i
-      const int i = warp + 8 * j;
+    for (int m = 0; m < 4; ++m) {
+      const int i = warp + 16 * m;
       float kx[4], qx[4], ex[4];
-      unpack4_bf16(in[jj].k, kx);
-      unpack4_bf16(in[jj].q, qx);
-      ex[0] = in[jj].b.x * kx[0]; ex[1] = in[jj].b.y * kx[1]; ex[2] = in[jj].b.z * kx[2]; ex[3] = in[jj].b.w * kx[3];
+      unpack4_bf16(in[m].k, kx);
+      unpack4_bf16(in[m].q, qx);
+      ex[0] = in[m].b.x * kx[0]; ex[1] = in[m].b.y * kx[1]; ex[2] = in[m].b.z * kx[2]; ex[3] = in[m].b.w * kx[3];
       float o_eb[4], o_qb[4], o_ke[4], o_em[4], o_qm[4], o_km[4], o_x1[4], o_x2[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -358,7 +388,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           if (mm < m) pre *= Pq[mm][c];
           if (mm > m) suf *= Pq[mm][c];
         }
-        const float f = fw[j][c];               // Π_{quarter start ≤ s ≤ i} α
+        const float f = fw[m][c];               // Π_{quarter start ≤ s ≤ i} α
         const float rf = __fdividef(1.f, f);
         const float bw = P * rf;                // Π_{i < s ≤ quarter end} α
         const float g = pre * f;                // γ_i
@@ -387,195 +417,196 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           o_x2[c] = 0.f;
         }
       }
-      st8(slot, SL_QB + sw_off(i, c4, BS_ROW64), pack4(o_qb, false));
-      st8(slot, SL_KE + sw_off(i, c4, BS_ROW64), pack4(o_ke, false));
-      st8(smem, P_EB + sw_off(i, c4, BS_ROW64), pack4(o_eb, false));
-      st8(smem, P_GM + sw_off(i, c4, BS_ROW128), pack4(o_em, gram_bf16));
-      st8(smem, P_GM + sw_off(64 + i, c4, BS_ROW128), pack4(o_qm, gram_bf16));
-      st8(smem, P_KM + sw_off(i, c4, BS_ROW64), pack4(o_km, gram_bf16));
+      st8(slot, SL_QB + col64 + i * 128, pack4(o_qb, false));
+      st8(slot, SL_KE + col64 + i * 128, pack4(o_ke, false));
+      st8(smem, P_EB + col64 + i * 128, pack4(o_eb, false));
+      st8(smem, P_GM + col128 + i * 128, pack4(o_em, gram_bf16));
+      st8(smem, P_GM + col128 + (64 + i) * 128, pack4(o_qm, gram_bf16));
+      st8(smem, P_KM + col64 + i * 128, pack4(o_km, gram_bf16));
       if (m >= 2) {
-        st8(smem, P_GB + sw_off(i, c4, BS_ROW128), pack4(o_x1, gram_bf16));
-        st8(smem, P_GB + sw_off(64 + i, c4, BS_ROW128), pack4(o_x2, gram_bf16));
+        st8(smem, P_GB + col128 + i * 128, pack4(o_x1, gram_bf16));
+        st8(smem, P_GB + col128 + (64 + i) * 128, pack4(o_x2, gram_bf16));
       } else {
-        st8(smem, P_KB + sw_off(i, c4, BS_ROW128), pack4(o_x1, gram_bf16));
+        st8(smem, P_KB + col128 + i * 128, pack4(o_x1, gram_bf16));
       }
     }
-    // keep the next batch's loads from being hoisted above this one (register
-    // pressure): one batch of rows in flight at a time
-    asm volatile("" ::: "memory");
-  }
-  sync_for_mma();
-
-  // -------- Gram MMAs: [T; Aqk] candidates
-  uint32_t phase = 0;
-  if (tid == 0) {
-    const uint32_t gm = smem_u32(smem + P_GM), km = smem_u32(smem + P_KM);
-    const uint32_t gb = smem_u32(smem + P_GB), kb = smem_u32(smem + P_KB);
+    // the next item's inputs: issued now, consumed at the top of the next pass
+    {
+      const int nxt = item + (int)gridDim.x;
+      if (nxt < n_items) {
+        const Item in_ = decode_item(a, c_begin, nxt);
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      mma16(tmem + PT_GM, desc_k_sw(gm, ks, BS_ROW128), desc_k_sw(km, ks, BS_ROW64),
-            idesc_16(128, 64, false, false, gram_bf16), ks > 0);
-      mma16(tmem + PT_GB, desc_k_sw(gb, ks, BS_ROW128), desc_k_sw(kb, ks, BS_ROW128),
-            idesc_16(128, 32, false, false, gram_bf16), ks > 0);
+        for (int j = 0; j < 4; ++j) {
+          const int i = warp + 16 * j;
+          load_token(src, in_.bi, in_.t0 + i, in_.h, in_.hq, c4, i < in_.Lc, in[j]);
+        }
+      }
     }
-    mma_commit(bar);
-  }
-  __syncwarp();
-  wait_mma(bar, phase, sflag);
+    sync_for_mma();
 
-  // -------- T (fp32, shared) and Aqk (fp16, workspace) from TMEM
-  float* sT = reinterpret_cast<float*>(smem + P_T);
-  float* sI = reinterpret_cast<float*>(smem + P_I);
-  float* sX = reinterpret_cast<float*>(smem + P_X);
-  const int lq = warp & 3;
-  const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
-  const int row = lq * 32 + lane;
-  const bool lo = warp < 4;
-  {
-    // lanes 0..63: rows of T; lanes 64..127: rows of Aqk. Warps 0-3 take
-    // columns 0..31, warps 4-7 columns 32..63.
-    const bool is_t = row < 64;
-    const int i = row & 63;
-    const int j0 = lo ? 0 : 32;
+    // -------- Gram MMAs: [T; Aqk] candidates
+    if (tid == 0) {
+      const uint64_t gm = desc_k_sw(smem_u32(smem + P_GM), 0, BS_ROW128);
+      const uint64_t km = desc_k_sw(smem_u32(smem + P_KM), 0, BS_ROW64);
+      const uint64_t gb = desc_k_sw(smem_u32(smem + P_GB), 0, BS_ROW128);
+      const uint64_t kb = desc_k_sw(smem_u32(smem + P_KB), 0, BS_ROW128);
+      const uint32_t id_m = idesc_16(128, 64, false, false, gram_bf16);
+      const uint32_t id_b = idesc_16(128, 32, false, false, gram_bf16);
 #pragma unroll
-    for (int jb = 0; jb < 32; jb += 16) {
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma16(tmem + PT_GM, gm + k_step_sw(ks, BS_ROW128), km + k_step_sw(ks, BS_ROW64), id_m, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma16(tmem + PT_GB, gb + k_step_sw(ks, BS_ROW128), kb + k_step_sw(ks, BS_ROW128), id_b, ks > 0);
+      mma_commit(bar);
+    }
+    __syncwarp();
+    wait_mma(bar, phase, sflag);
+
+    // -------- T (fp32, shared) and Aqk (fp16, workspace) from TMEM. Lanes
+    // 0..63 hold rows of T, lanes 64..127 rows of Aqk; the four warps of a
+    // lane quarter take 16 columns each.
+    {
+      const bool is_t = row < 64;
+      const int i = row & 63;
+      const int j0 = 16 * cgp;
       float dm[16], db[16];
-      tmem_ld16(t_lane + PT_GM + j0 + jb, dm);
-      tmem_ld16(t_lane + PT_GB + jb, db);
+      tmem_ld16(t_lane + PT_GM + j0, dm);
+      tmem_ld16(t_lane + PT_GB + (j0 & 31), db);
       tmem_wait_ld();
       float v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        const int j = j0 + jb + u;
+        const int j = j0 + u;
         const bool keep = is_t ? (j < i) : (j <= i);
         const bool same = (j >> 5) == (i >> 5);
-        const float x = same ? dm[u] : (j0 == 0 ? db[u] : 0.f);
+        const float x = same ? dm[u] : (j0 < 32 ? db[u] : 0.f);
         v[u] = keep ? x : 0.f;
       }
       if (is_t) {
 #pragma unroll
         for (int u = 0; u < 16; u += 4)
-          *reinterpret_cast<float4*>(sT + i * TS + j0 + jb + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+          *reinterpret_cast<float4*>(sT + i * TS + j0 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
       } else {
-        st16(slot, SL_AQ + sw_off(i, j0 + jb, BS_ROW64), pack8_f16(v));
-        st16(slot, SL_AQ + sw_off(i, j0 + jb + 8, BS_ROW64), pack8_f16(v + 8));
+        st16(slot, SL_AQ + sw_off(i, j0, BS_ROW64), pack8_f16(v));
+        st16(slot, SL_AQ + sw_off(i, j0 + 8, BS_ROW64), pack8_f16(v + 8));
       }
     }
-  }
-  __syncthreads();
+    __syncthreads();
 
-  // -------- A = (I + T)⁻¹, blocked
-  // level 0: the four 16 × 16 diagonal blocks by forward substitution, one
-  // column per thread; the other threads zero the two upper-right 16 × 16
-  // blocks of the 32-halves (read by the level-2 products).
-  if (tid < 64) {
-    const int blk = tid >> 4, j = tid & 15, base = blk * 16;
-    float x[16];
+    // -------- A = (I + T)⁻¹, blocked
+    // level 0: the four 16 × 16 diagonal blocks by forward substitution, one
+    // column per thread; the others zero the upper-right 16 × 16 block of each
+    // 32-half (read by the level-2 products).
+    if (tid < 64) {
+      const int blk = tid >> 4, j = tid & 15, base = blk * 16;
+      float x[16];
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      float acc = (ii == j) ? 1.f : 0.f;
+      for (int ii = 0; ii < 16; ++ii) {
+        float acc = (ii == j) ? 1.f : 0.f;
 #pragma unroll
-      for (int l = 0; l < ii; ++l)
-        if (l >= j) acc -= sT[(base + ii) * TS + base + l] * x[l];
-      x[ii] = (ii >= j) ? acc : 0.f;
+        for (int l = 0; l < ii; ++l)
+          if (l >= j) acc -= sT[(base + ii) * TS + base + l] * x[l];
+        x[ii] = (ii >= j) ? acc : 0.f;
+      }
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) sI[(base + ii) * TS + base + j] = x[ii];
+    } else {
+      for (int o = tid - 64; o < 512; o += NP - 64) {
+        const int hf = o >> 8, ii = (o >> 4) & 15, jj = o & 15;
+        sI[(hf * 32 + ii) * TS + hf * 32 + 16 + jj] = 0.f;
+      }
     }
+    __syncthreads();
+    // level 1: X21 = −I22 T21 I11 in each 32-half (one entry per thread)
+    {
+      const int hf = tid >> 8, ii = (tid >> 4) & 15, jj = tid & 15;
+      const int r0 = hf * 32 + 16, c0 = hf * 32;
+      float acc = 0.f;
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) sI[(base + ii) * TS + base + j] = x[ii];
-  } else {
-    for (int o = tid - 64; o < 512; o += NT - 64) {
-      const int hf = o >> 8, ii = (o >> 4) & 15, jj = o & 15;
-      sI[(hf * 32 + ii) * TS + hf * 32 + 16 + jj] = 0.f;
+      for (int l = 0; l < 16; ++l) acc += sT[(r0 + ii) * TS + c0 + l] * sI[(c0 + l) * TS + c0 + jj];
+      sX[(hf * 16 + ii) * 36 + jj] = acc;
     }
-  }
-  __syncthreads();
-  // level 1: X21 = −I22 T21 I11 in each 32-half (thread: 4 columns)
-  if (tid < 128) {
-    const int hf = tid >> 6, ii = (tid >> 2) & 15, jq = (tid & 3) * 4;
-    const int r0 = hf * 32 + 16, c0 = hf * 32;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    __syncthreads();
+    {
+      const int hf = tid >> 8, ii = (tid >> 4) & 15, jj = tid & 15;
+      const int r0 = hf * 32 + 16, c0 = hf * 32;
+      float acc = 0.f;
 #pragma unroll
-    for (int l = 0; l < 16; ++l) {
-      const float t = sT[(r0 + ii) * TS + c0 + l];
-      const float4 iv = *reinterpret_cast<const float4*>(sI + (c0 + l) * TS + c0 + jq);
-      acc[0] += t * iv.x; acc[1] += t * iv.y; acc[2] += t * iv.z; acc[3] += t * iv.w;
+      for (int l = 0; l < 16; ++l) acc += sI[(r0 + ii) * TS + r0 + l] * sX[(hf * 16 + l) * 36 + jj];
+      sI[(r0 + ii) * TS + c0 + jj] = -acc;
     }
-    *reinterpret_cast<float4*>(sX + (hf * 16 + ii) * 36 + jq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  }
-  __syncthreads();
-  if (tid < 128) {
-    const int hf = tid >> 6, ii = (tid >> 2) & 15, jq = (tid & 3) * 4;
-    const int r0 = hf * 32 + 16, c0 = hf * 32;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int l = 0; l < 16; ++l) {
-      const float t = sI[(r0 + ii) * TS + r0 + l];
-      const float4 xv = *reinterpret_cast<const float4*>(sX + (hf * 16 + l) * 36 + jq);
-      acc[0] += t * xv.x; acc[1] += t * xv.y; acc[2] += t * xv.z; acc[3] += t * xv.w;
-    }
-    *reinterpret_cast<float4*>(sI + (r0 + ii) * TS + c0 + jq) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-  }
-  __syncthreads();
-  // level 2: X_QP = −I_QQ T_QP I_PP (thread: row ii, 4 columns)
-  {
-    const int ii = tid >> 3, jq = (tid & 7) * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    __syncthreads();
+    // level 2: X_QP = −I_QQ T_QP I_PP (thread: row ii, 2 columns)
+    {
+      const int ii = tid >> 4, jp = (tid & 15) * 2;
+      float a0 = 0.f, a1 = 0.f;
 #pragma unroll 8
-    for (int l = 0; l < 32; ++l) {
-      const float t = sT[(32 + ii) * TS + l];
-      const float4 iv = *reinterpret_cast<const float4*>(sI + l * TS + jq);
-      acc[0] += t * iv.x; acc[1] += t * iv.y; acc[2] += t * iv.z; acc[3] += t * iv.w;
+      for (int l = 0; l < 32; ++l) {
+        const float t = sT[(32 + ii) * TS + l];
+        const float2 iv = *reinterpret_cast<const float2*>(sI + l * TS + jp);
+        a0 += t * iv.x; a1 += t * iv.y;
+      }
+      *reinterpret_cast<float2*>(sX + ii * 36 + jp) = make_float2(a0, a1);
     }
-    *reinterpret_cast<float4*>(sX + ii * 36 + jq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  }
-  __syncthreads();
-  {
-    const int ii = tid >> 3, jq = (tid & 7) * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    __syncthreads();
+    {
+      const int ii = tid >> 4, jp = (tid & 15) * 2;
+      float a0 = 0.f, a1 = 0.f;
 #pragma unroll 8
-    for (int l = 0; l < 32; ++l) {
-      const float t = sI[(32 + ii) * TS + 32 + l];
-      const float4 xv = *reinterpret_cast<const float4*>(sX + l * 36 + jq);
-      acc[0] += t * xv.x; acc[1] += t * xv.y; acc[2] += t * xv.z; acc[3] += t * xv.w;
+      for (int l = 0; l < 32; ++l) {
+        const float t = sI[(32 + ii) * TS + 32 + l];
+        const float2 xv = *reinterpret_cast<const float2*>(sX + l * 36 + jp);
+        a0 += t * xv.x; a1 += t * xv.y;
+      }
+      *reinterpret_cast<float2*>(sI + (32 + ii) * TS + jp) = make_float2(-a0, -a1);
     }
-    *reinterpret_cast<float4*>(sI + (32 + ii) * TS + jq) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-  }
-  __syncthreads();
-  // pack A (lower triangle; zeros above the diagonal)
-  for (int o = tid; o < C * 8; o += NT) {
-    const int i = o >> 3, j0 = (o & 7) * 8;
-    float x[8];
+    __syncthreads();
+    // pack A (lower triangle; zeros above the diagonal), one 8-wide piece per thread
+    {
+      const int i = tid >> 3, j0 = (tid & 7) * 8;
+      float x[8];
+      const float4 p0 = *reinterpret_cast<const float4*>(sI + i * TS + j0);
+      const float4 p1 = *reinterpret_cast<const float4*>(sI + i * TS + j0 + 4);
+      x[0] = p0.x; x[1] = p0.y; x[2] = p0.z; x[3] = p0.w; x[4] = p1.x; x[5] = p1.y; x[6] = p1.z; x[7] = p1.w;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = (j0 + u <= i) ? sI[i * TS + j0 + u] : 0.f;
-    st16(smem, P_AINV + sw_off(i, j0, BS_ROW64), pack8_f16(x));
-  }
-  sync_for_mma();
+      for (int u = 0; u < 8; ++u) x[u] = (j0 + u <= i) ? x[u] : 0.f;
+      st16(smem, P_AINV + sw_off(i, j0, BS_ROW64), pack8_f16(x));
+    }
+    sync_for_mma();
 
-  // -------- Yᵀ = Ēᵀ Aᵀ, U_wᵀ = Zᵀ Aᵀ
-  if (tid == 0) {
-    const uint32_t eb = smem_u32(smem + P_EB), z = smem_u32(smem + P_Z);
-    const uint32_t ai = smem_u32(smem + P_AINV);
+    // -------- Yᵀ = Ēᵀ Aᵀ, U_wᵀ = Zᵀ Aᵀ
+    if (tid == 0) {
+      const uint64_t eb = desc_mn_sw(smem_u32(smem + P_EB), 0, BS_ROW64);
+      const uint64_t z = desc_mn_sw(smem_u32(smem + P_Z), 0, BS_ROW64);
+      const uint64_t ai = desc_k_sw(smem_u32(smem + P_AINV), 0, BS_ROW64);
 #pragma unroll
-    for (int ks = 0; ks < C / 16; ++ks) {
-      const uint64_t bdesc = desc_k_sw(ai, ks, BS_ROW64);
-      mma16(tmem + PT_YT, desc_mn_sw(eb, ks, BS_ROW64), bdesc, idesc_f16(128, 64, true, false), ks > 0);
-      mma16(tmem + PT_UW, desc_mn_sw(z, ks, BS_ROW64), bdesc, idesc_f16(128, 64, true, false), ks > 0);
+      for (int ks = 0; ks < C / 16; ++ks)
+        mma16(tmem + PT_YT, eb + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
+              ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks)
+        mma16(tmem + PT_UW, z + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
+              ks > 0);
+      mma_commit(bar);
     }
-    mma_commit(bar);
-  }
-  __syncwarp();
-  wait_mma(bar, phase, sflag);
-  {
-    // warps 0-3: Yᵀ rows (key lanes); warps 4-7: U_wᵀ rows (dv lanes)
-    const uint32_t col = lo ? PT_YT : PT_UW;
-    const int dst = lo ? SL_YT : SL_UW;
-#pragma unroll
-    for (int cb = 0; cb < C; cb += 16) {
-      float v[16];
-      tmem_ld16(t_lane + col + cb, v);
+    __syncwarp();
+    wait_mma(bar, phase, sflag);
+    {
+      // column groups 0, 1: Yᵀ rows (key lanes); 2, 3: U_wᵀ rows (dv lanes)
+      const uint32_t col = (cgp < 2 ? PT_YT : PT_UW) + 32u * (uint32_t)(cgp & 1);
+      const int dst = cgp < 2 ? SL_YT : SL_UW;
+      const int cb0 = 32 * (cgp & 1);
+      float v[32];
+      tmem_ld16(t_lane + col, v);
+      tmem_ld16(t_lane + col + 16, v + 16);
       tmem_wait_ld();
-      st16(slot, dst + sw_off(row, cb, BS_ROW128), pack8_f16(v));
-      st16(slot, dst + sw_off(row, cb + 8, BS_ROW128), pack8_f16(v + 8));
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 8) st16(slot, dst + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
     }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
   }
   if (*sflag && tid == 0) atomicOr(static_cast<int*>(a.workspace), 1);
   fence_before_sync();
@@ -868,12 +899,15 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   auto scan = o_bf16 ? chunk_scan_kernel<__nv_bfloat16> : chunk_scan_kernel<float>;
   if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM)) != cudaSuccess) return e;
 
+  int dev = 0, sms = 148;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const float* s_in = a.S0;
   for (int c0 = 0; c0 < nchunks; c0 += seg) {
     const int n = std::min(seg, nchunks - c0);
     const bool last = c0 + n >= nchunks;
     float* s_out = last ? a.ST : carry;
-    chunk_prep_kernel<<<BH * n, NT, P_SMEM, s>>>(a, c0, n);
+    chunk_prep_kernel<<<std::min(BH * n, sms), NP, P_SMEM, s>>>(a, c0, n);
     scan<<<BH, NT, S_SMEM, s>>>(a, c0, n, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;
