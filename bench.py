@@ -7,6 +7,11 @@ token per step, fp32 states [256,48,128,128]) is timed in the same run and
 reported under "decode".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill_t32768|prefill_t4096] [--decode-workload decode_b256|decode_b64]
+                    [--decode-steps N] [--e2e-steps N]
+
+(--workload prefill_t4096 / --decode-workload decode_b64 are the small cases
+the ncu captures run; --decode-steps 0 / --e2e-steps 0 skip those parts.)
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own sequence
 (independent problems, no data-path collective); value = tokens of all ranks /
@@ -20,6 +25,7 @@ workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -36,6 +42,14 @@ METRIC = "prefill tokens/s (48 Vheads x 128^2, T=32K) + % tensor peak; decode HB
 PREFILL = "prefill_t32768"
 DECODE = "decode_b256"
 L2_BYTES = 126 * 2**20
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the two prefill
+# launches of one call, from an ncu capture of prefill_t4096 scaled by 8 to the
+# T=32768 workload (traffic grows with the number of chunks), and the hash of
+# the kernel sources it was taken on; with other sources the figure is stale
+# and the bench reports null.
+TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
+TRAFFIC = {"sha1": None, "bytes_per_call": None, "profile": None}
 
 
 def peaks():
@@ -81,6 +95,21 @@ def decode_bytes(w, o_bytes=2):
     state = B * w.H_v * d * d * 4 * 2
     io = B * w.H_qk * d * 2 * 2 + B * w.H_v * d * 2 + B * w.H_v * d * 4 * 3 + B * w.H_v * d * o_bytes
     return state + io
+
+
+def kernel_sources_sha1():
+    h = hashlib.sha1()
+    for rel in TRAFFIC_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """Per-call DRAM traffic of the prefill kernels if it was captured on the current sources."""
+    if TRAFFIC["sha1"] is None or TRAFFIC["sha1"] != kernel_sources_sha1():
+        return None
+    return TRAFFIC["bytes_per_call"]
 
 
 # ------------------------------------------------------------------ clocks
@@ -236,6 +265,9 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=PREFILL, choices=[PREFILL, "prefill_t4096"],
+                    help="prefill workload to time (the small one is for profiler captures)")
+    ap.add_argument("--decode-workload", default=DECODE, choices=[DECODE, "decode_b64"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -262,7 +294,7 @@ def main():
             dist.barrier()
 
     pk = peaks()
-    w = workload(PREFILL)
+    w = workload(args.workload)
     stream = torch.cuda.Stream(device=dev)
     inp = make_inputs(w, seed=rank_seed(rank), device=dev)
     o = torch.empty((w.B, w.T, w.H_v, w.d), dtype=torch.bfloat16, device=dev)
@@ -270,7 +302,9 @@ def main():
     p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk)
     ws_bytes = gdn2.chunk_fwd_workspace(p)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    launches_per_call = 1
+    # the tensor-core path (the one that takes a workspace) launches a prep and
+    # a scan kernel per call when the workspace holds the whole sequence
+    launches_per_call = 2 if ws_bytes > 0 else 1
 
     def prefill_call():
         gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None, chunk=w.chunk,
@@ -299,17 +333,56 @@ def main():
 
     nbytes = prefill_bytes(w)
     flops = prefill_flops(w)
-    kernel_s = ms * 1e-3  # one launch per call
+    kernel_s = ms * 1e-3  # one call: the prep and scan launches back to back on one stream
     achieved_gbs = nbytes / kernel_s / 1e9
     tflops = flops / kernel_s / 1e12
+    traffic = measured_traffic() if w.name == PREFILL else None
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / pk["hbm_gbs"], "traffic": None,
+                "frac": achieved_gbs / pk["hbm_gbs"], "traffic": traffic,
                 "peak_source": pk["source"],
-                "kernel": "gdn2 chunk_fwd", "alg_bytes_per_launch": nbytes, "alg_flops_per_launch": flops,
-                "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"]}
+                "kernel": "gdn2_chunk_fwd call (chunk_prep_kernel + chunk_scan_kernel)",
+                "launches_per_call": launches_per_call, "alg_bytes_per_launch": nbytes,
+                "alg_flops_per_launch": flops, "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"]}
 
     # ---------------------------------------------------------------- decode
-    dw = workload(DECODE)
+    decode = None
+    dw = workload(args.decode_workload) if args.decode_steps > 0 else None
+    if dw is not None:
+        decode = run_decode(args, dw, dev, stream, barrier, pk, world)
+
+    # ---------------------------------------------------------------- end to end
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step)
+
+    # ---------------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        heads, tokens = w.H_v, 8192
+        rate, dt, used = cpu_oracle_rate(w, heads, tokens)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
+               "sample": f"{heads} V heads x {tokens} tokens of the T={w.T} layer workload "
+                         f"({dt:.1f} s, layer tokens = tokens x heads/{w.H_v})"}
+
+    clocks = clk.summary()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(args, dw, dev, stream, barrier, pk, world):
+    import torch
+    from delta_rule_linear_gdn_b200 import gdn2
+    from delta_rule_linear_gdn_b200.inputs import make_decode_pool
     pool = make_decode_pool(dw, pool=16, device=dev)
     S = pool["S0"].clone()
     od = torch.empty((dw.B, dw.H_v, dw.d), dtype=torch.bfloat16, device=dev)
@@ -340,8 +413,16 @@ def main():
                            "unit": "GB/s", "frac": dbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"],
                            "traffic": None, "alg_bytes_per_launch": dbytes},
               "tokens_per_s": dw.B * world / (dms * 1e-3)}
+    decode["gpu_launches"] = args.decode_steps
+    return decode
 
-    # ---------------------------------------------------------------- end to end
+
+def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):
+    """The same prefill through the public call with host buffers: pinned
+    host->device copies of the inputs, the call, device->host copies of o and
+    S_T, all on the timed stream."""
+    import torch
+    from delta_rule_linear_gdn_b200 import gdn2
     host = {k: inp[k].cpu().pin_memory() for k in ("q", "k", "v", "alpha", "b", "w")}
     dev_in = {k: torch.empty_like(inp[k]) for k in host}
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -370,31 +451,8 @@ def main():
     torch.cuda.synchronize()
     barrier()
     ems = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
-    e2e = {"value": tokens_per_step / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": ems}
-
-    # ---------------------------------------------------------------- CPU baseline
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        heads, tokens = w.H_v, 8192
-        rate, dt, used = cpu_oracle_rate(w, heads, tokens)
-        cpu = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
-               "sample": f"{heads} V heads x {tokens} tokens of the T=32768 layer workload "
-                         f"({dt:.1f} s, layer tokens = tokens x heads/48)"}
-
-    clocks = clk.summary()
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
-        }
-        print(json.dumps(line), flush=True)
-    return 0
+    return {"value": tokens_per_step / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
 
 if __name__ == "__main__":

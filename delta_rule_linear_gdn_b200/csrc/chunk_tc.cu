@@ -56,6 +56,7 @@
 // otherwise, chosen per chunk. The fp16 operands require |S| and |v| < 6e4.
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "tc_prims.cuh"
@@ -67,7 +68,6 @@ using namespace tc;
 
 constexpr int D = 128;            // d_k = d_v
 constexpr int C = 64;             // chunk
-constexpr int NT = 256;           // threads per CTA (8 warps)
 
 // ------------------------------------------------------------------ workspace
 // Word 0 of the workspace is the device status (nonzero: a wait gave up).
@@ -93,22 +93,18 @@ constexpr int BS_ROW64 = 8192;        // block stride of a 64-row tile
 // [32K, 64K) Gm: [Ē_mid ; Q̄_mid], 128 rows, BS 16K
 // [64K, 80K) Km: K̃_mid, 64 rows, BS 8K
 // [80K, 96K) Ē (64 tok × 128 key, BS 8K)   [96K, 112K) Z (64 tok × 128 dv)
-// Before pass 2, [32K, 66K) stages α for the cumulative products; after the
-// Gram MMAs, [32K, 71K) holds the fp32 arrays of the inverse and [0, 8K) the
-// fp16 A = (I+T)⁻¹ (64 × 64).
+// After the Gram MMAs, [32K, 71K) holds the fp32 arrays of the inverse and
+// [0, 8K) the fp16 A = (I+T)⁻¹ (64 × 64). Two CTAs of this layout fit one SM.
 constexpr int P_GB = 0;
 constexpr int P_KB = 0;
 constexpr int P_PQ = 8192;            // quarter products [4][128] fp32
 constexpr int P_RED = P_PQ + 4 * D * 4;
-static_assert(P_RED + 64 <= 12288, "quarter products must stay in the unused Gram rows");
+static_assert(P_RED + 32 <= 12288, "quarter products must stay in the unused Gram rows");
 constexpr int P_GM = 32768;
 constexpr int P_KM = 65536;
 constexpr int P_EB = 81920;
 constexpr int P_Z = 98304;
 constexpr int P_END = 114688;
-constexpr int SS = 132;               // α staging row stride (floats)
-constexpr int P_STG = P_GM;
-static_assert(P_STG + C * SS * 4 <= P_EB, "staging overlap");
 constexpr int P_AINV = 0;
 constexpr int TS = 68;                // fp32 row stride of T and its inverse
 constexpr int P_T = P_GM;             // T   [64][68]
@@ -128,8 +124,8 @@ constexpr int S_STAGE1 = SLOT;
 constexpr int S_ST = 2 * SLOT;        // Sᵀ fp16 [128 dv][128 key], BS 16K
 constexpr int S_UT = S_ST + D * D * 2;// Uᵀ fp16 [128 dv][64 tok]
 constexpr int S_OS = S_UT + D * C * 2;// output staging, 16 KB of [rows][128] TOut
-constexpr int S_BAR = S_OS + 16384;   // full[2], ys, st, o
-constexpr int S_TMEMP = S_BAR + 48;
+constexpr int S_BAR = S_OS + 16384;   // 13 mbarriers (see the scan kernel)
+constexpr int S_TMEMP = S_BAR + 128;
 constexpr int S_FLAG = S_TMEMP + 16;
 constexpr int S_SMEM = S_FLAG + 16;
 constexpr uint32_t ST_S = 0, ST_YS = 128, ST_O = 192, ST_COLS = 512;   // Oᵀ double-buffered: 192, 256
@@ -156,36 +152,6 @@ __device__ __forceinline__ void unpack8_f16(uint4 u, float* x) {
   }
 }
 
-// Key-side inputs of one token for 4 channels (coalesced: a warp reads whole
-// rows), and the pointers and sizes needed to load them, passed by value.
-struct KeyIn {
-  uint2 k, q;              // bf16 × 4
-  float4 b;                // fp32 × 4 (tied gates: β broadcast)
-};
-struct RowSrc {
-  const __nv_bfloat16 *k, *q;
-  const float* b;
-  int T, Hqk, Hv, full_gates;
-};
-
-__device__ __forceinline__ void load_key_row(RowSrc r_, int bi, int t, int h, int hq, int c4, bool valid, KeyIn& r) {
-  if (valid) {
-    const size_t tq = ((size_t)bi * r_.T + t) * r_.Hqk + hq;
-    const size_t gt = ((size_t)bi * r_.T + t) * r_.Hv + h;
-    r.k = __ldg(reinterpret_cast<const uint2*>(r_.k + tq * D + c4));
-    r.q = __ldg(reinterpret_cast<const uint2*>(r_.q + tq * D + c4));
-    if (r_.full_gates) {
-      r.b = __ldg(reinterpret_cast<const float4*>(r_.b + gt * D + c4));
-    } else {
-      const float beta = __ldg(r_.b + gt);
-      r.b = make_float4(beta, beta, beta, beta);
-    }
-  } else {
-    r.k = r.q = make_uint2(0, 0);
-    r.b = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
 __device__ __forceinline__ void wait_mma(uint64_t* bar, uint32_t& phase, int* sflag) {
   if (!mbar_wait(bar, phase)) atomicOr(sflag, 1);
   phase ^= 1u;
@@ -200,51 +166,23 @@ __device__ __forceinline__ void sync_for_mma() {
 }
 
 // =============================================================================
-// prep kernel: persistent, one 512-thread CTA per SM looping over the work
-// items (chunk of the segment, sequence, value head). Each item's inputs are
-// loaded in one round into registers; the next item's loads are issued as
-// soon as the current item's elementwise pass has consumed its registers, so
-// they arrive while the Gram, inverse and Yᵀ/U_wᵀ phases run.
+// prep kernel: persistent, two 256-thread CTAs per SM, each looping over the
+// work items (chunk of the segment, sequence, value head). While one CTA waits
+// for its tensor-core products or runs the serial steps of the inverse, the
+// other CTA on the SM runs its elementwise passes.
 // =============================================================================
-constexpr int NP = 512;               // prep threads (16 warps)
+constexpr int NP = 256;               // prep threads (8 warps)
 
-// Inputs of one token for 4 channels (a warp reads whole rows).
-struct TokIn {
-  float4 al, b, w;
-  uint2 k, q, v;
-};
 struct PrepSrc {
   const float *alpha, *b, *w;
   const __nv_bfloat16 *k, *q, *v;
-  int T, Hqk, Hv, mode;
 };
 
-__device__ __forceinline__ void load_token(const PrepSrc& p, int bi, int t, int h, int hq, int c4, bool valid,
-                                           TokIn& r) {
-  if (valid) {
-    const size_t gt = ((size_t)bi * p.T + t) * p.Hv + h;
-    const size_t tq = ((size_t)bi * p.T + t) * p.Hqk + hq;
-    if (p.mode == GDN2_GATES_GDN) {
-      const float sa = __ldg(p.alpha + gt);
-      r.al = make_float4(sa, sa, sa, sa);
-    } else {
-      r.al = __ldg(reinterpret_cast<const float4*>(p.alpha + gt * D + c4));
-    }
-    if (p.mode == GDN2_GATES_FULL) {
-      r.b = __ldg(reinterpret_cast<const float4*>(p.b + gt * D + c4));
-      r.w = __ldg(reinterpret_cast<const float4*>(p.w + gt * D + c4));
-    } else {
-      const float beta = __ldg(p.b + gt);
-      r.b = r.w = make_float4(beta, beta, beta, beta);
-    }
-    r.k = __ldg(reinterpret_cast<const uint2*>(p.k + tq * D + c4));
-    r.q = __ldg(reinterpret_cast<const uint2*>(p.q + tq * D + c4));
-    r.v = __ldg(reinterpret_cast<const uint2*>(p.v + gt * D + c4));
-  } else {
-    r.al = make_float4(1.f, 1.f, 1.f, 1.f);
-    r.b = r.w = make_float4(0.f, 0.f, 0.f, 0.f);
-    r.k = r.q = r.v = make_uint2(0, 0);
-  }
+// fp32 gate of one token for 4 channels, or the token's scalar gate broadcast.
+__device__ __forceinline__ float4 gate4(const float* g, size_t gt, int c0, bool per_channel) {
+  if (per_channel) return __ldg(reinterpret_cast<const float4*>(g + gt * D + c0));
+  const float s = __ldg(g + gt);
+  return make_float4(s, s, s, s);
 }
 
 struct Item {
@@ -262,14 +200,13 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int
   return it;
 }
 
-__global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg) {
+__global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + P_BAR);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + P_TMEMP);
   int* sflag = reinterpret_cast<int*>(smem + P_FLAG);
   float* sPq = reinterpret_cast<float*>(smem + P_PQ);
   float* sred = reinterpret_cast<float*>(smem + P_RED);
-  float* stage = reinterpret_cast<float*>(smem + P_STG);
   float* sT = reinterpret_cast<float*>(smem + P_T);
   float* sI = reinterpret_cast<float*>(smem + P_I);
   float* sX = reinterpret_cast<float*>(smem + P_X);
@@ -292,57 +229,108 @@ __global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_be
   const int lq = warp & 3;                       // TMEM lane quarter of this warp
   const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
   const int row = lq * 32 + lane;
-  const int cgp = warp >> 2;                     // column group (0..3) among warps of a lane quarter
+  const int hc = warp >> 2;                      // which of the two warps of a lane quarter
 
-  // Element mapping: lane → 4 channels c4..c4+3 (a warp covers a whole row),
-  // warp w → token w + 16 j of quarter j (j = 0..3).
-  const int c4 = lane * 4;
-  // Swizzled offsets of this thread's 4-channel piece: every token it handles
-  // has row ≡ warp (mod 8), so only a multiple of 128 bytes depends on the row.
-  const uint32_t col64 = sw_off(warp & 7, c4, BS_ROW64) - (uint32_t)((warp & 7) * 128);
-  const uint32_t col128 = sw_off(warp & 7, c4, BS_ROW128) - (uint32_t)((warp & 7) * 128);
-  const PrepSrc src{a.alpha, a.b, a.w, static_cast<const __nv_bfloat16*>(a.k),
-                    static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.v),
-                    a.T, a.Hqk, a.Hv, a.gate_mode};
-  TokIn in[4];
-  int item = blockIdx.x;
-  if (item < n_items) {
-    const Item it = decode_item(a, c_begin, item);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int i = warp + 16 * j;
-      load_token(src, it.bi, it.t0 + i, it.h, it.hq, c4, i < it.Lc, in[j]);
-    }
-  }
+  // Element mapping of the elementwise passes: warp w takes quarter qt = w/2
+  // (tokens 16 qt .. 16 qt + 15) and channel half w%2; a lane takes 4 channels
+  // c0..c0+3 of the 8 tokens i0 + u (u = 0..7). Each memory access of a warp
+  // covers whole rows of 64 channels.
+  const int qt = warp >> 1, cg = lane & 15, tg = lane >> 4;
+  const int c0 = (warp & 1) * 64 + cg * 4;
+  const int i0 = 16 * qt + 8 * tg;
+  // Offset of this thread's 8-byte piece in row i0 + u of a swizzled tile,
+  // less the row's i·128 ((i0 + u) mod 8 = u); `blk` is the tile's block stride.
+  auto piece = [&](int u, int blk) -> uint32_t {
+    return (uint32_t)((warp & 1) * blk + ((((cg >> 1) ^ u) << 4) | ((cg & 1) << 3)));
+  };
+  const bool full = a.gate_mode == GDN2_GATES_FULL;
+  const bool alpha_pc = a.gate_mode != GDN2_GATES_GDN;
+  const PrepSrc src{a.alpha, a.b, full ? a.w : a.b, static_cast<const __nv_bfloat16*>(a.k),
+                    static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.v)};
+
   uint32_t phase = 0;
-  for (; item < n_items; item += gridDim.x) {
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const Item it = decode_item(a, c_begin, item);
     uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)it.bh * n_seg + it.cl) * SLOT;
+    const size_t tok0 = (size_t)it.bi * a.T + it.t0 + i0;    // token of u = 0
 
-    // -------- pass 1: α rows into the staging tile; the write side Z = w ⊙ v
-    // (which needs no decay) goes straight to its tile
+    // -------- pass 1: the write side Z = w ⊙ v (no decay) straight to its
+    // tile; α's forward products within the quarter. The key-side inputs of
+    // tokens u = 0..3 are requested here, those of u = 4..7 in pass 2.
+    float f[8][4];
+    float4 bq[4];
+    uint2 kk[4], qq[4];
+    const bool whole = it.Lc == C;              // every chunk but a sequence's last
+    auto load_key = [&](int u0) {
+      if (whole) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int i = warp + 16 * j;
-      *reinterpret_cast<float4*>(stage + i * SS + c4) = in[j].al;
-      float vx[4];
-      unpack4_bf16(in[j].v, vx);
-      st8(smem, P_Z + col64 + i * 128,
-          pack4_f16(in[j].w.x * vx[0], in[j].w.y * vx[1], in[j].w.z * vx[2], in[j].w.w * vx[3]));
-    }
-    __syncthreads();
-    // forward cumulative products down each channel within each quarter
-    {
-      const int c = tid & 127, q = tid >> 7;
-      float acc = 1.f;
+        for (int u = 0; u < 4; ++u) {
+          const size_t gt = (tok0 + u0 + u) * a.Hv + it.h;
+          const size_t tq = (tok0 + u0 + u) * a.Hqk + it.hq;
+          bq[u] = gate4(src.b, gt, c0, full);
+          kk[u] = __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0));
+          qq[u] = __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0));
+        }
+      } else {
 #pragma unroll
-      for (int s_ = 0; s_ < 16; ++s_) {
-        float* pp = stage + (16 * q + s_) * SS + c;
-        acc *= *pp;
-        *pp = acc;
+        for (int u = 0; u < 4; ++u) {
+          const bool ok = i0 + u0 + u < it.Lc;
+          const size_t gt = (tok0 + u0 + u) * a.Hv + it.h;
+          const size_t tq = (tok0 + u0 + u) * a.Hqk + it.hq;
+          bq[u] = ok ? gate4(src.b, gt, c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+          kk[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
+          qq[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
+        }
       }
-      sPq[q * D + c] = acc;
-      float mn = acc;
+    };
+    {
+      float4 wv[8];
+      uint2 vv[8];
+      if (whole) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const size_t gt = (tok0 + u) * a.Hv + it.h;
+          const float4 al = gate4(src.alpha, gt, c0, alpha_pc);
+          f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
+          wv[u] = gate4(src.w, gt, c0, full);
+          vv[u] = __ldg(reinterpret_cast<const uint2*>(src.v + gt * D + c0));
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const bool ok = i0 + u < it.Lc;
+          const size_t gt = (tok0 + u) * a.Hv + it.h;
+          const float4 al = ok ? gate4(src.alpha, gt, c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
+          f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
+          wv[u] = ok ? gate4(src.w, gt, c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+          vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + gt * D + c0)) : make_uint2(0, 0);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float vx[4];
+        unpack4_bf16(vv[u], vx);
+        st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
+            pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
+      }
+    }
+    load_key(0);
+    {
+      // within the thread's 8 tokens, then across the two token groups of the
+      // quarter (lanes l and l + 16)
+      float pq[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int u = 1; u < 8; ++u) f[u][c] *= f[u - 1][c];
+        const float y = __shfl_up_sync(0xffffffffu, f[7][c], 16);
+        const float ex = tg ? y : 1.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u][c] *= ex;
+        pq[c] = __shfl_sync(0xffffffffu, f[7][c], cg + 16);    // product over the quarter
+      }
+      if (tg == 0) *reinterpret_cast<float4*>(sPq + qt * D + c0) = make_float4(pq[0], pq[1], pq[2], pq[3]);
+      float mn = fminf(fminf(pq[0], pq[1]), fminf(pq[2], pq[3]));
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
       if (lane == 0) sred[warp] = mn;
@@ -360,87 +348,85 @@ __global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_be
       const float g = sPq[tid] * sPq[D + tid] * sPq[2 * D + tid] * sPq[3 * D + tid];
       reinterpret_cast<float*>(slot + SL_GC)[tid] = g;
     }
-    float fw[4][4], Pq[4][4];
+    // Per-channel factors of quarter qt from the quarter products P_m:
+    //   γ_i = pre · f_i,                      pre = Π_{m<qt} P_m
+    //   Π_{i<s≤63} α = (P_qt · suf) / f_i,      suf = Π_{m>qt} P_m
+    //   mid-reference factors: f_i / P_qt and P_qt / f_i (first quarter of a
+    //   half), f_i and 1 / f_i (second quarter);
+    //   half-boundary factors: P_2 f_i (quarter 3), f_i (quarter 2) for rows
+    //   of the second half; P_qt P_1 / f_i (quarter 0), P_qt / f_i (quarter 1)
+    //   for keys of the first half.
+    float pre[4], ps[4], se[4], sk[4], sx[4];
+    {
+      float P[4][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 v = *reinterpret_cast<const float4*>(stage + (warp + 16 * j) * SS + c4);
-      fw[j][0] = v.x; fw[j][1] = v.y; fw[j][2] = v.z; fw[j][3] = v.w;
-      const float4 pq = *reinterpret_cast<const float4*>(sPq + j * D + c4);
-      Pq[j][0] = pq.x; Pq[j][1] = pq.y; Pq[j][2] = pq.z; Pq[j][3] = pq.w;
-    }
-    __syncthreads();   // the staging tile is free from here on
-
-    // -------- pass 2: key-side operand tiles (token i = warp + 16 m is in quarter m)
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int i = warp + 16 * m;
-      float kx[4], qx[4], ex[4];
-      unpack4_bf16(in[m].k, kx);
-      unpack4_bf16(in[m].q, qx);
-      ex[0] = in[m].b.x * kx[0]; ex[1] = in[m].b.y * kx[1]; ex[2] = in[m].b.z * kx[2]; ex[3] = in[m].b.w * kx[3];
-      float o_eb[4], o_qb[4], o_ke[4], o_em[4], o_qm[4], o_km[4], o_x1[4], o_x2[4];
+      for (int m = 0; m < 4; ++m) {
+        const float4 v = *reinterpret_cast<const float4*>(sPq + m * D + c0);
+        P[m][0] = v.x; P[m][1] = v.y; P[m][2] = v.z; P[m][3] = v.w;
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float P = Pq[m][c];
-        float pre = 1.f, suf = 1.f;
+        float pr = 1.f, su = 1.f, own = P[0][c];
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-          if (mm < m) pre *= Pq[mm][c];
-          if (mm > m) suf *= Pq[mm][c];
+        for (int m = 0; m < 4; ++m) {
+          if (m < qt) pr *= P[m][c];
+          if (m > qt) su *= P[m][c];
+          if (m == qt) own = P[m][c];
         }
-        const float f = fw[m][c];               // Π_{quarter start ≤ s ≤ i} α
-        const float rf = __fdividef(1.f, f);
-        const float bw = P * rf;                // Π_{i < s ≤ quarter end} α
-        const float g = pre * f;                // γ_i
-        const float bk = bw * suf;              // Π_{i < s ≤ 63} α
-        o_eb[c] = ex[c] * g;
-        o_qb[c] = qx[c] * g;
-        o_ke[c] = kx[c] * bk;
-        float fe, fk;
-        if ((m & 1) == 0) {
-          fe = f * __fdividef(1.f, P);          // 1 / bw
-          fk = bw;
-        } else {
-          fe = f;
-          fk = rf;
-        }
-        o_em[c] = ex[c] * fe;
-        o_qm[c] = qx[c] * fe;
-        o_km[c] = kx[c] * fk;
-        if (m >= 2) {
-          const float fq = (m == 3 ? Pq[2][c] : 1.f) * f;
-          o_x1[c] = ex[c] * fq;
-          o_x2[c] = qx[c] * fq;
-        } else {
-          const float fb = bw * (m == 0 ? Pq[1][c] : 1.f);
-          o_x1[c] = kx[c] * fb;
-          o_x2[c] = 0.f;
-        }
-      }
-      st8(slot, SL_QB + col64 + i * 128, pack4(o_qb, false));
-      st8(slot, SL_KE + col64 + i * 128, pack4(o_ke, false));
-      st8(smem, P_EB + col64 + i * 128, pack4(o_eb, false));
-      st8(smem, P_GM + col128 + i * 128, pack4(o_em, gram_bf16));
-      st8(smem, P_GM + col128 + (64 + i) * 128, pack4(o_qm, gram_bf16));
-      st8(smem, P_KM + col64 + i * 128, pack4(o_km, gram_bf16));
-      if (m >= 2) {
-        st8(smem, P_GB + col128 + i * 128, pack4(o_x1, gram_bf16));
-        st8(smem, P_GB + col128 + (64 + i) * 128, pack4(o_x2, gram_bf16));
-      } else {
-        st8(smem, P_KB + col128 + i * 128, pack4(o_x1, gram_bf16));
+        pre[c] = pr;
+        ps[c] = own * su;
+        const bool even = (qt & 1) == 0;
+        se[c] = even ? rcp_approx(own) : 1.f;
+        sk[c] = even ? own : 1.f;
+        sx[c] = qt == 3 ? P[2][c] : (qt == 2 ? 1.f : (qt == 0 ? own * P[1][c] : own));
       }
     }
-    // the next item's inputs: issued now, consumed at the top of the next pass
-    {
-      const int nxt = item + (int)gridDim.x;
-      if (nxt < n_items) {
-        const Item in_ = decode_item(a, c_begin, nxt);
+
+    // -------- pass 2: key-side operand tiles, tile by tile per token
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = warp + 16 * j;
-          load_token(src, in_.bi, in_.t0 + i, in_.h, in_.hq, c4, i < in_.Lc, in[j]);
-        }
+    for (int u = 0; u < 8; ++u) {
+      if (u == 4) load_key(4);
+      const int uk = u & 3;
+      const uint32_t i128 = (uint32_t)(i0 + u) * 128;
+      const uint32_t p64 = i128 + piece(u, BS_ROW64), p128 = i128 + piece(u, BS_ROW128);
+      float kx[4], qx[4], e[4], rf[4], g[4], fe[4];
+      unpack4_bf16(kk[uk], kx);
+      unpack4_bf16(qq[uk], qx);
+      e[0] = bq[uk].x * kx[0]; e[1] = bq[uk].y * kx[1]; e[2] = bq[uk].z * kx[2]; e[3] = bq[uk].w * kx[3];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        rf[c] = rcp_approx(f[u][c]);
+        g[c] = pre[c] * f[u][c];
+        fe[c] = se[c] * f[u][c];
       }
+      float o[4];
+#define GDN2_TILE(dst, off, expr)                                             \
+  {                                                                           \
+    _Pragma("unroll") for (int c = 0; c < 4; ++c) o[c] = (expr);              \
+    st8(dst, off, pack4_f16(o[0], o[1], o[2], o[3]));                         \
+  }
+#define GDN2_GRAM_TILE(dst, off, expr)                                        \
+  {                                                                           \
+    _Pragma("unroll") for (int c = 0; c < 4; ++c) o[c] = (expr);              \
+    if (gram_bf16)                                                            \
+      st8(dst, off, pack4_bf16(o[0], o[1], o[2], o[3]));                      \
+    else                                                                      \
+      st8(dst, off, pack4_f16(o[0], o[1], o[2], o[3]));                       \
+  }
+      GDN2_TILE(slot, SL_QB + p64, qx[c] * g[c])
+      GDN2_TILE(slot, SL_KE + p64, kx[c] * (ps[c] * rf[c]))
+      GDN2_TILE(smem, P_EB + p64, e[c] * g[c])
+      GDN2_GRAM_TILE(smem, P_GM + p128, e[c] * fe[c])
+      GDN2_GRAM_TILE(smem, P_GM + 64 * 128 + p128, qx[c] * fe[c])
+      GDN2_GRAM_TILE(smem, P_KM + p64, kx[c] * (sk[c] * rf[c]))
+      if (qt >= 2) {
+        GDN2_GRAM_TILE(smem, P_GB + p128, e[c] * (sx[c] * f[u][c]))
+        GDN2_GRAM_TILE(smem, P_GB + 64 * 128 + p128, qx[c] * (sx[c] * f[u][c]))
+      } else {
+        GDN2_GRAM_TILE(smem, P_KB + p128, kx[c] * (sx[c] * rf[c]))
+      }
+#undef GDN2_TILE
+#undef GDN2_GRAM_TILE
     }
     sync_for_mma();
 
@@ -464,32 +450,36 @@ __global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_be
     wait_mma(bar, phase, sflag);
 
     // -------- T (fp32, shared) and Aqk (fp16, workspace) from TMEM. Lanes
-    // 0..63 hold rows of T, lanes 64..127 rows of Aqk; the four warps of a
-    // lane quarter take 16 columns each.
+    // 0..63 hold rows of T, lanes 64..127 rows of Aqk; the two warps of a lane
+    // quarter take 32 columns each (only columns < 32 need the half-boundary
+    // product: a row i ≥ 32 against a key j < 32).
     {
       const bool is_t = row < 64;
       const int i = row & 63;
-      const int j0 = 16 * cgp;
-      float dm[16], db[16];
+      const int j0 = 32 * hc;
+      float dm[32], db[32];
       tmem_ld16(t_lane + PT_GM + j0, dm);
-      tmem_ld16(t_lane + PT_GB + (j0 & 31), db);
+      tmem_ld16(t_lane + PT_GM + j0 + 16, dm + 16);
+      if (hc == 0) {
+        tmem_ld16(t_lane + PT_GB, db);
+        tmem_ld16(t_lane + PT_GB + 16, db + 16);
+      }
       tmem_wait_ld();
-      float v[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
+      for (int u = 0; u < 32; ++u) {
         const int j = j0 + u;
         const bool keep = is_t ? (j < i) : (j <= i);
         const bool same = (j >> 5) == (i >> 5);
-        const float x = same ? dm[u] : (j0 < 32 ? db[u] : 0.f);
-        v[u] = keep ? x : 0.f;
+        const float x = same ? dm[u] : (hc == 0 ? db[u] : 0.f);
+        dm[u] = keep ? x : 0.f;
       }
       if (is_t) {
 #pragma unroll
-        for (int u = 0; u < 16; u += 4)
-          *reinterpret_cast<float4*>(sT + i * TS + j0 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+        for (int u = 0; u < 32; u += 4)
+          *reinterpret_cast<float4*>(sT + i * TS + j0 + u) = make_float4(dm[u], dm[u + 1], dm[u + 2], dm[u + 3]);
       } else {
-        st16(slot, SL_AQ + sw_off(i, j0, BS_ROW64), pack8_f16(v));
-        st16(slot, SL_AQ + sw_off(i, j0 + 8, BS_ROW64), pack8_f16(v + 8));
+#pragma unroll
+        for (int cb = 0; cb < 32; cb += 8) st16(slot, SL_AQ + sw_off(i, j0 + cb, BS_ROW64), pack8_f16(dm + cb));
       }
     }
     __syncthreads();
@@ -518,60 +508,73 @@ __global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_be
       }
     }
     __syncthreads();
-    // level 1: X21 = −I22 T21 I11 in each 32-half (one entry per thread)
+    // level 1: X21 = −I22 T21 I11 in each 32-half (two entries per thread)
     {
-      const int hf = tid >> 8, ii = (tid >> 4) & 15, jj = tid & 15;
-      const int r0 = hf * 32 + 16, c0 = hf * 32;
-      float acc = 0.f;
-#pragma unroll
-      for (int l = 0; l < 16; ++l) acc += sT[(r0 + ii) * TS + c0 + l] * sI[(c0 + l) * TS + c0 + jj];
-      sX[(hf * 16 + ii) * 36 + jj] = acc;
-    }
-    __syncthreads();
-    {
-      const int hf = tid >> 8, ii = (tid >> 4) & 15, jj = tid & 15;
-      const int r0 = hf * 32 + 16, c0 = hf * 32;
-      float acc = 0.f;
-#pragma unroll
-      for (int l = 0; l < 16; ++l) acc += sI[(r0 + ii) * TS + r0 + l] * sX[(hf * 16 + l) * 36 + jj];
-      sI[(r0 + ii) * TS + c0 + jj] = -acc;
-    }
-    __syncthreads();
-    // level 2: X_QP = −I_QQ T_QP I_PP (thread: row ii, 2 columns)
-    {
-      const int ii = tid >> 4, jp = (tid & 15) * 2;
+      const int hf = tid >> 7, ii = (tid >> 3) & 15, jj = (tid & 7) * 2;
+      const int r0 = hf * 32 + 16, cc = hf * 32;
       float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int l = 0; l < 16; ++l) {
+        const float t = sT[(r0 + ii) * TS + cc + l];
+        const float2 iv = *reinterpret_cast<const float2*>(sI + (cc + l) * TS + cc + jj);
+        a0 += t * iv.x;
+        a1 += t * iv.y;
+      }
+      *reinterpret_cast<float2*>(sX + (hf * 16 + ii) * 36 + jj) = make_float2(a0, a1);
+    }
+    __syncthreads();
+    {
+      const int hf = tid >> 7, ii = (tid >> 3) & 15, jj = (tid & 7) * 2;
+      const int r0 = hf * 32 + 16, cc = hf * 32;
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int l = 0; l < 16; ++l) {
+        const float t = sI[(r0 + ii) * TS + r0 + l];
+        const float2 xv = *reinterpret_cast<const float2*>(sX + (hf * 16 + l) * 36 + jj);
+        a0 += t * xv.x;
+        a1 += t * xv.y;
+      }
+      *reinterpret_cast<float2*>(sI + (r0 + ii) * TS + cc + jj) = make_float2(-a0, -a1);
+    }
+    __syncthreads();
+    // level 2: X_QP = −I_QQ T_QP I_PP (thread: row ii, 4 columns)
+    {
+      const int ii = tid >> 3, jp = (tid & 7) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
       for (int l = 0; l < 32; ++l) {
         const float t = sT[(32 + ii) * TS + l];
-        const float2 iv = *reinterpret_cast<const float2*>(sI + l * TS + jp);
-        a0 += t * iv.x; a1 += t * iv.y;
+        const float4 iv = *reinterpret_cast<const float4*>(sI + l * TS + jp);
+        acc.x += t * iv.x; acc.y += t * iv.y; acc.z += t * iv.z; acc.w += t * iv.w;
       }
-      *reinterpret_cast<float2*>(sX + ii * 36 + jp) = make_float2(a0, a1);
+      *reinterpret_cast<float4*>(sX + ii * 36 + jp) = acc;
     }
     __syncthreads();
     {
-      const int ii = tid >> 4, jp = (tid & 15) * 2;
-      float a0 = 0.f, a1 = 0.f;
+      const int ii = tid >> 3, jp = (tid & 7) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
       for (int l = 0; l < 32; ++l) {
         const float t = sI[(32 + ii) * TS + 32 + l];
-        const float2 xv = *reinterpret_cast<const float2*>(sX + l * 36 + jp);
-        a0 += t * xv.x; a1 += t * xv.y;
+        const float4 xv = *reinterpret_cast<const float4*>(sX + l * 36 + jp);
+        acc.x += t * xv.x; acc.y += t * xv.y; acc.z += t * xv.z; acc.w += t * xv.w;
       }
-      *reinterpret_cast<float2*>(sI + (32 + ii) * TS + jp) = make_float2(-a0, -a1);
+      *reinterpret_cast<float4*>(sI + (32 + ii) * TS + jp) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
     }
     __syncthreads();
-    // pack A (lower triangle; zeros above the diagonal), one 8-wide piece per thread
+    // pack A (lower triangle; zeros above the diagonal), 16 entries per thread
     {
-      const int i = tid >> 3, j0 = (tid & 7) * 8;
-      float x[8];
-      const float4 p0 = *reinterpret_cast<const float4*>(sI + i * TS + j0);
-      const float4 p1 = *reinterpret_cast<const float4*>(sI + i * TS + j0 + 4);
-      x[0] = p0.x; x[1] = p0.y; x[2] = p0.z; x[3] = p0.w; x[4] = p1.x; x[5] = p1.y; x[6] = p1.z; x[7] = p1.w;
+      const int i = tid >> 2, j0 = (tid & 3) * 16;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = (j0 + u <= i) ? x[u] : 0.f;
-      st16(smem, P_AINV + sw_off(i, j0, BS_ROW64), pack8_f16(x));
+      for (int h8 = 0; h8 < 16; h8 += 8) {
+        float x[8];
+        const float4 p0 = *reinterpret_cast<const float4*>(sI + i * TS + j0 + h8);
+        const float4 p1 = *reinterpret_cast<const float4*>(sI + i * TS + j0 + h8 + 4);
+        x[0] = p0.x; x[1] = p0.y; x[2] = p0.z; x[3] = p0.w; x[4] = p1.x; x[5] = p1.y; x[6] = p1.z; x[7] = p1.w;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = (j0 + h8 + u <= i) ? x[u] : 0.f;
+        st16(smem, P_AINV + sw_off(i, j0 + h8, BS_ROW64), pack8_f16(x));
+      }
     }
     sync_for_mma();
 
@@ -593,16 +596,18 @@ __global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_be
     __syncwarp();
     wait_mma(bar, phase, sflag);
     {
-      // column groups 0, 1: Yᵀ rows (key lanes); 2, 3: U_wᵀ rows (dv lanes)
-      const uint32_t col = (cgp < 2 ? PT_YT : PT_UW) + 32u * (uint32_t)(cgp & 1);
-      const int dst = cgp < 2 ? SL_YT : SL_UW;
-      const int cb0 = 32 * (cgp & 1);
-      float v[32];
-      tmem_ld16(t_lane + col, v);
-      tmem_ld16(t_lane + col + 16, v + 16);
-      tmem_wait_ld();
+      // warps 0..3: Yᵀ rows (key lanes); warps 4..7: U_wᵀ rows (dv lanes)
+      const uint32_t col = hc == 0 ? PT_YT : PT_UW;
+      const int dst = hc == 0 ? SL_YT : SL_UW;
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) st16(slot, dst + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
+      for (int cb0 = 0; cb0 < 64; cb0 += 32) {
+        float v[32];
+        tmem_ld16(t_lane + col + cb0, v);
+        tmem_ld16(t_lane + col + cb0 + 16, v + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int cb = 0; cb < 32; cb += 8) st16(slot, dst + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
+      }
     }
     fence_before_sync();
     __syncthreads();
@@ -615,18 +620,43 @@ __global__ void __launch_bounds__(NP, 1) chunk_prep_kernel(ChunkArgs a, int c_be
 }
 
 // =============================================================================
-// scan kernel: one CTA per (sequence, value head), chunks of the segment in order
+// scan kernel: one CTA per (sequence, value head), chunks of the segment in
+// order. Warp 12 issues the tensor-core products and the slot copies (one
+// thread); warps 0..7 run the state chain, warps 8..11 write the outputs.
+// They hand over through mbarriers:
+//   MMA thread, chunk c:  (Y S)ᵀ [after each half of the fp16 Sᵀ copy] → Oᵀ =
+//     Sᵀ Q̄ᵀ → [after Uᵀ] Sᵀ += Uᵀ K_end in two 64-key halves → Oᵀ += Uᵀ Aqkᵀ →
+//     [when chunk c's products are done] copy of chunk c + 2's slot;
+//   chain warps, chunk c:  Uᵀ = U_wᵀ − (Y S)ᵀ → per key half: fp16 Sᵀ copy for
+//     chunk c + 1 and Sᵀ ← Sᵀ Γ_{c+1} in TMEM;
+//   output warps, chunk c:  Oᵀ (double-buffered in TMEM) → o.
 // =============================================================================
+constexpr int NS = 416;               // scan threads: 8 chain warps, 4 output warps, 1 MMA warp
+constexpr int NO = 128;               // output threads
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+__device__ __forceinline__ void out_sync() { asm volatile("bar.sync 2, 128;\n" ::: "memory"); }
+
 template <typename TOut>
-__global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, const float* S_in,
+__global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, const float* S_in,
                                                            float* S_out) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S_BAR);
-  uint64_t* bar_ys = full + 2;          // (Y S)ᵀ done
-  uint64_t* bar_st = full + 3;          // state update done
-  uint64_t* bar_o = full + 4;           // all MMAs of the chunk done
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_BAR);
+  uint64_t* full = bars;                // [2] slot copy landed in stage s
+  uint64_t* b_ys = bars + 2;            // (Y S)ᵀ done
+  uint64_t* b_sa = bars + 3;            // state update, keys 0..63, done
+  uint64_t* b_sb = bars + 4;            // state update, keys 64..127, done
+  uint64_t* b_o = bars + 5;             // every product of the chunk done
+  uint64_t* b_u = bars + 6;             // Uᵀ written
+  uint64_t* b_slo = bars + 7;           // fp16 Sᵀ keys 0..63 written (and TMEM scaled)
+  uint64_t* b_shi = bars + 8;           // keys 64..127
+  uint64_t* b_of = bars + 9;            // [2] Oᵀ buffer read out
+  uint64_t* b_ob = bars + 11;           // [2] Oᵀ buffer complete (one phase per use)
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + S_TMEMP);
   int* sflag = reinterpret_cast<int*>(smem + S_FLAG);
+  int* estop = sflag + 1;               // the chain warps' sample of the flag
+  int* ostop = sflag + 2;               // the output warps' sample
+  const volatile int* vflag = sflag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x;
@@ -635,13 +665,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   TOut* og = static_cast<TOut*>(a.o);
 
   if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    mbar_init(bar_ys, 1);
-    mbar_init(bar_st, 1);
-    mbar_init(bar_o, 1);
+    for (int i = 0; i < 13; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
-    *sflag = 0;
+    sflag[0] = 0;
+    sflag[1] = 0;
+    sflag[2] = 0;
   }
   if (warp == 0) {
     tmem_alloc(tmem_ptr, ST_COLS);
@@ -651,207 +679,267 @@ __global__ void __launch_bounds__(NT, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_ptr;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&full[0], SLOT_USED);
-    bulk_g2s(smem + S_STAGE0, slots, SLOT_USED, &full[0]);
-  }
 
-  const int lq = warp & 3;
-  const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
-  const int row = lq * 32 + lane;       // dv index j of Sᵀ[j][*]
-  const bool lo = warp < 4;
-
-  // Entry state: Sᵀ[j][c] = S[c][j]. The fp16 copy (operand of the first
-  // chunk's MMAs) is the state itself; TMEM holds it already multiplied by the
-  // first chunk's decay Γ, ready for the first update Sᵀ ← Sᵀ Γ + Uᵀ K_end.
-  if (!mbar_wait(&full[0], 0)) atomicOr(sflag, 1);
-  {
-    const float* gC = reinterpret_cast<const float*>(smem + S_STAGE0 + SL_GC);
-    const int c0 = lo ? 0 : 64;
-    const float* S0 = S_in ? S_in + (size_t)bh * D * D : nullptr;
-    for (int cb = c0; cb < c0 + 64; cb += 16) {
-      float v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = S0 ? __ldg(S0 + (size_t)(cb + u) * D + row) : 0.f;
-      st16(smem, S_ST + sw_off(row, cb, BS_ROW128), pack8_f16(v));
-      st16(smem, S_ST + sw_off(row, cb + 8, BS_ROW128), pack8_f16(v + 8));
-#pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] *= gC[cb + u];
-      tmem_st16(t_lane + ST_S + cb, v);
-    }
-    tmem_wait_st();
-  }
-  sync_for_mma();
-
-  // Output epilogue of a chunk: Oᵀ (TMEM buffer `ob`) → staging tile
-  // [rows][128] of TOut → contiguous 16-byte stores to o, O_ROWS tokens at a
-  // time. It runs while the next chunk's first MMAs execute.
-  constexpr int O_ROWS = 16384 / (D * (int)sizeof(TOut));   // 64 (bf16) or 32 (fp32)
-  auto out_epilogue = [&](uint32_t ob, int t0o, int Lco) {
-    TOut* so = reinterpret_cast<TOut*>(smem + S_OS);
-    const int c0 = lo ? 0 : 32;
-    float v[32];
-    tmem_ld16(t_lane + ob + c0, v);
-    tmem_ld16(t_lane + ob + c0 + 16, v + 16);
-    tmem_wait_ld();
-    constexpr int VEC = 16 / (int)sizeof(TOut);             // elements per 16 bytes
-    for (int r0 = 0; r0 < C; r0 += O_ROWS) {
-      if (r0 > 0) __syncthreads();
-      if (c0 >= r0 && c0 < r0 + O_ROWS) {
-#pragma unroll
-        for (int u = 0; u < 32; ++u) so[(c0 - r0 + u) * D + row] = from_f32<TOut>(a.scale * v[u]);
+  if (warp == 12) {
+    // ------------------------------------------------------------ MMA thread
+    if (lane == 0) {
+      int issued = 0, landed = 0;       // slot copies issued / seen complete
+      for (int c = 0; c < n_seg && c < 2; ++c) {
+        mbar_arrive_expect_tx(&full[c], SLOT_USED);
+        bulk_g2s(smem + (c ? S_STAGE1 : S_STAGE0), slots + (size_t)c * SLOT, SLOT_USED, &full[c]);
+        ++issued;
       }
-      __syncthreads();
-      const int nvec = O_ROWS * D / VEC;
-      for (int e = tid; e < nvec; e += NT) {
-        const int rr = e / (D / VEC), cc = (e % (D / VEC)) * VEC;
-        const int i = r0 + rr;
-        if (i < Lco)
-          *reinterpret_cast<uint4*>(og + (((size_t)bi * a.T + t0o + i) * a.Hv + h) * D + cc) =
-              *reinterpret_cast<const uint4*>(so + rr * D + cc);
-      }
-    }
-  };
-
-  uint32_t mphase = 0;
-  int issued = 1;                       // bulk copies issued (for the error path)
-  int waited = 1;
-  int prev_t0 = 0, prev_L = 0;          // chunk whose outputs are still in TMEM
-  for (int cl = 0; cl < n_seg; ++cl) {
-    const int s = cl & 1;
-    uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
-    uint8_t* nstg = smem + (s ? S_STAGE0 : S_STAGE1);
-    const int t0 = (c_begin + cl) * C;
-    const int Lc = min(C, a.T - t0);
-    const uint32_t ob = ST_O + 64u * (uint32_t)s;           // this chunk's Oᵀ buffer
-    // prefetch the next chunk into the other stage (free: its MMAs and reads
-    // finished before the barrier that closed the previous iteration)
-    if (cl + 1 < n_seg) {
-      if (tid == 0) {
-        mbar_arrive_expect_tx(&full[s ^ 1], SLOT_USED);
-        bulk_g2s(nstg, slots + (size_t)(cl + 1) * SLOT, SLOT_USED, &full[s ^ 1]);
-      }
-      ++issued;
-    }
-    // (Y S)ᵀ = Sᵀ Yᵀ (waited for right away), then Oᵀ = Sᵀ Q̄ᵀ
-    if (tid == 0) {
-      const uint64_t a0 = desc_k_sw(smem_u32(smem + S_ST), 0, BS_ROW128);
-      const uint64_t y0 = desc_mn_sw(smem_u32(stg + SL_YT), 0, BS_ROW128);
-      const uint64_t q0 = desc_k_sw(smem_u32(stg + SL_QB), 0, BS_ROW64);
+      const uint32_t id64 = idesc_f16(128, 64, false, false);
+      const uint32_t id64n = idesc_f16(128, 64, false, true);
+      const uint64_t sdesc0 = desc_k_sw(smem_u32(smem + S_ST), 0, BS_ROW128);
+      const uint64_t udesc0 = desc_k_sw(smem_u32(smem + S_UT), 0, BS_ROW128);
+      bool ok = true;
+      for (int c = 0; c < n_seg && ok; ++c) {
+        const int s = c & 1;
+        const uint32_t ph = (uint32_t)(c & 1);
+        uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
+        const uint32_t ob = ST_O + 64u * (uint32_t)s;
+        ok = mbar_wait_or_stop(&full[s], (uint32_t)((c >> 1) & 1), vflag);
+        if (!ok) break;
+        ++landed;
+        const uint64_t y0 = desc_mn_sw(smem_u32(stg + SL_YT), 0, BS_ROW128);
+        // (Y S)ᵀ = Sᵀ Yᵀ, keys 0..63 then 64..127 as the fp16 copy lands
+        ok = mbar_wait_or_stop(b_slo, ph, vflag);
+        if (!ok) break;
+        fence_after_sync();
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        mma16(tmem + ST_YS, a0 + k_step_sw(ks, BS_ROW128), y0 + mn_step_sw(ks), idesc_f16(128, 64, false, true),
-              ks > 0);
-      mma_commit(bar_ys);
+        for (int ks = 0; ks < 4; ++ks)
+          mma16(tmem + ST_YS, sdesc0 + k_step_sw(ks, BS_ROW128), y0 + mn_step_sw(ks), id64n, ks > 0);
+        ok = mbar_wait_or_stop(b_shi, ph, vflag);
+        if (!ok) break;
+        fence_after_sync();
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        mma16(tmem + ob, a0 + k_step_sw(ks, BS_ROW128), q0 + k_step_sw(ks, BS_ROW64),
-              idesc_f16(128, 64, false, false), ks > 0);
-    }
-    // meanwhile: the previous chunk's outputs (its MMAs completed before the
-    // barrier that closed the previous iteration)
-    if (cl > 0) out_epilogue(ST_O + 64u * (uint32_t)(s ^ 1), prev_t0, prev_L);
-    __syncwarp();
-    {
-      uint32_t ph = mphase;
-      wait_mma(bar_ys, ph, sflag);
-    }
-    // Uᵀ = U_wᵀ − (Y S)ᵀ
-    {
-      const int c0 = lo ? 0 : 32;
-      float ys[32], uw[32];
-      tmem_ld16(t_lane + ST_YS + c0, ys);
-      tmem_ld16(t_lane + ST_YS + c0 + 16, ys + 16);
+        for (int ks = 4; ks < 8; ++ks)
+          mma16(tmem + ST_YS, sdesc0 + k_step_sw(ks, BS_ROW128), y0 + mn_step_sw(ks), id64n, 1);
+        mma_commit(b_ys);
+        // Oᵀ = Sᵀ Q̄ᵀ into this chunk's buffer, once chunk c − 2 has left it
+        if (c >= 2) {
+          ok = mbar_wait_or_stop(&b_of[s], (uint32_t)(((c - 2) >> 1) & 1), vflag);
+          if (!ok) break;
+          fence_after_sync();
+        }
+        const uint64_t q0 = desc_k_sw(smem_u32(stg + SL_QB), 0, BS_ROW64);
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 8)
-        unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + sw_off(row, c0 + cb, BS_ROW128)), uw + cb);
-      tmem_wait_ld();
+        for (int ks = 0; ks < 8; ++ks)
+          mma16(tmem + ob, sdesc0 + k_step_sw(ks, BS_ROW128), q0 + k_step_sw(ks, BS_ROW64), id64, ks > 0);
+        // Sᵀ += Uᵀ K_end (two key halves), then Oᵀ += Uᵀ Aqkᵀ
+        ok = mbar_wait_or_stop(b_u, ph, vflag);
+        if (!ok) break;
+        fence_after_sync();
+        const uint64_t ke0 = desc_mn_sw(smem_u32(stg + SL_KE), 0, BS_ROW64);
+        const uint64_t ke1 = desc_mn_sw(smem_u32(stg + SL_KE + BS_ROW64), 0, BS_ROW64);
 #pragma unroll
-      for (int u = 0; u < 32; ++u) uw[u] -= ys[u];
+        for (int ks = 0; ks < 4; ++ks)
+          mma16(tmem + ST_S, udesc0 + k_step_sw(ks, BS_ROW128), ke0 + mn_step_sw(ks), id64n, 1);
+        mma_commit(b_sa);
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_UT + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(uw + cb));
-    }
-    sync_for_mma();
-    // Sᵀ += Uᵀ K_end (waited for by the state copy), then Oᵀ += Uᵀ Aqkᵀ
-    if (tid == 0) {
-      const uint64_t u0 = desc_k_sw(smem_u32(smem + S_UT), 0, BS_ROW128);
-      const uint64_t k0 = desc_mn_sw(smem_u32(stg + SL_KE), 0, BS_ROW64);
-      const uint64_t q0 = desc_k_sw(smem_u32(stg + SL_AQ), 0, BS_ROW64);
+        for (int ks = 0; ks < 4; ++ks)
+          mma16(tmem + ST_S + 64, udesc0 + k_step_sw(ks, BS_ROW128), ke1 + mn_step_sw(ks), id64n, 1);
+        mma_commit(b_sb);
+        const uint64_t aq0 = desc_k_sw(smem_u32(stg + SL_AQ), 0, BS_ROW64);
 #pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks)
-        mma16(tmem + ST_S, u0 + k_step_sw(ks, BS_ROW128), k0 + mn_step_sw(ks), idesc_f16(128, 128, false, true), 1);
-      mma_commit(bar_st);
-#pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks)
-        mma16(tmem + ob, u0 + k_step_sw(ks, BS_ROW128), q0 + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, false, false),
-              1);
-      mma_commit(bar_o);
-    }
-    __syncwarp();
-    {
-      uint32_t ph = mphase;
-      wait_mma(bar_st, ph, sflag);
-    }
-    // Next chunk's fp16 Sᵀ operand, then Sᵀ ← Sᵀ Γ_next in TMEM (the next
-    // slot's γ_C; its copy was issued at the top of this iteration).
-    const bool more = cl + 1 < n_seg;
-    if (more) {
-      if (!mbar_wait(&full[s ^ 1], ((cl + 1) >> 1) & 1)) atomicOr(sflag, 1);
-      ++waited;
-    }
-    {
-      const float* gN = reinterpret_cast<const float*>(nstg + SL_GC);
-      const int c0 = lo ? 0 : 64;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float v[32];
-        tmem_ld16(t_lane + ST_S + c0 + half * 32, v);
-        tmem_ld16(t_lane + ST_S + c0 + half * 32 + 16, v + 16);
-        tmem_wait_ld();
-#pragma unroll
-        for (int cb = 0; cb < 32; cb += 8)
-          st16(smem, S_ST + sw_off(row, c0 + half * 32 + cb, BS_ROW128), pack8_f16(v + cb));
-        if (more) {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] *= gN[c0 + half * 32 + u];
-          tmem_st16(t_lane + ST_S + c0 + half * 32, v);
-          tmem_st16(t_lane + ST_S + c0 + half * 32 + 16, v + 16);
+        for (int ks = 0; ks < 4; ++ks)
+          mma16(tmem + ob, udesc0 + k_step_sw(ks, BS_ROW128), aq0 + k_step_sw(ks, BS_ROW64), id64, 1);
+        mma_commit(b_o);
+        mma_commit(&b_ob[s]);
+        // stage s is free once this chunk's products are done: chunk c + 2
+        if (c + 2 < n_seg) {
+          ok = mbar_wait_or_stop(b_o, ph, vflag);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&full[s], SLOT_USED);
+          bulk_g2s(stg, slots + (size_t)(c + 2) * SLOT, SLOT_USED, &full[s]);
+          ++issued;
         }
       }
-      if (more) tmem_wait_st();
+      if (!ok) {
+        atomicOr(sflag, 1);
+        // copies still in flight complete (bounded) before shared memory is released
+        for (int k = landed; k < issued; ++k) mbar_wait(&full[k & 1], (uint32_t)((k >> 1) & 1), 1u << 16);
+      }
     }
-    {
-      uint32_t ph = mphase;
-      wait_mma(bar_o, ph, sflag);
-      mphase ^= 1u;                   // the three MMA barriers advance together
-    }
-    prev_t0 = t0;
-    prev_L = Lc;
-    sync_for_mma();
-    if (*sflag) break;
-  }
-  // the last chunk's outputs
-  if (!*sflag && n_seg > 0) out_epilogue(ST_O + 64u * (uint32_t)((n_seg - 1) & 1), prev_t0, prev_L);
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ chain warps
+    const int lq = warp & 3;
+    const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
+    const int row = lq * 32 + lane;     // dv index j of Sᵀ[j][*], Oᵀ[j][*]
+    const int hw = warp >> 2;           // which of the two warps of a lane quarter
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok && !mbar_wait_or_stop(bar, parity, vflag)) {
+        ok = false;
+        atomicOr(sflag, 1);
+      }
+      fence_after_sync();
+    };
+    // Publish this thread's fp16 operand writes and TMEM stores, then one
+    // arrival for all 256 epilogue threads.
+    auto publish = [&](uint64_t* bar) {
+      fence_async_smem();
+      fence_before_sync();
+      epi_sync();
+      if (tid == 0) mbar_arrive(bar);
+    };
 
-  if (S_out && !*sflag) {
-    const int c0 = lo ? 0 : 64;
-    float* ST = S_out + (size_t)bh * D * D;
-    for (int cb = c0; cb < c0 + 64; cb += 16) {
-      float v[16];
-      tmem_ld16(t_lane + ST_S + cb, v);
+    // Entry state: Sᵀ[j][c] = S[c][j]. The fp16 copy (operand of the first
+    // chunk's products) is the state itself; TMEM holds it multiplied by the
+    // first chunk's decay Γ, ready for the first update Sᵀ ← Sᵀ Γ + Uᵀ K_end.
+    wait(&full[0], 0);
+    {
+      const float* gC = reinterpret_cast<const float*>(smem + S_STAGE0 + SL_GC);
+      const float* S0 = S_in ? S_in + (size_t)bh * D * D : nullptr;
+      for (int cb = hw * 64; cb < hw * 64 + 64; cb += 16) {
+        float v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] = S0 ? __ldg(S0 + (size_t)(cb + u) * D + row) : 0.f;
+        st16(smem, S_ST + sw_off(row, cb, BS_ROW128), pack8_f16(v));
+        st16(smem, S_ST + sw_off(row, cb + 8, BS_ROW128), pack8_f16(v + 8));
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] *= gC[cb + u];
+        tmem_st16(t_lane + ST_S + cb, v);
+      }
+      tmem_wait_st();
+    }
+    publish(b_slo);
+    if (tid == 0) mbar_arrive(b_shi);
+
+    // fp16 copy of 32 key columns [k0, k0 + 32) of Sᵀ for the next chunk's
+    // products, and Sᵀ ← Sᵀ Γ_next in TMEM.
+    auto copy_state = [&](int k0, const float* gN) {
+      float v[32];
+      tmem_ld16(t_lane + ST_S + k0, v);
+      tmem_ld16(t_lane + ST_S + k0 + 16, v + 16);
       tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < 16; ++u) ST[(size_t)(cb + u) * D + row] = v[u];
+      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_ST + sw_off(row, k0 + cb, BS_ROW128), pack8_f16(v + cb));
+#pragma unroll
+      for (int u = 0; u < 32; ++u) v[u] *= gN[k0 + u];
+      tmem_st16(t_lane + ST_S + k0, v);
+      tmem_st16(t_lane + ST_S + k0 + 16, v + 16);
+      tmem_wait_st();
+    };
+
+    for (int c = 0; c < n_seg; ++c) {
+      const int s = c & 1;
+      const uint32_t ph = (uint32_t)(c & 1);
+      const uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
+      const uint8_t* nstg = smem + (s ? S_STAGE0 : S_STAGE1);
+      // Uᵀ = U_wᵀ − (Y S)ᵀ
+      wait(&full[s], (uint32_t)((c >> 1) & 1));
+      wait(b_ys, ph);
+      {
+        const int c0 = hw * 32;
+        float ys[32], uw[32];
+        tmem_ld16(t_lane + ST_YS + c0, ys);
+        tmem_ld16(t_lane + ST_YS + c0 + 16, ys + 16);
+#pragma unroll
+        for (int cb = 0; cb < 32; cb += 8)
+          unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + sw_off(row, c0 + cb, BS_ROW128)), uw + cb);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) uw[u] -= ys[u];
+#pragma unroll
+        for (int cb = 0; cb < 32; cb += 8) st16(smem, S_UT + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(uw + cb));
+      }
+      publish(b_u);
+      // the state for the next chunk, one key half at a time (barriers are
+      // reached by every epilogue thread whatever its own waits returned)
+      const bool more = c + 1 < n_seg;
+      if (more) wait(&full[s ^ 1], (uint32_t)(((c + 1) >> 1) & 1));
+      const float* gN = reinterpret_cast<const float*>(nstg + SL_GC);
+      wait(b_sa, ph);
+      if (more) {
+        copy_state(hw * 32, gN);
+        publish(b_slo);
+      }
+      wait(b_sb, ph);
+      if (more) {
+        copy_state(64 + hw * 32, gN);
+        publish(b_shi);
+      }
+      // stop together: every thread's flag update precedes the first barrier,
+      // one thread samples the flag, all read the sample after the second
+      if (!ok) atomicOr(sflag, 1);
+      epi_sync();
+      if (tid == 0) *estop = *vflag;
+      epi_sync();
+      if (*estop) {
+        ok = false;
+        break;
+      }
     }
-  }
-  if (*sflag && tid == 0) {
-    atomicOr(static_cast<int*>(a.workspace), 1);
-    // after an early exit a prefetched bulk copy may still be in flight:
-    // wait for it (bounded) before this CTA's shared memory is released
-    if (issued > waited) mbar_wait(&full[waited & 1], (waited >> 1) & 1, 1u << 16);
+    // S_T (the loop ran to its end on every thread or stopped on every thread)
+    const bool done = *estop == 0;
+    if (S_out && done && ok) {
+      float* ST = S_out + (size_t)bh * D * D;
+      for (int cb = hw * 64; cb < hw * 64 + 64; cb += 16) {
+        float v[16];
+        tmem_ld16(t_lane + ST_S + cb, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) ST[(size_t)(cb + u) * D + row] = v[u];
+      }
+    }
+    if (!ok) atomicOr(sflag, 1);
+  } else {
+    // ------------------------------------------------------------ output warps
+    // Oᵀ (TMEM buffer of chunk c) → staging tile [rows][128] of TOut →
+    // contiguous 16-byte stores to o, O_ROWS tokens at a time; the buffer is
+    // released as soon as it has been read.
+    const int lq = warp & 3;
+    const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
+    const int row = lq * 32 + lane;
+    const int otid = tid - 256;
+    bool ok = true;
+    TOut* so = reinterpret_cast<TOut*>(smem + S_OS);
+    constexpr int O_ROWS = 16384 / (D * (int)sizeof(TOut));   // 64 (bf16) or 32 (fp32)
+    constexpr int VEC = 16 / (int)sizeof(TOut);               // elements per 16 bytes
+    for (int c = 0; c < n_seg; ++c) {
+      const int s = c & 1;
+      const int t0 = (c_begin + c) * C;
+      const int Lc = min(C, a.T - t0);
+      if (ok && !mbar_wait_or_stop(&b_ob[s], (uint32_t)((c >> 1) & 1), vflag)) {
+        ok = false;
+        atomicOr(sflag, 1);
+      }
+      fence_after_sync();
+      float v[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld16(t_lane + ST_O + 64u * (uint32_t)s + 16 * q, v + 16 * q);
+      tmem_wait_ld();
+      fence_before_sync();
+#pragma unroll
+      for (int r0 = 0; r0 < C; r0 += O_ROWS) {
+#pragma unroll
+        for (int u = 0; u < O_ROWS; ++u) so[u * D + row] = from_f32<TOut>(a.scale * v[r0 + u]);
+        out_sync();
+        if (r0 == 0 && otid == 0) mbar_arrive(&b_of[s]);
+        const int nvec = O_ROWS * D / VEC;
+        for (int e = otid; e < nvec; e += NO) {
+          const int rr = e / (D / VEC), cc = (e % (D / VEC)) * VEC;
+          const int i = r0 + rr;
+          if (i < Lc)
+            *reinterpret_cast<uint4*>(og + (((size_t)bi * a.T + t0 + i) * a.Hv + h) * D + cc) =
+                *reinterpret_cast<const uint4*>(so + rr * D + cc);
+        }
+        out_sync();
+      }
+      // stop together (as the chain warps do)
+      if (!ok) atomicOr(sflag, 1);
+      out_sync();
+      if (otid == 0) *ostop = *vflag;
+      out_sync();
+      if (*ostop) break;
+    }
   }
   fence_before_sync();
   __syncthreads();
+  if (tid == 0 && *sflag) atomicOr(static_cast<int*>(a.workspace), 1);
   if (warp == 0) tmem_dealloc(tmem, ST_COLS);
 }
 
@@ -896,19 +984,29 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   if ((e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) !=
       cudaSuccess)
     return e;
+  // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
+  if ((e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+    return e;
   auto scan = o_bf16 ? chunk_scan_kernel<__nv_bfloat16> : chunk_scan_kernel<float>;
   if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM)) != cudaSuccess) return e;
 
   int dev = 0, sms = 148;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  // Persistent prep: two CTAs per SM. Two fit by shared memory (2 × 113 KB),
+  // registers (2 × 256 × 128) and tensor memory (2 × 256 of 512 columns); the
+  // occupancy calculator reports one for any kernel that allocates tensor
+  // memory, so the count is set here. CTAs beyond those resident would only
+  // start later (items are independent).
+  const int prep_ctas = sms * 2;
   const float* s_in = a.S0;
   for (int c0 = 0; c0 < nchunks; c0 += seg) {
     const int n = std::min(seg, nchunks - c0);
     const bool last = c0 + n >= nchunks;
     float* s_out = last ? a.ST : carry;
-    chunk_prep_kernel<<<std::min(BH * n, sms), NP, P_SMEM, s>>>(a, c0, n);
-    scan<<<BH, NT, S_SMEM, s>>>(a, c0, n, s_in, s_out);
+    chunk_prep_kernel<<<std::min(BH * n, prep_ctas), NP, P_SMEM, s>>>(a, c0, n);
+    scan<<<BH, NS, S_SMEM, s>>>(a, c0, n, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;
   }

@@ -191,6 +191,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint3
   return false;
 }
 
+// Bounded wait that also gives up as soon as *stop becomes nonzero (another
+// thread of the CTA met an error); returns true only if the phase completed.
+__device__ __forceinline__ bool mbar_wait_or_stop(uint64_t* mbar, uint32_t parity, const volatile int* stop,
+                                                  uint32_t limit = (1u << 22)) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    if (mbar_try_wait(mbar, parity)) return true;
+    if ((i & 15u) == 15u && *stop) return false;
+  }
+  return false;
+}
+
+// Plain arrive (count 1) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(mbar)) : "memory");
+}
+
 // Arrive on an mbarrier and add `bytes` to the transaction count it waits for.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(bytes)
@@ -206,6 +222,14 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
           smem_u32(dst_smem)),
       "l"(src_gmem), "r"(bytes), "r"(smem_u32(mbar))
       : "memory");
+}
+
+// Approximate reciprocal (the PTX rcp.approx.ftz.f32 instruction: at most
+// one ulp of error, subnormal inputs and results flushed to zero).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 // Pack 8 floats to 8 bf16 (16 bytes), round to nearest even.

@@ -14,6 +14,7 @@ Conceito: 16 QK heads serving 48 V heads, head dimension 128):
   2     prefill_t32768               B=1,T=32768, 16/48, d=128, chunk 64, bf16, alpha mean 4
   3     decode_b256                  B=256 sequences, one token per step, 16/48, d=128
   4     conv_prefill_b8_t8192        B=8,T=8192, 16/48, d=128, conv k=4 + L2 fused, S0 != 0
+  5     decode_b64                   B=64 sequences (profiler-sized decode), 16/48, d=128
 
 Value distributions: q,k ~ N(0,1) rows scaled to unit length (raw N(0,1) when
 the conv + L2 norm is fused into the kernel); v ~ N(0,1); alpha = sigmoid(N(mu,1))
@@ -52,6 +53,8 @@ WORKLOADS = [
     Workload("prefill_t32768", 1, 32768, 16, 48, 128, 64, "bf16", 4.0, "zeros"),
     Workload("decode_b256", 256, 1, 16, 48, 128, 64, "bf16", 3.0, "normal", decode_steps=1000),
     Workload("conv_prefill_b8_t8192", 8, 8192, 16, 48, 128, 64, "bf16", 3.0, "normal", conv=True),
+    # a quarter of the decode batch: the case profiler captures run on
+    Workload("decode_b64", 64, 1, 16, 48, 128, 64, "bf16", 3.0, "normal", decode_steps=1000),
 ]
 
 BY_NAME = {w.name: w for w in WORKLOADS}
