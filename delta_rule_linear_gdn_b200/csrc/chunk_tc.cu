@@ -74,11 +74,11 @@ constexpr int C = 64;             // chunk
 // Slots follow, one per (sequence, value head, chunk of the segment). Tiles
 // are swizzled; "BS" is the byte stride between 64-column blocks.
 constexpr size_t WS_HEAD = 256;
-constexpr int SL_YT = 0;              // Yᵀ   fp16 [128 key][64 tok]   (MN-major B of (YS)ᵀ)
-constexpr int SL_UW = 16384;          // U_wᵀ fp16 [128 dv][64 tok]
-constexpr int SL_QB = 32768;          // Q̄    fp16 [64 tok][128 key]  BS 8192 (K-major B of Oᵀ)
-constexpr int SL_KE = 49152;          // K_end fp16 [64 tok][128 key] BS 8192 (MN-major B of Sᵀ)
-constexpr int SL_AQ = 65536;          // Aqk  fp16 [64 i][64 j]        (K-major B of Oᵀ)
+constexpr int SL_YT = 0;              // Yᵀ   fp16 [128 key][64 tok]  ┐ Zᵀ = [Yᵀ | Q̄ᵀ]: the two
+constexpr int SL_QT = 16384;          // Q̄ᵀ   fp16 [128 key][64 tok]  ┘ 64-column blocks, BS 16384
+constexpr int SL_UW = 32768;          // U_wᵀ fp16 [128 dv][64 tok]
+constexpr int SL_KE = 49152;          // K_end fp16 [64 tok][128 key] BS 8192
+constexpr int SL_AQ = 65536;          // −Aqk fp16 [64 i][64 j]
 constexpr int SL_GC = 73728;          // γ_C  fp32 [128]
 constexpr int SLOT_USED = 74240;      // bytes copied per chunk
 constexpr int SLOT = 74752;           // slot stride (1 KB multiple)
@@ -119,16 +119,15 @@ constexpr int P_SMEM = P_FLAG + 16;
 constexpr uint32_t PT_GM = 0, PT_GB = 64, PT_YT = 128, PT_UW = 192, PT_COLS = 256;
 
 // ------------------------------------------------------------------ scan smem
-constexpr int S_STAGE0 = 0;
-constexpr int S_STAGE1 = SLOT;
-constexpr int S_ST = 2 * SLOT;        // Sᵀ fp16 [128 dv][128 key], BS 16K
-constexpr int S_UT = S_ST + D * D * 2;// Uᵀ fp16 [128 dv][64 tok]
-constexpr int S_OS = S_UT + D * C * 2;// output staging, 16 KB of [rows][128] TOut
-constexpr int S_BAR = S_OS + 16384;   // 13 mbarriers (see the scan kernel)
+// Two stages (see the scan kernel for their layout), then:
+constexpr int S_SH = 2 * 66560;       // −S fp16 [128 key][64 dv]
+constexpr int S_U = S_SH + 16384;     // U fp16 [64 tok][64 dv]
+constexpr int S_I = S_U + 8192;       // [I_64; 0] fp16 [128][64]
+constexpr int S_BAR = S_I + 16384;    // 10 mbarriers (see the scan kernel)
 constexpr int S_TMEMP = S_BAR + 128;
 constexpr int S_FLAG = S_TMEMP + 16;
 constexpr int S_SMEM = S_FLAG + 16;
-constexpr uint32_t ST_S = 0, ST_YS = 128, ST_O = 192, ST_COLS = 512;   // Oᵀ double-buffered: 192, 256
+constexpr uint32_t ST_S = 0, ST_D = 64, ST_COLS = 256;   // S (64 columns), D double-buffered: 64, 128
 
 __device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
   *reinterpret_cast<uint4*>(base + off) = v;
@@ -141,15 +140,6 @@ __device__ __forceinline__ void unpack4_bf16(uint2 u, float* x) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
   const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
   x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
-__device__ __forceinline__ void unpack8_f16(uint4 u, float* x) {
-  const __half2* h = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(h[i]);
-    x[2 * i] = f.x;
-    x[2 * i + 1] = f.y;
-  }
 }
 
 __device__ __forceinline__ void wait_mma(uint64_t* bar, uint32_t& phase, int* sflag) {
@@ -383,6 +373,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
 
     // -------- pass 2: key-side operand tiles, tile by tile per token
+    uint32_t qpk[4][4];
+    float qlo[4];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (u == 4) load_key(4);
@@ -413,7 +405,14 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     else                                                                      \
       st8(dst, off, pack4_f16(o[0], o[1], o[2], o[3]));                       \
   }
-      GDN2_TILE(slot, SL_QB + p64, qx[c] * g[c])
+      // Q̄ᵀ: each key's token pairs packed as they are produced
+      if ((u & 1) == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qlo[c] = qx[c] * g[c];
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qpk[c][u >> 1] = pack2_f16(qlo[c], qx[c] * g[c]);
+      }
       GDN2_TILE(slot, SL_KE + p64, kx[c] * (ps[c] * rf[c]))
       GDN2_TILE(smem, P_EB + p64, e[c] * g[c])
       GDN2_GRAM_TILE(smem, P_GM + p128, e[c] * fe[c])
@@ -428,6 +427,10 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #undef GDN2_TILE
 #undef GDN2_GRAM_TILE
     }
+    // Q̄ᵀ [key][tok]: the thread's 8 tokens of each of its keys form one 16-byte chunk
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      st16(slot, SL_QT + sw_off(c0 + c, i0, BS_ROW128), make_uint4(qpk[c][0], qpk[c][1], qpk[c][2], qpk[c][3]));
     sync_for_mma();
 
     // -------- Gram MMAs: [T; Aqk] candidates
@@ -478,6 +481,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
         for (int u = 0; u < 32; u += 4)
           *reinterpret_cast<float4*>(sT + i * TS + j0 + u) = make_float4(dm[u], dm[u + 1], dm[u + 2], dm[u + 3]);
       } else {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) dm[u] = -dm[u];            // the scan adds −Aqk·U
 #pragma unroll
         for (int cb = 0; cb < 32; cb += 8) st16(slot, SL_AQ + sw_off(i, j0 + cb, BS_ROW64), pack8_f16(dm + cb));
       }
@@ -620,52 +625,75 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 }
 
 // =============================================================================
-// scan kernel: one CTA per (sequence, value head), chunks of the segment in
-// order. Warp 12 issues the tensor-core products and the slot copies (one
-// thread); warps 0..7 run the state chain, warps 8..11 write the outputs.
-// They hand over through mbarriers:
-//   MMA thread, chunk c:  (Y S)ᵀ [after each half of the fp16 Sᵀ copy] → Oᵀ =
-//     Sᵀ Q̄ᵀ → [after Uᵀ] Sᵀ += Uᵀ K_end in two 64-key halves → Oᵀ += Uᵀ Aqkᵀ →
-//     [when chunk c's products are done] copy of chunk c + 2's slot;
-//   chain warps, chunk c:  Uᵀ = U_wᵀ − (Y S)ᵀ → per key half: fp16 Sᵀ copy for
-//     chunk c + 1 and Sᵀ ← Sᵀ Γ_{c+1} in TMEM;
-//   output warps, chunk c:  Oᵀ (double-buffered in TMEM) → o.
+// scan kernel: two CTAs per (sequence, value head), each owning one 64-wide
+// half of d_v (the recurrence never mixes d_v columns), walking the chunks of
+// the segment in order. Per chunk c, with the state S (d_k × 64, fp32 in TMEM,
+// one key per lane) and Z = [Y; Q̄] stacked along the rows:
+//   D  = Z (−S) + [I; 0] U_w  → rows 0..63: U = U_w − Y S, rows 64..127: −Q̄ S
+//   S ← Γ S + K_endᵀ U        (TMEM holds Γ S already)
+//   D_rows 64..127 −= Aqk U   → −O / scale
+// Every product has M = 128. Warp 8 issues the products and the slot copies
+// (one thread); warps with TMEM lanes 0..63 write U, those with lanes 64..127
+// write the outputs of the previous chunk, and all eight copy the state (fp16
+// −S for the next chunk's products, TMEM ← S·Γ_next).
 // =============================================================================
-constexpr int NS = 416;               // scan threads: 8 chain warps, 4 output warps, 1 MMA warp
-constexpr int NO = 128;               // output threads
+constexpr int NS = 288;               // scan threads: 8 epilogue warps + 1 MMA warp
+
+// Stage (one chunk's operands for this half), filled by three bulk copies.
+constexpr int SG_ZT = 0;              // Zᵀ = [Yᵀ | Q̄ᵀ]  [128 key][128 tok], BS 16384
+constexpr int SG_UW = 32768;          // U_wᵀ rows of this half [64 dv][64 tok]
+constexpr int SG_KE = 40960;          // K_end [64 tok][128 key], BS 8192
+constexpr int SG_AQ = 57344;          // −Aqk [64][64] (must follow K_end: see the O product)
+constexpr int SG_GC = 65536;          // γ_C [128] fp32
+constexpr int SG_BYTES = 32768 + 8192 + (SLOT_USED - SL_KE);
+constexpr int STAGE = 66560;          // stage stride (1 KB multiple)
+static_assert(S_SH == 2 * STAGE, "scan shared-memory layout");
+static_assert(SG_AQ == SG_KE + 16384 && SG_GC == SG_AQ + 8192, "stage tail copied in one piece");
+static_assert(SL_AQ == SL_KE + 16384 && SL_GC == SL_AQ + 8192, "slot tail copied in one piece");
+static_assert(SG_GC + 512 <= STAGE, "stage size");
+
+// 16 bytes of output: 8 bf16 or 4 fp32 values of sc · x.
+template <typename TOut> __device__ __forceinline__ uint4 pack_out(const float* x, float sc);
+template <> __device__ __forceinline__ uint4 pack_out<__nv_bfloat16>(const float* x, float sc) {
+  float y[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) y[k] = sc * x[k];
+  return pack8_bf16(y);
+}
+template <> __device__ __forceinline__ uint4 pack_out<float>(const float* x, float sc) {
+  return make_uint4(__float_as_uint(sc * x[0]), __float_as_uint(sc * x[1]), __float_as_uint(sc * x[2]),
+                    __float_as_uint(sc * x[3]));
+}
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
-__device__ __forceinline__ void out_sync() { asm volatile("bar.sync 2, 128;\n" ::: "memory"); }
+__device__ __forceinline__ void u_sync() { asm volatile("bar.sync 2, 128;\n" ::: "memory"); }
+__device__ __forceinline__ void o_sync() { asm volatile("bar.sync 3, 128;\n" ::: "memory"); }
 
 template <typename TOut>
 __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, const float* S_in,
                                                            float* S_out) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_BAR);
-  uint64_t* full = bars;                // [2] slot copy landed in stage s
-  uint64_t* b_ys = bars + 2;            // (Y S)ᵀ done
-  uint64_t* b_sa = bars + 3;            // state update, keys 0..63, done
-  uint64_t* b_sb = bars + 4;            // state update, keys 64..127, done
-  uint64_t* b_o = bars + 5;             // every product of the chunk done
-  uint64_t* b_u = bars + 6;             // Uᵀ written
-  uint64_t* b_slo = bars + 7;           // fp16 Sᵀ keys 0..63 written (and TMEM scaled)
-  uint64_t* b_shi = bars + 8;           // keys 64..127
-  uint64_t* b_of = bars + 9;            // [2] Oᵀ buffer read out
-  uint64_t* b_ob = bars + 11;           // [2] Oᵀ buffer complete (one phase per use)
+  uint64_t* full = bars;                // [2] stage s loaded
+  uint64_t* b_d = bars + 2;             // Z(−S) + [I;0]U_w done (U and −Q̄S in D)
+  uint64_t* b_u = bars + 3;             // U written (fp16)
+  uint64_t* b_s = bars + 4;             // state update done
+  uint64_t* b_sh = bars + 5;            // fp16 −S written and TMEM scaled
+  uint64_t* b_o = bars + 6;             // [2] D buffer holds the chunk's −O
+  uint64_t* b_of = bars + 8;            // [2] D buffer read out
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + S_TMEMP);
   int* sflag = reinterpret_cast<int*>(smem + S_FLAG);
-  int* estop = sflag + 1;               // the chain warps' sample of the flag
-  int* ostop = sflag + 2;               // the output warps' sample
+  volatile int* estop = sflag + 1;      // [2] the epilogue warps' samples of the flag
   const volatile int* vflag = sflag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x >> 1, half = blockIdx.x & 1;
   const int h = bh % a.Hv, bi = bh / a.Hv;
   const uint8_t* slots = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + (size_t)bh * n_seg * SLOT;
   TOut* og = static_cast<TOut*>(a.o);
 
   if (tid == 0) {
-    for (int i = 0; i < 13; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     sflag[0] = 0;
     sflag[1] = 0;
@@ -680,79 +708,72 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   fence_after_sync();
   const uint32_t tmem = *tmem_ptr;
 
-  if (warp == 12) {
+  if (warp == 8) {
     // ------------------------------------------------------------ MMA thread
     if (lane == 0) {
-      int issued = 0, landed = 0;       // slot copies issued / seen complete
+      auto load = [&](int c) {
+        uint8_t* stg = smem + (c & 1) * STAGE;
+        const uint8_t* sl = slots + (size_t)c * SLOT;
+        mbar_arrive_expect_tx(&full[c & 1], SG_BYTES);
+        bulk_g2s(stg + SG_ZT, sl + SL_YT, 32768, &full[c & 1]);
+        bulk_g2s(stg + SG_UW, sl + SL_UW + half * 8192, 8192, &full[c & 1]);
+        bulk_g2s(stg + SG_KE, sl + SL_KE, SLOT_USED - SL_KE, &full[c & 1]);
+      };
+      int issued = 0, landed = 0;       // chunks whose copies were issued / seen complete
       for (int c = 0; c < n_seg && c < 2; ++c) {
-        mbar_arrive_expect_tx(&full[c], SLOT_USED);
-        bulk_g2s(smem + (c ? S_STAGE1 : S_STAGE0), slots + (size_t)c * SLOT, SLOT_USED, &full[c]);
+        load(c);
         ++issued;
       }
-      const uint32_t id64 = idesc_f16(128, 64, false, false);
-      const uint32_t id64n = idesc_f16(128, 64, false, true);
-      const uint64_t sdesc0 = desc_k_sw(smem_u32(smem + S_ST), 0, BS_ROW128);
-      const uint64_t udesc0 = desc_k_sw(smem_u32(smem + S_UT), 0, BS_ROW128);
+      const uint32_t id_zs = idesc_f16(128, 64, true, true);     // Zᵀ (MN) × −S (MN)
+      const uint32_t id_iu = idesc_f16(128, 64, false, false);   // [I;0] (K) × U_wᵀ (K)
+      const uint32_t id_kn = idesc_f16(128, 64, true, true);     // K_endᵀ (MN) × U (MN)
+      const uint32_t id_au = idesc_f16(128, 64, false, true);    // [·;−Aqk] (K) × U (MN)
+      const uint64_t sh0 = desc_mn_sw(smem_u32(smem + S_SH), 0, BS_ROW128);
+      const uint64_t u0 = desc_mn_sw(smem_u32(smem + S_U), 0, BS_ROW64);
+      const uint64_t i0 = desc_k_sw(smem_u32(smem + S_I), 0, BS_ROW128);
       bool ok = true;
       for (int c = 0; c < n_seg && ok; ++c) {
         const int s = c & 1;
         const uint32_t ph = (uint32_t)(c & 1);
-        uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
-        const uint32_t ob = ST_O + 64u * (uint32_t)s;
-        ok = mbar_wait_or_stop(&full[s], (uint32_t)((c >> 1) & 1), vflag);
+        uint8_t* stg = smem + s * STAGE;
+        const uint32_t db = ST_D + 64u * (uint32_t)s;
+        ok = mbar_wait_or_stop(&full[s], (uint32_t)((c >> 1) & 1), vflag) &&
+             (c < 2 || mbar_wait_or_stop(&b_of[s], (uint32_t)(((c - 2) >> 1) & 1), vflag));
         if (!ok) break;
         ++landed;
-        const uint64_t y0 = desc_mn_sw(smem_u32(stg + SL_YT), 0, BS_ROW128);
-        // (Y S)ᵀ = Sᵀ Yᵀ, keys 0..63 then 64..127 as the fp16 copy lands
-        ok = mbar_wait_or_stop(b_slo, ph, vflag);
+        fence_after_sync();
+        // D = [I; 0] U_w (needs no state: issued ahead), then D += Z (−S)
+        const uint64_t z0 = desc_mn_sw(smem_u32(stg + SG_ZT), 0, BS_ROW128);
+        const uint64_t w0 = desc_k_sw(smem_u32(stg + SG_UW), 0, BS_ROW64);
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma16(tmem + db, i0 + k_step_sw(ks, BS_ROW128), w0 + k_step_sw(ks, BS_ROW64), id_iu, ks > 0);
+        ok = mbar_wait_or_stop(b_sh, ph, vflag);
         if (!ok) break;
         fence_after_sync();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma16(tmem + ST_YS, sdesc0 + k_step_sw(ks, BS_ROW128), y0 + mn_step_sw(ks), id64n, ks > 0);
-        ok = mbar_wait_or_stop(b_shi, ph, vflag);
-        if (!ok) break;
-        fence_after_sync();
-#pragma unroll
-        for (int ks = 4; ks < 8; ++ks)
-          mma16(tmem + ST_YS, sdesc0 + k_step_sw(ks, BS_ROW128), y0 + mn_step_sw(ks), id64n, 1);
-        mma_commit(b_ys);
-        // Oᵀ = Sᵀ Q̄ᵀ into this chunk's buffer, once chunk c − 2 has left it
-        if (c >= 2) {
-          ok = mbar_wait_or_stop(&b_of[s], (uint32_t)(((c - 2) >> 1) & 1), vflag);
-          if (!ok) break;
-          fence_after_sync();
-        }
-        const uint64_t q0 = desc_k_sw(smem_u32(stg + SL_QB), 0, BS_ROW64);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma16(tmem + ob, sdesc0 + k_step_sw(ks, BS_ROW128), q0 + k_step_sw(ks, BS_ROW64), id64, ks > 0);
-        // Sᵀ += Uᵀ K_end (two key halves), then Oᵀ += Uᵀ Aqkᵀ
+        for (int ks = 0; ks < D / 16; ++ks) mma16(tmem + db, z0 + mn_step_sw(ks), sh0 + mn_step_sw(ks), id_zs, 1);
+        mma_commit(b_d);
+        // S += K_endᵀ U (TMEM holds Γ S), then D_rows 64..127 += (−Aqk) U; the
+        // A operand of the latter starts 64 rows before −Aqk (in K_end), whose
+        // products land in rows 0..63, already read out as U.
         ok = mbar_wait_or_stop(b_u, ph, vflag);
         if (!ok) break;
         fence_after_sync();
-        const uint64_t ke0 = desc_mn_sw(smem_u32(stg + SL_KE), 0, BS_ROW64);
-        const uint64_t ke1 = desc_mn_sw(smem_u32(stg + SL_KE + BS_ROW64), 0, BS_ROW64);
+        const uint64_t ke0 = desc_mn_sw(smem_u32(stg + SG_KE), 0, BS_ROW64);
+        const uint64_t aq0 = desc_k_sw(smem_u32(stg + SG_AQ - 8192), 0, BS_ROW64);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma16(tmem + ST_S, udesc0 + k_step_sw(ks, BS_ROW128), ke0 + mn_step_sw(ks), id64n, 1);
-        mma_commit(b_sa);
+        for (int ks = 0; ks < C / 16; ++ks) mma16(tmem + ST_S, ke0 + mn_step_sw(ks), u0 + mn_step_sw(ks), id_kn, 1);
+        mma_commit(b_s);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma16(tmem + ST_S + 64, udesc0 + k_step_sw(ks, BS_ROW128), ke1 + mn_step_sw(ks), id64n, 1);
-        mma_commit(b_sb);
-        const uint64_t aq0 = desc_k_sw(smem_u32(stg + SL_AQ), 0, BS_ROW64);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma16(tmem + ob, udesc0 + k_step_sw(ks, BS_ROW128), aq0 + k_step_sw(ks, BS_ROW64), id64, 1);
-        mma_commit(b_o);
-        mma_commit(&b_ob[s]);
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma16(tmem + db, aq0 + k_step_sw(ks, BS_ROW64), u0 + mn_step_sw(ks), id_au, 1);
+        mma_commit(&b_o[s]);
         // stage s is free once this chunk's products are done: chunk c + 2
         if (c + 2 < n_seg) {
-          ok = mbar_wait_or_stop(b_o, ph, vflag);
+          ok = mbar_wait_or_stop(&b_o[s], (uint32_t)((c >> 1) & 1), vflag);
           if (!ok) break;
-          mbar_arrive_expect_tx(&full[s], SLOT_USED);
-          bulk_g2s(stg, slots + (size_t)(c + 2) * SLOT, SLOT_USED, &full[s]);
+          load(c + 2);
           ++issued;
         }
       }
@@ -763,12 +784,14 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       }
     }
     __syncwarp();
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ chain warps
+  } else {
+    // ------------------------------------------------------------ epilogue warps
     const int lq = warp & 3;
     const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
-    const int row = lq * 32 + lane;     // dv index j of Sᵀ[j][*], Oᵀ[j][*]
-    const int hw = warp >> 2;           // which of the two warps of a lane quarter
+    const int row = lq * 32 + lane;     // TMEM lane: a key of S; a row of D
+    const int c0 = (warp >> 2) * 32;    // this warp's 32 of the half's 64 columns
+    const bool u_warp = lq < 2;         // D rows 0..63 (U) or 64..127 (outputs)
+    const int dv0 = half * 64 + c0;     // first d_v column of this thread's 32
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok && !mbar_wait_or_stop(bar, parity, vflag)) {
@@ -777,165 +800,142 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       }
       fence_after_sync();
     };
-    // Publish this thread's fp16 operand writes and TMEM stores, then one
-    // arrival for all 256 epilogue threads.
-    auto publish = [&](uint64_t* bar) {
-      fence_async_smem();
-      fence_before_sync();
-      epi_sync();
-      if (tid == 0) mbar_arrive(bar);
-    };
 
-    // Entry state: Sᵀ[j][c] = S[c][j]. The fp16 copy (operand of the first
-    // chunk's products) is the state itself; TMEM holds it multiplied by the
-    // first chunk's decay Γ, ready for the first update Sᵀ ← Sᵀ Γ + Uᵀ K_end.
+    // Constant [I_64; 0] (rows × 64 columns) and the entry state: fp16 −S for
+    // the first chunk's products, TMEM ← S · Γ of the first chunk.
+    {
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = (row == c0 + cb + u) ? 1.f : 0.f;
+        st16(smem, S_I + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(x));
+      }
+    }
     wait(&full[0], 0);
     {
-      const float* gC = reinterpret_cast<const float*>(smem + S_STAGE0 + SL_GC);
-      const float* S0 = S_in ? S_in + (size_t)bh * D * D : nullptr;
-      for (int cb = hw * 64; cb < hw * 64 + 64; cb += 16) {
-        float v[16];
+      const float g = reinterpret_cast<const float*>(smem + SG_GC)[row];
+      const float* S0 = S_in ? S_in + ((size_t)bh * D + row) * D + dv0 : nullptr;
+      float v[32];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] = S0 ? __ldg(S0 + (size_t)(cb + u) * D + row) : 0.f;
-        st16(smem, S_ST + sw_off(row, cb, BS_ROW128), pack8_f16(v));
-        st16(smem, S_ST + sw_off(row, cb + 8, BS_ROW128), pack8_f16(v + 8));
-#pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] *= gC[cb + u];
-        tmem_st16(t_lane + ST_S + cb, v);
+      for (int u = 0; u < 32; u += 4) {
+        const float4 x = S0 ? __ldg(reinterpret_cast<const float4*>(S0 + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
       }
+      float n[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) n[u] = -v[u];
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(n + cb));
+#pragma unroll
+      for (int u = 0; u < 32; ++u) v[u] *= g;
+      tmem_st16(t_lane + ST_S + c0, v);
+      tmem_st16(t_lane + ST_S + c0 + 16, v + 16);
       tmem_wait_st();
     }
-    publish(b_slo);
-    if (tid == 0) mbar_arrive(b_shi);
+    fence_async_smem();
+    fence_before_sync();
+    epi_sync();
+    if (tid == 0) mbar_arrive(b_sh);
 
-    // fp16 copy of 32 key columns [k0, k0 + 32) of Sᵀ for the next chunk's
-    // products, and Sᵀ ← Sᵀ Γ_next in TMEM.
-    auto copy_state = [&](int k0, const float* gN) {
+    // Outputs of chunk cc from D buffer `db`: row 64 + i of D is token i; this
+    // thread writes 32 contiguous d_v values of it.
+    auto out_rows = [&](int cc, uint32_t db, uint64_t* freed) {
+      const int t0o = (c_begin + cc) * C;
+      const int Lco = min(C, a.T - t0o);
       float v[32];
-      tmem_ld16(t_lane + ST_S + k0, v);
-      tmem_ld16(t_lane + ST_S + k0 + 16, v + 16);
+      tmem_ld16(t_lane + db + c0, v);
+      tmem_ld16(t_lane + db + c0 + 16, v + 16);
       tmem_wait_ld();
+      fence_before_sync();
+      o_sync();
+      if (tid == 64) mbar_arrive(freed);           // first thread of the output warps
+      const int i = row - 64;
+      if (i < Lco) {
+        TOut* dst = og + (((size_t)bi * a.T + t0o + i) * a.Hv + h) * D + dv0;
+        constexpr int VEC = 16 / (int)sizeof(TOut);
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_ST + sw_off(row, k0 + cb, BS_ROW128), pack8_f16(v + cb));
-#pragma unroll
-      for (int u = 0; u < 32; ++u) v[u] *= gN[k0 + u];
-      tmem_st16(t_lane + ST_S + k0, v);
-      tmem_st16(t_lane + ST_S + k0 + 16, v + 16);
-      tmem_wait_st();
+        for (int u = 0; u < 32; u += VEC) *reinterpret_cast<uint4*>(dst + u) = pack_out<TOut>(v + u, -a.scale);
+      }
     };
 
+    bool stopped = false;
     for (int c = 0; c < n_seg; ++c) {
       const int s = c & 1;
       const uint32_t ph = (uint32_t)(c & 1);
-      const uint8_t* stg = smem + (s ? S_STAGE1 : S_STAGE0);
-      const uint8_t* nstg = smem + (s ? S_STAGE0 : S_STAGE1);
-      // Uᵀ = U_wᵀ − (Y S)ᵀ
-      wait(&full[s], (uint32_t)((c >> 1) & 1));
-      wait(b_ys, ph);
-      {
-        const int c0 = hw * 32;
-        float ys[32], uw[32];
-        tmem_ld16(t_lane + ST_YS + c0, ys);
-        tmem_ld16(t_lane + ST_YS + c0 + 16, ys + 16);
-#pragma unroll
-        for (int cb = 0; cb < 32; cb += 8)
-          unpack8_f16(*reinterpret_cast<const uint4*>(stg + SL_UW + sw_off(row, c0 + cb, BS_ROW128)), uw + cb);
+      const uint32_t db = ST_D + 64u * (uint32_t)s;
+      if (u_warp) {
+        // U (rows 0..63 of D) → fp16 tile [tok][dv]
+        wait(b_d, ph);
+        float v[32];
+        tmem_ld16(t_lane + db + c0, v);
+        tmem_ld16(t_lane + db + c0 + 16, v + 16);
         tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 32; ++u) uw[u] -= ys[u];
-#pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(smem, S_UT + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(uw + cb));
+        for (int cb = 0; cb < 32; cb += 8) st16(smem, S_U + sw_off(row, c0 + cb, BS_ROW64), pack8_f16(v + cb));
+        fence_async_smem();
+        fence_before_sync();
+        u_sync();
+        if (tid == 0) mbar_arrive(b_u);
+      } else if (c > 0) {
+        // outputs of the previous chunk
+        wait(&b_o[s ^ 1], (uint32_t)(((c - 1) >> 1) & 1));
+        out_rows(c - 1, ST_D + 64u * (uint32_t)(s ^ 1), &b_of[s ^ 1]);
       }
-      publish(b_u);
-      // the state for the next chunk, one key half at a time (barriers are
-      // reached by every epilogue thread whatever its own waits returned)
+      // the state: fp16 −S for the next chunk and TMEM ← S · Γ_next; S_T after the last
       const bool more = c + 1 < n_seg;
       if (more) wait(&full[s ^ 1], (uint32_t)(((c + 1) >> 1) & 1));
-      const float* gN = reinterpret_cast<const float*>(nstg + SL_GC);
-      wait(b_sa, ph);
-      if (more) {
-        copy_state(hw * 32, gN);
-        publish(b_slo);
+      wait(b_s, ph);
+      {
+        float v[32];
+        tmem_ld16(t_lane + ST_S + c0, v);
+        tmem_ld16(t_lane + ST_S + c0 + 16, v + 16);
+        tmem_wait_ld();
+        if (more) {
+          float n[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) n[u] = -v[u];
+#pragma unroll
+          for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(n + cb));
+          const float g = reinterpret_cast<const float*>(smem + (s ^ 1) * STAGE + SG_GC)[row];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] *= g;
+          tmem_st16(t_lane + ST_S + c0, v);
+          tmem_st16(t_lane + ST_S + c0 + 16, v + 16);
+          tmem_wait_st();
+        } else if (S_out && ok) {
+          float* ST = S_out + ((size_t)bh * D + row) * D + dv0;
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(ST + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+        }
       }
-      wait(b_sb, ph);
-      if (more) {
-        copy_state(64 + hw * 32, gN);
-        publish(b_shi);
-      }
-      // stop together: every thread's flag update precedes the first barrier,
-      // one thread samples the flag, all read the sample after the second
+      // One barrier per chunk publishes the state and carries the stop
+      // decision: thread 0 samples the error flag just before it, every thread
+      // reads the sample just after it (a flag raised later is seen one chunk
+      // later; the waits in between return at once).
       if (!ok) atomicOr(sflag, 1);
+      if (more) {
+        fence_async_smem();
+        fence_before_sync();
+      }
+      // (two sample slots: slot c & 1 is rewritten only in chunk c + 2, after
+      // every thread has passed the barrier of chunk c + 1)
+      if (tid == 0) estop[c & 1] = *vflag;
       epi_sync();
-      if (tid == 0) *estop = *vflag;
-      epi_sync();
-      if (*estop) {
+      if (more && tid == 0) mbar_arrive(b_sh);
+      if (estop[c & 1] != 0) {
         ok = false;
+        stopped = true;
         break;
       }
     }
-    // S_T (the loop ran to its end on every thread or stopped on every thread)
-    const bool done = *estop == 0;
-    if (S_out && done && ok) {
-      float* ST = S_out + (size_t)bh * D * D;
-      for (int cb = hw * 64; cb < hw * 64 + 64; cb += 16) {
-        float v[16];
-        tmem_ld16(t_lane + ST_S + cb, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; ++u) ST[(size_t)(cb + u) * D + row] = v[u];
-      }
+    // the last chunk's outputs (every epilogue thread left the loop the same way)
+    if (!stopped && n_seg > 0 && !u_warp) {
+      const int s = (n_seg - 1) & 1;
+      wait(&b_o[s], (uint32_t)(((n_seg - 1) >> 1) & 1));
+      out_rows(n_seg - 1, ST_D + 64u * (uint32_t)s, &b_of[s]);
     }
     if (!ok) atomicOr(sflag, 1);
-  } else {
-    // ------------------------------------------------------------ output warps
-    // Oᵀ (TMEM buffer of chunk c) → staging tile [rows][128] of TOut →
-    // contiguous 16-byte stores to o, O_ROWS tokens at a time; the buffer is
-    // released as soon as it has been read.
-    const int lq = warp & 3;
-    const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
-    const int row = lq * 32 + lane;
-    const int otid = tid - 256;
-    bool ok = true;
-    TOut* so = reinterpret_cast<TOut*>(smem + S_OS);
-    constexpr int O_ROWS = 16384 / (D * (int)sizeof(TOut));   // 64 (bf16) or 32 (fp32)
-    constexpr int VEC = 16 / (int)sizeof(TOut);               // elements per 16 bytes
-    for (int c = 0; c < n_seg; ++c) {
-      const int s = c & 1;
-      const int t0 = (c_begin + c) * C;
-      const int Lc = min(C, a.T - t0);
-      if (ok && !mbar_wait_or_stop(&b_ob[s], (uint32_t)((c >> 1) & 1), vflag)) {
-        ok = false;
-        atomicOr(sflag, 1);
-      }
-      fence_after_sync();
-      float v[64];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(t_lane + ST_O + 64u * (uint32_t)s + 16 * q, v + 16 * q);
-      tmem_wait_ld();
-      fence_before_sync();
-#pragma unroll
-      for (int r0 = 0; r0 < C; r0 += O_ROWS) {
-#pragma unroll
-        for (int u = 0; u < O_ROWS; ++u) so[u * D + row] = from_f32<TOut>(a.scale * v[r0 + u]);
-        out_sync();
-        if (r0 == 0 && otid == 0) mbar_arrive(&b_of[s]);
-        const int nvec = O_ROWS * D / VEC;
-        for (int e = otid; e < nvec; e += NO) {
-          const int rr = e / (D / VEC), cc = (e % (D / VEC)) * VEC;
-          const int i = r0 + rr;
-          if (i < Lc)
-            *reinterpret_cast<uint4*>(og + (((size_t)bi * a.T + t0 + i) * a.Hv + h) * D + cc) =
-                *reinterpret_cast<const uint4*>(so + rr * D + cc);
-        }
-        out_sync();
-      }
-      // stop together (as the chain warps do)
-      if (!ok) atomicOr(sflag, 1);
-      out_sync();
-      if (otid == 0) *ostop = *vflag;
-      out_sync();
-      if (*ostop) break;
-    }
   }
   fence_before_sync();
   __syncthreads();
@@ -1006,7 +1006,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     const bool last = c0 + n >= nchunks;
     float* s_out = last ? a.ST : carry;
     chunk_prep_kernel<<<std::min(BH * n, prep_ctas), NP, P_SMEM, s>>>(a, c0, n);
-    scan<<<BH, NS, S_SMEM, s>>>(a, c0, n, s_in, s_out);
+    scan<<<BH * 2, NS, S_SMEM, s>>>(a, c0, n, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;
   }

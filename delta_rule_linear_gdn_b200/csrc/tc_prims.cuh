@@ -255,6 +255,12 @@ __device__ __forceinline__ uint4 pack8_f16(const float* x) {
 }
 __device__ __forceinline__ uint4 pack8(const float* x, bool bf16) { return bf16 ? pack8_bf16(x) : pack8_f16(x); }
 
+// Pack 2 floats to 2 fp16 (the first in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack2_f16(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // Pack 4 floats to 4 16-bit values (8 bytes).
 __device__ __forceinline__ uint2 pack4_f16(float a, float b, float c, float d) {
   uint2 u;
