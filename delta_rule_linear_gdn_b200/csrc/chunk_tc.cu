@@ -136,6 +136,11 @@ __device__ __forceinline__ void st8(uint8_t* base, uint32_t off, uint2 v) {
   *reinterpret_cast<uint2*>(base + off) = v;
 }
 
+__device__ __forceinline__ void unpack4_f16(uint2 u, float* x) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+  const float2 a = __half22float2(h[0]), b = __half22float2(h[1]);
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
 __device__ __forceinline__ void unpack4_bf16(uint2 u, float* x) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
   const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
@@ -165,8 +170,17 @@ constexpr int NP = 256;               // prep threads (8 warps)
 
 struct PrepSrc {
   const float *alpha, *b, *w;
-  const __nv_bfloat16 *k, *q, *v;
+  const uint16_t *k, *q, *v;      // bf16, or fp16 when preprocessed
 };
+
+// 4 q/k/v values: bf16 from the caller's tensors, fp16 from the preprocessed copies.
+template <bool F16IN>
+__device__ __forceinline__ void unpack4_in(uint2 u, float* x) {
+  if (F16IN)
+    unpack4_f16(u, x);
+  else
+    unpack4_bf16(u, x);
+}
 
 // fp32 gate of one token for 4 channels, or the token's scalar gate broadcast.
 __device__ __forceinline__ float4 gate4(const float* g, size_t gt, int c0, bool per_channel) {
@@ -190,6 +204,7 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int
   return it;
 }
 
+template <bool F16IN>
 __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + P_BAR);
@@ -235,14 +250,15 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   };
   const bool full = a.gate_mode == GDN2_GATES_FULL;
   const bool alpha_pc = a.gate_mode != GDN2_GATES_GDN;
-  const PrepSrc src{a.alpha, a.b, full ? a.w : a.b, static_cast<const __nv_bfloat16*>(a.k),
-                    static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.v)};
+  const PrepSrc src{a.alpha, a.b, full ? a.w : a.b, static_cast<const uint16_t*>(a.k),
+                    static_cast<const uint16_t*>(a.q), static_cast<const uint16_t*>(a.v)};
 
   uint32_t phase = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const Item it = decode_item(a, c_begin, item);
     uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)it.bh * n_seg + it.cl) * SLOT;
-    const size_t tok0 = (size_t)it.bi * a.T + it.t0 + i0;    // token of u = 0
+    const size_t tok0 = (size_t)it.bi * a.T + it.t0 + i0;    // gate row of u = 0
+    const size_t qtok0 = (size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i0;   // q, k, v row of u = 0
 
     // -------- pass 1: the write side Z = w ⊙ v (no decay) straight to its
     // tile; α's forward products within the quarter. The key-side inputs of
@@ -256,7 +272,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const size_t gt = (tok0 + u0 + u) * a.Hv + it.h;
-          const size_t tq = (tok0 + u0 + u) * a.Hqk + it.hq;
+          const size_t tq = (qtok0 + u0 + u) * a.Hqk + it.hq;
           bq[u] = gate4(src.b, gt, c0, full);
           kk[u] = __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0));
           qq[u] = __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0));
@@ -266,7 +282,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
         for (int u = 0; u < 4; ++u) {
           const bool ok = i0 + u0 + u < it.Lc;
           const size_t gt = (tok0 + u0 + u) * a.Hv + it.h;
-          const size_t tq = (tok0 + u0 + u) * a.Hqk + it.hq;
+          const size_t tq = (qtok0 + u0 + u) * a.Hqk + it.hq;
           bq[u] = ok ? gate4(src.b, gt, c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
           kk[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
           qq[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
@@ -283,7 +299,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           const float4 al = gate4(src.alpha, gt, c0, alpha_pc);
           f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
           wv[u] = gate4(src.w, gt, c0, full);
-          vv[u] = __ldg(reinterpret_cast<const uint2*>(src.v + gt * D + c0));
+          vv[u] = __ldg(reinterpret_cast<const uint2*>(src.v + ((qtok0 + u) * a.Hv + it.h) * D + c0));
         }
       } else {
 #pragma unroll
@@ -293,13 +309,14 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           const float4 al = ok ? gate4(src.alpha, gt, c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
           f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
           wv[u] = ok ? gate4(src.w, gt, c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
-          vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + gt * D + c0)) : make_uint2(0, 0);
+          vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + ((qtok0 + u) * a.Hv + it.h) * D + c0))
+                     : make_uint2(0, 0);
         }
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         float vx[4];
-        unpack4_bf16(vv[u], vx);
+        unpack4_in<F16IN>(vv[u], vx);
         st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
             pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
       }
@@ -382,8 +399,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       const uint32_t i128 = (uint32_t)(i0 + u) * 128;
       const uint32_t p64 = i128 + piece(u, BS_ROW64), p128 = i128 + piece(u, BS_ROW128);
       float kx[4], qx[4], e[4], rf[4], g[4], fe[4];
-      unpack4_bf16(kk[uk], kx);
-      unpack4_bf16(qq[uk], qx);
+      unpack4_in<F16IN>(kk[uk], kx);
+      unpack4_in<F16IN>(qq[uk], qx);
       e[0] = bq[uk].x * kx[0]; e[1] = bq[uk].y * kx[1]; e[2] = bq[uk].z * kx[2]; e[3] = bq[uk].w * kx[3];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -943,51 +960,158 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   if (warp == 0) tmem_dealloc(tmem, ST_COLS);
 }
 
+// =============================================================================
+// Load step of the tensor-core prefill when the depthwise causal convolution
+// (kernel 4, taps W[c][0..3] on tokens t−3..t, zero history) and/or the L2
+// normalisation of q, k (after the conv) are requested: q, k, v of the tokens
+// [t_begin, t_begin + Tseg) of every sequence → fp16 copies [B][Tseg][H][D]
+// that the prep kernel reads instead of the caller's tensors. One thread owns
+// 8 consecutive channels and walks the CTA's tokens with the last three inputs
+// in registers; the 16 threads of one head's 128 channels are one half-warp,
+// which reduces the sum of squares.
+// =============================================================================
+constexpr int QP_THREADS = 256;
+constexpr int QP_TOK = 64;            // tokens per CTA
+
+__global__ void __launch_bounds__(QP_THREADS) qkv_prep_kernel(ChunkArgs a, int t_begin, int Tseg, __half* qo,
+                                                              __half* ko, __half* vo) {
+  const int groups = (2 * a.Hqk + a.Hv) * (D / 8);
+  const int g = blockIdx.x * QP_THREADS + threadIdx.x;
+  if (g >= groups) return;            // whole half-warps: groups is a multiple of 16
+  const int bi = blockIdx.z;
+  const int lane = threadIdx.x & 31;
+  const unsigned hmask = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
+  const int ch = g * 8;               // channel in [q | k | v]
+  const int which = ch < a.Hqk * D ? 0 : (ch < 2 * a.Hqk * D ? 1 : 2);
+  const int cw = ch - (which == 0 ? 0 : (which == 1 ? a.Hqk * D : 2 * a.Hqk * D));   // channel within the tensor
+  const int H = which == 2 ? a.Hv : a.Hqk;
+  const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(which == 0 ? a.q : (which == 1 ? a.k : a.v));
+  __half* dst = which == 0 ? qo : (which == 1 ? ko : vo);
+  const bool conv = a.conv_w != nullptr;
+  const bool norm = a.l2norm && which < 2;
+  float W[8][4];
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) W[c][j] = conv ? __ldg(a.conv_w + (size_t)(ch + c) * 4 + j) : (j == 3 ? 1.f : 0.f);
+
+  const int tl0 = blockIdx.y * QP_TOK;                  // first token of this CTA, relative to t_begin
+  const int tl1 = min(tl0 + QP_TOK, Tseg);
+  const size_t row = (size_t)H * D;                     // elements per token
+  const __nv_bfloat16* base = src + (size_t)bi * a.T * row + cw;
+  auto load8 = [&](int t, float* x) {
+    if (t < 0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x[c] = 0.f;
+      return;
+    }
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + (size_t)t * row));
+    float lo[4], hi[4];
+    unpack4_bf16(make_uint2(u.x, u.y), lo);
+    unpack4_bf16(make_uint2(u.z, u.w), hi);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      x[c] = lo[c];
+      x[4 + c] = hi[c];
+    }
+  };
+  float x3[8], x2[8], x1[8];                            // inputs of t−3, t−2, t−1
+  const int t_abs0 = t_begin + tl0;
+  load8(conv ? t_abs0 - 3 : -1, x3);
+  load8(conv ? t_abs0 - 2 : -1, x2);
+  load8(conv ? t_abs0 - 1 : -1, x1);
+  for (int tl = tl0; tl < tl1; ++tl) {
+    float x0[8], y[8];
+    load8(t_begin + tl, x0);
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      y[c] = W[c][0] * x3[c] + W[c][1] * x2[c] + W[c][2] * x1[c] + W[c][3] * x0[c];
+      ss += y[c] * y[c];
+    }
+    if (norm) {
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(hmask, ss, off);
+      const float inv = rsqrtf(ss + kL2Eps);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) y[c] *= inv;
+    }
+    *reinterpret_cast<uint4*>(dst + ((size_t)bi * Tseg + tl) * row + cw) = pack8_f16(y);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      x3[c] = x2[c];
+      x2[c] = x1[c];
+      x1[c] = x0[c];
+    }
+  }
+}
+
+// Bytes of the preprocessed q, k, v copies for `tokens` tokens of every sequence.
+size_t qkv_prep_bytes(const ChunkArgs& a, size_t tokens) {
+  return (size_t)a.B * tokens * (size_t)(2 * a.Hqk + a.Hv) * D * sizeof(__half);
+}
+
 size_t state_bytes(const ChunkArgs& a) { return (size_t)a.B * a.Hv * D * D * sizeof(float); }
 
 }  // namespace
 
 bool chunk_tc_supported(const ChunkArgs& a, int qkv_bf16) {
-  return qkv_bf16 && a.dk == D && a.dv == D && a.chunk == C && a.conv_w == nullptr && !a.l2norm;
+  return qkv_bf16 && a.dk == D && a.dv == D && a.chunk == C;
 }
+
+namespace {
+bool needs_qkv_prep(const ChunkArgs& a) { return a.conv_w != nullptr || a.l2norm; }
+// Workspace per chunk of a segment: the slots of every sequence-head and,
+// with the conv / L2 load step, the preprocessed q, k, v of its tokens.
+size_t bytes_per_chunk(const ChunkArgs& a) {
+  return (size_t)a.B * a.Hv * SLOT + (needs_qkv_prep(a) ? qkv_prep_bytes(a, C) : 0);
+}
+}  // namespace
 
 // Workspace for the whole sequence in one segment.
 size_t chunk_tc_workspace(const ChunkArgs& a) {
   const size_t nchunks = (a.T + C - 1) / C;
-  return WS_HEAD + (size_t)a.B * a.Hv * nchunks * SLOT;
+  return WS_HEAD + nchunks * bytes_per_chunk(a);
 }
 
 size_t chunk_tc_min_workspace(const ChunkArgs& a, bool carry_state) {
-  return WS_HEAD + (size_t)a.B * a.Hv * SLOT + (carry_state ? state_bytes(a) : 0);
+  return WS_HEAD + bytes_per_chunk(a) + (carry_state ? state_bytes(a) : 0);
 }
 
-// Runs the chunks in segments when the workspace holds fewer chunk slots than
-// the sequence has; the state is carried between segments through S_T (or,
-// when S_T is NULL, through the end of the workspace).
+// Runs the chunks in segments when the workspace holds fewer chunks than the
+// sequence has; the state is carried between segments through S_T (or, when
+// S_T is NULL, through the end of the workspace). Workspace: status word,
+// slots [B·H_v][seg], preprocessed q|k|v of seg·C tokens (conv / L2 only),
+// carried state (only when needed).
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   const int BH = a.B * a.Hv;
   const int nchunks = (a.T + C - 1) / C;
   if (a.ws_bytes < WS_HEAD) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(a.workspace, 0, sizeof(int), s);
   if (e != cudaSuccess || BH == 0 || nchunks == 0) return e;
-  size_t slot_bytes = a.ws_bytes - WS_HEAD;
-  int seg = (int)std::min<size_t>(nchunks, slot_bytes / ((size_t)BH * SLOT));
+  const bool pre = needs_qkv_prep(a);
+  const size_t per_chunk = bytes_per_chunk(a);
+  size_t avail = a.ws_bytes - WS_HEAD;
+  int seg = (int)std::min<size_t>(nchunks, avail / per_chunk);
   float* carry = a.ST;
+  uint8_t* const ws = static_cast<uint8_t*>(a.workspace);
   if (seg < nchunks && carry == nullptr) {
     const size_t sb = state_bytes(a);
-    slot_bytes = slot_bytes > sb ? slot_bytes - sb : 0;
-    seg = (int)std::min<size_t>(nchunks, slot_bytes / ((size_t)BH * SLOT));
-    carry = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + WS_HEAD + (size_t)BH * seg * SLOT);
+    avail = avail > sb ? avail - sb : 0;
+    seg = (int)std::min<size_t>(nchunks, avail / per_chunk);
+    carry = reinterpret_cast<float*>(ws + WS_HEAD + (size_t)seg * per_chunk);
   }
   if (seg < 1) return cudaErrorInvalidValue;
+  __half* qkv = reinterpret_cast<__half*>(ws + WS_HEAD + (size_t)BH * seg * SLOT);
 
-  if ((e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) !=
-      cudaSuccess)
-    return e;
-  // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
-  if ((e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
-    return e;
+  for (auto prep : {chunk_prep_kernel<false>, chunk_prep_kernel<true>}) {
+    if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) != cudaSuccess)
+      return e;
+    // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
+    if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
+  }
   auto scan = o_bf16 ? chunk_scan_kernel<__nv_bfloat16> : chunk_scan_kernel<float>;
   if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM)) != cudaSuccess) return e;
 
@@ -1000,12 +1124,34 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   // memory, so the count is set here. CTAs beyond those resident would only
   // start later (items are independent).
   const int prep_ctas = sms * 2;
+  const int qp_groups = (2 * a.Hqk + a.Hv) * (D / 8);
   const float* s_in = a.S0;
   for (int c0 = 0; c0 < nchunks; c0 += seg) {
     const int n = std::min(seg, nchunks - c0);
     const bool last = c0 + n >= nchunks;
     float* s_out = last ? a.ST : carry;
-    chunk_prep_kernel<<<std::min(BH * n, prep_ctas), NP, P_SMEM, s>>>(a, c0, n);
+    const int grid = std::min(BH * n, prep_ctas);
+    if (pre) {
+      const int t_begin = c0 * C;
+      const int Tseg = std::min(n * C, a.T - t_begin);
+      __half* qo = qkv;
+      __half* ko = qo + (size_t)a.B * Tseg * a.Hqk * D;
+      __half* vo = ko + (size_t)a.B * Tseg * a.Hqk * D;
+      const dim3 qgrid((qp_groups + QP_THREADS - 1) / QP_THREADS, (Tseg + QP_TOK - 1) / QP_TOK, a.B);
+      qkv_prep_kernel<<<qgrid, QP_THREADS, 0, s>>>(a, t_begin, Tseg, qo, ko, vo);
+      ChunkArgs ap = a;
+      ap.q = qo;
+      ap.k = ko;
+      ap.v = vo;
+      ap.qkv_T = Tseg;
+      ap.qkv_t0 = t_begin;
+      ap.qkv_f16 = 1;
+      ap.conv_w = nullptr;
+      ap.l2norm = 0;
+      chunk_prep_kernel<true><<<grid, NP, P_SMEM, s>>>(ap, c0, n);
+    } else {
+      chunk_prep_kernel<false><<<grid, NP, P_SMEM, s>>>(a, c0, n);
+    }
     scan<<<BH * 2, NS, S_SMEM, s>>>(a, c0, n, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;

@@ -188,7 +188,7 @@ def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_
 
 
 def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=64, scale=1.0,
-                      gate_mode="full", stream=None):
+                      gate_mode="full", l2norm_qk=False, conv_w=None, stream=None):
     """Chunked prefill through ``gdn2_chunk_fwd_noalloc``: the library takes the
     kernel's scratch from its own fixed device array, so nothing is allocated
     for the call. ``o`` and ``S_T`` (or None) are caller-provided outputs (the
@@ -201,11 +201,11 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=
     H_v, d_v = v.shape[2], v.shape[3]
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check(t, name, q.dtype)
-    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S0", S0), ("S_T", S_T)):
+    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S0", S0), ("S_T", S_T), ("conv_w", conv_w)):
         _check(t, name, torch.float32)
     _check(o, "o")
     p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
-                    o_dtype=_dtype_code(o.dtype), gate_mode=gate_mode)
+                    o_dtype=_dtype_code(o.dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk, conv_w=conv_w)
     st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
             _ptr(S_T), _stream_handle(stream))
     if st != OK:

@@ -71,3 +71,20 @@ def test_noalloc_rejects_configurations_without_scratch():
     fn = gdn2.lib().gdn2_chunk_fwd_noalloc
     fn.argtypes = [ctypes.POINTER(gdn2.Params)] + [ctypes.c_void_p] * 10
     assert fn(None, *[None] * 10) == gdn2.ERR_INVALID_ARG
+
+
+def test_noalloc_conv_l2norm_segments_carry_conv_history():
+    """With the conv / L2 load step the fixed array holds fewer chunks; a
+    2-sequence, 2000-token call runs in several segments whose first tokens
+    take their conv history from the previous segment."""
+    w = replace(workload("conv_prefill_b8_t8192"), B=2, T=2000, H_qk=2, H_v=6)
+    inp = make_inputs(w, seed=29, device="cuda")
+    args = (inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"])
+    o_ref, S_ref = gdn2.chunk_fwd(*args, chunk=64, o_dtype=torch.float32, conv_w=inp["conv_w"], l2norm_qk=True)
+    o = torch.full_like(o_ref, float("nan"))
+    S = torch.full_like(S_ref, float("nan"))
+    gdn2.chunk_fwd_noalloc(*args, o=o, S_T=S, chunk=64, conv_w=inp["conv_w"], l2norm_qk=True)
+    torch.cuda.synchronize()
+    assert_close(o, np64(o_ref), TOL_BF16, "o")
+    assert_close(S, np64(S_ref), TOL_BF16, "S_T")
+    assert torch.equal(o, o_ref) and torch.equal(S, S_ref)
