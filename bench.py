@@ -41,6 +41,7 @@ if ROOT not in sys.path:
 METRIC = "prefill tokens/s (48 Vheads x 128^2, T=32K) + % tensor peak; decode HBM GB/s"
 PREFILL = "prefill_t32768"
 DECODE = "decode_b256"
+CONV = "conv_prefill_b8_t8192"
 L2_BYTES = 126 * 2**20
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the two prefill
@@ -131,7 +132,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
         except (OSError, FileNotFoundError):
@@ -259,7 +260,7 @@ def config_dict(w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
@@ -268,6 +269,8 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=[PREFILL, "prefill_t4096"],
                     help="prefill workload to time (the small one is for profiler captures)")
     ap.add_argument("--decode-workload", default=DECODE, choices=[DECODE, "decode_b64"])
+    ap.add_argument("--conv-steps", type=int, default=5,
+                    help="timed calls of the conv + L2 workload (B=8, T=8192); 0 skips it")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -350,6 +353,11 @@ def main():
     if dw is not None:
         decode = run_decode(args, dw, dev, stream, barrier, pk, world)
 
+    # ---------------------------------------------------------------- conv + L2 load step
+    conv = None
+    if args.conv_steps > 0:
+        conv = run_conv(args, dev, stream, barrier, pk, world)
+
     # ---------------------------------------------------------------- end to end
     e2e = None
     if args.e2e_steps > 0:
@@ -374,6 +382,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
+            "conv_prefill": conv,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -415,6 +424,49 @@ def run_decode(args, dw, dev, stream, barrier, pk, world):
               "tokens_per_s": dw.B * world / (dms * 1e-3)}
     decode["gpu_launches"] = args.decode_steps
     return decode
+
+
+def run_conv(args, dev, stream, barrier, pk, world):
+    """The B=8, T=8192 workload with the depthwise causal conv on q, k, v and
+    the L2 norm of q, k fused into the load step (three launches per call)."""
+    import torch
+    from delta_rule_linear_gdn_b200 import gdn2
+    from delta_rule_linear_gdn_b200.inputs import make_inputs, workload
+    cw = workload(CONV)
+    rank = int(os.environ.get("RANK", "0"))
+    inp = make_inputs(cw, seed=rank_seed(rank), device=dev)
+    o = torch.empty((cw.B, cw.T, cw.H_v, cw.d), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((cw.B, cw.H_v, cw.d, cw.d), dtype=torch.float32, device=dev)
+    p = gdn2.make_params(cw.B, cw.T, cw.H_qk, cw.H_v, cw.d, cw.d, chunk=cw.chunk, l2norm_qk=True,
+                         conv_w=inp["conv_w"])
+    ws = torch.empty(max(gdn2.chunk_fwd_workspace(p), 1), dtype=torch.uint8, device=dev)
+
+    def call():
+        gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"], chunk=cw.chunk,
+                       conv_w=inp["conv_w"], l2norm_qk=True, o=o, S_T=S_T, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    torch.cuda.synchronize()
+    barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.conv_steps):
+            call()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    cms = max_over_ranks(c0.elapsed_time(c1) / args.conv_steps, dev)
+    nbytes = prefill_bytes(cw, s0=True)
+    gbs = nbytes / (cms * 1e-3) / 1e9
+    return {"workload": f"{cw.name}: B={cw.B} T={cw.T} H_qk={cw.H_qk} H_v={cw.H_v} d={cw.d} chunk={cw.chunk}, "
+                        f"depthwise causal conv k=4 on q,k,v and L2 norm of q,k in the load step, S0 given",
+            "ms_per_call": cms, "tokens_per_s": cw.B * cw.T * world / (cms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes},
+            "gpu_launches": 3 * args.conv_steps}
 
 
 def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):

@@ -106,6 +106,11 @@ constexpr int P_EB = 81920;
 constexpr int P_Z = 98304;
 constexpr int P_END = 114688;
 constexpr int P_AINV = 0;
+// level-2 inverse tiles (fp16, 128-byte rows), in the Gram operand space
+constexpr int P_L2I = 0;              // A11, MN-major B  (32 rows)
+constexpr int P_L2P = 4096;           // P = T21 A11, MN-major B (32 rows)
+constexpr int P_L2T = 8192;           // T21, K-major A (first 32 of 128 rows)
+constexpr int P_L2J = 12288;          // A22, K-major A (first 32 of 128 rows)
 constexpr int TS = 68;                // fp32 row stride of T and its inverse
 constexpr int P_T = P_GM;             // T   [64][68]
 constexpr int P_I = P_T + C * TS * 4; // inv [64][68]
@@ -117,6 +122,7 @@ constexpr int P_FLAG = P_TMEMP + 16;
 constexpr int P_SMEM = P_FLAG + 16;
 // prep TMEM columns
 constexpr uint32_t PT_GM = 0, PT_GB = 64, PT_YT = 128, PT_UW = 192, PT_COLS = 256;
+constexpr uint32_t PT_L2P = 0, PT_L2A = 64;   // level-2 inverse accumulators (after the Gram read-out)
 
 // ------------------------------------------------------------------ scan smem
 // Two stages (see the scan kernel for their layout), then:
@@ -559,29 +565,57 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       *reinterpret_cast<float2*>(sI + (r0 + ii) * TS + cc + jj) = make_float2(-a0, -a1);
     }
     __syncthreads();
-    // level 2: X_QP = −I_QQ T_QP I_PP (thread: row ii, 4 columns)
-    {
-      const int ii = tid >> 3, jp = (tid & 7) * 4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-      for (int l = 0; l < 32; ++l) {
-        const float t = sT[(32 + ii) * TS + l];
-        const float4 iv = *reinterpret_cast<const float4*>(sI + l * TS + jp);
-        acc.x += t * iv.x; acc.y += t * iv.y; acc.z += t * iv.z; acc.w += t * iv.w;
-      }
-      *reinterpret_cast<float4*>(sX + ii * 36 + jp) = acc;
+    // level 2 on the tensor cores: P = T21 A11, then A21 = −A22 P (32 × 32
+    // blocks, fp16 operands, fp32 accumulation). The tiles live in the Gram
+    // operand space, free since the Gram products: T21 and A22 are the first
+    // 32 rows of two K-major 128-row A operands (the rows after them only
+    // produce accumulator rows ≥ 32, which are not read), A11 and P are
+    // 32-row MN-major B operands (their columns ≥ 32 only produce accumulator
+    // columns ≥ 32).
+    for (int q = tid; q < 384; q += NP) {
+      const int t = q >> 7, r = (q >> 2) & 31, cb = (q & 3) * 8;
+      const float* src = t == 0 ? sT + (32 + r) * TS + cb : (t == 1 ? sI + r * TS + cb : sI + (32 + r) * TS + 32 + cb);
+      const float4 p0 = *reinterpret_cast<const float4*>(src);
+      const float4 p1 = *reinterpret_cast<const float4*>(src + 4);
+      const float x[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      st16(smem, (t == 0 ? P_L2T : (t == 1 ? P_L2I : P_L2J)) + sw_off(r, cb, BS_ROW64), pack8_f16(x));
     }
-    __syncthreads();
-    {
-      const int ii = tid >> 3, jp = (tid & 7) * 4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-      for (int l = 0; l < 32; ++l) {
-        const float t = sI[(32 + ii) * TS + 32 + l];
-        const float4 xv = *reinterpret_cast<const float4*>(sX + l * 36 + jp);
-        acc.x += t * xv.x; acc.y += t * xv.y; acc.z += t * xv.z; acc.w += t * xv.w;
-      }
-      *reinterpret_cast<float4*>(sI + (32 + ii) * TS + jp) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    sync_for_mma();
+    if (tid == 0) {
+      const uint64_t a1 = desc_k_sw(smem_u32(smem + P_L2T), 0, BS_ROW64);
+      const uint64_t b1 = desc_mn_sw(smem_u32(smem + P_L2I), 0, BS_ROW64);
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks)
+        mma16(tmem + PT_L2P, a1 + k_step_sw(ks, BS_ROW64), b1 + mn_step_sw(ks), idesc_f16(128, 64, false, true), ks > 0);
+      mma_commit(bar);
+    }
+    __syncwarp();
+    wait_mma(bar, phase, sflag);
+    if (lq == 0) {   // P rows 0..31: TMEM lanes 0..31 (warps 0 and 4, 16 columns each)
+      float v[16];
+      tmem_ld16(t_lane + PT_L2P + 16 * hc, v);
+      tmem_wait_ld();
+      st16(smem, P_L2P + sw_off(lane, 16 * hc, BS_ROW64), pack8_f16(v));
+      st16(smem, P_L2P + sw_off(lane, 16 * hc + 8, BS_ROW64), pack8_f16(v + 8));
+    }
+    sync_for_mma();
+    if (tid == 0) {
+      const uint64_t a2 = desc_k_sw(smem_u32(smem + P_L2J), 0, BS_ROW64);
+      const uint64_t b2 = desc_mn_sw(smem_u32(smem + P_L2P), 0, BS_ROW64);
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks)
+        mma16(tmem + PT_L2A, a2 + k_step_sw(ks, BS_ROW64), b2 + mn_step_sw(ks), idesc_f16(128, 64, false, true), ks > 0);
+      mma_commit(bar);
+    }
+    __syncwarp();
+    wait_mma(bar, phase, sflag);
+    if (lq == 0) {   // A21 = −(A22 P): rows 32..63 of A, columns 0..31
+      float v[16];
+      tmem_ld16(t_lane + PT_L2A + 16 * hc, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; u += 4)
+        *reinterpret_cast<float4*>(sI + (32 + lane) * TS + 16 * hc + u) = make_float4(-v[u], -v[u + 1], -v[u + 2], -v[u + 3]);
     }
     __syncthreads();
     // pack A (lower triangle; zeros above the diagonal), 16 entries per thread
@@ -971,9 +1005,9 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
 // which reduces the sum of squares.
 // =============================================================================
 constexpr int QP_THREADS = 256;
-constexpr int QP_TOK = 64;            // tokens per CTA
+constexpr int QP_TOK = 12;            // tokens per CTA; a thread's 3 + 12 input rows are loaded at once
 
-__global__ void __launch_bounds__(QP_THREADS) qkv_prep_kernel(ChunkArgs a, int t_begin, int Tseg, __half* qo,
+__global__ void __launch_bounds__(QP_THREADS, 2) qkv_prep_kernel(ChunkArgs a, int t_begin, int Tseg, __half* qo,
                                                               __half* ko, __half* vo) {
   const int groups = (2 * a.Hqk + a.Hv) * (D / 8);
   const int g = blockIdx.x * QP_THREADS + threadIdx.x;
@@ -989,40 +1023,37 @@ __global__ void __launch_bounds__(QP_THREADS) qkv_prep_kernel(ChunkArgs a, int t
   __half* dst = which == 0 ? qo : (which == 1 ? ko : vo);
   const bool conv = a.conv_w != nullptr;
   const bool norm = a.l2norm && which < 2;
+
+  const int tl0 = blockIdx.y * QP_TOK;                  // first token of this CTA, relative to t_begin
+  const int nt = min(QP_TOK, Tseg - tl0);
+  const size_t row = (size_t)H * D;                     // elements per token
+  const __nv_bfloat16* base = src + (size_t)bi * a.T * row + cw;
+  // rows t_begin + tl0 − 3 .. t_begin + tl0 + nt − 1 (zero before the sequence start)
+  uint4 raw[QP_TOK + 3];
+#pragma unroll
+  for (int r = 0; r < QP_TOK + 3; ++r) {
+    const int t = t_begin + tl0 - 3 + r;
+    const bool in = r < nt + 3 && t >= 0 && (conv || r >= 3);
+    raw[r] = in ? __ldg(reinterpret_cast<const uint4*>(base + (size_t)t * row)) : make_uint4(0, 0, 0, 0);
+  }
   float W[8][4];
 #pragma unroll
   for (int c = 0; c < 8; ++c)
 #pragma unroll
     for (int j = 0; j < 4; ++j) W[c][j] = conv ? __ldg(a.conv_w + (size_t)(ch + c) * 4 + j) : (j == 3 ? 1.f : 0.f);
 
-  const int tl0 = blockIdx.y * QP_TOK;                  // first token of this CTA, relative to t_begin
-  const int tl1 = min(tl0 + QP_TOK, Tseg);
-  const size_t row = (size_t)H * D;                     // elements per token
-  const __nv_bfloat16* base = src + (size_t)bi * a.T * row + cw;
-  auto load8 = [&](int t, float* x) {
-    if (t < 0) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) x[c] = 0.f;
-      return;
-    }
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + (size_t)t * row));
-    float lo[4], hi[4];
-    unpack4_bf16(make_uint2(u.x, u.y), lo);
-    unpack4_bf16(make_uint2(u.z, u.w), hi);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      x[c] = lo[c];
-      x[4 + c] = hi[c];
-    }
+  auto unpack8 = [](uint4 u, float* x) {
+    unpack4_bf16(make_uint2(u.x, u.y), x);
+    unpack4_bf16(make_uint2(u.z, u.w), x + 4);
   };
   float x3[8], x2[8], x1[8];                            // inputs of t−3, t−2, t−1
-  const int t_abs0 = t_begin + tl0;
-  load8(conv ? t_abs0 - 3 : -1, x3);
-  load8(conv ? t_abs0 - 2 : -1, x2);
-  load8(conv ? t_abs0 - 1 : -1, x1);
-  for (int tl = tl0; tl < tl1; ++tl) {
+  unpack8(raw[0], x3);
+  unpack8(raw[1], x2);
+  unpack8(raw[2], x1);
+#pragma unroll
+  for (int r = 0; r < QP_TOK; ++r) {
     float x0[8], y[8];
-    load8(t_begin + tl, x0);
+    unpack8(raw[r + 3], x0);
     float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -1036,7 +1067,7 @@ __global__ void __launch_bounds__(QP_THREADS) qkv_prep_kernel(ChunkArgs a, int t
 #pragma unroll
       for (int c = 0; c < 8; ++c) y[c] *= inv;
     }
-    *reinterpret_cast<uint4*>(dst + ((size_t)bi * Tseg + tl) * row + cw) = pack8_f16(y);
+    if (r < nt) *reinterpret_cast<uint4*>(dst + ((size_t)bi * Tseg + tl0 + r) * row + cw) = pack8_f16(y);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       x3[c] = x2[c];
