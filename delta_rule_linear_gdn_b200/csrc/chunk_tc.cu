@@ -1004,11 +1004,11 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
 // in registers; the 16 threads of one head's 128 channels are one half-warp,
 // which reduces the sum of squares.
 // =============================================================================
-constexpr int QP_THREADS = 256;
-constexpr int QP_TOK = 12;            // tokens per CTA; a thread's 3 + 12 input rows are loaded at once
+constexpr int QP_THREADS = 512;
+constexpr int QP_TOK = 64;            // tokens per CTA, in blocks of 8 rows loaded together
 
-__global__ void __launch_bounds__(QP_THREADS, 2) qkv_prep_kernel(ChunkArgs a, int t_begin, int Tseg, __half* qo,
-                                                              __half* ko, __half* vo) {
+__global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, int t_begin, int Tseg, __half* qo,
+                                                                 __half* ko, __half* vo) {
   const int groups = (2 * a.Hqk + a.Hv) * (D / 8);
   const int g = blockIdx.x * QP_THREADS + threadIdx.x;
   if (g >= groups) return;            // whole half-warps: groups is a multiple of 16
@@ -1024,55 +1024,68 @@ __global__ void __launch_bounds__(QP_THREADS, 2) qkv_prep_kernel(ChunkArgs a, in
   const bool conv = a.conv_w != nullptr;
   const bool norm = a.l2norm && which < 2;
 
+  float W[8][4];                      // taps of this thread's 8 channels (identity without the conv)
+  if (conv) {
+    const float4* wp = reinterpret_cast<const float4*>(a.conv_w + (size_t)ch * 4);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 t = __ldg(wp + c);
+      W[c][0] = t.x; W[c][1] = t.y; W[c][2] = t.z; W[c][3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) { W[c][0] = W[c][1] = W[c][2] = 0.f; W[c][3] = 1.f; }
+  }
   const int tl0 = blockIdx.y * QP_TOK;                  // first token of this CTA, relative to t_begin
   const int nt = min(QP_TOK, Tseg - tl0);
   const size_t row = (size_t)H * D;                     // elements per token
   const __nv_bfloat16* base = src + (size_t)bi * a.T * row + cw;
-  // rows t_begin + tl0 − 3 .. t_begin + tl0 + nt − 1 (zero before the sequence start)
-  uint4 raw[QP_TOK + 3];
-#pragma unroll
-  for (int r = 0; r < QP_TOK + 3; ++r) {
-    const int t = t_begin + tl0 - 3 + r;
-    const bool in = r < nt + 3 && t >= 0 && (conv || r >= 3);
-    raw[r] = in ? __ldg(reinterpret_cast<const uint4*>(base + (size_t)t * row)) : make_uint4(0, 0, 0, 0);
-  }
-  float W[8][4];
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) W[c][j] = conv ? __ldg(a.conv_w + (size_t)(ch + c) * 4 + j) : (j == 3 ? 1.f : 0.f);
-
+  auto load = [&](int tl) -> uint4 {                    // token t_begin + tl (zero outside the sequence / CTA)
+    const int t = t_begin + tl;
+    return (tl < tl0 + nt && t >= 0) ? __ldg(reinterpret_cast<const uint4*>(base + (size_t)t * row))
+                                     : make_uint4(0, 0, 0, 0);
+  };
   auto unpack8 = [](uint4 u, float* x) {
     unpack4_bf16(make_uint2(u.x, u.y), x);
     unpack4_bf16(make_uint2(u.z, u.w), x + 4);
   };
   float x3[8], x2[8], x1[8];                            // inputs of t−3, t−2, t−1
-  unpack8(raw[0], x3);
-  unpack8(raw[1], x2);
-  unpack8(raw[2], x1);
+  {
+    const uint4 h3 = conv ? load(tl0 - 3) : make_uint4(0, 0, 0, 0);
+    const uint4 h2 = conv ? load(tl0 - 2) : make_uint4(0, 0, 0, 0);
+    const uint4 h1 = conv ? load(tl0 - 1) : make_uint4(0, 0, 0, 0);
+    unpack8(h3, x3);
+    unpack8(h2, x2);
+    unpack8(h1, x1);
+  }
+  for (int b0 = 0; b0 < nt; b0 += 8) {
+    uint4 raw[8];
 #pragma unroll
-  for (int r = 0; r < QP_TOK; ++r) {
-    float x0[8], y[8];
-    unpack8(raw[r + 3], x0);
-    float ss = 0.f;
+    for (int r = 0; r < 8; ++r) raw[r] = load(tl0 + b0 + r);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      y[c] = W[c][0] * x3[c] + W[c][1] * x2[c] + W[c][2] * x1[c] + W[c][3] * x0[c];
-      ss += y[c] * y[c];
-    }
-    if (norm) {
+    for (int r = 0; r < 8; ++r) {
+      float x0[8], y[8];
+      unpack8(raw[r], x0);
+      float ss = 0.f;
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(hmask, ss, off);
-      const float inv = rsqrtf(ss + kL2Eps);
+      for (int c = 0; c < 8; ++c) {
+        y[c] = W[c][0] * x3[c] + W[c][1] * x2[c] + W[c][2] * x1[c] + W[c][3] * x0[c];
+        ss += y[c] * y[c];
+      }
+      if (norm) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) y[c] *= inv;
-    }
-    if (r < nt) *reinterpret_cast<uint4*>(dst + ((size_t)bi * Tseg + tl0 + r) * row + cw) = pack8_f16(y);
+        for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(hmask, ss, off);
+        const float inv = rsqrtf(ss + kL2Eps);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      x3[c] = x2[c];
-      x2[c] = x1[c];
-      x1[c] = x0[c];
+        for (int c = 0; c < 8; ++c) y[c] *= inv;
+      }
+      if (b0 + r < nt) *reinterpret_cast<uint4*>(dst + ((size_t)bi * Tseg + tl0 + b0 + r) * row + cw) = pack8_f16(y);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        x3[c] = x2[c];
+        x2[c] = x1[c];
+        x1[c] = x0[c];
+      }
     }
   }
 }
