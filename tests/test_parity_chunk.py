@@ -91,19 +91,22 @@ def test_bf16_d128_chunk64(gate_mode):
     torch.testing.assert_close(S16, S, rtol=0, atol=0)
 
 
-@pytest.mark.parametrize("conv", [True, False])
-def test_bf16_d128_conv_and_l2norm_tensor_core(conv):
+@pytest.mark.parametrize("conv,gate_mode", [(True, "full"), (False, "full"), (True, "kda"), (True, "gdn")])
+def test_bf16_d128_conv_and_l2norm_tensor_core(conv, gate_mode):
     """The load step (depthwise causal conv, L2 norm of q, k) ahead of the
     tensor-core prefill: two sequences with a ragged tail, so the conv history
-    crosses chunk boundaries but never sequence boundaries."""
+    crosses chunk boundaries but never sequence boundaries; all gate layouts."""
     w = small(T=200, B=2, H_qk=2, H_v=6, d=128, chunk=64, qkv="bf16", s0="normal", conv=True)
-    inp = make_inputs(w, seed=31)
+    inp = make_inputs(w, seed=31, gate_mode=gate_mode)
     if not conv:
         inp = dict(inp, conv_w=None)
-    o, S = run(inp, chunk=64, l2norm_qk=True, o_dtype=torch.float32)
-    o_ref, S_ref = oracle_chunk(inp, l2norm_qk=True)
+    o, S = run(inp, chunk=64, gate_mode=gate_mode, l2norm_qk=True, o_dtype=torch.float32)
+    o_ref, S_ref = oracle_chunk(inp, gate_mode=gate_mode, l2norm_qk=True)
     assert_close(o, o_ref, TOL_BF16, "o")
     assert_close(S, S_ref, TOL_BF16, "S_T")
+    o16, S16 = run(inp, chunk=64, gate_mode=gate_mode, l2norm_qk=True)
+    assert_bf16_rounding(o16, o, "o bf16")
+    torch.testing.assert_close(S16, S, rtol=0, atol=0)
 
 
 def test_empty_sequence_copies_state():
