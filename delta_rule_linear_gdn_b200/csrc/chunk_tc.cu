@@ -106,11 +106,15 @@ constexpr int P_EB = 81920;
 constexpr int P_Z = 98304;
 constexpr int P_END = 114688;
 constexpr int P_AINV = 0;
+constexpr int P_YS = P_GM;            // Yᵀ then U_wᵀ (16 KB each), staged for the bulk stores
+constexpr int P_AQS = 16384;          // −Aqk (8 KB) staged for its bulk store: in Gb's block 1,
+                                      // read only as don't-care rows by the level-2 products
 // level-2 inverse tiles (fp16, 128-byte rows), in the Gram operand space
 constexpr int P_L2I = 0;              // A11, MN-major B  (32 rows)
 constexpr int P_L2P = 4096;           // P = T21 A11, MN-major B (32 rows)
 constexpr int P_L2T = 8192;           // T21, K-major A (first 32 of 128 rows)
 constexpr int P_L2J = 12288;          // A22, K-major A (first 32 of 128 rows)
+static_assert(P_AQS >= P_L2J + 4096 && P_AQS + 8192 <= 32768, "staging of -Aqk clear of the level-2 tiles");
 constexpr int TS = 68;                // fp32 row stride of T and its inverse
 constexpr int P_T = P_GM;             // T   [64][68]
 constexpr int P_I = P_T + C * TS * 4; // inv [64][68]
@@ -348,6 +352,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       for (int off = 16; off > 0; off >>= 1) mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
       if (lane == 0) sred[warp] = mn;
     }
+    if (tid == 0) bulk_wait_read_all();   // the previous item's Yᵀ, U_wᵀ staging is read
     __syncthreads();
     bool gram_bf16;
     {
@@ -507,10 +512,15 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #pragma unroll
         for (int u = 0; u < 32; ++u) dm[u] = -dm[u];            // the scan adds −Aqk·U
 #pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(slot, SL_AQ + sw_off(i, j0 + cb, BS_ROW64), pack8_f16(dm + cb));
+        for (int cb = 0; cb < 32; cb += 8) st16(smem, P_AQS + sw_off(i, j0 + cb, BS_ROW64), pack8_f16(dm + cb));
       }
     }
+    fence_async_smem();
     __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(slot + SL_AQ, smem + P_AQS, 8192);   // −Aqk, byte for byte the slot's layout
+      bulk_commit();
+    }
 
     // -------- A = (I + T)⁻¹, blocked
     // level 0: the four 16 × 16 diagonal blocks by forward substitution, one
@@ -652,9 +662,11 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     __syncwarp();
     wait_mma(bar, phase, sflag);
     {
-      // warps 0..3: Yᵀ rows (key lanes); warps 4..7: U_wᵀ rows (dv lanes)
+      // warps 0..3: Yᵀ rows (key lanes); warps 4..7: U_wᵀ rows (dv lanes),
+      // staged in the (now free) Gram operand space and stored by two bulk
+      // copies, byte for byte the slot's layout
       const uint32_t col = hc == 0 ? PT_YT : PT_UW;
-      const int dst = hc == 0 ? SL_YT : SL_UW;
+      const int stg = P_YS + hc * 16384;
 #pragma unroll
       for (int cb0 = 0; cb0 < 64; cb0 += 32) {
         float v[32];
@@ -662,13 +674,20 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
         tmem_ld16(t_lane + col + cb0 + 16, v + 16);
         tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(slot, dst + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
+        for (int cb = 0; cb < 32; cb += 8) st16(smem, stg + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
       }
     }
+    fence_async_smem();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
+    if (tid == 0) {
+      bulk_s2g(slot + SL_YT, smem + P_YS, 16384);
+      bulk_s2g(slot + SL_UW, smem + P_YS + 16384, 16384);
+      bulk_commit();
+    }
   }
+  if (tid == 0) bulk_wait_all();      // the last item's copies
   if (*sflag && tid == 0) atomicOr(static_cast<int*>(a.workspace), 1);
   fence_before_sync();
   __syncthreads();

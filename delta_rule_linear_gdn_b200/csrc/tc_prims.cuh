@@ -224,6 +224,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       : "memory");
 }
 
+// Bulk (non-tensor) asynchronous copy shared → global of `bytes` (multiple of
+// 16, both addresses 16-byte aligned), tracked by the issuing thread's bulk
+// groups: commit, then wait until the source may be overwritten (.read) or
+// until the writes are done.
+__device__ __forceinline__ void bulk_s2g(void* dst_gmem, const void* src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst_gmem),
+               "r"(smem_u32(src_smem)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
 // Approximate reciprocal (the PTX rcp.approx.ftz.f32 instruction: at most
 // one ulp of error, subnormal inputs and results flushed to zero).
 __device__ __forceinline__ float rcp_approx(float x) {
