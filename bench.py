@@ -371,9 +371,12 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads, tokens = w.H_v, 8192
         rate, dt, used = cpu_oracle_rate(w, heads, tokens)
+        rate1, dt1, _ = cpu_oracle_rate(w, 1, tokens, threads=1)
         cpu = {"value": rate, "unit": "tokens/s", "cores": used, "kind": "oracle",
                "sample": f"{heads} V heads x {tokens} tokens of the T={w.T} layer workload "
-                         f"({dt:.1f} s, layer tokens = tokens x heads/{w.H_v})"}
+                         f"({dt:.1f} s, layer tokens = tokens x heads/{w.H_v})",
+               "single_core_value": rate1,
+               "single_core_sample": f"1 V head x {tokens} tokens on one thread ({dt1:.1f} s)"}
 
     clocks = clk.summary()
     if world > 1:
