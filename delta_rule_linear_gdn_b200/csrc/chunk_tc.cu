@@ -400,61 +400,61 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       }
     }
 
-    // -------- pass 2: key-side operand tiles, tile by tile per token
+    // -------- pass 2: key-side operand tiles, tile by tile per token; one
+    // copy of the loop per Gram operand type, so each packs only its own
     uint32_t qpk[4][4];
     float qlo[4];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (u == 4) load_key(4);
-      const int uk = u & 3;
-      const uint32_t i128 = (uint32_t)(i0 + u) * 128;
-      const uint32_t p64 = i128 + piece(u, BS_ROW64), p128 = i128 + piece(u, BS_ROW128);
-      float kx[4], qx[4], e[4], rf[4], g[4], fe[4];
-      unpack4_in<F16IN>(kk[uk], kx);
-      unpack4_in<F16IN>(qq[uk], qx);
-      e[0] = bq[uk].x * kx[0]; e[1] = bq[uk].y * kx[1]; e[2] = bq[uk].z * kx[2]; e[3] = bq[uk].w * kx[3];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        rf[c] = rcp_approx(f[u][c]);
-        g[c] = pre[c] * f[u][c];
-        fe[c] = se[c] * f[u][c];
-      }
-      float o[4];
 #define GDN2_TILE(dst, off, expr)                                             \
   {                                                                           \
     _Pragma("unroll") for (int c = 0; c < 4; ++c) o[c] = (expr);              \
     st8(dst, off, pack4_f16(o[0], o[1], o[2], o[3]));                         \
   }
-#define GDN2_GRAM_TILE(dst, off, expr)                                        \
+#define GDN2_GRAM_TILE(dst, off, expr, BF)                                    \
   {                                                                           \
     _Pragma("unroll") for (int c = 0; c < 4; ++c) o[c] = (expr);              \
-    if (gram_bf16)                                                            \
-      st8(dst, off, pack4_bf16(o[0], o[1], o[2], o[3]));                      \
-    else                                                                      \
-      st8(dst, off, pack4_f16(o[0], o[1], o[2], o[3]));                       \
+    st8(dst, off, (BF) ? pack4_bf16(o[0], o[1], o[2], o[3]) : pack4_f16(o[0], o[1], o[2], o[3])); \
   }
-      // Q̄ᵀ: each key's token pairs packed as they are produced
-      if ((u & 1) == 0) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) qlo[c] = qx[c] * g[c];
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) qpk[c][u >> 1] = pack2_f16(qlo[c], qx[c] * g[c]);
-      }
-      GDN2_TILE(slot, SL_KE + p64, kx[c] * (ps[c] * rf[c]))
-      GDN2_TILE(smem, P_EB + p64, e[c] * g[c])
-      GDN2_GRAM_TILE(smem, P_GM + p128, e[c] * fe[c])
-      GDN2_GRAM_TILE(smem, P_GM + 64 * 128 + p128, qx[c] * fe[c])
-      GDN2_GRAM_TILE(smem, P_KM + p64, kx[c] * (sk[c] * rf[c]))
-      if (qt >= 2) {
-        GDN2_GRAM_TILE(smem, P_GB + p128, e[c] * (sx[c] * f[u][c]))
-        GDN2_GRAM_TILE(smem, P_GB + 64 * 128 + p128, qx[c] * (sx[c] * f[u][c]))
-      } else {
-        GDN2_GRAM_TILE(smem, P_KB + p128, kx[c] * (sx[c] * rf[c]))
-      }
-#undef GDN2_TILE
-#undef GDN2_GRAM_TILE
+#define GDN2_PASS2(BF)                                                                          \
+  _Pragma("unroll") for (int u = 0; u < 8; ++u) {                                               \
+    if (u == 4) load_key(4);                                                                    \
+    const int uk = u & 3;                                                                       \
+    const uint32_t i128 = (uint32_t)(i0 + u) * 128;                                             \
+    const uint32_t p64 = i128 + piece(u, BS_ROW64), p128 = i128 + piece(u, BS_ROW128);          \
+    float kx[4], qx[4], e[4], rf[4], g[4], fe[4], o[4];                                         \
+    unpack4_in<F16IN>(kk[uk], kx);                                                              \
+    unpack4_in<F16IN>(qq[uk], qx);                                                              \
+    e[0] = bq[uk].x * kx[0]; e[1] = bq[uk].y * kx[1]; e[2] = bq[uk].z * kx[2]; e[3] = bq[uk].w * kx[3]; \
+    _Pragma("unroll") for (int c = 0; c < 4; ++c) {                                             \
+      rf[c] = rcp_approx(f[u][c]);                                                              \
+      g[c] = pre[c] * f[u][c];                                                                  \
+      fe[c] = se[c] * f[u][c];                                                                  \
+    }                                                                                           \
+    /* Q̄ᵀ: each key's token pairs packed as they are produced */                              \
+    if ((u & 1) == 0) {                                                                         \
+      _Pragma("unroll") for (int c = 0; c < 4; ++c) qlo[c] = qx[c] * g[c];                     \
+    } else {                                                                                    \
+      _Pragma("unroll") for (int c = 0; c < 4; ++c) qpk[c][u >> 1] = pack2_f16(qlo[c], qx[c] * g[c]); \
+    }                                                                                           \
+    GDN2_TILE(slot, SL_KE + p64, kx[c] * (ps[c] * rf[c]))                                       \
+    GDN2_TILE(smem, P_EB + p64, e[c] * g[c])                                                    \
+    GDN2_GRAM_TILE(smem, P_GM + p128, e[c] * fe[c], BF)                                         \
+    GDN2_GRAM_TILE(smem, P_GM + 64 * 128 + p128, qx[c] * fe[c], BF)                             \
+    GDN2_GRAM_TILE(smem, P_KM + p64, kx[c] * (sk[c] * rf[c]), BF)                               \
+    if (qt >= 2) {                                                                              \
+      GDN2_GRAM_TILE(smem, P_GB + p128, e[c] * (sx[c] * f[u][c]), BF)                           \
+      GDN2_GRAM_TILE(smem, P_GB + 64 * 128 + p128, qx[c] * (sx[c] * f[u][c]), BF)               \
+    } else {                                                                                    \
+      GDN2_GRAM_TILE(smem, P_KB + p128, kx[c] * (sx[c] * rf[c]), BF)                            \
+    }                                                                                           \
+  }
+    if (gram_bf16) {
+      GDN2_PASS2(true)
+    } else {
+      GDN2_PASS2(false)
     }
+#undef GDN2_PASS2
+#undef GDN2_GRAM_TILE
+#undef GDN2_TILE
     // Q̄ᵀ [key][tok]: the thread's 8 tokens of each of its keys form one 16-byte chunk
 #pragma unroll
     for (int c = 0; c < 4; ++c)
