@@ -50,9 +50,9 @@ L2_BYTES = 126 * 2**20
 # the kernel sources it was taken on; with other sources the figure is stale
 # and the bench reports null.
 TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
-TRAFFIC = {"sha1": "a7065507281ee5004884522d91b4a4a89310a89e",
-           # (387.1 + 191.1 + 228.1 + 36.3) MB at T=4096, times 8
-           "bytes_per_call": 6_741_000_192,
+TRAFFIC = {"sha1": "1363a36cfe9b7a5c1ec8a2a42e9c8fa3656ec197",
+           # (386.1 + 191.7 + 228.1 + 37.6) MB at T=4096, times 8
+           "bytes_per_call": 6_747_873_280,
            "profile": "profiles/chunk_prep_scan_t4096_ncu.md"}
 
 
