@@ -263,75 +263,46 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   const PrepSrc src{a.alpha, a.b, full ? a.w : a.b, static_cast<const uint16_t*>(a.k),
                     static_cast<const uint16_t*>(a.q), static_cast<const uint16_t*>(a.v)};
 
+  // Input schedule of an item: α of the thread's 8 tokens and the key side
+  // (b, k, q) of tokens 0..3 first; the key side of token u + 4 as soon as
+  // token u is packed (its registers are free); w and v after pass 2, their
+  // latency covered by the Gram products. (Requesting the next item's inputs
+  // earlier than this needs registers the 2-CTA/SM budget does not have.)
+  float f[8][4];                   // α, then its forward products within the quarter
+  float4 bq[4];
+  uint2 kk[4], qq[4];
+  auto gate_row = [&](const Item& it, int u) -> size_t {
+    return ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hv + it.h;
+  };
+  auto qkv_tok = [&](const Item& it, int u) -> size_t {
+    return (size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i0 + u;
+  };
+  auto load_key1 = [&](const Item& it, int u, int s) {
+    const bool ok = it.Lc == C || i0 + u < it.Lc;
+    const size_t tq = qkv_tok(it, u) * a.Hqk + it.hq;
+    bq[s] = ok ? gate4(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+    kk[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
+    qq[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
+  };
+  auto load_alpha_key0 = [&](int item_) {
+    const Item it = decode_item(a, c_begin, item_);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const bool ok = it.Lc == C || i0 + u < it.Lc;
+      const float4 al = ok ? gate4(src.alpha, gate_row(it, u), c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
+      f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) load_key1(it, u, u);
+  };
+
   uint32_t phase = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const Item it = decode_item(a, c_begin, item);
     uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)it.bh * n_seg + it.cl) * SLOT;
-    const size_t tok0 = (size_t)it.bi * a.T + it.t0 + i0;    // gate row of u = 0
-    const size_t qtok0 = (size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i0;   // q, k, v row of u = 0
+    load_alpha_key0(item);
 
-    // -------- pass 1: the write side Z = w ⊙ v (no decay) straight to its
-    // tile; α's forward products within the quarter. The key-side inputs of
-    // tokens u = 0..3 are requested here, those of u = 4..7 in pass 2.
-    float f[8][4];
-    float4 bq[4];
-    uint2 kk[4], qq[4];
-    const bool whole = it.Lc == C;              // every chunk but a sequence's last
-    auto load_key = [&](int u0) {
-      if (whole) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const size_t gt = (tok0 + u0 + u) * a.Hv + it.h;
-          const size_t tq = (qtok0 + u0 + u) * a.Hqk + it.hq;
-          bq[u] = gate4(src.b, gt, c0, full);
-          kk[u] = __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0));
-          qq[u] = __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0));
-        }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const bool ok = i0 + u0 + u < it.Lc;
-          const size_t gt = (tok0 + u0 + u) * a.Hv + it.h;
-          const size_t tq = (qtok0 + u0 + u) * a.Hqk + it.hq;
-          bq[u] = ok ? gate4(src.b, gt, c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
-          kk[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
-          qq[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
-        }
-      }
-    };
-    {
-      float4 wv[8];
-      uint2 vv[8];
-      if (whole) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const size_t gt = (tok0 + u) * a.Hv + it.h;
-          const float4 al = gate4(src.alpha, gt, c0, alpha_pc);
-          f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
-          wv[u] = gate4(src.w, gt, c0, full);
-          vv[u] = __ldg(reinterpret_cast<const uint2*>(src.v + ((qtok0 + u) * a.Hv + it.h) * D + c0));
-        }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const bool ok = i0 + u < it.Lc;
-          const size_t gt = (tok0 + u) * a.Hv + it.h;
-          const float4 al = ok ? gate4(src.alpha, gt, c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
-          f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
-          wv[u] = ok ? gate4(src.w, gt, c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
-          vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + ((qtok0 + u) * a.Hv + it.h) * D + c0))
-                     : make_uint2(0, 0);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float vx[4];
-        unpack4_in<F16IN>(vv[u], vx);
-        st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
-            pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
-      }
-    }
-    load_key(0);
+    // -------- pass 1: α's forward products within the quarter
     {
       // within the thread's 8 tokens, then across the two token groups of the
       // quarter (lanes l and l + 16)
@@ -373,8 +344,11 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     //   half), f_i and 1 / f_i (second quarter);
     //   half-boundary factors: P_2 f_i (quarter 3), f_i (quarter 2) for rows
     //   of the second half; P_qt P_1 / f_i (quarter 0), P_qt / f_i (quarter 1)
-    //   for keys of the first half.
-    float pre[4], ps[4], se[4], sk[4], sx[4];
+    //   for keys of the first half. In every quarter these are the
+    //   mid-reference factor times one constant: P_2 for rows (quarters 2,
+    //   3), P_1 for keys (quarters 0, 1); likewise the K_end factor is the
+    //   key's mid-reference factor times suf (even quarter) or P_qt · suf (odd).
+    float pre[4], se[4], sk[4], ke[4], xb[4];
     {
       float P[4][4];
 #pragma unroll
@@ -392,11 +366,11 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           if (m == qt) own = P[m][c];
         }
         pre[c] = pr;
-        ps[c] = own * su;
         const bool even = (qt & 1) == 0;
         se[c] = even ? rcp_approx(own) : 1.f;
         sk[c] = even ? own : 1.f;
-        sx[c] = qt == 3 ? P[2][c] : (qt == 2 ? 1.f : (qt == 0 ? own * P[1][c] : own));
+        ke[c] = even ? su : own * su;            // K_end row = K̃_mid row · ke
+        xb[c] = qt >= 2 ? P[2][c] : P[1][c];     // boundary row = mid row · xb
       }
     }
 
@@ -416,7 +390,6 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   }
 #define GDN2_PASS2(BF)                                                                          \
   _Pragma("unroll") for (int u = 0; u < 8; ++u) {                                               \
-    if (u == 4) load_key(4);                                                                    \
     const int uk = u & 3;                                                                       \
     const uint32_t i128 = (uint32_t)(i0 + u) * 128;                                             \
     const uint32_t p64 = i128 + piece(u, BS_ROW64), p128 = i128 + piece(u, BS_ROW128);          \
@@ -435,17 +408,24 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     } else {                                                                                    \
       _Pragma("unroll") for (int c = 0; c < 4; ++c) qpk[c][u >> 1] = pack2_f16(qlo[c], qx[c] * g[c]); \
     }                                                                                           \
-    GDN2_TILE(slot, SL_KE + p64, kx[c] * (ps[c] * rf[c]))                                       \
-    GDN2_TILE(smem, P_EB + p64, e[c] * g[c])                                                    \
-    GDN2_GRAM_TILE(smem, P_GM + p128, e[c] * fe[c], BF)                                         \
-    GDN2_GRAM_TILE(smem, P_GM + 64 * 128 + p128, qx[c] * fe[c], BF)                             \
-    GDN2_GRAM_TILE(smem, P_KM + p64, kx[c] * (sk[c] * rf[c]), BF)                               \
-    if (qt >= 2) {                                                                              \
-      GDN2_GRAM_TILE(smem, P_GB + p128, e[c] * (sx[c] * f[u][c]), BF)                           \
-      GDN2_GRAM_TILE(smem, P_GB + 64 * 128 + p128, qx[c] * (sx[c] * f[u][c]), BF)               \
-    } else {                                                                                    \
-      GDN2_GRAM_TILE(smem, P_KB + p128, kx[c] * (sx[c] * rf[c]), BF)                            \
+    float km[4], gme[4], gmq[4];                                                                \
+    _Pragma("unroll") for (int c = 0; c < 4; ++c) {                                             \
+      km[c] = kx[c] * (sk[c] * rf[c]);                                                          \
+      gme[c] = e[c] * fe[c];                                                                    \
+      gmq[c] = qx[c] * fe[c];                                                                   \
     }                                                                                           \
+    GDN2_TILE(slot, SL_KE + p64, km[c] * ke[c])                                                 \
+    GDN2_TILE(smem, P_EB + p64, e[c] * g[c])                                                    \
+    GDN2_GRAM_TILE(smem, P_GM + p128, gme[c], BF)                                               \
+    GDN2_GRAM_TILE(smem, P_GM + 64 * 128 + p128, gmq[c], BF)                                    \
+    GDN2_GRAM_TILE(smem, P_KM + p64, km[c], BF)                                                 \
+    if (qt >= 2) {                                                                              \
+      GDN2_GRAM_TILE(smem, P_GB + p128, gme[c] * xb[c], BF)                                     \
+      GDN2_GRAM_TILE(smem, P_GB + 64 * 128 + p128, gmq[c] * xb[c], BF)                          \
+    } else {                                                                                    \
+      GDN2_GRAM_TILE(smem, P_KB + p128, km[c] * xb[c], BF)                                      \
+    }                                                                                           \
+    if (u < 4) load_key1(it, u + 4, u);                                                         \
   }
     if (gram_bf16) {
       GDN2_PASS2(true)
@@ -455,6 +435,16 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #undef GDN2_PASS2
 #undef GDN2_GRAM_TILE
 #undef GDN2_TILE
+    // the write side, consumed after the Gram products
+    float4 wv[8];
+    uint2 vv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const bool ok = it.Lc == C || i0 + u < it.Lc;
+      wv[u] = ok ? gate4(src.w, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+      vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
+                 : make_uint2(0, 0);
+    }
     // Q̄ᵀ [key][tok]: the thread's 8 tokens of each of its keys form one 16-byte chunk
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -478,6 +468,14 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       mma_commit(bar);
     }
     __syncwarp();
+    // Z = w ⊙ v (no decay) to its tile, read by the Y/U_w products
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      float vx[4];
+      unpack4_in<F16IN>(vv[u], vx);
+      st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
+          pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
+    }
     wait_mma(bar, phase, sflag);
 
     // -------- T (fp32, shared) and Aqk (fp16, workspace) from TMEM. Lanes
@@ -521,6 +519,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       bulk_s2g(slot + SL_AQ, smem + P_AQS, 8192);   // −Aqk, byte for byte the slot's layout
       bulk_commit();
     }
+
 
     // -------- A = (I + T)⁻¹, blocked
     // level 0: the four 16 × 16 diagonal blocks by forward substitution, one
