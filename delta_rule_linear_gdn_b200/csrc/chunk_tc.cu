@@ -478,39 +478,31 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
     wait_mma(bar, phase, sflag);
 
-    // -------- T (fp32, shared) and Aqk (fp16, workspace) from TMEM. Lanes
+    // -------- T (fp32, shared) and −Aqk (fp16, staged) from TMEM. Lanes
     // 0..63 hold rows of T, lanes 64..127 rows of Aqk; the two warps of a lane
-    // quarter take 32 columns each (only columns < 32 need the half-boundary
-    // product: a row i ≥ 32 against a key j < 32).
+    // quarter take 32 columns each. Every case is warp-uniform: a row i ≥ 32
+    // against keys j < 32 takes the half-boundary product, the other pairs
+    // the mid-reference product. The inverse reads only the strictly lower
+    // part of T, so T is stored unmasked; Aqk is masked to j ≤ i.
     {
-      const bool is_t = row < 64;
       const int i = row & 63;
       const int j0 = 32 * hc;
-      float dm[32], db[32];
-      tmem_ld16(t_lane + PT_GM + j0, dm);
-      tmem_ld16(t_lane + PT_GM + j0 + 16, dm + 16);
-      if (hc == 0) {
-        tmem_ld16(t_lane + PT_GB, db);
-        tmem_ld16(t_lane + PT_GB + 16, db + 16);
-      }
+      const bool bnd = hc == 0 && i >= 32;
+      const uint32_t col = bnd ? PT_GB : PT_GM + j0;
+      float d[32];
+      tmem_ld16(t_lane + col, d);
+      tmem_ld16(t_lane + col + 16, d + 16);
       tmem_wait_ld();
-#pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        const int j = j0 + u;
-        const bool keep = is_t ? (j < i) : (j <= i);
-        const bool same = (j >> 5) == (i >> 5);
-        const float x = same ? dm[u] : (hc == 0 ? db[u] : 0.f);
-        dm[u] = keep ? x : 0.f;
-      }
-      if (is_t) {
+      if (row < 64) {
 #pragma unroll
         for (int u = 0; u < 32; u += 4)
-          *reinterpret_cast<float4*>(sT + i * TS + j0 + u) = make_float4(dm[u], dm[u + 1], dm[u + 2], dm[u + 3]);
+          *reinterpret_cast<float4*>(sT + i * TS + j0 + u) = make_float4(d[u], d[u + 1], d[u + 2], d[u + 3]);
       } else {
+        const int li = bnd ? 31 : (hc == 1 && i < 32 ? -1 : (i & 31));   // keep column u ≤ li
 #pragma unroll
-        for (int u = 0; u < 32; ++u) dm[u] = -dm[u];            // the scan adds −Aqk·U
+        for (int u = 0; u < 32; ++u) d[u] = u <= li ? -d[u] : 0.f;
 #pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(smem, P_AQS + sw_off(i, j0 + cb, BS_ROW64), pack8_f16(dm + cb));
+        for (int cb = 0; cb < 32; cb += 8) st16(smem, P_AQS + sw_off(i, j0 + cb, BS_ROW64), pack8_f16(d + cb));
       }
     }
     fence_async_smem();
@@ -747,7 +739,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   uint64_t* b_d = bars + 2;             // Z(−S) + [I;0]U_w done (U and −Q̄S in D)
   uint64_t* b_u = bars + 3;             // U written (fp16)
   uint64_t* b_s = bars + 4;             // state update done
-  uint64_t* b_sh = bars + 5;            // fp16 −S written and TMEM scaled
+  uint64_t* b_sh = bars + 5;            // fp16 −S written (one arrival per epilogue warp)
   uint64_t* b_o = bars + 6;             // [2] D buffer holds the chunk's −O
   uint64_t* b_of = bars + 8;            // [2] D buffer read out
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + S_TMEMP);
@@ -762,7 +754,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   TOut* og = static_cast<TOut*>(a.o);
 
   if (tid == 0) {
-    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], &bars[i] == b_sh ? 8 : 1);   // b_sh: one per epilogue warp
     fence_mbar_init();
     sflag[0] = 0;
     sflag[1] = 0;
@@ -771,6 +763,18 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   if (warp == 0) {
     tmem_alloc(tmem_ptr, ST_COLS);
     tmem_relinquish();
+  }
+  if (warp < 8) {
+    // constant [I_64; 0] (128 rows × 64 columns), in place before any product
+    const int r = (warp & 3) * 32 + lane, cq = (warp >> 2) * 32;
+#pragma unroll
+    for (int cb = 0; cb < 32; cb += 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = (r == cq + cb + u) ? 1.f : 0.f;
+      st16(smem, S_I + sw_off(r, cq + cb, BS_ROW128), pack8_f16(x));
+    }
+    fence_async_smem();
   }
   fence_before_sync();
   __syncthreads();
@@ -870,17 +874,8 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       fence_after_sync();
     };
 
-    // Constant [I_64; 0] (rows × 64 columns) and the entry state: fp16 −S for
-    // the first chunk's products, TMEM ← S · Γ of the first chunk.
-    {
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) {
-        float x[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = (row == c0 + cb + u) ? 1.f : 0.f;
-        st16(smem, S_I + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(x));
-      }
-    }
+    // The entry state: fp16 −S for the first chunk's products, TMEM ← S · Γ
+    // of the first chunk.
     wait(&full[0], 0);
     {
       const float g = reinterpret_cast<const float*>(smem + SG_GC)[row];
@@ -904,8 +899,8 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
     }
     fence_async_smem();
     fence_before_sync();
-    epi_sync();
-    if (tid == 0) mbar_arrive(b_sh);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_sh);
 
     // Outputs of chunk cc from D buffer `db`: row 64 + i of D is token i; this
     // thread writes 32 contiguous d_v values of it.
@@ -966,6 +961,11 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
           for (int u = 0; u < 32; ++u) n[u] = -v[u];
 #pragma unroll
           for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(n + cb));
+          // publish this warp's part of −S at once: the next products need
+          // only that; the TMEM state is scaled while they run
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_sh);
           const float g = reinterpret_cast<const float*>(smem + (s ^ 1) * STAGE + SG_GC)[row];
 #pragma unroll
           for (int u = 0; u < 32; ++u) v[u] *= g;
@@ -978,20 +978,18 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
           for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(ST + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
         }
       }
-      // One barrier per chunk publishes the state and carries the stop
-      // decision: thread 0 samples the error flag just before it, every thread
-      // reads the sample just after it (a flag raised later is seen one chunk
-      // later; the waits in between return at once).
+      // One barrier per chunk orders the scaled TMEM state before the next
+      // state update (issued after U, which the U warps publish only after
+      // this barrier) and carries the stop decision: thread 0 samples the
+      // error flag just before it, every thread reads the sample just after it
+      // (a flag raised later is seen one chunk later; the waits in between
+      // return at once).
       if (!ok) atomicOr(sflag, 1);
-      if (more) {
-        fence_async_smem();
-        fence_before_sync();
-      }
+      if (more) fence_before_sync();
       // (two sample slots: slot c & 1 is rewritten only in chunk c + 2, after
       // every thread has passed the barrier of chunk c + 1)
       if (tid == 0) estop[c & 1] = *vflag;
       epi_sync();
-      if (more && tid == 0) mbar_arrive(b_sh);
       if (estop[c & 1] != 0) {
         ok = false;
         stopped = true;
