@@ -50,9 +50,9 @@ L2_BYTES = 126 * 2**20
 # the kernel sources it was taken on; with other sources the figure is stale
 # and the bench reports null.
 TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
-TRAFFIC = {"sha1": "1363a36cfe9b7a5c1ec8a2a42e9c8fa3656ec197",
-           # (386.1 + 191.7 + 228.1 + 37.6) MB at T=4096, times 8
-           "bytes_per_call": 6_747_873_280,
+TRAFFIC = {"sha1": "16d0da025ec8024f6807e720aaefae0131bd2e8b",
+           # (385.97 + 193.10 + 228.10 + 34.44) MB at T=4096, times 8
+           "bytes_per_call": 6_732_920_832,
            "profile": "profiles/chunk_prep_scan_t4096_ncu.md"}
 
 
@@ -119,25 +119,68 @@ def measured_traffic():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a timed region."""
+    """SM clock and throttle-reason samples during a timed region, read through
+    NVML every 5 ms (falls back to `nvidia-smi -lms 50` without the NVML
+    bindings). Reads only; no setting of the GPU is touched."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
         self.proc = None
         self.lines = []
+        self.sm = []
+        self.mx = None
+        self.reasons = set()
         self._t = None
+        self._stop = threading.Event()
+        self._nvml = None
+
+    def _nvml_loop(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                bits = int(get_reasons(h))
+                for name, bit in self.REASON_BITS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.005)
 
     def __enter__(self):
         try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            idx = torch.cuda._get_nvml_device_index(self.cuda_index)
+            h = nv.nvmlDeviceGetHandleByIndex(idx)
+            self.mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self._nvml = nv
+            self._t = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self._t.start()
+            return self
+        except Exception:
+            self._nvml = None
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", f"--id={self.cuda_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
+            # nvidia-smi takes a while to print its first sample: the timed
+            # region starts only once it samples (bounded wait)
+            t_end = time.time() + 5.0
+            while not self.lines and time.time() < t_end and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.lines.clear()
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -147,17 +190,23 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            if self._t is not None:
-                self._t.join(timeout=2)
+        if self._t is not None:
+            self._t.join(timeout=2)
+        if self._nvml is not None:
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons = list(self.sm), self.mx, set(self.reasons)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
@@ -172,9 +221,9 @@ class ClockSampler:
                 if val.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
 # ------------------------------------------------------------------ reference arm
