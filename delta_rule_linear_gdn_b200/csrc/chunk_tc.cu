@@ -214,8 +214,22 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int
   return it;
 }
 
+// Where the slots of a launch live: chunk c_begin + j of sequence-head bh is
+// slot bh · stride + off + j of the workspace (stride: slots per
+// sequence-head in the workspace; off: the launch's first chunk there).
+struct SlotMap {
+  int stride, off;
+};
+__device__ __forceinline__ size_t slot_index(SlotMap m, int bh, int j) {
+  return (size_t)bh * m.stride + m.off + j;
+}
+
+// Items are taken in order (chunk-major, value head fastest): by a fixed stride
+// of the grid, or, with `counter`, one at a time from that device counter
+// (zero before the launch), so that CTAs which start late take fewer.
 template <bool F16IN>
-__global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg) {
+__global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
+                                                           int* counter) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + P_BAR);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + P_TMEMP);
@@ -226,12 +240,15 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   float* sI = reinterpret_cast<float*>(smem + P_I);
   float* sX = reinterpret_cast<float*>(smem + P_X);
 
+  int* s_item = sflag + 1;               // the next item, when taken from the counter
+
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_items = a.B * a.Hv * n_seg;
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
     *sflag = 0;
+    *s_item = counter ? atomicAdd(counter, 1) : 0;
   }
   if (warp == 0) {
     tmem_alloc(tmem_ptr, PT_COLS);
@@ -297,9 +314,9 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   };
 
   uint32_t phase = 0;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+  for (int item = counter ? *s_item : (int)blockIdx.x; item < n_items;) {
     const Item it = decode_item(a, c_begin, item);
-    uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + ((size_t)it.bh * n_seg + it.cl) * SLOT;
+    uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + slot_index(sm, it.bh, it.cl) * SLOT;
     load_alpha_key0(item);
 
     // -------- pass 1: α's forward products within the quarter
@@ -325,6 +342,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
     if (tid == 0) bulk_wait_read_all();   // the previous item's Yᵀ, U_wᵀ staging is read
     __syncthreads();
+    // every thread has read s_item for this item (at the end of the previous one)
+    if (counter && tid == 0) *s_item = atomicAdd(counter, 1);
     bool gram_bf16;
     {
       float mall = sred[0];
@@ -677,12 +696,17 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       bulk_s2g(slot + SL_UW, smem + P_YS + 16384, 16384);
       bulk_commit();
     }
+    item = counter ? *s_item : item + (int)gridDim.x;   // written before the barriers above
   }
   if (tid == 0) bulk_wait_all();      // the last item's copies
   if (*sflag && tid == 0) atomicOr(static_cast<int*>(a.workspace), 1);
   fence_before_sync();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, PT_COLS);
+  // Launched beside the previous segment's scan, this grid completes only
+  // after it: the next scan, ordered after this grid, then also follows that
+  // scan (whose final state it reads).
+  griddep_wait();
 }
 
 // =============================================================================
@@ -731,8 +755,8 @@ __device__ __forceinline__ void u_sync() { asm volatile("bar.sync 2, 128;\n" :::
 __device__ __forceinline__ void o_sync() { asm volatile("bar.sync 3, 128;\n" ::: "memory"); }
 
 template <typename TOut>
-__global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, const float* S_in,
-                                                           float* S_out) {
+__global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
+                                                           const float* S_in, float* S_out) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_BAR);
   uint64_t* full = bars;                // [2] stage s loaded
@@ -749,8 +773,11 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x >> 1, half = blockIdx.x & 1;
+  // resident: the next segment's prep, launched as a programmatic dependent,
+  // may take the SMs this grid leaves free
+  griddep_launch_dependents();
   const int h = bh % a.Hv, bi = bh / a.Hv;
-  const uint8_t* slots = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + (size_t)bh * n_seg * SLOT;
+  const uint8_t* slots = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + slot_index(sm, bh, 0) * SLOT;
   TOut* og = static_cast<TOut*>(a.o);
 
   if (tid == 0) {
@@ -1138,16 +1165,47 @@ size_t chunk_tc_min_workspace(const ChunkArgs& a, bool carry_state) {
   return WS_HEAD + bytes_per_chunk(a) + (carry_state ? state_bytes(a) : 0);
 }
 
+namespace {
+// The scan of segment k and the prep of segment k + 1 overlap when the scan
+// leaves SMs idle (fewer (sequence, V head, half) chains than SMs) and the
+// workspace holds every chunk's slot: the prep is launched as a programmatic
+// dependent of the scan, so it starts once the scan's CTAs are resident and
+// takes the SMs they leave free (items from a counter, so that CTAs which start
+// only when the scan ends take fewer); it does not complete before the scan.
+constexpr int OVERLAP_SEGMENTS = 4;     // segments of an overlapped call
+constexpr int OVERLAP_MIN_CHUNKS = 32;  // per segment
+constexpr int OVERLAP_LAST_MIN = 16;    // chunks of the last segment, at least
+constexpr int MAX_COUNTERS = (int)(WS_HEAD / sizeof(int)) - 1;   // item counters after the status word
+
+template <typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Args...), int grid, int block, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+}  // namespace
+
 // Runs the chunks in segments when the workspace holds fewer chunks than the
 // sequence has; the state is carried between segments through S_T (or, when
-// S_T is NULL, through the end of the workspace). Workspace: status word,
-// slots [B·H_v][seg], preprocessed q|k|v of seg·C tokens (conv / L2 only),
-// carried state (only when needed).
+// S_T is NULL, through the end of the workspace). Workspace: status word and
+// item counters (256 bytes), slots [B·H_v][seg], preprocessed q|k|v of seg·C
+// tokens (conv / L2 only), carried state (only when needed). With the whole
+// sequence in the workspace and SMs left idle by the scan, the segments are
+// pipelined (see the note on overlapped segments above).
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   const int BH = a.B * a.Hv;
   const int nchunks = (a.T + C - 1) / C;
   if (a.ws_bytes < WS_HEAD) return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(a.workspace, 0, sizeof(int), s);
+  cudaError_t e = cudaMemsetAsync(a.workspace, 0, WS_HEAD, s);   // status word and counters
   if (e != cudaSuccess || BH == 0 || nchunks == 0) return e;
   const bool pre = needs_qkv_prep(a);
   const size_t per_chunk = bytes_per_chunk(a);
@@ -1181,15 +1239,31 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   // Persistent prep: two CTAs per SM. Two fit by shared memory (2 × 113 KB),
   // registers (2 × 256 × 128) and tensor memory (2 × 256 of 512 columns); the
   // occupancy calculator reports one for any kernel that allocates tensor
-  // memory, so the count is set here. CTAs beyond those resident would only
-  // start later (items are independent).
+  // memory, so the count is set here.
   const int prep_ctas = sms * 2;
   const int qp_groups = (2 * a.Hqk + a.Hv) * (D / 8);
+
+  // overlapped segments: whole sequence in the workspace, idle SMs beside the
+  // scan, no load step (its kernel would wait for the scan), S_T given (the
+  // state passes from segment to segment through it)
+  int nseg_ov = 0;
+  if (seg == nchunks && !pre && a.ST != nullptr && BH * 2 < sms && nchunks >= 2 * OVERLAP_MIN_CHUNKS)
+    nseg_ov = std::min(std::min(OVERLAP_SEGMENTS, nchunks / OVERLAP_MIN_CHUNKS), MAX_COUNTERS);
+
+  // Segment lengths. Overlapped: the last scan has no prep beside it, so the
+  // last segment is short (1/16 of the chunks, at least OVERLAP_LAST_MIN) and
+  // the others share the rest equally.
+  const int n_last = nseg_ov > 0 ? std::max(OVERLAP_LAST_MIN, nchunks / 16) : 0;
+  const int step = nseg_ov > 0 ? (nchunks - n_last + nseg_ov - 2) / (nseg_ov - 1) : seg;
   const float* s_in = a.S0;
-  for (int c0 = 0; c0 < nchunks; c0 += seg) {
-    const int n = std::min(seg, nchunks - c0);
+  int k = 0;
+  for (int c0 = 0; c0 < nchunks; ++k) {
+    const int n = nseg_ov > 0 && k == nseg_ov - 1 ? nchunks - c0 : std::min(step, nchunks - c0);
     const bool last = c0 + n >= nchunks;
     float* s_out = last ? a.ST : carry;
+    // overlapped: every chunk has its own slot; otherwise the segment's slots start at 0
+    const SlotMap sm = nseg_ov > 0 ? SlotMap{nchunks, c0} : SlotMap{seg, 0};
+    int* counter = nseg_ov > 0 ? reinterpret_cast<int*>(ws) + 1 + k : nullptr;
     const int grid = std::min(BH * n, prep_ctas);
     if (pre) {
       const int t_begin = c0 * C;
@@ -1208,13 +1282,18 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       ap.qkv_f16 = 1;
       ap.conv_w = nullptr;
       ap.l2norm = 0;
-      chunk_prep_kernel<true><<<grid, NP, P_SMEM, s>>>(ap, c0, n);
+      chunk_prep_kernel<true><<<grid, NP, P_SMEM, s>>>(ap, c0, n, sm, counter);
+    } else if (nseg_ov > 0 && k > 0) {
+      if ((e = launch_dependent(chunk_prep_kernel<false>, grid, NP, P_SMEM, s, a, c0, n, sm, counter)) !=
+          cudaSuccess)
+        return e;
     } else {
-      chunk_prep_kernel<false><<<grid, NP, P_SMEM, s>>>(a, c0, n);
+      chunk_prep_kernel<false><<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter);
     }
-    scan<<<BH * 2, NS, S_SMEM, s>>>(a, c0, n, s_in, s_out);
+    scan<<<BH * 2, NS, S_SMEM, s>>>(a, c0, n, sm, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;
+    c0 += n;
   }
   return cudaSuccess;
 }

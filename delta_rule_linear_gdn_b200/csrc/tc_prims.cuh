@@ -237,6 +237,16 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
+// Programmatic dependent launch: a kernel launched after this one with
+// programmatic stream serialization may start once every CTA of this one has
+// executed launch_dependents (or exited); griddep_wait blocks until the grids
+// this one depends on have completed and their writes are visible (it returns
+// at once for a kernel launched without that attribute).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // Approximate reciprocal (the PTX rcp.approx.ftz.f32 instruction: at most
 // one ulp of error, subnormal inputs and results flushed to zero).
 __device__ __forceinline__ float rcp_approx(float x) {

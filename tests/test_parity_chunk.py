@@ -152,6 +152,31 @@ def test_chunk_size_invariance_and_split_sequence():
     torch.testing.assert_close(Sb, outs[1][1], rtol=1e-5, atol=1e-5)
 
 
+def test_overlapped_segments_match_one_pass_and_oracle():
+    """Few heads and many chunks: the call pipelines its segments (each
+    segment's scan beside the next segment's prep, the state carried through
+    S_T). Same results, bit for bit, as the single-pass schedule (no S_T
+    requested) and as the no-alloc call, whose fixed 32 MB scratch holds about
+    half the chunks and so runs in plain segments; and the oracle's within the
+    bf16-path bound. Ragged tail, nonzero entry state."""
+    w = small(T=64 * 70 + 37, B=1, H_qk=4, H_v=12, d=128, chunk=64, qkv="bf16", s0="normal")
+    inp = make_inputs(w, seed=41)
+    c = to_cuda(inp)
+    args = (c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], c["S0"])
+    o, S = gdn2.chunk_fwd(*args, chunk=64, o_dtype=torch.float32)
+    o1, _ = gdn2.chunk_fwd(*args, chunk=64, o_dtype=torch.float32, want_state=False)
+    o2, S2 = torch.empty_like(o), torch.empty_like(S)
+    gdn2.chunk_fwd_noalloc(*args, o=o2, S_T=S2, chunk=64)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(o1, o, rtol=0, atol=0)
+    torch.testing.assert_close(o2, o, rtol=0, atol=0)
+    torch.testing.assert_close(S2, S, rtol=0, atol=0)
+    ref = oracle_chunk(inp, heads=[(0, 0), (0, 11)])
+    for (bi, h), (o_ref, S_ref) in ref.items():
+        assert_close(o[bi:bi + 1, :, h:h + 1], o_ref, TOL_BF16, f"o[{bi},{h}]")
+        assert_close(S[bi:bi + 1, h:h + 1], S_ref, TOL_BF16, f"S_T[{bi},{h}]")
+
+
 def test_decode_steps_equal_chunked_prefill():
     w = small(T=48, B=2, H_qk=2, H_v=4, d=32, s0="normal")
     inp = make_inputs(w, seed=11)
