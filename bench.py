@@ -44,16 +44,16 @@ DECODE = "decode_b256"
 CONV = "conv_prefill_b8_t8192"
 L2_BYTES = 126 * 2**20
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the two prefill
-# launches of one call, from an ncu capture of prefill_t4096 scaled by 8 to the
-# T=32768 workload (traffic grows with the number of chunks), and the hash of
-# the kernel sources it was taken on; with other sources the figure is stale
-# and the bench reports null.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the prefill
+# launches of one call (4 segments: a prep and a scan each), from a
+# single-pass ncu capture of the T=32768 workload itself, and the hash of the
+# kernel sources it was taken on; with other sources the figure is stale and
+# the bench reports null.
 TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
-TRAFFIC = {"sha1": "16d0da025ec8024f6807e720aaefae0131bd2e8b",
-           # (385.97 + 193.10 + 228.10 + 34.44) MB at T=4096, times 8
-           "bytes_per_call": 6_732_920_832,
-           "profile": "profiles/chunk_prep_scan_t4096_ncu.md"}
+TRAFFIC = {"sha1": "a7c61a1d9240277c3c02f13836e8ab20d114637a",
+           # reads 4.922 GB + writes 2.007 GB over the 8 launches of one call
+           "bytes_per_call": 6_929_130_496,
+           "profile": "profiles/prefill_t32768_dram_traffic.md"}
 
 
 def peaks():
@@ -99,6 +99,23 @@ def decode_bytes(w, o_bytes=2):
     state = B * w.H_v * d * d * 4 * 2
     io = B * w.H_qk * d * 2 * 2 + B * w.H_v * d * 2 + B * w.H_v * d * 4 * 3 + B * w.H_v * d * o_bytes
     return state + io
+
+
+def tc_launches_per_call(w, ws_bytes, dev):
+    """Kernel launches of one gdn2_chunk_fwd call of workload w with S_T given
+    and the whole sequence in the workspace: a prep and a scan kernel per
+    segment; the call pipelines 2 to 4 segments when the scan's (sequence,
+    V head, half) chains leave SMs idle and the sequence has at least 64
+    chunks (the launcher's rule), else it runs one segment. The SIMT path
+    (no workspace) is one launch."""
+    if ws_bytes == 0:
+        return 1
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    nchunks = (w.T + 63) // 64
+    if not w.conv and nchunks >= 64 and 2 * w.B * w.H_v < sms:
+        return 2 * min(4, nchunks // 32)
+    return 2
 
 
 def kernel_sources_sha1():
@@ -357,9 +374,7 @@ def main():
     p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk)
     ws_bytes = gdn2.chunk_fwd_workspace(p)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    # the tensor-core path (the one that takes a workspace) launches a prep and
-    # a scan kernel per call when the workspace holds the whole sequence
-    launches_per_call = 2 if ws_bytes > 0 else 1
+    launches_per_call = tc_launches_per_call(w, ws_bytes, dev)
 
     def prefill_call():
         gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None, chunk=w.chunk,
@@ -395,7 +410,7 @@ def main():
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved_gbs / pk["hbm_gbs"], "traffic": traffic,
                 "peak_source": pk["source"],
-                "kernel": "gdn2_chunk_fwd call (chunk_prep_kernel + chunk_scan_kernel)",
+                "kernel": "gdn2_chunk_fwd call (chunk_prep_kernel + chunk_scan_kernel per segment)",
                 "launches_per_call": launches_per_call, "alg_bytes_per_launch": nbytes,
                 "alg_flops_per_launch": flops, "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"]}
 
