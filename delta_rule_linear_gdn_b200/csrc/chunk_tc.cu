@@ -106,6 +106,7 @@ constexpr int P_EB = 81920;
 constexpr int P_Z = 98304;
 constexpr int P_END = 114688;
 constexpr int P_AINV = 0;
+constexpr int P_KES = P_Z;            // K_end staged for its bulk store (Z is written after the store has read it)
 constexpr int P_YS = P_GM;            // Yᵀ then U_wᵀ (16 KB each), staged for the bulk stores
 constexpr int P_AQS = 16384;          // −Aqk (8 KB) staged for its bulk store: in Gb's block 1,
                                       // read only as don't-care rows by the level-2 products
@@ -433,7 +434,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       gme[c] = e[c] * fe[c];                                                                    \
       gmq[c] = qx[c] * fe[c];                                                                   \
     }                                                                                           \
-    GDN2_TILE(slot, SL_KE + p64, km[c] * ke[c])                                                 \
+    GDN2_TILE(smem, P_KES + p64, km[c] * ke[c])                                                 \
     GDN2_TILE(smem, P_EB + p64, e[c] * g[c])                                                    \
     GDN2_GRAM_TILE(smem, P_GM + p128, gme[c], BF)                                               \
     GDN2_GRAM_TILE(smem, P_GM + 64 * 128 + p128, gmq[c], BF)                                    \
@@ -485,16 +486,10 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       for (int ks = 0; ks < D / 16; ++ks)
         mma16(tmem + PT_GB, gb + k_step_sw(ks, BS_ROW128), kb + k_step_sw(ks, BS_ROW128), id_b, ks > 0);
       mma_commit(bar);
+      bulk_s2g(slot + SL_KE, smem + P_KES, 16384);   // K_end, byte for byte the slot's layout
+      bulk_commit();
     }
     __syncwarp();
-    // Z = w ⊙ v (no decay) to its tile, read by the Y/U_w products
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float vx[4];
-      unpack4_in<F16IN>(vv[u], vx);
-      st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
-          pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
-    }
     wait_mma(bar, phase, sflag);
 
     // -------- T (fp32, shared) and −Aqk (fp16, staged) from TMEM. Lanes
@@ -525,12 +520,22 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       }
     }
     fence_async_smem();
+    if (tid == 0) bulk_wait_read_all();   // K_end's staging is read: the Z tile may be written
     __syncthreads();
     if (tid == 0) {
       bulk_s2g(slot + SL_AQ, smem + P_AQS, 8192);   // −Aqk, byte for byte the slot's layout
       bulk_commit();
     }
 
+
+    // Z = w ⊙ v (no decay) to its tile, read by the Y/U_w products
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      float vx[4];
+      unpack4_in<F16IN>(vv[u], vx);
+      st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
+          pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
+    }
 
     // -------- A = (I + T)⁻¹, blocked
     // level 0: the four 16 × 16 diagonal blocks by forward substitution, one
