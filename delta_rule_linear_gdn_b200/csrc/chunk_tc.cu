@@ -93,8 +93,9 @@ constexpr int BS_ROW64 = 8192;        // block stride of a 64-row tile
 // [32K, 64K) Gm: [Ē_mid ; Q̄_mid], 128 rows, BS 16K
 // [64K, 80K) Km: K̃_mid, 64 rows, BS 8K
 // [80K, 96K) Ē (64 tok × 128 key, BS 8K)   [96K, 112K) Z (64 tok × 128 dv)
-// After the Gram MMAs, [32K, 71K) holds the fp32 arrays of the inverse and
-// [0, 8K) the fp16 A = (I+T)⁻¹ (64 × 64). Two CTAs of this layout fit one SM.
+// After the Gram MMAs, [24K, 63K) holds the fp32 arrays of the inverse,
+// [0, 8K) the fp16 A = (I+T)⁻¹ (64 × 64), and [64K, 80K) Q̄ᵀ and [96K, 112K)
+// K_end wait there for their bulk stores. Two CTAs of this layout fit one SM.
 constexpr int P_GB = 0;
 constexpr int P_KB = 0;
 constexpr int P_PQ = 8192;            // quarter products [4][128] fp32
@@ -107,6 +108,7 @@ constexpr int P_Z = 98304;
 constexpr int P_END = 114688;
 constexpr int P_AINV = 0;
 constexpr int P_KES = P_Z;            // K_end staged for its bulk store (Z is written after the store has read it)
+constexpr int P_QTS = P_KM;           // Q̄ᵀ staged for its bulk store (after the Gram products have read K̃_mid)
 constexpr int P_YS = P_GM;            // Yᵀ then U_wᵀ (16 KB each), staged for the bulk stores
 constexpr int P_AQS = 16384;          // −Aqk (8 KB) staged for its bulk store: in Gb's block 1,
                                       // read only as don't-care rows by the level-2 products
@@ -117,10 +119,10 @@ constexpr int P_L2T = 8192;           // T21, K-major A (first 32 of 128 rows)
 constexpr int P_L2J = 12288;          // A22, K-major A (first 32 of 128 rows)
 static_assert(P_AQS >= P_L2J + 4096 && P_AQS + 8192 <= 32768, "staging of -Aqk clear of the level-2 tiles");
 constexpr int TS = 68;                // fp32 row stride of T and its inverse
-constexpr int P_T = P_GM;             // T   [64][68]
+constexpr int P_T = 24576;            // T   [64][68] (after the Gram products; clear of −Aqk's staging)
 constexpr int P_I = P_T + C * TS * 4; // inv [64][68]
 constexpr int P_X = P_I + C * TS * 4; // tmp [32][36]
-static_assert(P_X + 32 * 36 * 4 <= P_EB, "prep smem overlap");
+static_assert(P_T >= P_AQS + 8192 && P_X + 32 * 36 * 4 <= P_QTS, "prep smem overlap");
 constexpr int P_BAR = P_END;
 constexpr int P_TMEMP = P_BAR + 16;
 constexpr int P_FLAG = P_TMEMP + 16;
@@ -465,10 +467,6 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
                  : make_uint2(0, 0);
     }
-    // Q̄ᵀ [key][tok]: the thread's 8 tokens of each of its keys form one 16-byte chunk
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      st16(slot, SL_QT + sw_off(c0 + c, i0, BS_ROW128), make_uint4(qpk[c][0], qpk[c][1], qpk[c][2], qpk[c][3]));
     sync_for_mma();
 
     // -------- Gram MMAs: [T; Aqk] candidates
@@ -491,6 +489,10 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
     __syncwarp();
     wait_mma(bar, phase, sflag);
+    // Q̄ᵀ [key][tok], staged: the thread's 8 tokens of each of its keys form one 16-byte chunk
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      st16(smem, P_QTS + sw_off(c0 + c, i0, BS_ROW128), make_uint4(qpk[c][0], qpk[c][1], qpk[c][2], qpk[c][3]));
 
     // -------- T (fp32, shared) and −Aqk (fp16, staged) from TMEM. Lanes
     // 0..63 hold rows of T, lanes 64..127 rows of Aqk; the two warps of a lane
@@ -523,7 +525,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     if (tid == 0) bulk_wait_read_all();   // K_end's staging is read: the Z tile may be written
     __syncthreads();
     if (tid == 0) {
-      bulk_s2g(slot + SL_AQ, smem + P_AQS, 8192);   // −Aqk, byte for byte the slot's layout
+      bulk_s2g(slot + SL_AQ, smem + P_AQS, 8192);   // −Aqk and Q̄ᵀ, byte for byte the slot's layout
+      bulk_s2g(slot + SL_QT, smem + P_QTS, 16384);
       bulk_commit();
     }
 
