@@ -19,21 +19,22 @@
 // Two kernels, following the pages' split between the parallel intra-chunk
 // work and the single inter-chunk sweep ("Pipeline Triton da versão por
 // chunks"):
-//   * prep: one CTA per (chunk, sequence, value head), all in parallel. It
-//     builds T and Aqk (tensor cores), inverts I + T (fp32), forms Yᵀ and U_wᵀ
-//     (tensor cores) and writes the chunk's scan operands — Yᵀ, U_wᵀ, Q̄, K_end,
-//     Aqk as fp16 tiles already in the MMA shared-memory layout, and γ_C — to
-//     one 73 KB workspace slot.
-//   * scan: one CTA per (sequence, value head) walks the chunks in order. It
-//     streams the slots into shared memory with bulk copies (double-buffered,
-//     chunk c+1 in flight while c computes) and runs
-//         (Y S)ᵀ = Sᵀ Yᵀ,  Oᵀ = Sᵀ Q̄ᵀ,  Uᵀ = U_wᵀ − (Y S)ᵀ,
-//         Sᵀ ← Sᵀ Γ + Uᵀ K_end,  Oᵀ += Uᵀ Aqkᵀ,
-//     with the fp32 state Sᵀ resident in TMEM and an fp16 copy in shared
-//     memory feeding the next chunk's MMAs.
-// Everything is computed transposed so that every MMA has M = 128. All MMA
-// operand tiles use the 128-byte-swizzled layout (see tc_prims.cuh), so that
-// a warp writing or reading whole rows is free of bank conflicts.
+//   * prep: persistent CTAs over the (chunk, sequence, value head) items,
+//     all independent. Per item it builds T and Aqk (tensor cores), inverts
+//     I + T (fp32 blocks, then a tensor-core merge), forms Yᵀ and U_wᵀ
+//     (tensor cores) and writes the chunk's scan operands — −Yᵀ, −Q̄ᵀ, U_wᵀ,
+//     K_end, −Aqk as fp16 tiles already in the MMA shared-memory layout, and
+//     γ_C — to one 73 KB workspace slot, every tile by a bulk copy.
+//   * scan: two CTAs per (sequence, value head), one per 64-column half of
+//     d_v, walk the chunks in order. They stream the slots into shared memory
+//     with bulk copies (double-buffered, chunk c+1 in flight while c computes)
+//     and run, with Z = [Y; Q̄] stacked so that every product has M = 128,
+//         D = (−Z) S + [I; 0] U_w   (rows 0..63: U = U_w − Y S; rows 64..127: −Q̄ S)
+//         S ← Γ S + K_endᵀ U,       D_rows 64..127 += (−Aqk) U  (= −O / scale),
+//     with the fp32 state resident in TMEM and an fp16 copy in shared memory
+//     feeding the next chunk's products.
+// All MMA operand tiles use the 128-byte-swizzled layout (see tc_prims.cuh),
+// so that a warp writing or reading whole rows is free of bank conflicts.
 //
 // Decay factors of the Gram matrices. Π_{j<s≤i} α is split into two factors
 // about a reference token so that one factor multiplies row i and the other
@@ -74,8 +75,8 @@ constexpr int C = 64;             // chunk
 // Slots follow, one per (sequence, value head, chunk of the segment). Tiles
 // are swizzled; "BS" is the byte stride between 64-column blocks.
 constexpr size_t WS_HEAD = 256;
-constexpr int SL_YT = 0;              // Yᵀ   fp16 [128 key][64 tok]  ┐ Zᵀ = [Yᵀ | Q̄ᵀ]: the two
-constexpr int SL_QT = 16384;          // Q̄ᵀ   fp16 [128 key][64 tok]  ┘ 64-column blocks, BS 16384
+constexpr int SL_YT = 0;              // −Yᵀ  fp16 [128 key][64 tok]  ┐ −Zᵀ = [−Yᵀ | −Q̄ᵀ]: the two
+constexpr int SL_QT = 16384;          // −Q̄ᵀ  fp16 [128 key][64 tok]  ┘ 64-column blocks, BS 16384
 constexpr int SL_UW = 32768;          // U_wᵀ fp16 [128 dv][64 tok]
 constexpr int SL_KE = 49152;          // K_end fp16 [64 tok][128 key] BS 8192
 constexpr int SL_AQ = 65536;          // −Aqk fp16 [64 i][64 j]
@@ -133,7 +134,7 @@ constexpr uint32_t PT_L2P = 0, PT_L2A = 64;   // level-2 inverse accumulators (a
 
 // ------------------------------------------------------------------ scan smem
 // Two stages (see the scan kernel for their layout), then:
-constexpr int S_SH = 2 * 66560;       // −S fp16 [128 key][64 dv]
+constexpr int S_SH = 2 * 66560;       // S fp16 [128 key][64 dv]
 constexpr int S_U = S_SH + 16384;     // U fp16 [64 tok][64 dv]
 constexpr int S_I = S_U + 8192;       // [I_64; 0] fp16 [128][64]
 constexpr int S_BAR = S_I + 16384;    // 10 mbarriers (see the scan kernel)
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       reinterpret_cast<float*>(slot + SL_GC)[tid] = g;
     }
     // Per-channel factors of quarter qt from the quarter products P_m:
-    //   γ_i = pre · f_i,                      pre = Π_{m<qt} P_m
+    //   γ_i = pre · f_i,                      pre = Π_{m<qt} P_m  (held negated: see below)
     //   Π_{i<s≤63} α = (P_qt · suf) / f_i,      suf = Π_{m>qt} P_m
     //   mid-reference factors: f_i / P_qt and P_qt / f_i (first quarter of a
     //   half), f_i and 1 / f_i (second quarter);
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           if (m > qt) su *= P[m][c];
           if (m == qt) own = P[m][c];
         }
-        pre[c] = pr;
+        pre[c] = -pr;                            // Ē and Q̄ leave with the sign the scan wants
         const bool even = (qt & 1) == 0;
         se[c] = even ? rcp_approx(own) : 1.f;
         sk[c] = even ? own : 1.f;
@@ -525,7 +526,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     if (tid == 0) bulk_wait_read_all();   // K_end's staging is read: the Z tile may be written
     __syncthreads();
     if (tid == 0) {
-      bulk_s2g(slot + SL_AQ, smem + P_AQS, 8192);   // −Aqk and Q̄ᵀ, byte for byte the slot's layout
+      bulk_s2g(slot + SL_AQ, smem + P_AQS, 8192);   // −Aqk and −Q̄ᵀ, byte for byte the slot's layout
       bulk_s2g(slot + SL_QT, smem + P_QTS, 16384);
       bulk_commit();
     }
@@ -662,7 +663,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
     sync_for_mma();
 
-    // -------- Yᵀ = Ēᵀ Aᵀ, U_wᵀ = Zᵀ Aᵀ
+    // -------- −Yᵀ = −Ēᵀ Aᵀ, U_wᵀ = Zᵀ Aᵀ (Ē carries the sign, Z here is the write side w ⊙ v)
     if (tid == 0) {
       const uint64_t eb = desc_mn_sw(smem_u32(smem + P_EB), 0, BS_ROW64);
       const uint64_t z = desc_mn_sw(smem_u32(smem + P_Z), 0, BS_ROW64);
@@ -722,18 +723,18 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 // half of d_v (the recurrence never mixes d_v columns), walking the chunks of
 // the segment in order. Per chunk c, with the state S (d_k × 64, fp32 in TMEM,
 // one key per lane) and Z = [Y; Q̄] stacked along the rows:
-//   D  = Z (−S) + [I; 0] U_w  → rows 0..63: U = U_w − Y S, rows 64..127: −Q̄ S
+//   D  = (−Z) S + [I; 0] U_w  → rows 0..63: U = U_w − Y S, rows 64..127: −Q̄ S
 //   S ← Γ S + K_endᵀ U        (TMEM holds Γ S already)
 //   D_rows 64..127 −= Aqk U   → −O / scale
 // Every product has M = 128. Warp 8 issues the products and the slot copies
 // (one thread); warps with TMEM lanes 0..63 write U, those with lanes 64..127
 // write the outputs of the previous chunk, and all eight copy the state (fp16
-// −S for the next chunk's products, TMEM ← S·Γ_next).
+// S for the next chunk's products, TMEM ← S·Γ_next).
 // =============================================================================
 constexpr int NS = 288;               // scan threads: 8 epilogue warps + 1 MMA warp
 
 // Stage (one chunk's operands for this half), filled by three bulk copies.
-constexpr int SG_ZT = 0;              // Zᵀ = [Yᵀ | Q̄ᵀ]  [128 key][128 tok], BS 16384
+constexpr int SG_ZT = 0;              // −Zᵀ = [−Yᵀ | −Q̄ᵀ]  [128 key][128 tok], BS 16384
 constexpr int SG_UW = 32768;          // U_wᵀ rows of this half [64 dv][64 tok]
 constexpr int SG_KE = 40960;          // K_end [64 tok][128 key], BS 8192
 constexpr int SG_AQ = 57344;          // −Aqk [64][64] (must follow K_end: see the O product)
@@ -768,10 +769,10 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_BAR);
   uint64_t* full = bars;                // [2] stage s loaded
-  uint64_t* b_d = bars + 2;             // Z(−S) + [I;0]U_w done (U and −Q̄S in D)
+  uint64_t* b_d = bars + 2;             // (−Z)S + [I;0]U_w done (U and −Q̄S in D)
   uint64_t* b_u = bars + 3;             // U written (fp16)
   uint64_t* b_s = bars + 4;             // state update done
-  uint64_t* b_sh = bars + 5;            // fp16 −S written (one arrival per epilogue warp)
+  uint64_t* b_sh = bars + 5;            // fp16 S written (one arrival per epilogue warp)
   uint64_t* b_o = bars + 6;             // [2] D buffer holds the chunk's −O
   uint64_t* b_of = bars + 8;            // [2] D buffer read out
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + S_TMEMP);
@@ -832,7 +833,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         load(c);
         ++issued;
       }
-      const uint32_t id_zs = idesc_f16(128, 64, true, true);     // Zᵀ (MN) × −S (MN)
+      const uint32_t id_zs = idesc_f16(128, 64, true, true);     // −Zᵀ (MN) × S (MN)
       const uint32_t id_iu = idesc_f16(128, 64, false, false);   // [I;0] (K) × U_wᵀ (K)
       const uint32_t id_kn = idesc_f16(128, 64, true, true);     // K_endᵀ (MN) × U (MN)
       const uint32_t id_au = idesc_f16(128, 64, false, true);    // [·;−Aqk] (K) × U (MN)
@@ -850,7 +851,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         if (!ok) break;
         ++landed;
         fence_after_sync();
-        // D = [I; 0] U_w (needs no state: issued ahead), then D += Z (−S)
+        // D = [I; 0] U_w (needs no state: issued ahead), then D += (−Z) S
         const uint64_t z0 = desc_mn_sw(smem_u32(stg + SG_ZT), 0, BS_ROW128);
         const uint64_t w0 = desc_k_sw(smem_u32(stg + SG_UW), 0, BS_ROW64);
 #pragma unroll
@@ -909,7 +910,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       fence_after_sync();
     };
 
-    // The entry state: fp16 −S for the first chunk's products, TMEM ← S · Γ
+    // The entry state: fp16 S for the first chunk's products, TMEM ← S · Γ
     // of the first chunk.
     wait(&full[0], 0);
     {
@@ -921,11 +922,8 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         const float4 x = S0 ? __ldg(reinterpret_cast<const float4*>(S0 + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
         v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
       }
-      float n[32];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) n[u] = -v[u];
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(n + cb));
+      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
 #pragma unroll
       for (int u = 0; u < 32; ++u) v[u] *= g;
       tmem_st16(t_lane + ST_S + c0, v);
@@ -981,7 +979,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         wait(&b_o[s ^ 1], (uint32_t)(((c - 1) >> 1) & 1));
         out_rows(c - 1, ST_D + 64u * (uint32_t)(s ^ 1), &b_of[s ^ 1]);
       }
-      // the state: fp16 −S for the next chunk and TMEM ← S · Γ_next; S_T after the last
+      // the state: fp16 S for the next chunk and TMEM ← S · Γ_next; S_T after the last
       const bool more = c + 1 < n_seg;
       if (more) wait(&full[s ^ 1], (uint32_t)(((c + 1) >> 1) & 1));
       wait(b_s, ph);
@@ -991,12 +989,9 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         tmem_ld16(t_lane + ST_S + c0 + 16, v + 16);
         tmem_wait_ld();
         if (more) {
-          float n[32];
 #pragma unroll
-          for (int u = 0; u < 32; ++u) n[u] = -v[u];
-#pragma unroll
-          for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(n + cb));
-          // publish this warp's part of −S at once: the next products need
+          for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
+          // publish this warp's part of S at once: the next products need
           // only that; the TMEM state is scaled while they run
           fence_async_smem();
           __syncwarp();
