@@ -132,17 +132,6 @@ constexpr int P_SMEM = P_FLAG + 16;
 constexpr uint32_t PT_GM = 0, PT_GB = 64, PT_YT = 128, PT_UW = 192, PT_COLS = 256;
 constexpr uint32_t PT_L2P = 0, PT_L2A = 64;   // level-2 inverse accumulators (after the Gram read-out)
 
-// ------------------------------------------------------------------ scan smem
-// Two stages (see the scan kernel for their layout), then:
-constexpr int S_SH = 2 * 66560;       // S fp16 [128 key][64 dv]
-constexpr int S_U = S_SH + 16384;     // U fp16 [64 tok][64 dv]
-constexpr int S_I = S_U + 8192;       // [I_64; 0] fp16 [128][64]
-constexpr int S_BAR = S_I + 16384;    // 10 mbarriers (see the scan kernel)
-constexpr int S_TMEMP = S_BAR + 128;
-constexpr int S_FLAG = S_TMEMP + 16;
-constexpr int S_SMEM = S_FLAG + 16;
-constexpr uint32_t ST_S = 0, ST_D = 64, ST_COLS = 256;   // S (64 columns), D double-buffered: 64, 128
-
 __device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
   *reinterpret_cast<uint4*>(base + off) = v;
 }
@@ -719,32 +708,54 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 }
 
 // =============================================================================
-// scan kernel: two CTAs per (sequence, value head), each owning one 64-wide
-// half of d_v (the recurrence never mixes d_v columns), walking the chunks of
-// the segment in order. Per chunk c, with the state S (d_k × 64, fp32 in TMEM,
-// one key per lane) and Z = [Y; Q̄] stacked along the rows:
+// scan kernel: one CTA per (sequence, value head, block of DV columns of d_v)
+// — DV = 64 (two CTAs per head) or 128 (one) — walking the chunks of the
+// segment in order; the recurrence never mixes d_v columns. Per chunk c, with
+// the state S (d_k × DV, fp32 in TMEM, one key per lane) and Z = [Y; Q̄]
+// stacked along the rows:
 //   D  = (−Z) S + [I; 0] U_w  → rows 0..63: U = U_w − Y S, rows 64..127: −Q̄ S
 //   S ← Γ S + K_endᵀ U        (TMEM holds Γ S already)
 //   D_rows 64..127 −= Aqk U   → −O / scale
-// Every product has M = 128. Warp 8 issues the products and the slot copies
-// (one thread); warps with TMEM lanes 0..63 write U, those with lanes 64..127
-// write the outputs of the previous chunk, and all eight copy the state (fp16
-// S for the next chunk's products, TMEM ← S·Γ_next).
+// Every product has M = 128 and N = DV. The last warp issues the products and
+// the slot copies (one thread); of the DV/8 epilogue warps (32 columns each,
+// DV/32 per TMEM lane quarter), those on lanes 0..63 write U, those on lanes
+// 64..127 write the outputs of the previous chunk, and all copy the state
+// (fp16 S for the next chunk's products, TMEM ← S·Γ_next). Two CTAs per head
+// finish a chunk sooner; one CTA per head does the work of two on one SM,
+// which pays when the half-width CTAs would need more waves than the SMs give.
 // =============================================================================
-constexpr int NS = 288;               // scan threads: 8 epilogue warps + 1 MMA warp
-
-// Stage (one chunk's operands for this half), filled by three bulk copies.
-constexpr int SG_ZT = 0;              // −Zᵀ = [−Yᵀ | −Q̄ᵀ]  [128 key][128 tok], BS 16384
-constexpr int SG_UW = 32768;          // U_wᵀ rows of this half [64 dv][64 tok]
-constexpr int SG_KE = 40960;          // K_end [64 tok][128 key], BS 8192
-constexpr int SG_AQ = 57344;          // −Aqk [64][64] (must follow K_end: see the O product)
-constexpr int SG_GC = 65536;          // γ_C [128] fp32
-constexpr int SG_BYTES = 32768 + 8192 + (SLOT_USED - SL_KE);
-constexpr int STAGE = 66560;          // stage stride (1 KB multiple)
-static_assert(S_SH == 2 * STAGE, "scan shared-memory layout");
-static_assert(SG_AQ == SG_KE + 16384 && SG_GC == SG_AQ + 8192, "stage tail copied in one piece");
+template <int DV>
+struct ScanLayout {
+  static_assert(DV == 64 || DV == 128, "d_v block of a scan CTA");
+  static constexpr int NE = DV * 4;              // epilogue threads
+  static constexpr int NS = NE + 32;             // + the MMA warp
+  // Stage: one chunk's operands for this CTA's columns. DV = 128 takes the
+  // slot byte for byte; DV = 64 takes its half of U_wᵀ and the rest.
+  static constexpr int ZT = 0;                   // −Zᵀ = [−Yᵀ | −Q̄ᵀ]  [128 key][128 tok], BS 16384
+  static constexpr int UW = 32768;               // U_wᵀ rows of the block [DV][64 tok]
+  static constexpr int KE = UW + DV * 128;       // K_end [64 tok][128 key], BS 8192
+  static constexpr int AQ = KE + 16384;          // −Aqk [64][64] (must follow K_end: see the O product)
+  static constexpr int GC = AQ + 8192;           // γ_C [128] fp32
+  static constexpr int BYTES = GC + 512;         // copied per chunk
+  static constexpr int STAGE = (BYTES + 1023) / 1024 * 1024;
+  static constexpr int SH = 2 * STAGE;           // S fp16 [128 key][DV], BS 16384
+  static constexpr int U = SH + 128 * DV * 2;    // U fp16 [64 tok][DV], BS 8192
+  static constexpr int I = U + 64 * DV * 2;      // [I_64; 0] fp16 [128][64]
+  static constexpr int BAR = I + 16384;          // 10 mbarriers
+  static constexpr int TMEMP = BAR + 128;
+  static constexpr int FLAG = TMEMP + 16;
+  static constexpr int SMEM = FLAG + 16;
+  static constexpr uint32_t T_S = 0, T_D = DV;   // TMEM: S (DV columns), D double-buffered
+  static constexpr uint32_t T_COLS = DV == 64 ? 256 : 512;
+};
+static_assert(ScanLayout<128>::ZT == SL_YT && ScanLayout<128>::UW == SL_UW && ScanLayout<128>::KE == SL_KE &&
+                  ScanLayout<128>::AQ == SL_AQ && ScanLayout<128>::GC == SL_GC && ScanLayout<128>::BYTES == SLOT_USED,
+              "a full-width stage is the slot");
 static_assert(SL_AQ == SL_KE + 16384 && SL_GC == SL_AQ + 8192, "slot tail copied in one piece");
-static_assert(SG_GC + 512 <= STAGE, "stage size");
+static_assert(ScanLayout<64>::SMEM <= 232448 && ScanLayout<128>::SMEM <= 232448, "scan shared memory");
+static_assert(ScanLayout<64>::SH % 1024 == 0 && ScanLayout<128>::SH % 1024 == 0 && ScanLayout<64>::U % 1024 == 0 &&
+                  ScanLayout<128>::U % 1024 == 0 && ScanLayout<64>::I % 1024 == 0 && ScanLayout<128>::I % 1024 == 0,
+              "swizzled tiles on 1 KB boundaries");
 
 // 16 bytes of output: 8 bf16 or 4 fp32 values of sc · x.
 template <typename TOut> __device__ __forceinline__ uint4 pack_out(const float* x, float sc);
@@ -759,15 +770,18 @@ template <> __device__ __forceinline__ uint4 pack_out<float>(const float* x, flo
                     __float_as_uint(sc * x[3]));
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
-__device__ __forceinline__ void u_sync() { asm volatile("bar.sync 2, 128;\n" ::: "memory"); }
-__device__ __forceinline__ void o_sync() { asm volatile("bar.sync 3, 128;\n" ::: "memory"); }
+// named barriers of the epilogue warps (all of them; those writing U; those writing outputs)
+template <int NE> __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(NE) : "memory"); }
+template <int NE> __device__ __forceinline__ void u_sync() { asm volatile("bar.sync 2, %0;\n" ::"n"(NE / 2) : "memory"); }
+template <int NE> __device__ __forceinline__ void o_sync() { asm volatile("bar.sync 3, %0;\n" ::"n"(NE / 2) : "memory"); }
 
-template <typename TOut>
-__global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
+template <typename TOut, int DV>
+__global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
                                                            const float* S_in, float* S_out) {
+  using L = ScanLayout<DV>;
+  constexpr int NE = L::NE;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
   uint64_t* full = bars;                // [2] stage s loaded
   uint64_t* b_d = bars + 2;             // (−Z)S + [I;0]U_w done (U and −Q̄S in D)
   uint64_t* b_u = bars + 3;             // U written (fp16)
@@ -775,13 +789,14 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   uint64_t* b_sh = bars + 5;            // fp16 S written (one arrival per epilogue warp)
   uint64_t* b_o = bars + 6;             // [2] D buffer holds the chunk's −O
   uint64_t* b_of = bars + 8;            // [2] D buffer read out
-  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + S_TMEMP);
-  int* sflag = reinterpret_cast<int*>(smem + S_FLAG);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::TMEMP);
+  int* sflag = reinterpret_cast<int*>(smem + L::FLAG);
   volatile int* estop = sflag + 1;      // [2] the epilogue warps' samples of the flag
   const volatile int* vflag = sflag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x >> 1, half = blockIdx.x & 1;
+  const int bh = DV == D ? (int)blockIdx.x : (int)blockIdx.x >> 1;
+  const int col0 = DV == D ? 0 : ((int)blockIdx.x & 1) * DV;   // first d_v column of this CTA
   // resident: the next segment's prep, launched as a programmatic dependent,
   // may take the SMs this grid leaves free
   griddep_launch_dependents();
@@ -790,14 +805,14 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   TOut* og = static_cast<TOut*>(a.o);
 
   if (tid == 0) {
-    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], &bars[i] == b_sh ? 8 : 1);   // b_sh: one per epilogue warp
+    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], &bars[i] == b_sh ? NE / 32 : 1);   // b_sh: one per epilogue warp
     fence_mbar_init();
     sflag[0] = 0;
     sflag[1] = 0;
     sflag[2] = 0;
   }
   if (warp == 0) {
-    tmem_alloc(tmem_ptr, ST_COLS);
+    tmem_alloc(tmem_ptr, L::T_COLS);
     tmem_relinquish();
   }
   if (warp < 8) {
@@ -808,7 +823,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       float x[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) x[u] = (r == cq + cb + u) ? 1.f : 0.f;
-      st16(smem, S_I + sw_off(r, cq + cb, BS_ROW128), pack8_f16(x));
+      st16(smem, L::I + sw_off(r, cq + cb, BS_ROW128), pack8_f16(x));
     }
     fence_async_smem();
   }
@@ -817,43 +832,47 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
   fence_after_sync();
   const uint32_t tmem = *tmem_ptr;
 
-  if (warp == 8) {
+  if (warp == NE / 32) {
     // ------------------------------------------------------------ MMA thread
     if (lane == 0) {
       auto load = [&](int c) {
-        uint8_t* stg = smem + (c & 1) * STAGE;
+        uint8_t* stg = smem + (c & 1) * L::STAGE;
         const uint8_t* sl = slots + (size_t)c * SLOT;
-        mbar_arrive_expect_tx(&full[c & 1], SG_BYTES);
-        bulk_g2s(stg + SG_ZT, sl + SL_YT, 32768, &full[c & 1]);
-        bulk_g2s(stg + SG_UW, sl + SL_UW + half * 8192, 8192, &full[c & 1]);
-        bulk_g2s(stg + SG_KE, sl + SL_KE, SLOT_USED - SL_KE, &full[c & 1]);
+        mbar_arrive_expect_tx(&full[c & 1], L::BYTES);
+        if (DV == D) {
+          bulk_g2s(stg, sl, L::BYTES, &full[c & 1]);
+        } else {
+          bulk_g2s(stg + L::ZT, sl + SL_YT, 32768, &full[c & 1]);
+          bulk_g2s(stg + L::UW, sl + SL_UW + col0 * 128, DV * 128, &full[c & 1]);
+          bulk_g2s(stg + L::KE, sl + SL_KE, SLOT_USED - SL_KE, &full[c & 1]);
+        }
       };
       int issued = 0, landed = 0;       // chunks whose copies were issued / seen complete
       for (int c = 0; c < n_seg && c < 2; ++c) {
         load(c);
         ++issued;
       }
-      const uint32_t id_zs = idesc_f16(128, 64, true, true);     // −Zᵀ (MN) × S (MN)
-      const uint32_t id_iu = idesc_f16(128, 64, false, false);   // [I;0] (K) × U_wᵀ (K)
-      const uint32_t id_kn = idesc_f16(128, 64, true, true);     // K_endᵀ (MN) × U (MN)
-      const uint32_t id_au = idesc_f16(128, 64, false, true);    // [·;−Aqk] (K) × U (MN)
-      const uint64_t sh0 = desc_mn_sw(smem_u32(smem + S_SH), 0, BS_ROW128);
-      const uint64_t u0 = desc_mn_sw(smem_u32(smem + S_U), 0, BS_ROW64);
-      const uint64_t i0 = desc_k_sw(smem_u32(smem + S_I), 0, BS_ROW128);
+      const uint32_t id_zs = idesc_f16(128, DV, true, true);     // −Zᵀ (MN) × S (MN)
+      const uint32_t id_iu = idesc_f16(128, DV, false, false);   // [I;0] (K) × U_wᵀ (K)
+      const uint32_t id_kn = idesc_f16(128, DV, true, true);     // K_endᵀ (MN) × U (MN)
+      const uint32_t id_au = idesc_f16(128, DV, false, true);    // [·;−Aqk] (K) × U (MN)
+      const uint64_t sh0 = desc_mn_sw(smem_u32(smem + L::SH), 0, BS_ROW128);
+      const uint64_t u0 = desc_mn_sw(smem_u32(smem + L::U), 0, BS_ROW64);
+      const uint64_t i0 = desc_k_sw(smem_u32(smem + L::I), 0, BS_ROW128);
       bool ok = true;
       for (int c = 0; c < n_seg && ok; ++c) {
         const int s = c & 1;
         const uint32_t ph = (uint32_t)(c & 1);
-        uint8_t* stg = smem + s * STAGE;
-        const uint32_t db = ST_D + 64u * (uint32_t)s;
+        uint8_t* stg = smem + s * L::STAGE;
+        const uint32_t db = L::T_D + (uint32_t)DV * (uint32_t)s;
         ok = mbar_wait_or_stop(&full[s], (uint32_t)((c >> 1) & 1), vflag) &&
              (c < 2 || mbar_wait_or_stop(&b_of[s], (uint32_t)(((c - 2) >> 1) & 1), vflag));
         if (!ok) break;
         ++landed;
         fence_after_sync();
         // D = [I; 0] U_w (needs no state: issued ahead), then D += (−Z) S
-        const uint64_t z0 = desc_mn_sw(smem_u32(stg + SG_ZT), 0, BS_ROW128);
-        const uint64_t w0 = desc_k_sw(smem_u32(stg + SG_UW), 0, BS_ROW64);
+        const uint64_t z0 = desc_mn_sw(smem_u32(stg + L::ZT), 0, BS_ROW128);
+        const uint64_t w0 = desc_k_sw(smem_u32(stg + L::UW), 0, BS_ROW64);   // DV rows, one K block
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
           mma16(tmem + db, i0 + k_step_sw(ks, BS_ROW128), w0 + k_step_sw(ks, BS_ROW64), id_iu, ks > 0);
@@ -869,10 +888,10 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         ok = mbar_wait_or_stop(b_u, ph, vflag);
         if (!ok) break;
         fence_after_sync();
-        const uint64_t ke0 = desc_mn_sw(smem_u32(stg + SG_KE), 0, BS_ROW64);
-        const uint64_t aq0 = desc_k_sw(smem_u32(stg + SG_AQ - 8192), 0, BS_ROW64);
+        const uint64_t ke0 = desc_mn_sw(smem_u32(stg + L::KE), 0, BS_ROW64);
+        const uint64_t aq0 = desc_k_sw(smem_u32(stg + L::AQ - 8192), 0, BS_ROW64);
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) mma16(tmem + ST_S, ke0 + mn_step_sw(ks), u0 + mn_step_sw(ks), id_kn, 1);
+        for (int ks = 0; ks < C / 16; ++ks) mma16(tmem + L::T_S, ke0 + mn_step_sw(ks), u0 + mn_step_sw(ks), id_kn, 1);
         mma_commit(b_s);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
@@ -898,9 +917,9 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
     const int lq = warp & 3;
     const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
     const int row = lq * 32 + lane;     // TMEM lane: a key of S; a row of D
-    const int c0 = (warp >> 2) * 32;    // this warp's 32 of the half's 64 columns
+    const int c0 = (warp >> 2) * 32;    // this warp's 32 of the CTA's DV columns
     const bool u_warp = lq < 2;         // D rows 0..63 (U) or 64..127 (outputs)
-    const int dv0 = half * 64 + c0;     // first d_v column of this thread's 32
+    const int dv0 = col0 + c0;          // first d_v column of this thread's 32
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok && !mbar_wait_or_stop(bar, parity, vflag)) {
@@ -914,7 +933,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
     // of the first chunk.
     wait(&full[0], 0);
     {
-      const float g = reinterpret_cast<const float*>(smem + SG_GC)[row];
+      const float g = reinterpret_cast<const float*>(smem + L::GC)[row];
       const float* S0 = S_in ? S_in + ((size_t)bh * D + row) * D + dv0 : nullptr;
       float v[32];
 #pragma unroll
@@ -923,11 +942,11 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
       }
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
+      for (int cb = 0; cb < 32; cb += 8) st16(smem, L::SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
 #pragma unroll
       for (int u = 0; u < 32; ++u) v[u] *= g;
-      tmem_st16(t_lane + ST_S + c0, v);
-      tmem_st16(t_lane + ST_S + c0 + 16, v + 16);
+      tmem_st16(t_lane + L::T_S + c0, v);
+      tmem_st16(t_lane + L::T_S + c0 + 16, v + 16);
       tmem_wait_st();
     }
     fence_async_smem();
@@ -945,7 +964,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       tmem_ld16(t_lane + db + c0 + 16, v + 16);
       tmem_wait_ld();
       fence_before_sync();
-      o_sync();
+      o_sync<NE>();
       if (tid == 64) mbar_arrive(freed);           // first thread of the output warps
       const int i = row - 64;
       if (i < Lco) {
@@ -960,7 +979,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
     for (int c = 0; c < n_seg; ++c) {
       const int s = c & 1;
       const uint32_t ph = (uint32_t)(c & 1);
-      const uint32_t db = ST_D + 64u * (uint32_t)s;
+      const uint32_t db = L::T_D + (uint32_t)DV * (uint32_t)s;
       if (u_warp) {
         // U (rows 0..63 of D) → fp16 tile [tok][dv]
         wait(b_d, ph);
@@ -969,15 +988,15 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
         tmem_ld16(t_lane + db + c0 + 16, v + 16);
         tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(smem, S_U + sw_off(row, c0 + cb, BS_ROW64), pack8_f16(v + cb));
+        for (int cb = 0; cb < 32; cb += 8) st16(smem, L::U + sw_off(row, c0 + cb, BS_ROW64), pack8_f16(v + cb));
         fence_async_smem();
         fence_before_sync();
-        u_sync();
+        u_sync<NE>();
         if (tid == 0) mbar_arrive(b_u);
       } else if (c > 0) {
         // outputs of the previous chunk
         wait(&b_o[s ^ 1], (uint32_t)(((c - 1) >> 1) & 1));
-        out_rows(c - 1, ST_D + 64u * (uint32_t)(s ^ 1), &b_of[s ^ 1]);
+        out_rows(c - 1, L::T_D + (uint32_t)DV * (uint32_t)(s ^ 1), &b_of[s ^ 1]);
       }
       // the state: fp16 S for the next chunk and TMEM ← S · Γ_next; S_T after the last
       const bool more = c + 1 < n_seg;
@@ -985,22 +1004,22 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       wait(b_s, ph);
       {
         float v[32];
-        tmem_ld16(t_lane + ST_S + c0, v);
-        tmem_ld16(t_lane + ST_S + c0 + 16, v + 16);
+        tmem_ld16(t_lane + L::T_S + c0, v);
+        tmem_ld16(t_lane + L::T_S + c0 + 16, v + 16);
         tmem_wait_ld();
         if (more) {
 #pragma unroll
-          for (int cb = 0; cb < 32; cb += 8) st16(smem, S_SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
+          for (int cb = 0; cb < 32; cb += 8) st16(smem, L::SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
           // publish this warp's part of S at once: the next products need
           // only that; the TMEM state is scaled while they run
           fence_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(b_sh);
-          const float g = reinterpret_cast<const float*>(smem + (s ^ 1) * STAGE + SG_GC)[row];
+          const float g = reinterpret_cast<const float*>(smem + (s ^ 1) * L::STAGE + L::GC)[row];
 #pragma unroll
           for (int u = 0; u < 32; ++u) v[u] *= g;
-          tmem_st16(t_lane + ST_S + c0, v);
-          tmem_st16(t_lane + ST_S + c0 + 16, v + 16);
+          tmem_st16(t_lane + L::T_S + c0, v);
+          tmem_st16(t_lane + L::T_S + c0 + 16, v + 16);
           tmem_wait_st();
         } else if (S_out && ok) {
           float* ST = S_out + ((size_t)bh * D + row) * D + dv0;
@@ -1019,7 +1038,7 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
       // (two sample slots: slot c & 1 is rewritten only in chunk c + 2, after
       // every thread has passed the barrier of chunk c + 1)
       if (tid == 0) estop[c & 1] = *vflag;
-      epi_sync();
+      epi_sync<NE>();
       if (estop[c & 1] != 0) {
         ok = false;
         stopped = true;
@@ -1030,14 +1049,14 @@ __global__ void __launch_bounds__(NS, 1) chunk_scan_kernel(ChunkArgs a, int c_be
     if (!stopped && n_seg > 0 && !u_warp) {
       const int s = (n_seg - 1) & 1;
       wait(&b_o[s], (uint32_t)(((n_seg - 1) >> 1) & 1));
-      out_rows(n_seg - 1, ST_D + 64u * (uint32_t)s, &b_of[s]);
+      out_rows(n_seg - 1, L::T_D + (uint32_t)DV * (uint32_t)s, &b_of[s]);
     }
     if (!ok) atomicOr(sflag, 1);
   }
   fence_before_sync();
   __syncthreads();
   if (tid == 0 && *sflag) atomicOr(static_cast<int*>(a.workspace), 1);
-  if (warp == 0) tmem_dealloc(tmem, ST_COLS);
+  if (warp == 0) tmem_dealloc(tmem, L::T_COLS);
 }
 
 // =============================================================================
@@ -1170,7 +1189,7 @@ size_t chunk_tc_min_workspace(const ChunkArgs& a, bool carry_state) {
 
 namespace {
 // The scan of segment k and the prep of segment k + 1 overlap when the scan
-// leaves SMs idle (fewer (sequence, V head, half) chains than SMs) and the
+// leaves SMs idle (fewer scan CTAs than SMs) and the
 // workspace holds every chunk's slot: the prep is launched as a programmatic
 // dependent of the scan, so it starts once the scan's CTAs are resident and
 // takes the SMs they leave free (items from a counter, so that CTAs which start
@@ -1233,12 +1252,21 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;
   }
-  auto scan = o_bf16 ? chunk_scan_kernel<__nv_bfloat16> : chunk_scan_kernel<float>;
-  if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM)) != cudaSuccess) return e;
-
   int dev = 0, sms = 148;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  // Scan width: half-width CTAs (two per head) finish a chunk sooner, but when
+  // they need more waves than the SMs give, full-width ones (one per head, a
+  // chunk in ≈1.7× the time, measured) finish the call sooner.
+  const int waves_half = (2 * BH + sms - 1) / sms, waves_full = (BH + sms - 1) / sms;
+  const bool full_width = 5 * waves_full < 3 * waves_half;
+  const int scan_ctas = full_width ? BH : 2 * BH;
+  auto scan = full_width ? (o_bf16 ? chunk_scan_kernel<__nv_bfloat16, 128> : chunk_scan_kernel<float, 128>)
+                         : (o_bf16 ? chunk_scan_kernel<__nv_bfloat16, 64> : chunk_scan_kernel<float, 64>);
+  const int scan_threads = full_width ? ScanLayout<128>::NS : ScanLayout<64>::NS;
+  const int scan_smem = full_width ? ScanLayout<128>::SMEM : ScanLayout<64>::SMEM;
+  if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
+    return e;
   // Persistent prep: two CTAs per SM. Two fit by shared memory (2 × 113 KB),
   // registers (2 × 256 × 128) and tensor memory (2 × 256 of 512 columns); the
   // occupancy calculator reports one for any kernel that allocates tensor
@@ -1250,7 +1278,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   // scan, no load step (its kernel would wait for the scan), S_T given (the
   // state passes from segment to segment through it)
   int nseg_ov = 0;
-  if (seg == nchunks && !pre && a.ST != nullptr && BH * 2 < sms && nchunks >= 2 * OVERLAP_MIN_CHUNKS)
+  if (seg == nchunks && !pre && a.ST != nullptr && scan_ctas < sms && nchunks >= 2 * OVERLAP_MIN_CHUNKS)
     nseg_ov = std::min(std::min(OVERLAP_SEGMENTS, nchunks / OVERLAP_MIN_CHUNKS), MAX_COUNTERS);
 
   // Segment lengths. Overlapped: the last scan has no prep beside it, so the
@@ -1293,7 +1321,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     } else {
       chunk_prep_kernel<false><<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter);
     }
-    scan<<<BH * 2, NS, S_SMEM, s>>>(a, c0, n, sm, s_in, s_out);
+    scan<<<scan_ctas, scan_threads, scan_smem, s>>>(a, c0, n, sm, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;
     c0 += n;

@@ -177,6 +177,21 @@ def test_overlapped_segments_match_one_pass_and_oracle():
         assert_close(S[bi:bi + 1, h:h + 1], S_ref, TOL_BF16, f"S_T[{bi},{h}]")
 
 
+@pytest.mark.parametrize("gate_mode", ["full", "gdn"])
+def test_full_width_scan_many_heads(gate_mode):
+    """Two sequences of the 48-V-head layer: twice as many half-width scan CTAs
+    as one wave holds, so the launcher runs one full-width (d_v = 128) scan CTA
+    per head. Ragged tail, nonzero entry state; sampled heads of both
+    sequences against the oracle."""
+    w = small(T=150, B=2, H_qk=16, H_v=48, d=128, chunk=64, qkv="bf16", s0="normal")
+    inp = make_inputs(w, seed=43, gate_mode=gate_mode)
+    o, S = run(inp, chunk=64, gate_mode=gate_mode, o_dtype=torch.float32)
+    ref = oracle_chunk(inp, gate_mode=gate_mode, heads=[(0, 0), (0, 47), (1, 1), (1, 30)])
+    for (bi, h), (o_ref, S_ref) in ref.items():
+        assert_close(o[bi:bi + 1, :, h:h + 1], o_ref, TOL_BF16, f"o[{bi},{h}]")
+        assert_close(S[bi:bi + 1, h:h + 1], S_ref, TOL_BF16, f"S_T[{bi},{h}]")
+
+
 def test_decode_steps_equal_chunked_prefill():
     w = small(T=48, B=2, H_qk=2, H_v=4, d=32, s0="normal")
     inp = make_inputs(w, seed=11)
