@@ -103,19 +103,24 @@ def decode_bytes(w, o_bytes=2):
 
 def tc_launches_per_call(w, ws_bytes, dev):
     """Kernel launches of one gdn2_chunk_fwd call of workload w with S_T given
-    and the whole sequence in the workspace: a prep and a scan kernel per
-    segment; the call pipelines 2 to 4 segments when the scan's (sequence,
-    V head, half) chains leave SMs idle and the sequence has at least 64
-    chunks (the launcher's rule), else it runs one segment. The SIMT path
-    (no workspace) is one launch."""
+    and the whole sequence in the workspace, by the launcher's rules: the scan
+    runs 2·B·H_v half-width CTAs, or B·H_v full-width ones when the half-width
+    grid would need ≥ 5/3 as many waves; when the scan grid leaves SMs idle,
+    the sequence has at least 64 chunks and no load step (conv / L2 norm) is
+    fused, the call pipelines 2 to 4 segments (a prep and a scan each), else
+    it runs one segment (a prep and a scan, plus the load step if fused). The
+    SIMT path (no workspace) is one launch."""
     if ws_bytes == 0:
         return 1
     import torch
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    bh = w.B * w.H_v
+    waves_half, waves_full = -(-2 * bh // sms), -(-bh // sms)
+    scan_ctas = bh if 5 * waves_full < 3 * waves_half else 2 * bh
     nchunks = (w.T + 63) // 64
-    if not w.conv and nchunks >= 64 and 2 * w.B * w.H_v < sms:
+    if not w.conv and nchunks >= 64 and scan_ctas < sms:
         return 2 * min(4, nchunks // 32)
-    return 2
+    return 3 if w.conv else 2
 
 
 def kernel_sources_sha1():
