@@ -56,6 +56,9 @@
 // fp16 when every quarter product of α exceeds 2^-14, bf16 (fp32 range)
 // otherwise, chosen per chunk. The fp16 operands require |S| and |v| < 6e4.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <type_traits>
 
@@ -110,6 +113,9 @@ constexpr int P_END = 114688;
 constexpr int P_AINV = 0;
 constexpr int P_KES = P_Z;            // K_end staged for its bulk store (Z is written after the store has read it)
 constexpr int P_QTS = P_KM;           // Q̄ᵀ staged for its bulk store (after the Gram products have read K̃_mid)
+constexpr int P_ALPHA = P_EB;         // α of the next item (fp32 [64 tok][128 ch], 32 KB), loaded by TMA once
+                                      // the Y/U_w products have read Ē and Z; read by pass 1
+static_assert(P_ALPHA + C * D * 4 == P_END, "α tile over the Ē and Z tiles");
 constexpr int P_YS = P_GM;            // Yᵀ then U_wᵀ (16 KB each), staged for the bulk stores
 constexpr int P_AQS = 16384;          // −Aqk (8 KB) staged for its bulk store: in Gb's block 1,
                                       // read only as don't-care rows by the level-2 products
@@ -222,9 +228,11 @@ __device__ __forceinline__ size_t slot_index(SlotMap m, int bh, int j) {
 // (zero before the launch), so that CTAs which start late take fewer.
 template <bool F16IN>
 __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
-                                                           int* counter) {
+                                                           int* counter, const __grid_constant__ CUtensorMap amap,
+                                                           int use_amap) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + P_BAR);
+  uint64_t* bar_a = bar + 1;            // the α tile has landed
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + P_TMEMP);
   int* sflag = reinterpret_cast<int*>(smem + P_FLAG);
   float* sPq = reinterpret_cast<float*>(smem + P_PQ);
@@ -239,6 +247,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   const int n_items = a.B * a.Hv * n_seg;
   if (tid == 0) {
     mbar_init(bar, 1);
+    mbar_init(bar_a, 1);
     fence_mbar_init();
     *sflag = 0;
     *s_item = counter ? atomicAdd(counter, 1) : 0;
@@ -294,19 +303,40 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     kk[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
     qq[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
   };
+  // The per-channel α tile of an item comes by one TMA copy (rows of the
+  // tensor map [B·T][H_v][128]), requested by thread 0 one item ahead.
+  auto fetch_alpha = [&](int item_) {
+    const Item nx = decode_item(a, c_begin, item_);
+    mbar_arrive_expect_tx(bar_a, C * D * 4);
+    tma_load_3d(smem + P_ALPHA, &amap, 0, nx.h, nx.bi * a.T + nx.t0, bar_a);
+  };
+  uint32_t phase_a = 0;
   auto load_alpha_key0 = [&](int item_) {
     const Item it = decode_item(a, c_begin, item_);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const bool ok = it.Lc == C || i0 + u < it.Lc;
-      const float4 al = ok ? gate4(src.alpha, gate_row(it, u), c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
-      f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
-    }
-#pragma unroll
     for (int u = 0; u < 4; ++u) load_key1(it, u, u);
+    if (use_amap) {
+      wait_mma(bar_a, phase_a, sflag);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool ok = it.Lc == C || i0 + u < it.Lc;    // rows past the sequence's end: α = 1
+        const float4 al = ok ? *reinterpret_cast<const float4*>(smem + P_ALPHA + (i0 + u) * (D * 4) + c0 * 4)
+                             : make_float4(1.f, 1.f, 1.f, 1.f);
+        f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool ok = it.Lc == C || i0 + u < it.Lc;
+        const float4 al = ok ? gate4(src.alpha, gate_row(it, u), c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
+        f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
+      }
+    }
   };
 
   uint32_t phase = 0;
+  if (use_amap && tid == 0 && (counter ? *s_item : (int)blockIdx.x) < n_items)
+    fetch_alpha(counter ? *s_item : (int)blockIdx.x);
   for (int item = counter ? *s_item : (int)blockIdx.x; item < n_items;) {
     const Item it = decode_item(a, c_begin, item);
     uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + slot_index(sm, it.bh, it.cl) * SLOT;
@@ -669,6 +699,11 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
     __syncwarp();
     wait_mma(bar, phase, sflag);
+    // the products have read Ē and Z: their space takes the next item's α
+    if (use_amap && tid == 0) {
+      const int nx = counter ? *s_item : item + (int)gridDim.x;
+      if (nx < n_items) fetch_alpha(nx);
+    }
     {
       // warps 0..3: Yᵀ rows (key lanes); warps 4..7: U_wᵀ rows (dv lanes),
       // staged in the (now free) Gram operand space and stored by two bulk
@@ -1216,6 +1251,30 @@ cudaError_t launch_dependent(void (*kernel)(Args...), int grid, int block, size_
 }
 }  // namespace
 
+namespace {
+// Tensor map of the per-channel α gates [B·T][H_v][128] fp32 for the prep's
+// tile loads (box: 64 tokens × 1 head × 128 channels). false if the driver
+// entry point is unavailable (the prep then reads α with plain loads).
+bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
+  static PFN_cuTensorMapEncodeTiled encode = [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      fn = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+  }();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.Hv, (cuuint64_t)a.B * (cuuint64_t)a.T};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)a.Hv * D * 4};   // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(a.alpha), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
 // Runs the chunks in segments when the workspace holds fewer chunks than the
 // sequence has; the state is carried between segments through S_T (or, when
 // S_T is NULL, through the end of the workspace). Workspace: status word and
@@ -1272,6 +1331,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   // occupancy calculator reports one for any kernel that allocates tensor
   // memory, so the count is set here.
   const int prep_ctas = sms * 2;
+  CUtensorMap amap{};
+  const int use_amap = a.gate_mode != GDN2_GATES_GDN && a.alpha != nullptr && encode_alpha_map(a, &amap) ? 1 : 0;
   const int qp_groups = (2 * a.Hqk + a.Hv) * (D / 8);
 
   // overlapped segments: whole sequence in the workspace, idle SMs beside the
@@ -1313,13 +1374,14 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       ap.qkv_f16 = 1;
       ap.conv_w = nullptr;
       ap.l2norm = 0;
-      chunk_prep_kernel<true><<<grid, NP, P_SMEM, s>>>(ap, c0, n, sm, counter);
+      chunk_prep_kernel<true><<<grid, NP, P_SMEM, s>>>(ap, c0, n, sm, counter, amap, use_amap);
     } else if (nseg_ov > 0 && k > 0) {
-      if ((e = launch_dependent(chunk_prep_kernel<false>, grid, NP, P_SMEM, s, a, c0, n, sm, counter)) !=
+      if ((e = launch_dependent(chunk_prep_kernel<false>, grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap,
+                                use_amap)) !=
           cudaSuccess)
         return e;
     } else {
-      chunk_prep_kernel<false><<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter);
+      chunk_prep_kernel<false><<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter, amap, use_amap);
     }
     scan<<<scan_ctas, scan_threads, scan_smem, s>>>(a, c0, n, sm, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

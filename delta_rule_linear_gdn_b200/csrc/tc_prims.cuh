@@ -224,6 +224,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       : "memory");
 }
 
+// Tiled tensor copy global → shared of one box of a 3-D tensor map (no
+// multicast), completing on `mbar` as transactions. The innermost coordinate
+// x times the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* tmap, int x, int y, int z, uint64_t* mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n"
+      ::"r"(smem_u32(dst_smem)), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(mbar))
+      : "memory");
+}
+
 // Bulk (non-tensor) asynchronous copy shared → global of `bytes` (multiple of
 // 16, both addresses 16-byte aligned), tracked by the issuing thread's bulk
 // groups: commit, then wait until the source may be overwritten (.read) or
