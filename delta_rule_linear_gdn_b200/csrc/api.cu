@@ -32,6 +32,7 @@ gdn2_status check_common(const gdn2_params* p, bool decode) {
   if (p->qkv_dtype != GDN2_F32 && p->qkv_dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
   if (p->o_dtype != GDN2_F32 && p->o_dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
   if (p->gate_mode < GDN2_GATES_FULL || p->gate_mode > GDN2_GATES_GDN) return GDN2_ERR_INVALID_ARG;
+  if (p->gate_logits != 0 && p->gate_logits != 1) return GDN2_ERR_INVALID_ARG;
   if (p->precision != GDN2_PREC_DEFAULT && p->precision != GDN2_PREC_FP32) return GDN2_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return GDN2_ERR_INVALID_ARG;
   if (p->d_k != p->d_v || !supported_dim(p->d_k)) return GDN2_ERR_UNSUPPORTED;
@@ -51,9 +52,10 @@ Sizes sizes(const gdn2_params* p, size_t tokens) {
   const size_t dk = p->d_k, dv = p->d_v;
   s.qk = tokens * p->H_qk * dk * dsize(p->qkv_dtype);
   s.v = tokens * p->H_v * dv * dsize(p->qkv_dtype);
-  s.ga = tokens * p->H_v * (p->gate_mode == GDN2_GATES_GDN ? 1 : dk) * 4;
-  s.gb = tokens * p->H_v * (p->gate_mode == GDN2_GATES_FULL ? dk : 1) * 4;
-  s.gw = p->gate_mode == GDN2_GATES_FULL ? tokens * p->H_v * dv * 4 : 0;
+  const size_t gsz = p->gate_logits ? 2 : 4;   // bf16 logits or fp32 values
+  s.ga = tokens * p->H_v * (p->gate_mode == GDN2_GATES_GDN ? 1 : dk) * gsz;
+  s.gb = tokens * p->H_v * (p->gate_mode == GDN2_GATES_FULL ? dk : 1) * gsz;
+  s.gw = p->gate_mode == GDN2_GATES_FULL ? tokens * p->H_v * dv * gsz : 0;
   s.st = (size_t)p->B * p->H_v * dk * dv * 4;
   return s;
 }
@@ -74,6 +76,7 @@ ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, co
   a.qkv_T = p->T;
   a.qkv_t0 = 0;
   a.qkv_f16 = 0;
+  a.gate_logits = p->gate_logits;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S0 = S0; a.o = o; a.ST = S_T;
   a.workspace = ws; a.ws_bytes = ws_bytes;
   return a;
@@ -186,7 +189,7 @@ gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k,
 
   DecodeArgs a;
   a.B = p->B; a.Hqk = p->H_qk; a.Hv = p->H_v; a.d = p->d_k; a.scale = p->scale;
-  a.gate_mode = p->gate_mode; a.l2norm = p->l2norm_qk != 0;
+  a.gate_mode = p->gate_mode; a.l2norm = p->l2norm_qk != 0; a.gate_logits = p->gate_logits;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S = S; a.o = o;
   cudaError_t e = launch_decode(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16,
                                 static_cast<cudaStream_t>(stream));

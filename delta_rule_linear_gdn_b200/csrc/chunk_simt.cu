@@ -117,8 +117,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         qv = load_conv(qg + qk0, qk_tok, t, conv ? wq + c * 4 : nullptr, conv);
         kv = load_conv(kg + qk0, qk_tok, t, conv ? wk + c * 4 : nullptr, conv);
         const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
-        gv = logf(mode == GDN2_GATES_GDN ? a.alpha[gt] : a.alpha[gt * D + c]);
-        bv = (mode == GDN2_GATES_FULL) ? a.b[gt * D + c] : a.b[gt];
+        gv = logf(gate_at(a.alpha, mode == GDN2_GATES_GDN ? gt : gt * D + c, a.gate_logits));
+        bv = gate_at(a.b, (mode == GDN2_GATES_FULL) ? gt * D + c : gt, a.gate_logits);
       }
       sq[i * DP + c] = qv;
       sk[i * DP + c] = kv;
@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
         const float vv = load_conv(vg + (size_t)bi * a.T * v_tok + (size_t)h * D + col0 + c, v_tok, t,
                                    conv ? wv + (col0 + c) * 4 : nullptr, conv);
-        const float wv_ = (mode == GDN2_GATES_FULL) ? a.w[gt * D + col0 + c] : a.b[gt];
+        const float wv_ = (mode == GDN2_GATES_FULL) ? gate_at(a.w, gt * D + col0 + c, a.gate_logits)
+                                                    : gate_at(a.b, gt, a.gate_logits);
         zv = wv_ * vv;
       }
       sz[i * DVT + c] = zv;

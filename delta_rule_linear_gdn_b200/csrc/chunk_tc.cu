@@ -191,10 +191,22 @@ __device__ __forceinline__ void unpack4_in(uint2 u, float* x) {
     unpack4_bf16(u, x);
 }
 
-// fp32 gate of one token for 4 channels, or the token's scalar gate broadcast.
+// Gate of one token for 4 channels, or the token's scalar gate broadcast: the
+// fp32 values, or σ of the bf16 logits (LG).
+template <bool LG>
 __device__ __forceinline__ float4 gate4(const float* g, size_t gt, int c0, bool per_channel) {
-  if (per_channel) return __ldg(reinterpret_cast<const float4*>(g + gt * D + c0));
-  const float s = __ldg(g + gt);
+  if (!LG) {
+    if (per_channel) return __ldg(reinterpret_cast<const float4*>(g + gt * D + c0));
+    const float s = __ldg(g + gt);
+    return make_float4(s, s, s, s);
+  }
+  const uint16_t* h = reinterpret_cast<const uint16_t*>(g);
+  if (per_channel) {
+    float x[4];
+    unpack4_bf16(__ldg(reinterpret_cast<const uint2*>(h + gt * D + c0)), x);
+    return make_float4(sigmoid_f32(x[0]), sigmoid_f32(x[1]), sigmoid_f32(x[2]), sigmoid_f32(x[3]));
+  }
+  const float s = sigmoid_f32(__uint_as_float((uint32_t)__ldg(h + gt) << 16));
   return make_float4(s, s, s, s);
 }
 
@@ -226,7 +238,7 @@ __device__ __forceinline__ size_t slot_index(SlotMap m, int bh, int j) {
 // Items are taken in order (chunk-major, value head fastest): by a fixed stride
 // of the grid, or, with `counter`, one at a time from that device counter
 // (zero before the launch), so that CTAs which start late take fewer.
-template <bool F16IN>
+template <bool F16IN, bool LG>
 __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
                                                            int* counter, const __grid_constant__ CUtensorMap amap,
                                                            int use_amap) {
@@ -299,7 +311,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   auto load_key1 = [&](const Item& it, int u, int s) {
     const bool ok = it.Lc == C || i0 + u < it.Lc;
     const size_t tq = qkv_tok(it, u) * a.Hqk + it.hq;
-    bq[s] = ok ? gate4(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+    bq[s] = ok ? gate4<LG>(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
     kk[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
     qq[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
   };
@@ -307,7 +319,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   // tensor map [B·T][H_v][128]), requested by thread 0 one item ahead.
   auto fetch_alpha = [&](int item_) {
     const Item nx = decode_item(a, c_begin, item_);
-    mbar_arrive_expect_tx(bar_a, C * D * 4);
+    mbar_arrive_expect_tx(bar_a, C * D * (LG ? 2 : 4));
     tma_load_3d(smem + P_ALPHA, &amap, 0, nx.h, nx.bi * a.T + nx.t0, bar_a);
   };
   uint32_t phase_a = 0;
@@ -320,15 +332,21 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const bool ok = it.Lc == C || i0 + u < it.Lc;    // rows past the sequence's end: α = 1
-        const float4 al = ok ? *reinterpret_cast<const float4*>(smem + P_ALPHA + (i0 + u) * (D * 4) + c0 * 4)
-                             : make_float4(1.f, 1.f, 1.f, 1.f);
+        float4 al = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (ok && LG) {
+          float x[4];
+          unpack4_bf16(*reinterpret_cast<const uint2*>(smem + P_ALPHA + (i0 + u) * (D * 2) + c0 * 2), x);
+          al = make_float4(sigmoid_f32(x[0]), sigmoid_f32(x[1]), sigmoid_f32(x[2]), sigmoid_f32(x[3]));
+        } else if (ok) {
+          al = *reinterpret_cast<const float4*>(smem + P_ALPHA + (i0 + u) * (D * 4) + c0 * 4);
+        }
         f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
       }
     } else {
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const bool ok = it.Lc == C || i0 + u < it.Lc;
-        const float4 al = ok ? gate4(src.alpha, gate_row(it, u), c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
+        const float4 al = ok ? gate4<LG>(src.alpha, gate_row(it, u), c0, alpha_pc) : make_float4(1.f, 1.f, 1.f, 1.f);
         f[u][0] = al.x; f[u][1] = al.y; f[u][2] = al.z; f[u][3] = al.w;
       }
     }
@@ -483,7 +501,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const bool ok = it.Lc == C || i0 + u < it.Lc;
-      wv[u] = ok ? gate4(src.w, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+      wv[u] = ok ? gate4<LG>(src.w, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
       vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
                  : make_uint2(0, 0);
     }
@@ -1252,10 +1270,11 @@ cudaError_t launch_dependent(void (*kernel)(Args...), int grid, int block, size_
 }  // namespace
 
 namespace {
-// Tensor map of the per-channel α gates [B·T][H_v][128] fp32 for the prep's
+// Tensor map of the per-channel α gates [B·T][H_v][128] (fp32, or bf16 logits) for the prep's
 // tile loads (box: 64 tokens × 1 head × 128 channels). false if the driver
 // entry point is unavailable (the prep then reads α with plain loads).
 bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
+  const cuuint64_t esz = a.gate_logits ? 2 : 4;
   static PFN_cuTensorMapEncodeTiled encode = [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -1266,10 +1285,11 @@ bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
   }();
   if (encode == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.Hv, (cuuint64_t)a.B * (cuuint64_t)a.T};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)a.Hv * D * 4};   // bytes, dims 1 and 2
+  const cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)a.Hv * D * esz};   // bytes, dims 1 and 2
   const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(a.alpha), dims, strides, box, estr,
+  return encode(m, a.gate_logits ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                const_cast<float*>(a.alpha), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1303,7 +1323,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   if (seg < 1) return cudaErrorInvalidValue;
   __half* qkv = reinterpret_cast<__half*>(ws + WS_HEAD + (size_t)BH * seg * SLOT);
 
-  for (auto prep : {chunk_prep_kernel<false>, chunk_prep_kernel<true>}) {
+  for (auto prep : {chunk_prep_kernel<false, false>, chunk_prep_kernel<true, false>, chunk_prep_kernel<false, true>,
+                     chunk_prep_kernel<true, true>}) {
     if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) != cudaSuccess)
       return e;
     // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
@@ -1374,14 +1395,16 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       ap.qkv_f16 = 1;
       ap.conv_w = nullptr;
       ap.l2norm = 0;
-      chunk_prep_kernel<true><<<grid, NP, P_SMEM, s>>>(ap, c0, n, sm, counter, amap, use_amap);
+      (a.gate_logits ? chunk_prep_kernel<true, true> : chunk_prep_kernel<true, false>)<<<grid, NP, P_SMEM, s>>>(
+          ap, c0, n, sm, counter, amap, use_amap);
     } else if (nseg_ov > 0 && k > 0) {
-      if ((e = launch_dependent(chunk_prep_kernel<false>, grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap,
-                                use_amap)) !=
+      if ((e = launch_dependent(a.gate_logits ? chunk_prep_kernel<false, true> : chunk_prep_kernel<false, false>,
+                                grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap, use_amap)) !=
           cudaSuccess)
         return e;
     } else {
-      chunk_prep_kernel<false><<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter, amap, use_amap);
+      (a.gate_logits ? chunk_prep_kernel<false, true> : chunk_prep_kernel<false, false>)<<<grid, NP, P_SMEM, s>>>(
+          a, c0, n, sm, counter, amap, use_amap);
     }
     scan<<<scan_ctas, scan_threads, scan_smem, s>>>(a, c0, n, sm, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

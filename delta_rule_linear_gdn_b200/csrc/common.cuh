@@ -21,6 +21,13 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // The epsilon of the fused L2 normalisation: x · (Σx² + eps)^(−1/2).
 constexpr float kL2Eps = 1e-6f;
 
+// Gate element i of a gate tensor: the fp32 value, or σ(x) of the bf16 logit
+// x when the gates are given as logits (gdn2_params.gate_logits).
+__device__ __forceinline__ float sigmoid_f32(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float gate_at(const float* g, size_t i, bool logits) {
+  return logits ? sigmoid_f32(__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[i])) : g[i];
+}
+
 // Arguments of one launch, already validated by the host entry points.
 struct ChunkArgs {
   int B, T, Hqk, Hv, dk, dv, chunk;
@@ -39,6 +46,7 @@ struct ChunkArgs {
   // values when the tensor-core prefill reads its own preprocessed copies),
   // and whether they hold fp16 instead of the input dtype.
   int qkv_T, qkv_t0, qkv_f16;
+  int gate_logits;   // gates are bf16 logits (σ applied in the kernels)
 };
 
 struct DecodeArgs {
@@ -50,6 +58,7 @@ struct DecodeArgs {
   const float *alpha, *b, *w;
   float* S;
   void* o;
+  int gate_logits;   // gates are bf16 logits (σ applied in the kernels)
 };
 
 // Launchers (return cudaSuccess or the launch error).

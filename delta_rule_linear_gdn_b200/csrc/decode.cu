@@ -64,11 +64,11 @@ decode_kernel(DecodeArgs a) {
   for (int i = tid; i < D; i += NT) {
     s_q[i] = to_f32(qg[i]);
     s_k[i] = to_f32(kg[i]);
-    s_a[i] = (a.gate_mode == GDN2_GATES_GDN) ? a.alpha[bh] : a.alpha[(size_t)bh * D + i];
+    s_a[i] = gate_at(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? (size_t)bh : (size_t)bh * D + i, a.gate_logits);
   }
-  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : a.b[bh];
+  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at(a.b, bh, a.gate_logits);
   for (int j = tid; j < COLS; j += NT) {
-    const float wj = (a.gate_mode == GDN2_GATES_FULL) ? a.w[(size_t)bh * D + col0 + j] : beta;
+    const float wj = (a.gate_mode == GDN2_GATES_FULL) ? gate_at(a.w, (size_t)bh * D + col0 + j, a.gate_logits) : beta;
     s_z[j] = wj * to_f32(vg[j]);
   }
   __syncthreads();
@@ -100,7 +100,7 @@ decode_kernel(DecodeArgs a) {
   const float iq = s_scalar[0], ik = s_scalar[1], kq = s_scalar[2];
   for (int i = tid; i < D; i += NT) {
     const float kk = s_k[i] * ik;
-    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? a.b[(size_t)bh * D + i] : beta;
+    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? gate_at(a.b, (size_t)bh * D + i, a.gate_logits) : beta;
     s_e[i] = bb * kk;
   }
   __syncthreads();

@@ -41,7 +41,7 @@ class Params(ctypes.Structure):
         ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("chunk", ctypes.c_int),
         ("scale", ctypes.c_float), ("qkv_dtype", ctypes.c_int), ("o_dtype", ctypes.c_int),
         ("gate_mode", ctypes.c_int), ("precision", ctypes.c_int), ("l2norm_qk", ctypes.c_int),
-        ("conv_w", ctypes.c_void_p),
+        ("conv_w", ctypes.c_void_p), ("gate_logits", ctypes.c_int),
     ]
 
 
@@ -109,11 +109,11 @@ def _stream_handle(stream):
 
 
 def make_params(B, T, H_qk, H_v, d_k, d_v, *, chunk=64, scale=1.0, qkv_dtype=BF16, o_dtype=BF16,
-                gate_mode="full", precision="default", l2norm_qk=False, conv_w=None) -> Params:
+                gate_mode="full", precision="default", l2norm_qk=False, conv_w=None, gate_logits=False) -> Params:
     return Params(int(B), int(T), int(H_qk), int(H_v), int(d_k), int(d_v), int(chunk), float(scale),
                   int(qkv_dtype), int(o_dtype), GATES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode),
                   PRECISION[precision] if isinstance(precision, str) else int(precision),
-                  1 if l2norm_qk else 0, _ptr(conv_w))
+                  1 if l2norm_qk else 0, _ptr(conv_w), 1 if gate_logits else 0)
 
 
 def _check(t, name, dtype=None):
@@ -133,19 +133,23 @@ def chunk_fwd_workspace(params: Params) -> int:
 
 def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_mode="full",
               precision="default", l2norm_qk=False, conv_w=None, o_dtype=None, o=None, S_T=None,
-              workspace=None, stream=None, want_state=True):
-    """Chunked prefill. q,k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; gates fp32 per
-    ``gate_mode``; S0 [B,H_v,d_k,d_v] fp32 or None. Returns (o, S_T)."""
+              workspace=None, stream=None, want_state=True, gate_logits=False):
+    """Chunked prefill. q,k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; gates per
+    ``gate_mode``: fp32 values, or bf16 logits with ``gate_logits`` (the kernels
+    apply the sigmoid); S0 [B,H_v,d_k,d_v] fp32 or None. Returns (o, S_T)."""
     B, T, H_qk, d_k = q.shape
     H_v, d_v = v.shape[2], v.shape[3]
     o_dtype = q.dtype if o_dtype is None else o_dtype
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check(t, name, q.dtype)
-    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S0", S0), ("conv_w", conv_w)):
+    gdt = torch.bfloat16 if gate_logits else torch.float32
+    for name, t in (("alpha", alpha), ("b", b), ("w", w)):
+        _check(t, name, gdt)
+    for name, t in (("S0", S0), ("conv_w", conv_w)):
         _check(t, name, torch.float32)
     p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
                     o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, precision=precision,
-                    l2norm_qk=l2norm_qk, conv_w=conv_w)
+                    l2norm_qk=l2norm_qk, conv_w=conv_w, gate_logits=gate_logits)
     if o is None:
         o = torch.empty((B, T, H_v, d_v), dtype=o_dtype, device=q.device)
     if S_T is None and want_state:
@@ -165,18 +169,22 @@ def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_m
 
 
 def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_qk=False, o_dtype=None,
-                o=None, stream=None):
-    """One decode step. q,k [B,H_qk,d_k]; v [B,H_v,d_v]; gates fp32 without the
-    T axis; S [B,H_v,d_k,d_v] fp32 updated in place. Returns o [B,H_v,d_v]."""
+                o=None, stream=None, gate_logits=False):
+    """One decode step. q,k [B,H_qk,d_k]; v [B,H_v,d_v]; gates without the T
+    axis (fp32 values, or bf16 logits with ``gate_logits``); S [B,H_v,d_k,d_v]
+    fp32 updated in place. Returns o [B,H_v,d_v]."""
     B, H_qk, d_k = q.shape
     H_v, d_v = v.shape[1], v.shape[2]
     o_dtype = q.dtype if o_dtype is None else o_dtype
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check(t, name, q.dtype)
-    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S", S)):
-        _check(t, name, torch.float32)
+    gdt = torch.bfloat16 if gate_logits else torch.float32
+    for name, t in (("alpha", alpha), ("b", b), ("w", w)):
+        _check(t, name, gdt)
+    _check(S, "S", torch.float32)
     p = make_params(B, 1, H_qk, H_v, d_k, d_v, scale=scale, qkv_dtype=_dtype_code(q.dtype),
-                    o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk)
+                    o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk,
+                    gate_logits=gate_logits)
     if o is None:
         o = torch.empty((B, H_v, d_v), dtype=o_dtype, device=q.device)
     _check(o, "o", o_dtype)
@@ -188,7 +196,7 @@ def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_
 
 
 def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=64, scale=1.0,
-                      gate_mode="full", l2norm_qk=False, conv_w=None, stream=None):
+                      gate_mode="full", l2norm_qk=False, conv_w=None, stream=None, gate_logits=False):
     """Chunked prefill through ``gdn2_chunk_fwd_noalloc``: the library takes the
     kernel's scratch from its own fixed device array, so nothing is allocated
     for the call. ``o`` and ``S_T`` (or None) are caller-provided outputs (the
@@ -201,11 +209,15 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=
     H_v, d_v = v.shape[2], v.shape[3]
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check(t, name, q.dtype)
-    for name, t in (("alpha", alpha), ("b", b), ("w", w), ("S0", S0), ("S_T", S_T), ("conv_w", conv_w)):
+    gdt = torch.bfloat16 if gate_logits else torch.float32
+    for name, t in (("alpha", alpha), ("b", b), ("w", w)):
+        _check(t, name, gdt)
+    for name, t in (("S0", S0), ("S_T", S_T), ("conv_w", conv_w)):
         _check(t, name, torch.float32)
     _check(o, "o")
     p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
-                    o_dtype=_dtype_code(o.dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk, conv_w=conv_w)
+                    o_dtype=_dtype_code(o.dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk, conv_w=conv_w,
+                    gate_logits=gate_logits)
     st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
             _ptr(S_T), _stream_handle(stream))
     if st != OK:

@@ -95,14 +95,16 @@ def _qkv_dtype(w: Workload):
     return torch.bfloat16 if w.qkv_dtype == "bf16" else torch.float32
 
 
-def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: str = "full"):
+def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: str = "full",
+                gate_logits: bool = False):
     """Draw one batch of inputs for workload ``w``.
 
     gate_mode "full": alpha, b [B,T,Hv,dk], w [B,T,Hv,dv].
     gate_mode "kda":  alpha [B,T,Hv,dk] (mean alpha_mu), b = beta [B,T,Hv], w = None.
     gate_mode "gdn":  alpha [B,T,Hv] (mean 4), b = beta [B,T,Hv], w = None.
     Returns a dict of tensors on ``device`` (q,k,v in the workload's dtype;
-    gates, S0 and conv weights float32).
+    gates float32 sigmoids of normal draws, or with ``gate_logits`` those
+    draws themselves rounded to bf16; S0 and conv weights float32).
     """
     if seed is None:
         seed = WORKLOADS.index(BY_NAME[w.name]) if w.name in BY_NAME else 0
@@ -118,17 +120,18 @@ def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: s
     v = _normal((B, T, Hv, d), _gen(seed, 3, dev), dev)
     dt = _qkv_dtype(w)
     out["q"], out["k"], out["v"] = q.to(dt), k.to(dt), v.to(dt)
+    gate = (lambda x: x.to(torch.bfloat16)) if gate_logits else torch.sigmoid
     if gate_mode == "full":
-        out["alpha"] = torch.sigmoid(_normal((B, T, Hv, d), _gen(seed, 4, dev), dev, mean=w.alpha_mu))
-        out["b"] = torch.sigmoid(_normal((B, T, Hv, d), _gen(seed, 5, dev), dev))
-        out["w"] = torch.sigmoid(_normal((B, T, Hv, d), _gen(seed, 6, dev), dev))
+        out["alpha"] = gate(_normal((B, T, Hv, d), _gen(seed, 4, dev), dev, mean=w.alpha_mu))
+        out["b"] = gate(_normal((B, T, Hv, d), _gen(seed, 5, dev), dev))
+        out["w"] = gate(_normal((B, T, Hv, d), _gen(seed, 6, dev), dev))
     elif gate_mode == "kda":
-        out["alpha"] = torch.sigmoid(_normal((B, T, Hv, d), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
-        out["b"] = torch.sigmoid(_normal((B, T, Hv), _gen(seed, 5, dev), dev))
+        out["alpha"] = gate(_normal((B, T, Hv, d), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
+        out["b"] = gate(_normal((B, T, Hv), _gen(seed, 5, dev), dev))
         out["w"] = None
     elif gate_mode == "gdn":
-        out["alpha"] = torch.sigmoid(_normal((B, T, Hv), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
-        out["b"] = torch.sigmoid(_normal((B, T, Hv), _gen(seed, 5, dev), dev))
+        out["alpha"] = gate(_normal((B, T, Hv), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
+        out["b"] = gate(_normal((B, T, Hv), _gen(seed, 5, dev), dev))
         out["w"] = None
     else:
         raise ValueError(gate_mode)
@@ -144,12 +147,13 @@ def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: s
 
 
 def make_decode_pool(w: Workload, pool: int = 16, seed: int | None = None, device="cpu",
-                     gate_mode: str = "full"):
+                     gate_mode: str = "full", gate_logits: bool = False):
     """Per-step decode inputs: ``pool`` independent one-token step sets, cycled by
     the caller, plus the initial state. Tensors carry a leading pool axis."""
     if seed is None:
         seed = 3
-    steps = make_inputs(replace(w, T=pool, s0="zeros"), seed=seed, device=device, gate_mode=gate_mode)
+    steps = make_inputs(replace(w, T=pool, s0="zeros"), seed=seed, device=device, gate_mode=gate_mode,
+                        gate_logits=gate_logits)
     # [B, pool, ...] -> [pool, B, ...]
     for key in ("q", "k", "v", "alpha", "b", "w"):
         if steps[key] is not None:

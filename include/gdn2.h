@@ -22,8 +22,9 @@
  *    owned by the caller. The library allocates nothing, keeps no state
  *    between calls and never synchronises: all work is enqueued on `stream`
  *    (a cudaStream_t passed as void*; NULL = the legacy default stream).
- *  - q, k, v, o are bf16 or fp32 (see gdn2_params); gates, S0/S_T/S, conv
- *    weights are always fp32.
+ *  - q, k, v, o are bf16 or fp32 (see gdn2_params); gates are fp32 values or
+ *    bf16 logits (gdn2_params.gate_logits); S0/S_T/S and conv weights are
+ *    always fp32.
  *  - Every pointer must be 16-byte aligned.
  *  - Arguments are validated on the host before any launch. A rejected call
  *    enqueues nothing and returns GDN2_ERR_INVALID_ARG (bad pointer, shape,
@@ -97,6 +98,13 @@ typedef struct {
                      recurrence ("Gated DeltaNet: o mixer em 48 das 64
                      camadas", Conceito). Tap 3 weights the current token.
                      gdn2_chunk_fwd only.                                     */
+  int gate_logits; /* 0: alpha, b, w hold the gate values (fp32). 1: they hold
+                     bf16 logits x and the kernels use σ(x) = 1 / (1 + e^(−x)),
+                     the sigmoid the pages put on the gate projections
+                     ("BigSaaS – Posts", section "Implementação Prática: Como
+                     Funciona a Camada de Atenção do DeltaNet-2"); same
+                     shapes, half the bytes. The pointers keep their float*
+                     type and are read as bf16.                               */
 } gdn2_params;
 
 /* Human-readable name of a status code (static string, never NULL). */

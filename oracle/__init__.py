@@ -21,6 +21,10 @@ Functions and the passages they follow:
   assume normalised keys: "Uma análise das variantes de atenção linear da
   família DeltaNet", Notação e ordem da derivação).
 * :func:`preprocess` -- conv then L2 norm, in that order.
+* :func:`gates_from_logits` -- the gates as the sigmoid of their projections'
+  outputs ("BigSaaS – Posts", section "Implementação Prática: Como Funciona a
+  Camada de Atenção do DeltaNet-2": erase and write gates pass through a
+  sigmoid so that they lie between 0 and 1).
 
 Pins: every function above is checked in ``tests/test_oracle_pins.py`` against
 closed forms, special cases and brute force (no function is parity-unpinned).
@@ -156,6 +160,13 @@ def preprocess(q, k, v, conv_w=None, l2norm_qk: bool = False):
         q = l2norm(q)
         k = l2norm(k)
     return q, k, v
+
+
+def gates_from_logits(x):
+    """σ(x) = 1 / (1 + e^(−x)) elementwise, float64 (x: gate logits)."""
+    x = _f64(x)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-x))
 
 
 def rel_err(got, ref) -> float:

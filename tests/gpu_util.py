@@ -14,22 +14,26 @@ def np64(t):
     return None if t is None else t.detach().to(torch.float64).cpu().numpy()
 
 
-def oracle_gates(mode, alpha, b, w, d_k, d_v):
-    """Per-channel float64 gates for the oracle from the tensors the kernel gets."""
+def oracle_gates(mode, alpha, b, w, d_k, d_v, gate_logits=False):
+    """Per-channel float64 gates for the oracle from the tensors the kernel gets
+    (bf16 logits pass through the oracle's sigmoid first)."""
+    f = oracle.gates_from_logits if gate_logits else (lambda x: x)
+    alpha, b = f(np64(alpha)), f(np64(b))
+    w = None if w is None else f(np64(w))
     if mode == "full":
-        return np64(alpha), np64(b), np64(w)
-    return oracle.expand_tied_gates(mode, np64(alpha), np64(b), d_k, d_v)
+        return alpha, b, w
+    return oracle.expand_tied_gates(mode, alpha, b, d_k, d_v)
 
 
 def oracle_chunk(inp, gate_mode="full", scale=1.0, l2norm_qk=False, S0=None, threads=0,
-                 heads=None):
+                 heads=None, gate_logits=False):
     """Oracle (o, S_T) for a chunk_fwd input dict. ``heads`` optionally restricts
     to a list of (sequence, value head) pairs; returns dict keyed by pair then."""
     q, k, v = np64(inp["q"]), np64(inp["k"]), np64(inp["v"])
     d_k, d_v = q.shape[-1], v.shape[-1]
     conv_w = np64(inp.get("conv_w"))
     S0 = np64(inp.get("S0")) if S0 is None else np64(S0)
-    alpha, b, w = oracle_gates(gate_mode, inp["alpha"], inp["b"], inp.get("w"), d_k, d_v)
+    alpha, b, w = oracle_gates(gate_mode, inp["alpha"], inp["b"], inp.get("w"), d_k, d_v, gate_logits)
     if heads is None:
         qp, kp, vp = oracle.preprocess(q, k, v, conv_w, l2norm_qk)
         return oracle.gdn2_forward(qp, kp, vp, alpha, b, w, S0, scale=scale, threads=threads)

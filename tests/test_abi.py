@@ -47,8 +47,12 @@ def test_status_strings_and_version(L):
 
 def _params(**kw):
     base = dict(B=1, T=64, H_qk=1, H_v=1, d_k=16, d_v=16, chunk=16, qkv_dtype=gdn2.F32, o_dtype=gdn2.F32)
+    raw_logits = kw.pop("gate_logits", None)
     base.update(kw)
-    return gdn2.make_params(**base)
+    p = gdn2.make_params(**base)
+    if raw_logits is not None:
+        p.gate_logits = int(raw_logits)   # raw field value, including invalid ones
+    return p
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
@@ -74,6 +78,7 @@ def _call_chunk(L, p, **ptrs):
     (dict(gate_mode=5), gdn2.ERR_INVALID_ARG),
     (dict(precision=3), gdn2.ERR_INVALID_ARG),
     (dict(scale=float("nan")), gdn2.ERR_INVALID_ARG),
+    (dict(gate_logits=2), gdn2.ERR_INVALID_ARG),
 ])
 def test_chunk_rejects_bad_params(L, kw, expect):
     assert _call_chunk(L, _params(**kw)) == expect
@@ -106,6 +111,13 @@ def test_decode_rejects_conv_and_bad_args(L):
     args[6] = None  # S
     assert L.gdn2_decode_step(ctypes.byref(p), *args, None) == gdn2.ERR_INVALID_ARG
     assert L.gdn2_decode_step(None, *[FAKE] * 8, None) == gdn2.ERR_INVALID_ARG
+
+
+def test_gate_logits_field_follows_conv_w():
+    # the C struct ends with conv_w then gate_logits: the mirror keeps that order
+    names = [f[0] for f in gdn2.Params._fields_]
+    assert names[-2:] == ["conv_w", "gate_logits"]
+    assert gdn2.make_params(1, 1, 1, 1, 16, 16, gate_logits=True).gate_logits == 1
 
 
 def test_workspace_query_is_host_only(L):

@@ -387,3 +387,21 @@ def test_rel_err_metric():
     assert oracle.rel_err(ref, ref) == 0.0
     got = ref + np.array([0.0, 0.5])
     assert abs(oracle.rel_err(got, ref) - 0.5 / np.sqrt(12.5)) < 1e-15
+
+
+def test_gates_from_logits_closed_forms():
+    """σ(0) = 1/2, σ(ln 3) = 3/4 and σ(−ln 3) = 1/4 exactly in closed form;
+    σ(x) + σ(−x) = 1; increasing; saturates to 0 and 1 without NaN."""
+    s = oracle.gates_from_logits(np.array([0.0, np.log(3.0), -np.log(3.0)]))
+    np.testing.assert_allclose(s, [0.5, 0.75, 0.25], rtol=0, atol=1e-15)
+    x = _rng(50).standard_normal(1000) * 6.0
+    np.testing.assert_allclose(oracle.gates_from_logits(x) + oracle.gates_from_logits(-x), 1.0, rtol=0,
+                               atol=1e-15)
+    xs = np.sort(x)
+    assert np.all(np.diff(oracle.gates_from_logits(xs)) >= 0)
+    ext = oracle.gates_from_logits(np.array([-1000.0, 1000.0]))
+    assert ext[0] == 0.0 and ext[1] == 1.0
+    # the odds: σ(x) / σ(−x) = e^x
+    xm = x[np.abs(x) < 30]
+    np.testing.assert_allclose(oracle.gates_from_logits(xm) / oracle.gates_from_logits(-xm), np.exp(xm),
+                               rtol=1e-12)

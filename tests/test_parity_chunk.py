@@ -192,6 +192,42 @@ def test_full_width_scan_many_heads(gate_mode):
         assert_close(S[bi:bi + 1, h:h + 1], S_ref, TOL_BF16, f"S_T[{bi},{h}]")
 
 
+@pytest.mark.parametrize("gate_mode", ["full", "kda", "gdn"])
+def test_gate_logits_tensor_core_and_fp32_paths(gate_mode):
+    """Gates given as bf16 logits, σ applied in the kernels: the tensor-core
+    prefill (with its TMA-loaded α tile in the per-channel modes) and the fp32
+    path against the oracle on σ of the same logits; ragged tail, nonzero
+    entry state, two sequences."""
+    w = small(T=200, B=2, H_qk=2, H_v=6, d=128, chunk=64, qkv="bf16", s0="normal")
+    inp = make_inputs(w, seed=47, gate_mode=gate_mode, gate_logits=True)
+    o, S = run(inp, chunk=64, gate_mode=gate_mode, o_dtype=torch.float32, gate_logits=True)
+    o32, S32 = run(inp, chunk=64, gate_mode=gate_mode, o_dtype=torch.float32, gate_logits=True, precision="fp32")
+    o_ref, S_ref = oracle_chunk(inp, gate_mode=gate_mode, gate_logits=True)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(S, S_ref, TOL_BF16, "S_T")
+    assert_close(o32, o_ref, TOL_FP32, "o fp32 path")
+    assert_close(S32, S_ref, TOL_FP32, "S_T fp32 path")
+
+
+def test_gate_logits_long_sequence_overlapped():
+    """Logit gates through the pipelined schedule (few heads, 80 chunks): the
+    same results as the gate values σ(logits) computed ahead on the host, to
+    within the two sigmoids' rounding."""
+    w = small(T=64 * 80, B=1, H_qk=2, H_v=6, d=128, chunk=64, qkv="bf16", s0="normal")
+    inp = make_inputs(w, seed=53, gate_logits=True)
+    o, S = run(inp, chunk=64, o_dtype=torch.float32, gate_logits=True)
+    vals = dict(inp, alpha=torch.sigmoid(inp["alpha"].float()), b=torch.sigmoid(inp["b"].float()),
+                w=torch.sigmoid(inp["w"].float()))
+    o2, S2 = run(vals, chunk=64, o_dtype=torch.float32)
+    ref = oracle_chunk(inp, gate_logits=True, heads=[(0, 0), (0, 5)])
+    for (bi, h), (o_ref, S_ref) in ref.items():
+        assert_close(o[bi:bi + 1, :, h:h + 1], o_ref, TOL_BF16, f"o[{bi},{h}]")
+        assert_close(S[bi:bi + 1, h:h + 1], S_ref, TOL_BF16, f"S_T[{bi},{h}]")
+    for got, want, name in ((o, o2, "o"), (S, S2, "S_T")):
+        rel = ((got - want).abs().max() / want.pow(2).mean().sqrt()).item()
+        assert rel <= 5e-3, (name, rel)
+
+
 def test_decode_steps_equal_chunked_prefill():
     w = small(T=48, B=2, H_qk=2, H_v=4, d=32, s0="normal")
     inp = make_inputs(w, seed=11)

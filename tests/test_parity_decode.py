@@ -39,6 +39,28 @@ def test_decode_steps_vs_oracle(d, gate_mode, qkv):
     assert_close(S, S_ref, TOL_FP32, "S")
 
 
+@pytest.mark.parametrize("d", [16, 128])
+@pytest.mark.parametrize("gate_mode", ["full", "kda", "gdn"])
+def test_decode_gate_logits_vs_oracle(d, gate_mode):
+    """Gates given as bf16 logits (the kernel applies the sigmoid): the oracle
+    takes σ of the same logits in float64."""
+    w = replace(workload(0), B=3, T=5, H_qk=2, H_v=6, d=d, qkv_dtype="bf16", s0="normal")
+    inp = make_inputs(w, seed=d + 7, gate_mode=gate_mode, gate_logits=True)
+    assert inp["alpha"].dtype == torch.bfloat16
+    S = inp["S0"].cuda().clone()
+    outs = []
+    for t in range(w.T):
+        s = {k: (None if v is None else v.cuda()) for k, v in _step_inputs(inp, t).items()}
+        outs.append(gdn2.decode_step(s["q"], s["k"], s["v"], s["alpha"], s["b"], s["w"], S,
+                                     gate_mode=gate_mode, o_dtype=torch.float32, gate_logits=True))
+    torch.cuda.synchronize()
+    a, b, w_ = oracle_gates(gate_mode, inp["alpha"], inp["b"], inp["w"], d, d, gate_logits=True)
+    o_ref, S_ref = oracle.gdn2_forward(np64(inp["q"]), np64(inp["k"]), np64(inp["v"]), a, b, w_,
+                                       np64(inp["S0"]))
+    assert_close(torch.stack(outs, 1), o_ref, TOL_FP32, "o")
+    assert_close(S, S_ref, TOL_FP32, "S")
+
+
 def test_decode_l2norm_and_scale_bf16_out():
     w = replace(workload(0), B=4, T=3, H_qk=1, H_v=3, d=128, qkv_dtype="bf16", s0="normal", conv=True)
     inp = make_inputs(w, seed=3)   # conv=True: raw (unnormalised) q, k
