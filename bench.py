@@ -69,18 +69,18 @@ def peaks():
 
 # ------------------------------------------------------------------ accounting
 
-def prefill_bytes(w, gate_mode="full", o_bytes=2, s0=False):
+def prefill_bytes(w, gate_mode="full", o_bytes=2, s0=False, gate_bytes=4):
     """Algorithmic HBM bytes of one chunk_fwd call: every input read once, every
-    output written once."""
+    output written once (gate_bytes: 4 for fp32 gate values, 2 for bf16 logits)."""
     tok = w.B * w.T
     qkb = 2 if w.qkv_dtype == "bf16" else 4
     n = tok * w.H_qk * w.d * qkb * 2 + tok * w.H_v * w.d * qkb
     if gate_mode == "full":
-        n += tok * w.H_v * w.d * 4 * 3
+        n += tok * w.H_v * w.d * gate_bytes * 3
     elif gate_mode == "kda":
-        n += tok * w.H_v * (w.d + 1) * 4
+        n += tok * w.H_v * (w.d + 1) * gate_bytes
     else:
-        n += tok * w.H_v * 2 * 4
+        n += tok * w.H_v * 2 * gate_bytes
     n += tok * w.H_v * w.d * o_bytes
     n += w.B * w.H_v * w.d * w.d * 4 * (2 if s0 else 1)
     if w.conv:
@@ -343,6 +343,8 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=[PREFILL, "prefill_t4096"],
                     help="prefill workload to time (the small one is for profiler captures)")
     ap.add_argument("--decode-workload", default=DECODE, choices=[DECODE, "decode_b64"])
+    ap.add_argument("--logits-steps", type=int, default=20,
+                    help="timed calls of the T=32768 prefill with bf16 gate logits; 0 skips it")
     ap.add_argument("--conv-steps", type=int, default=5,
                     help="timed calls of the conv + L2 workload (B=8, T=8192); 0 skips it")
     args = ap.parse_args()
@@ -430,6 +432,11 @@ def main():
     if args.conv_steps > 0:
         conv = run_conv(args, dev, stream, barrier, pk, world)
 
+    # ---------------------------------------------------------------- gates as bf16 logits
+    logits = None
+    if args.logits_steps > 0:
+        logits = run_logits(args, w, dev, stream, barrier, pk, world)
+
     # ---------------------------------------------------------------- end to end
     e2e = None
     if args.e2e_steps > 0:
@@ -457,7 +464,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
-            "conv_prefill": conv,
+            "conv_prefill": conv, "prefill_gate_logits": logits,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -542,6 +549,46 @@ def run_conv(args, dev, stream, barrier, pk, world):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes},
             "gpu_launches": 3 * args.conv_steps}
+
+
+def run_logits(args, w, dev, stream, barrier, pk, world):
+    """The headline layer and length with the gates given as bf16 logits (the
+    kernels apply the sigmoid): half the gate bytes of the fp32 values."""
+    import torch
+    from delta_rule_linear_gdn_b200 import gdn2
+    from delta_rule_linear_gdn_b200.inputs import make_inputs
+    rank = int(os.environ.get("RANK", "0"))
+    inp = make_inputs(w, seed=rank_seed(rank), device=dev, gate_logits=True)
+    o = torch.empty((w.B, w.T, w.H_v, w.d), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((w.B, w.H_v, w.d, w.d), dtype=torch.float32, device=dev)
+    p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk, gate_logits=True)
+    ws = torch.empty(max(gdn2.chunk_fwd_workspace(p), 1), dtype=torch.uint8, device=dev)
+
+    def call():
+        gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None, chunk=w.chunk,
+                       o=o, S_T=S_T, workspace=ws, stream=stream, gate_logits=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    torch.cuda.synchronize()
+    barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.logits_steps):
+            call()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    lms = max_over_ranks(c0.elapsed_time(c1) / args.logits_steps, dev)
+    nbytes = prefill_bytes(w, gate_bytes=2)
+    gbs = nbytes / (lms * 1e-3) / 1e9
+    return {"workload": f"{w.name} with the gates as bf16 logits (sigmoid in the kernels)",
+            "ms_per_call": lms, "tokens_per_s": w.B * w.T * world / (lms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes},
+            "gpu_launches": args.logits_steps * tc_launches_per_call(w, gdn2.chunk_fwd_workspace(p), dev)}
 
 
 def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):
