@@ -29,6 +29,10 @@ __device__ __forceinline__ float sigmoid_f32(float x) { return __fdividef(1.f, 1
 __device__ __forceinline__ float gate_at(const float* g, size_t i, bool logits) {
   return logits ? sigmoid_f32(__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[i])) : g[i];
 }
+template <bool LG> __device__ __forceinline__ float gate_at(const float* g, size_t i) {
+  if (LG) return sigmoid_f32(__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[i]));
+  return g[i];
+}
 
 // Arguments of one launch, already validated by the host entry points.
 struct ChunkArgs {

@@ -25,7 +25,7 @@ namespace {
 
 constexpr int kRowGroups = 16;
 
-template <int D, int COLS, typename TIn, typename TOut>
+template <int D, int COLS, typename TIn, typename TOut, bool LG>
 __global__ void __launch_bounds__((COLS / 4) * kRowGroups)
 decode_kernel(DecodeArgs a) {
   constexpr int CG = COLS / 4;            // column groups (float4 each)
@@ -64,11 +64,11 @@ decode_kernel(DecodeArgs a) {
   for (int i = tid; i < D; i += NT) {
     s_q[i] = to_f32(qg[i]);
     s_k[i] = to_f32(kg[i]);
-    s_a[i] = gate_at(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? (size_t)bh : (size_t)bh * D + i, a.gate_logits);
+    s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? (size_t)bh : (size_t)bh * D + i);
   }
-  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at(a.b, bh, a.gate_logits);
+  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at<LG>(a.b, bh);
   for (int j = tid; j < COLS; j += NT) {
-    const float wj = (a.gate_mode == GDN2_GATES_FULL) ? gate_at(a.w, (size_t)bh * D + col0 + j, a.gate_logits) : beta;
+    const float wj = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.w, (size_t)bh * D + col0 + j) : beta;
     s_z[j] = wj * to_f32(vg[j]);
   }
   __syncthreads();
@@ -100,7 +100,7 @@ decode_kernel(DecodeArgs a) {
   const float iq = s_scalar[0], ik = s_scalar[1], kq = s_scalar[2];
   for (int i = tid; i < D; i += NT) {
     const float kk = s_k[i] * ik;
-    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? gate_at(a.b, (size_t)bh * D + i, a.gate_logits) : beta;
+    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.b, (size_t)bh * D + i) : beta;
     s_e[i] = bb * kk;
   }
   __syncthreads();
@@ -164,7 +164,10 @@ template <int D, int COLS, typename TIn, typename TOut>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t s) {
   const int grid = a.B * a.Hv * (D / COLS);
   if (grid == 0) return cudaSuccess;
-  decode_kernel<D, COLS, TIn, TOut><<<grid, (COLS / 4) * kRowGroups, 0, s>>>(a);
+  if (a.gate_logits)
+    decode_kernel<D, COLS, TIn, TOut, true><<<grid, (COLS / 4) * kRowGroups, 0, s>>>(a);
+  else
+    decode_kernel<D, COLS, TIn, TOut, false><<<grid, (COLS / 4) * kRowGroups, 0, s>>>(a);
   return cudaGetLastError();
 }
 
