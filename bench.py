@@ -326,7 +326,8 @@ def config_dict(w):
     return {"workload": f"{w.name}: B={w.B} T={w.T} H_qk={w.H_qk} H_v={w.H_v} d={w.d} chunk={w.chunk} "
                         f"{w.qkv_dtype} q,k,v, fp32 per-channel gates, S0=0",
             "global_batch": w.B, "seq_len": w.T, "parallelism": "independent sequences per GPU",
-            "l2": "no flush: each step reads ~3.5 GB of inputs, > 126 MB L2"}
+            "l2": f"no flush: each step moves {prefill_bytes(w) / 1e9:.2f} GB (inputs read once, "
+                  f"o written once), > 126 MB L2"}
 
 
 # ------------------------------------------------------------------ our arm
