@@ -66,6 +66,26 @@ gdn2_status check_gate_ptrs(const gdn2_params* p, const float* alpha, const floa
   return GDN2_OK;
 }
 
+// Conv history buffers: only with a conv, 16-byte aligned; the outgoing
+// history overlaps nothing else of the call, and no output overlaps the
+// incoming history. `ins` / `outs` are the call's other inputs / outputs.
+struct Range { const void* p; size_t n; };
+gdn2_status check_conv_state(const gdn2_params* p, const Range* ins, int n_in, const Range* outs, int n_out) {
+  const void* hin = p->conv_state_in;
+  void* hout = p->conv_state_out;
+  if (!p->conv_w && (hin || hout)) return GDN2_ERR_INVALID_ARG;
+  if (!aligned16(hin) || !aligned16(hout)) return GDN2_ERR_INVALID_ARG;
+  const size_t hb = (size_t)p->B * 3 * ((size_t)2 * p->H_qk * p->d_k + (size_t)p->H_v * p->d_v) *
+                    dsize(p->qkv_dtype);
+  if (overlaps(hout, hb, hin, hb)) return GDN2_ERR_INVALID_ARG;
+  for (int i = 0; i < n_in; ++i)
+    if (overlaps(hout, hb, ins[i].p, ins[i].n)) return GDN2_ERR_INVALID_ARG;
+  for (int i = 0; i < n_out; ++i)
+    if (overlaps(hout, hb, outs[i].p, outs[i].n) || overlaps(hin, hb, outs[i].p, outs[i].n))
+      return GDN2_ERR_INVALID_ARG;
+  return GDN2_OK;
+}
+
 ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, const void* v,
                           const float* alpha, const float* b, const float* w, const float* S0, void* o,
                           float* S_T, void* ws, size_t ws_bytes) {
@@ -77,6 +97,8 @@ ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, co
   a.qkv_t0 = 0;
   a.qkv_f16 = 0;
   a.gate_logits = p->gate_logits;
+  a.conv_in = p->conv_state_in;
+  a.conv_out = p->conv_state_out;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S0 = S0; a.o = o; a.ST = S_T;
   a.workspace = ws; a.ws_bytes = ws_bytes;
   return a;
@@ -115,6 +137,12 @@ gdn2_status gdn2::chunk_fwd_checked(const gdn2_params* p, const void* q, const v
   }
   if (S0 && S_T && S0 != S_T && overlaps(S0, sz.st, S_T, sz.st)) return GDN2_ERR_INVALID_ARG;
   if (overlaps(o, o_bytes, S_T, sz.st)) return GDN2_ERR_INVALID_ARG;
+  {
+    const Range cin[] = {{q, sz.qk}, {k, sz.qk}, {v, sz.v}, {alpha, sz.ga}, {b, sz.gb},
+                         {w, sz.gw}, {S0, sz.st}, {p->conv_w, conv_bytes}};
+    const Range cout[] = {{o, o_bytes}, {S_T, sz.st}, {workspace, ws_bytes}};
+    if ((st = check_conv_state(p, cin, 8, cout, 3)) != GDN2_OK) return st;
+  }
 
   ChunkArgs a = make_chunk_args(p, q, k, v, alpha, b, w, S0, o, S_T, workspace, ws_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -130,6 +158,7 @@ gdn2_status gdn2::chunk_fwd_checked(const gdn2_params* p, const void* q, const v
   } else {
     e = launch_chunk_simt(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16, s);
   }
+  if (e == cudaSuccess) e = launch_conv_state(a, p->qkv_dtype == GDN2_BF16, s);
   return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
 }
 
@@ -167,30 +196,35 @@ gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k,
                              void* stream) {
   gdn2_status st = check_common(p, true);
   if (st != GDN2_OK) return st;
-  if (p->conv_w != nullptr) return GDN2_ERR_UNSUPPORTED;
   const size_t tokens = (size_t)p->B;
   if (tokens > 0) {
     if (!q || !k || !v || !o || !S) return GDN2_ERR_INVALID_ARG;
     if ((st = check_gate_ptrs(p, alpha, b, w)) != GDN2_OK) return st;
   }
-  const void* ptrs[] = {q, k, v, alpha, b, w, S, o};
+  const void* ptrs[] = {q, k, v, alpha, b, w, S, o, p->conv_w};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return GDN2_ERR_INVALID_ARG;
   const Sizes sz = sizes(p, tokens);
   const size_t o_bytes = tokens * p->H_v * p->d_v * dsize(p->o_dtype);
-  struct R { const void* p; size_t n; } ins[] = {{q, sz.qk}, {k, sz.qk}, {v, sz.v}, {alpha, sz.ga},
-                                                  {b, sz.gb}, {w, sz.gw}};
-  for (const R& r : ins) {
+  const size_t conv_bytes = ((size_t)2 * p->H_qk * p->d_k + (size_t)p->H_v * p->d_v) * 4 * sizeof(float);
+  const Range ins[] = {{q, sz.qk}, {k, sz.qk}, {v, sz.v}, {alpha, sz.ga}, {b, sz.gb}, {w, sz.gw},
+                       {p->conv_w, conv_bytes}};
+  for (const Range& r : ins) {
     if (overlaps(o, o_bytes, r.p, r.n)) return GDN2_ERR_INVALID_ARG;
     if (overlaps(S, sz.st, r.p, r.n)) return GDN2_ERR_INVALID_ARG;
   }
   if (overlaps(o, o_bytes, S, sz.st)) return GDN2_ERR_INVALID_ARG;
+  {
+    const Range outs[] = {{o, o_bytes}, {S, sz.st}};
+    if ((st = check_conv_state(p, ins, 7, outs, 2)) != GDN2_OK) return st;
+  }
   if (tokens == 0) return GDN2_OK;
 
   DecodeArgs a;
   a.B = p->B; a.Hqk = p->H_qk; a.Hv = p->H_v; a.d = p->d_k; a.scale = p->scale;
   a.gate_mode = p->gate_mode; a.l2norm = p->l2norm_qk != 0; a.gate_logits = p->gate_logits;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S = S; a.o = o;
+  a.conv_w = p->conv_w; a.conv_in = p->conv_state_in; a.conv_out = p->conv_state_out;
   cudaError_t e = launch_decode(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16,
                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;

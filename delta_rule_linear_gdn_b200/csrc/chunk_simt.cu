@@ -39,15 +39,17 @@ struct SimtSmem {
 
 template <typename TIn>
 __device__ __forceinline__ float load_conv(const TIn* base, size_t tok_stride, int t, const float* wrow,
-                                           bool conv) {
+                                           bool conv, const TIn* hist, size_t hist_stride) {
   // base points at token 0 of this channel; tok_stride is the element stride
-  // between consecutive tokens.
+  // between consecutive tokens. hist (or NULL: zeros) points at row 0 of the
+  // channel's history, whose row 3 + t holds the input of token t < 0.
   if (!conv) return to_f32(base[(size_t)t * tok_stride]);
   float acc = 0.f;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int src = t - 3 + j;
     if (src >= 0) acc += wrow[j] * to_f32(base[(size_t)src * tok_stride]);
+    else if (hist) acc += wrow[j] * to_f32(hist[(size_t)(3 + src) * hist_stride]);
   }
   return acc;
 }
@@ -94,6 +96,11 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
   const float* wq = conv ? a.conv_w + (size_t)(hq * D) * 4 : nullptr;
   const float* wk = conv ? a.conv_w + (size_t)(a.Hqk * D + hq * D) * 4 : nullptr;
   const float* wv = conv ? a.conv_w + (size_t)(2 * a.Hqk * D + h * D) * 4 : nullptr;
+  const size_t hstride = 2 * qk_tok + v_tok;   // channels of the conv history rows
+  const TIn* hist = static_cast<const TIn*>(a.conv_in);
+  const TIn* hq_ = hist ? hist + (size_t)bi * 3 * hstride + (size_t)hq * D : nullptr;
+  const TIn* hk_ = hist ? hist + (size_t)bi * 3 * hstride + qk_tok + (size_t)hq * D : nullptr;
+  const TIn* hv_ = hist ? hist + (size_t)bi * 3 * hstride + 2 * qk_tok + (size_t)h * D + col0 : nullptr;
 
   // Entry state tile.
   for (int idx = tid; idx < D * DVT; idx += kThreads) {
@@ -114,8 +121,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
       if (i < Lc) {
         const int t = t0 + i;
         const size_t qk0 = (size_t)bi * a.T * qk_tok + (size_t)hq * D + c;
-        qv = load_conv(qg + qk0, qk_tok, t, conv ? wq + c * 4 : nullptr, conv);
-        kv = load_conv(kg + qk0, qk_tok, t, conv ? wk + c * 4 : nullptr, conv);
+        qv = load_conv(qg + qk0, qk_tok, t, conv ? wq + c * 4 : nullptr, conv, hq_ ? hq_ + c : nullptr, hstride);
+        kv = load_conv(kg + qk0, qk_tok, t, conv ? wk + c * 4 : nullptr, conv, hk_ ? hk_ + c : nullptr, hstride);
         const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
         gv = logf(gate_at(a.alpha, mode == GDN2_GATES_GDN ? gt : gt * D + c, a.gate_logits));
         bv = gate_at(a.b, (mode == GDN2_GATES_FULL) ? gt * D + c : gt, a.gate_logits);
@@ -132,7 +139,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         const int t = t0 + i;
         const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
         const float vv = load_conv(vg + (size_t)bi * a.T * v_tok + (size_t)h * D + col0 + c, v_tok, t,
-                                   conv ? wv + (col0 + c) * 4 : nullptr, conv);
+                                   conv ? wv + (col0 + c) * 4 : nullptr, conv, hv_ ? hv_ + c : nullptr, hstride);
         const float wv_ = (mode == GDN2_GATES_FULL) ? gate_at(a.w, gt * D + col0 + c, a.gate_logits)
                                                     : gate_at(a.b, gt, a.gate_logits);
         zv = wv_ * vv;

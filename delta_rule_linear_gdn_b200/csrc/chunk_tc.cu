@@ -1167,11 +1167,21 @@ __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, in
     unpack4_bf16(make_uint2(u.x, u.y), x);
     unpack4_bf16(make_uint2(u.z, u.w), x + 4);
   };
+  // Inputs before the CTA's first token: from the sequence, or for tokens
+  // before 0 from the caller's conv history [B, 3, channels] (zeros without).
+  const size_t hrow = (size_t)(2 * a.Hqk + a.Hv) * D;
+  const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.conv_in);
+  auto hload = [&](int tl) -> uint4 {
+    const int t = t_begin + tl;
+    if (t >= 0) return load(tl);
+    if (hist == nullptr) return make_uint4(0, 0, 0, 0);
+    return __ldg(reinterpret_cast<const uint4*>(hist + ((size_t)bi * 3 + 3 + t) * hrow + ch));
+  };
   float x3[8], x2[8], x1[8];                            // inputs of t−3, t−2, t−1
   {
-    const uint4 h3 = conv ? load(tl0 - 3) : make_uint4(0, 0, 0, 0);
-    const uint4 h2 = conv ? load(tl0 - 2) : make_uint4(0, 0, 0, 0);
-    const uint4 h1 = conv ? load(tl0 - 1) : make_uint4(0, 0, 0, 0);
+    const uint4 h3 = conv ? hload(tl0 - 3) : make_uint4(0, 0, 0, 0);
+    const uint4 h2 = conv ? hload(tl0 - 2) : make_uint4(0, 0, 0, 0);
+    const uint4 h1 = conv ? hload(tl0 - 1) : make_uint4(0, 0, 0, 0);
     unpack8(h3, x3);
     unpack8(h2, x2);
     unpack8(h1, x1);

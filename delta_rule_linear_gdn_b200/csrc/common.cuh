@@ -53,6 +53,10 @@ struct ChunkArgs {
   // and whether they hold fp16 instead of the input dtype.
   int qkv_T, qkv_t0, qkv_f16;
   int gate_logits;   // gates are bf16 logits (σ applied in the kernels)
+  // Conv history [B, 3, 2·Hqk·dk + Hv·dv] in the input dtype (NULL = zeros)
+  // and the buffer that receives the history after the last token (or NULL).
+  const void* conv_in;
+  void* conv_out;
 };
 
 struct DecodeArgs {
@@ -65,6 +69,9 @@ struct DecodeArgs {
   float* S;
   void* o;
   int gate_logits;   // gates are bf16 logits (σ applied in the kernels)
+  const float* conv_w;   // conv taps [2·Hqk·d + Hv·d, 4] or NULL (no conv)
+  const void* conv_in;   // conv history before this token, or NULL (zeros)
+  void* conv_out;        // history after this token, or NULL
 };
 
 // Launchers (return cudaSuccess or the launch error).
@@ -77,6 +84,9 @@ bool chunk_tc_supported(const ChunkArgs& a, int qkv_bf16);
 size_t chunk_tc_workspace(const ChunkArgs& a);
 size_t chunk_tc_min_workspace(const ChunkArgs& a, bool carry_state);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s);
+// Writes a.conv_out: the three pre-conv inputs that end at token T−1 of each
+// sequence (history from a.conv_in shifted in when T < 3).
+cudaError_t launch_conv_state(const ChunkArgs& a, int qkv_bf16, cudaStream_t s);
 
 // gdn2_chunk_fwd after argument checks; `segmented_ok` accepts a workspace
 // between the minimum and the full size.

@@ -12,6 +12,14 @@
 // with e = b ⊙ k, z = w ⊙ v. Both reductions run on the decayed state in the
 // same register pass, so the state is read from HBM once and written once.
 //
+// With the depthwise causal conv (kernel 4, "Gated DeltaNet: o mixer em 48
+// das 64 camadas", Conceito) the step convolves its q, k, v channels with the
+// three previous inputs held in the caller's conv history, normalises q, k
+// after the conv when asked, and writes the shifted history to a second
+// buffer (never the one it reads, since several CTAs read each q, k channel).
+// The q, k channels of a QK head are written by the CTA of its first value
+// head and first column tile; each CTA writes its own v channels.
+//
 // Work split: one CTA per (sequence, value head, tile of COLS value columns).
 // Thread (cg, rg) owns 4 consecutive columns (one float4) of rows
 // rg, rg+16, rg+32, ...: a warp instruction covers whole 4·COLS-byte row
@@ -25,7 +33,7 @@ namespace {
 
 constexpr int kRowGroups = 16;
 
-template <int D, int COLS, typename TIn, typename TOut, bool LG>
+template <int D, int COLS, typename TIn, typename TOut, bool LG, bool CONV>
 __global__ void __launch_bounds__((COLS / 4) * kRowGroups)
 decode_kernel(DecodeArgs a) {
   constexpr int CG = COLS / 4;            // column groups (float4 each)
@@ -61,15 +69,48 @@ decode_kernel(DecodeArgs a) {
   const TIn* qg = static_cast<const TIn*>(a.q) + ((size_t)bi * a.Hqk + hq) * D;
   const TIn* kg = static_cast<const TIn*>(a.k) + ((size_t)bi * a.Hqk + hq) * D;
   const TIn* vg = static_cast<const TIn*>(a.v) + (size_t)bh * D + col0;
+  // Conv history rows [B, 3, channels]; channel offsets of q, k and v.
+  const size_t ctot = (size_t)(2 * a.Hqk + a.Hv) * D;
+  const size_t hbase = (size_t)bi * 3 * ctot;
+  const size_t cq = (size_t)hq * D, ck = (size_t)(a.Hqk + hq) * D, cv = (size_t)2 * a.Hqk * D + (size_t)h * D + col0;
+  const TIn* hin = static_cast<const TIn*>(a.conv_in);
+  auto conv1 = [&](TIn xr, size_t ch) -> float {   // y = Σ_j W[ch][j] x_{t−3+j}
+    const float x = to_f32(xr);
+    if (!CONV) return x;
+    const float4 wt = __ldg(reinterpret_cast<const float4*>(a.conv_w) + ch);
+    float y = wt.w * x;
+    if (hin) {
+      const TIn* hp = hin + hbase + ch;
+      y += wt.x * to_f32(hp[0]) + wt.y * to_f32(hp[ctot]) + wt.z * to_f32(hp[2 * ctot]);
+    }
+    return y;
+  };
   for (int i = tid; i < D; i += NT) {
-    s_q[i] = to_f32(qg[i]);
-    s_k[i] = to_f32(kg[i]);
+    s_q[i] = conv1(qg[i], cq + i);
+    s_k[i] = conv1(kg[i], ck + i);
     s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? (size_t)bh : (size_t)bh * D + i);
   }
   const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at<LG>(a.b, bh);
   for (int j = tid; j < COLS; j += NT) {
     const float wj = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.w, (size_t)bh * D + col0 + j) : beta;
-    s_z[j] = wj * to_f32(vg[j]);
+    s_z[j] = wj * conv1(vg[j], cv + j);
+  }
+  if (CONV && a.conv_out) {
+    // Shifted history: rows 1, 2 of the incoming history, then this token.
+    TIn* hout = static_cast<TIn*>(a.conv_out);
+    auto shift = [&](size_t ch, TIn xr) {
+      const TIn zero = from_f32<TIn>(0.f);
+      hout[hbase + ch] = hin ? hin[hbase + ctot + ch] : zero;
+      hout[hbase + ctot + ch] = hin ? hin[hbase + 2 * ctot + ch] : zero;
+      hout[hbase + 2 * ctot + ch] = xr;
+    };
+    if (tile == 0 && h % (a.Hv / a.Hqk) == 0) {
+      for (int i = tid; i < D; i += NT) {
+        shift(cq + i, qg[i]);
+        shift(ck + i, kg[i]);
+      }
+    }
+    for (int j = tid; j < COLS; j += NT) shift(cv + j, vg[j]);
   }
   __syncthreads();
   if (tid < 32) {
@@ -164,10 +205,14 @@ template <int D, int COLS, typename TIn, typename TOut>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t s) {
   const int grid = a.B * a.Hv * (D / COLS);
   if (grid == 0) return cudaSuccess;
+  constexpr int NT = (COLS / 4) * kRowGroups;
+  const bool conv = a.conv_w != nullptr;
   if (a.gate_logits)
-    decode_kernel<D, COLS, TIn, TOut, true><<<grid, (COLS / 4) * kRowGroups, 0, s>>>(a);
+    (conv ? decode_kernel<D, COLS, TIn, TOut, true, true> : decode_kernel<D, COLS, TIn, TOut, true, false>)
+        <<<grid, NT, 0, s>>>(a);
   else
-    decode_kernel<D, COLS, TIn, TOut, false><<<grid, (COLS / 4) * kRowGroups, 0, s>>>(a);
+    (conv ? decode_kernel<D, COLS, TIn, TOut, false, true> : decode_kernel<D, COLS, TIn, TOut, false, false>)
+        <<<grid, NT, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -42,6 +42,7 @@ class Params(ctypes.Structure):
         ("scale", ctypes.c_float), ("qkv_dtype", ctypes.c_int), ("o_dtype", ctypes.c_int),
         ("gate_mode", ctypes.c_int), ("precision", ctypes.c_int), ("l2norm_qk", ctypes.c_int),
         ("conv_w", ctypes.c_void_p), ("gate_logits", ctypes.c_int),
+        ("conv_state_in", ctypes.c_void_p), ("conv_state_out", ctypes.c_void_p),
     ]
 
 
@@ -109,11 +110,26 @@ def _stream_handle(stream):
 
 
 def make_params(B, T, H_qk, H_v, d_k, d_v, *, chunk=64, scale=1.0, qkv_dtype=BF16, o_dtype=BF16,
-                gate_mode="full", precision="default", l2norm_qk=False, conv_w=None, gate_logits=False) -> Params:
+                gate_mode="full", precision="default", l2norm_qk=False, conv_w=None, gate_logits=False,
+                conv_state_in=None, conv_state_out=None) -> Params:
     return Params(int(B), int(T), int(H_qk), int(H_v), int(d_k), int(d_v), int(chunk), float(scale),
                   int(qkv_dtype), int(o_dtype), GATES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode),
                   PRECISION[precision] if isinstance(precision, str) else int(precision),
-                  1 if l2norm_qk else 0, _ptr(conv_w), 1 if gate_logits else 0)
+                  1 if l2norm_qk else 0, _ptr(conv_w), 1 if gate_logits else 0,
+                  _ptr(conv_state_in), _ptr(conv_state_out))
+
+
+def conv_state_shape(B, H_qk, H_v, d_k, d_v):
+    """Shape of a conv history buffer: [B, 3, 2·H_qk·d_k + H_v·d_v] (q | k | v channels)."""
+    return (B, 3, 2 * H_qk * d_k + H_v * d_v)
+
+
+def _check_conv_state(t, name, qkv_dtype, shape):
+    if t is None:
+        return
+    _check(t, name, qkv_dtype)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
 def _check(t, name, dtype=None):
@@ -133,10 +149,14 @@ def chunk_fwd_workspace(params: Params) -> int:
 
 def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_mode="full",
               precision="default", l2norm_qk=False, conv_w=None, o_dtype=None, o=None, S_T=None,
-              workspace=None, stream=None, want_state=True, gate_logits=False):
+              workspace=None, stream=None, want_state=True, gate_logits=False, conv_state_in=None,
+              conv_state_out=None):
     """Chunked prefill. q,k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; gates per
     ``gate_mode``: fp32 values, or bf16 logits with ``gate_logits`` (the kernels
-    apply the sigmoid); S0 [B,H_v,d_k,d_v] fp32 or None. Returns (o, S_T)."""
+    apply the sigmoid); S0 [B,H_v,d_k,d_v] fp32 or None. With ``conv_w``, the
+    conv history before token 0 comes from ``conv_state_in`` (None: zeros) and
+    the history after the last token is written to ``conv_state_out`` (both
+    :func:`conv_state_shape`, q's dtype, distinct buffers). Returns (o, S_T)."""
     B, T, H_qk, d_k = q.shape
     H_v, d_v = v.shape[2], v.shape[3]
     o_dtype = q.dtype if o_dtype is None else o_dtype
@@ -147,9 +167,13 @@ def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_m
         _check(t, name, gdt)
     for name, t in (("S0", S0), ("conv_w", conv_w)):
         _check(t, name, torch.float32)
+    hshape = conv_state_shape(B, H_qk, H_v, d_k, d_v)
+    _check_conv_state(conv_state_in, "conv_state_in", q.dtype, hshape)
+    _check_conv_state(conv_state_out, "conv_state_out", q.dtype, hshape)
     p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
                     o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, precision=precision,
-                    l2norm_qk=l2norm_qk, conv_w=conv_w, gate_logits=gate_logits)
+                    l2norm_qk=l2norm_qk, conv_w=conv_w, gate_logits=gate_logits,
+                    conv_state_in=conv_state_in, conv_state_out=conv_state_out)
     if o is None:
         o = torch.empty((B, T, H_v, d_v), dtype=o_dtype, device=q.device)
     if S_T is None and want_state:
@@ -169,10 +193,13 @@ def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_m
 
 
 def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_qk=False, o_dtype=None,
-                o=None, stream=None, gate_logits=False):
+                o=None, stream=None, gate_logits=False, conv_w=None, conv_state_in=None, conv_state_out=None):
     """One decode step. q,k [B,H_qk,d_k]; v [B,H_v,d_v]; gates without the T
     axis (fp32 values, or bf16 logits with ``gate_logits``); S [B,H_v,d_k,d_v]
-    fp32 updated in place. Returns o [B,H_v,d_v]."""
+    fp32 updated in place. With ``conv_w`` the step's conv reads
+    ``conv_state_in`` (None: zeros) and writes the shifted history to
+    ``conv_state_out`` (a second buffer: swap the two between steps).
+    Returns o [B,H_v,d_v]."""
     B, H_qk, d_k = q.shape
     H_v, d_v = v.shape[1], v.shape[2]
     o_dtype = q.dtype if o_dtype is None else o_dtype
@@ -182,9 +209,14 @@ def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_
     for name, t in (("alpha", alpha), ("b", b), ("w", w)):
         _check(t, name, gdt)
     _check(S, "S", torch.float32)
+    _check(conv_w, "conv_w", torch.float32)
+    hshape = conv_state_shape(B, H_qk, H_v, d_k, d_v)
+    _check_conv_state(conv_state_in, "conv_state_in", q.dtype, hshape)
+    _check_conv_state(conv_state_out, "conv_state_out", q.dtype, hshape)
     p = make_params(B, 1, H_qk, H_v, d_k, d_v, scale=scale, qkv_dtype=_dtype_code(q.dtype),
                     o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk,
-                    gate_logits=gate_logits)
+                    gate_logits=gate_logits, conv_w=conv_w, conv_state_in=conv_state_in,
+                    conv_state_out=conv_state_out)
     if o is None:
         o = torch.empty((B, H_v, d_v), dtype=o_dtype, device=q.device)
     _check(o, "o", o_dtype)

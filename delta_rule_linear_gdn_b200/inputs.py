@@ -146,6 +146,15 @@ def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: s
     return out
 
 
+def make_conv_state(w: Workload, seed: int, device="cpu"):
+    """A conv history [B, 3, 2·Hqk·d + Hv·d] in the workload's q,k,v dtype: the
+    pre-conv inputs of three earlier tokens (standard normal draws, the
+    distribution of the conv workload's q, k, v), channels q | k | v."""
+    dev = torch.device(device)
+    x = _normal((w.B, 3, (2 * w.H_qk + w.H_v) * w.d), _gen(seed, 9, dev), dev)
+    return x.to(_qkv_dtype(w))
+
+
 def make_decode_pool(w: Workload, pool: int = 16, seed: int | None = None, device="cpu",
                      gate_mode: str = "full", gate_logits: bool = False):
     """Per-step decode inputs: ``pool`` independent one-token step sets, cycled by

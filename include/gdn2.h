@@ -35,6 +35,7 @@
  *    for gdn2_chunk_fwd (α ∈ [0,1] for gdn2_decode_step), b, w ∈ [0,1];
  *    q, k of unit length unless l2norm_qk is set.
  *  - Output buffers must not alias inputs, except S0 == S_T (in place).
+ *    conv_state_out never aliases conv_state_in.
  */
 #ifndef GDN2_H_
 #define GDN2_H_
@@ -93,11 +94,12 @@ typedef struct {
   int l2norm_qk;  /* nonzero: normalise q and k (after the conv) inside the
                      kernel: x · (Σx² + 1e-6)^(-1/2)                          */
   const float* conv_w; /* NULL, or device weights [2·H_qk·d_k + H_v·d_v, 4] of
-                     the depthwise causal conv (kernel 4, no bias, zero
-                     history) applied to q | k | v channels before the
-                     recurrence ("Gated DeltaNet: o mixer em 48 das 64
-                     camadas", Conceito). Tap 3 weights the current token.
-                     gdn2_chunk_fwd only.                                     */
+                     the depthwise causal conv (kernel 4, no bias) applied to
+                     q | k | v channels before the recurrence ("Gated
+                     DeltaNet: o mixer em 48 das 64 camadas", Conceito):
+                     y_t = Σ_j W[c][j]·x_{t−3+j}, so tap 3 weights the
+                     current token. The three inputs before the first token
+                     come from conv_state_in (zeros when it is NULL).        */
   int gate_logits; /* 0: alpha, b, w hold the gate values (fp32). 1: they hold
                      bf16 logits x and the kernels use σ(x) = 1 / (1 + e^(−x)),
                      the sigmoid the pages put on the gate projections
@@ -105,6 +107,19 @@ typedef struct {
                      Funciona a Camada de Atenção do DeltaNet-2"); same
                      shapes, half the bytes. The pointers keep their float*
                      type and are read as bf16.                               */
+  const void* conv_state_in; /* NULL, or device [B, 3, 2·H_qk·d_k + H_v·d_v] in
+                     qkv_dtype: per sequence the three pre-conv inputs that
+                     precede this call's first token, oldest first, channels
+                     ordered q | k | v as in conv_w. NULL means zero history
+                     (a sequence's start). Needs conv_w.                      */
+  void* conv_state_out; /* NULL, or device buffer of the same layout, written
+                     with the three pre-conv inputs ending at this call's last
+                     token (with T < 3, the tail of conv_state_in shifted in;
+                     T = 0 copies it). Feed it as the next call's
+                     conv_state_in: together the two carry the conv across
+                     split prefills and decode steps. Must not overlap
+                     conv_state_in or any other argument (swap two buffers
+                     between calls). Needs conv_w.                            */
 } gdn2_params;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -155,7 +170,9 @@ GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const v
  * query-read reduction), with the GDN-2 gates. Each state is read once from
  * HBM and written once.
  *
- *   q, k   [B,H_qk,d_k]     qkv_dtype (l2norm_qk honoured; conv_w must be NULL)
+ *   q, k   [B,H_qk,d_k]     qkv_dtype (conv_w and l2norm_qk honoured: the
+ *                           step's conv reads conv_state_in and writes
+ *                           conv_state_out, a ping-pong pair across steps)
  *   v      [B,H_v,d_v]      qkv_dtype
  *   alpha, b, w             fp32, gate_mode layouts without the T axis
  *   S      [B,H_v,d_k,d_v]  fp32, read and overwritten with the new state

@@ -21,6 +21,10 @@ Functions and the passages they follow:
   assume normalised keys: "Uma análise das variantes de atenção linear da
   família DeltaNet", Notação e ordem da derivação).
 * :func:`preprocess` -- conv then L2 norm, in that order.
+* :func:`conv_state_after` -- the conv's three-token history after a call, so
+  that a sequence split into calls (prefill pieces, decode steps) convolves
+  exactly as one call over all its tokens (same page: the conv is causal
+  over the token stream, which a split does not change).
 * :func:`gates_from_logits` -- the gates as the sigmoid of their projections'
   outputs ("BigSaaS – Posts", section "Implementação Prática: Como Funciona a
   Camada de Atenção do DeltaNet-2": erase and write gates pass through a
@@ -120,16 +124,43 @@ def expand_tied_gates(mode: str, alpha, beta, d_k: int, d_v: int):
     return alpha, b, w
 
 
-def causal_conv4(x, W):
-    """x [B,T,C], W [C,4] -> y [B,T,C] (depthwise causal conv, zero history)."""
+def causal_conv4(x, W, history=None):
+    """x [B,T,C], W [C,4] -> y [B,T,C] (depthwise causal conv).
+
+    ``history`` [B,3,C] holds the three inputs before token 0, oldest first
+    (None: zeros). The conv is then the zero-history conv of the stream
+    ``history ++ x`` with its first three outputs dropped: the definition of a
+    conv that continues over earlier tokens."""
     x = _f64(x)
     W = _f64(W)
     B, T, C = x.shape
     assert W.shape == (C, 4)
+    if history is not None:
+        h = _f64(history)
+        assert h.shape == (B, 3, C)
+        return causal_conv4(np.concatenate([h, x], axis=1), W)[:, 3:]
     y = np.zeros_like(x)
     if _load().oracle_causal_conv4(B, T, C, _ptr(x), _ptr(W), _ptr(y)) != 0:
         raise ValueError("oracle_causal_conv4 rejected its arguments")
     return y
+
+
+def conv_inputs(q, k, v):
+    """The conv's input channels per token: [B,T, Hqk·dk | Hqk·dk | Hv·dv]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hqk, dk = q.shape
+    nq, nv = Hqk * dk, v.shape[2] * v.shape[3]
+    return np.concatenate([q.reshape(B, T, nq), k.reshape(B, T, nq), v.reshape(B, T, nv)], axis=2)
+
+
+def conv_state_after(q, k, v, conv_state=None):
+    """The conv history after the last token: the last three rows of
+    ``conv_state ++ inputs`` ([B,3,C], oldest first; zeros stand in for a
+    missing ``conv_state``)."""
+    x = conv_inputs(q, k, v)
+    B, _, C = x.shape
+    h = np.zeros((B, 3, C)) if conv_state is None else _f64(conv_state)
+    return np.concatenate([h, x], axis=1)[:, -3:]
 
 
 def l2norm(x, eps: float = L2NORM_EPS):
@@ -143,9 +174,10 @@ def l2norm(x, eps: float = L2NORM_EPS):
     return y
 
 
-def preprocess(q, k, v, conv_w=None, l2norm_qk: bool = False):
+def preprocess(q, k, v, conv_w=None, l2norm_qk: bool = False, conv_state=None):
     """Optional depthwise causal conv on q, k, v (weights [Hqk·dk + Hqk·dk + Hv·dv, 4],
-    rows ordered q | k | v), then optional L2 normalisation of q and k."""
+    rows ordered q | k | v; history ``conv_state`` [B,3,channels] in the same
+    channel order, None for zeros), then optional L2 normalisation of q and k."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, T, Hqk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
@@ -153,9 +185,13 @@ def preprocess(q, k, v, conv_w=None, l2norm_qk: bool = False):
         W = _f64(conv_w)
         nq = Hqk * dk
         assert W.shape == (2 * nq + Hv * dv, 4)
-        q = causal_conv4(q.reshape(B, T, nq), W[:nq]).reshape(q.shape)
-        k = causal_conv4(k.reshape(B, T, nq), W[nq:2 * nq]).reshape(k.shape)
-        v = causal_conv4(v.reshape(B, T, Hv * dv), W[2 * nq:]).reshape(v.shape)
+        h = [None] * 3
+        if conv_state is not None:
+            hs = _f64(conv_state)
+            h = [hs[:, :, :nq], hs[:, :, nq:2 * nq], hs[:, :, 2 * nq:]]
+        q = causal_conv4(q.reshape(B, T, nq), W[:nq], h[0]).reshape(q.shape)
+        k = causal_conv4(k.reshape(B, T, nq), W[nq:2 * nq], h[1]).reshape(k.shape)
+        v = causal_conv4(v.reshape(B, T, Hv * dv), W[2 * nq:], h[2]).reshape(v.shape)
     if l2norm_qk:
         q = l2norm(q)
         k = l2norm(k)

@@ -26,17 +26,20 @@ def oracle_gates(mode, alpha, b, w, d_k, d_v, gate_logits=False):
 
 
 def oracle_chunk(inp, gate_mode="full", scale=1.0, l2norm_qk=False, S0=None, threads=0,
-                 heads=None, gate_logits=False):
-    """Oracle (o, S_T) for a chunk_fwd input dict. ``heads`` optionally restricts
-    to a list of (sequence, value head) pairs; returns dict keyed by pair then."""
+                 heads=None, gate_logits=False, conv_state=None):
+    """Oracle (o, S_T) for a chunk_fwd input dict (``conv_state``: the conv
+    history before token 0, or None). ``heads`` optionally restricts to a list of
+    (sequence, value head) pairs; returns dict keyed by pair then."""
     q, k, v = np64(inp["q"]), np64(inp["k"]), np64(inp["v"])
     d_k, d_v = q.shape[-1], v.shape[-1]
     conv_w = np64(inp.get("conv_w"))
+    conv_state = np64(conv_state)
     S0 = np64(inp.get("S0")) if S0 is None else np64(S0)
     alpha, b, w = oracle_gates(gate_mode, inp["alpha"], inp["b"], inp.get("w"), d_k, d_v, gate_logits)
     if heads is None:
-        qp, kp, vp = oracle.preprocess(q, k, v, conv_w, l2norm_qk)
+        qp, kp, vp = oracle.preprocess(q, k, v, conv_w, l2norm_qk, conv_state)
         return oracle.gdn2_forward(qp, kp, vp, alpha, b, w, S0, scale=scale, threads=threads)
+    assert conv_state is None, "per-head oracle runs take no conv history"
     Hqk, Hv = q.shape[2], v.shape[2]
     g = Hv // Hqk
     out = {}

@@ -103,21 +103,54 @@ def test_chunk_rejects_aliased_output(L):
     assert _call_chunk(L, p, S_T=FAKE * 8 + 64) == gdn2.ERR_INVALID_ARG
 
 
-def test_decode_rejects_conv_and_bad_args(L):
-    p = _params(conv_w=FAKE * 20)
-    args = [FAKE * (i + 1) for i in range(8)]
-    assert L.gdn2_decode_step(ctypes.byref(p), *args, None) == gdn2.ERR_UNSUPPORTED
+def test_decode_rejects_bad_args(L):
     p = _params()
+    args = [FAKE * (i + 1) for i in range(8)]
     args[6] = None  # S
     assert L.gdn2_decode_step(ctypes.byref(p), *args, None) == gdn2.ERR_INVALID_ARG
     assert L.gdn2_decode_step(None, *[FAKE] * 8, None) == gdn2.ERR_INVALID_ARG
 
 
-def test_gate_logits_field_follows_conv_w():
-    # the C struct ends with conv_w then gate_logits: the mirror keeps that order
+def _call_decode(L, p, **ptrs):
+    names = ["q", "k", "v", "alpha", "b", "w", "S", "o"]
+    vals = {n: FAKE * (i + 1) for i, n in enumerate(names)}
+    vals.update(ptrs)
+    return L.gdn2_decode_step(ctypes.byref(p), *[vals[n] for n in names], None)
+
+
+def test_conv_state_validation(L):
+    # history buffers at 64 KiB multiples past the other arguments (576 bytes each here)
+    hin, hout, conv_w = FAKE * 30, FAKE * 31, FAKE * 20
+    for call in (_call_chunk, _call_decode):
+        # history without a conv
+        assert call(L, _params(conv_state_in=hin)) == gdn2.ERR_INVALID_ARG
+        assert call(L, _params(conv_state_out=hout)) == gdn2.ERR_INVALID_ARG
+        # misaligned
+        assert call(L, _params(conv_w=conv_w, conv_state_out=hout + 8)) == gdn2.ERR_INVALID_ARG
+        # outgoing history on the incoming one (also in place), or on an input
+        assert call(L, _params(conv_w=conv_w, conv_state_in=hin, conv_state_out=hin)) == gdn2.ERR_INVALID_ARG
+        assert call(L, _params(conv_w=conv_w, conv_state_in=hin, conv_state_out=hin + 512)) == gdn2.ERR_INVALID_ARG
+        assert call(L, _params(conv_w=conv_w, conv_state_out=FAKE * 2)) == gdn2.ERR_INVALID_ARG
+        assert call(L, _params(conv_w=conv_w, conv_state_out=conv_w)) == gdn2.ERR_INVALID_ARG
+    # the output o written over the incoming history
+    assert _call_chunk(L, _params(conv_w=conv_w, conv_state_in=hin), o=hin) == gdn2.ERR_INVALID_ARG
+    assert _call_decode(L, _params(conv_w=conv_w, conv_state_in=hin), o=hin) == gdn2.ERR_INVALID_ARG
+    assert _call_decode(L, _params(conv_w=conv_w, conv_state_in=hin), S=hin - 256) == gdn2.ERR_INVALID_ARG
+
+
+def _header_param_fields():
+    text = open(HEADER).read()
+    body = text[text.index("typedef struct {"):text.index("} gdn2_params;")]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    return re.findall(r"(\w+)\s*;", body)
+
+
+def test_params_mirror_matches_header_field_order():
     names = [f[0] for f in gdn2.Params._fields_]
-    assert names[-2:] == ["conv_w", "gate_logits"]
+    assert names == _header_param_fields()
+    assert names[-4:] == ["conv_w", "gate_logits", "conv_state_in", "conv_state_out"]
     assert gdn2.make_params(1, 1, 1, 1, 16, 16, gate_logits=True).gate_logits == 1
+    assert gdn2.conv_state_shape(2, 16, 48, 128, 128) == (2, 3, 10240)
 
 
 def test_workspace_query_is_host_only(L):

@@ -356,6 +356,51 @@ def test_conv_current_token_tap_and_causality():
     np.testing.assert_array_equal(y[0, :, 0], [0, 0, 4, 3, 2, 1])
 
 
+def test_conv_history_taps_closed_form():
+    """With only tap j set, y_t = W[c][j]·x_{t−3+j}: the first outputs read the
+    history rows oldest first (row 0 = token −3), then the tokens themselves."""
+    hist = np.array([[[10.0], [20.0], [30.0]]])      # tokens −3, −2, −1
+    x = np.array([[[1.0], [2.0], [3.0], [4.0]]])
+    for j, ref in ((0, [10, 20, 30, 1]), (1, [20, 30, 1, 2]), (2, [30, 1, 2, 3]), (3, [1, 2, 3, 4])):
+        W = np.zeros((1, 4))
+        W[0, j] = 2.0
+        y = oracle.causal_conv4(x, W, hist)
+        np.testing.assert_array_equal(y[0, :, 0], 2.0 * np.array(ref, dtype=float))
+
+
+def test_conv_split_equals_whole_and_state_rows():
+    """Convolving a sequence in pieces, each starting from the history the
+    previous piece leaves (conv_state_after), equals one conv of the whole
+    sequence: the conv is causal over the token stream. Pieces shorter than
+    three tokens shift the older history through."""
+    r = _rng(33)
+    B, T, Hqk, Hv, dk, dv = 2, 13, 1, 2, 3, 2
+    q = r.standard_normal((B, T, Hqk, dk))
+    k = r.standard_normal((B, T, Hqk, dk))
+    v = r.standard_normal((B, T, Hv, dv))
+    W = r.standard_normal((2 * Hqk * dk + Hv * dv, 4))
+    whole = oracle.preprocess(q, k, v, W, l2norm_qk=True)
+    for cuts in ([0, 5, 13], [0, 1, 2, 3, 13], [0, 2, 4, 6, 7, 13], [0, 13, 13]):
+        state = None
+        parts = []
+        for t0, t1 in zip(cuts[:-1], cuts[1:]):
+            sl = slice(t0, t1)
+            parts.append(oracle.preprocess(q[:, sl], k[:, sl], v[:, sl], W, l2norm_qk=True, conv_state=state))
+            state = oracle.conv_state_after(q[:, sl], k[:, sl], v[:, sl], state)
+        for i in range(3):
+            got = np.concatenate([p[i] for p in parts], axis=1)
+            np.testing.assert_allclose(got, whole[i], rtol=0, atol=1e-13)
+        # the final history holds the inputs of tokens T−3, T−2, T−1, channels q | k | v
+        last = np.concatenate([q[:, -3:].reshape(B, 3, -1), k[:, -3:].reshape(B, 3, -1),
+                               v[:, -3:].reshape(B, 3, -1)], axis=2)
+        np.testing.assert_array_equal(state, last)
+    # one token after a given history: rows 1, 2 of it, then the token
+    h = r.standard_normal((B, 3, 2 * Hqk * dk + Hv * dv))
+    s1 = oracle.conv_state_after(q[:, :1], k[:, :1], v[:, :1], h)
+    np.testing.assert_array_equal(s1[:, :2], h[:, 1:])
+    np.testing.assert_array_equal(s1[:, 2], oracle.conv_inputs(q[:, :1], k[:, :1], v[:, :1])[:, 0])
+
+
 def test_l2norm_matches_numpy():
     r = _rng(31)
     x = r.standard_normal((3, 7, 9))
