@@ -33,6 +33,7 @@ gdn2_status check_common(const gdn2_params* p, bool decode) {
   if (p->o_dtype != GDN2_F32 && p->o_dtype != GDN2_BF16) return GDN2_ERR_INVALID_ARG;
   if (p->gate_mode < GDN2_GATES_FULL || p->gate_mode > GDN2_GATES_GDN) return GDN2_ERR_INVALID_ARG;
   if (p->gate_logits != 0 && p->gate_logits != 1) return GDN2_ERR_INVALID_ARG;
+  if (p->gate_heads != GDN2_GATE_HEADS_V && p->gate_heads != GDN2_GATE_HEADS_QK) return GDN2_ERR_INVALID_ARG;
   if (p->precision != GDN2_PREC_DEFAULT && p->precision != GDN2_PREC_FP32) return GDN2_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return GDN2_ERR_INVALID_ARG;
   if (p->d_k != p->d_v || !supported_dim(p->d_k)) return GDN2_ERR_UNSUPPORTED;
@@ -53,8 +54,9 @@ Sizes sizes(const gdn2_params* p, size_t tokens) {
   s.qk = tokens * p->H_qk * dk * dsize(p->qkv_dtype);
   s.v = tokens * p->H_v * dv * dsize(p->qkv_dtype);
   const size_t gsz = p->gate_logits ? 2 : 4;   // bf16 logits or fp32 values
-  s.ga = tokens * p->H_v * (p->gate_mode == GDN2_GATES_GDN ? 1 : dk) * gsz;
-  s.gb = tokens * p->H_v * (p->gate_mode == GDN2_GATES_FULL ? dk : 1) * gsz;
+  const size_t hg = p->gate_heads == GDN2_GATE_HEADS_QK ? p->H_qk : p->H_v;   // heads of alpha and b
+  s.ga = tokens * hg * (p->gate_mode == GDN2_GATES_GDN ? 1 : dk) * gsz;
+  s.gb = tokens * hg * (p->gate_mode == GDN2_GATES_FULL ? dk : 1) * gsz;
   s.gw = p->gate_mode == GDN2_GATES_FULL ? tokens * p->H_v * dv * gsz : 0;
   s.st = (size_t)p->B * p->H_v * dk * dv * 4;
   return s;
@@ -99,6 +101,7 @@ ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, co
   a.gate_logits = p->gate_logits;
   a.conv_in = p->conv_state_in;
   a.conv_out = p->conv_state_out;
+  a.Hg = p->gate_heads == GDN2_GATE_HEADS_QK ? p->H_qk : p->H_v;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S0 = S0; a.o = o; a.ST = S_T;
   a.workspace = ws; a.ws_bytes = ws_bytes;
   return a;
@@ -225,6 +228,7 @@ gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k,
   a.gate_mode = p->gate_mode; a.l2norm = p->l2norm_qk != 0; a.gate_logits = p->gate_logits;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S = S; a.o = o;
   a.conv_w = p->conv_w; a.conv_in = p->conv_state_in; a.conv_out = p->conv_state_out;
+  a.Hg = p->gate_heads == GDN2_GATE_HEADS_QK ? p->H_qk : p->H_v;
   cudaError_t e = launch_decode(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16,
                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;

@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
   const int h = bh % a.Hv;
   const int bi = bh / a.Hv;
   const int hq = h / (a.Hv / a.Hqk);
+  const int hg = a.Hg == a.Hv ? h : hq;     // head of alpha and b
   const int col0 = tile * DVT;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = a.chunk;
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         const size_t qk0 = (size_t)bi * a.T * qk_tok + (size_t)hq * D + c;
         qv = load_conv(qg + qk0, qk_tok, t, conv ? wq + c * 4 : nullptr, conv, hq_ ? hq_ + c : nullptr, hstride);
         kv = load_conv(kg + qk0, qk_tok, t, conv ? wk + c * 4 : nullptr, conv, hk_ ? hk_ + c : nullptr, hstride);
-        const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
+        const size_t gt = ((size_t)bi * a.T + t) * a.Hg + hg;   // row of alpha, b
         gv = logf(gate_at(a.alpha, mode == GDN2_GATES_GDN ? gt : gt * D + c, a.gate_logits));
         bv = gate_at(a.b, (mode == GDN2_GATES_FULL) ? gt * D + c : gt, a.gate_logits);
       }
@@ -137,11 +138,12 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
       float zv = 0.f;
       if (i < Lc) {
         const int t = t0 + i;
-        const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;
+        const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;     // row of w
+        const size_t gtb = ((size_t)bi * a.T + t) * a.Hg + hg;   // row of b (= β, tied modes)
         const float vv = load_conv(vg + (size_t)bi * a.T * v_tok + (size_t)h * D + col0 + c, v_tok, t,
                                    conv ? wv + (col0 + c) * 4 : nullptr, conv, hv_ ? hv_ + c : nullptr, hstride);
         const float wv_ = (mode == GDN2_GATES_FULL) ? gate_at(a.w, gt * D + col0 + c, a.gate_logits)
-                                                    : gate_at(a.b, gt, a.gate_logits);
+                                                    : gate_at(a.b, gtb, a.gate_logits);
         zv = wv_ * vv;
       }
       sz[i * DVT + c] = zv;

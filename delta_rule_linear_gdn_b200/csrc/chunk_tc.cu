@@ -302,8 +302,13 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   float f[8][4];                   // α, then its forward products within the quarter
   float4 bq[4];
   uint2 kk[4], qq[4];
+  // rows of alpha, b (per value head, or shared per QK head) and of w
+  const bool g_qk = a.Hg != a.Hv;
   auto gate_row = [&](const Item& it, int u) -> size_t {
-    return ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hv + it.h;
+    return ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hg + (g_qk ? it.hq : it.h);
+  };
+  auto w_row = [&](const Item& it, int u) -> size_t {
+    return full ? ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hv + it.h : gate_row(it, u);
   };
   auto qkv_tok = [&](const Item& it, int u) -> size_t {
     return (size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i0 + u;
@@ -320,7 +325,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   auto fetch_alpha = [&](int item_) {
     const Item nx = decode_item(a, c_begin, item_);
     mbar_arrive_expect_tx(bar_a, C * D * (LG ? 2 : 4));
-    tma_load_3d(smem + P_ALPHA, &amap, 0, nx.h, nx.bi * a.T + nx.t0, bar_a);
+    tma_load_3d(smem + P_ALPHA, &amap, 0, a.Hg != a.Hv ? nx.hq : nx.h, nx.bi * a.T + nx.t0, bar_a);
   };
   uint32_t phase_a = 0;
   auto load_alpha_key0 = [&](int item_) {
@@ -501,7 +506,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const bool ok = it.Lc == C || i0 + u < it.Lc;
-      wv[u] = ok ? gate4<LG>(src.w, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+      wv[u] = ok ? gate4<LG>(src.w, w_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
       vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
                  : make_uint2(0, 0);
     }
@@ -1280,9 +1285,10 @@ cudaError_t launch_dependent(void (*kernel)(Args...), int grid, int block, size_
 }  // namespace
 
 namespace {
-// Tensor map of the per-channel α gates [B·T][H_v][128] (fp32, or bf16 logits) for the prep's
-// tile loads (box: 64 tokens × 1 head × 128 channels). false if the driver
-// entry point is unavailable (the prep then reads α with plain loads).
+// Tensor map of the per-channel α gates [B·T][H_g][128] (fp32, or bf16 logits; H_g heads own
+// them: H_v, or H_qk when shared) for the prep's tile loads (box: 64 tokens × 1 head × 128
+// channels). false if the driver entry point is unavailable (the prep then reads α with
+// plain loads).
 bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
   const cuuint64_t esz = a.gate_logits ? 2 : 4;
   static PFN_cuTensorMapEncodeTiled encode = [] {
@@ -1294,8 +1300,8 @@ bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
   }();
   if (encode == nullptr) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.Hv, (cuuint64_t)a.B * (cuuint64_t)a.T};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)a.Hv * D * esz};   // bytes, dims 1 and 2
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.Hg, (cuuint64_t)a.B * (cuuint64_t)a.T};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)a.Hg * D * esz};   // bytes, dims 1 and 2
   const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
   const cuuint32_t estr[3] = {1, 1, 1};
   return encode(m, a.gate_logits ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,

@@ -57,6 +57,7 @@ struct ChunkArgs {
   // and the buffer that receives the history after the last token (or NULL).
   const void* conv_in;
   void* conv_out;
+  int Hg;            // heads of alpha and b: Hv, or Hqk when the value heads of a QK head share them
 };
 
 struct DecodeArgs {
@@ -72,6 +73,7 @@ struct DecodeArgs {
   const float* conv_w;   // conv taps [2·Hqk·d + Hv·d, 4] or NULL (no conv)
   const void* conv_in;   // conv history before this token, or NULL (zeros)
   void* conv_out;        // history after this token, or NULL
+  int Hg;                // heads of alpha and b (Hv, or Hqk when shared per QK head)
 };
 
 // Launchers (return cudaSuccess or the launch error).

@@ -48,6 +48,7 @@ decode_kernel(DecodeArgs a) {
   const int h = bh % a.Hv;
   const int bi = bh / a.Hv;
   const int hq = h / (a.Hv / a.Hqk);
+  const size_t bg = (size_t)bi * a.Hg + (a.Hg == a.Hv ? h : hq);   // row of alpha, b
   const int tid = threadIdx.x;
   const int cg = tid % CG;
   const int rg = tid / CG;
@@ -88,9 +89,9 @@ decode_kernel(DecodeArgs a) {
   for (int i = tid; i < D; i += NT) {
     s_q[i] = conv1(qg[i], cq + i);
     s_k[i] = conv1(kg[i], ck + i);
-    s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? (size_t)bh : (size_t)bh * D + i);
+    s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
   }
-  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at<LG>(a.b, bh);
+  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at<LG>(a.b, bg);
   for (int j = tid; j < COLS; j += NT) {
     const float wj = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.w, (size_t)bh * D + col0 + j) : beta;
     s_z[j] = wj * conv1(vg[j], cv + j);
@@ -141,7 +142,7 @@ decode_kernel(DecodeArgs a) {
   const float iq = s_scalar[0], ik = s_scalar[1], kq = s_scalar[2];
   for (int i = tid; i < D; i += NT) {
     const float kk = s_k[i] * ik;
-    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.b, (size_t)bh * D + i) : beta;
+    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.b, bg * D + i) : beta;
     s_e[i] = bb * kk;
   }
   __syncthreads();

@@ -43,6 +43,7 @@ class Params(ctypes.Structure):
         ("gate_mode", ctypes.c_int), ("precision", ctypes.c_int), ("l2norm_qk", ctypes.c_int),
         ("conv_w", ctypes.c_void_p), ("gate_logits", ctypes.c_int),
         ("conv_state_in", ctypes.c_void_p), ("conv_state_out", ctypes.c_void_p),
+        ("gate_heads", ctypes.c_int),
     ]
 
 
@@ -111,17 +112,42 @@ def _stream_handle(stream):
 
 def make_params(B, T, H_qk, H_v, d_k, d_v, *, chunk=64, scale=1.0, qkv_dtype=BF16, o_dtype=BF16,
                 gate_mode="full", precision="default", l2norm_qk=False, conv_w=None, gate_logits=False,
-                conv_state_in=None, conv_state_out=None) -> Params:
+                conv_state_in=None, conv_state_out=None, gates_per_qk_head=False) -> Params:
     return Params(int(B), int(T), int(H_qk), int(H_v), int(d_k), int(d_v), int(chunk), float(scale),
                   int(qkv_dtype), int(o_dtype), GATES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode),
                   PRECISION[precision] if isinstance(precision, str) else int(precision),
                   1 if l2norm_qk else 0, _ptr(conv_w), 1 if gate_logits else 0,
-                  _ptr(conv_state_in), _ptr(conv_state_out))
+                  _ptr(conv_state_in), _ptr(conv_state_out), 1 if gates_per_qk_head else 0)
 
 
 def conv_state_shape(B, H_qk, H_v, d_k, d_v):
     """Shape of a conv history buffer: [B, 3, 2·H_qk·d_k + H_v·d_v] (q | k | v channels)."""
     return (B, 3, 2 * H_qk * d_k + H_v * d_v)
+
+
+def _check_shapes(lead, H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates_per_qk_head, states=(),
+                  conv_w=None):
+    """Shapes of everything the call reads or writes, so that no kernel indexes
+    past a tensor: ``lead`` is (B, T) or (B,); ``states`` are [B,H_v,d_k,d_v]."""
+    mode = GATES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode)
+    Hg = H_qk if gates_per_qk_head else H_v
+    want = {"k": lead + (H_qk, d_k), "v": lead + (H_v, d_v)}
+    if mode == GATES["full"]:
+        want.update(alpha=lead + (Hg, d_k), b=lead + (Hg, d_k), w=lead + (H_v, d_v))
+    elif mode == GATES["kda"]:
+        want.update(alpha=lead + (Hg, d_k), b=lead + (Hg,))
+    else:
+        want.update(alpha=lead + (Hg,), b=lead + (Hg,))
+    got = {"k": k, "v": v, "alpha": alpha, "b": b, "w": w}
+    for name, shape in want.items():
+        t = got[name]
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+    for name, t in states:
+        if t is not None and tuple(t.shape) != (lead[0], H_v, d_k, d_v):
+            raise ValueError(f"{name} must have shape {(lead[0], H_v, d_k, d_v)}, got {tuple(t.shape)}")
+    if conv_w is not None and tuple(conv_w.shape) != (2 * H_qk * d_k + H_v * d_v, 4):
+        raise ValueError(f"conv_w must have shape {(2 * H_qk * d_k + H_v * d_v, 4)}, got {tuple(conv_w.shape)}")
 
 
 def _check_conv_state(t, name, qkv_dtype, shape):
@@ -150,13 +176,15 @@ def chunk_fwd_workspace(params: Params) -> int:
 def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_mode="full",
               precision="default", l2norm_qk=False, conv_w=None, o_dtype=None, o=None, S_T=None,
               workspace=None, stream=None, want_state=True, gate_logits=False, conv_state_in=None,
-              conv_state_out=None):
+              conv_state_out=None, gates_per_qk_head=False):
     """Chunked prefill. q,k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; gates per
     ``gate_mode``: fp32 values, or bf16 logits with ``gate_logits`` (the kernels
     apply the sigmoid); S0 [B,H_v,d_k,d_v] fp32 or None. With ``conv_w``, the
     conv history before token 0 comes from ``conv_state_in`` (None: zeros) and
     the history after the last token is written to ``conv_state_out`` (both
-    :func:`conv_state_shape`, q's dtype, distinct buffers). Returns (o, S_T)."""
+    :func:`conv_state_shape`, q's dtype, distinct buffers). With
+    ``gates_per_qk_head`` alpha and b have H_qk heads, shared by the value
+    heads of each QK head. Returns (o, S_T)."""
     B, T, H_qk, d_k = q.shape
     H_v, d_v = v.shape[2], v.shape[3]
     o_dtype = q.dtype if o_dtype is None else o_dtype
@@ -167,18 +195,23 @@ def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_m
         _check(t, name, gdt)
     for name, t in (("S0", S0), ("conv_w", conv_w)):
         _check(t, name, torch.float32)
+    _check_shapes((B, T), H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates_per_qk_head,
+                  states=(("S0", S0), ("S_T", S_T)), conv_w=conv_w)
     hshape = conv_state_shape(B, H_qk, H_v, d_k, d_v)
     _check_conv_state(conv_state_in, "conv_state_in", q.dtype, hshape)
     _check_conv_state(conv_state_out, "conv_state_out", q.dtype, hshape)
     p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
                     o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, precision=precision,
                     l2norm_qk=l2norm_qk, conv_w=conv_w, gate_logits=gate_logits,
-                    conv_state_in=conv_state_in, conv_state_out=conv_state_out)
+                    conv_state_in=conv_state_in, conv_state_out=conv_state_out,
+                    gates_per_qk_head=gates_per_qk_head)
     if o is None:
         o = torch.empty((B, T, H_v, d_v), dtype=o_dtype, device=q.device)
     if S_T is None and want_state:
         S_T = torch.empty((B, H_v, d_k, d_v), dtype=torch.float32, device=q.device)
     _check(o, "o", o_dtype)
+    if tuple(o.shape) != (B, T, H_v, d_v):
+        raise ValueError(f"o must have shape {(B, T, H_v, d_v)}, got {tuple(o.shape)}")
     _check(S_T, "S_T", torch.float32)
     need = chunk_fwd_workspace(p)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
@@ -193,13 +226,14 @@ def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_m
 
 
 def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_qk=False, o_dtype=None,
-                o=None, stream=None, gate_logits=False, conv_w=None, conv_state_in=None, conv_state_out=None):
+                o=None, stream=None, gate_logits=False, conv_w=None, conv_state_in=None, conv_state_out=None,
+                gates_per_qk_head=False):
     """One decode step. q,k [B,H_qk,d_k]; v [B,H_v,d_v]; gates without the T
     axis (fp32 values, or bf16 logits with ``gate_logits``); S [B,H_v,d_k,d_v]
     fp32 updated in place. With ``conv_w`` the step's conv reads
     ``conv_state_in`` (None: zeros) and writes the shifted history to
-    ``conv_state_out`` (a second buffer: swap the two between steps).
-    Returns o [B,H_v,d_v]."""
+    ``conv_state_out`` (a second buffer: swap the two between steps). With
+    ``gates_per_qk_head`` alpha and b have H_qk heads. Returns o [B,H_v,d_v]."""
     B, H_qk, d_k = q.shape
     H_v, d_v = v.shape[1], v.shape[2]
     o_dtype = q.dtype if o_dtype is None else o_dtype
@@ -210,16 +244,20 @@ def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_
         _check(t, name, gdt)
     _check(S, "S", torch.float32)
     _check(conv_w, "conv_w", torch.float32)
+    _check_shapes((B,), H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates_per_qk_head,
+                  states=(("S", S),), conv_w=conv_w)
     hshape = conv_state_shape(B, H_qk, H_v, d_k, d_v)
     _check_conv_state(conv_state_in, "conv_state_in", q.dtype, hshape)
     _check_conv_state(conv_state_out, "conv_state_out", q.dtype, hshape)
     p = make_params(B, 1, H_qk, H_v, d_k, d_v, scale=scale, qkv_dtype=_dtype_code(q.dtype),
                     o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk,
                     gate_logits=gate_logits, conv_w=conv_w, conv_state_in=conv_state_in,
-                    conv_state_out=conv_state_out)
+                    conv_state_out=conv_state_out, gates_per_qk_head=gates_per_qk_head)
     if o is None:
         o = torch.empty((B, H_v, d_v), dtype=o_dtype, device=q.device)
     _check(o, "o", o_dtype)
+    if tuple(o.shape) != (B, H_v, d_v):
+        raise ValueError(f"o must have shape {(B, H_v, d_v)}, got {tuple(o.shape)}")
     st = lib().gdn2_decode_step(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
                                 _ptr(S), _ptr(o), _stream_handle(stream))
     if st != OK:
@@ -228,7 +266,8 @@ def decode_step(q, k, v, alpha, b, w, S, *, scale=1.0, gate_mode="full", l2norm_
 
 
 def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=64, scale=1.0,
-                      gate_mode="full", l2norm_qk=False, conv_w=None, stream=None, gate_logits=False):
+                      gate_mode="full", l2norm_qk=False, conv_w=None, stream=None, gate_logits=False,
+                      gates_per_qk_head=False):
     """Chunked prefill through ``gdn2_chunk_fwd_noalloc``: the library takes the
     kernel's scratch from its own fixed device array, so nothing is allocated
     for the call. ``o`` and ``S_T`` (or None) are caller-provided outputs (the
@@ -247,9 +286,13 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=
     for name, t in (("S0", S0), ("S_T", S_T), ("conv_w", conv_w)):
         _check(t, name, torch.float32)
     _check(o, "o")
+    _check_shapes((B, T), H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates_per_qk_head,
+                  states=(("S0", S0), ("S_T", S_T)), conv_w=conv_w)
+    if tuple(o.shape) != (B, T, H_v, d_v):
+        raise ValueError(f"o must have shape {(B, T, H_v, d_v)}, got {tuple(o.shape)}")
     p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
                     o_dtype=_dtype_code(o.dtype), gate_mode=gate_mode, l2norm_qk=l2norm_qk, conv_w=conv_w,
-                    gate_logits=gate_logits)
+                    gate_logits=gate_logits, gates_per_qk_head=gates_per_qk_head)
     st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
             _ptr(S_T), _stream_handle(stream))
     if st != OK:

@@ -96,7 +96,7 @@ def _qkv_dtype(w: Workload):
 
 
 def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: str = "full",
-                gate_logits: bool = False):
+                gate_logits: bool = False, gates_per_qk_head: bool = False):
     """Draw one batch of inputs for workload ``w``.
 
     gate_mode "full": alpha, b [B,T,Hv,dk], w [B,T,Hv,dv].
@@ -104,7 +104,8 @@ def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: s
     gate_mode "gdn":  alpha [B,T,Hv] (mean 4), b = beta [B,T,Hv], w = None.
     Returns a dict of tensors on ``device`` (q,k,v in the workload's dtype;
     gates float32 sigmoids of normal draws, or with ``gate_logits`` those
-    draws themselves rounded to bf16; S0 and conv weights float32).
+    draws themselves rounded to bf16; S0 and conv weights float32). With
+    ``gates_per_qk_head`` alpha and b (beta) have H_qk heads instead of H_v.
     """
     if seed is None:
         seed = WORKLOADS.index(BY_NAME[w.name]) if w.name in BY_NAME else 0
@@ -121,17 +122,18 @@ def make_inputs(w: Workload, seed: int | None = None, device="cpu", gate_mode: s
     dt = _qkv_dtype(w)
     out["q"], out["k"], out["v"] = q.to(dt), k.to(dt), v.to(dt)
     gate = (lambda x: x.to(torch.bfloat16)) if gate_logits else torch.sigmoid
+    Hg = Hqk if gates_per_qk_head else Hv     # heads of alpha and b
     if gate_mode == "full":
-        out["alpha"] = gate(_normal((B, T, Hv, d), _gen(seed, 4, dev), dev, mean=w.alpha_mu))
-        out["b"] = gate(_normal((B, T, Hv, d), _gen(seed, 5, dev), dev))
+        out["alpha"] = gate(_normal((B, T, Hg, d), _gen(seed, 4, dev), dev, mean=w.alpha_mu))
+        out["b"] = gate(_normal((B, T, Hg, d), _gen(seed, 5, dev), dev))
         out["w"] = gate(_normal((B, T, Hv, d), _gen(seed, 6, dev), dev))
     elif gate_mode == "kda":
-        out["alpha"] = gate(_normal((B, T, Hv, d), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
-        out["b"] = gate(_normal((B, T, Hv), _gen(seed, 5, dev), dev))
+        out["alpha"] = gate(_normal((B, T, Hg, d), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
+        out["b"] = gate(_normal((B, T, Hg), _gen(seed, 5, dev), dev))
         out["w"] = None
     elif gate_mode == "gdn":
-        out["alpha"] = gate(_normal((B, T, Hv), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
-        out["b"] = gate(_normal((B, T, Hv), _gen(seed, 5, dev), dev))
+        out["alpha"] = gate(_normal((B, T, Hg), _gen(seed, 4, dev), dev, mean=TIED_ALPHA_MU))
+        out["b"] = gate(_normal((B, T, Hg), _gen(seed, 5, dev), dev))
         out["w"] = None
     else:
         raise ValueError(gate_mode)
@@ -156,13 +158,13 @@ def make_conv_state(w: Workload, seed: int, device="cpu"):
 
 
 def make_decode_pool(w: Workload, pool: int = 16, seed: int | None = None, device="cpu",
-                     gate_mode: str = "full", gate_logits: bool = False):
+                     gate_mode: str = "full", gate_logits: bool = False, gates_per_qk_head: bool = False):
     """Per-step decode inputs: ``pool`` independent one-token step sets, cycled by
     the caller, plus the initial state. Tensors carry a leading pool axis."""
     if seed is None:
         seed = 3
     steps = make_inputs(replace(w, T=pool, s0="zeros"), seed=seed, device=device, gate_mode=gate_mode,
-                        gate_logits=gate_logits)
+                        gate_logits=gate_logits, gates_per_qk_head=gates_per_qk_head)
     # [B, pool, ...] -> [pool, B, ...]
     for key in ("q", "k", "v", "alpha", "b", "w"):
         if steps[key] is not None:

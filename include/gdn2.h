@@ -63,11 +63,23 @@ typedef enum {
 
 typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
 
-/* Gate layouts ([B,T,...] for gdn2_chunk_fwd; drop T for gdn2_decode_step):
- *   GDN2_GATES_FULL  alpha [B,T,H_v,d_k], b [B,T,H_v,d_k], w [B,T,H_v,d_v]
- *   GDN2_GATES_KDA   alpha [B,T,H_v,d_k], b = beta [B,T,H_v], w = NULL
- *   GDN2_GATES_GDN   alpha [B,T,H_v],     b = beta [B,T,H_v], w = NULL      */
+/* Gate layouts ([B,T,...] for gdn2_chunk_fwd; drop T for gdn2_decode_step),
+ * with H_g = H_v (gdn2_params.gate_heads = GDN2_GATE_HEADS_V) or H_g = H_qk
+ * (GDN2_GATE_HEADS_QK: alpha and b shared by the value heads of a QK head):
+ *   GDN2_GATES_FULL  alpha [B,T,H_g,d_k], b [B,T,H_g,d_k], w [B,T,H_v,d_v]
+ *   GDN2_GATES_KDA   alpha [B,T,H_g,d_k], b = beta [B,T,H_g], w = NULL
+ *   GDN2_GATES_GDN   alpha [B,T,H_g],     b = beta [B,T,H_g], w = NULL      */
 typedef enum { GDN2_GATES_FULL = 0, GDN2_GATES_KDA = 1, GDN2_GATES_GDN = 2 } gdn2_gate_mode;
+
+/* Which heads own the decay and erase gates (alpha, b; beta in the tied
+ * modes). The pages do not say; GDN2_GATE_HEADS_V gives every value head (the
+ * owner of a state) its own. GDN2_GATE_HEADS_QK shares them among the value
+ * heads that read one query/key head (value head h uses the gates of QK head
+ * h / (H_v / H_qk)): both gate the key axis, which those heads share; w, on
+ * the value axis, stays per value head. Same results as GDN2_GATE_HEADS_V
+ * with each gate row repeated for the heads of its group, H_v/H_qk times
+ * fewer gate bytes.                                                          */
+typedef enum { GDN2_GATE_HEADS_V = 0, GDN2_GATE_HEADS_QK = 1 } gdn2_gate_heads;
 
 /* Arithmetic of gdn2_chunk_fwd:
  *   GDN2_PREC_DEFAULT  bf16 q,k,v with d_k = d_v = 128 and chunk 64 run on the
@@ -120,6 +132,7 @@ typedef struct {
                      split prefills and decode steps. Must not overlap
                      conv_state_in or any other argument (swap two buffers
                      between calls). Needs conv_w.                            */
+  int gate_heads;  /* gdn2_gate_heads of alpha and b (0: per value head)       */
 } gdn2_params;
 
 /* Human-readable name of a status code (static string, never NULL). */

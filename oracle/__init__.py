@@ -15,6 +15,8 @@ Functions and the passages they follow:
 * :func:`expand_tied_gates` -- the reductions of the same section: tying
   ``b_t`` and ``w_t`` to one scalar ``β_t`` gives KDA; tying ``α_t`` to a
   scalar as well gives Gated DeltaNet.
+* :func:`gates_for_value_heads` -- gates shared per query/key head, given to
+  each value head of the group (its contiguous head grouping).
 * :func:`causal_conv4` -- depthwise causal convolution with kernel 4
   ("Gated DeltaNet: o mixer em 48 das 64 camadas", Conceito).
 * :func:`l2norm` -- row-wise L2 normalisation of queries and keys (the pages
@@ -122,6 +124,17 @@ def expand_tied_gates(mode: str, alpha, beta, d_k: int, d_v: int):
     elif mode != "kda":
         raise ValueError(mode)
     return alpha, b, w
+
+
+def gates_for_value_heads(g, H_v: int, axis: int = 2):
+    """Gates owned by query/key heads, head axis ``axis`` ([B,T,H_qk,...]; 1
+    for one step's [B,H_qk,...]), repeated for the value heads that read each
+    QK head: value head h takes QK head h // (H_v / H_qk), the contiguous
+    grouping of "Gated DeltaNet: o mixer em 48 das 64 camadas", Conceito."""
+    g = _f64(g)
+    H_qk = g.shape[axis]
+    assert H_v % H_qk == 0
+    return np.repeat(g, H_v // H_qk, axis=axis)
 
 
 def causal_conv4(x, W, history=None):

@@ -14,19 +14,23 @@ def np64(t):
     return None if t is None else t.detach().to(torch.float64).cpu().numpy()
 
 
-def oracle_gates(mode, alpha, b, w, d_k, d_v, gate_logits=False):
+def oracle_gates(mode, alpha, b, w, d_k, d_v, gate_logits=False, H_v=None, head_axis=2):
     """Per-channel float64 gates for the oracle from the tensors the kernel gets
-    (bf16 logits pass through the oracle's sigmoid first)."""
+    (bf16 logits pass through the oracle's sigmoid first; with ``H_v``, alpha
+    and b are owned by QK heads and given to each value head of the group)."""
     f = oracle.gates_from_logits if gate_logits else (lambda x: x)
     alpha, b = f(np64(alpha)), f(np64(b))
     w = None if w is None else f(np64(w))
+    if H_v is not None:
+        alpha = oracle.gates_for_value_heads(alpha, H_v, head_axis)
+        b = oracle.gates_for_value_heads(b, H_v, head_axis)
     if mode == "full":
         return alpha, b, w
     return oracle.expand_tied_gates(mode, alpha, b, d_k, d_v)
 
 
 def oracle_chunk(inp, gate_mode="full", scale=1.0, l2norm_qk=False, S0=None, threads=0,
-                 heads=None, gate_logits=False, conv_state=None):
+                 heads=None, gate_logits=False, conv_state=None, gates_per_qk_head=False):
     """Oracle (o, S_T) for a chunk_fwd input dict (``conv_state``: the conv
     history before token 0, or None). ``heads`` optionally restricts to a list of
     (sequence, value head) pairs; returns dict keyed by pair then."""
@@ -35,7 +39,8 @@ def oracle_chunk(inp, gate_mode="full", scale=1.0, l2norm_qk=False, S0=None, thr
     conv_w = np64(inp.get("conv_w"))
     conv_state = np64(conv_state)
     S0 = np64(inp.get("S0")) if S0 is None else np64(S0)
-    alpha, b, w = oracle_gates(gate_mode, inp["alpha"], inp["b"], inp.get("w"), d_k, d_v, gate_logits)
+    alpha, b, w = oracle_gates(gate_mode, inp["alpha"], inp["b"], inp.get("w"), d_k, d_v, gate_logits,
+                               H_v=v.shape[2] if gates_per_qk_head else None)
     if heads is None:
         qp, kp, vp = oracle.preprocess(q, k, v, conv_w, l2norm_qk, conv_state)
         return oracle.gdn2_forward(qp, kp, vp, alpha, b, w, S0, scale=scale, threads=threads)

@@ -47,11 +47,11 @@ def test_status_strings_and_version(L):
 
 def _params(**kw):
     base = dict(B=1, T=64, H_qk=1, H_v=1, d_k=16, d_v=16, chunk=16, qkv_dtype=gdn2.F32, o_dtype=gdn2.F32)
-    raw_logits = kw.pop("gate_logits", None)
+    raw = {f: kw.pop(f) for f in ("gate_logits", "gate_heads") if f in kw}
     base.update(kw)
     p = gdn2.make_params(**base)
-    if raw_logits is not None:
-        p.gate_logits = int(raw_logits)   # raw field value, including invalid ones
+    for f, val in raw.items():
+        setattr(p, f, int(val))           # raw field value, including invalid ones
     return p
 
 
@@ -79,6 +79,7 @@ def _call_chunk(L, p, **ptrs):
     (dict(precision=3), gdn2.ERR_INVALID_ARG),
     (dict(scale=float("nan")), gdn2.ERR_INVALID_ARG),
     (dict(gate_logits=2), gdn2.ERR_INVALID_ARG),
+    (dict(gate_heads=2), gdn2.ERR_INVALID_ARG),
 ])
 def test_chunk_rejects_bad_params(L, kw, expect):
     assert _call_chunk(L, _params(**kw)) == expect
@@ -148,7 +149,7 @@ def _header_param_fields():
 def test_params_mirror_matches_header_field_order():
     names = [f[0] for f in gdn2.Params._fields_]
     assert names == _header_param_fields()
-    assert names[-4:] == ["conv_w", "gate_logits", "conv_state_in", "conv_state_out"]
+    assert names[-5:] == ["conv_w", "gate_logits", "conv_state_in", "conv_state_out", "gate_heads"]
     assert gdn2.make_params(1, 1, 1, 1, 16, 16, gate_logits=True).gate_logits == 1
     assert gdn2.conv_state_shape(2, 16, 48, 128, 128) == (2, 3, 10240)
 

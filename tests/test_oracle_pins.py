@@ -427,6 +427,35 @@ def test_preprocess_order_conv_then_norm():
     np.testing.assert_array_equal(vp, vc)
 
 
+def test_gates_for_value_heads_mapping_and_group_symmetry():
+    """Value head h takes the gates of QK head h // (H_v/H_qk) (contiguous
+    groups); and with gates shared, the heads of one group that also get the
+    same v and w run identical recurrences (a consequence of sharing q, k and
+    the key-side gates), while heads of different groups do not."""
+    B, T, Hqk, Hv, d = 1, 6, 2, 6, 4
+    g = np.arange(B * T * Hqk * d, dtype=float).reshape(B, T, Hqk, d)
+    e = oracle.gates_for_value_heads(g, Hv)
+    assert e.shape == (B, T, Hv, d)
+    for h in range(Hv):
+        np.testing.assert_array_equal(e[:, :, h], g[:, :, h // 3])
+    s = np.arange(4, dtype=float).reshape(2, 2)          # one step: [B, H_qk]
+    np.testing.assert_array_equal(oracle.gates_for_value_heads(s, 4, axis=1), [[0, 0, 1, 1], [2, 2, 3, 3]])
+    r = _rng(34)
+    q = _unit(r.standard_normal((B, T, Hqk, d)))
+    k = _unit(r.standard_normal((B, T, Hqk, d)))
+    v1 = r.standard_normal((B, T, 1, d))
+    w1 = 1.0 / (1.0 + np.exp(-r.standard_normal((B, T, 1, d))))
+    v, w = np.repeat(v1, Hv, axis=2), np.repeat(w1, Hv, axis=2)
+    a = oracle.gates_for_value_heads(1.0 / (1.0 + np.exp(-3.0 - r.standard_normal((B, T, Hqk, d)))), Hv)
+    b = oracle.gates_for_value_heads(1.0 / (1.0 + np.exp(-r.standard_normal((B, T, Hqk, d)))), Hv)
+    qv, kv = np.repeat(q, 3, axis=2), np.repeat(k, 3, axis=2)
+    o, S = oracle.gdn2_forward(qv, kv, v, a, b, w)
+    for h in (1, 2):
+        np.testing.assert_array_equal(o[:, :, h], o[:, :, 0])
+        np.testing.assert_array_equal(S[:, h], S[:, 0])
+    assert np.abs(o[:, :, 3] - o[:, :, 0]).max() > 1e-3
+
+
 def test_rel_err_metric():
     ref = np.array([3.0, -4.0])
     assert oracle.rel_err(ref, ref) == 0.0
