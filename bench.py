@@ -4,14 +4,17 @@ One step = one chunked prefill (gdn2_chunk_fwd) of the 48-V-head, d=128 layer
 over T=32768 tokens of one sequence (bf16 q,k,v, fp32 per-channel gates,
 chunk 64), inputs resident in HBM. The decode workload (B=256 sequences, one
 token per step, fp32 states [256,48,128,128]) is timed in the same run and
-reported under "decode".
+reported under "decode"; so are the conv + L2 prefill (B=8, T=8192,
+"conv_prefill") and the headline prefill with other gate layouts (bf16
+logits, "prefill_gate_logits"; alpha and b per QK head, "prefill_qk_gates").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill_t32768|prefill_t4096] [--decode-workload decode_b256|decode_b64]
-                    [--decode-steps N] [--e2e-steps N]
+                    [--decode-steps N] [--conv-steps N] [--e2e-steps N] [--logits-steps N]
+                    [--qk-gates-steps N]
 
 (--workload prefill_t4096 / --decode-workload decode_b64 are the small cases
-the ncu captures run; --decode-steps 0 / --e2e-steps 0 skip those parts.)
+the ncu captures run; a count of 0 skips that part.)
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own sequence
 (independent problems, no data-path collective); value = tokens of all ranks /
@@ -69,18 +72,20 @@ def peaks():
 
 # ------------------------------------------------------------------ accounting
 
-def prefill_bytes(w, gate_mode="full", o_bytes=2, s0=False, gate_bytes=4):
+def prefill_bytes(w, gate_mode="full", o_bytes=2, s0=False, gate_bytes=4, qk_gates=False):
     """Algorithmic HBM bytes of one chunk_fwd call: every input read once, every
-    output written once (gate_bytes: 4 for fp32 gate values, 2 for bf16 logits)."""
+    output written once (gate_bytes: 4 for fp32 gate values, 2 for bf16 logits;
+    qk_gates: alpha and b owned by the QK heads, H_qk of them)."""
     tok = w.B * w.T
     qkb = 2 if w.qkv_dtype == "bf16" else 4
     n = tok * w.H_qk * w.d * qkb * 2 + tok * w.H_v * w.d * qkb
+    hg = w.H_qk if qk_gates else w.H_v
     if gate_mode == "full":
-        n += tok * w.H_v * w.d * gate_bytes * 3
+        n += tok * (2 * hg + w.H_v) * w.d * gate_bytes
     elif gate_mode == "kda":
-        n += tok * w.H_v * (w.d + 1) * gate_bytes
+        n += tok * hg * (w.d + 1) * gate_bytes
     else:
-        n += tok * w.H_v * 2 * gate_bytes
+        n += tok * hg * 2 * gate_bytes
     n += tok * w.H_v * w.d * o_bytes
     n += w.B * w.H_v * w.d * w.d * 4 * (2 if s0 else 1)
     if w.conv:
@@ -346,6 +351,8 @@ def main():
     ap.add_argument("--decode-workload", default=DECODE, choices=[DECODE, "decode_b64"])
     ap.add_argument("--logits-steps", type=int, default=20,
                     help="timed calls of the T=32768 prefill with bf16 gate logits; 0 skips it")
+    ap.add_argument("--qk-gates-steps", type=int, default=20,
+                    help="timed calls of the T=32768 prefill with alpha, b per QK head; 0 skips it")
     ap.add_argument("--conv-steps", type=int, default=5,
                     help="timed calls of the conv + L2 workload (B=8, T=8192); 0 skips it")
     args = ap.parse_args()
@@ -436,7 +443,10 @@ def main():
     # ---------------------------------------------------------------- gates as bf16 logits
     logits = None
     if args.logits_steps > 0:
-        logits = run_logits(args, w, dev, stream, barrier, pk, world)
+        logits = run_gate_variant(args.logits_steps, w, dev, stream, barrier, pk, world, gate_logits=True)
+    qk_gates = None
+    if args.qk_gates_steps > 0:
+        qk_gates = run_gate_variant(args.qk_gates_steps, w, dev, stream, barrier, pk, world, qk=True)
 
     # ---------------------------------------------------------------- end to end
     e2e = None
@@ -465,7 +475,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
-            "conv_prefill": conv, "prefill_gate_logits": logits,
+            "conv_prefill": conv, "prefill_gate_logits": logits, "prefill_qk_gates": qk_gates,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -552,22 +562,24 @@ def run_conv(args, dev, stream, barrier, pk, world):
             "gpu_launches": 3 * args.conv_steps}
 
 
-def run_logits(args, w, dev, stream, barrier, pk, world):
-    """The headline layer and length with the gates given as bf16 logits (the
-    kernels apply the sigmoid): half the gate bytes of the fp32 values."""
+def run_gate_variant(steps, w, dev, stream, barrier, pk, world, gate_logits=False, qk=False):
+    """The headline layer and length with another gate layout: bf16 logits
+    (the kernels apply the sigmoid; half the gate bytes), or alpha and b owned
+    by the QK heads (a third of their bytes at 48 V / 16 QK heads)."""
     import torch
     from delta_rule_linear_gdn_b200 import gdn2
     from delta_rule_linear_gdn_b200.inputs import make_inputs
     rank = int(os.environ.get("RANK", "0"))
-    inp = make_inputs(w, seed=rank_seed(rank), device=dev, gate_logits=True)
+    inp = make_inputs(w, seed=rank_seed(rank), device=dev, gate_logits=gate_logits, gates_per_qk_head=qk)
     o = torch.empty((w.B, w.T, w.H_v, w.d), dtype=torch.bfloat16, device=dev)
     S_T = torch.empty((w.B, w.H_v, w.d, w.d), dtype=torch.float32, device=dev)
-    p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk, gate_logits=True)
+    p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk, gate_logits=gate_logits,
+                         gates_per_qk_head=qk)
     ws = torch.empty(max(gdn2.chunk_fwd_workspace(p), 1), dtype=torch.uint8, device=dev)
 
     def call():
         gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None, chunk=w.chunk,
-                       o=o, S_T=S_T, workspace=ws, stream=stream, gate_logits=True)
+                       o=o, S_T=S_T, workspace=ws, stream=stream, gate_logits=gate_logits, gates_per_qk_head=qk)
 
     with torch.cuda.stream(stream):
         for _ in range(3):
@@ -577,19 +589,21 @@ def run_logits(args, w, dev, stream, barrier, pk, world):
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     c0.record(stream)
     with torch.cuda.stream(stream):
-        for _ in range(args.logits_steps):
+        for _ in range(steps):
             call()
     c1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    lms = max_over_ranks(c0.elapsed_time(c1) / args.logits_steps, dev)
-    nbytes = prefill_bytes(w, gate_bytes=2)
+    lms = max_over_ranks(c0.elapsed_time(c1) / steps, dev)
+    nbytes = prefill_bytes(w, gate_bytes=2 if gate_logits else 4, qk_gates=qk)
     gbs = nbytes / (lms * 1e-3) / 1e9
-    return {"workload": f"{w.name} with the gates as bf16 logits (sigmoid in the kernels)",
+    what = ("the gates as bf16 logits (sigmoid in the kernels)" if gate_logits else
+            "alpha and b per QK head (shared by its 3 value heads), fp32")
+    return {"workload": f"{w.name} with {what}",
             "ms_per_call": lms, "tokens_per_s": w.B * w.T * world / (lms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes},
-            "gpu_launches": args.logits_steps * tc_launches_per_call(w, gdn2.chunk_fwd_workspace(p), dev)}
+            "gpu_launches": steps * tc_launches_per_call(w, gdn2.chunk_fwd_workspace(p), dev)}
 
 
 def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):

@@ -238,7 +238,10 @@ __device__ __forceinline__ size_t slot_index(SlotMap m, int bh, int j) {
 // Items are taken in order (chunk-major, value head fastest): by a fixed stride
 // of the grid, or, with `counter`, one at a time from that device counter
 // (zero before the launch), so that CTAs which start late take fewer.
-template <bool F16IN, bool LG>
+// F16IN: q, k, v are the load step's fp16 copies; LG: the gates are bf16
+// logits; QKG: alpha and b belong to the QK heads (one compiled copy each, so
+// that no form pays for the others' addressing at the register limit).
+template <bool F16IN, bool LG, bool QKG>
 __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
                                                            int* counter, const __grid_constant__ CUtensorMap amap,
                                                            int use_amap) {
@@ -303,9 +306,9 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   float4 bq[4];
   uint2 kk[4], qq[4];
   // rows of alpha, b (per value head, or shared per QK head) and of w
-  const bool g_qk = a.Hg != a.Hv;
   auto gate_row = [&](const Item& it, int u) -> size_t {
-    return ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hg + (g_qk ? it.hq : it.h);
+    const size_t r = (size_t)it.bi * a.T + it.t0 + i0 + u;
+    return QKG ? r * a.Hqk + it.hq : r * a.Hv + it.h;
   };
   auto w_row = [&](const Item& it, int u) -> size_t {
     return full ? ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hv + it.h : gate_row(it, u);
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   auto fetch_alpha = [&](int item_) {
     const Item nx = decode_item(a, c_begin, item_);
     mbar_arrive_expect_tx(bar_a, C * D * (LG ? 2 : 4));
-    tma_load_3d(smem + P_ALPHA, &amap, 0, a.Hg != a.Hv ? nx.hq : nx.h, nx.bi * a.T + nx.t0, bar_a);
+    tma_load_3d(smem + P_ALPHA, &amap, 0, QKG ? nx.hq : nx.h, nx.bi * a.T + nx.t0, bar_a);
   };
   uint32_t phase_a = 0;
   auto load_alpha_key0 = [&](int item_) {
@@ -1339,8 +1342,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   if (seg < 1) return cudaErrorInvalidValue;
   __half* qkv = reinterpret_cast<__half*>(ws + WS_HEAD + (size_t)BH * seg * SLOT);
 
-  for (auto prep : {chunk_prep_kernel<false, false>, chunk_prep_kernel<true, false>, chunk_prep_kernel<false, true>,
-                     chunk_prep_kernel<true, true>}) {
+  for (auto prep : {chunk_prep_kernel<false, false, false>, chunk_prep_kernel<true, false, false>,
+                     chunk_prep_kernel<false, true, false>, chunk_prep_kernel<true, true, false>,
+                     chunk_prep_kernel<false, false, true>, chunk_prep_kernel<true, false, true>,
+                     chunk_prep_kernel<false, true, true>, chunk_prep_kernel<true, true, true>}) {
     if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) != cudaSuccess)
       return e;
     // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
@@ -1371,6 +1376,15 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   CUtensorMap amap{};
   const int use_amap = a.gate_mode != GDN2_GATES_GDN && a.alpha != nullptr && encode_alpha_map(a, &amap) ? 1 : 0;
   const int qp_groups = (2 * a.Hqk + a.Hv) * (D / 8);
+  const bool qkg = a.Hg != a.Hv;
+  using PrepFn = void (*)(ChunkArgs, int, int, SlotMap, int*, const CUtensorMap, int);
+  auto prep_fn = [&](bool f16in) -> PrepFn {
+    if (f16in)
+      return a.gate_logits ? (qkg ? chunk_prep_kernel<true, true, true> : chunk_prep_kernel<true, true, false>)
+                           : (qkg ? chunk_prep_kernel<true, false, true> : chunk_prep_kernel<true, false, false>);
+    return a.gate_logits ? (qkg ? chunk_prep_kernel<false, true, true> : chunk_prep_kernel<false, true, false>)
+                         : (qkg ? chunk_prep_kernel<false, false, true> : chunk_prep_kernel<false, false, false>);
+  };
 
   // overlapped segments: whole sequence in the workspace, idle SMs beside the
   // scan, no load step (its kernel would wait for the scan), S_T given (the
@@ -1411,15 +1425,15 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       ap.qkv_f16 = 1;
       ap.conv_w = nullptr;
       ap.l2norm = 0;
-      (a.gate_logits ? chunk_prep_kernel<true, true> : chunk_prep_kernel<true, false>)<<<grid, NP, P_SMEM, s>>>(
+      prep_fn(true)<<<grid, NP, P_SMEM, s>>>(
           ap, c0, n, sm, counter, amap, use_amap);
     } else if (nseg_ov > 0 && k > 0) {
-      if ((e = launch_dependent(a.gate_logits ? chunk_prep_kernel<false, true> : chunk_prep_kernel<false, false>,
+      if ((e = launch_dependent(prep_fn(false),
                                 grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap, use_amap)) !=
           cudaSuccess)
         return e;
     } else {
-      (a.gate_logits ? chunk_prep_kernel<false, true> : chunk_prep_kernel<false, false>)<<<grid, NP, P_SMEM, s>>>(
+      prep_fn(false)<<<grid, NP, P_SMEM, s>>>(
           a, c0, n, sm, counter, amap, use_amap);
     }
     scan<<<scan_ctas, scan_threads, scan_smem, s>>>(a, c0, n, sm, s_in, s_out);
