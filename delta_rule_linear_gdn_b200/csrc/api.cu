@@ -23,6 +23,22 @@ bool overlaps(const void* p, size_t n, const void* q, size_t m) {
 
 size_t dsize(int dtype) { return dtype == GDN2_BF16 ? 2 : 4; }
 
+// Sequences that own a state: n_seqs for packed sequences of different lengths, else B.
+size_t n_states(const gdn2_params* p) { return p->cu_seqlens ? (size_t)p->n_seqs : (size_t)p->B; }
+
+// Packed sequences (cu_seqlens): one row of B, 1..GDN2_MAX_SEQS sequences whose
+// host offsets start at 0, never decrease and end at T.
+gdn2_status check_varlen(const gdn2_params* p, bool decode) {
+  if (!p->cu_seqlens) return p->n_seqs == 0 ? GDN2_OK : GDN2_ERR_INVALID_ARG;
+  if (decode) return GDN2_ERR_INVALID_ARG;
+  if (p->B != 1 || p->n_seqs < 1 || p->n_seqs > GDN2_MAX_SEQS) return GDN2_ERR_INVALID_ARG;
+  const int* cu = p->cu_seqlens;
+  if (cu[0] != 0 || cu[p->n_seqs] != p->T) return GDN2_ERR_INVALID_ARG;
+  for (int n = 0; n < p->n_seqs; ++n)
+    if (cu[n + 1] < cu[n]) return GDN2_ERR_INVALID_ARG;
+  return GDN2_OK;
+}
+
 // Shared shape/enum checks. tokens = B*T (chunk) or B (decode).
 gdn2_status check_common(const gdn2_params* p, bool decode) {
   if (!p) return GDN2_ERR_INVALID_ARG;
@@ -36,6 +52,7 @@ gdn2_status check_common(const gdn2_params* p, bool decode) {
   if (p->gate_heads != GDN2_GATE_HEADS_V && p->gate_heads != GDN2_GATE_HEADS_QK) return GDN2_ERR_INVALID_ARG;
   if (p->precision != GDN2_PREC_DEFAULT && p->precision != GDN2_PREC_FP32) return GDN2_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return GDN2_ERR_INVALID_ARG;
+  if (check_varlen(p, decode) != GDN2_OK) return GDN2_ERR_INVALID_ARG;
   if (p->d_k != p->d_v || !supported_dim(p->d_k)) return GDN2_ERR_UNSUPPORTED;
   // Element counts must fit comfortably in 63 bits and grid sizes in 31.
   const double elems = (double)p->B * (decode ? 1.0 : (double)p->T) * p->H_v * p->d_k;
@@ -58,7 +75,7 @@ Sizes sizes(const gdn2_params* p, size_t tokens) {
   s.ga = tokens * hg * (p->gate_mode == GDN2_GATES_GDN ? 1 : dk) * gsz;
   s.gb = tokens * hg * (p->gate_mode == GDN2_GATES_FULL ? dk : 1) * gsz;
   s.gw = p->gate_mode == GDN2_GATES_FULL ? tokens * p->H_v * dv * gsz : 0;
-  s.st = (size_t)p->B * p->H_v * dk * dv * 4;
+  s.st = n_states(p) * p->H_v * dk * dv * 4;
   return s;
 }
 
@@ -77,7 +94,7 @@ gdn2_status check_conv_state(const gdn2_params* p, const Range* ins, int n_in, c
   void* hout = p->conv_state_out;
   if (!p->conv_w && (hin || hout)) return GDN2_ERR_INVALID_ARG;
   if (!aligned16(hin) || !aligned16(hout)) return GDN2_ERR_INVALID_ARG;
-  const size_t hb = (size_t)p->B * 3 * ((size_t)2 * p->H_qk * p->d_k + (size_t)p->H_v * p->d_v) *
+  const size_t hb = n_states(p) * 3 * ((size_t)2 * p->H_qk * p->d_k + (size_t)p->H_v * p->d_v) *
                     dsize(p->qkv_dtype);
   if (overlaps(hout, hb, hin, hb)) return GDN2_ERR_INVALID_ARG;
   for (int i = 0; i < n_in; ++i)
@@ -102,6 +119,16 @@ ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, co
   a.conv_in = p->conv_state_in;
   a.conv_out = p->conv_state_out;
   a.Hg = p->gate_heads == GDN2_GATE_HEADS_QK ? p->H_qk : p->H_v;
+  a.nseq = 0;
+  if (p->cu_seqlens) {
+    // B becomes the number of sequences; the 64-token chunks of the
+    // tensor-core prefill start anew in every sequence.
+    a.nseq = p->n_seqs;
+    a.B = p->n_seqs;
+    a.cu_chk[0] = 0;
+    for (int n = 0; n <= p->n_seqs; ++n) a.cu_tok[n] = p->cu_seqlens[n];
+    for (int n = 0; n < p->n_seqs; ++n) a.cu_chk[n + 1] = a.cu_chk[n] + (a.cu_tok[n + 1] - a.cu_tok[n] + 63) / 64;
+  }
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S0 = S0; a.o = o; a.ST = S_T;
   a.workspace = ws; a.ws_bytes = ws_bytes;
   return a;

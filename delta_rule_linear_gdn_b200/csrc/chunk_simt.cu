@@ -109,10 +109,12 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
     sS[idx] = a.S0 ? a.S0[((size_t)bh * D + r) * D + col0 + c] : 0.f;
   }
 
-  const int nchunks = (a.T + C - 1) / C;
+  const size_t tok0 = seq_tok0(a, bi);     // first token of the sequence in the buffers
+  const int Tn = seq_len(a, bi);
+  const int nchunks = (Tn + C - 1) / C;
   for (int ck = 0; ck < nchunks; ++ck) {
     const int t0 = ck * C;
-    const int Lc = min(C, a.T - t0);
+    const int Lc = min(C, Tn - t0);
     __syncthreads();
 
     // 1. Load q, k, log α, b (key side) and z = w ⊙ v (value tile).
@@ -121,10 +123,10 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
       float qv = 0.f, kv = 0.f, gv = 0.f, bv = 0.f;
       if (i < Lc) {
         const int t = t0 + i;
-        const size_t qk0 = (size_t)bi * a.T * qk_tok + (size_t)hq * D + c;
+        const size_t qk0 = tok0 * qk_tok + (size_t)hq * D + c;
         qv = load_conv(qg + qk0, qk_tok, t, conv ? wq + c * 4 : nullptr, conv, hq_ ? hq_ + c : nullptr, hstride);
         kv = load_conv(kg + qk0, qk_tok, t, conv ? wk + c * 4 : nullptr, conv, hk_ ? hk_ + c : nullptr, hstride);
-        const size_t gt = ((size_t)bi * a.T + t) * a.Hg + hg;   // row of alpha, b
+        const size_t gt = (tok0 + t) * a.Hg + hg;   // row of alpha, b
         gv = logf(gate_at(a.alpha, mode == GDN2_GATES_GDN ? gt : gt * D + c, a.gate_logits));
         bv = gate_at(a.b, (mode == GDN2_GATES_FULL) ? gt * D + c : gt, a.gate_logits);
       }
@@ -138,9 +140,9 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
       float zv = 0.f;
       if (i < Lc) {
         const int t = t0 + i;
-        const size_t gt = ((size_t)bi * a.T + t) * a.Hv + h;     // row of w
-        const size_t gtb = ((size_t)bi * a.T + t) * a.Hg + hg;   // row of b (= β, tied modes)
-        const float vv = load_conv(vg + (size_t)bi * a.T * v_tok + (size_t)h * D + col0 + c, v_tok, t,
+        const size_t gt = (tok0 + t) * a.Hv + h;     // row of w
+        const size_t gtb = (tok0 + t) * a.Hg + hg;   // row of b (= β, tied modes)
+        const float vv = load_conv(vg + tok0 * v_tok + (size_t)h * D + col0 + c, v_tok, t,
                                    conv ? wv + (col0 + c) * 4 : nullptr, conv, hv_ ? hv_ + c : nullptr, hstride);
         const float wv_ = (mode == GDN2_GATES_FULL) ? gate_at(a.w, gt * D + col0 + c, a.gate_logits)
                                                     : gate_at(a.b, gtb, a.gate_logits);
@@ -249,7 +251,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
       if (i >= Lc) continue;
       float acc = sP[i * DVT + c];
       for (int j = 0; j <= i; ++j) acc += sA[i * CP + j] * sz[j * DVT + c];
-      og[(((size_t)bi * a.T + t0 + i) * a.Hv + h) * D + col0 + c] = from_f32<TOut>(a.scale * acc);
+      og[((tok0 + t0 + i) * a.Hv + h) * D + col0 + c] = from_f32<TOut>(a.scale * acc);
     }
     // 8. State S ← Diag(γ_C) S + K_endᵀ U.
     for (int idx = tid; idx < D * DVT; idx += kThreads) {

@@ -60,6 +60,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <climits>
 #include <type_traits>
 
 #include "common.cuh"
@@ -210,24 +211,11 @@ __device__ __forceinline__ float4 gate4(const float* g, size_t gt, int c0, bool 
   return make_float4(s, s, s, s);
 }
 
-struct Item {
-  int bh, cl, h, bi, hq, t0, Lc;
-};
-__device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int item) {
-  Item it;
-  it.bh = item % (a.B * a.Hv);      // value head fastest: heads sharing q, k run together
-  it.cl = item / (a.B * a.Hv);
-  it.h = it.bh % a.Hv;
-  it.bi = it.bh / a.Hv;
-  it.hq = it.h / (a.Hv / a.Hqk);
-  it.t0 = (c_begin + it.cl) * C;
-  it.Lc = min(C, a.T - it.t0);
-  return it;
-}
-
 // Where the slots of a launch live: chunk c_begin + j of sequence-head bh is
 // slot bh · stride + off + j of the workspace (stride: slots per
 // sequence-head in the workspace; off: the launch's first chunk there).
+// Packed sequences of different lengths: the nc chunks of sequence n, value
+// head h are slots cu_chk[n] · H_v + h · nc + j.
 struct SlotMap {
   int stride, off;
 };
@@ -235,13 +223,55 @@ __device__ __forceinline__ size_t slot_index(SlotMap m, int bh, int j) {
   return (size_t)bh * m.stride + m.off + j;
 }
 
+// A work item: chunk cl of sequence bi (bh = bi · H_v + h), tokens t0 .. t0 +
+// Lc − 1 of the q, k, v buffers (bi is 0 for packed sequences, whose t0 is
+// already in the packed stream), and its slot.
+struct Item {
+  int bh, cl, h, bi, hq, t0, Lc;
+  size_t slot;
+};
+template <bool VL>
+__device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int item, SlotMap sm) {
+  Item it;
+  if (VL) {
+    // item = global chunk · H_v + value head; the sequence is the last n with
+    // cu_chk[n] ≤ the chunk (empty sequences own no chunk and are passed over)
+    it.h = item % a.Hv;
+    const int g = item / a.Hv;
+    int lo = 0, hi = a.nseq;            // cu_chk[lo] ≤ g < cu_chk[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (a.cu_chk[mid] <= g) lo = mid; else hi = mid;
+    }
+    const int nc = a.cu_chk[lo + 1] - a.cu_chk[lo];
+    it.bi = 0;
+    it.bh = lo * a.Hv + it.h;
+    it.cl = g - a.cu_chk[lo];
+    it.hq = it.h / (a.Hv / a.Hqk);
+    it.t0 = a.cu_tok[lo] + it.cl * C;
+    it.Lc = min(C, a.cu_tok[lo + 1] - it.t0);
+    it.slot = (size_t)a.cu_chk[lo] * a.Hv + (size_t)it.h * nc + it.cl;
+  } else {
+    it.bh = item % (a.B * a.Hv);      // value head fastest: heads sharing q, k run together
+    it.cl = item / (a.B * a.Hv);
+    it.h = it.bh % a.Hv;
+    it.bi = it.bh / a.Hv;
+    it.hq = it.h / (a.Hv / a.Hqk);
+    it.t0 = (c_begin + it.cl) * C;
+    it.Lc = min(C, a.T - it.t0);
+    it.slot = slot_index(sm, it.bh, it.cl);
+  }
+  return it;
+}
+
 // Items are taken in order (chunk-major, value head fastest): by a fixed stride
 // of the grid, or, with `counter`, one at a time from that device counter
 // (zero before the launch), so that CTAs which start late take fewer.
 // F16IN: q, k, v are the load step's fp16 copies; LG: the gates are bf16
-// logits; QKG: alpha and b belong to the QK heads (one compiled copy each, so
-// that no form pays for the others' addressing at the register limit).
-template <bool F16IN, bool LG, bool QKG>
+// logits; QKG: alpha and b belong to the QK heads; VL: sequences of different
+// lengths packed along T (one compiled copy each, so that no form pays for the
+// others' addressing at the register limit).
+template <bool F16IN, bool LG, bool QKG, bool VL>
 __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
                                                            int* counter, const __grid_constant__ CUtensorMap amap,
                                                            int use_amap) {
@@ -259,7 +289,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   int* s_item = sflag + 1;               // the next item, when taken from the counter
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_items = a.B * a.Hv * n_seg;
+  const int n_items = VL ? a.cu_chk[a.nseq] * a.Hv : a.B * a.Hv * n_seg;
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(bar_a, 1);
@@ -326,13 +356,13 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   // The per-channel α tile of an item comes by one TMA copy (rows of the
   // tensor map [B·T][H_v][128]), requested by thread 0 one item ahead.
   auto fetch_alpha = [&](int item_) {
-    const Item nx = decode_item(a, c_begin, item_);
+    const Item nx = decode_item<VL>(a, c_begin, item_, sm);
     mbar_arrive_expect_tx(bar_a, C * D * (LG ? 2 : 4));
     tma_load_3d(smem + P_ALPHA, &amap, 0, QKG ? nx.hq : nx.h, nx.bi * a.T + nx.t0, bar_a);
   };
   uint32_t phase_a = 0;
   auto load_alpha_key0 = [&](int item_) {
-    const Item it = decode_item(a, c_begin, item_);
+    const Item it = decode_item<VL>(a, c_begin, item_, sm);
 #pragma unroll
     for (int u = 0; u < 4; ++u) load_key1(it, u, u);
     if (use_amap) {
@@ -364,8 +394,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   if (use_amap && tid == 0 && (counter ? *s_item : (int)blockIdx.x) < n_items)
     fetch_alpha(counter ? *s_item : (int)blockIdx.x);
   for (int item = counter ? *s_item : (int)blockIdx.x; item < n_items;) {
-    const Item it = decode_item(a, c_begin, item);
-    uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + slot_index(sm, it.bh, it.cl) * SLOT;
+    const Item it = decode_item<VL>(a, c_begin, item, sm);
+    uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + it.slot * SLOT;
     load_alpha_key0(item);
 
     // -------- pass 1: α's forward products within the quarter
@@ -837,8 +867,8 @@ template <int NE> __device__ __forceinline__ void u_sync() { asm volatile("bar.s
 template <int NE> __device__ __forceinline__ void o_sync() { asm volatile("bar.sync 3, %0;\n" ::"n"(NE / 2) : "memory"); }
 
 template <typename TOut, int DV>
-__global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
-                                                           const float* S_in, float* S_out) {
+__global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg_arg,
+                                                           SlotMap sm, const float* S_in, float* S_out) {
   using L = ScanLayout<DV>;
   constexpr int NE = L::NE;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -862,8 +892,24 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   // may take the SMs this grid leaves free
   griddep_launch_dependents();
   const int h = bh % a.Hv, bi = bh / a.Hv;
-  const uint8_t* slots = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + slot_index(sm, bh, 0) * SLOT;
+  // This CTA's chunks, their slots, and its tokens in the o buffer: the
+  // launch's segment of sequence bi, or all chunks of packed sequence bi.
+  const int n_seg = a.nseq ? a.cu_chk[bi + 1] - a.cu_chk[bi] : n_seg_arg;
+  const size_t slot0 = a.nseq ? (size_t)a.cu_chk[bi] * a.Hv + (size_t)h * n_seg : slot_index(sm, bh, 0);
+  const size_t tok0 = a.nseq ? (size_t)a.cu_tok[bi] : (size_t)bi * a.T + (size_t)c_begin * C;
+  const int trem = a.nseq ? a.cu_tok[bi + 1] - a.cu_tok[bi] : a.T - c_begin * C;
+  const uint8_t* slots = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + slot0 * SLOT;
   TOut* og = static_cast<TOut*>(a.o);
+  if (n_seg == 0) {
+    // an empty packed sequence: its final state is its initial one
+    if (S_out) {
+      for (int idx = tid; idx < D * DV; idx += L::NS) {
+        const size_t e = ((size_t)bh * D + idx / DV) * D + col0 + idx % DV;
+        S_out[e] = S_in ? S_in[e] : 0.f;
+      }
+    }
+    return;
+  }
 
   if (tid == 0) {
     for (int i = 0; i < 10; ++i) mbar_init(&bars[i], &bars[i] == b_sh ? NE / 32 : 1);   // b_sh: one per epilogue warp
@@ -1018,8 +1064,8 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
     // Outputs of chunk cc from D buffer `db`: row 64 + i of D is token i; this
     // thread writes 32 contiguous d_v values of it.
     auto out_rows = [&](int cc, uint32_t db, uint64_t* freed) {
-      const int t0o = (c_begin + cc) * C;
-      const int Lco = min(C, a.T - t0o);
+      const int t0o = cc * C;
+      const int Lco = min(C, trem - t0o);
       float v[32];
       tmem_ld16(t_lane + db + c0, v);
       tmem_ld16(t_lane + db + c0 + 16, v + 16);
@@ -1029,7 +1075,7 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
       if (tid == 64) mbar_arrive(freed);           // first thread of the output warps
       const int i = row - 64;
       if (i < Lco) {
-        TOut* dst = og + (((size_t)bi * a.T + t0o + i) * a.Hv + h) * D + dv0;
+        TOut* dst = og + ((tok0 + t0o + i) * a.Hv + h) * D + dv0;
         constexpr int VEC = 16 / (int)sizeof(TOut);
 #pragma unroll
         for (int u = 0; u < 32; u += VEC) *reinterpret_cast<uint4*>(dst + u) = pack_out<TOut>(v + u, -a.scale);
@@ -1122,13 +1168,16 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
 
 // =============================================================================
 // Load step of the tensor-core prefill when the depthwise causal convolution
-// (kernel 4, taps W[c][0..3] on tokens t−3..t, zero history) and/or the L2
-// normalisation of q, k (after the conv) are requested: q, k, v of the tokens
-// [t_begin, t_begin + Tseg) of every sequence → fp16 copies [B][Tseg][H][D]
-// that the prep kernel reads instead of the caller's tensors. One thread owns
-// 8 consecutive channels and walks the CTA's tokens with the last three inputs
-// in registers; the 16 threads of one head's 128 channels are one half-warp,
-// which reduces the sum of squares.
+// (kernel 4, taps W[c][0..3] on tokens t−3..t; before a sequence's first
+// token, its history from conv_in, or zeros) and/or the L2 normalisation of
+// q, k (after the conv) are requested: q, k, v of the tokens [t_begin, t_begin
+// + Tseg) of every sequence → fp16 copies [B][Tseg][H][D] that the prep
+// kernel reads instead of the caller's tensors. One thread owns 8 consecutive
+// channels and walks the CTA's tokens with the last three inputs in
+// registers; the 16 threads of one head's 128 channels are one half-warp,
+// which reduces the sum of squares. Packed sequences (one row of tokens):
+// at each sequence start the three inputs restart from that sequence's
+// history.
 // =============================================================================
 constexpr int QP_THREADS = 512;
 constexpr int QP_TOK = 64;            // tokens per CTA, in blocks of 8 rows loaded together
@@ -1138,7 +1187,7 @@ __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, in
   const int groups = (2 * a.Hqk + a.Hv) * (D / 8);
   const int g = blockIdx.x * QP_THREADS + threadIdx.x;
   if (g >= groups) return;            // whole half-warps: groups is a multiple of 16
-  const int bi = blockIdx.z;
+  const int bi = blockIdx.z;           // 0 for packed sequences
   const int lane = threadIdx.x & 31;
   const unsigned hmask = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
   const int ch = g * 8;               // channel in [q | k | v]
@@ -1179,11 +1228,28 @@ __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, in
   // before 0 from the caller's conv history [B, 3, channels] (zeros without).
   const size_t hrow = (size_t)(2 * a.Hqk + a.Hv) * D;
   const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.conv_in);
+  // The sequence of the CTA's first token (packed: the last n with
+  // cu_tok[n] ≤ it, which passes over empty sequences) and its first token.
+  int sq = bi, s_start = 0;
+  if (a.nseq) {
+    const int tf = t_begin + tl0;
+    int lo = 0, hi = a.nseq;            // cu_tok[lo] ≤ tf < cu_tok[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (a.cu_tok[mid] <= tf) lo = mid; else hi = mid;
+    }
+    sq = lo;
+    s_start = a.cu_tok[lo];
+  }
+  // Row j (token −3 + j of the sequence) of sequence n's history, or zeros.
+  auto hist_row = [&](int n, int j) -> uint4 {
+    if (hist == nullptr) return make_uint4(0, 0, 0, 0);
+    return __ldg(reinterpret_cast<const uint4*>(hist + ((size_t)n * 3 + j) * hrow + ch));
+  };
   auto hload = [&](int tl) -> uint4 {
     const int t = t_begin + tl;
-    if (t >= 0) return load(tl);
-    if (hist == nullptr) return make_uint4(0, 0, 0, 0);
-    return __ldg(reinterpret_cast<const uint4*>(hist + ((size_t)bi * 3 + 3 + t) * hrow + ch));
+    if (t >= s_start) return load(tl);
+    return hist_row(sq, 3 + t - s_start);
   };
   float x3[8], x2[8], x1[8];                            // inputs of t−3, t−2, t−1
   {
@@ -1194,12 +1260,22 @@ __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, in
     unpack8(h2, x2);
     unpack8(h1, x1);
   }
+  int next_start = a.nseq ? a.cu_tok[sq + 1] : INT_MAX;   // first token of the next sequence
   for (int b0 = 0; b0 < nt; b0 += 8) {
     uint4 raw[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) raw[r] = load(tl0 + b0 + r);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
+      if (conv && t_begin + tl0 + b0 + r == next_start && b0 + r < nt) {
+        // a packed sequence starts here (the same token for the whole CTA):
+        // the three previous inputs are its history
+        while (a.cu_tok[sq + 1] <= next_start) ++sq;
+        next_start = a.cu_tok[sq + 1];
+        unpack8(hist_row(sq, 0), x3);
+        unpack8(hist_row(sq, 1), x2);
+        unpack8(hist_row(sq, 2), x1);
+      }
       float x0[8], y[8];
       unpack8(raw[r], x0);
       float ss = 0.f;
@@ -1228,7 +1304,8 @@ __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, in
 
 // Bytes of the preprocessed q, k, v copies for `tokens` tokens of every sequence.
 size_t qkv_prep_bytes(const ChunkArgs& a, size_t tokens) {
-  return (size_t)a.B * tokens * (size_t)(2 * a.Hqk + a.Hv) * D * sizeof(__half);
+  const size_t rows = a.nseq ? 1 : (size_t)a.B;   // packed sequences share one row of tokens
+  return rows * tokens * (size_t)(2 * a.Hqk + a.Hv) * D * sizeof(__half);
 }
 
 size_t state_bytes(const ChunkArgs& a) { return (size_t)a.B * a.Hv * D * D * sizeof(float); }
@@ -1248,13 +1325,17 @@ size_t bytes_per_chunk(const ChunkArgs& a) {
 }
 }  // namespace
 
-// Workspace for the whole sequence in one segment.
+// Workspace for the whole sequence in one segment (packed sequences: the
+// slots of all their chunks and the load step's copies of all tokens).
 size_t chunk_tc_workspace(const ChunkArgs& a) {
+  if (a.nseq)
+    return WS_HEAD + (size_t)a.cu_chk[a.nseq] * a.Hv * SLOT + (needs_qkv_prep(a) ? qkv_prep_bytes(a, a.T) : 0);
   const size_t nchunks = (a.T + C - 1) / C;
   return WS_HEAD + nchunks * bytes_per_chunk(a);
 }
 
 size_t chunk_tc_min_workspace(const ChunkArgs& a, bool carry_state) {
+  if (a.nseq) return chunk_tc_workspace(a);   // packed sequences run in one pass
   return WS_HEAD + bytes_per_chunk(a) + (carry_state ? state_bytes(a) : 0);
 }
 
@@ -1303,7 +1384,8 @@ bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
   }();
   if (encode == nullptr) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.Hg, (cuuint64_t)a.B * (cuuint64_t)a.T};
+  const cuuint64_t rows = a.nseq ? (cuuint64_t)a.T : (cuuint64_t)a.B * (cuuint64_t)a.T;   // token rows
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.Hg, rows};
   const cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)a.Hg * D * esz};   // bytes, dims 1 and 2
   const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
   const cuuint32_t estr[3] = {1, 1, 1};
@@ -1321,38 +1403,59 @@ bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
 // tokens (conv / L2 only), carried state (only when needed). With the whole
 // sequence in the workspace and SMs left idle by the scan, the segments are
 // pipelined (see the note on overlapped segments above).
+using PrepFn = void (*)(ChunkArgs, int, int, SlotMap, int*, const CUtensorMap, int);
+template <bool VL>
+PrepFn prep_variant(bool f16in, bool lg, bool qkg) {
+  if (f16in)
+    return lg ? (qkg ? chunk_prep_kernel<true, true, true, VL> : chunk_prep_kernel<true, true, false, VL>)
+              : (qkg ? chunk_prep_kernel<true, false, true, VL> : chunk_prep_kernel<true, false, false, VL>);
+  return lg ? (qkg ? chunk_prep_kernel<false, true, true, VL> : chunk_prep_kernel<false, true, false, VL>)
+            : (qkg ? chunk_prep_kernel<false, false, true, VL> : chunk_prep_kernel<false, false, false, VL>);
+}
+
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
+  const bool vl = a.nseq > 0;
   const int BH = a.B * a.Hv;
-  const int nchunks = (a.T + C - 1) / C;
+  // chunks per sequence; for packed sequences all chunks of all of them
+  const int nchunks = vl ? a.cu_chk[a.nseq] : (a.T + C - 1) / C;
   if (a.ws_bytes < WS_HEAD) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(a.workspace, 0, WS_HEAD, s);   // status word and counters
-  if (e != cudaSuccess || BH == 0 || nchunks == 0) return e;
+  if (e != cudaSuccess || BH == 0) return e;
+  if (nchunks == 0 && !vl) return e;
   const bool pre = needs_qkv_prep(a);
-  const size_t per_chunk = bytes_per_chunk(a);
-  size_t avail = a.ws_bytes - WS_HEAD;
-  int seg = (int)std::min<size_t>(nchunks, avail / per_chunk);
   float* carry = a.ST;
   uint8_t* const ws = static_cast<uint8_t*>(a.workspace);
-  if (seg < nchunks && carry == nullptr) {
-    const size_t sb = state_bytes(a);
-    avail = avail > sb ? avail - sb : 0;
+  int seg = nchunks;
+  size_t slot_bytes = (size_t)a.Hv * nchunks * SLOT;
+  if (vl) {
+    // packed sequences run in one pass with every chunk's slot in the workspace
+    if (a.ws_bytes < chunk_tc_workspace(a)) return cudaErrorInvalidValue;
+  } else {
+    const size_t per_chunk = bytes_per_chunk(a);
+    size_t avail = a.ws_bytes - WS_HEAD;
     seg = (int)std::min<size_t>(nchunks, avail / per_chunk);
-    carry = reinterpret_cast<float*>(ws + WS_HEAD + (size_t)seg * per_chunk);
+    if (seg < nchunks && carry == nullptr) {
+      const size_t sb = state_bytes(a);
+      avail = avail > sb ? avail - sb : 0;
+      seg = (int)std::min<size_t>(nchunks, avail / per_chunk);
+      carry = reinterpret_cast<float*>(ws + WS_HEAD + (size_t)seg * per_chunk);
+    }
+    if (seg < 1) return cudaErrorInvalidValue;
+    slot_bytes = (size_t)BH * seg * SLOT;
   }
-  if (seg < 1) return cudaErrorInvalidValue;
-  __half* qkv = reinterpret_cast<__half*>(ws + WS_HEAD + (size_t)BH * seg * SLOT);
+  __half* qkv = reinterpret_cast<__half*>(ws + WS_HEAD + slot_bytes);
 
-  for (auto prep : {chunk_prep_kernel<false, false, false>, chunk_prep_kernel<true, false, false>,
-                     chunk_prep_kernel<false, true, false>, chunk_prep_kernel<true, true, false>,
-                     chunk_prep_kernel<false, false, true>, chunk_prep_kernel<true, false, true>,
-                     chunk_prep_kernel<false, true, true>, chunk_prep_kernel<true, true, true>}) {
-    if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) != cudaSuccess)
-      return e;
-    // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
-    if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
-      return e;
-  }
+  for (bool f16 : {false, true})
+    for (bool lg : {false, true})
+      for (bool qg : {false, true}) {
+        const PrepFn prep = vl ? prep_variant<true>(f16, lg, qg) : prep_variant<false>(f16, lg, qg);
+        if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) != cudaSuccess)
+          return e;
+        // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
+        if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                      cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+          return e;
+      }
   int dev = 0, sms = 148;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -1377,20 +1480,15 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   const int use_amap = a.gate_mode != GDN2_GATES_GDN && a.alpha != nullptr && encode_alpha_map(a, &amap) ? 1 : 0;
   const int qp_groups = (2 * a.Hqk + a.Hv) * (D / 8);
   const bool qkg = a.Hg != a.Hv;
-  using PrepFn = void (*)(ChunkArgs, int, int, SlotMap, int*, const CUtensorMap, int);
   auto prep_fn = [&](bool f16in) -> PrepFn {
-    if (f16in)
-      return a.gate_logits ? (qkg ? chunk_prep_kernel<true, true, true> : chunk_prep_kernel<true, true, false>)
-                           : (qkg ? chunk_prep_kernel<true, false, true> : chunk_prep_kernel<true, false, false>);
-    return a.gate_logits ? (qkg ? chunk_prep_kernel<false, true, true> : chunk_prep_kernel<false, true, false>)
-                         : (qkg ? chunk_prep_kernel<false, false, true> : chunk_prep_kernel<false, false, false>);
+    return vl ? prep_variant<true>(f16in, a.gate_logits != 0, qkg) : prep_variant<false>(f16in, a.gate_logits != 0, qkg);
   };
 
   // overlapped segments: whole sequence in the workspace, idle SMs beside the
   // scan, no load step (its kernel would wait for the scan), S_T given (the
   // state passes from segment to segment through it)
   int nseg_ov = 0;
-  if (seg == nchunks && !pre && a.ST != nullptr && scan_ctas < sms && nchunks >= 2 * OVERLAP_MIN_CHUNKS)
+  if (!vl && seg == nchunks && !pre && a.ST != nullptr && scan_ctas < sms && nchunks >= 2 * OVERLAP_MIN_CHUNKS)
     nseg_ov = std::min(std::min(OVERLAP_SEGMENTS, nchunks / OVERLAP_MIN_CHUNKS), MAX_COUNTERS);
 
   // Segment lengths. Overlapped: the last scan has no prep beside it, so the
@@ -1400,21 +1498,27 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   const int step = nseg_ov > 0 ? (nchunks - n_last + nseg_ov - 2) / (nseg_ov - 1) : seg;
   const float* s_in = a.S0;
   int k = 0;
-  for (int c0 = 0; c0 < nchunks; ++k) {
+  // (packed sequences: one pass, also when every sequence is empty, so that
+  // the scan copies their states)
+  for (int c0 = 0; c0 < nchunks || (vl && k == 0); ++k) {
     const int n = nseg_ov > 0 && k == nseg_ov - 1 ? nchunks - c0 : std::min(step, nchunks - c0);
     const bool last = c0 + n >= nchunks;
     float* s_out = last ? a.ST : carry;
     // overlapped: every chunk has its own slot; otherwise the segment's slots start at 0
     const SlotMap sm = nseg_ov > 0 ? SlotMap{nchunks, c0} : SlotMap{seg, 0};
     int* counter = nseg_ov > 0 ? reinterpret_cast<int*>(ws) + 1 + k : nullptr;
-    const int grid = std::min(BH * n, prep_ctas);
-    if (pre) {
-      const int t_begin = c0 * C;
-      const int Tseg = std::min(n * C, a.T - t_begin);
+    const int items = vl ? nchunks * a.Hv : BH * n;
+    const int grid = std::min(items, prep_ctas);
+    if (items == 0) {
+      // nothing to prepare (packed sequences, all empty)
+    } else if (pre) {
+      const int t_begin = vl ? 0 : c0 * C;
+      const int Tseg = vl ? a.T : std::min(n * C, a.T - t_begin);
+      const int rows = vl ? 1 : a.B;
       __half* qo = qkv;
-      __half* ko = qo + (size_t)a.B * Tseg * a.Hqk * D;
-      __half* vo = ko + (size_t)a.B * Tseg * a.Hqk * D;
-      const dim3 qgrid((qp_groups + QP_THREADS - 1) / QP_THREADS, (Tseg + QP_TOK - 1) / QP_TOK, a.B);
+      __half* ko = qo + (size_t)rows * Tseg * a.Hqk * D;
+      __half* vo = ko + (size_t)rows * Tseg * a.Hqk * D;
+      const dim3 qgrid((qp_groups + QP_THREADS - 1) / QP_THREADS, (Tseg + QP_TOK - 1) / QP_TOK, rows);
       qkv_prep_kernel<<<qgrid, QP_THREADS, 0, s>>>(a, t_begin, Tseg, qo, ko, vo);
       ChunkArgs ap = a;
       ap.q = qo;

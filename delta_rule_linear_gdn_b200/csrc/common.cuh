@@ -58,7 +58,22 @@ struct ChunkArgs {
   const void* conv_in;
   void* conv_out;
   int Hg;            // heads of alpha and b: Hv, or Hqk when the value heads of a QK head share them
+  // Sequences of different lengths packed along T (nseq > 0): B is then
+  // nseq (states and conv histories per sequence), tokens are addressed in
+  // the packed stream, sequence n is [cu_tok[n], cu_tok[n+1]) and owns the
+  // 64-token chunks [cu_chk[n], cu_chk[n+1]) of the tensor-core prefill.
+  int nseq;
+  int cu_tok[GDN2_MAX_SEQS + 1];
+  int cu_chk[GDN2_MAX_SEQS + 1];
 };
+
+// First token (in the q, k, v, o buffers) and length of sequence bi.
+__host__ __device__ __forceinline__ size_t seq_tok0(const ChunkArgs& a, int bi) {
+  return a.nseq ? (size_t)a.cu_tok[bi] : (size_t)bi * a.T;
+}
+__host__ __device__ __forceinline__ int seq_len(const ChunkArgs& a, int bi) {
+  return a.nseq ? a.cu_tok[bi + 1] - a.cu_tok[bi] : a.T;
+}
 
 struct DecodeArgs {
   int B, Hqk, Hv, d;

@@ -4,8 +4,9 @@
 // camadas", Conceito) reads the three inputs before each token. A prefill
 // that continues an earlier one (or is followed by decode steps) needs those
 // three inputs of the earlier call: this kernel writes them, per sequence and
-// channel of q | k | v, as rows j = 0, 1, 2 holding the input of token
-// T − 3 + j (oldest first). Rows before token 0 come from the incoming history
+// channel of q | k | v, as rows j = 0, 1, 2 holding the input of the
+// sequence's token T − 3 + j (oldest first; T its length, also for sequences
+// packed along one row). Rows before token 0 come from the incoming history
 // (or are zero without one), which makes the chain of calls equal to one call
 // over the concatenated tokens. The rows are copied bit for bit, in the input
 // dtype.
@@ -38,12 +39,14 @@ __global__ void __launch_bounds__(kCsThreads) conv_state_kernel(ChunkArgs a) {
   const TIn* hin = static_cast<const TIn*>(a.conv_in);
   TIn* hout = static_cast<TIn*>(a.conv_out);
   // Read all three rows before writing any (rows of one channel only).
+  const size_t tok0 = seq_tok0(a, bi);   // the sequence's first token in the q, k, v buffers
+  const int len = seq_len(a, bi);
   TIn r[3];
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
-    const int t = a.T - 3 + j;
+    const int t = len - 3 + j;           // token of the sequence
     if (t >= 0) {
-      r[j] = src[((size_t)bi * a.T + t) * row + cw];
+      r[j] = src[(tok0 + t) * row + cw];
     } else if (hin) {
       r[j] = hin[((size_t)bi * 3 + 3 + t) * ctot + ch];
     } else {

@@ -48,6 +48,7 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_params* p, con
                                                        const float* w, const float* S0, void* o, float* S_T,
                                                        void* stream) {
   if (!p) return GDN2_ERR_INVALID_ARG;
+  if (p->cu_seqlens) return GDN2_ERR_UNSUPPORTED;   // packed sequences need every chunk's slot at once
   // Only the tensor-core prefill uses scratch; it is the configuration this
   // call serves (every other configuration runs without scratch through
   // gdn2_chunk_fwd).

@@ -26,6 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn2.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+MAX_SEQS = 384   # GDN2_MAX_SEQS: sequences per packed (cu_seqlens) call
 F32, BF16 = 0, 1
 GATES = {"full": 0, "kda": 1, "gdn": 2}
 PRECISION = {"default": 0, "fp32": 1}
@@ -43,7 +44,7 @@ class Params(ctypes.Structure):
         ("gate_mode", ctypes.c_int), ("precision", ctypes.c_int), ("l2norm_qk", ctypes.c_int),
         ("conv_w", ctypes.c_void_p), ("gate_logits", ctypes.c_int),
         ("conv_state_in", ctypes.c_void_p), ("conv_state_out", ctypes.c_void_p),
-        ("gate_heads", ctypes.c_int),
+        ("gate_heads", ctypes.c_int), ("n_seqs", ctypes.c_int), ("cu_seqlens", ctypes.c_void_p),
     ]
 
 
@@ -112,12 +113,24 @@ def _stream_handle(stream):
 
 def make_params(B, T, H_qk, H_v, d_k, d_v, *, chunk=64, scale=1.0, qkv_dtype=BF16, o_dtype=BF16,
                 gate_mode="full", precision="default", l2norm_qk=False, conv_w=None, gate_logits=False,
-                conv_state_in=None, conv_state_out=None, gates_per_qk_head=False) -> Params:
+                conv_state_in=None, conv_state_out=None, gates_per_qk_head=False, cu_seqlens=None) -> Params:
+    """``cu_seqlens``: None, or a ctypes c_int array of N + 1 token offsets
+    (see :func:`cu_seqlens_array`), which must stay alive while the Params are
+    used."""
     return Params(int(B), int(T), int(H_qk), int(H_v), int(d_k), int(d_v), int(chunk), float(scale),
                   int(qkv_dtype), int(o_dtype), GATES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode),
                   PRECISION[precision] if isinstance(precision, str) else int(precision),
                   1 if l2norm_qk else 0, _ptr(conv_w), 1 if gate_logits else 0,
-                  _ptr(conv_state_in), _ptr(conv_state_out), 1 if gates_per_qk_head else 0)
+                  _ptr(conv_state_in), _ptr(conv_state_out), 1 if gates_per_qk_head else 0,
+                  0 if cu_seqlens is None else len(cu_seqlens) - 1,
+                  None if cu_seqlens is None else ctypes.cast(cu_seqlens, ctypes.c_void_p).value)
+
+
+def cu_seqlens_array(cu_seqlens):
+    """Host int32 offsets (list, tuple, numpy or CPU tensor) as the ctypes array
+    the C call reads."""
+    vals = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    return (ctypes.c_int * len(vals))(*vals)
 
 
 def conv_state_shape(B, H_qk, H_v, d_k, d_v):
@@ -126,9 +139,11 @@ def conv_state_shape(B, H_qk, H_v, d_k, d_v):
 
 
 def _check_shapes(lead, H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates_per_qk_head, states=(),
-                  conv_w=None):
+                  conv_w=None, n_states=None):
     """Shapes of everything the call reads or writes, so that no kernel indexes
-    past a tensor: ``lead`` is (B, T) or (B,); ``states`` are [B,H_v,d_k,d_v]."""
+    past a tensor: ``lead`` is (B, T) or (B,); ``states`` are
+    [n_states (default B),H_v,d_k,d_v]."""
+    ns = lead[0] if n_states is None else n_states
     mode = GATES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode)
     Hg = H_qk if gates_per_qk_head else H_v
     want = {"k": lead + (H_qk, d_k), "v": lead + (H_v, d_v)}
@@ -144,8 +159,8 @@ def _check_shapes(lead, H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates
         if t is not None and tuple(t.shape) != shape:
             raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
     for name, t in states:
-        if t is not None and tuple(t.shape) != (lead[0], H_v, d_k, d_v):
-            raise ValueError(f"{name} must have shape {(lead[0], H_v, d_k, d_v)}, got {tuple(t.shape)}")
+        if t is not None and tuple(t.shape) != (ns, H_v, d_k, d_v):
+            raise ValueError(f"{name} must have shape {(ns, H_v, d_k, d_v)}, got {tuple(t.shape)}")
     if conv_w is not None and tuple(conv_w.shape) != (2 * H_qk * d_k + H_v * d_v, 4):
         raise ValueError(f"conv_w must have shape {(2 * H_qk * d_k + H_v * d_v, 4)}, got {tuple(conv_w.shape)}")
 
@@ -176,7 +191,7 @@ def chunk_fwd_workspace(params: Params) -> int:
 def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_mode="full",
               precision="default", l2norm_qk=False, conv_w=None, o_dtype=None, o=None, S_T=None,
               workspace=None, stream=None, want_state=True, gate_logits=False, conv_state_in=None,
-              conv_state_out=None, gates_per_qk_head=False):
+              conv_state_out=None, gates_per_qk_head=False, cu_seqlens=None):
     """Chunked prefill. q,k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; gates per
     ``gate_mode``: fp32 values, or bf16 logits with ``gate_logits`` (the kernels
     apply the sigmoid); S0 [B,H_v,d_k,d_v] fp32 or None. With ``conv_w``, the
@@ -184,9 +199,13 @@ def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_m
     the history after the last token is written to ``conv_state_out`` (both
     :func:`conv_state_shape`, q's dtype, distinct buffers). With
     ``gates_per_qk_head`` alpha and b have H_qk heads, shared by the value
-    heads of each QK head. Returns (o, S_T)."""
+    heads of each QK head. With ``cu_seqlens`` (host offsets, N + 1 of them)
+    the tensors hold N sequences of different lengths packed along T (B = 1),
+    and S0, S_T and the conv histories have N rows. Returns (o, S_T)."""
     B, T, H_qk, d_k = q.shape
     H_v, d_v = v.shape[2], v.shape[3]
+    cu = None if cu_seqlens is None else cu_seqlens_array(cu_seqlens)
+    NS = B if cu is None else len(cu) - 1    # sequences that own a state
     o_dtype = q.dtype if o_dtype is None else o_dtype
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check(t, name, q.dtype)
@@ -196,24 +215,24 @@ def chunk_fwd(q, k, v, alpha, b, w=None, S0=None, *, chunk=64, scale=1.0, gate_m
     for name, t in (("S0", S0), ("conv_w", conv_w)):
         _check(t, name, torch.float32)
     _check_shapes((B, T), H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates_per_qk_head,
-                  states=(("S0", S0), ("S_T", S_T)), conv_w=conv_w)
-    hshape = conv_state_shape(B, H_qk, H_v, d_k, d_v)
+                  states=(("S0", S0), ("S_T", S_T)), conv_w=conv_w, n_states=NS)
+    hshape = conv_state_shape(NS, H_qk, H_v, d_k, d_v)
     _check_conv_state(conv_state_in, "conv_state_in", q.dtype, hshape)
     _check_conv_state(conv_state_out, "conv_state_out", q.dtype, hshape)
     p = make_params(B, T, H_qk, H_v, d_k, d_v, chunk=chunk, scale=scale, qkv_dtype=_dtype_code(q.dtype),
                     o_dtype=_dtype_code(o_dtype), gate_mode=gate_mode, precision=precision,
                     l2norm_qk=l2norm_qk, conv_w=conv_w, gate_logits=gate_logits,
                     conv_state_in=conv_state_in, conv_state_out=conv_state_out,
-                    gates_per_qk_head=gates_per_qk_head)
+                    gates_per_qk_head=gates_per_qk_head, cu_seqlens=cu)
     if o is None:
         o = torch.empty((B, T, H_v, d_v), dtype=o_dtype, device=q.device)
     if S_T is None and want_state:
-        S_T = torch.empty((B, H_v, d_k, d_v), dtype=torch.float32, device=q.device)
+        S_T = torch.empty((NS, H_v, d_k, d_v), dtype=torch.float32, device=q.device)
     _check(o, "o", o_dtype)
     if tuple(o.shape) != (B, T, H_v, d_v):
         raise ValueError(f"o must have shape {(B, T, H_v, d_v)}, got {tuple(o.shape)}")
     _check(S_T, "S_T", torch.float32)
-    need = chunk_fwd_workspace(p)
+    need = chunk_fwd_workspace(p)   # (reads the offsets too)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

@@ -133,7 +133,23 @@ typedef struct {
                      conv_state_in or any other argument (swap two buffers
                      between calls). Needs conv_w.                            */
   int gate_heads;  /* gdn2_gate_heads of alpha and b (0: per value head)       */
+  int n_seqs;      /* gdn2_chunk_fwd with cu_seqlens: number of sequences N   */
+  const int* cu_seqlens; /* NULL (B sequences of T tokens each), or a HOST
+                     array of n_seqs + 1 token offsets for sequences of
+                     different lengths packed along T: sequence n is tokens
+                     [cu_seqlens[n], cu_seqlens[n+1]) of q, k, v, gates and o,
+                     with cu_seqlens[0] = 0, non-decreasing (empty sequences
+                     allowed), cu_seqlens[n_seqs] = T. Then B must be 1, the
+                     states S0, S_T and the conv histories have n_seqs rows in
+                     place of B, every sequence starts its own chunks, state
+                     and conv history, and 1 <= n_seqs <= GDN2_MAX_SEQS. Read
+                     during the call only; gdn2_chunk_fwd_workspace needs it
+                     too. gdn2_chunk_fwd only (not decode, not noalloc).      */
 } gdn2_params;
+
+/* Most sequences one varlen gdn2_chunk_fwd call takes (their offsets travel
+ * with the launches). */
+#define GDN2_MAX_SEQS 384
 
 /* Human-readable name of a status code (static string, never NULL). */
 GDN2_API const char* gdn2_status_str(gdn2_status s);

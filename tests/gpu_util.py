@@ -83,3 +83,34 @@ def assert_close(got, ref, tol, what):
     err = oracle.rel_err(np64(got) if torch.is_tensor(got) else got, ref)
     assert np.isfinite(err) and err <= tol, f"{what}: max|err|/RMS(ref) = {err:.3e} > {tol:.1e}"
     return err
+
+
+def split_packed(inp, cu, n):
+    """Sequence n of a packed input dict ([1, T, ...] tensors, offsets cu) as
+    its own one-sequence input dict (S0 row n). Fresh copies: a slice of a
+    per-token scalar gate can start off the 16-byte alignment the C calls ask
+    for."""
+    t0, t1 = int(cu[n]), int(cu[n + 1])
+    out = {}
+    for key, t in inp.items():
+        if t is None or key == "conv_w":
+            out[key] = t
+        elif key == "S0":
+            out[key] = t[n:n + 1].clone()
+        else:
+            out[key] = t[:, t0:t1].clone()
+    return out
+
+
+def oracle_packed(inp, cu, conv_state=None, **kw):
+    """Oracle (o [1,T,H_v,d_v], S_T [N,H_v,d_k,d_v]) of packed sequences: each
+    sequence on its own, from its own state and conv history."""
+    N = len(cu) - 1
+    os_, Ss = [], []
+    for n in range(N):
+        part = split_packed(inp, cu, n)
+        hist = None if conv_state is None else conv_state[n:n + 1]
+        o, S = oracle_chunk(part, conv_state=hist, **kw)
+        os_.append(o)
+        Ss.append(S)
+    return np.concatenate(os_, axis=1), np.concatenate(Ss, axis=0)

@@ -139,6 +139,44 @@ def test_conv_state_validation(L):
     assert _call_decode(L, _params(conv_w=conv_w, conv_state_in=hin), S=hin - 256) == gdn2.ERR_INVALID_ARG
 
 
+def test_varlen_validation_and_workspace(L):
+    """Packed sequences (cu_seqlens, host offsets): every malformed table is
+    refused before any launch; the workspace of the tensor-core path holds a
+    slot per chunk of every sequence."""
+    def vp(cu, **kw):
+        arr = gdn2.cu_seqlens_array(cu)
+        base = dict(B=1, T=int(cu[-1]), H_qk=1, H_v=2, d_k=16, d_v=16, chunk=16, qkv_dtype=gdn2.F32,
+                    o_dtype=gdn2.F32, cu_seqlens=arr)
+        base.update(kw)
+        return gdn2.make_params(**base), arr
+    for cu, kw in (([1, 5], {}), ([0, 5, 3, 9], {}), ([0, 4, 9], dict(T=10)), ([0, 4, 9], dict(B=2))):
+        p, keep = vp(cu, **kw)
+        assert _call_chunk(L, p) == gdn2.ERR_INVALID_ARG, (cu, kw)
+    p, keep = vp(list(range(gdn2.MAX_SEQS + 2)))            # one sequence too many
+    assert _call_chunk(L, p) == gdn2.ERR_INVALID_ARG
+    p = _params()
+    p.n_seqs = 2                                            # a count without offsets
+    assert _call_chunk(L, p) == gdn2.ERR_INVALID_ARG
+    p, keep = vp([0, 3, 7])
+    assert _call_decode(L, p) == gdn2.ERR_INVALID_ARG       # decode has no packed form
+    fn = L.gdn2_chunk_fwd_noalloc
+    fn.argtypes = [ctypes.POINTER(gdn2.Params)] + [ctypes.c_void_p] * 10
+    fn.restype = ctypes.c_int
+    assert fn(ctypes.byref(p), *[FAKE * (i + 1) for i in range(9)], None) == gdn2.ERR_UNSUPPORTED
+    # S0 sized for B = 1 rather than for the 3 sequences overlaps o placed right after it
+    p, keep = vp([0, 3, 7, 7], H_v=1)
+    s0_one = 16 * 16 * 4
+    assert _call_chunk(L, p, S0=FAKE * 7, o=FAKE * 7 + s0_one) == gdn2.ERR_INVALID_ARG
+    # tensor-core workspace: 256-byte header + one 74,752-byte slot per (chunk, value head)
+    cu = [0, 130, 130, 131, 331]                            # chunks of 64: 3, 0, 1, 4
+    arr = gdn2.cu_seqlens_array(cu)
+    p = gdn2.make_params(1, 331, 2, 6, 128, 128, chunk=64, cu_seqlens=arr)
+    assert gdn2.chunk_fwd_workspace(p) == 256 + 8 * 6 * 74752
+    # with the conv / L2 load step: plus fp16 copies of all 331 tokens' q | k | v
+    p = gdn2.make_params(1, 331, 2, 6, 128, 128, chunk=64, cu_seqlens=arr, l2norm_qk=True)
+    assert gdn2.chunk_fwd_workspace(p) == 256 + 8 * 6 * 74752 + 331 * (2 * 2 + 6) * 128 * 2
+
+
 def _header_param_fields():
     text = open(HEADER).read()
     body = text[text.index("typedef struct {"):text.index("} gdn2_params;")]
@@ -149,7 +187,8 @@ def _header_param_fields():
 def test_params_mirror_matches_header_field_order():
     names = [f[0] for f in gdn2.Params._fields_]
     assert names == _header_param_fields()
-    assert names[-5:] == ["conv_w", "gate_logits", "conv_state_in", "conv_state_out", "gate_heads"]
+    assert names[-7:] == ["conv_w", "gate_logits", "conv_state_in", "conv_state_out", "gate_heads", "n_seqs",
+                          "cu_seqlens"]
     assert gdn2.make_params(1, 1, 1, 1, 16, 16, gate_logits=True).gate_logits == 1
     assert gdn2.conv_state_shape(2, 16, 48, 128, 128) == (2, 3, 10240)
 
