@@ -1182,6 +1182,7 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
 constexpr int QP_THREADS = 512;
 constexpr int QP_TOK = 64;            // tokens per CTA, in blocks of 8 rows loaded together
 
+template <bool VL>
 __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, int t_begin, int Tseg, __half* qo,
                                                                  __half* ko, __half* vo) {
   const int groups = (2 * a.Hqk + a.Hv) * (D / 8);
@@ -1231,7 +1232,7 @@ __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, in
   // The sequence of the CTA's first token (packed: the last n with
   // cu_tok[n] ≤ it, which passes over empty sequences) and its first token.
   int sq = bi, s_start = 0;
-  if (a.nseq) {
+  if (VL) {
     const int tf = t_begin + tl0;
     int lo = 0, hi = a.nseq;            // cu_tok[lo] ≤ tf < cu_tok[hi]
     while (hi - lo > 1) {
@@ -1260,14 +1261,14 @@ __global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, in
     unpack8(h2, x2);
     unpack8(h1, x1);
   }
-  int next_start = a.nseq ? a.cu_tok[sq + 1] : INT_MAX;   // first token of the next sequence
+  int next_start = VL ? a.cu_tok[sq + 1] : INT_MAX;   // first token of the next sequence
   for (int b0 = 0; b0 < nt; b0 += 8) {
     uint4 raw[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) raw[r] = load(tl0 + b0 + r);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      if (conv && t_begin + tl0 + b0 + r == next_start && b0 + r < nt) {
+      if (VL && conv && t_begin + tl0 + b0 + r == next_start && b0 + r < nt) {
         // a packed sequence starts here (the same token for the whole CTA):
         // the three previous inputs are its history
         while (a.cu_tok[sq + 1] <= next_start) ++sq;
@@ -1519,7 +1520,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       __half* ko = qo + (size_t)rows * Tseg * a.Hqk * D;
       __half* vo = ko + (size_t)rows * Tseg * a.Hqk * D;
       const dim3 qgrid((qp_groups + QP_THREADS - 1) / QP_THREADS, (Tseg + QP_TOK - 1) / QP_TOK, rows);
-      qkv_prep_kernel<<<qgrid, QP_THREADS, 0, s>>>(a, t_begin, Tseg, qo, ko, vo);
+      (vl ? qkv_prep_kernel<true> : qkv_prep_kernel<false>)<<<qgrid, QP_THREADS, 0, s>>>(a, t_begin, Tseg, qo, ko, vo);
       ChunkArgs ap = a;
       ap.q = qo;
       ap.k = ko;
