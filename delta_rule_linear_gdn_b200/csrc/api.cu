@@ -206,7 +206,7 @@ const char* gdn2_status_str(gdn2_status s) {
   return "GDN2: unknown status";
 }
 
-int gdn2_version(void) { return 100; }
+int gdn2_version(void) { return 200; }   // 0.2.0: gdn2_params grew the gate, conv-history and packed-sequence fields
 
 size_t gdn2_chunk_fwd_workspace(const gdn2_params* p) {
   if (check_common(p, false) != GDN2_OK) return 0;

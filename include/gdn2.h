@@ -154,7 +154,9 @@ typedef struct {
 /* Human-readable name of a status code (static string, never NULL). */
 GDN2_API const char* gdn2_status_str(gdn2_status s);
 
-/* Library version as 10000*major + 100*minor + patch. */
+/* Library version as 10000*major + 100*minor + patch. 200 (0.2.0) takes the
+ * gdn2_params layout of this header, which extends 0.1.0's at the end; a
+ * caller built against an older header passes a struct too short for it. */
 GDN2_API int gdn2_version(void);
 
 /* Bytes of device workspace gdn2_chunk_fwd needs for `p` (0 if none). Returns
