@@ -108,3 +108,20 @@ def test_binding_rejects_gates_of_the_wrong_heads():
     cq = to_cuda(make_inputs(w, seed=63, gates_per_qk_head=True))
     with pytest.raises(ValueError):
         run(cq, chunk=16)
+
+
+def test_noalloc_with_qk_gates():
+    """The allocation-free call with gates per QK head: 79 chunks of 6
+    sequence-heads do not fit its 32 MiB scratch (74 do), so it runs in plain
+    segments; same results as the workspace call, bit for bit."""
+    w = replace(workload("prefill_t4096"), T=5000, H_qk=2, H_v=6, s0="normal")
+    inp = make_inputs(w, seed=64, gates_per_qk_head=True)
+    c = to_cuda(inp)
+    o, S = run(c, chunk=64, gates_per_qk_head=True)
+    o2 = torch.empty_like(o)
+    S2 = torch.empty_like(S)
+    gdn2.chunk_fwd_noalloc(c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], c["S0"], o=o2, S_T=S2,
+                           chunk=64, gates_per_qk_head=True)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(o2, o, rtol=0, atol=0)
+    torch.testing.assert_close(S2, S, rtol=0, atol=0)

@@ -154,3 +154,26 @@ def test_binding_shapes_for_packed_sequences():
         run(dict(c, S0=c["S0"][:1].contiguous()), cu, chunk=16)
     with pytest.raises(gdn2.GDN2Error):  # offsets that do not end at T
         run(c, [0, 5, 11], chunk=16)
+
+
+def test_packed_without_states_and_fp32_arithmetic_on_bf16():
+    """No initial states (zeros) and no final states requested, on the
+    tensor-core path; and GDN2_PREC_FP32 on bf16 inputs (the fp32 path reads
+    bf16 q, k, v) against the 1e-4 bar."""
+    lens = [90, 3, 0, 70]
+    w, cu, inp, tol = packed_inputs("tensor_core", lens, seed=78)
+    inp["S0"] = None
+    c = to_cuda(inp)
+    o, S = gdn2.chunk_fwd(c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], None, chunk=64,
+                          o_dtype=torch.float32, cu_seqlens=cu, want_state=False)
+    torch.cuda.synchronize()
+    assert S is None
+    o_ref, _ = oracle_packed(inp, cu)
+    assert_close(o, o_ref, TOL_BF16, "o without states")
+    o32, S32 = gdn2.chunk_fwd(c["q"], c["k"], c["v"], c["alpha"], c["b"], c["w"], None, chunk=64,
+                              o_dtype=torch.float32, cu_seqlens=cu, precision="fp32")
+    torch.cuda.synchronize()
+    o_ref2, S_ref2 = oracle_packed(inp, cu)
+    assert_close(o32, o_ref2, TOL_FP32, "o fp32 path")
+    assert_close(S32, S_ref2, TOL_FP32, "S_T fp32 path")
+    assert torch.count_nonzero(S32[2]) == 0                      # the empty sequence: zero state
