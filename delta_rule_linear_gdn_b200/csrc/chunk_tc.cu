@@ -33,6 +33,12 @@
 //         S ← Γ S + K_endᵀ U,       D_rows 64..127 += (−Aqk) U  (= −O / scale),
 //     with the fp32 state resident in TMEM and an fp16 copy in shared memory
 //     feeding the next chunk's products.
+// Forms selected by the call's parameters: gates as bf16 logits (σ applied
+// where they are read), α and b owned by the QK heads, the conv's history
+// from and to the caller (load step), and sequences of different lengths
+// packed along T (items and scan CTAs find their sequence's chunks and
+// tokens in offset tables passed with the launch). The prep has one compiled
+// copy per combination, so that no form pays for another's addressing.
 // All MMA operand tiles use the 128-byte-swizzled layout (see tc_prims.cuh),
 // so that a warp writing or reading whole rows is free of bank conflicts.
 //
