@@ -53,9 +53,9 @@ L2_BYTES = 126 * 2**20
 # kernel sources it was taken on; with other sources the figure is stale and
 # the bench reports null.
 TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
-TRAFFIC = {"sha1": "5d5a2334bb192c8982c08411810d029368ca55d8",
+TRAFFIC = {"sha1": "c303dc6434ed4a50c5ec5cd8cd600ff47ced5b3c",
            # reads 4.931 GB + writes 2.004 GB over the 8 launches of one call
-           "bytes_per_call": 6_934_754_816,
+           "bytes_per_call": 6_934_368_512,
            "profile": "profiles/prefill_t32768_dram_traffic.md"}
 
 
