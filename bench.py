@@ -5,13 +5,14 @@ over T=32768 tokens of one sequence (bf16 q,k,v, fp32 per-channel gates,
 chunk 64), inputs resident in HBM. The decode workload (B=256 sequences, one
 token per step, fp32 states [256,48,128,128]) is timed in the same run and
 reported under "decode"; so are the conv + L2 prefill (B=8, T=8192,
-"conv_prefill") and the headline prefill with other gate layouts (bf16
-logits, "prefill_gate_logits"; alpha and b per QK head, "prefill_qk_gates").
+"conv_prefill"), the headline prefill with other gate layouts (bf16
+logits, "prefill_gate_logits"; alpha and b per QK head, "prefill_qk_gates")
+and decode with the conv in the step ("decode_conv").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill_t32768|prefill_t4096] [--decode-workload decode_b256|decode_b64]
                     [--decode-steps N] [--conv-steps N] [--e2e-steps N] [--logits-steps N]
-                    [--qk-gates-steps N]
+                    [--qk-gates-steps N] [--decode-conv-steps N]
 
 (--workload prefill_t4096 / --decode-workload decode_b64 are the small cases
 the ncu captures run; a count of 0 skips that part.)
@@ -353,6 +354,8 @@ def main():
                     help="timed calls of the T=32768 prefill with bf16 gate logits; 0 skips it")
     ap.add_argument("--qk-gates-steps", type=int, default=20,
                     help="timed calls of the T=32768 prefill with alpha, b per QK head; 0 skips it")
+    ap.add_argument("--decode-conv-steps", type=int, default=200,
+                    help="timed decode steps with the conv and L2 norm in the step; 0 skips it")
     ap.add_argument("--conv-steps", type=int, default=5,
                     help="timed calls of the conv + L2 workload (B=8, T=8192); 0 skips it")
     args = ap.parse_args()
@@ -434,6 +437,9 @@ def main():
     dw = workload(args.decode_workload) if args.decode_steps > 0 else None
     if dw is not None:
         decode = run_decode(args, dw, dev, stream, barrier, pk, world)
+    decode_conv = None
+    if args.decode_conv_steps > 0:
+        decode_conv = run_decode(args, workload(args.decode_workload), dev, stream, barrier, pk, world, conv=True)
 
     # ---------------------------------------------------------------- conv + L2 load step
     conv = None
@@ -476,46 +482,68 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
             "conv_prefill": conv, "prefill_gate_logits": logits, "prefill_qk_gates": qk_gates,
+            "decode_conv": decode_conv,
         }
         print(json.dumps(line), flush=True)
     return 0
 
 
-def run_decode(args, dw, dev, stream, barrier, pk, world):
+def run_decode(args, dw, dev, stream, barrier, pk, world, conv=False):
+    """Consecutive decode steps of B sequences; with ``conv``, each step also
+    convolves q, k, v with the three previous inputs (history ping-ponged
+    between two buffers) and L2-normalises q, k."""
     import torch
     from delta_rule_linear_gdn_b200 import gdn2
-    from delta_rule_linear_gdn_b200.inputs import make_decode_pool
+    from delta_rule_linear_gdn_b200.inputs import CONV_STD, make_conv_state, make_decode_pool
     pool = make_decode_pool(dw, pool=16, device=dev)
     S = pool["S0"].clone()
     od = torch.empty((dw.B, dw.H_v, dw.d), dtype=torch.bfloat16, device=dev)
+    steps = args.decode_conv_steps if conv else args.decode_steps
+    kw = {}
+    hist = []
+    if conv:
+        nch = (2 * dw.H_qk + dw.H_v) * dw.d
+        g = torch.Generator(device=dev)
+        g.manual_seed(11)
+        kw = dict(conv_w=torch.randn((nch, 4), generator=g, device=dev) * CONV_STD, l2norm_qk=True)
+        hist = [make_conv_state(dw, seed=12, device=dev), torch.empty((dw.B, 3, nch), dtype=torch.bfloat16,
+                                                                       device=dev)]
 
     def decode_call(i):
-        gdn2.decode_step(pool["q"][i], pool["k"][i], pool["v"][i], pool["alpha"][i], pool["b"][i], pool["w"][i],
-                         S, o=od, stream=stream)
+        if conv:
+            kw["conv_state_in"], kw["conv_state_out"] = hist[i % 2], hist[(i + 1) % 2]
+        j = i % 16
+        gdn2.decode_step(pool["q"][j], pool["k"][j], pool["v"][j], pool["alpha"][j], pool["b"][j], pool["w"][j],
+                         S, o=od, stream=stream, **kw)
 
     with torch.cuda.stream(stream):
-        for i in range(5):
-            decode_call(i % 16)
+        for i in range(6):
+            decode_call(i)
     torch.cuda.synchronize()
     barrier()
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     d0.record(stream)
     with torch.cuda.stream(stream):
-        for i in range(args.decode_steps):
-            decode_call(i % 16)
+        for i in range(steps):
+            decode_call(i)
     d1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    dms = max_over_ranks(d0.elapsed_time(d1) / args.decode_steps, dev)
+    dms = max_over_ranks(d0.elapsed_time(d1) / steps, dev)
     dbytes = decode_bytes(dw)
+    what = ""
+    if conv:
+        nch = (2 * dw.H_qk + dw.H_v) * dw.d
+        dbytes += 2 * dw.B * 3 * nch * 2 + nch * 16      # history in and out (bf16), conv taps
+        what = ", depthwise causal conv k=4 (history ping-ponged) and L2 norm of q, k in the step"
     decode = {"workload": f"{dw.name}: B={dw.B} sequences, one token per step, H_qk={dw.H_qk} H_v={dw.H_v} "
-                          f"d={dw.d}, fp32 state, bf16 q,k,v,o, {args.decode_steps} consecutive steps",
+                          f"d={dw.d}, fp32 state, bf16 q,k,v,o, {steps} consecutive steps{what}",
               "us_per_step": dms * 1e3, "gbs": dbytes / (dms * 1e-3) / 1e9 * world,
               "roofline": {"bound": "hbm", "achieved": dbytes / (dms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                            "unit": "GB/s", "frac": dbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"],
                            "traffic": None, "alg_bytes_per_launch": dbytes},
               "tokens_per_s": dw.B * world / (dms * 1e-3)}
-    decode["gpu_launches"] = args.decode_steps
+    decode["gpu_launches"] = steps
     return decode
 
 
