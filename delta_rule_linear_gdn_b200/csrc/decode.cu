@@ -34,7 +34,7 @@ namespace {
 constexpr int kRowGroups = 16;
 
 template <int D, int COLS, typename TIn, typename TOut, bool LG, bool CONV>
-__global__ void __launch_bounds__((COLS / 4) * kRowGroups)
+__global__ void __launch_bounds__((COLS / 4) * kRowGroups, 4)
 decode_kernel(DecodeArgs a) {
   constexpr int CG = COLS / 4;            // column groups (float4 each)
   constexpr int NT = CG * kRowGroups;     // threads
@@ -86,10 +86,22 @@ decode_kernel(DecodeArgs a) {
     }
     return y;
   };
-  for (int i = tid; i < D; i += NT) {
-    s_q[i] = conv1(qg[i], cq + i);
-    s_k[i] = conv1(kg[i], ck + i);
-    s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
+  if (CONV) {
+    // q and k channels spread over all threads (warp-uniform halves): each
+    // thread waits for one channel's taps and history, not two
+    for (int i = tid; i < 2 * D; i += NT) {
+      const bool isq = i < D;
+      const int c = isq ? i : i - D;
+      (isq ? s_q : s_k)[c] = conv1(isq ? qg[c] : kg[c], (isq ? cq : ck) + c);
+    }
+    for (int i = tid; i < D; i += NT)
+      s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
+  } else {
+    for (int i = tid; i < D; i += NT) {
+      s_q[i] = conv1(qg[i], cq + i);
+      s_k[i] = conv1(kg[i], ck + i);
+      s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
+    }
   }
   const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at<LG>(a.b, bg);
   for (int j = tid; j < COLS; j += NT) {
