@@ -56,8 +56,7 @@ L2_BYTES = 126 * 2**20
 TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
 TRAFFIC = {"sha1": "c303dc6434ed4a50c5ec5cd8cd600ff47ced5b3c",
            # reads 4.931 GB + writes 2.004 GB over the 8 launches of one call
-           "bytes_per_call": 6_934_368_512,
-           "profile": "profiles/prefill_t32768_dram_traffic.md"}
+           "bytes_per_call": 6_934_368_512}
 
 
 def peaks():

@@ -28,7 +28,7 @@
  *  - Every pointer must be 16-byte aligned.
  *  - Arguments are validated on the host before any launch. A rejected call
  *    enqueues nothing and returns GDN2_ERR_INVALID_ARG (bad pointer, shape,
- *    alignment) or GDN2_ERR_UNSUPPORTED (a valid request this build has no
+ *    alignment) or GDN2_ERR_UNSUPPORTED (a valid request this library has no
  *    kernel for). A launch failure returns GDN2_ERR_CUDA. Nothing is thrown
  *    across the ABI.
  *  - Preconditions NOT checked on the device: gates finite with α ∈ (0,1]
@@ -96,7 +96,7 @@ typedef struct {
   int H_qk;       /* query/key heads                                          */
   int H_v;        /* value heads; H_v % H_qk == 0                             */
   int d_k;        /* key head dim: 16, 32, 64 or 128                          */
-  int d_v;        /* value head dim: equal to d_k in this build               */
+  int d_v;        /* value head dim: equal to d_k in this version             */
   int chunk;      /* chunk length C for gdn2_chunk_fwd: 16, 32 or 64          */
   float scale;    /* readout scale s                                          */
   int qkv_dtype;  /* gdn2_dtype of q, k, v                                    */
