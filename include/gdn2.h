@@ -133,7 +133,7 @@ typedef struct {
                      conv_state_in or any other argument (swap two buffers
                      between calls). Needs conv_w.                            */
   int gate_heads;  /* gdn2_gate_heads of alpha and b (0: per value head)       */
-  int n_seqs;      /* gdn2_chunk_fwd with cu_seqlens: number of sequences N   */
+  int n_seqs;      /* with cu_seqlens: number of sequences N; else 0          */
   const int* cu_seqlens; /* NULL (B sequences of T tokens each), or a HOST
                      array of n_seqs + 1 token offsets for sequences of
                      different lengths packed along T: sequence n is tokens
