@@ -456,6 +456,52 @@ def test_gates_for_value_heads_mapping_and_group_symmetry():
     assert np.abs(o[:, :, 3] - o[:, :, 0]).max() > 1e-3
 
 
+@pytest.mark.parametrize("C", [4, 16])
+def test_chunk_algebra_equals_token_loop(C):
+    """The chunked form the prefill kernels compute ("Chunkwise KDA" of the
+    hada.io page, with the decoupled gates of the GDN-2 summary, Metodologia
+    §3), written out in float64 from its equations, equals the token loop to
+    rounding: per chunk with entry state S and γ_i = Π_{s≤i} α_s,
+        T_ij = Σ_c e_ic k_jc γ_ic/γ_jc (j < i),  Aqk_ij = Σ_c q_ic k_jc γ_ic/γ_jc (j ≤ i),
+        Y = (I+T)⁻¹ Ē,  U_w = (I+T)⁻¹ Z,  U = U_w − Y S,
+        O = Q̄ S + Aqk U,  S ← Diag(γ_C) S + K_endᵀ U,
+    and the state update is the affine map S ← (Diag(γ_C) − K_endᵀ Y) S + K_endᵀ U_w."""
+    r = _rng(40 + C)
+    T, dk, dv = 3 * C + 1, 5, 3                      # a ragged last chunk
+    q = _unit(r.standard_normal((T, dk)))
+    k = _unit(r.standard_normal((T, dk)))
+    v = r.standard_normal((T, dv))
+    a = _sig(r.standard_normal((T, dk)) + 2.0)
+    b = _sig(r.standard_normal((T, dk)))
+    w = _sig(r.standard_normal((T, dv)))
+    S0 = 0.1 * r.standard_normal((dk, dv))
+    o_ref, S_ref = oracle.gdn2_forward(q[None, :, None], k[None, :, None], v[None, :, None], a[None, :, None],
+                                       b[None, :, None], w[None, :, None], S0[None, None])
+    S = S0.copy()
+    out = []
+    for t0 in range(0, T, C):
+        sl = slice(t0, min(T, t0 + C))
+        qc, kc, vc, ac, bc, wc = q[sl], k[sl], v[sl], a[sl], b[sl], w[sl]
+        L = qc.shape[0]
+        g = np.cumprod(ac, axis=0)                   # γ_i per key channel
+        e, z = bc * kc, wc * vc
+        Eb, Qb = e * g, qc * g                       # Ē, Q̄
+        Kt = kc / g                                  # K̃ (γ_i/γ_j = Ē_i·K̃_j)
+        Tm = np.tril(Eb @ Kt.T, -1)
+        Aqk = np.tril(Qb @ Kt.T)
+        Ainv = np.linalg.inv(np.eye(L) + Tm)
+        Y, Uw = Ainv @ Eb, Ainv @ z
+        U = Uw - Y @ S
+        out.append(Qb @ S + Aqk @ U)
+        Kend = kc * (g[-1] / g)                      # k_j ⊙ Π_{j<s≤L} α_s
+        S_aff = (np.diag(g[-1]) - Kend.T @ Y) @ S + Kend.T @ Uw
+        S = g[-1][:, None] * S + Kend.T @ U
+        np.testing.assert_allclose(S_aff, S, rtol=0, atol=1e-12)
+    o = np.concatenate(out)
+    np.testing.assert_allclose(o, o_ref[0, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S, S_ref[0, 0], rtol=0, atol=1e-12)
+
+
 def test_rel_err_metric():
     ref = np.array([3.0, -4.0])
     assert oracle.rel_err(ref, ref) == 0.0
