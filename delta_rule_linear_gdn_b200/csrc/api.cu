@@ -1,6 +1,7 @@
 // C ABI entry points: argument validation on the host, then one launch on the
 // caller's stream. See include/gdn2.h for the contract of each call.
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -131,8 +132,11 @@ ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, co
   }
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.w = w; a.S0 = S0; a.o = o; a.ST = S_T;
   a.workspace = ws; a.ws_bytes = ws_bytes;
+  a.stall_polls = 0;
   return a;
 }
+
+std::atomic<unsigned> g_scan_stall{0};
 
 bool use_tc(const gdn2_params* p, const ChunkArgs& a) {
   return p->precision == GDN2_PREC_DEFAULT && p->T > 0 && p->B > 0 &&
@@ -141,13 +145,29 @@ bool use_tc(const gdn2_params* p, const ChunkArgs& a) {
 
 }  // namespace
 
+gdn2_status gdn2::check_chunk_params(const gdn2_params* p) {
+  const gdn2_status st = check_common(p, false);
+  if (st != GDN2_OK) return st;
+  if (p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return GDN2_ERR_UNSUPPORTED;
+  return GDN2_OK;
+}
+
+unsigned gdn2::scan_stall_polls() { return g_scan_stall.load(std::memory_order_relaxed); }
+
+gdn2_status gdn2::read_device_status(const void* scratch, cudaStream_t stream) {
+  int word = 0;
+  if (cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  return word == 0 ? GDN2_OK : GDN2_ERR_TIMEOUT;
+}
+
 gdn2_status gdn2::chunk_fwd_checked(const gdn2_params* p, const void* q, const void* k, const void* v,
                                      const float* alpha, const float* b, const float* w, const float* S0,
                                      void* o, float* S_T, void* workspace, size_t ws_bytes, void* stream,
                                      bool segmented_ok) {
-  gdn2_status st = check_common(p, false);
+  gdn2_status st = check_chunk_params(p);
   if (st != GDN2_OK) return st;
-  if (p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return GDN2_ERR_UNSUPPORTED;
   const size_t tokens = (size_t)p->B * p->T;
   if (tokens > 0) {
     if (!q || !k || !v || !o) return GDN2_ERR_INVALID_ARG;
@@ -184,6 +204,7 @@ gdn2_status gdn2::chunk_fwd_checked(const gdn2_params* p, const void* q, const v
     if (need > 0 && (overlaps(workspace, ws_bytes, o, o_bytes) || overlaps(workspace, ws_bytes, S_T, sz.st)))
       return GDN2_ERR_INVALID_ARG;
     a.ws_bytes = segmented_ok ? ws_bytes : chunk_tc_workspace(a);
+    a.stall_polls = scan_stall_polls();
     e = launch_chunk_tc(a, p->o_dtype == GDN2_BF16, s);
   } else {
     e = launch_chunk_simt(a, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16, s);
@@ -220,6 +241,14 @@ gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const void* k, c
                            float* S_T, void* workspace, size_t ws_bytes, void* stream) {
   return gdn2::chunk_fwd_checked(p, q, k, v, alpha, b, w, S0, o, S_T, workspace, ws_bytes, stream, false);
 }
+
+gdn2_status gdn2_chunk_fwd_status(const void* workspace, void* stream) {
+  if (workspace == nullptr) return GDN2_OK;   // the fp32 path keeps no device status
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDN2_ERR_INVALID_ARG;
+  return gdn2::read_device_status(workspace, static_cast<cudaStream_t>(stream));
+}
+
+void gdn2_debug_set_scan_stall(unsigned polls) { g_scan_stall.store(polls, std::memory_order_relaxed); }
 
 gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k, const void* v,
                              const float* alpha, const float* b, const float* w, float* S, void* o,

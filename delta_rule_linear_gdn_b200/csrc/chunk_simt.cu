@@ -33,7 +33,7 @@ struct SimtSmem {
   static constexpr int DP = D + 1;        // padded row stride of [C][D] arrays
   static constexpr int CP = kCMax + 1;    // padded row stride of [C][C] arrays
   static constexpr size_t floats =
-      4 * (size_t)kCMax * DP + (size_t)D * DVT + 2 * (size_t)kCMax * CP + 2 * (size_t)kCMax * DVT + D;
+      5 * (size_t)kCMax * DP + (size_t)D * DVT + 2 * (size_t)kCMax * CP + 2 * (size_t)kCMax * DVT + D;
   static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
   float* sz = sA + kCMax * CP;             // [C][DVT] z, then W, then U
   float* sP = sz + kCMax * DVT;            // [C][DVT] Q̄ S
   float* sgC = sP + kCMax * DVT;           // [D] γ_C
+  float* sGl = sgC + D;                    // [C][DP] low part of G (G = sG + sGl)
 
   const int tile = blockIdx.x % TILES;
   const int bh = blockIdx.x / TILES;
@@ -127,7 +128,9 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         qv = load_conv(qg + qk0, qk_tok, t, conv ? wq + c * 4 : nullptr, conv, hq_ ? hq_ + c : nullptr, hstride);
         kv = load_conv(kg + qk0, qk_tok, t, conv ? wk + c * 4 : nullptr, conv, hk_ ? hk_ + c : nullptr, hstride);
         const size_t gt = (tok0 + t) * a.Hg + hg;   // row of alpha, b
-        gv = logf(gate_at(a.alpha, mode == GDN2_GATES_GDN ? gt : gt * D + c, a.gate_logits));
+        const size_t ai = mode == GDN2_GATES_GDN ? gt : gt * D + c;
+        gv = a.gate_logits ? log_sigmoid_f32(__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.alpha)[ai]))
+                           : logf(a.alpha[ai]);
         bv = gate_at(a.b, (mode == GDN2_GATES_FULL) ? gt * D + c : gt, a.gate_logits);
       }
       sq[i * DP + c] = qv;
@@ -176,12 +179,17 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         se[i * DP + c] *= kk;
       }
     }
-    // 3. Cumulative log decay per key channel.
+    // 3. Cumulative log decay per key channel, summed in double and kept as
+    // a float pair (hi + lo): after a run of strong decay |G| is large, and a
+    // difference G_i − G_j of two single floats would lose the small
+    // exponent that tokens after that run need.
     if (tid < D) {
-      float acc = 0.f;
+      double acc = 0.0;
       for (int i = 0; i < C; ++i) {
-        acc += sG[i * DP + tid];
-        sG[i * DP + tid] = acc;
+        acc += (double)sG[i * DP + tid];
+        const float hi = (float)acc;
+        sG[i * DP + tid] = hi;
+        sGl[i * DP + tid] = (float)(acc - (double)hi);
       }
     }
     __syncthreads();
@@ -192,7 +200,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         float tv = 0.f, av = 0.f;
         if (j <= i) {
           for (int c = 0; c < D; ++c) {
-            const float dec = expf(sG[i * DP + c] - sG[j * DP + c]);
+            const float dec = expf((sG[i * DP + c] - sG[j * DP + c]) + (sGl[i * DP + c] - sGl[j * DP + c]));
             const float kd = sk[j * DP + c] * dec;
             tv += se[i * DP + c] * kd;
             av += sq[i * DP + c] * kd;
@@ -206,14 +214,14 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
     // 4b. Absorb the decay: Ē = γ ⊙ e, Q̄ = γ ⊙ q, K_end = k ⊙ exp(G_C − G), γ_C.
     for (int idx = tid; idx < C * D; idx += kThreads) {
       const int i = idx / D, c = idx % D;
-      const float G = sG[i * DP + c];
-      const float Gc = sG[(C - 1) * DP + c];
-      const float g = expf(G);
+      const float G = sG[i * DP + c], Gl = sGl[i * DP + c];
+      const float Gc = sG[(C - 1) * DP + c], Gcl = sGl[(C - 1) * DP + c];
+      const float g = expf(G + Gl);
       se[i * DP + c] *= g;
       sq[i * DP + c] *= g;
-      sk[i * DP + c] *= expf(Gc - G);
+      sk[i * DP + c] *= expf((Gc - G) + (Gcl - Gl));
     }
-    if (tid < D) sgC[tid] = expf(sG[(C - 1) * DP + tid]);
+    if (tid < D) sgC[tid] = expf(sG[(C - 1) * DP + tid] + sGl[(C - 1) * DP + tid]);
     __syncthreads();
 
     // 5. W = Z − Ē S and P = Q̄ S for the tile.

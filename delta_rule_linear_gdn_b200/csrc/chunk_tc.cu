@@ -91,8 +91,13 @@ constexpr int SL_UW = 32768;          // U_wᵀ fp16 [128 dv][64 tok]
 constexpr int SL_KE = 49152;          // K_end fp16 [64 tok][128 key] BS 8192
 constexpr int SL_AQ = 65536;          // −Aqk fp16 [64 i][64 j]
 constexpr int SL_GC = 73728;          // γ_C  fp32 [128]
-constexpr int SLOT_USED = 74240;      // bytes copied per chunk
+constexpr int SL_WM = 74240;          // max |U_w| over the chunk (fp32; 16 bytes)
+constexpr int SLOT_USED = 74256;      // bytes copied per chunk
+constexpr int SL_FLAG = SLOT_USED;    // int: 1 = the slot is written by the exact kernel (not copied)
 constexpr int SLOT = 74752;           // slot stride (1 KB multiple)
+// Least α product over an aligned 16-token quarter (per channel) that the
+// prep's reciprocal factorisation takes; items below it run exactly.
+constexpr float kStrongDecay = 5.421010862427522e-20f;   // 2^-64
 constexpr int BS_ROW128 = 16384;      // block stride of a 128-row tile
 constexpr int BS_ROW64 = 8192;        // block stride of a 64-row tile
 
@@ -293,6 +298,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   float* sX = reinterpret_cast<float*>(smem + P_X);
 
   int* s_item = sflag + 1;               // the next item, when taken from the counter
+  uint32_t* s_wmax = reinterpret_cast<uint32_t*>(sflag + 2);   // max |U_w| of the item (float bits)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_items = VL ? a.cu_chk[a.nseq] * a.Hv : a.B * a.Hv * n_seg;
@@ -302,6 +308,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     fence_mbar_init();
     *sflag = 0;
     *s_item = counter ? atomicAdd(counter, 1) : 0;
+    *s_wmax = 0;
   }
   if (warp == 0) {
     tmem_alloc(tmem_ptr, PT_COLS);
@@ -429,13 +436,28 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     __syncthreads();
     // every thread has read s_item for this item (at the end of the previous one)
     if (counter && tid == 0) *s_item = atomicAdd(counter, 1);
-    bool gram_bf16;
+    bool gram_bf16, exact;
     {
       float mall = sred[0];
 #pragma unroll
       for (int w_ = 1; w_ < NP / 32; ++w_) mall = fminf(mall, sred[w_]);
       // every in-quarter forward/backward product is ≥ the quarter product
       gram_bf16 = !(mall > 6.103515625e-05f);   // 2^-14
+      // Below 2^-64 the reciprocal factors of the Gram operands leave the
+      // fp32 range (and an α product that underflows makes them inf): the
+      // item goes to the exact kernel (chunk_fix_kernel), which writes its
+      // slot before the scan reads it. The comparison is false for NaN too.
+      exact = !(mall >= kStrongDecay);
+    }
+    if (exact) {
+      if (tid == 0) *reinterpret_cast<int*>(slot + SL_FLAG) = 1;
+      // every thread has read the quarter minima and α (pass 1); thread 0's
+      // s_item is visible after this barrier
+      __syncthreads();
+      const int nx = counter ? *s_item : item + (int)gridDim.x;
+      if (use_amap && tid == 0 && nx < n_items) fetch_alpha(nx);
+      item = nx;
+      continue;
     }
     if (tid < D) {
       const float g = sPq[tid] * sPq[D + tid] * sPq[2 * D + tid] * sPq[3 * D + tid];
@@ -772,6 +794,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       // copies, byte for byte the slot's layout
       const uint32_t col = hc == 0 ? PT_YT : PT_UW;
       const int stg = P_YS + hc * 16384;
+      uint32_t wm = 0;                   // max |U_w| (the scan scales its state by it)
 #pragma unroll
       for (int cb0 = 0; cb0 < 64; cb0 += 32) {
         float v[32];
@@ -780,6 +803,14 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
         tmem_wait_ld();
 #pragma unroll
         for (int cb = 0; cb < 32; cb += 8) st16(smem, stg + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
+        if (hc == 1) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) wm = max(wm, __float_as_uint(v[u]) & 0x7fffffffu);
+        }
+      }
+      if (hc == 1) {
+        wm = __reduce_max_sync(0xffffffffu, wm);
+        if (lane == 0) atomicMax(s_wmax, wm);
       }
     }
     fence_async_smem();
@@ -790,6 +821,9 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       bulk_s2g(slot + SL_YT, smem + P_YS, 16384);
       bulk_s2g(slot + SL_UW, smem + P_YS + 16384, 16384);
       bulk_commit();
+      *reinterpret_cast<int*>(slot + SL_FLAG) = 0;   // written here, not by the exact kernel
+      *reinterpret_cast<uint32_t*>(slot + SL_WM) = *s_wmax;
+      *s_wmax = 0;                       // (the next item's maxima come after two barriers)
     }
     item = counter ? *s_item : item + (int)gridDim.x;   // written before the barriers above
   }
@@ -802,6 +836,240 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   // after it: the next scan, ordered after this grid, then also follows that
   // scan (whose final state it reads).
   griddep_wait();
+}
+
+// =============================================================================
+// Exact prep of the items the prep kernel flagged (decay too strong for its
+// reciprocal factors). Same algebra and same slot contents, in fp32 with the
+// decay of every pair formed as the running product Π_{j<s≤i} α_s — no
+// reciprocal and no logarithm — so it holds for every α ∈ [0, 1]:
+//     T_ij  = Σ_c e_ic k_jc Π_{j<s≤i} α_sc (j < i),  Aqk_ij likewise with q (j ≤ i)
+//     A = (I + T)⁻¹ (forward substitution), Y = A (γ ⊙ e), U_w = A (w ⊙ v),
+//     Q̄ = γ ⊙ q, K_end,j = k_j ⊙ Π_{j<s≤C} α_s, γ_C.
+// One CTA reads the flags of FX_ITEMS consecutive items and does the flagged
+// ones in turn; with nothing flagged it only reads the flags.
+// =============================================================================
+constexpr int FX_THREADS = 256;
+constexpr int FX_ITEMS = 32;
+constexpr int FX_LD = D + 4;          // fp32 row stride of the [64][128] arrays
+constexpr int FX_TS = C + 1;          // fp32 row stride of the [64][64] arrays
+constexpr size_t FX_SMEM = (size_t)(4 * C * FX_LD + 3 * C * FX_TS) * sizeof(float) + 16;   // + mask, max
+
+template <bool VL>
+__global__ void __launch_bounds__(FX_THREADS, 1) chunk_fix_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm) {
+  extern __shared__ __align__(16) float fsm[];
+  float* sAl = fsm;                     // α, later Z = w ⊙ v      [64][FX_LD]
+  float* sE = sAl + C * FX_LD;          // e = b ⊙ k, later Ē = γ ⊙ e
+  float* sK = sE + C * FX_LD;           // k, later K_end
+  float* sQ = sK + C * FX_LD;           // q, later Q̄ = γ ⊙ q
+  float* sT = sQ + C * FX_LD;           // T (strict lower)        [64][FX_TS]
+  float* sAq = sT + C * FX_TS;          // Aqk (lower incl.)
+  float* sI = sAq + C * FX_TS;          // (I + T)⁻¹
+  uint32_t* smask = reinterpret_cast<uint32_t*>(sI + C * FX_TS);
+  uint32_t* swm = smask + 1;            // max |U_w| of the item (float bits)
+
+  const int tid = threadIdx.x;
+  const int n_items = VL ? a.cu_chk[a.nseq] * a.Hv : a.B * a.Hv * n_seg;
+  const int first = (int)blockIdx.x * FX_ITEMS;
+  if (tid < 32) {
+    const int item = first + tid;
+    bool flagged = false;
+    if (item < n_items) {
+      const Item it = decode_item<VL>(a, c_begin, item, sm);
+      const uint8_t* slot = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + it.slot * SLOT;
+      flagged = *reinterpret_cast<const volatile int*>(slot + SL_FLAG) != 0;
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, flagged);
+    if (tid == 0) *smask = m;
+  }
+  __syncthreads();
+  uint32_t mask = *smask;
+  if (mask == 0) return;
+
+  const bool full = a.gate_mode == GDN2_GATES_FULL;
+  const bool alpha_pc = a.gate_mode != GDN2_GATES_GDN;
+  const bool lg = a.gate_logits != 0, qkg = a.Hg != a.Hv, f16 = a.qkv_f16 != 0;
+  auto in_val = [&](const void* p, size_t i) -> float {
+    return f16 ? __half2float(static_cast<const __half*>(p)[i]) : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+  };
+
+  while (mask) {
+    const int bit = __ffs(mask) - 1;
+    mask &= mask - 1;
+    const Item it = decode_item<VL>(a, c_begin, first + bit, sm);
+    uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + it.slot * SLOT;
+    __syncthreads();   // the previous item's arrays (and its max) are read
+    if (tid == 0) *swm = 0;
+
+    // ---- inputs (tokens past the sequence's end: α = 1, everything else 0)
+    for (int idx = tid; idx < C * D; idx += FX_THREADS) {
+      const int i = idx / D, c = idx % D;
+      float al = 1.f, e = 0.f, kx = 0.f, qx = 0.f;
+      if (i < it.Lc) {
+        const size_t r = (size_t)it.bi * a.T + it.t0 + i;
+        const size_t gr = qkg ? r * a.Hqk + it.hq : r * a.Hv + it.h;
+        const size_t tq = ((size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i) * a.Hqk + it.hq;
+        al = gate_at(a.alpha, alpha_pc ? gr * D + c : gr, lg);
+        kx = in_val(a.k, tq * D + c);
+        qx = in_val(a.q, tq * D + c);
+        e = gate_at(a.b, full ? gr * D + c : gr, lg) * kx;
+      }
+      sAl[i * FX_LD + c] = al;
+      sE[i * FX_LD + c] = e;
+      sK[i * FX_LD + c] = kx;
+      sQ[i * FX_LD + c] = qx;
+    }
+    __syncthreads();
+
+    // ---- T and Aqk. Thread (j, part) runs down column j over its 32
+    // channels c = 16m + 4·part + r, carrying Π_{j<s≤i} α_s per channel;
+    // the four parts of a column are adjacent lanes and add by shuffles.
+    {
+      const int j = tid >> 2, part = tid & 3;
+      float kj[32], dd[32];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float4 k4 = *reinterpret_cast<const float4*>(sK + j * FX_LD + 16 * m + 4 * part);
+        kj[4 * m] = k4.x; kj[4 * m + 1] = k4.y; kj[4 * m + 2] = k4.z; kj[4 * m + 3] = k4.w;
+      }
+#pragma unroll
+      for (int u = 0; u < 32; ++u) dd[u] = 1.f;
+      for (int i = (tid >> 5) * 8; i < C; ++i) {      // from the warp's first column
+        float at = 0.f, aa = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int off = i * FX_LD + 16 * m + 4 * part;
+          const float4 al = *reinterpret_cast<const float4*>(sAl + off);
+          const float4 e4 = *reinterpret_cast<const float4*>(sE + off);
+          const float4 q4 = *reinterpret_cast<const float4*>(sQ + off);
+          const float alv[4] = {al.x, al.y, al.z, al.w}, ev[4] = {e4.x, e4.y, e4.z, e4.w},
+                      qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int u = 4 * m + r;
+            dd[u] *= i > j ? alv[r] : 1.f;
+            const float kd = kj[u] * dd[u];
+            at = fmaf(ev[r], kd, at);
+            aa = fmaf(qv[r], kd, aa);
+          }
+        }
+        at += __shfl_xor_sync(0xffffffffu, at, 1);
+        aa += __shfl_xor_sync(0xffffffffu, aa, 1);
+        at += __shfl_xor_sync(0xffffffffu, at, 2);
+        aa += __shfl_xor_sync(0xffffffffu, aa, 2);
+        if (part == 0 && i >= j) {
+          sT[i * FX_TS + j] = i > j ? at : 0.f;
+          sAq[i * FX_TS + j] = aa;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- threads 0..127, channel c: γ_i (forward product), Ē, Q̄ in place;
+    // K_end (backward product) and γ_C. Threads 128..191: column j of
+    // (I + T)⁻¹ by forward substitution.
+    if (tid < D) {
+      const int c = tid;
+      float g = 1.f;
+      for (int i = 0; i < C; ++i) {
+        g *= sAl[i * FX_LD + c];
+        sE[i * FX_LD + c] *= g;
+        sQ[i * FX_LD + c] *= g;
+      }
+      reinterpret_cast<float*>(slot + SL_GC)[c] = g;
+      float p = 1.f;
+      for (int j = C - 1; j >= 0; --j) {
+        sK[j * FX_LD + c] *= p;
+        p *= sAl[j * FX_LD + c];
+      }
+    } else if (tid < D + C) {
+      const int j = tid - D;
+      for (int i = 0; i < C; ++i) {
+        float x = (i == j) ? 1.f : 0.f;
+        if (i > j) {
+          float acc = 0.f;
+          for (int l = j; l < i; ++l) acc = fmaf(sT[i * FX_TS + l], sI[l * FX_TS + j], acc);
+          x = -acc;
+        }
+        sI[i * FX_TS + j] = x;
+      }
+    }
+    __syncthreads();
+    // Z = w ⊙ v over the α array
+    for (int idx = tid; idx < C * D; idx += FX_THREADS) {
+      const int i = idx / D, c = idx % D;
+      float z = 0.f;
+      if (i < it.Lc) {
+        const size_t r = (size_t)it.bi * a.T + it.t0 + i;
+        const size_t wr = full ? (r * a.Hv + it.h) * D + c : (qkg ? r * a.Hqk + it.hq : r * a.Hv + it.h);
+        const size_t tv = ((size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i) * a.Hv + it.h;
+        z = gate_at(full ? a.w : a.b, wr, lg) * in_val(a.v, tv * D + c);
+      }
+      sAl[i * FX_LD + c] = z;
+    }
+    __syncthreads();
+
+    // ---- −Yᵀ (threads 0..127) and U_wᵀ (128..255): row c of the [128][64]
+    // fp16 tile, one thread each, from column c of Ē or Z.
+    {
+      const int c = tid & (D - 1);
+      const bool yside = tid < D;
+      const float* src = yside ? sE : sAl;
+      float acc[C];
+#pragma unroll
+      for (int i = 0; i < C; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < C; ++j) {
+        const float x = src[j * FX_LD + c];
+#pragma unroll
+        for (int i = j; i < C; ++i) acc[i] = fmaf(sI[i * FX_TS + j], x, acc[i]);
+      }
+      const float sg = yside ? -1.f : 1.f;
+      uint8_t* dst = slot + (yside ? SL_YT : SL_UW);
+      if (!yside) {
+        uint32_t wm = 0;
+#pragma unroll
+        for (int i = 0; i < C; ++i) wm = max(wm, __float_as_uint(acc[i]) & 0x7fffffffu);
+        wm = __reduce_max_sync(0xffffffffu, wm);
+        if ((tid & 31) == 0) atomicMax(swm, wm);
+      }
+#pragma unroll
+      for (int i0 = 0; i0 < C; i0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = sg * acc[i0 + u];
+        *reinterpret_cast<uint4*>(dst + sw_off(c, i0, BS_ROW128)) = pack8_f16(x);
+      }
+    }
+    // −Q̄ᵀ: row c (key) of a [128][64] tile, threads 0..127
+    if (tid < D) {
+      const int c = tid;
+#pragma unroll
+      for (int i0 = 0; i0 < C; i0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = -sQ[(i0 + u) * FX_LD + c];
+        *reinterpret_cast<uint4*>(slot + SL_QT + sw_off(c, i0, BS_ROW128)) = pack8_f16(x);
+      }
+    }
+    // K_end [64 tok][128 key]: 1024 pieces of 8 keys; −Aqk [64][64] masked j ≤ i: 512 pieces
+    for (int pc = tid; pc < C * D / 8; pc += FX_THREADS) {
+      const int j = pc >> 4, c0 = (pc & 15) * 8;
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = sK[j * FX_LD + c0 + u];
+      *reinterpret_cast<uint4*>(slot + SL_KE + sw_off(j, c0, BS_ROW64)) = pack8_f16(x);
+    }
+    for (int pc = tid; pc < C * C / 8; pc += FX_THREADS) {
+      const int i = pc >> 3, j0 = (pc & 7) * 8;
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = (j0 + u <= i) ? -sAq[i * FX_TS + j0 + u] : 0.f;
+      *reinterpret_cast<uint4*>(slot + SL_AQ + sw_off(i, j0, BS_ROW64)) = pack8_f16(x);
+    }
+    __syncthreads();
+    if (tid == 0) *reinterpret_cast<uint32_t*>(slot + SL_WM) = *swm;
+  }
 }
 
 // =============================================================================
@@ -833,12 +1101,13 @@ struct ScanLayout {
   static constexpr int KE = UW + DV * 128;       // K_end [64 tok][128 key], BS 8192
   static constexpr int AQ = KE + 16384;          // −Aqk [64][64] (must follow K_end: see the O product)
   static constexpr int GC = AQ + 8192;           // γ_C [128] fp32
-  static constexpr int BYTES = GC + 512;         // copied per chunk
+  static constexpr int WM = GC + 512;            // max |U_w| of the chunk (fp32)
+  static constexpr int BYTES = WM + 16;          // copied per chunk
   static constexpr int STAGE = (BYTES + 1023) / 1024 * 1024;
   static constexpr int SH = 2 * STAGE;           // S fp16 [128 key][DV], BS 16384
   static constexpr int U = SH + 128 * DV * 2;    // U fp16 [64 tok][DV], BS 8192
-  static constexpr int I = U + 64 * DV * 2;      // [I_64; 0] fp16 [128][64]
-  static constexpr int BAR = I + 16384;          // 10 mbarriers
+  static constexpr int RED = U + 64 * DV * 2;    // per-warp maxima of |S| [2][16] (float bits)
+  static constexpr int BAR = RED + 128;          // 11 mbarriers
   static constexpr int TMEMP = BAR + 128;
   static constexpr int FLAG = TMEMP + 16;
   static constexpr int SMEM = FLAG + 16;
@@ -846,12 +1115,13 @@ struct ScanLayout {
   static constexpr uint32_t T_COLS = DV == 64 ? 256 : 512;
 };
 static_assert(ScanLayout<128>::ZT == SL_YT && ScanLayout<128>::UW == SL_UW && ScanLayout<128>::KE == SL_KE &&
-                  ScanLayout<128>::AQ == SL_AQ && ScanLayout<128>::GC == SL_GC && ScanLayout<128>::BYTES == SLOT_USED,
+                  ScanLayout<128>::AQ == SL_AQ && ScanLayout<128>::GC == SL_GC && ScanLayout<128>::WM == SL_WM &&
+                  ScanLayout<128>::BYTES == SLOT_USED,
               "a full-width stage is the slot");
 static_assert(SL_AQ == SL_KE + 16384 && SL_GC == SL_AQ + 8192, "slot tail copied in one piece");
 static_assert(ScanLayout<64>::SMEM <= 232448 && ScanLayout<128>::SMEM <= 232448, "scan shared memory");
 static_assert(ScanLayout<64>::SH % 1024 == 0 && ScanLayout<128>::SH % 1024 == 0 && ScanLayout<64>::U % 1024 == 0 &&
-                  ScanLayout<128>::U % 1024 == 0 && ScanLayout<64>::I % 1024 == 0 && ScanLayout<128>::I % 1024 == 0,
+                  ScanLayout<128>::U % 1024 == 0,
               "swizzled tiles on 1 KB boundaries");
 
 // 16 bytes of output: 8 bf16 or 4 fp32 values of sc · x.
@@ -886,6 +1156,7 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   uint64_t* b_sh = bars + 5;            // fp16 S written (one arrival per epilogue warp)
   uint64_t* b_o = bars + 6;             // [2] D buffer holds the chunk's −O
   uint64_t* b_of = bars + 8;            // [2] D buffer read out
+  uint64_t* b_never = bars + 10;        // nothing arrives on it (the failure-path test hook waits here)
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::TMEMP);
   int* sflag = reinterpret_cast<int*>(smem + L::FLAG);
   volatile int* estop = sflag + 1;      // [2] the epilogue warps' samples of the flag
@@ -918,7 +1189,7 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   }
 
   if (tid == 0) {
-    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], &bars[i] == b_sh ? NE / 32 : 1);   // b_sh: one per epilogue warp
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], &bars[i] == b_sh ? NE / 32 : 1);   // b_sh: one per epilogue warp
     fence_mbar_init();
     sflag[0] = 0;
     sflag[1] = 0;
@@ -927,18 +1198,6 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   if (warp == 0) {
     tmem_alloc(tmem_ptr, L::T_COLS);
     tmem_relinquish();
-  }
-  if (warp < 8) {
-    // constant [I_64; 0] (128 rows × 64 columns), in place before any product
-    const int r = (warp & 3) * 32 + lane, cq = (warp >> 2) * 32;
-#pragma unroll
-    for (int cb = 0; cb < 32; cb += 8) {
-      float x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = (r == cq + cb + u) ? 1.f : 0.f;
-      st16(smem, L::I + sw_off(r, cq + cb, BS_ROW128), pack8_f16(x));
-    }
-    fence_async_smem();
   }
   fence_before_sync();
   __syncthreads();
@@ -966,13 +1225,14 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
         ++issued;
       }
       const uint32_t id_zs = idesc_f16(128, DV, true, true);     // −Zᵀ (MN) × S (MN)
-      const uint32_t id_iu = idesc_f16(128, DV, false, false);   // [I;0] (K) × U_wᵀ (K)
       const uint32_t id_kn = idesc_f16(128, DV, true, true);     // K_endᵀ (MN) × U (MN)
       const uint32_t id_au = idesc_f16(128, DV, false, true);    // [·;−Aqk] (K) × U (MN)
       const uint64_t sh0 = desc_mn_sw(smem_u32(smem + L::SH), 0, BS_ROW128);
       const uint64_t u0 = desc_mn_sw(smem_u32(smem + L::U), 0, BS_ROW64);
-      const uint64_t i0 = desc_k_sw(smem_u32(smem + L::I), 0, BS_ROW128);
-      bool ok = true;
+      // Failure-path test hook: a bounded wait that cannot complete, taken
+      // before any product is issued, so the give-up path below has only
+      // the two slot copies to drain.
+      bool ok = a.stall_polls == 0 || mbar_wait_or_stop(b_never, 0, vflag, a.stall_polls);
       for (int c = 0; c < n_seg && ok; ++c) {
         const int s = c & 1;
         const uint32_t ph = (uint32_t)(c & 1);
@@ -983,17 +1243,14 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
         if (!ok) break;
         ++landed;
         fence_after_sync();
-        // D = [I; 0] U_w (needs no state: issued ahead), then D += (−Z) S
+        // D = (−Z) S (the scaled state's fp16 copy; the U epilogue adds U_w)
         const uint64_t z0 = desc_mn_sw(smem_u32(stg + L::ZT), 0, BS_ROW128);
-        const uint64_t w0 = desc_k_sw(smem_u32(stg + L::UW), 0, BS_ROW64);   // DV rows, one K block
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          mma16(tmem + db, i0 + k_step_sw(ks, BS_ROW128), w0 + k_step_sw(ks, BS_ROW64), id_iu, ks > 0);
         ok = mbar_wait_or_stop(b_sh, ph, vflag);
         if (!ok) break;
         fence_after_sync();
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) mma16(tmem + db, z0 + mn_step_sw(ks), sh0 + mn_step_sw(ks), id_zs, 1);
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma16(tmem + db, z0 + mn_step_sw(ks), sh0 + mn_step_sw(ks), id_zs, ks > 0);
         mma_commit(b_d);
         // S += K_endᵀ U (TMEM holds Γ S), then D_rows 64..127 += (−Aqk) U; the
         // A operand of the latter starts 64 rows before −Aqk (in K_end), whose
@@ -1042,8 +1299,38 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
       fence_after_sync();
     };
 
-    // The entry state: fp16 S for the first chunk's products, TMEM ← S · Γ
-    // of the first chunk.
+    // Block floating point. Chunk c runs with a power-of-two scale 2^k_c on
+    // the state in TMEM, its fp16 copy, D and U, so that the 16-bit operands
+    // stay in fp16's range however small or large the state becomes: k_c is
+    // chosen, from the CTA-wide maximum of |S| at the chunk's entry and of
+    // |U_w| of the chunk (stored by the prep), to put the larger of the two
+    // in [2^8, 2^9), leaving 2^7 of headroom below fp16's largest value for
+    // U = U_w − Y S. Every epilogue thread derives the same k_c from the same
+    // shared maxima; the outputs and S_T are divided by 2^k_c.
+    uint32_t* red = reinterpret_cast<uint32_t*>(smem + L::RED);   // [2][16]: per-warp maxima, two buffers
+    auto cta_max = [&](const float* v, int buf) -> float {
+      uint32_t m = 0;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) m = max(m, __float_as_uint(v[u]) & 0x7fffffffu);
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (lane == 0) red[buf * 16 + warp] = m;
+      epi_sync<NE>();
+      uint32_t M = 0;
+#pragma unroll
+      for (int w_ = 0; w_ < NE / 32; ++w_) M = max(M, red[buf * 16 + w_]);
+      return __uint_as_float(M);
+    };
+    auto exp2i = [](int k) -> float { return __uint_as_float((uint32_t)(127 + k) << 23); };   // |k| ≤ 126
+    // k that brings `ref` (> 0) to [2^8, 2^9); a zero (or NaN) reference keeps k
+    auto pick_k = [](float ref, int k) -> int {
+      if (!(ref > 0.f)) return k;
+      const int e = (int)((__float_as_uint(ref) >> 23) & 0xffu) - 127;   // ⌊log2 ref⌋ (subnormal: −127)
+      return max(-60, min(60, 8 - e));
+    };
+    int k_cur = 0, k_prev = 0;          // scale exponents of chunk c and c − 1
+
+    // The entry state: fp16 2^k S for the first chunk's products, TMEM ←
+    // 2^k S · Γ of the first chunk.
     wait(&full[0], 0);
     {
       const float g = reinterpret_cast<const float*>(smem + L::GC)[row];
@@ -1054,6 +1341,12 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
         const float4 x = S0 ? __ldg(reinterpret_cast<const float4*>(S0 + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
         v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
       }
+      const float M = cta_max(v, 0);
+      k_cur = pick_k(fmaxf(M, *reinterpret_cast<const float*>(smem + L::WM)), 0);
+      k_prev = k_cur;
+      const float sg = exp2i(k_cur);
+#pragma unroll
+      for (int u = 0; u < 32; ++u) v[u] *= sg;
 #pragma unroll
       for (int cb = 0; cb < 32; cb += 8) st16(smem, L::SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
 #pragma unroll
@@ -1068,8 +1361,8 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
     if (lane == 0) mbar_arrive(b_sh);
 
     // Outputs of chunk cc from D buffer `db`: row 64 + i of D is token i; this
-    // thread writes 32 contiguous d_v values of it.
-    auto out_rows = [&](int cc, uint32_t db, uint64_t* freed) {
+    // thread writes 32 contiguous d_v values of it. D holds −2^k O / s.
+    auto out_rows = [&](int cc, uint32_t db, uint64_t* freed, int k) {
       const int t0o = cc * C;
       const int Lco = min(C, trem - t0o);
       float v[32];
@@ -1084,7 +1377,9 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
         TOut* dst = og + ((tok0 + t0o + i) * a.Hv + h) * D + dv0;
         constexpr int VEC = 16 / (int)sizeof(TOut);
 #pragma unroll
-        for (int u = 0; u < 32; u += VEC) *reinterpret_cast<uint4*>(dst + u) = pack_out<TOut>(v + u, -a.scale);
+        const float sc = -a.scale * exp2i(-k);
+#pragma unroll
+        for (int u = 0; u < 32; u += VEC) *reinterpret_cast<uint4*>(dst + u) = pack_out<TOut>(v + u, sc);
       }
     };
 
@@ -1094,12 +1389,21 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
       const uint32_t ph = (uint32_t)(c & 1);
       const uint32_t db = L::T_D + (uint32_t)DV * (uint32_t)s;
       if (u_warp) {
-        // U (rows 0..63 of D) → fp16 tile [tok][dv]
+        // U = 2^k (U_w − Y S): rows 0..63 of D (−2^k Y S) plus 2^k U_w from the
+        // stage's U_wᵀ tile [dv][tok] → fp16 tile [tok][dv]
+        wait(&full[s], (uint32_t)((c >> 1) & 1));   // (landed before D: makes the copy visible here)
         wait(b_d, ph);
         float v[32];
         tmem_ld16(t_lane + db + c0, v);
         tmem_ld16(t_lane + db + c0 + 16, v + 16);
         tmem_wait_ld();
+        {
+          const float sg = exp2i(k_cur);
+          const uint8_t* uw = smem + s * L::STAGE + L::UW;
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            v[u] = fmaf(sg, __half2float(*reinterpret_cast<const __half*>(uw + sw_off(c0 + u, row, 0))), v[u]);
+        }
 #pragma unroll
         for (int cb = 0; cb < 32; cb += 8) st16(smem, L::U + sw_off(row, c0 + cb, BS_ROW64), pack8_f16(v + cb));
         fence_async_smem();
@@ -1109,7 +1413,7 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
       } else if (c > 0) {
         // outputs of the previous chunk
         wait(&b_o[s ^ 1], (uint32_t)(((c - 1) >> 1) & 1));
-        out_rows(c - 1, L::T_D + (uint32_t)DV * (uint32_t)(s ^ 1), &b_of[s ^ 1]);
+        out_rows(c - 1, L::T_D + (uint32_t)DV * (uint32_t)(s ^ 1), &b_of[s ^ 1], k_prev);
       }
       // the state: fp16 S for the next chunk and TMEM ← S · Γ_next; S_T after the last
       const bool more = c + 1 < n_seg;
@@ -1119,8 +1423,17 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
         float v[32];
         tmem_ld16(t_lane + L::T_S + c0, v);
         tmem_ld16(t_lane + L::T_S + c0 + 16, v + 16);
-        tmem_wait_ld();
+        tmem_wait_ld();                   // 2^k_c S_{c+1}
         if (more) {
+          // the next chunk's scale, from max |S_{c+1}| and its max |U_w|
+          const float M = cta_max(v, (c + 1) & 1) * exp2i(-k_cur);
+          const float W = *reinterpret_cast<const float*>(smem + (s ^ 1) * L::STAGE + L::WM);
+          const int k_next = pick_k(fmaxf(M, W), k_cur);
+          const float r = exp2i(k_next - k_cur);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] *= r;
+          k_prev = k_cur;
+          k_cur = k_next;
 #pragma unroll
           for (int cb = 0; cb < 32; cb += 8) st16(smem, L::SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
           // publish this warp's part of S at once: the next products need
@@ -1134,10 +1447,15 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
           tmem_st16(t_lane + L::T_S + c0, v);
           tmem_st16(t_lane + L::T_S + c0 + 16, v + 16);
           tmem_wait_st();
-        } else if (S_out && ok) {
-          float* ST = S_out + ((size_t)bh * D + row) * D + dv0;
+        } else {
+          k_prev = k_cur;
+          if (S_out && ok) {
+            const float r = exp2i(-k_cur);
+            float* ST = S_out + ((size_t)bh * D + row) * D + dv0;
 #pragma unroll
-          for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(ST + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+            for (int u = 0; u < 32; u += 4)
+              *reinterpret_cast<float4*>(ST + u) = make_float4(r * v[u], r * v[u + 1], r * v[u + 2], r * v[u + 3]);
+          }
         }
       }
       // One barrier per chunk orders the scaled TMEM state before the next
@@ -1162,7 +1480,7 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
     if (!stopped && n_seg > 0 && !u_warp) {
       const int s = (n_seg - 1) & 1;
       wait(&b_o[s], (uint32_t)(((n_seg - 1) >> 1) & 1));
-      out_rows(n_seg - 1, L::T_D + (uint32_t)DV * (uint32_t)s, &b_of[s]);
+      out_rows(n_seg - 1, L::T_D + (uint32_t)DV * (uint32_t)s, &b_of[s], k_cur);
     }
     if (!ok) atomicOr(sflag, 1);
   }
@@ -1478,6 +1796,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   const int scan_smem = full_width ? ScanLayout<128>::SMEM : ScanLayout<64>::SMEM;
   if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
     return e;
+  auto fix = vl ? chunk_fix_kernel<true> : chunk_fix_kernel<false>;
+  if ((e = cudaFuncSetAttribute(fix, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FX_SMEM)) != cudaSuccess)
+    return e;
   // Persistent prep: two CTAs per SM. Two fit by shared memory (2 × 113 KB),
   // registers (2 × 256 × 128) and tensor memory (2 × 256 of 512 columns); the
   // occupancy calculator reports one for any kernel that allocates tensor
@@ -1516,6 +1837,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     int* counter = nseg_ov > 0 ? reinterpret_cast<int*>(ws) + 1 + k : nullptr;
     const int items = vl ? nchunks * a.Hv : BH * n;
     const int grid = std::min(items, prep_ctas);
+    ChunkArgs ap = a;        // the prep's view of q, k, v (the load step's copies with the conv / L2 norm)
     if (items == 0) {
       // nothing to prepare (packed sequences, all empty)
     } else if (pre) {
@@ -1527,7 +1849,6 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       __half* vo = ko + (size_t)rows * Tseg * a.Hqk * D;
       const dim3 qgrid((qp_groups + QP_THREADS - 1) / QP_THREADS, (Tseg + QP_TOK - 1) / QP_TOK, rows);
       (vl ? qkv_prep_kernel<true> : qkv_prep_kernel<false>)<<<qgrid, QP_THREADS, 0, s>>>(a, t_begin, Tseg, qo, ko, vo);
-      ChunkArgs ap = a;
       ap.q = qo;
       ap.k = ko;
       ap.v = vo;
@@ -1547,6 +1868,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       prep_fn(false)<<<grid, NP, P_SMEM, s>>>(
           a, c0, n, sm, counter, amap, use_amap);
     }
+    // the items whose decay the prep's factors cannot take, exactly
+    if (items > 0) fix<<<(items + FX_ITEMS - 1) / FX_ITEMS, FX_THREADS, FX_SMEM, s>>>(ap, c0, n, sm);
     scan<<<scan_ctas, scan_threads, scan_smem, s>>>(a, c0, n, sm, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;

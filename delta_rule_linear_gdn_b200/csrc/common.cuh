@@ -26,6 +26,10 @@ constexpr float kL2Eps = 1e-6f;
 // (the fast exponential and division intrinsics: a few ulp, far inside what
 // the gates feed, and a handful of instructions instead of a few dozen)
 __device__ __forceinline__ float sigmoid_f32(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// log σ(x) = −log(1 + e^(−x)), written as min(x, 0) − log1p(e^(−|x|)) so that
+// it stays finite for every finite x (σ(x) itself underflows to 0 below
+// x ≈ −87, where log would give −∞).
+__device__ __forceinline__ float log_sigmoid_f32(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
 __device__ __forceinline__ float gate_at(const float* g, size_t i, bool logits) {
   return logits ? sigmoid_f32(__bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[i])) : g[i];
 }
@@ -65,6 +69,9 @@ struct ChunkArgs {
   int nseq;
   int cu_tok[GDN2_MAX_SEQS + 1];
   int cu_chk[GDN2_MAX_SEQS + 1];
+  // Failure-path test hook (gdn2_debug_set_scan_stall): > 0 makes the scan
+  // wait first, for at most this many polls, on a barrier nothing signals.
+  unsigned stall_polls;
 };
 
 // First token (in the q, k, v, o buffers) and length of sequence bi.
@@ -104,6 +111,16 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s);
 // Writes a.conv_out: the three pre-conv inputs that end at token T−1 of each
 // sequence (history from a.conv_in shifted in when T < 3).
 cudaError_t launch_conv_state(const ChunkArgs& a, int qkv_bf16, cudaStream_t s);
+
+// Shape, enum and offset checks shared by the prefill entry points.
+gdn2_status check_chunk_params(const gdn2_params* p);
+
+// The polls the scan's stall hook waits (0: off).
+unsigned scan_stall_polls();
+
+// GDN2_OK or GDN2_ERR_TIMEOUT from the status word a tensor-core prefill
+// keeps at the start of its scratch, after the work on `stream` so far.
+gdn2_status read_device_status(const void* scratch, cudaStream_t stream);
 
 // gdn2_chunk_fwd after argument checks; `segmented_ok` accepts a workspace
 // between the minimum and the full size.

@@ -4,9 +4,11 @@
 //
 // The scratch is a file-scope __device__ array. Its host-side name is only a
 // stand-in for the device symbol, so host code never passes it to a kernel:
-// the device address is looked up once per device with cudaGetSymbolAddress
-// (with that device current) and cached. Every GPU that loads the library
-// holds the array until the process exits.
+// the device address is looked up per device with cudaGetSymbolAddress (with
+// that device current) and cached once the lookup has succeeded. The first
+// call on a device also loads the library's device code there, which is when
+// the array is reserved; every GPU that has done so holds it until the
+// process exits.
 
 #include <mutex>
 
@@ -20,23 +22,22 @@ constexpr size_t kNoAllocScratchBytes = 32u << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void* g_scratch[kMaxDevices];
-cudaError_t g_setup_status[kMaxDevices];
+std::mutex g_lock;
+void* g_scratch[kMaxDevices];   // device address per device, NULL until a lookup succeeded
 
-// Device address of the scratch array on the current device; the first call
-// per device performs the lookup.
+// Device address of the scratch array on the current device. A failed lookup
+// is not cached: the next call tries again.
 cudaError_t scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_once[dev], [dev]() {
+  std::lock_guard<std::mutex> guard(g_lock);
+  if (g_scratch[dev] == nullptr) {
     void* p = nullptr;
-    g_setup_status[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess) return e;
     g_scratch[dev] = p;
-  });
-  if (g_setup_status[dev] != cudaSuccess) return g_setup_status[dev];
+  }
   *out = g_scratch[dev];
   return cudaSuccess;
 }
@@ -47,7 +48,9 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_params* p, con
                                                        const void* v, const float* alpha, const float* b,
                                                        const float* w, const float* S0, void* o, float* S_T,
                                                        void* stream) {
-  if (!p) return GDN2_ERR_INVALID_ARG;
+  // invalid parameters get the statuses of gdn2_chunk_fwd
+  const gdn2_status st = gdn2::check_chunk_params(p);
+  if (st != GDN2_OK) return st;
   if (p->cu_seqlens) return GDN2_ERR_UNSUPPORTED;   // packed sequences need every chunk's slot at once
   // Only the tensor-core prefill uses scratch; it is the configuration this
   // call serves (every other configuration runs without scratch through
@@ -60,4 +63,10 @@ extern "C" GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_params* p, con
   // chunk slot per sequence-head exceeds the array gets GDN2_ERR_WORKSPACE.
   return gdn2::chunk_fwd_checked(p, q, k, v, alpha, b, w, S0, o, S_T, scratch, kNoAllocScratchBytes, stream,
                                  /*segmented_ok=*/true);
+}
+
+extern "C" GDN2_API gdn2_status gdn2_chunk_fwd_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return GDN2_ERR_CUDA;
+  return gdn2::read_device_status(scratch, static_cast<cudaStream_t>(stream));
 }

@@ -12,6 +12,9 @@ Entry points mirror the C ABI:
 * :func:`decode_step` -> ``gdn2_decode_step`` (one recurrent step, state in place)
 * :func:`chunk_fwd_noalloc` -> ``gdn2_chunk_fwd_noalloc`` (prefill with the library's
   own fixed scratch, for callers that cannot allocate device memory)
+* :func:`chunk_fwd_status` -> ``gdn2_chunk_fwd_status`` (device status of the last
+  call on a workspace), :func:`chunk_fwd_noalloc_status` -> ``gdn2_chunk_fwd_noalloc_status``
+* :func:`debug_set_scan_stall` -> ``gdn2_debug_set_scan_stall`` (failure-path test hook)
 * :func:`status_str`, :func:`version`
 """
 
@@ -32,7 +35,8 @@ GATES = {"full": 0, "kda": 1, "gdn": 2}
 PRECISION = {"default": 0, "fp32": 1}
 
 EXPORTS = ("gdn2_status_str", "gdn2_version", "gdn2_chunk_fwd_workspace", "gdn2_chunk_fwd",
-           "gdn2_decode_step")
+           "gdn2_decode_step", "gdn2_chunk_fwd_status", "gdn2_debug_set_scan_stall",
+           "gdn2_chunk_fwd_noalloc", "gdn2_chunk_fwd_noalloc_status")
 
 
 class Params(ctypes.Structure):
@@ -77,6 +81,12 @@ def lib():
         L.gdn2_chunk_fwd.restype = ctypes.c_int
         L.gdn2_decode_step.argtypes = [pp] + [vp] * 9
         L.gdn2_decode_step.restype = ctypes.c_int
+        L.gdn2_chunk_fwd_status.argtypes = [vp, vp]
+        L.gdn2_chunk_fwd_status.restype = ctypes.c_int
+        L.gdn2_chunk_fwd_noalloc_status.argtypes = [vp]
+        L.gdn2_chunk_fwd_noalloc_status.restype = ctypes.c_int
+        L.gdn2_debug_set_scan_stall.argtypes = [ctypes.c_uint]
+        L.gdn2_debug_set_scan_stall.restype = None
         _lib = L
     return _lib
 
@@ -317,3 +327,20 @@ def chunk_fwd_noalloc(q, k, v, alpha, b, w=None, S0=None, *, o, S_T=None, chunk=
     if st != OK:
         raise GDN2Error(st, "gdn2_chunk_fwd_noalloc")
     return o, S_T
+
+
+def chunk_fwd_status(workspace, stream=None) -> int:
+    """Status code of the device-side waits of the last :func:`chunk_fwd` that
+    ran with ``workspace`` (OK or ERR_TIMEOUT); synchronises the stream first."""
+    return int(lib().gdn2_chunk_fwd_status(_ptr(workspace), _stream_handle(stream)))
+
+
+def chunk_fwd_noalloc_status(stream=None) -> int:
+    """Status code of the last :func:`chunk_fwd_noalloc` on the current device."""
+    return int(lib().gdn2_chunk_fwd_noalloc_status(_stream_handle(stream)))
+
+
+def debug_set_scan_stall(polls: int) -> None:
+    """Failure-path test hook: polls > 0 makes every later tensor-core prefill's
+    scan give up on a wait before it issues any product; 0 turns it off."""
+    lib().gdn2_debug_set_scan_stall(int(polls))

@@ -32,8 +32,13 @@
  *    kernel for). A launch failure returns GDN2_ERR_CUDA. Nothing is thrown
  *    across the ABI.
  *  - Preconditions NOT checked on the device: gates finite with α ∈ (0,1]
- *    for gdn2_chunk_fwd (α ∈ [0,1] for gdn2_decode_step), b, w ∈ [0,1];
- *    q, k of unit length unless l2norm_qk is set.
+ *    for gdn2_chunk_fwd (α ∈ [0,1] for gdn2_decode_step), b, w ∈ [0,1]
+ *    (as bf16 logits: any finite value); q, k of unit length unless
+ *    l2norm_qk is set. The tensor-core prefill (see gdn2_precision) takes
+ *    any such α, however strong the decay (chunks whose per-channel α
+ *    product over 16 tokens falls below 2^-64 run an exact fp32 kernel);
+ *    its 16-bit operands also need |v|, |w ⊙ v| and the state entries |S|
+ *    below 6·10^4 (fp16 range). Larger values need GDN2_PREC_FP32.
  *  - Output buffers must not alias inputs, except S0 == S_T (in place).
  *    conv_state_out never aliases conv_state_in.
  */
@@ -58,7 +63,8 @@ typedef enum {
   GDN2_ERR_UNSUPPORTED = 2,
   GDN2_ERR_WORKSPACE = 3,
   GDN2_ERR_CUDA = 4,
-  GDN2_ERR_TIMEOUT = 5 /* reserved: no kernel here waits on another block */
+  GDN2_ERR_TIMEOUT = 5 /* a bounded wait inside a tensor-core kernel gave up
+                          (reported by gdn2_chunk_fwd_status, not by the call) */
 } gdn2_status;
 
 typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
@@ -193,6 +199,29 @@ GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const v
                            const float* S0, void* o, float* S_T,
                            void* workspace, size_t ws_bytes, void* stream);
 
+/* Device status of the last gdn2_chunk_fwd call that ran with `workspace`.
+ *
+ * The tensor-core kernels wait on their own asynchronous work (tensor-core
+ * products, bulk copies, hand-overs between warps) with bounded waits. A
+ * wait that gives up makes its block skip the rest of its work, wait
+ * (bounded) for its copies in flight, release its tensor memory and set a
+ * status word at the start of the workspace; the call itself has already
+ * returned GDN2_OK by then. This query waits for the work enqueued on
+ * `stream` so far (cudaStreamSynchronize) and reads that word: GDN2_OK, or
+ * GDN2_ERR_TIMEOUT when a wait gave up (o and S_T of that call are then not
+ * valid). Each gdn2_chunk_fwd call clears the word before its launches.
+ * workspace = NULL (calls that ran the fp32 path, which needs none) gives
+ * GDN2_OK. Returns GDN2_ERR_CUDA if the copy or the synchronisation fails. */
+GDN2_API gdn2_status gdn2_chunk_fwd_status(const void* workspace, void* stream);
+
+/* Testing hook of the failure path above: with polls > 0, the scan kernel of
+ * every later tensor-core prefill in this process first waits, at most
+ * `polls` polls, on a barrier that nothing signals, before it issues any
+ * tensor-core product, so it gives up, drains its two slot copies, releases
+ * its tensor memory and sets the status word. 0 (the default) turns it off.
+ * The pages have no counterpart. Not for production use.                     */
+GDN2_API void gdn2_debug_set_scan_stall(unsigned polls);
+
 /* One recurrent decode step for B sequences (one token each), state in place.
  *
  * The fused recurrent schedule ("Uma análise das variantes de atenção linear
@@ -214,10 +243,11 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const
 
 /* Chunked prefill that allocates nothing: the same computation as
  * gdn2_chunk_fwd for the configurations that run the tensor-core kernel
- * (bf16 q,k,v, d_k = d_v = 128, chunk 64, no conv, no fused L2 norm,
- * GDN2_PREC_DEFAULT), with the kernel's device scratch taken from a fixed
- * 32 MiB array compiled into the library instead of a caller-provided
- * workspace. The pages have no counterpart of this call.
+ * (bf16 q,k,v, d_k = d_v = 128, chunk 64, GDN2_PREC_DEFAULT; with or without
+ * the conv and the fused L2 norm; not packed sequences), with the kernel's
+ * device scratch taken from a fixed 32 MiB array compiled into the library
+ * instead of a caller-provided workspace. The pages have no counterpart of
+ * this call.
  *
  * It exists for callers that cannot hand the library device memory at call
  * time: plugin hosts and serving runtimes that budget all device memory up
@@ -227,15 +257,20 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const
  * routine.
  *
  *   Arguments: as gdn2_chunk_fwd, without workspace and ws_bytes.
- *   Scratch:   one array per GPU, held from library load until process exit.
- *              The sequence is processed in segments of as many 64-token
- *              chunks as the array holds for all B·H_v sequence-heads (73 KB
- *              per chunk and sequence-head; 9 chunks for B·H_v = 48), so long
- *              sequences take more launches than gdn2_chunk_fwd. The first
- *              call on each device looks up the array's device address (with
- *              that device current); make that first call before any stream
- *              capture. Each call clears the status word it uses before its
- *              launches; nothing else in the array needs to start at zero.
+ *   Scratch:   one array per GPU. The first call on a device loads the
+ *              library's device code there, which reserves the array, and
+ *              looks up its device address (with that device current); the
+ *              array is then held until the process exits. Make that first
+ *              call at set-up time, before any stream capture: a budgeting
+ *              host sees the reservation then, and an out-of-memory error
+ *              surfaces there. The sequence is processed in segments of as
+ *              many 64-token chunks as the array holds for all B·H_v
+ *              sequence-heads (73 KB per chunk and sequence-head, plus, with
+ *              the conv or the L2 norm, the fp16 copies of the chunk's q, k, v
+ *              for all sequences: 9 chunks for B·H_v = 48 without them), so
+ *              long sequences take more launches than gdn2_chunk_fwd. Each
+ *              call clears the status word it uses before its launches;
+ *              nothing else in the array needs to start at zero.
  *   Sharing:   every call on a device uses the same array, so calls whose
  *              work overlaps on the GPU (different streams, no ordering
  *              between them) race; order them on one stream or by events.
@@ -243,12 +278,18 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const
  *              tensor-core kernel (call gdn2_chunk_fwd: they need no
  *              scratch); GDN2_ERR_WORKSPACE if even one chunk per
  *              sequence-head does not fit (B·H_v above about 440);
- *              GDN2_ERR_CUDA if the address lookup fails; otherwise exactly
- *              the statuses of gdn2_chunk_fwd.                              */
+ *              GDN2_ERR_CUDA if the address lookup fails (not remembered:
+ *              a later call tries again); otherwise exactly the statuses of
+ *              gdn2_chunk_fwd, invalid parameters included.               */
 GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_params* p, const void* q, const void* k,
                                             const void* v, const float* alpha, const float* b,
                                             const float* w, const float* S0, void* o, float* S_T,
                                             void* stream);
+
+/* gdn2_chunk_fwd_status for the last gdn2_chunk_fwd_noalloc call on the
+ * current device (its status word is the first word of the library's array):
+ * synchronises `stream` first. The pages have no counterpart.                */
+GDN2_API gdn2_status gdn2_chunk_fwd_noalloc_status(void* stream);
 
 #ifdef __cplusplus
 }

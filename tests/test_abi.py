@@ -198,3 +198,21 @@ def test_workspace_query_is_host_only(L):
     assert gdn2.chunk_fwd_workspace(_params(B=-1)) == 0
     # the precise path needs no workspace
     assert gdn2.chunk_fwd_workspace(_params(precision=1)) == 0
+
+
+def test_noalloc_validates_like_chunk_fwd(L):
+    """gdn2_chunk_fwd_noalloc runs the shared validation first: invalid
+    parameters get the statuses of gdn2_chunk_fwd (not UNSUPPORTED), before
+    any CUDA call, and the status queries refuse a misaligned workspace."""
+    fn = L.gdn2_chunk_fwd_noalloc
+    fn.argtypes = [ctypes.POINTER(gdn2.Params)] + [ctypes.c_void_p] * 10
+    fn.restype = ctypes.c_int
+    ptrs = [FAKE * (i + 1) for i in range(9)]
+    for kw, expect in ((dict(B=-1), gdn2.ERR_INVALID_ARG), (dict(H_qk=2, H_v=3), gdn2.ERR_INVALID_ARG),
+                       (dict(gate_mode=5), gdn2.ERR_INVALID_ARG), (dict(chunk=48), gdn2.ERR_UNSUPPORTED),
+                       (dict(d_k=24, d_v=24), gdn2.ERR_UNSUPPORTED)):
+        assert fn(ctypes.byref(_params(**kw)), *ptrs, None) == expect, kw
+    # valid, but the fp32 path needs no scratch
+    assert fn(ctypes.byref(_params()), *ptrs, None) == gdn2.ERR_UNSUPPORTED
+    assert L.gdn2_chunk_fwd_status(FAKE + 16, None) == gdn2.ERR_INVALID_ARG
+    assert L.gdn2_chunk_fwd_status(None, None) == gdn2.OK

@@ -128,12 +128,12 @@ def test_full_size_decode_b256():
     # step 1 on the whole tensor
     x = {k: np64(pool[k][0])[:, None] for k in ("q", "k", "v", "alpha", "b", "w")}
     o1_ref, S1_ref = oracle.gdn2_forward(x["q"], x["k"], x["v"], x["alpha"], x["b"], x["w"], S0)
-    assert_close(o1, o1_ref[:, 0], TOL_BF16, "o step 1")
+    assert_close(o1, o1_ref[:, 0], TOL_FP32, "o step 1")
     assert_close(S1, S1_ref, TOL_FP32, "S step 1")
     # every step on a subset of sequences
     idx = [t % 16 for t in range(steps)]
     xs = {k: np.stack([np64(pool[k][i])[seqs] for i in idx], axis=1) for k in ("q", "k", "v", "alpha", "b", "w")}
     o_ref, S_ref = oracle.gdn2_forward(xs["q"], xs["k"], xs["v"], xs["alpha"], xs["b"], xs["w"], S0[seqs])
     got = torch.stack(outs, 1)
-    assert_close(got, o_ref, TOL_BF16, f"o {steps} steps")
+    assert_close(got, o_ref, TOL_FP32, f"o {steps} steps")
     assert_close(S[seqs], S_ref, TOL_FP32, f"S {steps} steps")
