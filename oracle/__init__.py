@@ -27,6 +27,16 @@ Functions and the passages they follow:
   that a sequence split into calls (prefill pieces, decode steps) convolves
   exactly as one call over all its tokens (same page: the conv is causal
   over the token stream, which a split does not change).
+* :func:`gdn2_backward` -- the gradients of ``<dO, o> + <dS_T, S_T>`` with
+  respect to every input of :func:`gdn2_forward`: reverse-mode
+  differentiation of the same token loop, written out step by step in C++
+  (``gdn2_oracle_bwd.cpp``); "Resumo Técnico: Gated DeltaNet-2", Metodologia
+  §3, "Passagem de Retropropagação Consciente de Portões".
+* :func:`tied_gate_grads`, :func:`grads_for_qk_heads`, :func:`logit_grads` --
+  the chain rule through the tied gates, the gates shared per query/key head
+  and the sigmoid of gate logits (sums and products of the per-channel
+  gradients, the transposes of :func:`expand_tied_gates`,
+  :func:`gates_for_value_heads` and :func:`gates_from_logits`).
 * :func:`gates_from_logits` -- the gates as the sigmoid of their projections'
   outputs ("BigSaaS – Posts", section "Implementação Prática: Como Funciona a
   Camada de Atenção do DeltaNet-2": erase and write gates pass through a
@@ -46,6 +56,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gdn2_oracle.cpp")
+_SRC_BWD = os.path.join(_HERE, "gdn2_oracle_bwd.cpp")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
@@ -54,8 +65,9 @@ L2NORM_EPS = 1e-6
 
 def build(force: bool = False) -> str:
     """Compile the C++ oracle with g++ (plain -O2, IEEE double)."""
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
-        cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", _SRC, "-o", _LIB_PATH]
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_BWD))
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest:
+        cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", _SRC, _SRC_BWD, "-o", _LIB_PATH]
         subprocess.run(cmd, check=True)
     return _LIB_PATH
 
@@ -72,6 +84,8 @@ def _load():
         lib.oracle_causal_conv4.restype = ctypes.c_int
         lib.oracle_l2norm.argtypes = [ctypes.c_longlong, ctypes.c_int, ctypes.c_double, dp, dp]
         lib.oracle_l2norm.restype = ctypes.c_int
+        lib.oracle_gdn2_backward.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [dp] * 16 + [ctypes.c_int]
+        lib.oracle_gdn2_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -106,6 +120,60 @@ def gdn2_forward(q, k, v, alpha, b, w, S0=None, scale: float = 1.0, threads: int
     if rc != 0:
         raise ValueError("oracle_gdn2_forward rejected its arguments")
     return o, ST
+
+
+def gdn2_backward(q, k, v, alpha, b, w, S0, dO, dS_T=None, scale: float = 1.0, threads: int = 0):
+    """Gradients of L = <dO, o> + <dS_T, S_T> for the inputs of
+    :func:`gdn2_forward` (same shapes; per-channel gates per value head).
+    S0 and dS_T may be None (zeros). Returns a dict with keys q, k, v, alpha,
+    b, w, S0 (float64)."""
+    q, k, v, alpha, b, w, dO = (_f64(x) for x in (q, k, v, alpha, b, w, dO))
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    assert k.shape == q.shape and v.shape[:2] == (B, T) and dO.shape == v.shape
+    assert alpha.shape == (B, T, Hv, dk) and b.shape == (B, T, Hv, dk) and w.shape == (B, T, Hv, dv)
+    S0 = None if S0 is None else _f64(S0)
+    dS_T = None if dS_T is None else _f64(dS_T)
+    for s_ in (S0, dS_T):
+        assert s_ is None or s_.shape == (B, Hv, dk, dv)
+    g = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v), "alpha": np.zeros_like(alpha),
+         "b": np.zeros_like(b), "w": np.zeros_like(w), "S0": np.zeros((B, Hv, dk, dv))}
+    rc = _load().oracle_gdn2_backward(B, T, Hqk, Hv, dk, dv, float(scale), _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                                      _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["alpha"]), _ptr(g["b"]),
+                                      _ptr(g["w"]), _ptr(g["S0"]), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_gdn2_backward rejected its arguments")
+    return g
+
+
+def tied_gate_grads(mode: str, dalpha, db, dw):
+    """Chain rule through :func:`expand_tied_gates`: "kda" gives dβ = Σ_c db_c +
+    Σ_v dw_v (per token and head) and the per-channel dα; "gdn" also sums dα
+    over the channels. Returns (dalpha, dbeta)."""
+    dalpha, db, dw = _f64(dalpha), _f64(db), _f64(dw)
+    dbeta = db.sum(axis=-1) + dw.sum(axis=-1)
+    if mode == "gdn":
+        dalpha = dalpha.sum(axis=-1)
+    elif mode != "kda":
+        raise ValueError(mode)
+    return dalpha, dbeta
+
+
+def grads_for_qk_heads(g, H_qk: int, axis: int = 2):
+    """Chain rule through :func:`gates_for_value_heads`: the gradient of a gate
+    shared by the value heads of a query/key head is the sum over those heads."""
+    g = _f64(g)
+    H_v = g.shape[axis]
+    assert H_v % H_qk == 0
+    shape = g.shape[:axis] + (H_qk, H_v // H_qk) + g.shape[axis + 1:]
+    return g.reshape(shape).sum(axis=axis + 1)
+
+
+def logit_grads(dgate, x):
+    """Chain rule through :func:`gates_from_logits`: dL/dx = dL/dσ · σ(x)(1 − σ(x))."""
+    s = gates_from_logits(x)
+    return _f64(dgate) * s * (1.0 - s)
 
 
 def expand_tied_gates(mode: str, alpha, beta, d_k: int, d_v: int):
