@@ -250,6 +250,72 @@ gdn2_status gdn2_chunk_fwd_status(const void* workspace, void* stream) {
 
 void gdn2_debug_set_scan_stall(unsigned polls) { g_scan_stall.store(polls, std::memory_order_relaxed); }
 
+size_t gdn2_chunk_bwd_workspace(const gdn2_params* p) {
+  if (check_chunk_params(p) != GDN2_OK || p->conv_w || p->l2norm_qk || p->cu_seqlens) return 0;
+  return chunk_bwd_workspace(p->B, p->H_v, p->T, p->d_k);
+}
+
+gdn2_status gdn2_chunk_bwd(const gdn2_params* p, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* b, const float* w, const float* S0, const void* dO,
+                           const float* dS_T, float* dq, float* dk, float* dv, float* dalpha, float* db, float* dw,
+                           float* dS0, void* workspace, size_t ws_bytes, void* stream) {
+  gdn2_status st = check_chunk_params(p);
+  if (st != GDN2_OK) return st;
+  // the fused conv / L2 norm and packed sequences have no backward here
+  if (p->conv_w || p->l2norm_qk || p->cu_seqlens || p->conv_state_in || p->conv_state_out)
+    return GDN2_ERR_UNSUPPORTED;
+  const size_t tokens = (size_t)p->B * p->T;
+  const bool full = p->gate_mode == GDN2_GATES_FULL;
+  if (tokens > 0) {
+    if (!q || !k || !v || !dO || !dq || !dk || !dv || !dalpha || !db) return GDN2_ERR_INVALID_ARG;
+    if ((st = check_gate_ptrs(p, alpha, b, w)) != GDN2_OK) return st;
+    if (full ? dw == nullptr : dw != nullptr) return GDN2_ERR_INVALID_ARG;
+  }
+  const void* ptrs[] = {q, k, v, alpha, b, w, S0, dO, dS_T, dq, dk, dv, dalpha, db, dw, dS0, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return GDN2_ERR_INVALID_ARG;
+  const Sizes sz = sizes(p, tokens);
+  const size_t do_bytes = tokens * p->H_v * p->d_v * dsize(p->o_dtype);
+  const size_t f32 = sizeof(float);
+  const size_t ga32 = sz.ga / (p->gate_logits ? 2 : 4) * f32, gb32 = sz.gb / (p->gate_logits ? 2 : 4) * f32,
+               gw32 = sz.gw / (p->gate_logits ? 2 : 4) * f32;
+  const size_t qk32 = tokens * p->H_qk * p->d_k * f32, v32 = tokens * p->H_v * p->d_v * f32;
+  const Range ins[] = {{q, sz.qk}, {k, sz.qk}, {v, sz.v}, {alpha, sz.ga}, {b, sz.gb}, {w, sz.gw},
+                       {S0, sz.st}, {dO, do_bytes}, {dS_T, sz.st}};
+  const Range outs[] = {{dq, qk32}, {dk, qk32}, {dv, v32}, {dalpha, ga32}, {db, gb32}, {dw, gw32}, {dS0, sz.st},
+                        {workspace, ws_bytes}};
+  for (int i = 0; i < 8; ++i) {
+    for (const Range& r : ins)
+      if (overlaps(outs[i].p, outs[i].n, r.p, r.n)) return GDN2_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j)
+      if (overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return GDN2_ERR_INVALID_ARG;
+  }
+  const size_t need = chunk_bwd_workspace(p->B, p->H_v, p->T, p->d_k);
+  if (tokens > 0 && (workspace == nullptr || ws_bytes < need)) return GDN2_ERR_WORKSPACE;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (p->B > 0 && p->T == 0 && dS0) {
+    // no token: S_T = S0, so dS0 = dS_T
+    e = dS_T ? cudaMemcpyAsync(dS0, dS_T, sz.st, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(dS0, 0, sz.st, s);
+    return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+  }
+  if (tokens == 0) return GDN2_OK;
+  // the key-side and gate gradients are sums over CTAs (atomics)
+  for (const Range& r : {Range{dq, qk32}, Range{dk, qk32}, Range{dalpha, ga32}, Range{db, gb32}})
+    if (e == cudaSuccess) e = cudaMemsetAsync(const_cast<void*>(r.p), 0, r.n, s);
+  if (e != cudaSuccess) return GDN2_ERR_CUDA;
+  BwdArgs a;
+  a.B = p->B; a.T = p->T; a.Hqk = p->H_qk; a.Hv = p->H_v;
+  a.Hg = p->gate_heads == GDN2_GATE_HEADS_QK ? p->H_qk : p->H_v;
+  a.gate_mode = p->gate_mode; a.gate_logits = p->gate_logits; a.scale = p->scale;
+  a.q = q; a.k = k; a.v = v; a.dO = dO; a.alpha = alpha; a.b = b; a.w = w; a.S0 = S0; a.dST = dS_T;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dalpha = dalpha; a.db = db; a.dw = dw; a.dS0 = dS0;
+  a.ckpt = static_cast<float*>(workspace);
+  e = launch_chunk_bwd(a, p->d_k, p->qkv_dtype == GDN2_BF16, p->o_dtype == GDN2_BF16, s);
+  return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
 gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const void* k, const void* v,
                              const float* alpha, const float* b, const float* w, float* S, void* o,
                              void* stream) {

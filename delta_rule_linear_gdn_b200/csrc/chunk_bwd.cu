@@ -1,0 +1,529 @@
+// Backward pass of the chunked prefill, exact fp32 SIMT arithmetic.
+//
+// Gradients of L = <dO, o> + <dS_T, S_T> for the recurrence ("Resumo Técnico:
+// Gated DeltaNet-2", Metodologia §1) with respect to q, k, v, the gates and S0,
+// in the chunked form of the forward ("Uma análise das variantes de atenção
+// linear da família DeltaNet", "Chunkwise KDA"; the decoupled gates of the
+// GDN-2 summary, Metodologia §3, whose backward pass carries the per-channel
+// erase and write gates through the gradients of the WY factors). Per chunk
+// of C tokens with entry state S, cumulative decays γ_i = Π_{s≤i} α_s, and the
+// pairwise decay D_ij = Π_{j<s≤i} α_s (per key channel):
+//     T_ij = Σ_c e_ic k_jc D_ijc (j < i),  Aqk_ij = Σ_c q_ic k_jc D_ijc (j ≤ i)
+//     A = (I + T)⁻¹,  R = Z − Ē S,  U = A R,  O = s (Q̄ S + Aqk U),
+//     S' = Γ S + K_endᵀ U,  Ē = γ ⊙ e, Q̄ = γ ⊙ q, K_end,j = k_j ⊙ Π_{j<s≤C} α_s.
+// Going back through the chunk with dO and dS' (the gradient of S'):
+//     dU = s Aqkᵀ dO + K_end dS',   dR = Aᵀ dU  (= dZ),
+//     dS = s Q̄ᵀ dO + Γ dS' − Ēᵀ dR  (carried to the previous chunk),
+//     dT_ij = −Σ_v dR_iv U_jv (j < i),   dAqk_ij = s Σ_v dO_iv U_jv (j ≤ i),
+//     dQ̄ = s dO Sᵀ,  dĒ = −dR Sᵀ,  dK_end = U dS'ᵀ,  dΓ_c = Σ_v dS'_cv S_cv,
+// then through the decays in log space (G_i = Σ_{s≤i} log α_s): every factor
+// is exp of a difference of G, so its gradient lands on the G of both ends,
+// and dlog α_s = Σ_{i≥s} dG_i. The Gram gradients use the running products
+// of α (no reciprocal, no logarithm), as the forward's exact kernel does, so
+// every α ∈ (0, 1] is taken.
+//
+// One CTA per (sequence, value head, tile of DVT value columns): the state's
+// columns evolve independently, so each CTA first runs the forward over all
+// chunks, writing its columns of each chunk's entry state to a checkpoint
+// buffer, then walks the chunks in reverse carrying its columns of dS. The
+// gradients of v and w are per column and written once; those of q, k, α and
+// b are sums over all columns (and over the value heads of a query/key head)
+// and are added with atomics into buffers the launcher zeroes.
+
+#include "common.cuh"
+
+namespace gdn2 {
+namespace {
+
+constexpr int BC = 16;        // chunk of the backward pass
+constexpr int BT = 256;       // threads
+
+template <int D>
+struct BwdSmem {
+  static constexpr int DVT = D < 64 ? D : 64;   // value columns per CTA
+  static constexpr int DP = D + 1;              // row strides (padded against bank conflicts)
+  static constexpr int CP = BC + 1;
+  static constexpr int VP = DVT + 1;
+  // [BC][DP] ×11: q, k, b, α, e, γ, bk (Π_{i<s<BC} α), and the gradients of q, k, e, G
+  // [BC][CP] ×5:  T, A = (I+T)⁻¹, Aqk, dT, dAqk
+  // [BC][VP] ×6:  Z (then R, then dR), U, dO, dU, v, w
+  // [D][VP] ×3:   S, dS', dS
+  // [D]:          γ_C
+  static constexpr size_t floats = 11 * BC * DP + 5 * BC * CP + 6 * BC * VP + 3 * D * VP + D;
+  static constexpr size_t bytes = floats * sizeof(float);
+};
+static_assert(BwdSmem<128>::bytes <= 232448, "backward shared memory");
+
+template <int D, typename TIn, typename TdO>
+__global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
+  using L = BwdSmem<D>;
+  constexpr int DVT = L::DVT, DP = L::DP, CP = L::CP, VP = L::VP;
+  constexpr int TILES = D / DVT;
+  constexpr int CPT = D / 16;   // channels per thread of the pairwise passes
+  extern __shared__ float sm[];
+  float* sQ = sm;
+  float* sK = sQ + BC * DP;
+  float* sB = sK + BC * DP;
+  float* sAl = sB + BC * DP;
+  float* sE = sAl + BC * DP;
+  float* sGm = sE + BC * DP;
+  float* sBk = sGm + BC * DP;
+  float* gQ = sBk + BC * DP;
+  float* gK = gQ + BC * DP;
+  float* gE = gK + BC * DP;
+  float* gG = gE + BC * DP;
+  float* sT = gG + BC * DP;
+  float* sA = sT + BC * CP;
+  float* sAq = sA + BC * CP;
+  float* sdT = sAq + BC * CP;
+  float* sdAq = sdT + BC * CP;
+  float* tZ = sdAq + BC * CP;
+  float* tU = tZ + BC * VP;
+  float* tdO = tU + BC * VP;
+  float* tdU = tdO + BC * VP;
+  float* tV = tdU + BC * VP;
+  float* tW = tV + BC * VP;
+  float* sS = tW + BC * VP;
+  float* sdS = sS + D * VP;
+  float* sdSn = sdS + D * VP;
+  float* sgC = sdSn + D * VP;
+
+  const int tile = blockIdx.x % TILES, bh = blockIdx.x / TILES;
+  const int h = bh % a.Hv, bi = bh / a.Hv;
+  const int hq = h / (a.Hv / a.Hqk);
+  const int hg = a.Hg == a.Hv ? h : hq;
+  const int col0 = tile * DVT;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool full = a.gate_mode == GDN2_GATES_FULL, alpha_pc = a.gate_mode != GDN2_GATES_GDN;
+  const bool lg = a.gate_logits != 0;
+  const int T = a.T, N = (T + BC - 1) / BC;
+  const float s = a.scale;
+  const TIn* qg = static_cast<const TIn*>(a.q);
+  const TIn* kg = static_cast<const TIn*>(a.k);
+  const TIn* vg = static_cast<const TIn*>(a.v);
+  const TdO* og = static_cast<const TdO*>(a.dO);
+  float* ckpt = a.ckpt + (size_t)bh * N * D * D;   // [N][D][D]; this CTA owns columns col0 ..
+
+  // ---- one chunk's inputs: key side [BC][D], value side of the tile [BC][DVT]
+  auto load_chunk = [&](int c, bool grads) {
+    const int t0 = c * BC, Lc = min(BC, T - t0);
+    for (int idx = tid; idx < BC * D; idx += BT) {
+      const int i = idx / D, cc = idx % D;
+      float q = 0.f, k = 0.f, al = 1.f, bb = 0.f;
+      if (i < Lc) {
+        const size_t t = (size_t)bi * T + t0 + i;
+        const size_t qk = (t * a.Hqk + hq) * D + cc;
+        q = to_f32(qg[qk]);
+        k = to_f32(kg[qk]);
+        const size_t gr = t * a.Hg + hg;
+        al = gate_at(a.alpha, alpha_pc ? gr * D + cc : gr, lg);
+        bb = gate_at(a.b, full ? gr * D + cc : gr, lg);
+      }
+      sQ[i * DP + cc] = q;
+      sK[i * DP + cc] = k;
+      sAl[i * DP + cc] = al;
+      sB[i * DP + cc] = bb;
+      sE[i * DP + cc] = bb * k;
+    }
+    for (int idx = tid; idx < BC * DVT; idx += BT) {
+      const int i = idx / DVT, v = idx % DVT;
+      float vv = 0.f, ww = 0.f, d = 0.f;
+      if (i < Lc) {
+        const size_t t = (size_t)bi * T + t0 + i;
+        const size_t vi = (t * a.Hv + h) * D + col0 + v;
+        vv = to_f32(vg[vi]);
+        ww = full ? gate_at(a.w, vi, lg) : gate_at(a.b, t * a.Hg + hg, lg);
+        if (grads) d = to_f32(og[vi]);
+      }
+      tV[i * VP + v] = vv;
+      tW[i * VP + v] = ww;
+      tZ[i * VP + v] = ww * vv;
+      tdO[i * VP + v] = d;
+    }
+  };
+
+  // ---- γ (forward products), bk (backward products), γ_C; then T, Aqk by
+  // running products per (column j, 16-channel part). Warp w owns columns
+  // 2w, 2w + 1 and runs its rows from 2w.
+  auto decays_and_gram = [&]() {
+    if (tid < D) {
+      const int c = tid;
+      float g = 1.f;
+      for (int i = 0; i < BC; ++i) {
+        g *= sAl[i * DP + c];
+        sGm[i * DP + c] = g;
+      }
+      sgC[c] = g;
+      float p = 1.f;
+      for (int i = BC - 1; i >= 0; --i) {
+        sBk[i * DP + c] = p;
+        p *= sAl[i * DP + c];
+      }
+    }
+    const int j = tid >> 4, part = tid & 15;
+    float kj[CPT], dd[CPT];
+#pragma unroll
+    for (int m = 0; m < CPT; ++m) {
+      kj[m] = sK[j * DP + part + 16 * m];
+      dd[m] = 1.f;
+    }
+    for (int i = warp * 2; i < BC; ++i) {
+      float at = 0.f, aa = 0.f;
+#pragma unroll
+      for (int m = 0; m < CPT; ++m) {
+        const int c = part + 16 * m;
+        dd[m] *= i > j ? sAl[i * DP + c] : 1.f;
+        const float kd = kj[m] * dd[m];
+        at = fmaf(sE[i * DP + c], kd, at);
+        aa = fmaf(sQ[i * DP + c], kd, aa);
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        at += __shfl_xor_sync(0xffffffffu, at, off);
+        aa += __shfl_xor_sync(0xffffffffu, aa, off);
+      }
+      if (part == 0 && i >= j) {
+        sT[i * CP + j] = i > j ? at : 0.f;
+        sAq[i * CP + j] = aa;
+      }
+    }
+  };
+
+  // A = (I + T)⁻¹ by forward substitution, one column per thread; R = Z − Ē S.
+  auto inverse_and_R = [&]() {
+    if (tid < BC) {
+      const int j = tid;
+      for (int i = 0; i < BC; ++i) {
+        float x = i == j ? 1.f : 0.f;
+        if (i > j) {
+          float acc = 0.f;
+          for (int l = j; l < i; ++l) acc = fmaf(sT[i * CP + l], sA[l * CP + j], acc);
+          x = -acc;
+        }
+        sA[i * CP + j] = x;
+      }
+    }
+    for (int idx = tid; idx < BC * DVT; idx += BT) {
+      const int i = idx / DVT, v = idx % DVT;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) acc = fmaf(sGm[i * DP + c] * sE[i * DP + c], sS[c * VP + v], acc);
+      tZ[i * VP + v] -= acc;
+    }
+  };
+  // U = A R
+  auto solve_U = [&]() {
+    for (int idx = tid; idx < BC * DVT; idx += BT) {
+      const int i = idx / DVT, v = idx % DVT;
+      float acc = 0.f;
+      for (int j = 0; j <= i; ++j) acc = fmaf(sA[i * CP + j], tZ[j * VP + v], acc);
+      tU[i * VP + v] = acc;
+    }
+  };
+
+  // ------------------------------------------------------------------ forward
+  for (int idx = tid; idx < D * DVT; idx += BT) {
+    const int r = idx / DVT, v = idx % DVT;
+    sS[r * VP + v] = a.S0 ? a.S0[((size_t)bh * D + r) * D + col0 + v] : 0.f;
+  }
+  for (int c = 0; c < N; ++c) {
+    __syncthreads();
+    for (int idx = tid; idx < D * DVT; idx += BT) {
+      const int r = idx / DVT, v = idx % DVT;
+      ckpt[((size_t)c * D + r) * D + col0 + v] = sS[r * VP + v];
+    }
+    load_chunk(c, false);
+    __syncthreads();
+    decays_and_gram();
+    __syncthreads();
+    inverse_and_R();
+    __syncthreads();
+    solve_U();
+    __syncthreads();
+    // S ← Γ S + K_endᵀ U
+    for (int idx = tid; idx < D * DVT; idx += BT) {
+      const int r = idx / DVT, v = idx % DVT;
+      float acc = sgC[r] * sS[r * VP + v];
+      for (int j = 0; j < BC; ++j) acc = fmaf(sK[j * DP + r] * sBk[j * DP + r], tU[j * VP + v], acc);
+      sS[r * VP + v] = acc;
+    }
+  }
+
+  // ------------------------------------------------------------------ backward
+  float* dSp = sdS;     // dS' (gradient of the chunk's exit state)
+  float* dSn = sdSn;    // dS of its entry state
+  __syncthreads();
+  for (int idx = tid; idx < D * DVT; idx += BT) {
+    const int r = idx / DVT, v = idx % DVT;
+    dSp[r * VP + v] = a.dST ? a.dST[((size_t)bh * D + r) * D + col0 + v] : 0.f;
+  }
+  for (int c = N - 1; c >= 0; --c) {
+    const int t0 = c * BC, Lc = min(BC, T - t0);
+    __syncthreads();
+    for (int idx = tid; idx < D * DVT; idx += BT) {
+      const int r = idx / DVT, v = idx % DVT;
+      sS[r * VP + v] = ckpt[((size_t)c * D + r) * D + col0 + v];
+    }
+    load_chunk(c, true);
+    __syncthreads();
+    decays_and_gram();
+    __syncthreads();
+    inverse_and_R();
+    __syncthreads();
+    solve_U();
+    __syncthreads();
+    // dU = s Aqkᵀ dO + K_end dS'
+    for (int idx = tid; idx < BC * DVT; idx += BT) {
+      const int j = idx / DVT, v = idx % DVT;
+      float acc = 0.f;
+      for (int i = j; i < BC; ++i) acc = fmaf(sAq[i * CP + j], tdO[i * VP + v], acc);
+      acc *= s;
+#pragma unroll 8
+      for (int cc = 0; cc < D; ++cc) acc = fmaf(sK[j * DP + cc] * sBk[j * DP + cc], dSp[cc * VP + v], acc);
+      tdU[j * VP + v] = acc;
+    }
+    __syncthreads();
+    // dR = Aᵀ dU, into the R array
+    for (int idx = tid; idx < BC * DVT; idx += BT) {
+      const int i = idx / DVT, v = idx % DVT;
+      float acc = 0.f;
+      for (int j = i; j < BC; ++j) acc = fmaf(sA[j * CP + i], tdU[j * VP + v], acc);
+      tZ[i * VP + v] = acc;
+    }
+    __syncthreads();
+    float* tdR = tZ;
+    // dS of the entry state
+    for (int idx = tid; idx < D * DVT; idx += BT) {
+      const int r = idx / DVT, v = idx % DVT;
+      float acc = 0.f;
+      for (int i = 0; i < BC; ++i)
+        acc = fmaf(sGm[i * DP + r], fmaf(s * sQ[i * DP + r], tdO[i * VP + v], -sE[i * DP + r] * tdR[i * VP + v]),
+                   acc);
+      dSn[r * VP + v] = fmaf(sgC[r], dSp[r * VP + v], acc);
+    }
+    // dv = dR ⊙ w; dw = dR ⊙ v (per channel), or its sum into dβ (tied gates)
+    for (int idx = tid; idx < BC * DVT; idx += BT) {
+      const int i = idx / DVT, v = idx % DVT;
+      if (i >= Lc) continue;
+      const size_t t = (size_t)bi * T + t0 + i;
+      const size_t vi = (t * a.Hv + h) * D + col0 + v;
+      const float dr = tdR[i * VP + v], ww = tW[i * VP + v];
+      a.dv[vi] = dr * ww;
+      if (full) a.dw[vi] = dr * tV[i * VP + v] * (lg ? ww * (1.f - ww) : 1.f);
+    }
+    if (!full) {
+      // Σ_v dR ⊙ v per token, one warp per token
+      for (int i = warp; i < Lc; i += BT / 32) {
+        float acc = 0.f;
+        for (int v = lane; v < DVT; v += 32) acc = fmaf(tdR[i * VP + v], tV[i * VP + v], acc);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+          const float beta = tW[i * VP];
+          atomicAdd(a.db + ((size_t)bi * T + t0 + i) * a.Hg + hg, acc * (lg ? beta * (1.f - beta) : 1.f));
+        }
+      }
+    }
+    // dT, dAqk
+    {
+      const int i = tid >> 4, j = tid & 15;
+      float x = 0.f, y = 0.f;
+      if (j <= i) {
+        for (int v = 0; v < DVT; ++v) {
+          const float u = tU[j * VP + v];
+          x = fmaf(tdR[i * VP + v], u, x);
+          y = fmaf(tdO[i * VP + v], u, y);
+        }
+      }
+      sdT[i * CP + j] = j < i ? -x : 0.f;
+      sdAq[i * CP + j] = j <= i ? s * y : 0.f;
+    }
+    // per (i, c): dQ̄ = s dO Sᵀ, dĒ = −dR Sᵀ, dK_end = U dS'ᵀ, and what they give
+    // q, e, k and G directly
+    for (int idx = tid; idx < BC * D; idx += BT) {
+      const int i = idx / D, cc = idx % D;
+      float dq_ = 0.f, de_ = 0.f, dke = 0.f;
+#pragma unroll 8
+      for (int v = 0; v < DVT; ++v) {
+        const float sv = sS[cc * VP + v];
+        dq_ = fmaf(tdO[i * VP + v], sv, dq_);
+        de_ = fmaf(tdR[i * VP + v], sv, de_);
+        dke = fmaf(tU[i * VP + v], dSp[cc * VP + v], dke);
+      }
+      dq_ *= s;
+      de_ = -de_;
+      const float g = sGm[i * DP + cc], bk = sBk[i * DP + cc];
+      gQ[i * DP + cc] = g * dq_;
+      gE[i * DP + cc] = g * de_;
+      gK[i * DP + cc] = bk * dke;
+      gG[i * DP + cc] = g * (sQ[i * DP + cc] * dq_ + sE[i * DP + cc] * de_) - sK[i * DP + cc] * bk * dke;
+    }
+    __syncthreads();
+    // G at the chunk's last token: from K_end (Σ_j K_end,j ⊙ dK_end,j) and Γ
+    if (tid < D) {
+      const int cc = tid;
+      float acc = 0.f;
+      for (int j = 0; j < BC; ++j) acc = fmaf(sK[j * DP + cc], gK[j * DP + cc], acc);
+      float dg = 0.f;
+      for (int v = 0; v < DVT; ++v) dg = fmaf(dSp[cc * VP + v], sS[cc * VP + v], dg);
+      gG[(BC - 1) * DP + cc] += fmaf(sgC[cc], dg, acc);
+    }
+    __syncthreads();
+    // Gram gradients, key side: thread (j, part) runs i up from j with D_ij
+    {
+      const int j = tid >> 4, part = tid & 15;
+      float dd[CPT], ak[CPT], ag[CPT], kj[CPT];
+#pragma unroll
+      for (int m = 0; m < CPT; ++m) {
+        dd[m] = 1.f;
+        ak[m] = 0.f;
+        ag[m] = 0.f;
+        kj[m] = sK[j * DP + part + 16 * m];
+      }
+      for (int i = j; i < BC; ++i) {
+        const float ct = sdT[i * CP + j], ca = sdAq[i * CP + j];
+#pragma unroll
+        for (int m = 0; m < CPT; ++m) {
+          const int cc = part + 16 * m;
+          dd[m] *= i > j ? sAl[i * DP + cc] : 1.f;
+          const float x = fmaf(ct, sE[i * DP + cc], ca * sQ[i * DP + cc]) * dd[m];
+          ak[m] += x;
+          ag[m] = fmaf(x, kj[m], ag[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < CPT; ++m) {
+        const int cc = part + 16 * m;
+        gK[j * DP + cc] += ak[m];
+        gG[j * DP + cc] -= ag[m];
+      }
+    }
+    __syncthreads();
+    // query / erase side: thread (i, part) runs j down from i with D_ij
+    {
+      const int i = tid >> 4, part = tid & 15;
+      float dd[CPT], ae[CPT], aq[CPT], ag[CPT];
+#pragma unroll
+      for (int m = 0; m < CPT; ++m) {
+        dd[m] = 1.f;
+        ae[m] = 0.f;
+        aq[m] = 0.f;
+        ag[m] = 0.f;
+      }
+      for (int j = i; j >= 0; --j) {
+        const float ct = sdT[i * CP + j], ca = sdAq[i * CP + j];
+#pragma unroll
+        for (int m = 0; m < CPT; ++m) {
+          const int cc = part + 16 * m;
+          if (j < i) dd[m] *= sAl[(j + 1) * DP + cc];
+          const float kd = sK[j * DP + cc] * dd[m];
+          ae[m] = fmaf(ct, kd, ae[m]);
+          aq[m] = fmaf(ca, kd, aq[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < CPT; ++m) {
+        const int cc = part + 16 * m;
+        ag[m] = fmaf(ae[m], sE[i * DP + cc], aq[m] * sQ[i * DP + cc]);
+        gE[i * DP + cc] += ae[m];
+        gQ[i * DP + cc] += aq[m];
+        gG[i * DP + cc] += ag[m];
+      }
+    }
+    __syncthreads();
+    // dlog α_s = Σ_{i≥s} dG_i per channel (into gG)
+    if (tid < D) {
+      const int cc = tid;
+      float acc = 0.f;
+      for (int i = BC - 1; i >= 0; --i) {
+        acc += gG[i * DP + cc];
+        gG[i * DP + cc] = acc;
+      }
+    }
+    __syncthreads();
+    // gradients of this tile's columns into q, k, α, b (per channel) by
+    // atomics; scalar gates (tied β, scalar α) as per-token sums
+    for (int i = warp; i < Lc; i += BT / 32) {
+      const size_t t = (size_t)bi * T + t0 + i;
+      const size_t qk = (t * a.Hqk + hq) * D;
+      const size_t gr = t * a.Hg + hg;
+      float sa = 0.f, sb = 0.f;
+      for (int cc = lane; cc < D; cc += 32) {
+        const float k = sK[i * DP + cc], ge = gE[i * DP + cc], al = sAl[i * DP + cc], bb = sB[i * DP + cc];
+        atomicAdd(a.dq + qk + cc, gQ[i * DP + cc]);
+        atomicAdd(a.dk + qk + cc, fmaf(ge, bb, gK[i * DP + cc]));
+        const float dlog = gG[i * DP + cc];
+        const float da = lg ? dlog * (1.f - al) : dlog / al;   // d/dα of log α = 1/α; d/dx of log σ(x) = 1 − σ
+        const float db_ = ge * k;
+        if (alpha_pc) atomicAdd(a.dalpha + gr * D + cc, da);
+        else sa += dlog;
+        if (full) atomicAdd(a.db + gr * D + cc, db_ * (lg ? bb * (1.f - bb) : 1.f));
+        else sb += db_;
+      }
+      if (!alpha_pc || !full) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          sa += __shfl_xor_sync(0xffffffffu, sa, off);
+          sb += __shfl_xor_sync(0xffffffffu, sb, off);
+        }
+        if (lane == 0) {
+          if (!alpha_pc) {
+            const float al = sAl[i * DP];
+            atomicAdd(a.dalpha + gr, lg ? sa * (1.f - al) : sa / al);
+          }
+          if (!full) {
+            const float beta = sB[i * DP];
+            atomicAdd(a.db + gr, sb * (lg ? beta * (1.f - beta) : 1.f));
+          }
+        }
+      }
+    }
+    float* tmp = dSp;
+    dSp = dSn;
+    dSn = tmp;
+  }
+  __syncthreads();
+  if (a.dS0) {
+    for (int idx = tid; idx < D * DVT; idx += BT) {
+      const int r = idx / DVT, v = idx % DVT;
+      a.dS0[((size_t)bh * D + r) * D + col0 + v] = dSp[r * VP + v];
+    }
+  }
+}
+
+template <int D, typename TIn, typename TdO>
+cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
+  using L = BwdSmem<D>;
+  const int grid = a.B * a.Hv * (D / L::DVT);
+  if (grid == 0) return cudaSuccess;
+  auto kfn = chunk_bwd_kernel<D, TIn, TdO>;
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
+  if (e != cudaSuccess) return e;
+  kfn<<<grid, BT, L::bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename TIn, typename TdO>
+cudaError_t launch_bwd_d(const BwdArgs& a, int d, cudaStream_t st) {
+  switch (d) {
+    case 16: return launch_bwd_t<16, TIn, TdO>(a, st);
+    case 32: return launch_bwd_t<32, TIn, TdO>(a, st);
+    case 64: return launch_bwd_t<64, TIn, TdO>(a, st);
+    case 128: return launch_bwd_t<128, TIn, TdO>(a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+size_t chunk_bwd_workspace(int n_states, int H_v, int T, int d) {
+  return (size_t)n_states * H_v * (size_t)((T + BC - 1) / BC) * d * d * sizeof(float);
+}
+
+cudaError_t launch_chunk_bwd(const BwdArgs& a, int d, int qkv_bf16, int do_bf16, cudaStream_t st) {
+  if (qkv_bf16)
+    return do_bf16 ? launch_bwd_d<__nv_bfloat16, __nv_bfloat16>(a, d, st) : launch_bwd_d<__nv_bfloat16, float>(a, d, st);
+  return do_bf16 ? launch_bwd_d<float, __nv_bfloat16>(a, d, st) : launch_bwd_d<float, float>(a, d, st);
+}
+
+}  // namespace gdn2

@@ -98,6 +98,16 @@ struct DecodeArgs {
   int Hg;                // heads of alpha and b (Hv, or Hqk when shared per QK head)
 };
 
+// Arguments of the backward pass (gdn2_chunk_bwd), validated on the host.
+struct BwdArgs {
+  int B, T, Hqk, Hv, Hg, gate_mode, gate_logits;
+  float scale;
+  const void *q, *k, *v, *dO;          // q, k, v in the input dtype; dO in the output dtype
+  const float *alpha, *b, *w, *S0, *dST;
+  float *dq, *dk, *dv, *dalpha, *db, *dw, *dS0;
+  float* ckpt;                         // workspace: every chunk's entry state
+};
+
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_decode(const DecodeArgs& a, int qkv_bf16, int o_bf16, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, int qkv_bf16, int o_bf16, cudaStream_t s);
@@ -111,6 +121,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s);
 // Writes a.conv_out: the three pre-conv inputs that end at token T−1 of each
 // sequence (history from a.conv_in shifted in when T < 3).
 cudaError_t launch_conv_state(const ChunkArgs& a, int qkv_bf16, cudaStream_t s);
+
+// Backward pass: workspace bytes and launcher.
+size_t chunk_bwd_workspace(int n_states, int H_v, int T, int d);
+cudaError_t launch_chunk_bwd(const BwdArgs& a, int d, int qkv_bf16, int do_bf16, cudaStream_t s);
 
 // Shape, enum and offset checks shared by the prefill entry points.
 gdn2_status check_chunk_params(const gdn2_params* p);

@@ -12,6 +12,8 @@ Entry points mirror the C ABI:
 * :func:`decode_step` -> ``gdn2_decode_step`` (one recurrent step, state in place)
 * :func:`chunk_fwd_noalloc` -> ``gdn2_chunk_fwd_noalloc`` (prefill with the library's
   own fixed scratch, for callers that cannot allocate device memory)
+* :func:`chunk_bwd` -> ``gdn2_chunk_bwd`` (gradients of the prefill), with
+  :func:`chunk_bwd_workspace` -> ``gdn2_chunk_bwd_workspace``
 * :func:`chunk_fwd_status` -> ``gdn2_chunk_fwd_status`` (device status of the last
   call on a workspace), :func:`chunk_fwd_noalloc_status` -> ``gdn2_chunk_fwd_noalloc_status``
 * :func:`debug_set_scan_stall` -> ``gdn2_debug_set_scan_stall`` (failure-path test hook)
@@ -36,7 +38,8 @@ PRECISION = {"default": 0, "fp32": 1}
 
 EXPORTS = ("gdn2_status_str", "gdn2_version", "gdn2_chunk_fwd_workspace", "gdn2_chunk_fwd",
            "gdn2_decode_step", "gdn2_chunk_fwd_status", "gdn2_debug_set_scan_stall",
-           "gdn2_chunk_fwd_noalloc", "gdn2_chunk_fwd_noalloc_status")
+           "gdn2_chunk_fwd_noalloc", "gdn2_chunk_fwd_noalloc_status", "gdn2_chunk_bwd",
+           "gdn2_chunk_bwd_workspace")
 
 
 class Params(ctypes.Structure):
@@ -81,6 +84,10 @@ def lib():
         L.gdn2_chunk_fwd.restype = ctypes.c_int
         L.gdn2_decode_step.argtypes = [pp] + [vp] * 9
         L.gdn2_decode_step.restype = ctypes.c_int
+        L.gdn2_chunk_bwd_workspace.argtypes = [pp]
+        L.gdn2_chunk_bwd_workspace.restype = ctypes.c_size_t
+        L.gdn2_chunk_bwd.argtypes = [pp] + [vp] * 17 + [ctypes.c_size_t, vp]
+        L.gdn2_chunk_bwd.restype = ctypes.c_int
         L.gdn2_chunk_fwd_status.argtypes = [vp, vp]
         L.gdn2_chunk_fwd_status.restype = ctypes.c_int
         L.gdn2_chunk_fwd_noalloc_status.argtypes = [vp]
@@ -344,3 +351,48 @@ def debug_set_scan_stall(polls: int) -> None:
     """Failure-path test hook: polls > 0 makes every later tensor-core prefill's
     scan give up on a wait before it issues any product; 0 turns it off."""
     lib().gdn2_debug_set_scan_stall(int(polls))
+
+
+def chunk_bwd_workspace(params: Params) -> int:
+    return int(lib().gdn2_chunk_bwd_workspace(ctypes.byref(params)))
+
+
+def chunk_bwd(q, k, v, alpha, b, w, S0, dO, dS_T=None, *, scale=1.0, gate_mode="full", gate_logits=False,
+              gates_per_qk_head=False, precision="default", workspace=None, stream=None, want_dS0=True):
+    """Gradients of <dO, o> + <dS_T, S_T> for :func:`chunk_fwd`'s inputs (same
+    argument forms; dO in o's dtype, dS_T fp32 or None). Returns a dict of fp32
+    tensors q, k, v, alpha, b, w (None in the tied modes, where b holds dβ), S0
+    (None without ``want_dS0``)."""
+    B, T, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, q.dtype)
+    gdt = torch.bfloat16 if gate_logits else torch.float32
+    for name, t in (("alpha", alpha), ("b", b), ("w", w)):
+        _check(t, name, gdt)
+    _check(dO, "dO")
+    for name, t in (("S0", S0), ("dS_T", dS_T)):
+        _check(t, name, torch.float32)
+    _check_shapes((B, T), H_qk, H_v, d_k, d_v, k, v, alpha, b, w, gate_mode, gates_per_qk_head,
+                  states=(("S0", S0), ("dS_T", dS_T)))
+    if tuple(dO.shape) != (B, T, H_v, d_v):
+        raise ValueError(f"dO must have shape {(B, T, H_v, d_v)}, got {tuple(dO.shape)}")
+    p = make_params(B, T, H_qk, H_v, d_k, d_v, scale=scale, qkv_dtype=_dtype_code(q.dtype),
+                    o_dtype=_dtype_code(dO.dtype), gate_mode=gate_mode, precision=precision,
+                    gate_logits=gate_logits, gates_per_qk_head=gates_per_qk_head)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"q": torch.empty(q.shape, **f32), "k": torch.empty(k.shape, **f32), "v": torch.empty(v.shape, **f32),
+         "alpha": torch.empty(alpha.shape, **f32), "b": torch.empty(b.shape, **f32),
+         "w": None if w is None else torch.empty(w.shape, **f32),
+         "S0": torch.empty((B, H_v, d_k, d_v), **f32) if want_dS0 else None}
+    need = chunk_bwd_workspace(p)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdn2_chunk_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b), _ptr(w),
+                              _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]),
+                              _ptr(g["alpha"]), _ptr(g["b"]), _ptr(g["w"]), _ptr(g["S0"]), _ptr(workspace),
+                              ws_bytes, _stream_handle(stream))
+    if st != OK:
+        raise GDN2Error(st, "gdn2_chunk_bwd")
+    return g

@@ -199,6 +199,46 @@ GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const v
                            const float* S0, void* o, float* S_T,
                            void* workspace, size_t ws_bytes, void* stream);
 
+/* Bytes of device workspace gdn2_chunk_bwd needs for `p` (0 if the call is
+ * not supported or the parameters are invalid): every 16-token chunk's entry
+ * state, B·H_v·ceil(T/16)·d_k·d_v·4 bytes. */
+GDN2_API size_t gdn2_chunk_bwd_workspace(const gdn2_params* p);
+
+/* Backward pass of gdn2_chunk_fwd: the gradients of
+ *     L = <dO, o> + <dS_T, S_T>
+ * with respect to q, k, v, the gates and S0, for upstream gradients dO (of o)
+ * and dS_T (of the final state), i.e. the vector-Jacobian product of the
+ * chunked prefill ("Resumo Técnico: Gated DeltaNet-2", Metodologia §3,
+ * "Passagem de Retropropagação Consciente de Portões": the per-channel erase
+ * and write gates enter the gradients of the WY factors). Chunked, exact fp32
+ * arithmetic: the forward is recomputed from checkpoints of every 16-token
+ * chunk's entry state (kept in the workspace), then the chunks are walked in
+ * reverse carrying dS; within a chunk the gradients go through (I + T)⁻¹, the
+ * Gram matrices and the decays in closed form.
+ *
+ *   q, k, v, alpha, b, w, S0   the forward's inputs (layouts, dtypes and gate
+ *                              forms as gdn2_chunk_fwd; S0 may be NULL)
+ *   dO     [B,T,H_v,d_v]       o_dtype, upstream gradient of o
+ *   dS_T   [B,H_v,d_k,d_v]     fp32 upstream gradient of S_T, or NULL (zeros)
+ *   dq, dk [B,T,H_qk,d_k]      fp32, written (the sums over the value heads of
+ *                              each query/key head)
+ *   dv     [B,T,H_v,d_v]       fp32, written
+ *   dalpha, db, dw             fp32, the shapes of alpha, b, w (tied modes: db
+ *                              is dβ and dw is NULL; with gate_logits the
+ *                              gradients of the logits; with gates per QK head
+ *                              the sums over the value heads of the group)
+ *   dS0    [B,H_v,d_k,d_v]     fp32 gradient of S0, written; may be NULL
+ *   workspace                  at least gdn2_chunk_bwd_workspace(p) bytes
+ * Outputs must not overlap each other or any input. Preconditions as for
+ * gdn2_chunk_fwd with α ∈ (0,1] (the gradient of α divides by α). Not
+ * supported (GDN2_ERR_UNSUPPORTED): the fused conv or L2 norm, conv
+ * histories, packed sequences. Every precision setting runs the fp32 kernel. */
+GDN2_API gdn2_status gdn2_chunk_bwd(const gdn2_params* p, const void* q, const void* k, const void* v,
+                                    const float* alpha, const float* b, const float* w, const float* S0,
+                                    const void* dO, const float* dS_T, float* dq, float* dk, float* dv,
+                                    float* dalpha, float* db, float* dw, float* dS0, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
 /* Device status of the last gdn2_chunk_fwd call that ran with `workspace`.
  *
  * The tensor-core kernels wait on their own asynchronous work (tensor-core

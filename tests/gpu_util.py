@@ -11,7 +11,11 @@ TOL_BF16 = 2e-2   # bf16 operands, fp32 accumulate
 
 
 def np64(t):
-    return None if t is None else t.detach().to(torch.float64).cpu().numpy()
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64, copy=False)
+    return t.detach().to(torch.float64).cpu().numpy()
 
 
 def oracle_gates(mode, alpha, b, w, d_k, d_v, gate_logits=False, H_v=None, head_axis=2):
