@@ -112,9 +112,10 @@ def tc_launches_per_call(w, ws_bytes, dev):
     runs 2·B·H_v half-width CTAs, or B·H_v full-width ones when the half-width
     grid would need ≥ 5/3 as many waves; when the scan grid leaves SMs idle,
     the sequence has at least 64 chunks and no load step (conv / L2 norm) is
-    fused, the call pipelines 2 to 4 segments (a prep and a scan each), else
-    it runs one segment (a prep and a scan, plus the load step if fused). The
-    SIMT path (no workspace) is one launch."""
+    fused, the call pipelines 2 to 4 segments, else it runs one segment; a
+    segment is a prep, the exact kernel for strongly decaying chunks and a
+    scan, plus the load step if fused. The SIMT path (no workspace) is one
+    launch."""
     if ws_bytes == 0:
         return 1
     import torch
@@ -124,8 +125,8 @@ def tc_launches_per_call(w, ws_bytes, dev):
     scan_ctas = bh if 5 * waves_full < 3 * waves_half else 2 * bh
     nchunks = (w.T + 63) // 64
     if not w.conv and nchunks >= 64 and scan_ctas < sms:
-        return 2 * min(4, nchunks // 32)
-    return 3 if w.conv else 2
+        return 3 * min(4, nchunks // 32)
+    return 4 if w.conv else 3
 
 
 def kernel_sources_sha1():
@@ -357,6 +358,11 @@ def main():
                     help="timed decode steps with the conv and L2 norm in the step; 0 skips it")
     ap.add_argument("--conv-steps", type=int, default=5,
                     help="timed calls of the conv + L2 workload (B=8, T=8192); 0 skips it")
+    ap.add_argument("--tied-steps", type=int, default=20,
+                    help="timed calls of the T=32768 prefill with the tied gates of KDA and of Gated DeltaNet")
+    ap.add_argument("--t4096-steps", type=int, default=50, help="timed calls of the T=4096 prefill; 0 skips it")
+    ap.add_argument("--bwd-steps", type=int, default=3,
+                    help="timed calls of the backward pass on the B=8, T=8192 training shape; 0 skips it")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -453,6 +459,17 @@ def main():
     if args.qk_gates_steps > 0:
         qk_gates = run_gate_variant(args.qk_gates_steps, w, dev, stream, barrier, pk, world, qk=True)
 
+    tied = {}
+    if args.tied_steps > 0:
+        for mode in ("kda", "gdn"):
+            tied[mode] = run_gate_variant(args.tied_steps, w, dev, stream, barrier, pk, world, gate_mode=mode)
+    t4096 = None
+    if args.t4096_steps > 0 and w.name != "prefill_t4096":
+        t4096 = run_gate_variant(args.t4096_steps, workload("prefill_t4096"), dev, stream, barrier, pk, world)
+    bwd = None
+    if args.bwd_steps > 0:
+        bwd = run_bwd(args, dev, stream, barrier, pk, world)
+
     # ---------------------------------------------------------------- end to end
     e2e = None
     if args.e2e_steps > 0:
@@ -481,7 +498,8 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
             "conv_prefill": conv, "prefill_gate_logits": logits, "prefill_qk_gates": qk_gates,
-            "decode_conv": decode_conv,
+            "decode_conv": decode_conv, "prefill_kda": tied.get("kda"), "prefill_gdn": tied.get("gdn"),
+            "prefill_t4096": t4096, "backward": bwd,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -586,27 +604,31 @@ def run_conv(args, dev, stream, barrier, pk, world):
             "ms_per_call": cms, "tokens_per_s": cw.B * cw.T * world / (cms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes},
-            "gpu_launches": 3 * args.conv_steps}
+            "gpu_launches": 4 * args.conv_steps}
 
 
-def run_gate_variant(steps, w, dev, stream, barrier, pk, world, gate_logits=False, qk=False):
-    """The headline layer and length with another gate layout: bf16 logits
-    (the kernels apply the sigmoid; half the gate bytes), or alpha and b owned
-    by the QK heads (a third of their bytes at 48 V / 16 QK heads)."""
+def run_gate_variant(steps, w, dev, stream, barrier, pk, world, gate_logits=False, qk=False, gate_mode="full"):
+    """A prefill leg with another gate layout or length: bf16 logits (the
+    kernels apply the sigmoid; half the gate bytes), alpha and b owned by the
+    QK heads (a third of their bytes at 48 V / 16 QK heads), the tied gates of
+    KDA (beta scalar) and Gated DeltaNet (alpha and beta scalar), or another
+    workload with the headline's gates."""
     import torch
     from delta_rule_linear_gdn_b200 import gdn2
     from delta_rule_linear_gdn_b200.inputs import make_inputs
     rank = int(os.environ.get("RANK", "0"))
-    inp = make_inputs(w, seed=rank_seed(rank), device=dev, gate_logits=gate_logits, gates_per_qk_head=qk)
+    inp = make_inputs(w, seed=rank_seed(rank), device=dev, gate_logits=gate_logits, gates_per_qk_head=qk,
+                      gate_mode=gate_mode)
     o = torch.empty((w.B, w.T, w.H_v, w.d), dtype=torch.bfloat16, device=dev)
     S_T = torch.empty((w.B, w.H_v, w.d, w.d), dtype=torch.float32, device=dev)
     p = gdn2.make_params(w.B, w.T, w.H_qk, w.H_v, w.d, w.d, chunk=w.chunk, gate_logits=gate_logits,
-                         gates_per_qk_head=qk)
+                         gates_per_qk_head=qk, gate_mode=gate_mode)
     ws = torch.empty(max(gdn2.chunk_fwd_workspace(p), 1), dtype=torch.uint8, device=dev)
 
     def call():
         gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None, chunk=w.chunk,
-                       o=o, S_T=S_T, workspace=ws, stream=stream, gate_logits=gate_logits, gates_per_qk_head=qk)
+                       o=o, S_T=S_T, workspace=ws, stream=stream, gate_logits=gate_logits, gates_per_qk_head=qk,
+                       gate_mode=gate_mode)
 
     with torch.cuda.stream(stream):
         for _ in range(3):
@@ -622,15 +644,92 @@ def run_gate_variant(steps, w, dev, stream, barrier, pk, world, gate_logits=Fals
     torch.cuda.synchronize()
     barrier()
     lms = max_over_ranks(c0.elapsed_time(c1) / steps, dev)
-    nbytes = prefill_bytes(w, gate_bytes=2 if gate_logits else 4, qk_gates=qk)
+    nbytes = prefill_bytes(w, gate_bytes=2 if gate_logits else 4, qk_gates=qk, gate_mode=gate_mode)
     gbs = nbytes / (lms * 1e-3) / 1e9
+    tflops = prefill_flops(w) / (lms * 1e-3) / 1e12
     what = ("the gates as bf16 logits (sigmoid in the kernels)" if gate_logits else
-            "alpha and b per QK head (shared by its 3 value heads), fp32")
-    return {"workload": f"{w.name} with {what}",
+            "alpha and b per QK head (shared by its 3 value heads), fp32" if qk else
+            "tied gates b = w = beta (KDA): per-channel alpha, scalar beta, fp32" if gate_mode == "kda" else
+            "tied gates (Gated DeltaNet): scalar alpha and scalar beta, fp32" if gate_mode == "gdn" else
+            "fp32 per-channel gates")
+    return {"workload": f"{w.name}: B={w.B} T={w.T} H_qk={w.H_qk} H_v={w.H_v} d={w.d} chunk={w.chunk} with {what}",
             "ms_per_call": lms, "tokens_per_s": w.B * w.T * world / (lms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes},
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes,
+                         "alg_flops_per_launch": prefill_flops(w), "tensor_tflops": tflops,
+                         "tensor_frac": tflops / pk["bf16_tflops"]},
             "gpu_launches": steps * tc_launches_per_call(w, gdn2.chunk_fwd_workspace(p), dev)}
+
+
+def bwd_flops(w):
+    """FLOPs of one gdn2_chunk_bwd call, counting its d²-scaled products per
+    token and value head: the forward pass's E-bar S and K_endᵀ U (4d²), and in
+    the reverse pass E-bar S again (2d²), K_end dS' (2d²), the carried dS
+    (Q-barᵀ dO and E-barᵀ dR, 4d²), dQ-bar, dE-bar and dK_end (6d²): 18d²."""
+    return w.B * w.T * w.H_v * 18 * w.d * w.d
+
+
+def alu_peak_tflops(dev):
+    """fp32 FMA peak of the CUDA cores: SMs × 128 lanes × 2 FLOP × the maximum
+    SM clock (MEASURED_PEAKS' sm_max_mhz, else 1965 MHz)."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = 1965.0
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def run_bwd(args, dev, stream, barrier, pk, world):
+    """The backward pass (gdn2_chunk_bwd) on the training-shape workload: B=8,
+    T=8192, 48 V heads, the recurrence's inputs (unit q, k), nonzero S0,
+    upstream gradients of o (bf16) and of S_T."""
+    import torch
+    from dataclasses import replace
+    from delta_rule_linear_gdn_b200 import gdn2
+    from delta_rule_linear_gdn_b200.inputs import make_inputs, workload
+    rank = int(os.environ.get("RANK", "0"))
+    bw = replace(workload(CONV), conv=False)
+    inp = make_inputs(bw, seed=rank_seed(rank), device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(21)
+    dO = torch.randn((bw.B, bw.T, bw.H_v, bw.d), generator=g, device=dev).to(torch.bfloat16)
+    dST = torch.randn((bw.B, bw.H_v, bw.d, bw.d), generator=g, device=dev)
+    p = gdn2.make_params(bw.B, bw.T, bw.H_qk, bw.H_v, bw.d, bw.d, chunk=bw.chunk)
+    ws = torch.empty(gdn2.chunk_bwd_workspace(p), dtype=torch.uint8, device=dev)
+
+    def call():
+        return gdn2.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"], dO, dST,
+                              workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    torch.cuda.synchronize()
+    barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.bwd_steps):
+            call()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    bms = max_over_ranks(c0.elapsed_time(c1) / args.bwd_steps, dev)
+    flops = bwd_flops(bw)
+    tf = flops / (bms * 1e-3) / 1e12
+    peak = alu_peak_tflops(dev)
+    return {"workload": f"{bw.name} recurrence inputs (no conv): B={bw.B} T={bw.T} H_qk={bw.H_qk} H_v={bw.H_v} "
+                        f"d={bw.d}, bf16 q,k,v,dO, fp32 per-channel gates, S0 and dS_T given; gradients of "
+                        f"q,k,v,alpha,b,w,S0 in fp32",
+            "ms_per_call": bms, "tokens_per_s": bw.B * bw.T * world / (bms * 1e-3),
+            "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "traffic": None, "alg_flops_per_launch": flops,
+                         "peak_source": "derived: SMs x 128 fp32 lanes x 2 FLOP x max SM clock"},
+            "workspace_bytes": gdn2.chunk_bwd_workspace(p),
+            "gpu_launches": args.bwd_steps}
 
 
 def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):

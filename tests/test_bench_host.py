@@ -42,3 +42,15 @@ def test_weak_scaling_value_and_config_note():
     assert bench.weak_value(32768, 4, 2.0) == 32768 * 4 / 2e-3
     note = bench.config_dict(workload("prefill_t32768"))["l2"]
     assert "3.49 GB" in note and "126 MB" in note
+
+
+def test_tied_gate_bytes_and_backward_flops():
+    w = workload("prefill_t32768")
+    qk, v, o, st = TOK * HQK * D * 2 * 2, TOK * HV * D * 2, TOK * HV * D * 2, HV * D * D * 4
+    # KDA: alpha per channel, beta one scalar per (token, value head)
+    assert bench.prefill_bytes(w, gate_mode="kda") == qk + v + o + st + TOK * HV * (D + 1) * 4
+    # Gated DeltaNet: alpha and beta scalars
+    assert bench.prefill_bytes(w, gate_mode="gdn") == qk + v + o + st + TOK * HV * 2 * 4
+    # backward: 18 d^2 per token and value head (B=8, T=8192)
+    bw = workload("conv_prefill_b8_t8192")
+    assert bench.bwd_flops(bw) == 8 * 8192 * HV * 18 * D * D
