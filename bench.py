@@ -111,11 +111,10 @@ def tc_launches_per_call(w, ws_bytes, dev):
     and the whole sequence in the workspace, by the launcher's rules: the scan
     runs 2·B·H_v half-width CTAs, or B·H_v full-width ones when the half-width
     grid would need ≥ 5/3 as many waves; when the scan grid leaves SMs idle,
-    the sequence has at least 64 chunks and no load step (conv / L2 norm) is
-    fused, the call pipelines 2 to 4 segments, else it runs one segment; a
-    segment is a prep, the exact kernel for strongly decaying chunks and a
-    scan, plus the load step if fused. The SIMT path (no workspace) is one
-    launch."""
+    and the sequence has at least 64 chunks, the call pipelines 2 to 4
+    segments, else it runs one segment; a segment is a prep (with the conv
+    and L2 norm in its load when asked for), the exact kernel for strongly
+    decaying chunks and a scan. The SIMT path (no workspace) is one launch."""
     if ws_bytes == 0:
         return 1
     import torch
@@ -124,9 +123,9 @@ def tc_launches_per_call(w, ws_bytes, dev):
     waves_half, waves_full = -(-2 * bh // sms), -(-bh // sms)
     scan_ctas = bh if 5 * waves_full < 3 * waves_half else 2 * bh
     nchunks = (w.T + 63) // 64
-    if not w.conv and nchunks >= 64 and scan_ctas < sms:
+    if nchunks >= 64 and scan_ctas < sms:
         return 3 * min(4, nchunks // 32)
-    return 4 if w.conv else 3
+    return 3
 
 
 def kernel_sources_sha1():
@@ -446,7 +445,7 @@ def main():
     if args.decode_conv_steps > 0:
         decode_conv = run_decode(args, workload(args.decode_workload), dev, stream, barrier, pk, world, conv=True)
 
-    # ---------------------------------------------------------------- conv + L2 load step
+    # ---------------------------------------------------------------- conv + L2 fused into the load
     conv = None
     if args.conv_steps > 0:
         conv = run_conv(args, dev, stream, barrier, pk, world)
@@ -566,7 +565,8 @@ def run_decode(args, dw, dev, stream, barrier, pk, world, conv=False):
 
 def run_conv(args, dev, stream, barrier, pk, world):
     """The B=8, T=8192 workload with the depthwise causal conv on q, k, v and
-    the L2 norm of q, k fused into the load step (three launches per call)."""
+    the L2 norm of q, k fused into the prep's load (prep, exact kernel and
+    scan: three launches per call)."""
     import torch
     from delta_rule_linear_gdn_b200 import gdn2
     from delta_rule_linear_gdn_b200.inputs import make_inputs, workload
@@ -600,11 +600,12 @@ def run_conv(args, dev, stream, barrier, pk, world):
     nbytes = prefill_bytes(cw, s0=True)
     gbs = nbytes / (cms * 1e-3) / 1e9
     return {"workload": f"{cw.name}: B={cw.B} T={cw.T} H_qk={cw.H_qk} H_v={cw.H_v} d={cw.d} chunk={cw.chunk}, "
-                        f"depthwise causal conv k=4 on q,k,v and L2 norm of q,k in the load step, S0 given",
+                        f"depthwise causal conv k=4 on q,k,v and L2 norm of q,k fused into the prep's load, "
+                        f"S0 given",
             "ms_per_call": cms, "tokens_per_s": cw.B * cw.T * world / (cms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": nbytes},
-            "gpu_launches": 4 * args.conv_steps}
+            "gpu_launches": 3 * args.conv_steps}
 
 
 def run_gate_variant(steps, w, dev, stream, barrier, pk, world, gate_logits=False, qk=False, gate_mode="full"):

@@ -113,9 +113,6 @@ ChunkArgs make_chunk_args(const gdn2_params* p, const void* q, const void* k, co
   a.B = p->B; a.T = p->T; a.Hqk = p->H_qk; a.Hv = p->H_v; a.dk = p->d_k; a.dv = p->d_v;
   a.chunk = p->chunk; a.scale = p->scale; a.gate_mode = p->gate_mode; a.l2norm = p->l2norm_qk != 0;
   a.conv_w = p->conv_w;
-  a.qkv_T = p->T;
-  a.qkv_t0 = 0;
-  a.qkv_f16 = 0;
   a.gate_logits = p->gate_logits;
   a.conv_in = p->conv_state_in;
   a.conv_out = p->conv_state_out;

@@ -33,12 +33,14 @@
 //         S ← Γ S + K_endᵀ U,       D_rows 64..127 += (−Aqk) U  (= −O / scale),
 //     with the fp32 state resident in TMEM and an fp16 copy in shared memory
 //     feeding the next chunk's products.
-// Forms selected by the call's parameters: gates as bf16 logits (σ applied
-// where they are read), α and b owned by the QK heads, the conv's history
-// from and to the caller (load step), and sequences of different lengths
-// packed along T (items and scan CTAs find their sequence's chunks and
-// tokens in offset tables passed with the launch). The prep has one compiled
-// copy per combination, so that no form pays for another's addressing.
+// Forms selected by the call's parameters: the depthwise causal conv and the
+// L2 norm of q, k fused into the prep's load (with the conv's history from
+// the caller before a sequence's first token), gates as bf16 logits (σ
+// applied where they are read), α and b owned by the QK heads, and sequences
+// of different lengths packed along T (items and scan CTAs find their
+// sequence's chunks and tokens in offset tables passed with the launch). The
+// prep has one compiled copy per combination, so that no form pays for
+// another's addressing.
 // All MMA operand tiles use the 128-byte-swizzled layout (see tc_prims.cuh),
 // so that a warp writing or reading whole rows is free of bank conflicts.
 //
@@ -116,7 +118,8 @@ constexpr int P_GB = 0;
 constexpr int P_KB = 0;
 constexpr int P_PQ = 8192;            // quarter products [4][128] fp32
 constexpr int P_RED = P_PQ + 4 * D * 4;
-static_assert(P_RED + 32 <= 12288, "quarter products must stay in the unused Gram rows");
+constexpr int P_SUMS = P_RED + 32;    // fused load: per-half sums of squares of k, q [2][64 tok][2] fp32
+static_assert(P_SUMS + 2 * C * 2 * 4 <= 12288, "quarter products and sums must stay in the unused Gram rows");
 constexpr int P_GM = 32768;
 constexpr int P_KM = 65536;
 constexpr int P_EB = 81920;
@@ -157,15 +160,20 @@ __device__ __forceinline__ void st8(uint8_t* base, uint32_t off, uint2 v) {
   *reinterpret_cast<uint2*>(base + off) = v;
 }
 
+// (element 0 in the low half; no address of the argument is taken, so that
+// the packed words stay in registers whatever the inlining order)
 __device__ __forceinline__ void unpack4_f16(uint2 u, float* x) {
-  const __half2* h = reinterpret_cast<const __half2*>(&u);
-  const float2 a = __half22float2(h[0]), b = __half22float2(h[1]);
-  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  x[0] = __half2float(__ushort_as_half((unsigned short)(u.x & 0xffffu)));
+  x[1] = __half2float(__ushort_as_half((unsigned short)(u.x >> 16)));
+  x[2] = __half2float(__ushort_as_half((unsigned short)(u.y & 0xffffu)));
+  x[3] = __half2float(__ushort_as_half((unsigned short)(u.y >> 16)));
 }
+// bf16 is the upper half of an fp32: widening is a shift.
 __device__ __forceinline__ void unpack4_bf16(uint2 u, float* x) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  x[0] = __uint_as_float(u.x << 16);
+  x[1] = __uint_as_float(u.x & 0xffff0000u);
+  x[2] = __uint_as_float(u.y << 16);
+  x[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
 __device__ __forceinline__ void wait_mma(uint64_t* bar, uint32_t& phase, int* sflag) {
@@ -191,17 +199,8 @@ constexpr int NP = 256;               // prep threads (8 warps)
 
 struct PrepSrc {
   const float *alpha, *b, *w;
-  const uint16_t *k, *q, *v;      // bf16, or fp16 when preprocessed
+  const uint16_t *k, *q, *v;      // bf16
 };
-
-// 4 q/k/v values: bf16 from the caller's tensors, fp16 from the preprocessed copies.
-template <bool F16IN>
-__device__ __forceinline__ void unpack4_in(uint2 u, float* x) {
-  if (F16IN)
-    unpack4_f16(u, x);
-  else
-    unpack4_bf16(u, x);
-}
 
 // Gate of one token for 4 channels, or the token's scalar gate broadcast: the
 // fp32 values, or σ of the bf16 logits (LG).
@@ -278,11 +277,12 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int
 // Items are taken in order (chunk-major, value head fastest): by a fixed stride
 // of the grid, or, with `counter`, one at a time from that device counter
 // (zero before the launch), so that CTAs which start late take fewer.
-// F16IN: q, k, v are the load step's fp16 copies; LG: the gates are bf16
-// logits; QKG: alpha and b belong to the QK heads; VL: sequences of different
-// lengths packed along T (one compiled copy each, so that no form pays for the
+// CV: the depthwise causal conv and/or the L2 norm of q, k are fused into the
+// load (see the fused-load steps below); LG: the gates are bf16 logits; QKG:
+// alpha and b belong to the QK heads; VL: sequences of different lengths
+// packed along T (one compiled copy each, so that no form pays for the
 // others' addressing at the register limit).
-template <bool F16IN, bool LG, bool QKG, bool VL>
+template <bool CV, bool LG, bool QKG, bool VL>
 __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
                                                            int* counter, const __grid_constant__ CUtensorMap amap,
                                                            int use_amap) {
@@ -357,14 +357,16 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     return full ? ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hv + it.h : gate_row(it, u);
   };
   auto qkv_tok = [&](const Item& it, int u) -> size_t {
-    return (size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i0 + u;
+    return (size_t)it.bi * a.T + it.t0 + i0 + u;
   };
   auto load_key1 = [&](const Item& it, int u, int s) {
     const bool ok = it.Lc == C || i0 + u < it.Lc;
     const size_t tq = qkv_tok(it, u) * a.Hqk + it.hq;
     bq[s] = ok ? gate4<LG>(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
-    kk[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
-    qq[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
+    if constexpr (!CV) {   // (CV: k and q come from pass 0)
+      kk[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
+      qq[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
+    }
   };
   // The per-channel α tile of an item comes by one TMA copy (rows of the
   // tensor map [B·T][H_v][128]), requested by thread 0 one item ahead.
@@ -403,12 +405,97 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
   };
 
+  // ---- fused load (CV). Raw bf16 rows of 4 channels: token t0 + r of the
+  // item's row of tokens, the sequence's conv history for tokens before its
+  // first one (zeros without a history), zeros past its end.
+  const uint16_t* hist = static_cast<const uint16_t*>(a.conv_in);
+  const size_t hrow = (size_t)(2 * a.Hqk + a.Hv) * D;
+  auto raw4 = [&](const uint16_t* base, int H, int hh, int choff, const Item& it, int r) -> uint2 {
+    const int t = it.t0 + r;
+    const int sq = VL ? it.bh / a.Hv : it.bi;   // the sequence (its history row)
+    const int seq0 = VL ? a.cu_tok[sq] : 0;     // and its first token in the row of tokens
+    if (t >= seq0) {
+      if (r >= it.Lc) return make_uint2(0, 0);
+      return __ldg(reinterpret_cast<const uint2*>(base + (((size_t)it.bi * a.T + t) * H + hh) * D + c0));
+    }
+    if (hist == nullptr) return make_uint2(0, 0);
+    return __ldg(reinterpret_cast<const uint2*>(hist + ((size_t)sq * 3 + 3 + (t - seq0)) * hrow + choff + c0));
+  };
+  // Channel c of y_t = Σ_j W[c][j] · x_{t−3+j}: x holds the raw rows of
+  // tokens t−3 .. t (in x[u] .. x[u + 3]), W the taps of the 4 channels.
+  auto conv4 = [](const uint2* x, int u, const float4* W, float* y) {
+    float x0[4], x1[4], x2[4], x3[4];
+    unpack4_bf16(x[u], x0);
+    unpack4_bf16(x[u + 1], x1);
+    unpack4_bf16(x[u + 2], x2);
+    unpack4_bf16(x[u + 3], x3);
+    y[0] = W[0].x * x0[0] + W[0].y * x1[0] + W[0].z * x2[0] + W[0].w * x3[0];
+    y[1] = W[1].x * x0[1] + W[1].y * x1[1] + W[1].z * x2[1] + W[1].w * x3[1];
+    y[2] = W[2].x * x0[2] + W[2].y * x1[2] + W[2].z * x2[2] + W[2].w * x3[2];
+    y[3] = W[3].x * x0[3] + W[3].y * x1[3] + W[3].z * x2[3] + W[3].w * x3[3];
+  };
+  float* ssum = reinterpret_cast<float*>(smem + P_SUMS);   // [k, q][64 tokens][channel half]
+  // Pass 0 (CV): k and q of the thread's 8 tokens and 4 channels, convolved,
+  // stored un-normalised as fp16 in exactly the bytes of the Gm tile (Ē and Q̄
+  // halves) that this thread overwrites in pass 2 after reading them back; the
+  // token's sum of squares over the warp's 64 channels to shared memory (the
+  // two channel halves are added, and the norm applied, in pass 2, after the
+  // barrier that follows pass 1).
+  // (the raw rows of both k and q are requested before the wait for the
+  // previous item's stores, so that their latency overlaps it)
+  auto fused_qk = [&](const Item& it) {
+    const bool conv = a.conv_w != nullptr;
+    uint2 xs[2][11];
+#pragma unroll
+    for (int arr = 0; arr < 2; ++arr) {
+#pragma unroll
+      for (int j = 0; j < 11; ++j)
+        xs[arr][j] = (conv || j >= 3) ? raw4(arr == 0 ? src.k : src.q, a.Hqk, it.hq,
+                                             (arr == 0 ? a.Hqk * D : 0) + it.hq * D, it, i0 - 3 + j)
+                                      : make_uint2(0, 0);
+    }
+    // the previous item's stores still read the Gram space: wait, then fill it
+    if (tid == 0) bulk_wait_read_all();
+    __syncthreads();
+#pragma unroll
+    for (int arr = 0; arr < 2; ++arr) {
+      const int choff = (arr == 0 ? a.Hqk * D : 0) + it.hq * D;
+      const uint2* x = xs[arr];
+      float4 W[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        W[c] = conv ? __ldg(reinterpret_cast<const float4*>(a.conv_w + (size_t)(choff + c0 + c) * 4))
+                    : make_float4(0.f, 0.f, 0.f, 1.f);
+      float ss[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float y[4];
+        conv4(x, u, W, y);
+        ss[u] = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
+        st8(smem, P_GM + (arr ? 64 * 128 : 0) + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW128),
+            pack4_f16(y[0], y[1], y[2], y[3]));
+      }
+      if (a.l2norm) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+#pragma unroll
+          for (int off = 1; off < 16; off <<= 1) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
+        }
+        if (cg == 0) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ssum[(arr * C + i0 + u) * 2 + (warp & 1)] = ss[u];
+        }
+      }
+    }
+  };
+
   uint32_t phase = 0;
   if (use_amap && tid == 0 && (counter ? *s_item : (int)blockIdx.x) < n_items)
     fetch_alpha(counter ? *s_item : (int)blockIdx.x);
   for (int item = counter ? *s_item : (int)blockIdx.x; item < n_items;) {
     const Item it = decode_item<VL>(a, c_begin, item, sm);
     uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + it.slot * SLOT;
+    if constexpr (CV) fused_qk(it);
     load_alpha_key0(item);
 
     // -------- pass 1: α's forward products within the quarter
@@ -436,6 +523,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     __syncthreads();
     // every thread has read s_item for this item (at the end of the previous one)
     if (counter && tid == 0) *s_item = atomicAdd(counter, 1);
+
     bool gram_bf16, exact;
     {
       float mall = sred[0];
@@ -520,8 +608,19 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     const uint32_t i128 = (uint32_t)(i0 + u) * 128;                                             \
     const uint32_t p64 = i128 + piece(u, BS_ROW64), p128 = i128 + piece(u, BS_ROW128);          \
     float kx[4], qx[4], e[4], rf[4], g[4], fe[4], o[4];                                         \
-    unpack4_in<F16IN>(kk[uk], kx);                                                              \
-    unpack4_in<F16IN>(qq[uk], qx);                                                              \
+    if constexpr (CV) {                                                                         \
+      unpack4_f16(*reinterpret_cast<const uint2*>(smem + P_GM + p128), kx);                     \
+      unpack4_f16(*reinterpret_cast<const uint2*>(smem + P_GM + 64 * 128 + p128), qx);          \
+      if (a.l2norm) {                                                                           \
+        const int ti = i0 + u;                                                                  \
+        const float nk = rsqrtf(ssum[ti * 2] + ssum[ti * 2 + 1] + kL2Eps);                      \
+        const float nq = rsqrtf(ssum[(C + ti) * 2] + ssum[(C + ti) * 2 + 1] + kL2Eps);          \
+        _Pragma("unroll") for (int c = 0; c < 4; ++c) { kx[c] *= nk; qx[c] *= nq; }             \
+      }                                                                                         \
+    } else {                                                                                    \
+      unpack4_bf16(kk[uk], kx);                                                                 \
+      unpack4_bf16(qq[uk], qx);                                                                 \
+    }                                                                                           \
     e[0] = bq[uk].x * kx[0]; e[1] = bq[uk].y * kx[1]; e[2] = bq[uk].z * kx[2]; e[3] = bq[uk].w * kx[3]; \
     _Pragma("unroll") for (int c = 0; c < 4; ++c) {                                             \
       rf[c] = rcp_approx(f[u][c]);                                                              \
@@ -563,13 +662,21 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #undef GDN2_TILE
     // the write side, consumed after the Gram products
     float4 wv[8];
-    uint2 vv[8];
+    constexpr int NV = CV ? 11 : 8;   // CV: raw v of the 8 tokens and the 3 before them (conv at the Z step)
+    uint2 vv[NV];
+    const int choff_v = 2 * a.Hqk * D + it.h * D;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const bool ok = it.Lc == C || i0 + u < it.Lc;
       wv[u] = ok ? gate4<LG>(src.w, w_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
-      vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
-                 : make_uint2(0, 0);
+      if constexpr (!CV)
+        vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
+                   : make_uint2(0, 0);
+    }
+    if constexpr (CV) {
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+        vv[j] = (a.conv_w != nullptr || j >= 3) ? raw4(src.v, a.Hv, it.h, choff_v, it, i0 - 3 + j) : make_uint2(0, 0);
     }
     sync_for_mma();
 
@@ -635,11 +742,20 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
 
 
-    // Z = w ⊙ v (no decay) to its tile, read by the Y/U_w products
+    // Z = w ⊙ v (no decay) to its tile, read by the Y/U_w products (CV: v
+    // convolved here, from its raw rows)
+    float4 Wv[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      Wv[c] = CV && a.conv_w ? __ldg(reinterpret_cast<const float4*>(a.conv_w + (size_t)(choff_v + c0 + c) * 4))
+                             : make_float4(0.f, 0.f, 0.f, 1.f);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       float vx[4];
-      unpack4_in<F16IN>(vv[u], vx);
+      if constexpr (CV)
+        conv4(vv, u, Wv, vx);
+      else
+        unpack4_bf16(vv[u], vx);
       st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
           pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
     }
@@ -788,6 +904,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       const int nx = counter ? *s_item : item + (int)gridDim.x;
       if (nx < n_items) fetch_alpha(nx);
     }
+
     {
       // warps 0..3: Yᵀ rows (key lanes); warps 4..7: U_wᵀ rows (dv lanes),
       // staged in the (now free) Gram operand space and stored by two bulk
@@ -888,9 +1005,25 @@ __global__ void __launch_bounds__(FX_THREADS, 1) chunk_fix_kernel(ChunkArgs a, i
 
   const bool full = a.gate_mode == GDN2_GATES_FULL;
   const bool alpha_pc = a.gate_mode != GDN2_GATES_GDN;
-  const bool lg = a.gate_logits != 0, qkg = a.Hg != a.Hv, f16 = a.qkv_f16 != 0;
-  auto in_val = [&](const void* p, size_t i) -> float {
-    return f16 ? __half2float(static_cast<const __half*>(p)[i]) : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+  const bool lg = a.gate_logits != 0, qkg = a.Hg != a.Hv;
+  const bool conv = a.conv_w != nullptr;
+  const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.conv_in);
+  const size_t hrow = (size_t)(2 * a.Hqk + a.Hv) * D;
+  // channel c of tensor x (H heads, head hh, conv channels from choff) at
+  // token i of the item, after the conv when there is one: y_t = Σ_j W[c][j]
+  // x_{t−3+j}, with the sequence's history rows before its first token
+  auto in_val = [&](const void* x, int H, int hh, int choff, const Item& it, int i, int c) -> float {
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    const int sq = VL ? it.bh / a.Hv : it.bi;   // the sequence (its history row)
+    const int seq0 = VL ? a.cu_tok[sq] : 0;     // and its first token in the row of tokens
+    auto raw = [&](int r) -> float {
+      const int t = it.t0 + r;
+      if (t >= seq0) return __bfloat162float(xb[(((size_t)it.bi * a.T + t) * H + hh) * D + c]);
+      return hist ? __bfloat162float(hist[((size_t)sq * 3 + 3 + (t - seq0)) * hrow + choff + c]) : 0.f;
+    };
+    if (!conv) return raw(i);
+    const float4 W = __ldg(reinterpret_cast<const float4*>(a.conv_w + (size_t)(choff + c) * 4));
+    return W.x * raw(i - 3) + W.y * raw(i - 2) + W.z * raw(i - 1) + W.w * raw(i);
   };
 
   while (mask) {
@@ -901,23 +1034,41 @@ __global__ void __launch_bounds__(FX_THREADS, 1) chunk_fix_kernel(ChunkArgs a, i
     __syncthreads();   // the previous item's arrays (and its max) are read
     if (tid == 0) *swm = 0;
 
-    // ---- inputs (tokens past the sequence's end: α = 1, everything else 0)
+    // ---- inputs (tokens past the sequence's end: α = 1, everything else 0);
+    // q, k after the conv, then L2-normalised by rows; then e = b ⊙ k
     for (int idx = tid; idx < C * D; idx += FX_THREADS) {
       const int i = idx / D, c = idx % D;
-      float al = 1.f, e = 0.f, kx = 0.f, qx = 0.f;
+      float al = 1.f, bb = 0.f, kx = 0.f, qx = 0.f;
       if (i < it.Lc) {
         const size_t r = (size_t)it.bi * a.T + it.t0 + i;
         const size_t gr = qkg ? r * a.Hqk + it.hq : r * a.Hv + it.h;
-        const size_t tq = ((size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i) * a.Hqk + it.hq;
         al = gate_at(a.alpha, alpha_pc ? gr * D + c : gr, lg);
-        kx = in_val(a.k, tq * D + c);
-        qx = in_val(a.q, tq * D + c);
-        e = gate_at(a.b, full ? gr * D + c : gr, lg) * kx;
+        kx = in_val(a.k, a.Hqk, it.hq, a.Hqk * D + it.hq * D, it, i, c);
+        qx = in_val(a.q, a.Hqk, it.hq, it.hq * D, it, i, c);
+        bb = gate_at(a.b, full ? gr * D + c : gr, lg);
       }
       sAl[i * FX_LD + c] = al;
-      sE[i * FX_LD + c] = e;
+      sE[i * FX_LD + c] = bb;
       sK[i * FX_LD + c] = kx;
       sQ[i * FX_LD + c] = qx;
+    }
+    __syncthreads();
+    if (a.l2norm) {
+      const int lane = tid & 31;
+      for (int row = tid >> 5; row < 2 * C; row += FX_THREADS / 32) {
+        float* x = (row < C ? sK : sQ) + (row % C) * FX_LD;
+        float ss = 0.f;
+        for (int c = lane; c < D; c += 32) ss += x[c] * x[c];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv = rsqrtf(ss + kL2Eps);
+        for (int c = lane; c < D; c += 32) x[c] *= inv;
+      }
+      __syncthreads();
+    }
+    for (int idx = tid; idx < C * D; idx += FX_THREADS) {
+      const int i = idx / D, c = idx % D;
+      sE[i * FX_LD + c] *= sK[i * FX_LD + c];
     }
     __syncthreads();
 
@@ -1002,8 +1153,7 @@ __global__ void __launch_bounds__(FX_THREADS, 1) chunk_fix_kernel(ChunkArgs a, i
       if (i < it.Lc) {
         const size_t r = (size_t)it.bi * a.T + it.t0 + i;
         const size_t wr = full ? (r * a.Hv + it.h) * D + c : (qkg ? r * a.Hqk + it.hq : r * a.Hv + it.h);
-        const size_t tv = ((size_t)it.bi * a.qkv_T + (it.t0 - a.qkv_t0) + i) * a.Hv + it.h;
-        z = gate_at(full ? a.w : a.b, wr, lg) * in_val(a.v, tv * D + c);
+        z = gate_at(full ? a.w : a.b, wr, lg) * in_val(a.v, a.Hv, it.h, 2 * a.Hqk * D + it.h * D, it, i, c);
       }
       sAl[i * FX_LD + c] = z;
     }
@@ -1376,7 +1526,6 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
       if (i < Lco) {
         TOut* dst = og + ((tok0 + t0o + i) * a.Hv + h) * D + dv0;
         constexpr int VEC = 16 / (int)sizeof(TOut);
-#pragma unroll
         const float sc = -a.scale * exp2i(-k);
 #pragma unroll
         for (int u = 0; u < 32; u += VEC) *reinterpret_cast<uint4*>(dst + u) = pack_out<TOut>(v + u, sc);
@@ -1490,149 +1639,6 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   if (warp == 0) tmem_dealloc(tmem, L::T_COLS);
 }
 
-// =============================================================================
-// Load step of the tensor-core prefill when the depthwise causal convolution
-// (kernel 4, taps W[c][0..3] on tokens t−3..t; before a sequence's first
-// token, its history from conv_in, or zeros) and/or the L2 normalisation of
-// q, k (after the conv) are requested: q, k, v of the tokens [t_begin, t_begin
-// + Tseg) of every sequence → fp16 copies [B][Tseg][H][D] that the prep
-// kernel reads instead of the caller's tensors. One thread owns 8 consecutive
-// channels and walks the CTA's tokens with the last three inputs in
-// registers; the 16 threads of one head's 128 channels are one half-warp,
-// which reduces the sum of squares. Packed sequences (one row of tokens):
-// at each sequence start the three inputs restart from that sequence's
-// history.
-// =============================================================================
-constexpr int QP_THREADS = 512;
-constexpr int QP_TOK = 64;            // tokens per CTA, in blocks of 8 rows loaded together
-
-template <bool VL>
-__global__ void __launch_bounds__(QP_THREADS, 1) qkv_prep_kernel(ChunkArgs a, int t_begin, int Tseg, __half* qo,
-                                                                 __half* ko, __half* vo) {
-  const int groups = (2 * a.Hqk + a.Hv) * (D / 8);
-  const int g = blockIdx.x * QP_THREADS + threadIdx.x;
-  if (g >= groups) return;            // whole half-warps: groups is a multiple of 16
-  const int bi = blockIdx.z;           // 0 for packed sequences
-  const int lane = threadIdx.x & 31;
-  const unsigned hmask = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
-  const int ch = g * 8;               // channel in [q | k | v]
-  const int which = ch < a.Hqk * D ? 0 : (ch < 2 * a.Hqk * D ? 1 : 2);
-  const int cw = ch - (which == 0 ? 0 : (which == 1 ? a.Hqk * D : 2 * a.Hqk * D));   // channel within the tensor
-  const int H = which == 2 ? a.Hv : a.Hqk;
-  const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(which == 0 ? a.q : (which == 1 ? a.k : a.v));
-  __half* dst = which == 0 ? qo : (which == 1 ? ko : vo);
-  const bool conv = a.conv_w != nullptr;
-  const bool norm = a.l2norm && which < 2;
-
-  float W[8][4];                      // taps of this thread's 8 channels (identity without the conv)
-  if (conv) {
-    const float4* wp = reinterpret_cast<const float4*>(a.conv_w + (size_t)ch * 4);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float4 t = __ldg(wp + c);
-      W[c][0] = t.x; W[c][1] = t.y; W[c][2] = t.z; W[c][3] = t.w;
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) { W[c][0] = W[c][1] = W[c][2] = 0.f; W[c][3] = 1.f; }
-  }
-  const int tl0 = blockIdx.y * QP_TOK;                  // first token of this CTA, relative to t_begin
-  const int nt = min(QP_TOK, Tseg - tl0);
-  const size_t row = (size_t)H * D;                     // elements per token
-  const __nv_bfloat16* base = src + (size_t)bi * a.T * row + cw;
-  auto load = [&](int tl) -> uint4 {                    // token t_begin + tl (zero outside the sequence / CTA)
-    const int t = t_begin + tl;
-    return (tl < tl0 + nt && t >= 0) ? __ldg(reinterpret_cast<const uint4*>(base + (size_t)t * row))
-                                     : make_uint4(0, 0, 0, 0);
-  };
-  auto unpack8 = [](uint4 u, float* x) {
-    unpack4_bf16(make_uint2(u.x, u.y), x);
-    unpack4_bf16(make_uint2(u.z, u.w), x + 4);
-  };
-  // Inputs before the CTA's first token: from the sequence, or for tokens
-  // before 0 from the caller's conv history [B, 3, channels] (zeros without).
-  const size_t hrow = (size_t)(2 * a.Hqk + a.Hv) * D;
-  const __nv_bfloat16* hist = static_cast<const __nv_bfloat16*>(a.conv_in);
-  // The sequence of the CTA's first token (packed: the last n with
-  // cu_tok[n] ≤ it, which passes over empty sequences) and its first token.
-  int sq = bi, s_start = 0;
-  if (VL) {
-    const int tf = t_begin + tl0;
-    int lo = 0, hi = a.nseq;            // cu_tok[lo] ≤ tf < cu_tok[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (a.cu_tok[mid] <= tf) lo = mid; else hi = mid;
-    }
-    sq = lo;
-    s_start = a.cu_tok[lo];
-  }
-  // Row j (token −3 + j of the sequence) of sequence n's history, or zeros.
-  auto hist_row = [&](int n, int j) -> uint4 {
-    if (hist == nullptr) return make_uint4(0, 0, 0, 0);
-    return __ldg(reinterpret_cast<const uint4*>(hist + ((size_t)n * 3 + j) * hrow + ch));
-  };
-  auto hload = [&](int tl) -> uint4 {
-    const int t = t_begin + tl;
-    if (t >= s_start) return load(tl);
-    return hist_row(sq, 3 + t - s_start);
-  };
-  float x3[8], x2[8], x1[8];                            // inputs of t−3, t−2, t−1
-  {
-    const uint4 h3 = conv ? hload(tl0 - 3) : make_uint4(0, 0, 0, 0);
-    const uint4 h2 = conv ? hload(tl0 - 2) : make_uint4(0, 0, 0, 0);
-    const uint4 h1 = conv ? hload(tl0 - 1) : make_uint4(0, 0, 0, 0);
-    unpack8(h3, x3);
-    unpack8(h2, x2);
-    unpack8(h1, x1);
-  }
-  int next_start = VL ? a.cu_tok[sq + 1] : INT_MAX;   // first token of the next sequence
-  for (int b0 = 0; b0 < nt; b0 += 8) {
-    uint4 raw[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) raw[r] = load(tl0 + b0 + r);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (VL && conv && t_begin + tl0 + b0 + r == next_start && b0 + r < nt) {
-        // a packed sequence starts here (the same token for the whole CTA):
-        // the three previous inputs are its history
-        while (a.cu_tok[sq + 1] <= next_start) ++sq;
-        next_start = a.cu_tok[sq + 1];
-        unpack8(hist_row(sq, 0), x3);
-        unpack8(hist_row(sq, 1), x2);
-        unpack8(hist_row(sq, 2), x1);
-      }
-      float x0[8], y[8];
-      unpack8(raw[r], x0);
-      float ss = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        y[c] = W[c][0] * x3[c] + W[c][1] * x2[c] + W[c][2] * x1[c] + W[c][3] * x0[c];
-        ss += y[c] * y[c];
-      }
-      if (norm) {
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(hmask, ss, off);
-        const float inv = rsqrtf(ss + kL2Eps);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) y[c] *= inv;
-      }
-      if (b0 + r < nt) *reinterpret_cast<uint4*>(dst + ((size_t)bi * Tseg + tl0 + b0 + r) * row + cw) = pack8_f16(y);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        x3[c] = x2[c];
-        x2[c] = x1[c];
-        x1[c] = x0[c];
-      }
-    }
-  }
-}
-
-// Bytes of the preprocessed q, k, v copies for `tokens` tokens of every sequence.
-size_t qkv_prep_bytes(const ChunkArgs& a, size_t tokens) {
-  const size_t rows = a.nseq ? 1 : (size_t)a.B;   // packed sequences share one row of tokens
-  return rows * tokens * (size_t)(2 * a.Hqk + a.Hv) * D * sizeof(__half);
-}
-
 size_t state_bytes(const ChunkArgs& a) { return (size_t)a.B * a.Hv * D * D * sizeof(float); }
 
 }  // namespace
@@ -1642,19 +1648,16 @@ bool chunk_tc_supported(const ChunkArgs& a, int qkv_bf16) {
 }
 
 namespace {
-bool needs_qkv_prep(const ChunkArgs& a) { return a.conv_w != nullptr || a.l2norm; }
-// Workspace per chunk of a segment: the slots of every sequence-head and,
-// with the conv / L2 load step, the preprocessed q, k, v of its tokens.
-size_t bytes_per_chunk(const ChunkArgs& a) {
-  return (size_t)a.B * a.Hv * SLOT + (needs_qkv_prep(a) ? qkv_prep_bytes(a, C) : 0);
-}
+// the conv and/or the L2 norm run in the prep's load
+bool fused_load(const ChunkArgs& a) { return a.conv_w != nullptr || a.l2norm; }
+// Workspace per chunk of a segment: the slots of every sequence-head.
+size_t bytes_per_chunk(const ChunkArgs& a) { return (size_t)a.B * a.Hv * SLOT; }
 }  // namespace
 
 // Workspace for the whole sequence in one segment (packed sequences: the
-// slots of all their chunks and the load step's copies of all tokens).
+// slots of all their chunks).
 size_t chunk_tc_workspace(const ChunkArgs& a) {
-  if (a.nseq)
-    return WS_HEAD + (size_t)a.cu_chk[a.nseq] * a.Hv * SLOT + (needs_qkv_prep(a) ? qkv_prep_bytes(a, a.T) : 0);
+  if (a.nseq) return WS_HEAD + (size_t)a.cu_chk[a.nseq] * a.Hv * SLOT;
   const size_t nchunks = (a.T + C - 1) / C;
   return WS_HEAD + nchunks * bytes_per_chunk(a);
 }
@@ -1724,14 +1727,14 @@ bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
 // Runs the chunks in segments when the workspace holds fewer chunks than the
 // sequence has; the state is carried between segments through S_T (or, when
 // S_T is NULL, through the end of the workspace). Workspace: status word and
-// item counters (256 bytes), slots [B·H_v][seg], preprocessed q|k|v of seg·C
-// tokens (conv / L2 only), carried state (only when needed). With the whole
+// item counters (256 bytes), slots [B·H_v][seg], carried state (only when
+// needed). With the whole
 // sequence in the workspace and SMs left idle by the scan, the segments are
 // pipelined (see the note on overlapped segments above).
 using PrepFn = void (*)(ChunkArgs, int, int, SlotMap, int*, const CUtensorMap, int);
 template <bool VL>
-PrepFn prep_variant(bool f16in, bool lg, bool qkg) {
-  if (f16in)
+PrepFn prep_variant(bool cv, bool lg, bool qkg) {
+  if (cv)
     return lg ? (qkg ? chunk_prep_kernel<true, true, true, VL> : chunk_prep_kernel<true, true, false, VL>)
               : (qkg ? chunk_prep_kernel<true, false, true, VL> : chunk_prep_kernel<true, false, false, VL>);
   return lg ? (qkg ? chunk_prep_kernel<false, true, true, VL> : chunk_prep_kernel<false, true, false, VL>)
@@ -1747,11 +1750,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(a.workspace, 0, WS_HEAD, s);   // status word and counters
   if (e != cudaSuccess || BH == 0) return e;
   if (nchunks == 0 && !vl) return e;
-  const bool pre = needs_qkv_prep(a);
+  const bool cv = fused_load(a);
   float* carry = a.ST;
   uint8_t* const ws = static_cast<uint8_t*>(a.workspace);
   int seg = nchunks;
-  size_t slot_bytes = (size_t)a.Hv * nchunks * SLOT;
   if (vl) {
     // packed sequences run in one pass with every chunk's slot in the workspace
     if (a.ws_bytes < chunk_tc_workspace(a)) return cudaErrorInvalidValue;
@@ -1766,11 +1768,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
       carry = reinterpret_cast<float*>(ws + WS_HEAD + (size_t)seg * per_chunk);
     }
     if (seg < 1) return cudaErrorInvalidValue;
-    slot_bytes = (size_t)BH * seg * SLOT;
   }
-  __half* qkv = reinterpret_cast<__half*>(ws + WS_HEAD + slot_bytes);
 
-  for (bool f16 : {false, true})
+  for (bool f16 : {false, true})   // (the fused-load copy and the plain one)
     for (bool lg : {false, true})
       for (bool qg : {false, true}) {
         const PrepFn prep = vl ? prep_variant<true>(f16, lg, qg) : prep_variant<false>(f16, lg, qg);
@@ -1806,17 +1806,13 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   const int prep_ctas = sms * 2;
   CUtensorMap amap{};
   const int use_amap = a.gate_mode != GDN2_GATES_GDN && a.alpha != nullptr && encode_alpha_map(a, &amap) ? 1 : 0;
-  const int qp_groups = (2 * a.Hqk + a.Hv) * (D / 8);
   const bool qkg = a.Hg != a.Hv;
-  auto prep_fn = [&](bool f16in) -> PrepFn {
-    return vl ? prep_variant<true>(f16in, a.gate_logits != 0, qkg) : prep_variant<false>(f16in, a.gate_logits != 0, qkg);
-  };
+  const PrepFn prep = vl ? prep_variant<true>(cv, a.gate_logits != 0, qkg) : prep_variant<false>(cv, a.gate_logits != 0, qkg);
 
   // overlapped segments: whole sequence in the workspace, idle SMs beside the
-  // scan, no load step (its kernel would wait for the scan), S_T given (the
-  // state passes from segment to segment through it)
+  // scan, S_T given (the state passes from segment to segment through it)
   int nseg_ov = 0;
-  if (!vl && seg == nchunks && !pre && a.ST != nullptr && scan_ctas < sms && nchunks >= 2 * OVERLAP_MIN_CHUNKS)
+  if (!vl && seg == nchunks && a.ST != nullptr && scan_ctas < sms && nchunks >= 2 * OVERLAP_MIN_CHUNKS)
     nseg_ov = std::min(std::min(OVERLAP_SEGMENTS, nchunks / OVERLAP_MIN_CHUNKS), MAX_COUNTERS);
 
   // Segment lengths. Overlapped: the last scan has no prep beside it, so the
@@ -1837,39 +1833,16 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     int* counter = nseg_ov > 0 ? reinterpret_cast<int*>(ws) + 1 + k : nullptr;
     const int items = vl ? nchunks * a.Hv : BH * n;
     const int grid = std::min(items, prep_ctas);
-    ChunkArgs ap = a;        // the prep's view of q, k, v (the load step's copies with the conv / L2 norm)
     if (items == 0) {
       // nothing to prepare (packed sequences, all empty)
-    } else if (pre) {
-      const int t_begin = vl ? 0 : c0 * C;
-      const int Tseg = vl ? a.T : std::min(n * C, a.T - t_begin);
-      const int rows = vl ? 1 : a.B;
-      __half* qo = qkv;
-      __half* ko = qo + (size_t)rows * Tseg * a.Hqk * D;
-      __half* vo = ko + (size_t)rows * Tseg * a.Hqk * D;
-      const dim3 qgrid((qp_groups + QP_THREADS - 1) / QP_THREADS, (Tseg + QP_TOK - 1) / QP_TOK, rows);
-      (vl ? qkv_prep_kernel<true> : qkv_prep_kernel<false>)<<<qgrid, QP_THREADS, 0, s>>>(a, t_begin, Tseg, qo, ko, vo);
-      ap.q = qo;
-      ap.k = ko;
-      ap.v = vo;
-      ap.qkv_T = Tseg;
-      ap.qkv_t0 = t_begin;
-      ap.qkv_f16 = 1;
-      ap.conv_w = nullptr;
-      ap.l2norm = 0;
-      prep_fn(true)<<<grid, NP, P_SMEM, s>>>(
-          ap, c0, n, sm, counter, amap, use_amap);
     } else if (nseg_ov > 0 && k > 0) {
-      if ((e = launch_dependent(prep_fn(false),
-                                grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap, use_amap)) !=
-          cudaSuccess)
+      if ((e = launch_dependent(prep, grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap, use_amap)) != cudaSuccess)
         return e;
     } else {
-      prep_fn(false)<<<grid, NP, P_SMEM, s>>>(
-          a, c0, n, sm, counter, amap, use_amap);
+      prep<<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter, amap, use_amap);
     }
     // the items whose decay the prep's factors cannot take, exactly
-    if (items > 0) fix<<<(items + FX_ITEMS - 1) / FX_ITEMS, FX_THREADS, FX_SMEM, s>>>(ap, c0, n, sm);
+    if (items > 0) fix<<<(items + FX_ITEMS - 1) / FX_ITEMS, FX_THREADS, FX_SMEM, s>>>(a, c0, n, sm);
     scan<<<scan_ctas, scan_threads, scan_smem, s>>>(a, c0, n, sm, s_in, s_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     s_in = carry;

@@ -51,11 +51,6 @@ struct ChunkArgs {
   float* ST;
   void* workspace;
   size_t ws_bytes;
-  // Addressing of q, k, v: tokens per sequence in their buffers and the
-  // absolute token of their row 0 (T and 0 for the caller's tensors; other
-  // values when the tensor-core prefill reads its own preprocessed copies),
-  // and whether they hold fp16 instead of the input dtype.
-  int qkv_T, qkv_t0, qkv_f16;
   int gate_logits;   // gates are bf16 logits (σ applied in the kernels)
   // Conv history [B, 3, 2·Hqk·dk + Hv·dv] in the input dtype (NULL = zeros)
   // and the buffer that receives the history after the last token (or NULL).

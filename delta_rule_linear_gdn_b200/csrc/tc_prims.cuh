@@ -265,49 +265,35 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-// Pack 8 floats to 8 bf16 (16 bytes), round to nearest even.
-__device__ __forceinline__ uint4 pack8_bf16(const float* x) {
-  uint4 u;
-  __nv_bfloat162 h;
-  h = __floats2bfloat162_rn(x[0], x[1]); u.x = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2bfloat162_rn(x[2], x[3]); u.y = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2bfloat162_rn(x[4], x[5]); u.z = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2bfloat162_rn(x[6], x[7]); u.w = *reinterpret_cast<uint32_t*>(&h);
-  return u;
+// Pairs of floats to 16-bit pairs (the first value in the low half), round to
+// nearest even, one cvt each; no address is taken, so that the packed words
+// stay in registers whatever the inlining order.
+__device__ __forceinline__ uint32_t pack2_f16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
 }
 
-// Pack 8 floats to 8 fp16 (16 bytes), round to nearest even.
+// Pack 8 floats to 8 bf16 / fp16 (16 bytes).
+__device__ __forceinline__ uint4 pack8_bf16(const float* x) {
+  return make_uint4(pack2_bf16(x[0], x[1]), pack2_bf16(x[2], x[3]), pack2_bf16(x[4], x[5]), pack2_bf16(x[6], x[7]));
+}
 __device__ __forceinline__ uint4 pack8_f16(const float* x) {
-  uint4 u;
-  __half2 h;
-  h = __floats2half2_rn(x[0], x[1]); u.x = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2half2_rn(x[2], x[3]); u.y = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2half2_rn(x[4], x[5]); u.z = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2half2_rn(x[6], x[7]); u.w = *reinterpret_cast<uint32_t*>(&h);
-  return u;
+  return make_uint4(pack2_f16(x[0], x[1]), pack2_f16(x[2], x[3]), pack2_f16(x[4], x[5]), pack2_f16(x[6], x[7]));
 }
 __device__ __forceinline__ uint4 pack8(const float* x, bool bf16) { return bf16 ? pack8_bf16(x) : pack8_f16(x); }
 
-// Pack 2 floats to 2 fp16 (the first in the low half), round to nearest even.
-__device__ __forceinline__ uint32_t pack2_f16(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 // Pack 4 floats to 4 16-bit values (8 bytes).
 __device__ __forceinline__ uint2 pack4_f16(float a, float b, float c, float d) {
-  uint2 u;
-  __half2 h;
-  h = __floats2half2_rn(a, b); u.x = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2half2_rn(c, d); u.y = *reinterpret_cast<uint32_t*>(&h);
-  return u;
+  return make_uint2(pack2_f16(a, b), pack2_f16(c, d));
 }
 __device__ __forceinline__ uint2 pack4_bf16(float a, float b, float c, float d) {
-  uint2 u;
-  __nv_bfloat162 h;
-  h = __floats2bfloat162_rn(a, b); u.x = *reinterpret_cast<uint32_t*>(&h);
-  h = __floats2bfloat162_rn(c, d); u.y = *reinterpret_cast<uint32_t*>(&h);
-  return u;
+  return make_uint2(pack2_bf16(a, b), pack2_bf16(c, d));
 }
 __device__ __forceinline__ uint2 pack4(const float* x, bool bf16) {
   return bf16 ? pack4_bf16(x[0], x[1], x[2], x[3]) : pack4_f16(x[0], x[1], x[2], x[3]);

@@ -172,9 +172,9 @@ def test_varlen_validation_and_workspace(L):
     arr = gdn2.cu_seqlens_array(cu)
     p = gdn2.make_params(1, 331, 2, 6, 128, 128, chunk=64, cu_seqlens=arr)
     assert gdn2.chunk_fwd_workspace(p) == 256 + 8 * 6 * 74752
-    # with the conv / L2 load step: plus fp16 copies of all 331 tokens' q | k | v
+    # the conv / L2 norm run in the prep's own load: no extra workspace
     p = gdn2.make_params(1, 331, 2, 6, 128, 128, chunk=64, cu_seqlens=arr, l2norm_qk=True)
-    assert gdn2.chunk_fwd_workspace(p) == 256 + 8 * 6 * 74752 + 331 * (2 * 2 + 6) * 128 * 2
+    assert gdn2.chunk_fwd_workspace(p) == 256 + 8 * 6 * 74752
 
 
 def _header_param_fields():
