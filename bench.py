@@ -360,6 +360,9 @@ def main():
     ap.add_argument("--tied-steps", type=int, default=20,
                     help="timed calls of the T=32768 prefill with the tied gates of KDA and of Gated DeltaNet")
     ap.add_argument("--t4096-steps", type=int, default=50, help="timed calls of the T=4096 prefill; 0 skips it")
+    ap.add_argument("--cp-steps", type=int, default=5,
+                    help="with N > 1 ranks: timed calls of the T=32768 sequence split across the ranks "
+                         "(context-parallel prefill, strong scaling); 0 skips it")
     ap.add_argument("--bwd-steps", type=int, default=3,
                     help="timed calls of the backward pass on the B=8, T=8192 training shape; 0 skips it")
     args = ap.parse_args()
@@ -468,6 +471,9 @@ def main():
     bwd = None
     if args.bwd_steps > 0:
         bwd = run_bwd(args, dev, stream, barrier, pk, world)
+    cp_leg = None
+    if args.cp_steps > 0 and world > 1:
+        cp_leg = run_context_parallel(args, w, dev, stream, barrier, world)
 
     # ---------------------------------------------------------------- end to end
     e2e = None
@@ -498,7 +504,7 @@ def main():
             "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
             "conv_prefill": conv, "prefill_gate_logits": logits, "prefill_qk_gates": qk_gates,
             "decode_conv": decode_conv, "prefill_kda": tied.get("kda"), "prefill_gdn": tied.get("gdn"),
-            "prefill_t4096": t4096, "backward": bwd,
+            "prefill_t4096": t4096, "backward": bwd, "prefill_context_parallel": cp_leg,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -731,6 +737,40 @@ def run_bwd(args, dev, stream, barrier, pk, world):
                          "peak_source": "derived: SMs x 128 fp32 lanes x 2 FLOP x max SM clock"},
             "workspace_bytes": gdn2.chunk_bwd_workspace(p),
             "gpu_launches": args.bwd_steps}
+
+
+def run_context_parallel(args, w, dev, stream, barrier, world):
+    """The headline sequence split across the ranks: rank r runs tokens
+    [r·T/N, (r+1)·T/N) and the ranks join through the affine maps of their
+    segments (one all-gather); tokens of the one sequence / max-over-ranks
+    time ("strong" scaling)."""
+    import torch
+    from dataclasses import replace
+    from delta_rule_linear_gdn_b200 import context_parallel as cp
+    from delta_rule_linear_gdn_b200.inputs import make_inputs
+    rank = int(os.environ.get("RANK", "0"))
+    seg = replace(w, T=w.T // world)
+    inp = make_inputs(seg, seed=rank_seed(rank), device=dev)   # this rank's segment
+
+    def call():
+        with torch.cuda.stream(stream):
+            cp.chunk_fwd_context_parallel(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(args.cp_steps):
+        call()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(c0.elapsed_time(c1) / args.cp_steps, dev)
+    return {"workload": f"{w.name} split into {world} segments of {seg.T} tokens, one per rank",
+            "ms_per_call": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "scaling": "strong",
+            "gpu_launches": args.cp_steps * (3 * tc_launches_per_call(seg, 1, dev) + world - 1)}
 
 
 def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):

@@ -239,6 +239,24 @@ gdn2_status gdn2_chunk_fwd(const gdn2_params* p, const void* q, const void* k, c
   return gdn2::chunk_fwd_checked(p, q, k, v, alpha, b, w, S0, o, S_T, workspace, ws_bytes, stream, false);
 }
 
+gdn2_status gdn2_state_affine(const gdn2_params* p, const float* M, const float* N, const float* S_in,
+                              float* S_out, void* stream) {
+  if (!p || p->B < 0 || p->H_v <= 0 || p->d_k <= 0 || p->d_v <= 0) return GDN2_ERR_INVALID_ARG;
+  if (p->d_k != p->d_v || !supported_dim(p->d_k) || p->d_k < 32) return GDN2_ERR_UNSUPPORTED;
+  const size_t n = (size_t)p->B * p->H_v;
+  if (n == 0) return GDN2_OK;
+  if (!M || !S_out) return GDN2_ERR_INVALID_ARG;
+  const void* ptrs[] = {M, N, S_in, S_out};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return GDN2_ERR_INVALID_ARG;
+  const size_t sb = n * p->d_k * p->d_v * sizeof(float), mb = n * p->d_k * p->d_k * sizeof(float);
+  // S_out may be S_in; nothing else overlaps it
+  if (overlaps(S_out, sb, M, mb) || overlaps(S_out, sb, N, sb)) return GDN2_ERR_INVALID_ARG;
+  if (S_in && S_in != S_out && overlaps(S_out, sb, S_in, sb)) return GDN2_ERR_INVALID_ARG;
+  const cudaError_t e = launch_state_affine((int)n, p->d_k, p->d_v, M, N, S_in, S_out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
 gdn2_status gdn2_chunk_fwd_status(const void* workspace, void* stream) {
   if (workspace == nullptr) return GDN2_OK;   // the fp32 path keeps no device status
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return GDN2_ERR_INVALID_ARG;

@@ -117,6 +117,11 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s);
 // sequence (history from a.conv_in shifted in when T < 3).
 cudaError_t launch_conv_state(const ChunkArgs& a, int qkv_bf16, cudaStream_t s);
 
+// S_out = M · S_in + N for n states (M [n][dk][dk]; N, S_in, S_out [n][dk][dv];
+// N or S_in NULL = zeros; S_out may be S_in).
+cudaError_t launch_state_affine(int n, int dk, int dv, const float* M, const float* N, const float* S_in,
+                                float* S_out, cudaStream_t s);
+
 // Backward pass: workspace bytes and launcher.
 size_t chunk_bwd_workspace(int n_states, int H_v, int T, int d);
 cudaError_t launch_chunk_bwd(const BwdArgs& a, int d, int qkv_bf16, int do_bf16, cudaStream_t s);

@@ -14,6 +14,8 @@ Entry points mirror the C ABI:
   own fixed scratch, for callers that cannot allocate device memory)
 * :func:`chunk_bwd` -> ``gdn2_chunk_bwd`` (gradients of the prefill), with
   :func:`chunk_bwd_workspace` -> ``gdn2_chunk_bwd_workspace``
+* :func:`state_affine` -> ``gdn2_state_affine`` (S_out = M S_in + N per head: the
+  affine map of a segment, for context-parallel prefill)
 * :func:`chunk_fwd_status` -> ``gdn2_chunk_fwd_status`` (device status of the last
   call on a workspace), :func:`chunk_fwd_noalloc_status` -> ``gdn2_chunk_fwd_noalloc_status``
 * :func:`debug_set_scan_stall` -> ``gdn2_debug_set_scan_stall`` (failure-path test hook)
@@ -39,7 +41,7 @@ PRECISION = {"default": 0, "fp32": 1}
 EXPORTS = ("gdn2_status_str", "gdn2_version", "gdn2_chunk_fwd_workspace", "gdn2_chunk_fwd",
            "gdn2_decode_step", "gdn2_chunk_fwd_status", "gdn2_debug_set_scan_stall",
            "gdn2_chunk_fwd_noalloc", "gdn2_chunk_fwd_noalloc_status", "gdn2_chunk_bwd",
-           "gdn2_chunk_bwd_workspace")
+           "gdn2_chunk_bwd_workspace", "gdn2_state_affine")
 
 
 class Params(ctypes.Structure):
@@ -88,6 +90,8 @@ def lib():
         L.gdn2_chunk_bwd_workspace.restype = ctypes.c_size_t
         L.gdn2_chunk_bwd.argtypes = [pp] + [vp] * 17 + [ctypes.c_size_t, vp]
         L.gdn2_chunk_bwd.restype = ctypes.c_int
+        L.gdn2_state_affine.argtypes = [pp] + [vp] * 5
+        L.gdn2_state_affine.restype = ctypes.c_int
         L.gdn2_chunk_fwd_status.argtypes = [vp, vp]
         L.gdn2_chunk_fwd_status.restype = ctypes.c_int
         L.gdn2_chunk_fwd_noalloc_status.argtypes = [vp]
@@ -396,3 +400,25 @@ def chunk_bwd(q, k, v, alpha, b, w, S0, dO, dS_T=None, *, scale=1.0, gate_mode="
     if st != OK:
         raise GDN2Error(st, "gdn2_chunk_bwd")
     return g
+
+
+def state_affine(M, N, S_in, S_out=None, stream=None):
+    """S_out = M · S_in + N per (sequence, value head): M [B,H_v,d_k,d_k]; N,
+    S_in [B,H_v,d_k,d_v] (either may be None = zeros). S_out may be S_in (in
+    place); a new tensor when None. Returns S_out."""
+    B, H_v, d_k, _ = M.shape
+    ref = N if N is not None else S_in
+    d_v = ref.shape[-1] if ref is not None else d_k
+    for name, t in (("M", M), ("N", N), ("S_in", S_in)):
+        _check(t, name, torch.float32)
+    if S_out is None:
+        S_out = torch.empty((B, H_v, d_k, d_v), dtype=torch.float32, device=M.device)
+    _check(S_out, "S_out", torch.float32)
+    for name, t in (("N", N), ("S_in", S_in), ("S_out", S_out)):
+        if t is not None and tuple(t.shape) != (B, H_v, d_k, d_v):
+            raise ValueError(f"{name} must have shape {(B, H_v, d_k, d_v)}, got {tuple(t.shape)}")
+    p = make_params(B, 0, 1, H_v, d_k, d_v)
+    st = lib().gdn2_state_affine(ctypes.byref(p), _ptr(M), _ptr(N), _ptr(S_in), _ptr(S_out), _stream_handle(stream))
+    if st != OK:
+        raise GDN2Error(st, "gdn2_state_affine")
+    return S_out

@@ -239,6 +239,29 @@ GDN2_API gdn2_status gdn2_chunk_bwd(const gdn2_params* p, const void* q, const v
                                     float* dalpha, float* db, float* dw, float* dS0, void* workspace,
                                     size_t ws_bytes, void* stream);
 
+/* The affine map of a segment applied to states, for carrying a sequence
+ * split into segments (context-parallel prefill):
+ *
+ *     S_out = M · S_in + N      per (sequence, value head)
+ *
+ * Over a segment of tokens the recurrence maps its entry state affinely to
+ * its exit state (every token's step S ↦ (I − k eᵀ) Diag(α) S + k zᵀ is
+ * affine: "Resumo Técnico: Gated DeltaNet-2", Metodologia §1); the state sweep
+ * is the one sequential step of the chunked form ("Uma análise das variantes
+ * de atenção linear da família DeltaNet", "Pipeline Triton da versão por
+ * chunks"). For a segment, M is gdn2_chunk_fwd's S_T from S0 = I with v = 0,
+ * and N its S_T from S0 = 0; composing them gives every segment's entry state.
+ *
+ *   p       B states per value head (B·H_v in all), d_k = d_v ∈ {32, 64, 128}
+ *   M       [B,H_v,d_k,d_k] fp32
+ *   N       [B,H_v,d_k,d_v] fp32, or NULL (zeros)
+ *   S_in    [B,H_v,d_k,d_v] fp32, or NULL (zeros)
+ *   S_out   [B,H_v,d_k,d_v] fp32, written; may equal S_in (in place); must
+ *           not overlap M or N
+ * fp32 arithmetic. Errors as gdn2_chunk_fwd (smaller d: GDN2_ERR_UNSUPPORTED). */
+GDN2_API gdn2_status gdn2_state_affine(const gdn2_params* p, const float* M, const float* N, const float* S_in,
+                                       float* S_out, void* stream);
+
 /* Device status of the last gdn2_chunk_fwd call that ran with `workspace`.
  *
  * The tensor-core kernels wait on their own asynchronous work (tensor-core
