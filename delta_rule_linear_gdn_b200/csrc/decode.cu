@@ -75,55 +75,57 @@ decode_kernel(DecodeArgs a) {
   const size_t hbase = (size_t)bi * 3 * ctot;
   const size_t cq = (size_t)hq * D, ck = (size_t)(a.Hqk + hq) * D, cv = (size_t)2 * a.Hqk * D + (size_t)h * D + col0;
   const TIn* hin = static_cast<const TIn*>(a.conv_in);
-  auto conv1 = [&](TIn xr, size_t ch) -> float {   // y = Σ_j W[ch][j] x_{t−3+j}
+  const TIn zero = from_f32<TIn>(0.f);
+  // y = Σ_j W[ch][j] x_{t−3+j}; the channel's history rows 1, 2 and its input
+  // are kept (in `keep`) for the shifted history written at the end
+  auto conv1 = [&](TIn xr, size_t ch, TIn* keep) -> float {
     const float x = to_f32(xr);
     if (!CONV) return x;
     const float4 wt = __ldg(reinterpret_cast<const float4*>(a.conv_w) + ch);
     float y = wt.w * x;
+    TIn h1 = zero, h2 = zero;
     if (hin) {
       const TIn* hp = hin + hbase + ch;
-      y += wt.x * to_f32(hp[0]) + wt.y * to_f32(hp[ctot]) + wt.z * to_f32(hp[2 * ctot]);
+      h1 = hp[ctot];
+      h2 = hp[2 * ctot];
+      y += wt.x * to_f32(hp[0]) + wt.y * to_f32(h1) + wt.z * to_f32(h2);
     }
+    keep[0] = h1;
+    keep[1] = h2;
+    keep[2] = xr;
     return y;
   };
+  // the shifted history of the channels this thread convolved (written after
+  // the state: nothing in the step waits for it)
+  constexpr int KQ = (2 * D + NT - 1) / NT;        // q, k channels per thread
+  TIn keep_qk[KQ][3], keep_v[3];
   if (CONV) {
     // q and k channels spread over all threads (warp-uniform halves): each
     // thread waits for one channel's taps and history, not two
-    for (int i = tid; i < 2 * D; i += NT) {
-      const bool isq = i < D;
-      const int c = isq ? i : i - D;
-      (isq ? s_q : s_k)[c] = conv1(isq ? qg[c] : kg[c], (isq ? cq : ck) + c);
+#pragma unroll
+    for (int m = 0; m < KQ; ++m) {
+      const int i = tid + m * NT;
+      if (i < 2 * D) {
+        const bool isq = i < D;
+        const int c = isq ? i : i - D;
+        (isq ? s_q : s_k)[c] = conv1(isq ? qg[c] : kg[c], (isq ? cq : ck) + c, keep_qk[m]);
+      }
     }
     for (int i = tid; i < D; i += NT)
       s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
   } else {
     for (int i = tid; i < D; i += NT) {
-      s_q[i] = conv1(qg[i], cq + i);
-      s_k[i] = conv1(kg[i], ck + i);
+      s_q[i] = to_f32(qg[i]);
+      s_k[i] = to_f32(kg[i]);
       s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
     }
   }
   const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at<LG>(a.b, bg);
-  for (int j = tid; j < COLS; j += NT) {
+  static_assert(COLS <= NT, "one v channel per thread at most");
+  if (tid < COLS) {
+    const int j = tid;
     const float wj = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.w, (size_t)bh * D + col0 + j) : beta;
-    s_z[j] = wj * conv1(vg[j], cv + j);
-  }
-  if (CONV && a.conv_out) {
-    // Shifted history: rows 1, 2 of the incoming history, then this token.
-    TIn* hout = static_cast<TIn*>(a.conv_out);
-    auto shift = [&](size_t ch, TIn xr) {
-      const TIn zero = from_f32<TIn>(0.f);
-      hout[hbase + ch] = hin ? hin[hbase + ctot + ch] : zero;
-      hout[hbase + ctot + ch] = hin ? hin[hbase + 2 * ctot + ch] : zero;
-      hout[hbase + 2 * ctot + ch] = xr;
-    };
-    if (tile == 0 && h % (a.Hv / a.Hqk) == 0) {
-      for (int i = tid; i < D; i += NT) {
-        shift(cq + i, qg[i]);
-        shift(ck + i, kg[i]);
-      }
-    }
-    for (int j = tid; j < COLS; j += NT) shift(cv + j, vg[j]);
+    s_z[j] = wj * (CONV ? conv1(vg[j], cv + j, keep_v) : to_f32(vg[j]));
   }
   __syncthreads();
   if (tid < 32) {
@@ -211,6 +213,25 @@ decode_kernel(DecodeArgs a) {
     float4 x = st[i];
     x.x += kr * u0; x.y += kr * u1; x.z += kr * u2; x.w += kr * u3;
     __stcs(Sg + (size_t)row * (D / 4), x);
+  }
+  if (CONV && a.conv_out) {
+    // Shifted history: rows 1, 2 of the incoming history, then this token.
+    // The q, k channels of a QK head are written by the CTA of its first
+    // value head and first column tile; every CTA writes its v channels.
+    TIn* hout = static_cast<TIn*>(a.conv_out);
+    auto shift = [&](size_t ch, const TIn* kp) {
+      hout[hbase + ch] = kp[0];
+      hout[hbase + ctot + ch] = kp[1];
+      hout[hbase + 2 * ctot + ch] = kp[2];
+    };
+    if (tile == 0 && h % (a.Hv / a.Hqk) == 0) {
+#pragma unroll
+      for (int m = 0; m < KQ; ++m) {
+        const int i = tid + m * NT;
+        if (i < 2 * D) shift(i < D ? cq + i : ck + (i - D), keep_qk[m]);
+      }
+    }
+    if (tid < COLS) shift(cv + tid, keep_v);
   }
 }
 
