@@ -363,6 +363,10 @@ def main():
     ap.add_argument("--cp-steps", type=int, default=5,
                     help="with N > 1 ranks: timed calls of the T=32768 sequence split across the ranks "
                          "(context-parallel prefill, strong scaling); 0 skips it")
+    ap.add_argument("--heads-steps", type=int, default=20,
+                    help="with N > 1 ranks: timed calls of the T=32768 layer with its heads split across the "
+                         "ranks (H_qk/N QK heads and the value heads that read them per rank, strong scaling); "
+                         "0 skips it")
     ap.add_argument("--bwd-steps", type=int, default=3,
                     help="timed calls of the backward pass on the B=8, T=8192 training shape; 0 skips it")
     args = ap.parse_args()
@@ -474,6 +478,9 @@ def main():
     cp_leg = None
     if args.cp_steps > 0 and world > 1:
         cp_leg = run_context_parallel(args, w, dev, stream, barrier, world)
+    heads_leg = None
+    if args.heads_steps > 0 and world > 1 and w.H_qk % world == 0:
+        heads_leg = run_head_split(args, w, dev, stream, barrier, world)
 
     # ---------------------------------------------------------------- end to end
     e2e = None
@@ -505,6 +512,7 @@ def main():
             "conv_prefill": conv, "prefill_gate_logits": logits, "prefill_qk_gates": qk_gates,
             "decode_conv": decode_conv, "prefill_kda": tied.get("kda"), "prefill_gdn": tied.get("gdn"),
             "prefill_t4096": t4096, "backward": bwd, "prefill_context_parallel": cp_leg,
+            "prefill_head_split": heads_leg,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -771,6 +779,49 @@ def run_context_parallel(args, w, dev, stream, barrier, world):
     return {"workload": f"{w.name} split into {world} segments of {seg.T} tokens, one per rank",
             "ms_per_call": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "scaling": "strong",
             "gpu_launches": args.cp_steps * (3 * tc_launches_per_call(seg, 1, dev) + world - 1)}
+
+
+def run_head_split(args, w, dev, stream, barrier, world):
+    """The headline layer with its heads split across the ranks: rank r runs
+    QK heads [r·H_qk/N, (r+1)·H_qk/N) and the value heads that read them, over
+    the whole sequence, with no exchange; tokens of the layer / max-over-ranks
+    time ("strong" scaling: the layer is fixed, each rank's share shrinks)."""
+    import torch
+    from dataclasses import replace
+    from delta_rule_linear_gdn_b200 import gdn2
+    from delta_rule_linear_gdn_b200.head_parallel import head_shard
+    from delta_rule_linear_gdn_b200.inputs import make_inputs
+    rank = int(os.environ.get("RANK", "0"))
+    qs, vs = head_shard(w.H_qk, w.H_v, rank, world)
+    mine = replace(w, H_qk=qs.stop - qs.start, H_v=vs.stop - vs.start)
+    inp = make_inputs(mine, seed=rank_seed(rank), device=dev)   # this rank's block of heads
+    o = torch.empty((mine.B, mine.T, mine.H_v, mine.d), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((mine.B, mine.H_v, mine.d, mine.d), dtype=torch.float32, device=dev)
+    p = gdn2.make_params(mine.B, mine.T, mine.H_qk, mine.H_v, mine.d, mine.d, chunk=mine.chunk)
+    ws_bytes = gdn2.chunk_fwd_workspace(p)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+
+    def call():
+        gdn2.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], None, chunk=mine.chunk,
+                       o=o, S_T=S_T, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    torch.cuda.synchronize()
+    barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.heads_steps):
+            call()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(c0.elapsed_time(c1) / args.heads_steps, dev)
+    return {"workload": f"{w.name} with {mine.H_qk} QK / {mine.H_v} V heads per rank on {world} ranks",
+            "ms_per_call": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3), "scaling": "strong",
+            "gpu_launches": args.heads_steps * tc_launches_per_call(mine, ws_bytes, dev)}
 
 
 def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):
