@@ -25,14 +25,15 @@
 //     (tensor cores) and writes the chunk's scan operands — −Yᵀ, −Q̄ᵀ, U_wᵀ,
 //     K_end, −Aqk as fp16 tiles already in the MMA shared-memory layout, and
 //     γ_C — to one 73 KB workspace slot, every tile by a bulk copy.
-//   * scan: two CTAs per (sequence, value head), one per 64-column half of
-//     d_v, walk the chunks in order. They stream the slots into shared memory
-//     with bulk copies (double-buffered, chunk c+1 in flight while c computes)
-//     and run, with Z = [Y; Q̄] stacked so that every product has M = 128,
-//         D = (−Z) S + [I; 0] U_w   (rows 0..63: U = U_w − Y S; rows 64..127: −Q̄ S)
-//         S ← Γ S + K_endᵀ U,       D_rows 64..127 += (−Aqk) U  (= −O / scale),
-//     with the fp32 state resident in TMEM and an fp16 copy in shared memory
-//     feeding the next chunk's products.
+//   * scan: one CTA per (sequence, value head) walks the chunks in order. It
+//     streams the slots into shared memory with bulk copies (double-buffered,
+//     chunk c+1 in flight while c computes) and holds the state transposed,
+//     Sᵀ in tensor memory with one value column per lane, so that the state
+//     and U are A operands read from tensor memory and the slot's tiles are B
+//     operands read from shared memory as the prep wrote them:
+//         Dᵀ = Sᵀ (−Zᵀ), Zᵀ = [Yᵀ | Q̄ᵀ]  (columns 0..63: −(Y S)ᵀ; 64..127: −(Q̄ S)ᵀ)
+//         Uᵀ = U_wᵀ + Dᵀ[:, 0..63],   Sᵀ ← Sᵀ Γ + Uᵀ K_end,
+//         Dᵀ[:, 64..127] += Uᵀ (−Aqkᵀ)  (= −Oᵀ / scale).
 // Forms selected by the call's parameters: the depthwise causal conv and the
 // L2 norm of q, k fused into the prep's load (with the conv's history from
 // the caller before a sequence's first token), gates as bf16 logits (σ
@@ -1223,98 +1224,84 @@ __global__ void __launch_bounds__(FX_THREADS, 1) chunk_fix_kernel(ChunkArgs a, i
 }
 
 // =============================================================================
-// scan kernel: one CTA per (sequence, value head, block of DV columns of d_v)
-// — DV = 64 (two CTAs per head) or 128 (one) — walking the chunks of the
-// segment in order; the recurrence never mixes d_v columns. Per chunk c, with
-// the state S (d_k × DV, fp32 in TMEM, one key per lane) and Z = [Y; Q̄]
-// stacked along the rows:
-//   D  = (−Z) S + [I; 0] U_w  → rows 0..63: U = U_w − Y S, rows 64..127: −Q̄ S
-//   S ← Γ S + K_endᵀ U        (TMEM holds Γ S already)
-//   D_rows 64..127 −= Aqk U   → −O / scale
-// Every product has M = 128 and N = DV. The last warp issues the products and
-// the slot copies (one thread); of the DV/8 epilogue warps (32 columns each,
-// DV/32 per TMEM lane quarter), those on lanes 0..63 write U, those on lanes
-// 64..127 write the outputs of the previous chunk, and all copy the state
-// (fp16 S for the next chunk's products, TMEM ← S·Γ_next). Two CTAs per head
-// finish a chunk sooner; one CTA per head does the work of two on one SM,
-// which pays when the half-width CTAs would need more waves than the SMs give.
+// scan kernel: one CTA per (sequence, value head), walking the chunks of the
+// segment in order with the state held transposed: Sᵀ (d_v × d_k, fp32) lives
+// in tensor memory with one value column of S per TMEM lane, so that both
+// operands that change along the sweep (the state and U) are A operands read
+// from tensor memory, and every chunk operand from the slot is a B operand
+// read from shared memory as the slot holds it. Per chunk c, with
+// Zᵀ = [Yᵀ | Q̄ᵀ] along the columns:
+//   Dᵀ = Sᵀ (−Zᵀ)                  columns 0..63: −(Y S)ᵀ, 64..127: −(Q̄ S)ᵀ
+//   Uᵀ = U_wᵀ + Dᵀ[:, 0..63]        (per lane, in the epilogue)
+//   Sᵀ ← Sᵀ Γ + Uᵀ K_end            (TMEM holds Sᵀ Γ already)
+//   Dᵀ[:, 64..127] += Uᵀ (−Aqkᵀ)    (= −Oᵀ / scale)
+// The recurrence never mixes d_v columns, so each lane's row of Sᵀ carries its
+// own block floating point scale. Four state warps (TMEM lane quarters;
+// thread r = value column r) turn Dᵀ's U part into the 16-bit A operand Uᵀ
+// and the new state into the 16-bit A operand Sᵀ (and back into TMEM times
+// the next chunk's Γ); four output warps (the same lanes) read the finished
+// chunks' outputs out of the other D buffer and store them; the last warp
+// issues the products and the slot copies (one thread). No operand is
+// written to shared memory during the sweep.
 // =============================================================================
-template <int DV>
 struct ScanLayout {
-  static_assert(DV == 64 || DV == 128, "d_v block of a scan CTA");
-  static constexpr int NE = DV * 4;              // epilogue threads
-  static constexpr int NS = NE + 32;             // + the MMA warp
-  // Stage: one chunk's operands for this CTA's columns. DV = 128 takes the
-  // slot byte for byte; DV = 64 takes its half of U_wᵀ and the rest.
-  static constexpr int ZT = 0;                   // −Zᵀ = [−Yᵀ | −Q̄ᵀ]  [128 key][128 tok], BS 16384
-  static constexpr int UW = 32768;               // U_wᵀ rows of the block [DV][64 tok]
-  static constexpr int KE = UW + DV * 128;       // K_end [64 tok][128 key], BS 8192
-  static constexpr int AQ = KE + 16384;          // −Aqk [64][64] (must follow K_end: see the O product)
-  static constexpr int GC = AQ + 8192;           // γ_C [128] fp32
-  static constexpr int WM = GC + 512;            // max |U_w| of the chunk (fp32)
-  static constexpr int BYTES = WM + 16;          // copied per chunk
-  static constexpr int STAGE = (BYTES + 1023) / 1024 * 1024;
-  static constexpr int SH = 2 * STAGE;           // S fp16 [128 key][DV], BS 16384
-  static constexpr int U = SH + 128 * DV * 2;    // U fp16 [64 tok][DV], BS 8192
-  static constexpr int RED = U + 64 * DV * 2;    // per-warp maxima of |S| [2][16] (float bits)
-  static constexpr int BAR = RED + 128;          // 11 mbarriers
-  static constexpr int TMEMP = BAR + 128;
-  static constexpr int FLAG = TMEMP + 16;
-  static constexpr int SMEM = FLAG + 16;
-  static constexpr uint32_t T_S = 0, T_D = DV;   // TMEM: S (DV columns), D double-buffered
-  static constexpr uint32_t T_COLS = DV == 64 ? 256 : 512;
+  static constexpr int STAGE = (SLOT_USED + 1023) / 1024 * 1024;   // one chunk's slot, byte for byte
+  static constexpr int BAR = 2 * STAGE;          // 16 mbarriers
+  static constexpr int KSC = BAR + 128;          // output scale per value column, chunks c mod 4: [4][128] fp32
+  static constexpr int OST = KSC + 4 * 128 * 4;  // outputs of chunks c mod 2, staged [64 tok][128] (fp32 or bf16)
+  static constexpr int FLAG = OST + 2 * C * D * 4;
+  static constexpr int TMEMP = FLAG + 16;
+  static constexpr int SMEM = TMEMP + 16;
+  static constexpr int NE = 128;                 // state threads (one per value column)
+  static constexpr int NO = 128;                 // output threads (one per value column)
+  static constexpr int NS = NE + NO + 32;        // + the MMA warp
+  // TMEM columns
+  static constexpr uint32_t T_S = 0;             // Sᵀ fp32 [128 d_v lanes][128 keys]
+  static constexpr uint32_t T_D = 128;           // Dᵀ fp32 [128][128 tokens], two buffers
+  static constexpr uint32_t T_SH = 384;          // Sᵀ fp16, key pairs [128][64]
+  static constexpr uint32_t T_UH = 448;          // Uᵀ fp16, token pairs [128][32]
+  static constexpr uint32_t T_COLS = 512;
 };
-static_assert(ScanLayout<128>::ZT == SL_YT && ScanLayout<128>::UW == SL_UW && ScanLayout<128>::KE == SL_KE &&
-                  ScanLayout<128>::AQ == SL_AQ && ScanLayout<128>::GC == SL_GC && ScanLayout<128>::WM == SL_WM &&
-                  ScanLayout<128>::BYTES == SLOT_USED,
-              "a full-width stage is the slot");
-static_assert(SL_AQ == SL_KE + 16384 && SL_GC == SL_AQ + 8192, "slot tail copied in one piece");
-static_assert(ScanLayout<64>::SMEM <= 232448 && ScanLayout<128>::SMEM <= 232448, "scan shared memory");
-static_assert(ScanLayout<64>::SH % 1024 == 0 && ScanLayout<128>::SH % 1024 == 0 && ScanLayout<64>::U % 1024 == 0 &&
-                  ScanLayout<128>::U % 1024 == 0,
-              "swizzled tiles on 1 KB boundaries");
+static_assert(ScanLayout::T_UH + 32 <= ScanLayout::T_COLS, "scan tensor memory");
+static_assert(ScanLayout::SMEM <= 232448, "scan shared memory");
 
-// 16 bytes of output: 8 bf16 or 4 fp32 values of sc · x.
-template <typename TOut> __device__ __forceinline__ uint4 pack_out(const float* x, float sc);
-template <> __device__ __forceinline__ uint4 pack_out<__nv_bfloat16>(const float* x, float sc) {
-  float y[8];
+// pairs of fp32 values as fp16 pairs, 16 columns of a TMEM A operand
+__device__ __forceinline__ void tmem_st16_f16(uint32_t taddr, const float* x) {
+  float p[16];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) y[k] = sc * x[k];
-  return pack8_bf16(y);
-}
-template <> __device__ __forceinline__ uint4 pack_out<float>(const float* x, float sc) {
-  return make_uint4(__float_as_uint(sc * x[0]), __float_as_uint(sc * x[1]), __float_as_uint(sc * x[2]),
-                    __float_as_uint(sc * x[3]));
+  for (int j = 0; j < 16; ++j) p[j] = __uint_as_float(pack2_f16(x[2 * j], x[2 * j + 1]));
+  tmem_st16(taddr, p);
 }
 
-// named barriers of the epilogue warps (all of them; those writing U; those writing outputs)
-template <int NE> __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(NE) : "memory"); }
-template <int NE> __device__ __forceinline__ void u_sync() { asm volatile("bar.sync 2, %0;\n" ::"n"(NE / 2) : "memory"); }
-template <int NE> __device__ __forceinline__ void o_sync() { asm volatile("bar.sync 3, %0;\n" ::"n"(NE / 2) : "memory"); }
+template <typename TOut> __device__ __forceinline__ void store_out(TOut* dst, float x);
+template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* dst, float x) {
+  *dst = __float2bfloat16_rn(x);
+}
+template <> __device__ __forceinline__ void store_out<float>(float* dst, float x) { *dst = x; }
 
-template <typename TOut, int DV>
-__global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg_arg,
-                                                           SlotMap sm, const float* S_in, float* S_out) {
-  using L = ScanLayout<DV>;
-  constexpr int NE = L::NE;
+template <typename TOut>
+__global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg_arg,
+                                                                      SlotMap sm, const float* S_in, float* S_out) {
+  using L = ScanLayout;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
   uint64_t* full = bars;                // [2] stage s loaded
-  uint64_t* b_d = bars + 2;             // (−Z)S + [I;0]U_w done (U and −Q̄S in D)
-  uint64_t* b_u = bars + 3;             // U written (fp16)
+  uint64_t* b_d = bars + 2;             // Sᵀ(−Zᵀ) done
+  uint64_t* b_u = bars + 3;             // fp16 Uᵀ written (one arrival per epilogue warp)
   uint64_t* b_s = bars + 4;             // state update done
-  uint64_t* b_sh = bars + 5;            // fp16 S written (one arrival per epilogue warp)
-  uint64_t* b_o = bars + 6;             // [2] D buffer holds the chunk's −O
-  uint64_t* b_of = bars + 8;            // [2] D buffer read out
-  uint64_t* b_never = bars + 10;        // nothing arrives on it (the failure-path test hook waits here)
+  uint64_t* b_sh = bars + 5;            // fp16 Sᵀ written (one arrival per epilogue warp)
+  uint64_t* b_o = bars + 6;             // [2] every product of the chunk in D buffer s done
+  uint64_t* b_fin = bars + 8;           // the products issued before a give-up have completed
+  uint64_t* b_never = bars + 9;         // nothing arrives on it (the failure-path test hook waits here)
+  uint64_t* b_k = bars + 10;            // [4] output scales of chunk c (c mod 4) written (one arrival per state warp)
+  uint64_t* b_of = bars + 14;           // [2] D buffer s read out (one arrival per output warp)
+  float* ksc = reinterpret_cast<float*>(smem + L::KSC);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::TMEMP);
   int* sflag = reinterpret_cast<int*>(smem + L::FLAG);
-  volatile int* estop = sflag + 1;      // [2] the epilogue warps' samples of the flag
   const volatile int* vflag = sflag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = DV == D ? (int)blockIdx.x : (int)blockIdx.x >> 1;
-  const int col0 = DV == D ? 0 : ((int)blockIdx.x & 1) * DV;   // first d_v column of this CTA
+  const int bh = (int)blockIdx.x;
   // resident: the next segment's prep, launched as a programmatic dependent,
   // may take the SMs this grid leaves free
   griddep_launch_dependents();
@@ -1330,8 +1317,8 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   if (n_seg == 0) {
     // an empty packed sequence: its final state is its initial one
     if (S_out) {
-      for (int idx = tid; idx < D * DV; idx += L::NS) {
-        const size_t e = ((size_t)bh * D + idx / DV) * D + col0 + idx % DV;
+      for (int idx = tid; idx < D * D; idx += L::NS) {
+        const size_t e = (size_t)bh * D * D + idx;
         S_out[e] = S_in ? S_in[e] : 0.f;
       }
     }
@@ -1339,11 +1326,9 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   }
 
   if (tid == 0) {
-    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], &bars[i] == b_sh ? NE / 32 : 1);   // b_sh: one per epilogue warp
+    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], i < 10 ? ((&bars[i] == b_sh || &bars[i] == b_u) ? L::NE / 32 : 1) : 4);
     fence_mbar_init();
     sflag[0] = 0;
-    sflag[1] = 0;
-    sflag[2] = 0;
   }
   if (warp == 0) {
     tmem_alloc(tmem_ptr, L::T_COLS);
@@ -1354,31 +1339,23 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
   fence_after_sync();
   const uint32_t tmem = *tmem_ptr;
 
-  if (warp == NE / 32) {
+  if (warp == (L::NE + L::NO) / 32) {
     // ------------------------------------------------------------ MMA thread
     if (lane == 0) {
       auto load = [&](int c) {
         uint8_t* stg = smem + (c & 1) * L::STAGE;
-        const uint8_t* sl = slots + (size_t)c * SLOT;
-        mbar_arrive_expect_tx(&full[c & 1], L::BYTES);
-        if (DV == D) {
-          bulk_g2s(stg, sl, L::BYTES, &full[c & 1]);
-        } else {
-          bulk_g2s(stg + L::ZT, sl + SL_YT, 32768, &full[c & 1]);
-          bulk_g2s(stg + L::UW, sl + SL_UW + col0 * 128, DV * 128, &full[c & 1]);
-          bulk_g2s(stg + L::KE, sl + SL_KE, SLOT_USED - SL_KE, &full[c & 1]);
-        }
+        mbar_arrive_expect_tx(&full[c & 1], SLOT_USED);
+        bulk_g2s(stg, slots + (size_t)c * SLOT, SLOT_USED, &full[c & 1]);
       };
       int issued = 0, landed = 0;       // chunks whose copies were issued / seen complete
+      bool any_mma = false;
       for (int c = 0; c < n_seg && c < 2; ++c) {
         load(c);
         ++issued;
       }
-      const uint32_t id_zs = idesc_f16(128, DV, true, true);     // −Zᵀ (MN) × S (MN)
-      const uint32_t id_kn = idesc_f16(128, DV, true, true);     // K_endᵀ (MN) × U (MN)
-      const uint32_t id_au = idesc_f16(128, DV, false, true);    // [·;−Aqk] (K) × U (MN)
-      const uint64_t sh0 = desc_mn_sw(smem_u32(smem + L::SH), 0, BS_ROW128);
-      const uint64_t u0 = desc_mn_sw(smem_u32(smem + L::U), 0, BS_ROW64);
+      const uint32_t id_zs = idesc_f16(128, 128, false, true);   // Sᵀ (TMEM) × −Zᵀ (MN)
+      const uint32_t id_uk = idesc_f16(128, 128, false, true);   // Uᵀ (TMEM) × K_end (MN)
+      const uint32_t id_ua = idesc_f16(128, 64, false, false);   // Uᵀ (TMEM) × −Aqkᵀ (K)
       // Failure-path test hook: a bounded wait that cannot complete, taken
       // before any product is issued, so the give-up path below has only
       // the two slot copies to drain.
@@ -1387,35 +1364,34 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
         const int s = c & 1;
         const uint32_t ph = (uint32_t)(c & 1);
         uint8_t* stg = smem + s * L::STAGE;
-        const uint32_t db = L::T_D + (uint32_t)DV * (uint32_t)s;
+        const uint32_t db = tmem + L::T_D + 128u * (uint32_t)s;
         ok = mbar_wait_or_stop(&full[s], (uint32_t)((c >> 1) & 1), vflag) &&
              (c < 2 || mbar_wait_or_stop(&b_of[s], (uint32_t)(((c - 2) >> 1) & 1), vflag));
         if (!ok) break;
         ++landed;
-        fence_after_sync();
-        // D = (−Z) S (the scaled state's fp16 copy; the U epilogue adds U_w)
-        const uint64_t z0 = desc_mn_sw(smem_u32(stg + L::ZT), 0, BS_ROW128);
         ok = mbar_wait_or_stop(b_sh, ph, vflag);
         if (!ok) break;
         fence_after_sync();
+        // Dᵀ = Sᵀ (−Zᵀ): K = the 128 keys
+        const uint64_t z0 = desc_mn_sw(smem_u32(stg + SL_YT), 0, BS_ROW128);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma16(tmem + db, z0 + mn_step_sw(ks), sh0 + mn_step_sw(ks), id_zs, ks > 0);
+          mma16_ts(db, tmem + L::T_SH + 8 * ks, z0 + mn_step_sw(ks), id_zs, ks > 0);
         mma_commit(b_d);
-        // S += K_endᵀ U (TMEM holds Γ S), then D_rows 64..127 += (−Aqk) U; the
-        // A operand of the latter starts 64 rows before −Aqk (in K_end), whose
-        // products land in rows 0..63, already read out as U.
+        any_mma = true;
         ok = mbar_wait_or_stop(b_u, ph, vflag);
         if (!ok) break;
         fence_after_sync();
-        const uint64_t ke0 = desc_mn_sw(smem_u32(stg + L::KE), 0, BS_ROW64);
-        const uint64_t aq0 = desc_k_sw(smem_u32(stg + L::AQ - 8192), 0, BS_ROW64);
+        // Sᵀ += Uᵀ K_end, then Dᵀ[:, 64..127] += Uᵀ (−Aqkᵀ): K = the 64 tokens
+        const uint64_t ke0 = desc_mn_sw(smem_u32(stg + SL_KE), 0, BS_ROW64);
+        const uint64_t aq0 = desc_k_sw(smem_u32(stg + SL_AQ), 0, BS_ROW64);
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) mma16(tmem + L::T_S, ke0 + mn_step_sw(ks), u0 + mn_step_sw(ks), id_kn, 1);
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma16_ts(tmem + L::T_S, tmem + L::T_UH + 8 * ks, ke0 + mn_step_sw(ks), id_uk, 1);
         mma_commit(b_s);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
-          mma16(tmem + db, aq0 + k_step_sw(ks, BS_ROW64), u0 + mn_step_sw(ks), id_au, 1);
+          mma16_ts(db + 64, tmem + L::T_UH + 8 * ks, aq0 + k_step_sw(ks, BS_ROW64), id_ua, 1);
         mma_commit(&b_o[s]);
         // stage s is free once this chunk's products are done: chunk c + 2
         if (c + 2 < n_seg) {
@@ -1427,49 +1403,100 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
       }
       if (!ok) {
         atomicOr(sflag, 1);
-        // copies still in flight complete (bounded) before shared memory is released
+        // products and copies still in flight complete (bounded) before
+        // tensor and shared memory are released
+        if (any_mma) {
+          mma_commit(b_fin);
+          mbar_wait(b_fin, 0, 1u << 16);
+        }
         for (int k = landed; k < issued; ++k) mbar_wait(&full[k & 1], (uint32_t)((k >> 1) & 1), 1u << 16);
       }
     }
     __syncwarp();
+  } else if (warp >= L::NE / 32) {
+    // ------------------------------------------------------------ output warps
+    // Chunk c's outputs: Dᵀ columns 64..127 of buffer c mod 2 hold −2^k Oᵀ / s
+    // (k: the column's scale in that chunk); row 64 + i is token i, and this
+    // thread writes its value column of it.
+    const int q = warp - L::NE / 32;
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    const int r = q * 32 + lane;
+    const size_t tstride = (size_t)a.Hv * D;
+    for (int c = 0; c < n_seg; ++c) {
+      const int s = c & 1;
+      // (the four output warps take the same way: each warp agrees on its
+      // waits, and the barrier below ORs the warps' failures)
+      bool okw = mbar_wait_or_stop(&b_o[s], (uint32_t)((c >> 1) & 1), vflag) &&
+                 mbar_wait_or_stop(&b_k[c & 3], (uint32_t)((c >> 2) & 1), vflag);
+      okw = __all_sync(0xffffffffu, okw);
+      TOut* st = reinterpret_cast<TOut*>(smem + L::OST + s * (C * D * 4));
+      if (okw) {
+        fence_after_sync();
+        const float sc = ksc[(c & 3) * 128 + r];
+        float v[C];
+#pragma unroll
+        for (int cb = 0; cb < C; cb += 16) tmem_ld16(t_lane + L::T_D + 128u * (uint32_t)s + 64 + cb, v + cb);
+        tmem_wait_ld();
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b_of[s]);
+        // through shared memory (this thread's column of the [token][d_v]
+        // tile), then whole rows in 16-byte pieces
+#pragma unroll
+        for (int i = 0; i < C; ++i) store_out<TOut>(st + i * D + r, sc * v[i]);
+      }
+      uint32_t failed;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.eq.u32 p, %1, 0;\n\t"
+          "barrier.cta.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+          : "=r"(failed)
+          : "r"((uint32_t)okw), "n"(L::NO)
+          : "memory");
+      if (failed) {
+        atomicOr(sflag, 1);
+        break;
+      }
+      const int t0o = c * C;
+      const int Lco = min(C, trem - t0o);
+      constexpr int PIECES = D * (int)sizeof(TOut) / 16;   // 16-byte pieces per row
+      TOut* dst = og + ((tok0 + t0o) * a.Hv + h) * D;
+      for (int idx = tid - L::NE; idx < C * PIECES; idx += L::NO) {
+        const int i = idx / PIECES, pc = idx % PIECES;
+        if (i < Lco)
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dst + (size_t)i * tstride) + pc * 16) =
+              *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(st + i * D) + pc * 16);
+      }
+    }
   } else {
-    // ------------------------------------------------------------ epilogue warps
-    const int lq = warp & 3;
-    const uint32_t t_lane = tmem + ((uint32_t)(lq * 32) << 16);
-    const int row = lq * 32 + lane;     // TMEM lane: a key of S; a row of D
-    const int c0 = (warp >> 2) * 32;    // this warp's 32 of the CTA's DV columns
-    const bool u_warp = lq < 2;         // D rows 0..63 (U) or 64..127 (outputs)
-    const int dv0 = col0 + c0;          // first d_v column of this thread's 32
+    // ------------------------------------------------------------ state warps
+    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    const int r = warp * 32 + lane;     // the value column this thread carries (TMEM lane)
     bool ok = true;
-    auto wait = [&](uint64_t* bar, uint32_t parity) {
-      if (ok && !mbar_wait_or_stop(bar, parity, vflag)) {
+    auto wait = [&](uint64_t* bar, uint32_t parity) {   // (the warp agrees on the outcome)
+      bool got = ok && mbar_wait_or_stop(bar, parity, vflag);
+      got = __all_sync(0xffffffffu, got);
+      if (ok && !got) {
         ok = false;
         atomicOr(sflag, 1);
       }
       fence_after_sync();
+      return ok;
+    };
+    auto publish = [&](uint64_t* bar) {   // this warp's TMEM stores are complete: one arrival
+      tmem_wait_st();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
     };
 
-    // Block floating point. Chunk c runs with a power-of-two scale 2^k_c on
-    // the state in TMEM, its fp16 copy, D and U, so that the 16-bit operands
-    // stay in fp16's range however small or large the state becomes: k_c is
-    // chosen, from the CTA-wide maximum of |S| at the chunk's entry and of
-    // |U_w| of the chunk (stored by the prep), to put the larger of the two
-    // in [2^8, 2^9), leaving 2^7 of headroom below fp16's largest value for
-    // U = U_w − Y S. Every epilogue thread derives the same k_c from the same
-    // shared maxima; the outputs and S_T are divided by 2^k_c.
-    uint32_t* red = reinterpret_cast<uint32_t*>(smem + L::RED);   // [2][16]: per-warp maxima, two buffers
-    auto cta_max = [&](const float* v, int buf) -> float {
-      uint32_t m = 0;
-#pragma unroll
-      for (int u = 0; u < 32; ++u) m = max(m, __float_as_uint(v[u]) & 0x7fffffffu);
-      m = __reduce_max_sync(0xffffffffu, m);
-      if (lane == 0) red[buf * 16 + warp] = m;
-      epi_sync<NE>();
-      uint32_t M = 0;
-#pragma unroll
-      for (int w_ = 0; w_ < NE / 32; ++w_) M = max(M, red[buf * 16 + w_]);
-      return __uint_as_float(M);
-    };
+    // Block floating point, per value column. Column r of chunk c runs with a
+    // power-of-two scale 2^k on its state in TMEM, its fp16 copy, its row of
+    // Dᵀ and of Uᵀ, so that the 16-bit operands stay in fp16's range however
+    // small or large the state becomes: k is chosen, from max |S| over the
+    // column at the chunk's entry and max |U_w| of the chunk (stored by the
+    // prep), to put the larger of the two in [2^8, 2^9), leaving 2^7 of
+    // headroom below fp16's largest value for U = U_w − Y S. The outputs
+    // and S_T of the column are divided by 2^k.
     auto exp2i = [](int k) -> float { return __uint_as_float((uint32_t)(127 + k) << 23); };   // |k| ≤ 126
     // k that brings `ref` (> 0) to [2^8, 2^9); a zero (or NaN) reference keeps k
     auto pick_k = [](float ref, int k) -> int {
@@ -1477,159 +1504,145 @@ __global__ void __launch_bounds__(ScanLayout<DV>::NS, 1) chunk_scan_kernel(Chunk
       const int e = (int)((__float_as_uint(ref) >> 23) & 0xffu) - 127;   // ⌊log2 ref⌋ (subnormal: −127)
       return max(-60, min(60, 8 - e));
     };
-    int k_cur = 0, k_prev = 0;          // scale exponents of chunk c and c − 1
-
-    // The entry state: fp16 2^k S for the first chunk's products, TMEM ←
-    // 2^k S · Γ of the first chunk.
-    wait(&full[0], 0);
-    {
-      const float g = reinterpret_cast<const float*>(smem + L::GC)[row];
-      const float* S0 = S_in ? S_in + ((size_t)bh * D + row) * D + dv0 : nullptr;
-      float v[32];
+    auto absmax = [](const float* x) -> float {   // max |x| over half a row (8 independent chains)
+      uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-      for (int u = 0; u < 32; u += 4) {
-        const float4 x = S0 ? __ldg(reinterpret_cast<const float4*>(S0 + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
-      }
-      const float M = cta_max(v, 0);
-      k_cur = pick_k(fmaxf(M, *reinterpret_cast<const float*>(smem + L::WM)), 0);
-      k_prev = k_cur;
-      const float sg = exp2i(k_cur);
+      for (int u = 0; u < D / 2; ++u) m[u & 7] = max(m[u & 7], __float_as_uint(x[u]) & 0x7fffffffu);
 #pragma unroll
-      for (int u = 0; u < 32; ++u) v[u] *= sg;
+      for (int j = 4; j > 0; j >>= 1)
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 8) st16(smem, L::SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
+        for (int i = 0; i < j; ++i) m[i] = max(m[i], m[i + j]);
+      return __uint_as_float(m[0]);
+    };
+    // the output scale of chunk c (−s / 2^k) for the output warps
+    auto post_scale = [&](int c, int kk) {
+      ksc[(c & 3) * 128 + r] = -a.scale * exp2i(-kk);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b_k[c & 3]);
+    };
+    auto times_gamma = [](float* x, const uint8_t* gsrc) {   // half a row times its 64 entries of γ_C
+      const float4* g4 = reinterpret_cast<const float4*>(gsrc);
 #pragma unroll
-      for (int u = 0; u < 32; ++u) v[u] *= g;
-      tmem_st16(t_lane + L::T_S + c0, v);
-      tmem_st16(t_lane + L::T_S + c0 + 16, v + 16);
-      tmem_wait_st();
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(b_sh);
-
-    // Outputs of chunk cc from D buffer `db`: row 64 + i of D is token i; this
-    // thread writes 32 contiguous d_v values of it. D holds −2^k O / s.
-    auto out_rows = [&](int cc, uint32_t db, uint64_t* freed, int k) {
-      const int t0o = cc * C;
-      const int Lco = min(C, trem - t0o);
-      float v[32];
-      tmem_ld16(t_lane + db + c0, v);
-      tmem_ld16(t_lane + db + c0 + 16, v + 16);
-      tmem_wait_ld();
-      fence_before_sync();
-      o_sync<NE>();
-      if (tid == 64) mbar_arrive(freed);           // first thread of the output warps
-      const int i = row - 64;
-      if (i < Lco) {
-        TOut* dst = og + ((tok0 + t0o + i) * a.Hv + h) * D + dv0;
-        constexpr int VEC = 16 / (int)sizeof(TOut);
-        const float sc = -a.scale * exp2i(-k);
-#pragma unroll
-        for (int u = 0; u < 32; u += VEC) *reinterpret_cast<uint4*>(dst + u) = pack_out<TOut>(v + u, sc);
+      for (int j = 0; j < D / 8; ++j) {
+        const float4 g = g4[j];
+        x[4 * j] *= g.x; x[4 * j + 1] *= g.y; x[4 * j + 2] *= g.z; x[4 * j + 3] *= g.w;
       }
     };
+    int k = 0;
+    constexpr int HK = D / 2;           // a row of Sᵀ is handled in two halves of 64 keys
+    float x[HK];
 
-    bool stopped = false;
-    for (int c = 0; c < n_seg; ++c) {
+    // The entry state: fp16 2^k Sᵀ for the first chunk's products, TMEM ←
+    // 2^k Sᵀ Γ of the first chunk.
+    wait(&full[0], 0);
+    {
+      const float* S0 = S_in ? S_in + (size_t)bh * D * D + r : nullptr;
+      auto load_half = [&](int hf) {
+#pragma unroll
+        for (int j = 0; j < HK; ++j) x[j] = S0 ? __ldg(S0 + (size_t)(hf * HK + j) * D) : 0.f;
+      };
+      float M = 0.f;
+      for (int hf = 0; hf < 2; ++hf) {
+        load_half(hf);
+        M = fmaxf(M, absmax(x));
+      }
+      k = pick_k(fmaxf(M, *reinterpret_cast<const float*>(smem + SL_WM)), 0);
+      post_scale(0, k);
+      const float sg = exp2i(k);
+      for (int hf = 0; hf < 2; ++hf) {
+        load_half(hf);
+#pragma unroll
+        for (int j = 0; j < HK; ++j) x[j] *= sg;
+#pragma unroll
+        for (int cb = 0; cb < HK; cb += 32) tmem_st16_f16(t_lane + L::T_SH + (hf * HK + cb) / 2, x + cb);
+        times_gamma(x, smem + SL_GC + hf * HK * 4);
+#pragma unroll
+        for (int cb = 0; cb < HK; cb += 16) tmem_st16(t_lane + L::T_S + hf * HK + cb, x + cb);
+      }
+      publish(b_sh);
+    }
+
+    for (int c = 0; c < n_seg && ok; ++c) {
       const int s = c & 1;
       const uint32_t ph = (uint32_t)(c & 1);
-      const uint32_t db = L::T_D + (uint32_t)DV * (uint32_t)s;
-      if (u_warp) {
-        // U = 2^k (U_w − Y S): rows 0..63 of D (−2^k Y S) plus 2^k U_w from the
-        // stage's U_wᵀ tile [dv][tok] → fp16 tile [tok][dv]
-        wait(&full[s], (uint32_t)((c >> 1) & 1));   // (landed before D: makes the copy visible here)
-        wait(b_d, ph);
-        float v[32];
-        tmem_ld16(t_lane + db + c0, v);
-        tmem_ld16(t_lane + db + c0 + 16, v + 16);
-        tmem_wait_ld();
-        {
-          const float sg = exp2i(k_cur);
-          const uint8_t* uw = smem + s * L::STAGE + L::UW;
-#pragma unroll
-          for (int u = 0; u < 32; ++u)
-            v[u] = fmaf(sg, __half2float(*reinterpret_cast<const __half*>(uw + sw_off(c0 + u, row, 0))), v[u]);
-        }
-#pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(smem, L::U + sw_off(row, c0 + cb, BS_ROW64), pack8_f16(v + cb));
-        fence_async_smem();
-        fence_before_sync();
-        u_sync<NE>();
-        if (tid == 0) mbar_arrive(b_u);
-      } else if (c > 0) {
-        // outputs of the previous chunk
-        wait(&b_o[s ^ 1], (uint32_t)(((c - 1) >> 1) & 1));
-        out_rows(c - 1, L::T_D + (uint32_t)DV * (uint32_t)(s ^ 1), &b_of[s ^ 1], k_prev);
-      }
-      // the state: fp16 S for the next chunk and TMEM ← S · Γ_next; S_T after the last
-      const bool more = c + 1 < n_seg;
-      if (more) wait(&full[s ^ 1], (uint32_t)(((c + 1) >> 1) & 1));
-      wait(b_s, ph);
+      const uint32_t db = L::T_D + 128u * (uint32_t)s;
+      const uint8_t* stg = smem + s * L::STAGE;
+      const int k_c = k;                  // this chunk's scale
+      // ---- Uᵀ = 2^k (U_wᵀ − (Y S)ᵀ): Dᵀ columns 0..63 plus 2^k U_w of the
+      // stage's U_wᵀ row r (tokens, 16-byte pieces swizzled) → fp16 A operand
+      if (!wait(&full[s], (uint32_t)((c >> 1) & 1)) || !wait(b_d, ph)) break;
       {
-        float v[32];
-        tmem_ld16(t_lane + L::T_S + c0, v);
-        tmem_ld16(t_lane + L::T_S + c0 + 16, v + 16);
-        tmem_wait_ld();                   // 2^k_c S_{c+1}
-        if (more) {
-          // the next chunk's scale, from max |S_{c+1}| and its max |U_w|
-          const float M = cta_max(v, (c + 1) & 1) * exp2i(-k_cur);
-          const float W = *reinterpret_cast<const float*>(smem + (s ^ 1) * L::STAGE + L::WM);
-          const int k_next = pick_k(fmaxf(M, W), k_cur);
-          const float r = exp2i(k_next - k_cur);
+        float v[C];
 #pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] *= r;
-          k_prev = k_cur;
-          k_cur = k_next;
+        for (int cb = 0; cb < C; cb += 16) tmem_ld16(t_lane + db + cb, v + cb);
+        tmem_wait_ld();
+        const float sg = exp2i(k_c);
+        const uint8_t* uw = stg + SL_UW + r * 128;
 #pragma unroll
-          for (int cb = 0; cb < 32; cb += 8) st16(smem, L::SH + sw_off(row, c0 + cb, BS_ROW128), pack8_f16(v + cb));
-          // publish this warp's part of S at once: the next products need
-          // only that; the TMEM state is scaled while they run
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(b_sh);
-          const float g = reinterpret_cast<const float*>(smem + (s ^ 1) * L::STAGE + L::GC)[row];
+        for (int j = 0; j < 8; ++j) {
+          const uint4 p = *reinterpret_cast<const uint4*>(uw + ((j ^ (r & 7)) << 4));
+          const uint32_t w4[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] *= g;
-          tmem_st16(t_lane + L::T_S + c0, v);
-          tmem_st16(t_lane + L::T_S + c0 + 16, v + 16);
-          tmem_wait_st();
-        } else {
-          k_prev = k_cur;
-          if (S_out && ok) {
-            const float r = exp2i(-k_cur);
-            float* ST = S_out + ((size_t)bh * D + row) * D + dv0;
-#pragma unroll
-            for (int u = 0; u < 32; u += 4)
-              *reinterpret_cast<float4*>(ST + u) = make_float4(r * v[u], r * v[u + 1], r * v[u + 2], r * v[u + 3]);
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[q2]));
+            v[8 * j + 2 * q2] = fmaf(sg, f.x, v[8 * j + 2 * q2]);
+            v[8 * j + 2 * q2 + 1] = fmaf(sg, f.y, v[8 * j + 2 * q2 + 1]);
           }
         }
+#pragma unroll
+        for (int cb = 0; cb < C; cb += 32) tmem_st16_f16(t_lane + L::T_UH + cb / 2, v + cb);
+        publish(b_u);
       }
-      // One barrier per chunk orders the scaled TMEM state before the next
-      // state update (issued after U, which the U warps publish only after
-      // this barrier) and carries the stop decision: thread 0 samples the
-      // error flag just before it, every thread reads the sample just after it
-      // (a flag raised later is seen one chunk later; the waits in between
-      // return at once).
-      if (!ok) atomicOr(sflag, 1);
-      if (more) fence_before_sync();
-      // (two sample slots: slot c & 1 is rewritten only in chunk c + 2, after
-      // every thread has passed the barrier of chunk c + 1)
-      if (tid == 0) estop[c & 1] = *vflag;
-      epi_sync<NE>();
-      if (estop[c & 1] != 0) {
-        ok = false;
-        stopped = true;
-        break;
+      // ---- the state: fp16 Sᵀ for the next chunk and TMEM ← Sᵀ Γ_next; S_T after the last
+      const bool more = c + 1 < n_seg;
+      if (more && !wait(&full[s ^ 1], (uint32_t)(((c + 1) >> 1) & 1))) break;
+      if (!wait(b_s, ph)) break;
+      auto ld_half = [&](int hf) {       // 2^k_c Sᵀ_{c+1}, keys hf·64 ..
+#pragma unroll
+        for (int cb = 0; cb < HK; cb += 16) tmem_ld16(t_lane + L::T_S + hf * HK + cb, x + cb);
+        tmem_wait_ld();
+      };
+      if (more) {
+        const uint8_t* nx = smem + (s ^ 1) * L::STAGE;
+        ld_half(0);
+        float M = absmax(x);
+        ld_half(1);
+        M = fmaxf(M, absmax(x)) * exp2i(-k_c);
+        k = pick_k(fmaxf(M, *reinterpret_cast<const float*>(nx + SL_WM)), k_c);
+        const float rs = exp2i(k - k_c);
+        // fp16 copy: the half in registers, then the other one
+#pragma unroll
+        for (int j = 0; j < HK; ++j) x[j] *= rs;
+#pragma unroll
+        for (int cb = 0; cb < HK; cb += 32) tmem_st16_f16(t_lane + L::T_SH + (HK + cb) / 2, x + cb);
+        ld_half(0);
+#pragma unroll
+        for (int j = 0; j < HK; ++j) x[j] *= rs;
+#pragma unroll
+        for (int cb = 0; cb < HK; cb += 32) tmem_st16_f16(t_lane + L::T_SH + cb / 2, x + cb);
+        publish(b_sh);
+        post_scale(c + 1, k);
+        // the TMEM state times Γ_next, while the next products run (complete
+        // before this warp's next arrival on b_u, which orders it before the
+        // next state update)
+        times_gamma(x, nx + SL_GC);
+#pragma unroll
+        for (int cb = 0; cb < HK; cb += 16) tmem_st16(t_lane + L::T_S + cb, x + cb);
+        ld_half(1);
+#pragma unroll
+        for (int j = 0; j < HK; ++j) x[j] *= rs;
+        times_gamma(x, nx + SL_GC + HK * 4);
+#pragma unroll
+        for (int cb = 0; cb < HK; cb += 16) tmem_st16(t_lane + L::T_S + HK + cb, x + cb);
+      } else if (S_out) {
+        const float rs = exp2i(-k_c);
+        float* ST = S_out + (size_t)bh * D * D + r;
+        for (int hf = 0; hf < 2; ++hf) {
+          ld_half(hf);
+#pragma unroll
+          for (int j = 0; j < HK; ++j) ST[(size_t)(hf * HK + j) * D] = rs * x[j];
+        }
       }
-    }
-    // the last chunk's outputs (every epilogue thread left the loop the same way)
-    if (!stopped && n_seg > 0 && !u_warp) {
-      const int s = (n_seg - 1) & 1;
-      wait(&b_o[s], (uint32_t)(((n_seg - 1) >> 1) & 1));
-      out_rows(n_seg - 1, L::T_D + (uint32_t)DV * (uint32_t)s, &b_of[s], k_cur);
     }
     if (!ok) atomicOr(sflag, 1);
   }
@@ -1784,16 +1797,11 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   int dev = 0, sms = 148;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  // Scan width: half-width CTAs (two per head) finish a chunk sooner, but when
-  // they need more waves than the SMs give, full-width ones (one per head, a
-  // chunk in ≈1.7× the time, measured) finish the call sooner.
-  const int waves_half = (2 * BH + sms - 1) / sms, waves_full = (BH + sms - 1) / sms;
-  const bool full_width = 5 * waves_full < 3 * waves_half;
-  const int scan_ctas = full_width ? BH : 2 * BH;
-  auto scan = full_width ? (o_bf16 ? chunk_scan_kernel<__nv_bfloat16, 128> : chunk_scan_kernel<float, 128>)
-                         : (o_bf16 ? chunk_scan_kernel<__nv_bfloat16, 64> : chunk_scan_kernel<float, 64>);
-  const int scan_threads = full_width ? ScanLayout<128>::NS : ScanLayout<64>::NS;
-  const int scan_smem = full_width ? ScanLayout<128>::SMEM : ScanLayout<64>::SMEM;
+  // Scan: one CTA per (sequence, value head).
+  const int scan_ctas = BH;
+  auto scan = o_bf16 ? chunk_scan_kernel<__nv_bfloat16> : chunk_scan_kernel<float>;
+  const int scan_threads = ScanLayout::NS;
+  const int scan_smem = ScanLayout::SMEM;
   if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
     return e;
   auto fix = vl ? chunk_fix_kernel<true> : chunk_fix_kernel<false>;

@@ -110,6 +110,20 @@ __device__ __forceinline__ void mma16(uint32_t tmem_d, uint64_t adesc, uint64_t 
 
 // Arrive on an mbarrier once every tcgen05 operation issued so far by this
 // thread has completed.
+// The same product with the A operand in tensor memory (M lanes, K 16-bit
+// elements packed two per 32-bit column, the lower half first): a_tmem is the
+// TMEM address of K step 0's columns, step ks at a_tmem + 8·ks.
+__device__ __forceinline__ void mma16_ts(uint32_t tmem_d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+      :
+      : "r"(tmem_d), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t* mbar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                    smem_u32(mbar))
