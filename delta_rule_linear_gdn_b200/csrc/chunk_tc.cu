@@ -1353,7 +1353,7 @@ __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs
         load(c);
         ++issued;
       }
-      const uint32_t id_zs = idesc_f16(128, 128, false, true);   // Sᵀ (TMEM) × −Zᵀ (MN)
+      const uint32_t id_zs = idesc_f16(128, 64, false, true);    // Sᵀ (TMEM) × −Yᵀ or −Q̄ᵀ (MN)
       const uint32_t id_uk = idesc_f16(128, 128, false, true);   // Uᵀ (TMEM) × K_end (MN)
       const uint32_t id_ua = idesc_f16(128, 64, false, false);   // Uᵀ (TMEM) × −Aqkᵀ (K)
       // Failure-path test hook: a bounded wait that cannot complete, taken
@@ -1372,12 +1372,18 @@ __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs
         ok = mbar_wait_or_stop(b_sh, ph, vflag);
         if (!ok) break;
         fence_after_sync();
-        // Dᵀ = Sᵀ (−Zᵀ): K = the 128 keys
-        const uint64_t z0 = desc_mn_sw(smem_u32(stg + SL_YT), 0, BS_ROW128);
+        // Dᵀ = Sᵀ (−Zᵀ), K = the 128 keys: the U part (−Yᵀ) first, which
+        // the epilogue waits for, then the output part (−Q̄ᵀ), which runs
+        // while the epilogue works
+        const uint64_t y0 = desc_mn_sw(smem_u32(stg + SL_YT), 0, BS_ROW128);
+        const uint64_t q0 = desc_mn_sw(smem_u32(stg + SL_QT), 0, BS_ROW128);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma16_ts(db, tmem + L::T_SH + 8 * ks, z0 + mn_step_sw(ks), id_zs, ks > 0);
+          mma16_ts(db, tmem + L::T_SH + 8 * ks, y0 + mn_step_sw(ks), id_zs, ks > 0);
         mma_commit(b_d);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma16_ts(db + 64, tmem + L::T_SH + 8 * ks, q0 + mn_step_sw(ks), id_zs, ks > 0);
         any_mma = true;
         ok = mbar_wait_or_stop(b_u, ph, vflag);
         if (!ok) break;
@@ -1505,14 +1511,14 @@ __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs
       return max(-60, min(60, 8 - e));
     };
     auto absmax = [](const float* x) -> float {   // max |x| over half a row (8 independent chains)
-      uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int u = 0; u < D / 2; ++u) m[u & 7] = max(m[u & 7], __float_as_uint(x[u]) & 0x7fffffffu);
+      for (int u = 0; u < D / 2; ++u) m[u & 7] = fmaxf(m[u & 7], fabsf(x[u]));
 #pragma unroll
       for (int j = 4; j > 0; j >>= 1)
 #pragma unroll
-        for (int i = 0; i < j; ++i) m[i] = max(m[i], m[i + j]);
-      return __uint_as_float(m[0]);
+        for (int i = 0; i < j; ++i) m[i] = fmaxf(m[i], m[i + j]);
+      return m[0];
     };
     // the output scale of chunk c (−s / 2^k) for the output warps
     auto post_scale = [&](int c, int kk) {
@@ -1568,14 +1574,12 @@ __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs
       const uint32_t db = L::T_D + 128u * (uint32_t)s;
       const uint8_t* stg = smem + s * L::STAGE;
       const int k_c = k;                  // this chunk's scale
-      // ---- Uᵀ = 2^k (U_wᵀ − (Y S)ᵀ): Dᵀ columns 0..63 plus 2^k U_w of the
-      // stage's U_wᵀ row r (tokens, 16-byte pieces swizzled) → fp16 A operand
-      if (!wait(&full[s], (uint32_t)((c >> 1) & 1)) || !wait(b_d, ph)) break;
+      // ---- Uᵀ = 2^k (U_wᵀ − (Y S)ᵀ): 2^k U_w of the stage's U_wᵀ row r
+      // (tokens, 16-byte pieces swizzled), taken while the product runs,
+      // plus Dᵀ columns 0..63 → fp16 A operand
+      if (!wait(&full[s], (uint32_t)((c >> 1) & 1))) break;
       {
-        float v[C];
-#pragma unroll
-        for (int cb = 0; cb < C; cb += 16) tmem_ld16(t_lane + db + cb, v + cb);
-        tmem_wait_ld();
+        float v[C], w[C];
         const float sg = exp2i(k_c);
         const uint8_t* uw = stg + SL_UW + r * 128;
 #pragma unroll
@@ -1585,10 +1589,16 @@ __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs
 #pragma unroll
           for (int q2 = 0; q2 < 4; ++q2) {
             const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[q2]));
-            v[8 * j + 2 * q2] = fmaf(sg, f.x, v[8 * j + 2 * q2]);
-            v[8 * j + 2 * q2 + 1] = fmaf(sg, f.y, v[8 * j + 2 * q2 + 1]);
+            w[8 * j + 2 * q2] = sg * f.x;
+            w[8 * j + 2 * q2 + 1] = sg * f.y;
           }
         }
+        if (!wait(b_d, ph)) break;
+#pragma unroll
+        for (int cb = 0; cb < C; cb += 16) tmem_ld16(t_lane + db + cb, v + cb);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < C; ++j) v[j] += w[j];
 #pragma unroll
         for (int cb = 0; cb < C; cb += 32) tmem_st16_f16(t_lane + L::T_UH + cb / 2, v + cb);
         publish(b_u);
