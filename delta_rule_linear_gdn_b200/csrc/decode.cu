@@ -60,13 +60,13 @@ decode_kernel(DecodeArgs a) {
   __shared__ float s_u[COLS];
   __shared__ float s_scalar[4];           // |q|⁻¹, |k|⁻¹, kᵀq
 
-  // Issue the state loads first: they are the only HBM-heavy traffic.
   float4* Sg = reinterpret_cast<float4*>(a.S + (size_t)bh * D * D + col0) + cg;
   float4 st[RPT];
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) st[i] = __ldcs(Sg + (size_t)(rg + kRowGroups * i) * (D / 4));
 
-  // Per-token vectors into shared memory (fp32).
+  // Per-token vectors into shared memory (fp32). Every small load of the
+  // step (q, k, v, their conv taps and history, the gates) is issued before
+  // the state loads, so that none of them waits behind the state stream and
+  // no load depends on another.
   const TIn* qg = static_cast<const TIn*>(a.q) + ((size_t)bi * a.Hqk + hq) * D;
   const TIn* kg = static_cast<const TIn*>(a.k) + ((size_t)bi * a.Hqk + hq) * D;
   const TIn* vg = static_cast<const TIn*>(a.v) + (size_t)bh * D + col0;
@@ -78,55 +78,81 @@ decode_kernel(DecodeArgs a) {
   const TIn zero = from_f32<TIn>(0.f);
   // y = Σ_j W[ch][j] x_{t−3+j}; the channel's history rows 1, 2 and its input
   // are kept (in `keep`) for the shifted history written at the end
-  auto conv1 = [&](TIn xr, size_t ch, TIn* keep) -> float {
-    const float x = to_f32(xr);
-    if (!CONV) return x;
-    const float4 wt = __ldg(reinterpret_cast<const float4*>(a.conv_w) + ch);
-    float y = wt.w * x;
-    TIn h1 = zero, h2 = zero;
+  // (loads of conv1: the taps, the history rows, the input)
+  struct ConvIn {
+    float4 wt;
+    TIn h0, h1, h2, x;
+  };
+  auto conv_load = [&](const TIn* xp, size_t ch) -> ConvIn {
+    ConvIn c;
+    c.x = *xp;
+    c.wt = __ldg(reinterpret_cast<const float4*>(a.conv_w) + ch);
+    c.h0 = c.h1 = c.h2 = zero;
     if (hin) {
       const TIn* hp = hin + hbase + ch;
-      h1 = hp[ctot];
-      h2 = hp[2 * ctot];
-      y += wt.x * to_f32(hp[0]) + wt.y * to_f32(h1) + wt.z * to_f32(h2);
+      c.h0 = hp[0];
+      c.h1 = hp[ctot];
+      c.h2 = hp[2 * ctot];
     }
-    keep[0] = h1;
-    keep[1] = h2;
-    keep[2] = xr;
-    return y;
+    return c;
+  };
+  auto conv1 = [&](const ConvIn& c, TIn* keep) -> float {
+    keep[0] = c.h1;
+    keep[1] = c.h2;
+    keep[2] = c.x;
+    return c.wt.x * to_f32(c.h0) + c.wt.y * to_f32(c.h1) + c.wt.z * to_f32(c.h2) + c.wt.w * to_f32(c.x);
   };
   // the shifted history of the channels this thread convolved (written after
   // the state: nothing in the step waits for it)
   constexpr int KQ = (2 * D + NT - 1) / NT;        // q, k channels per thread
   TIn keep_qk[KQ][3], keep_v[3];
-  if (CONV) {
-    // q and k channels spread over all threads (warp-uniform halves): each
-    // thread waits for one channel's taps and history, not two
-#pragma unroll
-    for (int m = 0; m < KQ; ++m) {
-      const int i = tid + m * NT;
-      if (i < 2 * D) {
-        const bool isq = i < D;
-        const int c = isq ? i : i - D;
-        (isq ? s_q : s_k)[c] = conv1(isq ? qg[c] : kg[c], (isq ? cq : ck) + c, keep_qk[m]);
-      }
-    }
-    for (int i = tid; i < D; i += NT)
-      s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
-  } else {
-    for (int i = tid; i < D; i += NT) {
-      s_q[i] = to_f32(qg[i]);
-      s_k[i] = to_f32(kg[i]);
-      s_a[i] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
-    }
-  }
-  const float beta = (a.gate_mode == GDN2_GATES_FULL) ? 0.f : gate_at<LG>(a.b, bg);
+  // this thread's channels: q/k channel tid + m·NT of the 2·D (q first;
+  // warp-uniform halves, so each thread waits for one channel's loads),
+  // α and b channels tid, tid + NT, ..., v channel tid < COLS
   static_assert(COLS <= NT, "one v channel per thread at most");
-  if (tid < COLS) {
-    const int j = tid;
-    const float wj = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.w, (size_t)bh * D + col0 + j) : beta;
-    s_z[j] = wj * (CONV ? conv1(vg[j], cv + j, keep_v) : to_f32(vg[j]));
+  ConvIn cin_qk[KQ], cin_v;
+  float xqk[KQ], av[(D + NT - 1) / NT], bv[(D + NT - 1) / NT];
+#pragma unroll
+  for (int m = 0; m < KQ; ++m) {
+    const int i = tid + m * NT;
+    if (i < 2 * D) {
+      const bool isq = i < D;
+      const int c = isq ? i : i - D;
+      if (CONV) cin_qk[m] = conv_load((isq ? qg : kg) + c, (isq ? cq : ck) + c);
+      else xqk[m] = to_f32((isq ? qg : kg)[c]);
+    }
   }
+  const bool full = a.gate_mode == GDN2_GATES_FULL;
+#pragma unroll
+  for (int m = 0; m * NT < D; ++m) {
+    const int i = tid + m * NT;
+    if (i < D) {
+      av[m] = gate_at<LG>(a.alpha, (a.gate_mode == GDN2_GATES_GDN) ? bg : bg * D + i);
+      bv[m] = full ? gate_at<LG>(a.b, bg * D + i) : 0.f;
+    }
+  }
+  const float beta = full ? 0.f : gate_at<LG>(a.b, bg);
+  float wj = 0.f, vx = 0.f;
+  if (tid < COLS) {
+    wj = full ? gate_at<LG>(a.w, (size_t)bh * D + col0 + tid) : beta;
+    if (CONV) cin_v = conv_load(vg + tid, cv + tid);
+    else vx = to_f32(vg[tid]);
+  }
+  // The state loads: the HBM-heavy traffic.
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) st[i] = __ldcs(Sg + (size_t)(rg + kRowGroups * i) * (D / 4));
+
+#pragma unroll
+  for (int m = 0; m < KQ; ++m) {
+    const int i = tid + m * NT;
+    if (i < 2 * D) (i < D ? s_q : s_k)[i < D ? i : i - D] = CONV ? conv1(cin_qk[m], keep_qk[m]) : xqk[m];
+  }
+#pragma unroll
+  for (int m = 0; m * NT < D; ++m) {
+    const int i = tid + m * NT;
+    if (i < D) s_a[i] = av[m];
+  }
+  if (tid < COLS) s_z[tid] = wj * (CONV ? conv1(cin_v, keep_v) : vx);
   __syncthreads();
   if (tid < 32) {
     float sq = 0.f, sk = 0.f, kq = 0.f;
@@ -154,10 +180,10 @@ decode_kernel(DecodeArgs a) {
   }
   __syncthreads();
   const float iq = s_scalar[0], ik = s_scalar[1], kq = s_scalar[2];
-  for (int i = tid; i < D; i += NT) {
-    const float kk = s_k[i] * ik;
-    const float bb = (a.gate_mode == GDN2_GATES_FULL) ? gate_at<LG>(a.b, bg * D + i) : beta;
-    s_e[i] = bb * kk;
+#pragma unroll
+  for (int m = 0; m * NT < D; ++m) {
+    const int i = tid + m * NT;
+    if (i < D) s_e[i] = (full ? bv[m] : beta) * (s_k[i] * ik);
   }
   __syncthreads();
 
