@@ -189,6 +189,22 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     }
   };
 
+  // Register tiles of the products below: warp w takes rows 2w, 2w + 1 of a
+  // BC-row result (or rows 16w .. 16w + 15 of a D-row one), lane l the value
+  // columns l, l + 32 (NV of them) or key columns l + 32 n (NK).
+  constexpr int NV = (DVT + 31) / 32, NK = (D + 31) / 32;
+  const int r2 = 2 * warp;
+  // Ē = γ ⊙ e, Q̄ = γ ⊙ q and K_end = k ⊙ bk, into the gradient arrays, which
+  // the backward sweep rewrites only after their last use.
+  auto absorbed = [&]() {
+    for (int idx = tid; idx < BC * D; idx += BT) {
+      const int i = idx / D, c = idx % D;
+      const float g = sGm[i * DP + c];
+      gE[i * DP + c] = g * sE[i * DP + c];
+      gQ[i * DP + c] = g * sQ[i * DP + c];
+      gK[i * DP + c] = sK[i * DP + c] * sBk[i * DP + c];
+    }
+  };
   // A = (I + T)⁻¹ by forward substitution, one column per thread; R = Z − Ē S.
   auto inverse_and_R = [&]() {
     if (tid < BC) {
@@ -203,12 +219,27 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
         sA[i * CP + j] = x;
       }
     }
-    for (int idx = tid; idx < BC * DVT; idx += BT) {
-      const int i = idx / DVT, v = idx % DVT;
-      float acc = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) acc = fmaf(sGm[i * DP + c] * sE[i * DP + c], sS[c * VP + v], acc);
-      tZ[i * VP + v] -= acc;
+    {
+      float acc[2][NV] = {};
+#pragma unroll 4
+      for (int c = 0; c < D; ++c) {
+        const float e0 = gE[r2 * DP + c], e1 = gE[(r2 + 1) * DP + c];
+#pragma unroll
+        for (int n = 0; n < NV; ++n) {
+          const int v = lane + 32 * n;
+          const float sv = v < DVT ? sS[c * VP + v] : 0.f;
+          acc[0][n] = fmaf(e0, sv, acc[0][n]);
+          acc[1][n] = fmaf(e1, sv, acc[1][n]);
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < NV; ++n) {
+        const int v = lane + 32 * n;
+        if (v < DVT) {
+          tZ[r2 * VP + v] -= acc[0][n];
+          tZ[(r2 + 1) * VP + v] -= acc[1][n];
+        }
+      }
     }
   };
   // U = A R
@@ -236,16 +267,39 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     __syncthreads();
     decays_and_gram();
     __syncthreads();
+    absorbed();
+    __syncthreads();
     inverse_and_R();
     __syncthreads();
     solve_U();
     __syncthreads();
-    // S ← Γ S + K_endᵀ U
-    for (int idx = tid; idx < D * DVT; idx += BT) {
-      const int r = idx / DVT, v = idx % DVT;
-      float acc = sgC[r] * sS[r * VP + v];
-      for (int j = 0; j < BC; ++j) acc = fmaf(sK[j * DP + r] * sBk[j * DP + r], tU[j * VP + v], acc);
-      sS[r * VP + v] = acc;
+    // S ← Γ S + K_endᵀ U (each thread updates its own entries in place)
+    for (int r0 = 16 * warp; r0 < D; r0 += 16 * (BT / 32)) {
+      float acc[16][NV];
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+#pragma unroll
+        for (int n = 0; n < NV; ++n) {
+          const int v = lane + 32 * n;
+          acc[m][n] = v < DVT ? sgC[r0 + m] * sS[(r0 + m) * VP + v] : 0.f;
+        }
+#pragma unroll 4
+      for (int j = 0; j < BC; ++j) {
+        float u[NV];
+#pragma unroll
+        for (int n = 0; n < NV; ++n) u[n] = lane + 32 * n < DVT ? tU[j * VP + lane + 32 * n] : 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float ke = gK[j * DP + r0 + m];
+#pragma unroll
+          for (int n = 0; n < NV; ++n) acc[m][n] = fmaf(ke, u[n], acc[m][n]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+#pragma unroll
+        for (int n = 0; n < NV; ++n)
+          if (lane + 32 * n < DVT) sS[(r0 + m) * VP + lane + 32 * n] = acc[m][n];
     }
   }
 
@@ -268,19 +322,44 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     __syncthreads();
     decays_and_gram();
     __syncthreads();
+    absorbed();
+    __syncthreads();
     inverse_and_R();
     __syncthreads();
     solve_U();
     __syncthreads();
     // dU = s Aqkᵀ dO + K_end dS'
-    for (int idx = tid; idx < BC * DVT; idx += BT) {
-      const int j = idx / DVT, v = idx % DVT;
-      float acc = 0.f;
-      for (int i = j; i < BC; ++i) acc = fmaf(sAq[i * CP + j], tdO[i * VP + v], acc);
-      acc *= s;
-#pragma unroll 8
-      for (int cc = 0; cc < D; ++cc) acc = fmaf(sK[j * DP + cc] * sBk[j * DP + cc], dSp[cc * VP + v], acc);
-      tdU[j * VP + v] = acc;
+    {
+      float aq[2][NV] = {}, ak[2][NV] = {};
+      for (int i = r2; i < BC; ++i) {
+        const float a0 = sAq[i * CP + r2], a1 = i > r2 ? sAq[i * CP + r2 + 1] : 0.f;
+#pragma unroll
+        for (int n = 0; n < NV; ++n) {
+          const int v = lane + 32 * n;
+          const float d = v < DVT ? tdO[i * VP + v] : 0.f;
+          aq[0][n] = fmaf(a0, d, aq[0][n]);
+          aq[1][n] = fmaf(a1, d, aq[1][n]);
+        }
+      }
+#pragma unroll 4
+      for (int cc = 0; cc < D; ++cc) {
+        const float k0 = gK[r2 * DP + cc], k1 = gK[(r2 + 1) * DP + cc];
+#pragma unroll
+        for (int n = 0; n < NV; ++n) {
+          const int v = lane + 32 * n;
+          const float p = v < DVT ? dSp[cc * VP + v] : 0.f;
+          ak[0][n] = fmaf(k0, p, ak[0][n]);
+          ak[1][n] = fmaf(k1, p, ak[1][n]);
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < NV; ++n) {
+        const int v = lane + 32 * n;
+        if (v < DVT) {
+          tdU[r2 * VP + v] = fmaf(s, aq[0][n], ak[0][n]);
+          tdU[(r2 + 1) * VP + v] = fmaf(s, aq[1][n], ak[1][n]);
+        }
+      }
     }
     __syncthreads();
     // dR = Aᵀ dU, into the R array
@@ -292,14 +371,37 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     }
     __syncthreads();
     float* tdR = tZ;
-    // dS of the entry state
-    for (int idx = tid; idx < D * DVT; idx += BT) {
-      const int r = idx / DVT, v = idx % DVT;
-      float acc = 0.f;
-      for (int i = 0; i < BC; ++i)
-        acc = fmaf(sGm[i * DP + r], fmaf(s * sQ[i * DP + r], tdO[i * VP + v], -sE[i * DP + r] * tdR[i * VP + v]),
-                   acc);
-      dSn[r * VP + v] = fmaf(sgC[r], dSp[r * VP + v], acc);
+    // dS of the entry state: Γ dS' + s Q̄ᵀ dO − Ēᵀ dR
+    for (int r0 = 16 * warp; r0 < D; r0 += 16 * (BT / 32)) {
+      float acc[16][NV];
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+#pragma unroll
+        for (int n = 0; n < NV; ++n) {
+          const int v = lane + 32 * n;
+          acc[m][n] = v < DVT ? sgC[r0 + m] * dSp[(r0 + m) * VP + v] : 0.f;
+        }
+#pragma unroll 2
+      for (int i = 0; i < BC; ++i) {
+        float od[NV], rd[NV];
+#pragma unroll
+        for (int n = 0; n < NV; ++n) {
+          const int v = lane + 32 * n;
+          od[n] = v < DVT ? s * tdO[i * VP + v] : 0.f;
+          rd[n] = v < DVT ? tdR[i * VP + v] : 0.f;
+        }
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float qb = gQ[i * DP + r0 + m], eb = gE[i * DP + r0 + m];
+#pragma unroll
+          for (int n = 0; n < NV; ++n) acc[m][n] = fmaf(qb, od[n], fmaf(-eb, rd[n], acc[m][n]));
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+#pragma unroll
+        for (int n = 0; n < NV; ++n)
+          if (lane + 32 * n < DVT) dSn[(r0 + m) * VP + lane + 32 * n] = acc[m][n];
     }
     // dv = dR ⊙ w; dw = dR ⊙ v (per channel), or its sum into dβ (tied gates)
     for (int idx = tid; idx < BC * DVT; idx += BT) {
@@ -339,24 +441,40 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
       sdAq[i * CP + j] = j <= i ? s * y : 0.f;
     }
     // per (i, c): dQ̄ = s dO Sᵀ, dĒ = −dR Sᵀ, dK_end = U dS'ᵀ, and what they give
-    // q, e, k and G directly
-    for (int idx = tid; idx < BC * D; idx += BT) {
-      const int i = idx / D, cc = idx % D;
-      float dq_ = 0.f, de_ = 0.f, dke = 0.f;
-#pragma unroll 8
+    // q, e, k and G directly (after every thread's last read of Q̄, Ē, K_end)
+    __syncthreads();
+    {
+      float aq[2][NK] = {}, ae[2][NK] = {}, ak[2][NK] = {};
+#pragma unroll 2
       for (int v = 0; v < DVT; ++v) {
-        const float sv = sS[cc * VP + v];
-        dq_ = fmaf(tdO[i * VP + v], sv, dq_);
-        de_ = fmaf(tdR[i * VP + v], sv, de_);
-        dke = fmaf(tU[i * VP + v], dSp[cc * VP + v], dke);
+        const float o0 = tdO[r2 * VP + v], o1 = tdO[(r2 + 1) * VP + v];
+        const float d0 = tdR[r2 * VP + v], d1 = tdR[(r2 + 1) * VP + v];
+        const float u0 = tU[r2 * VP + v], u1 = tU[(r2 + 1) * VP + v];
+#pragma unroll
+        for (int n = 0; n < NK; ++n) {
+          const int cc = lane + 32 * n;
+          const float sv = cc < D ? sS[cc * VP + v] : 0.f, pv = cc < D ? dSp[cc * VP + v] : 0.f;
+          aq[0][n] = fmaf(o0, sv, aq[0][n]);
+          aq[1][n] = fmaf(o1, sv, aq[1][n]);
+          ae[0][n] = fmaf(d0, sv, ae[0][n]);
+          ae[1][n] = fmaf(d1, sv, ae[1][n]);
+          ak[0][n] = fmaf(u0, pv, ak[0][n]);
+          ak[1][n] = fmaf(u1, pv, ak[1][n]);
+        }
       }
-      dq_ *= s;
-      de_ = -de_;
-      const float g = sGm[i * DP + cc], bk = sBk[i * DP + cc];
-      gQ[i * DP + cc] = g * dq_;
-      gE[i * DP + cc] = g * de_;
-      gK[i * DP + cc] = bk * dke;
-      gG[i * DP + cc] = g * (sQ[i * DP + cc] * dq_ + sE[i * DP + cc] * de_) - sK[i * DP + cc] * bk * dke;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int n = 0; n < NK; ++n) {
+          const int i = r2 + h2, cc = lane + 32 * n;
+          if (cc >= D) continue;
+          const float dq_ = s * aq[h2][n], de_ = -ae[h2][n], dke = ak[h2][n];
+          const float g = sGm[i * DP + cc], bk = sBk[i * DP + cc];
+          gQ[i * DP + cc] = g * dq_;
+          gE[i * DP + cc] = g * de_;
+          gK[i * DP + cc] = bk * dke;
+          gG[i * DP + cc] = g * (sQ[i * DP + cc] * dq_ + sE[i * DP + cc] * de_) - sK[i * DP + cc] * bk * dke;
+        }
     }
     __syncthreads();
     // G at the chunk's last token: from K_end (Σ_j K_end,j ⊙ dK_end,j) and Γ
