@@ -41,9 +41,9 @@ constexpr int BT = 256;       // threads
 template <int D>
 struct BwdSmem {
   static constexpr int DVT = D < 64 ? D : 64;   // value columns per CTA
-  static constexpr int DP = D + 1;              // row strides (padded against bank conflicts)
+  static constexpr int DP = D + 4;              // key rows: 16-byte multiples (broadcast rows load as float4)
   static constexpr int CP = BC + 1;
-  static constexpr int VP = DVT + 1;
+  static constexpr int VP = DVT + 1;            // (odd: column walks across lanes are conflict-free)
   // [BC][DP] ×11: q, k, b, α, e, γ, bk (Π_{i<s<BC} α), and the gradients of q, k, e, G
   // [BC][CP] ×5:  T, A = (I+T)⁻¹, Aqk, dT, dAqk
   // [BC][VP] ×6:  Z (then R, then dR), U, dO, dU, v, w
@@ -221,16 +221,20 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     }
     {
       float acc[2][NV] = {};
-#pragma unroll 4
-      for (int c = 0; c < D; ++c) {
-        const float e0 = gE[r2 * DP + c], e1 = gE[(r2 + 1) * DP + c];
+#pragma unroll 2
+      for (int c4 = 0; c4 < D; c4 += 4) {
+        const float4 e0 = *reinterpret_cast<const float4*>(gE + r2 * DP + c4);
+        const float4 e1 = *reinterpret_cast<const float4*>(gE + (r2 + 1) * DP + c4);
+        const float a0[4] = {e0.x, e0.y, e0.z, e0.w}, a1[4] = {e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-        for (int n = 0; n < NV; ++n) {
-          const int v = lane + 32 * n;
-          const float sv = v < DVT ? sS[c * VP + v] : 0.f;
-          acc[0][n] = fmaf(e0, sv, acc[0][n]);
-          acc[1][n] = fmaf(e1, sv, acc[1][n]);
-        }
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int n = 0; n < NV; ++n) {
+            const int v = lane + 32 * n;
+            const float sv = v < DVT ? sS[(c4 + t) * VP + v] : 0.f;
+            acc[0][n] = fmaf(a0[t], sv, acc[0][n]);
+            acc[1][n] = fmaf(a1[t], sv, acc[1][n]);
+          }
       }
 #pragma unroll
       for (int n = 0; n < NV; ++n) {
@@ -289,10 +293,13 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
 #pragma unroll
         for (int n = 0; n < NV; ++n) u[n] = lane + 32 * n < DVT ? tU[j * VP + lane + 32 * n] : 0.f;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float ke = gK[j * DP + r0 + m];
+        for (int m4 = 0; m4 < 16; m4 += 4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(gK + j * DP + r0 + m4);
+          const float ke[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-          for (int n = 0; n < NV; ++n) acc[m][n] = fmaf(ke, u[n], acc[m][n]);
+          for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int n = 0; n < NV; ++n) acc[m4 + t][n] = fmaf(ke[t], u[n], acc[m4 + t][n]);
         }
       }
 #pragma unroll
@@ -341,16 +348,20 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
           aq[1][n] = fmaf(a1, d, aq[1][n]);
         }
       }
-#pragma unroll 4
-      for (int cc = 0; cc < D; ++cc) {
-        const float k0 = gK[r2 * DP + cc], k1 = gK[(r2 + 1) * DP + cc];
+#pragma unroll 2
+      for (int c4 = 0; c4 < D; c4 += 4) {
+        const float4 q0 = *reinterpret_cast<const float4*>(gK + r2 * DP + c4);
+        const float4 q1 = *reinterpret_cast<const float4*>(gK + (r2 + 1) * DP + c4);
+        const float k0[4] = {q0.x, q0.y, q0.z, q0.w}, k1[4] = {q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-        for (int n = 0; n < NV; ++n) {
-          const int v = lane + 32 * n;
-          const float p = v < DVT ? dSp[cc * VP + v] : 0.f;
-          ak[0][n] = fmaf(k0, p, ak[0][n]);
-          ak[1][n] = fmaf(k1, p, ak[1][n]);
-        }
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int n = 0; n < NV; ++n) {
+            const int v = lane + 32 * n;
+            const float p = v < DVT ? dSp[(c4 + t) * VP + v] : 0.f;
+            ak[0][n] = fmaf(k0[t], p, ak[0][n]);
+            ak[1][n] = fmaf(k1[t], p, ak[1][n]);
+          }
       }
 #pragma unroll
       for (int n = 0; n < NV; ++n) {
@@ -391,10 +402,14 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
           rd[n] = v < DVT ? tdR[i * VP + v] : 0.f;
         }
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float qb = gQ[i * DP + r0 + m], eb = gE[i * DP + r0 + m];
+        for (int m4 = 0; m4 < 16; m4 += 4) {
+          const float4 q4 = *reinterpret_cast<const float4*>(gQ + i * DP + r0 + m4);
+          const float4 e4 = *reinterpret_cast<const float4*>(gE + i * DP + r0 + m4);
+          const float qb[4] = {q4.x, q4.y, q4.z, q4.w}, eb[4] = {e4.x, e4.y, e4.z, e4.w};
 #pragma unroll
-          for (int n = 0; n < NV; ++n) acc[m][n] = fmaf(qb, od[n], fmaf(-eb, rd[n], acc[m][n]));
+          for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int n = 0; n < NV; ++n) acc[m4 + t][n] = fmaf(qb[t], od[n], fmaf(-eb[t], rd[n], acc[m4 + t][n]));
         }
       }
 #pragma unroll
