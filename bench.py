@@ -49,14 +49,15 @@ CONV = "conv_prefill_b8_t8192"
 L2_BYTES = 126 * 2**20
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the prefill
-# launches of one call (4 segments: a prep and a scan each), from a
-# single-pass ncu capture of the T=32768 workload itself, and the hash of the
-# kernel sources it was taken on; with other sources the figure is stale and
-# the bench reports null.
+# launches of one T=32768 call, and the hash of the kernel sources they were
+# taken on (with other sources the figure is stale and the bench reports
+# null). Taken on the T=4096 case (its 2 segments' prep and scan launches,
+# 802.7 MB per call, 1.83x its algorithmic bytes) and scaled by the chunk
+# count (x8): the slot round trip, which is most of the excess, grows with the
+# chunks; the full-size workload is too large for a multi-metric capture.
 TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
-TRAFFIC = {"sha1": "c303dc6434ed4a50c5ec5cd8cd600ff47ced5b3c",
-           # reads 4.931 GB + writes 2.004 GB over the 8 launches of one call
-           "bytes_per_call": 6_934_368_512}
+TRAFFIC = {"sha1": "e7fd5b49375afc63974a1fc38c686b788b5f1654",
+           "bytes_per_call": 6421860352}
 
 
 def peaks():
@@ -367,6 +368,8 @@ def main():
                     help="with N > 1 ranks: timed calls of the T=32768 layer with its heads split across the "
                          "ranks (H_qk/N QK heads and the value heads that read them per rank, strong scaling); "
                          "0 skips it")
+    ap.add_argument("--bwd-workload", default=CONV, choices=[CONV, "prefill_t4096"],
+                    help="backward workload (the small one is for profiler captures)")
     ap.add_argument("--bwd-steps", type=int, default=3,
                     help="timed calls of the backward pass on the B=8, T=8192 training shape; 0 skips it")
     args = ap.parse_args()
@@ -700,13 +703,14 @@ def alu_peak_tflops(dev):
 def run_bwd(args, dev, stream, barrier, pk, world):
     """The backward pass (gdn2_chunk_bwd) on the training-shape workload: B=8,
     T=8192, 48 V heads, the recurrence's inputs (unit q, k), nonzero S0,
-    upstream gradients of o (bf16) and of S_T."""
+    upstream gradients of o (bf16) and of S_T (or, for profiler captures, the
+    T=4096 layer)."""
     import torch
     from dataclasses import replace
     from delta_rule_linear_gdn_b200 import gdn2
     from delta_rule_linear_gdn_b200.inputs import make_inputs, workload
     rank = int(os.environ.get("RANK", "0"))
-    bw = replace(workload(CONV), conv=False)
+    bw = replace(workload(args.bwd_workload), conv=False)
     inp = make_inputs(bw, seed=rank_seed(rank), device=dev)
     g = torch.Generator(device=dev)
     g.manual_seed(21)
