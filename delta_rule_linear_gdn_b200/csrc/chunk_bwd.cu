@@ -36,7 +36,7 @@ namespace gdn2 {
 namespace {
 
 constexpr int BC = 16;        // chunk of the backward pass
-constexpr int BT = 256;       // threads
+constexpr int BT = 512;       // threads (16 warps: one CTA per SM for its shared memory)
 
 template <int D>
 struct BwdSmem {
@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
   using L = BwdSmem<D>;
   constexpr int DVT = L::DVT, DP = L::DP, CP = L::CP, VP = L::VP;
   constexpr int TILES = D / DVT;
-  constexpr int CPT = D / 16;   // channels per thread of the pairwise passes
+  constexpr int CPT = (D + 31) / 32;   // channels per lane of the pairwise passes (one warp per row)
   extern __shared__ float sm[];
   float* sQ = sm;
   float* sK = sQ + BC * DP;
@@ -160,40 +160,51 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
         p *= sAl[i * DP + c];
       }
     }
-    const int j = tid >> 4, part = tid & 15;
+    // warp j takes key row j, lane l its channels l + 32 m
+    const int j = warp, part = lane;
     float kj[CPT], dd[CPT];
 #pragma unroll
     for (int m = 0; m < CPT; ++m) {
-      kj[m] = sK[j * DP + part + 16 * m];
+      kj[m] = part + 32 * m < D ? sK[j * DP + part + 32 * m] : 0.f;
       dd[m] = 1.f;
     }
-    for (int i = warp * 2; i < BC; ++i) {
+    for (int i = j; i < BC; ++i) {
       float at = 0.f, aa = 0.f;
 #pragma unroll
       for (int m = 0; m < CPT; ++m) {
-        const int c = part + 16 * m;
-        dd[m] *= i > j ? sAl[i * DP + c] : 1.f;
-        const float kd = kj[m] * dd[m];
-        at = fmaf(sE[i * DP + c], kd, at);
-        aa = fmaf(sQ[i * DP + c], kd, aa);
+        const int c = part + 32 * m;
+        if (c < D) {
+          dd[m] *= i > j ? sAl[i * DP + c] : 1.f;
+          const float kd = kj[m] * dd[m];
+          at = fmaf(sE[i * DP + c], kd, at);
+          aa = fmaf(sQ[i * DP + c], kd, aa);
+        }
       }
 #pragma unroll
-      for (int off = 1; off < 16; off <<= 1) {
+      for (int off = 1; off < 32; off <<= 1) {
         at += __shfl_xor_sync(0xffffffffu, at, off);
         aa += __shfl_xor_sync(0xffffffffu, aa, off);
       }
-      if (part == 0 && i >= j) {
+      if (part == 0) {
         sT[i * CP + j] = i > j ? at : 0.f;
         sAq[i * CP + j] = aa;
       }
     }
   };
 
-  // Register tiles of the products below: warp w takes rows 2w, 2w + 1 of a
-  // BC-row result (or rows 16w .. 16w + 15 of a D-row one), lane l the value
-  // columns l, l + 32 (NV of them) or key columns l + 32 n (NK).
+  // Register tiles of the products below. A BC-row result: warp w takes rows
+  // 2(w mod 8), 2(w mod 8) + 1 and, with lane l, the value columns
+  // l + 32(w/8 + 2n) (NVH of them) or key columns l + 32(w/8 + 2n) (NKH). A
+  // D-row result: warp w takes rows RW·w .. RW·w + RW − 1 and lane l the value
+  // columns l + 32n (NV).
+  constexpr int NW = BT / 32;
   constexpr int NV = (DVT + 31) / 32, NK = (D + 31) / 32;
-  const int r2 = 2 * warp;
+  constexpr int NVH = (NV + 1) / 2, NKH = (NK + 1) / 2;
+  constexpr int RW = D / NW > 0 ? D / NW : 1;
+  static_assert(BC == 16 && NW == 16, "row tiles assume 16 rows and 16 warps");
+  const int r2 = 2 * (warp & 7), wh = warp >> 3;
+  auto vcol = [&](int n) { return lane + 32 * (wh + 2 * n); };
+  auto kcol = [&](int n) { return lane + 32 * (wh + 2 * n); };
   // Ē = γ ⊙ e, Q̄ = γ ⊙ q and K_end = k ⊙ bk, into the gradient arrays, which
   // the backward sweep rewrites only after their last use.
   auto absorbed = [&]() {
@@ -220,7 +231,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
       }
     }
     {
-      float acc[2][NV] = {};
+      float acc[2][NVH] = {};
 #pragma unroll 2
       for (int c4 = 0; c4 < D; c4 += 4) {
         const float4 e0 = *reinterpret_cast<const float4*>(gE + r2 * DP + c4);
@@ -229,16 +240,16 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-          for (int n = 0; n < NV; ++n) {
-            const int v = lane + 32 * n;
+          for (int n = 0; n < NVH; ++n) {
+            const int v = vcol(n);
             const float sv = v < DVT ? sS[(c4 + t) * VP + v] : 0.f;
             acc[0][n] = fmaf(a0[t], sv, acc[0][n]);
             acc[1][n] = fmaf(a1[t], sv, acc[1][n]);
           }
       }
 #pragma unroll
-      for (int n = 0; n < NV; ++n) {
-        const int v = lane + 32 * n;
+      for (int n = 0; n < NVH; ++n) {
+        const int v = vcol(n);
         if (v < DVT) {
           tZ[r2 * VP + v] -= acc[0][n];
           tZ[(r2 + 1) * VP + v] -= acc[1][n];
@@ -278,10 +289,10 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     solve_U();
     __syncthreads();
     // S ← Γ S + K_endᵀ U (each thread updates its own entries in place)
-    for (int r0 = 16 * warp; r0 < D; r0 += 16 * (BT / 32)) {
-      float acc[16][NV];
+    for (int r0 = RW * warp; r0 < D; r0 += RW * NW) {
+      float acc[RW][NV];
 #pragma unroll
-      for (int m = 0; m < 16; ++m)
+      for (int m = 0; m < RW; ++m)
 #pragma unroll
         for (int n = 0; n < NV; ++n) {
           const int v = lane + 32 * n;
@@ -293,17 +304,14 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
 #pragma unroll
         for (int n = 0; n < NV; ++n) u[n] = lane + 32 * n < DVT ? tU[j * VP + lane + 32 * n] : 0.f;
 #pragma unroll
-        for (int m4 = 0; m4 < 16; m4 += 4) {
-          const float4 k4 = *reinterpret_cast<const float4*>(gK + j * DP + r0 + m4);
-          const float ke[4] = {k4.x, k4.y, k4.z, k4.w};
+        for (int m = 0; m < RW; ++m) {
+          const float ke = gK[j * DP + r0 + m];
 #pragma unroll
-          for (int t = 0; t < 4; ++t)
-#pragma unroll
-            for (int n = 0; n < NV; ++n) acc[m4 + t][n] = fmaf(ke[t], u[n], acc[m4 + t][n]);
+          for (int n = 0; n < NV; ++n) acc[m][n] = fmaf(ke, u[n], acc[m][n]);
         }
       }
 #pragma unroll
-      for (int m = 0; m < 16; ++m)
+      for (int m = 0; m < RW; ++m)
 #pragma unroll
         for (int n = 0; n < NV; ++n)
           if (lane + 32 * n < DVT) sS[(r0 + m) * VP + lane + 32 * n] = acc[m][n];
@@ -337,12 +345,12 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     __syncthreads();
     // dU = s Aqkᵀ dO + K_end dS'
     {
-      float aq[2][NV] = {}, ak[2][NV] = {};
+      float aq[2][NVH] = {}, ak[2][NVH] = {};
       for (int i = r2; i < BC; ++i) {
         const float a0 = sAq[i * CP + r2], a1 = i > r2 ? sAq[i * CP + r2 + 1] : 0.f;
 #pragma unroll
-        for (int n = 0; n < NV; ++n) {
-          const int v = lane + 32 * n;
+        for (int n = 0; n < NVH; ++n) {
+          const int v = vcol(n);
           const float d = v < DVT ? tdO[i * VP + v] : 0.f;
           aq[0][n] = fmaf(a0, d, aq[0][n]);
           aq[1][n] = fmaf(a1, d, aq[1][n]);
@@ -356,16 +364,16 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-          for (int n = 0; n < NV; ++n) {
-            const int v = lane + 32 * n;
+          for (int n = 0; n < NVH; ++n) {
+            const int v = vcol(n);
             const float p = v < DVT ? dSp[(c4 + t) * VP + v] : 0.f;
             ak[0][n] = fmaf(k0[t], p, ak[0][n]);
             ak[1][n] = fmaf(k1[t], p, ak[1][n]);
           }
       }
 #pragma unroll
-      for (int n = 0; n < NV; ++n) {
-        const int v = lane + 32 * n;
+      for (int n = 0; n < NVH; ++n) {
+        const int v = vcol(n);
         if (v < DVT) {
           tdU[r2 * VP + v] = fmaf(s, aq[0][n], ak[0][n]);
           tdU[(r2 + 1) * VP + v] = fmaf(s, aq[1][n], ak[1][n]);
@@ -383,10 +391,10 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     __syncthreads();
     float* tdR = tZ;
     // dS of the entry state: Γ dS' + s Q̄ᵀ dO − Ēᵀ dR
-    for (int r0 = 16 * warp; r0 < D; r0 += 16 * (BT / 32)) {
-      float acc[16][NV];
+    for (int r0 = RW * warp; r0 < D; r0 += RW * NW) {
+      float acc[RW][NV];
 #pragma unroll
-      for (int m = 0; m < 16; ++m)
+      for (int m = 0; m < RW; ++m)
 #pragma unroll
         for (int n = 0; n < NV; ++n) {
           const int v = lane + 32 * n;
@@ -402,18 +410,14 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
           rd[n] = v < DVT ? tdR[i * VP + v] : 0.f;
         }
 #pragma unroll
-        for (int m4 = 0; m4 < 16; m4 += 4) {
-          const float4 q4 = *reinterpret_cast<const float4*>(gQ + i * DP + r0 + m4);
-          const float4 e4 = *reinterpret_cast<const float4*>(gE + i * DP + r0 + m4);
-          const float qb[4] = {q4.x, q4.y, q4.z, q4.w}, eb[4] = {e4.x, e4.y, e4.z, e4.w};
+        for (int m = 0; m < RW; ++m) {
+          const float qb = gQ[i * DP + r0 + m], eb = gE[i * DP + r0 + m];
 #pragma unroll
-          for (int t = 0; t < 4; ++t)
-#pragma unroll
-            for (int n = 0; n < NV; ++n) acc[m4 + t][n] = fmaf(qb[t], od[n], fmaf(-eb[t], rd[n], acc[m4 + t][n]));
+          for (int n = 0; n < NV; ++n) acc[m][n] = fmaf(qb, od[n], fmaf(-eb, rd[n], acc[m][n]));
         }
       }
 #pragma unroll
-      for (int m = 0; m < 16; ++m)
+      for (int m = 0; m < RW; ++m)
 #pragma unroll
         for (int n = 0; n < NV; ++n)
           if (lane + 32 * n < DVT) dSn[(r0 + m) * VP + lane + 32 * n] = acc[m][n];
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
       }
     }
     // dT, dAqk
-    {
+    if (tid < BC * BC) {
       const int i = tid >> 4, j = tid & 15;
       float x = 0.f, y = 0.f;
       if (j <= i) {
@@ -459,15 +463,15 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     // q, e, k and G directly (after every thread's last read of Q̄, Ē, K_end)
     __syncthreads();
     {
-      float aq[2][NK] = {}, ae[2][NK] = {}, ak[2][NK] = {};
+      float aq[2][NKH] = {}, ae[2][NKH] = {}, ak[2][NKH] = {};
 #pragma unroll 2
       for (int v = 0; v < DVT; ++v) {
         const float o0 = tdO[r2 * VP + v], o1 = tdO[(r2 + 1) * VP + v];
         const float d0 = tdR[r2 * VP + v], d1 = tdR[(r2 + 1) * VP + v];
         const float u0 = tU[r2 * VP + v], u1 = tU[(r2 + 1) * VP + v];
 #pragma unroll
-        for (int n = 0; n < NK; ++n) {
-          const int cc = lane + 32 * n;
+        for (int n = 0; n < NKH; ++n) {
+          const int cc = kcol(n);
           const float sv = cc < D ? sS[cc * VP + v] : 0.f, pv = cc < D ? dSp[cc * VP + v] : 0.f;
           aq[0][n] = fmaf(o0, sv, aq[0][n]);
           aq[1][n] = fmaf(o1, sv, aq[1][n]);
@@ -480,8 +484,8 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-        for (int n = 0; n < NK; ++n) {
-          const int i = r2 + h2, cc = lane + 32 * n;
+        for (int n = 0; n < NKH; ++n) {
+          const int i = r2 + h2, cc = kcol(n);
           if (cc >= D) continue;
           const float dq_ = s * aq[h2][n], de_ = -ae[h2][n], dke = ak[h2][n];
           const float g = sGm[i * DP + cc], bk = sBk[i * DP + cc];
@@ -504,37 +508,41 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
     __syncthreads();
     // Gram gradients, key side: thread (j, part) runs i up from j with D_ij
     {
-      const int j = tid >> 4, part = tid & 15;
+      const int j = warp, part = lane;   // warp j: key row j, lane l: channels l + 32 m
       float dd[CPT], ak[CPT], ag[CPT], kj[CPT];
 #pragma unroll
       for (int m = 0; m < CPT; ++m) {
         dd[m] = 1.f;
         ak[m] = 0.f;
         ag[m] = 0.f;
-        kj[m] = sK[j * DP + part + 16 * m];
+        kj[m] = part + 32 * m < D ? sK[j * DP + part + 32 * m] : 0.f;
       }
       for (int i = j; i < BC; ++i) {
         const float ct = sdT[i * CP + j], ca = sdAq[i * CP + j];
 #pragma unroll
         for (int m = 0; m < CPT; ++m) {
-          const int cc = part + 16 * m;
-          dd[m] *= i > j ? sAl[i * DP + cc] : 1.f;
-          const float x = fmaf(ct, sE[i * DP + cc], ca * sQ[i * DP + cc]) * dd[m];
-          ak[m] += x;
-          ag[m] = fmaf(x, kj[m], ag[m]);
+          const int cc = part + 32 * m;
+          if (cc < D) {
+            dd[m] *= i > j ? sAl[i * DP + cc] : 1.f;
+            const float x = fmaf(ct, sE[i * DP + cc], ca * sQ[i * DP + cc]) * dd[m];
+            ak[m] += x;
+            ag[m] = fmaf(x, kj[m], ag[m]);
+          }
         }
       }
 #pragma unroll
       for (int m = 0; m < CPT; ++m) {
-        const int cc = part + 16 * m;
-        gK[j * DP + cc] += ak[m];
-        gG[j * DP + cc] -= ag[m];
+        const int cc = part + 32 * m;
+        if (cc < D) {
+          gK[j * DP + cc] += ak[m];
+          gG[j * DP + cc] -= ag[m];
+        }
       }
     }
     __syncthreads();
     // query / erase side: thread (i, part) runs j down from i with D_ij
     {
-      const int i = tid >> 4, part = tid & 15;
+      const int i = warp, part = lane;   // warp i: row i, lane l: channels l + 32 m
       float dd[CPT], ae[CPT], aq[CPT], ag[CPT];
 #pragma unroll
       for (int m = 0; m < CPT; ++m) {
@@ -547,16 +555,19 @@ __global__ void __launch_bounds__(BT, 1) chunk_bwd_kernel(BwdArgs a) {
         const float ct = sdT[i * CP + j], ca = sdAq[i * CP + j];
 #pragma unroll
         for (int m = 0; m < CPT; ++m) {
-          const int cc = part + 16 * m;
-          if (j < i) dd[m] *= sAl[(j + 1) * DP + cc];
-          const float kd = sK[j * DP + cc] * dd[m];
-          ae[m] = fmaf(ct, kd, ae[m]);
-          aq[m] = fmaf(ca, kd, aq[m]);
+          const int cc = part + 32 * m;
+          if (cc < D) {
+            if (j < i) dd[m] *= sAl[(j + 1) * DP + cc];
+            const float kd = sK[j * DP + cc] * dd[m];
+            ae[m] = fmaf(ct, kd, ae[m]);
+            aq[m] = fmaf(ca, kd, aq[m]);
+          }
         }
       }
 #pragma unroll
       for (int m = 0; m < CPT; ++m) {
-        const int cc = part + 16 * m;
+        const int cc = part + 32 * m;
+        if (cc >= D) continue;
         ag[m] = fmaf(ae[m], sE[i * DP + cc], aq[m] * sQ[i * DP + cc]);
         gE[i * DP + cc] += ae[m];
         gQ[i * DP + cc] += aq[m];
