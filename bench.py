@@ -110,19 +110,16 @@ def decode_bytes(w, o_bytes=2):
 def tc_launches_per_call(w, ws_bytes, dev):
     """Kernel launches of one gdn2_chunk_fwd call of workload w with S_T given
     and the whole sequence in the workspace, by the launcher's rules: the scan
-    runs 2·B·H_v half-width CTAs, or B·H_v full-width ones when the half-width
-    grid would need ≥ 5/3 as many waves; when the scan grid leaves SMs idle,
-    and the sequence has at least 64 chunks, the call pipelines 2 to 4
-    segments, else it runs one segment; a segment is a prep (with the conv
-    and L2 norm in its load when asked for), the exact kernel for strongly
-    decaying chunks and a scan. The SIMT path (no workspace) is one launch."""
+    runs one CTA per (sequence, value head); when that leaves SMs idle and the
+    sequence has at least 64 chunks, the call pipelines 2 to 4 segments, else
+    it runs one segment; a segment is a prep (with the conv and L2 norm in
+    its load when asked for), the exact kernel for strongly decaying chunks
+    and a scan. The SIMT path (no workspace) is one launch."""
     if ws_bytes == 0:
         return 1
     import torch
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    bh = w.B * w.H_v
-    waves_half, waves_full = -(-2 * bh // sms), -(-bh // sms)
-    scan_ctas = bh if 5 * waves_full < 3 * waves_half else 2 * bh
+    scan_ctas = w.B * w.H_v
     nchunks = (w.T + 63) // 64
     if nchunks >= 64 and scan_ctas < sms:
         return 3 * min(4, nchunks // 32)

@@ -328,10 +328,10 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_params* p, const void* q, const
  *              host sees the reservation then, and an out-of-memory error
  *              surfaces there. The sequence is processed in segments of as
  *              many 64-token chunks as the array holds for all B·H_v
- *              sequence-heads (73 KB per chunk and sequence-head, plus, with
- *              the conv or the L2 norm, the fp16 copies of the chunk's q, k, v
- *              for all sequences: 9 chunks for B·H_v = 48 without them), so
- *              long sequences take more launches than gdn2_chunk_fwd. Each
+ *              sequence-heads (73 KB per chunk and sequence-head, with or
+ *              without the conv and the L2 norm, which run inside the prep:
+ *              9 chunks for B·H_v = 48), so long sequences take more launches
+ *              than gdn2_chunk_fwd. Each
  *              call clears the status word it uses before its launches;
  *              nothing else in the array needs to start at zero.
  *   Sharing:   every call on a device uses the same array, so calls whose

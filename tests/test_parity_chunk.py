@@ -93,8 +93,8 @@ def test_bf16_d128_chunk64(gate_mode):
 
 @pytest.mark.parametrize("conv,gate_mode", [(True, "full"), (False, "full"), (True, "kda"), (True, "gdn")])
 def test_bf16_d128_conv_and_l2norm_tensor_core(conv, gate_mode):
-    """The load step (depthwise causal conv, L2 norm of q, k) ahead of the
-    tensor-core prefill: two sequences with a ragged tail, so the conv history
+    """The depthwise causal conv and the L2 norm of q, k in the tensor-core
+    prep's load: two sequences with a ragged tail, so the conv history
     crosses chunk boundaries but never sequence boundaries; all gate layouts."""
     w = small(T=200, B=2, H_qk=2, H_v=6, d=128, chunk=64, qkv="bf16", s0="normal", conv=True)
     inp = make_inputs(w, seed=31, gate_mode=gate_mode)
@@ -178,10 +178,9 @@ def test_overlapped_segments_match_one_pass_and_oracle():
 
 
 @pytest.mark.parametrize("gate_mode", ["full", "gdn"])
-def test_full_width_scan_many_heads(gate_mode):
-    """Two sequences of the 48-V-head layer: twice as many half-width scan CTAs
-    as one wave holds, so the launcher runs one full-width (d_v = 128) scan CTA
-    per head. Ragged tail, nonzero entry state; sampled heads of both
+def test_scan_two_sequences_many_heads(gate_mode):
+    """Two sequences of the 48-V-head layer (96 scan CTAs, one per sequence
+    and value head). Ragged tail, nonzero entry state; sampled heads of both
     sequences against the oracle."""
     w = small(T=150, B=2, H_qk=16, H_v=48, d=128, chunk=64, qkv="bf16", s0="normal")
     inp = make_inputs(w, seed=43, gate_mode=gate_mode)

@@ -74,7 +74,7 @@ def test_packed_equals_separate_and_oracle(path, gate_mode):
 
 @pytest.mark.parametrize("path", ["tensor_core", "fp32"])
 def test_packed_conv_histories(path):
-    """Conv + L2 norm in the load step: at every sequence start the conv reads
+    """Conv + L2 norm in the prep's load: at every sequence start the conv reads
     that sequence's own history (never the previous sequence's tokens), and
     each sequence's history after its last token is written."""
     lens = [70, 2, 0, 129, 5]

@@ -74,10 +74,11 @@ def test_noalloc_rejects_configurations_without_scratch():
 
 
 def test_noalloc_conv_l2norm_segments_carry_conv_history():
-    """With the conv / L2 load step the fixed array holds fewer chunks; a
-    2-sequence, 2000-token call runs in several segments whose first tokens
-    take their conv history from the previous segment."""
-    w = replace(workload("conv_prefill_b8_t8192"), B=2, T=2000, H_qk=2, H_v=6)
+    """The fixed array holds 37 chunks of this 12-sequence-head problem, so a
+    2-sequence, 3000-token call (47 chunks) with the conv and L2 norm runs in
+    two segments; the second segment's first tokens convolve with the last
+    inputs of the first. Bit for bit the one-pass call."""
+    w = replace(workload("conv_prefill_b8_t8192"), B=2, T=3000, H_qk=2, H_v=6)
     inp = make_inputs(w, seed=29, device="cuda")
     args = (inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"])
     o_ref, S_ref = gdn2.chunk_fwd(*args, chunk=64, o_dtype=torch.float32, conv_w=inp["conv_w"], l2norm_qk=True)
