@@ -325,10 +325,12 @@ def weak_value(units_per_rank: float, world: int, ms_max: float) -> float:
     return units_per_rank * world / (ms_max * 1e-3)
 
 
-def config_dict(w):
+def config_dict(w, heads_per_rank=None):
+    par = ("independent sequences per GPU" if heads_per_rank is None else
+           f"heads split across GPUs: {heads_per_rank[0]} QK / {heads_per_rank[1]} V heads per GPU")
     return {"workload": f"{w.name}: B={w.B} T={w.T} H_qk={w.H_qk} H_v={w.H_v} d={w.d} chunk={w.chunk} "
                         f"{w.qkv_dtype} q,k,v, fp32 per-channel gates, S0=0",
-            "global_batch": w.B, "seq_len": w.T, "parallelism": "independent sequences per GPU",
+            "global_batch": w.B, "seq_len": w.T, "parallelism": par,
             "l2": f"no flush: each step moves {prefill_bytes(w) / 1e9:.2f} GB (inputs read once, "
                   f"o written once), > 126 MB L2"}
 
@@ -361,6 +363,10 @@ def main():
     ap.add_argument("--cp-steps", type=int, default=5,
                     help="with N > 1 ranks: timed calls of the T=32768 sequence split across the ranks "
                          "(context-parallel prefill, strong scaling); 0 skips it")
+    ap.add_argument("--split", default="sequences", choices=["sequences", "heads"],
+                    help="with N > 1 ranks, what the headline line partitions: whole sequences per rank "
+                         "(weak scaling, the default) or the layer's heads (H_qk/N QK heads and the value heads "
+                         "that read them per rank, one sequence: strong scaling)")
     ap.add_argument("--heads-steps", type=int, default=20,
                     help="with N > 1 ranks: timed calls of the T=32768 layer with its heads split across the "
                          "ranks (H_qk/N QK heads and the value heads that read them per rank, strong scaling); "
@@ -395,7 +401,15 @@ def main():
             dist.barrier()
 
     pk = peaks()
-    w = workload(args.workload)
+    w_layer = workload(args.workload)
+    w = w_layer
+    heads_split = args.split == "heads" and world > 1
+    if heads_split:
+        # this rank's block of heads (see delta_rule_linear_gdn_b200/head_parallel.py)
+        from dataclasses import replace as _replace
+        from delta_rule_linear_gdn_b200.head_parallel import head_shard
+        qs, vs = head_shard(w_layer.H_qk, w_layer.H_v, rank, world)
+        w = _replace(w_layer, H_qk=qs.stop - qs.start, H_v=vs.stop - vs.start)
     stream = torch.cuda.Stream(device=dev)
     inp = make_inputs(w, seed=rank_seed(rank), device=dev)
     o = torch.empty((w.B, w.T, w.H_v, w.d), dtype=torch.bfloat16, device=dev)
@@ -427,15 +441,19 @@ def main():
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, dev)
-    tokens_per_step = w.B * w.T * world
-    value = weak_value(w.B * w.T, world, ms_max)
+    if heads_split:   # the ranks share one layer's tokens
+        tokens_per_step = w.B * w.T
+        value = tokens_per_step / (ms_max * 1e-3)
+    else:
+        tokens_per_step = w.B * w.T * world
+        value = weak_value(w.B * w.T, world, ms_max)
 
     nbytes = prefill_bytes(w)
     flops = prefill_flops(w)
     kernel_s = ms * 1e-3  # one call: the prep and scan launches back to back on one stream
     achieved_gbs = nbytes / kernel_s / 1e9
     tflops = flops / kernel_s / 1e12
-    traffic = measured_traffic() if w.name == PREFILL else None
+    traffic = measured_traffic() if w.name == PREFILL and not heads_split else None
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved_gbs / pk["hbm_gbs"], "traffic": traffic,
                 "peak_source": pk["source"],
@@ -505,8 +523,10 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(w),
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "strong" if heads_split else "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(w_layer, heads_per_rank=(w.H_qk, w.H_v) if heads_split else None),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * launches_per_call, "clocks": clocks, "decode": decode,
             "conv_prefill": conv, "prefill_gate_logits": logits, "prefill_qk_gates": qk_gates,
