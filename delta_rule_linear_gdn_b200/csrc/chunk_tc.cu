@@ -1834,9 +1834,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     nseg_ov = std::min(std::min(OVERLAP_SEGMENTS, nchunks / OVERLAP_MIN_CHUNKS), MAX_COUNTERS);
 
   // Segment lengths. Overlapped: the last scan has no prep beside it, so the
-  // last segment is short (1/16 of the chunks, at least OVERLAP_LAST_MIN) and
-  // the others share the rest equally.
-  const int n_last = nseg_ov > 0 ? std::max(OVERLAP_LAST_MIN, nchunks / 16) : 0;
+  // last segment is short (1/8 of the chunks, at least OVERLAP_LAST_MIN; 1/4,
+  // 1/6, 1/10, 1/16 and 1/32 measured slower at T=32768) and the others share
+  // the rest equally.
+  const int n_last = nseg_ov > 0 ? std::max(OVERLAP_LAST_MIN, nchunks / 8) : 0;
   const int step = nseg_ov > 0 ? (nchunks - n_last + nseg_ov - 2) / (nseg_ov - 1) : seg;
   const float* s_in = a.S0;
   int k = 0;
