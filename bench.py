@@ -355,7 +355,7 @@ def main():
                     help="timed calls of the T=32768 prefill with alpha, b per QK head; 0 skips it")
     ap.add_argument("--decode-conv-steps", type=int, default=200,
                     help="timed decode steps with the conv and L2 norm in the step; 0 skips it")
-    ap.add_argument("--conv-steps", type=int, default=5,
+    ap.add_argument("--conv-steps", type=int, default=10,
                     help="timed calls of the conv + L2 workload (B=8, T=8192); 0 skips it")
     ap.add_argument("--tied-steps", type=int, default=20,
                     help="timed calls of the T=32768 prefill with the tied gates of KDA and of Gated DeltaNet")
