@@ -98,6 +98,10 @@ constexpr int SL_WM = 74240;          // max |U_w| over the chunk (fp32; 16 byte
 constexpr int SLOT_USED = 74256;      // bytes copied per chunk
 constexpr int SL_FLAG = SLOT_USED;    // int: 1 = the slot is written by the exact kernel (not copied)
 constexpr int SLOT = 74752;           // slot stride (1 KB multiple)
+static_assert(SL_QT == SL_YT + 16384 && SL_UW == SL_QT + 16384 && SL_KE == SL_UW + 16384 &&
+                  SL_AQ == SL_KE + 16384 && SL_GC == SL_AQ + 8192 && SL_WM == SL_GC + 512 &&
+                  SLOT_USED == SL_WM + 16,
+              "slot layout: the head-shared tiles around the per-head U_w, then the per-head max");
 // Least α product over an aligned 16-token quarter (per channel) that the
 // prep's reciprocal factorisation takes; items below it run exactly.
 constexpr float kStrongDecay = 5.421010862427522e-20f;   // 2^-64
@@ -236,19 +240,24 @@ __device__ __forceinline__ size_t slot_index(SlotMap m, int bh, int j) {
 
 // A work item: chunk cl of sequence bi (bh = bi · H_v + h), tokens t0 .. t0 +
 // Lc − 1 of the q, k, v buffers (bi is 0 for packed sequences, whose t0 is
-// already in the packed stream), and its slot.
+// already in the packed stream), and its slot. With groups of G value heads
+// per item (the heads reading one QK head, when α and b belong to it), h is
+// the group's first head and the group's slots are slot + g · hstride.
 struct Item {
   int bh, cl, h, bi, hq, t0, Lc;
-  size_t slot;
+  size_t slot, hstride;
 };
-template <bool VL>
+template <bool VL, bool GROUPS = false>
 __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int item, SlotMap sm) {
   Item it;
+  // GROUPS: one item per group of G = H_v / H_qk value heads (ng per sequence)
+  const int G = GROUPS ? a.Hv / a.Hqk : 1;
+  const int ng = GROUPS ? a.Hqk : a.Hv;
   if (VL) {
-    // item = global chunk · H_v + value head; the sequence is the last n with
+    // item = global chunk · ng + head group; the sequence is the last n with
     // cu_chk[n] ≤ the chunk (empty sequences own no chunk and are passed over)
-    it.h = item % a.Hv;
-    const int g = item / a.Hv;
+    it.h = GROUPS ? (item % ng) * G : item % a.Hv;
+    const int g = item / ng;
     int lo = 0, hi = a.nseq;            // cu_chk[lo] ≤ g < cu_chk[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -262,6 +271,18 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int
     it.t0 = a.cu_tok[lo] + it.cl * C;
     it.Lc = min(C, a.cu_tok[lo + 1] - it.t0);
     it.slot = (size_t)a.cu_chk[lo] * a.Hv + (size_t)it.h * nc + it.cl;
+    it.hstride = (size_t)nc;
+  } else if (GROUPS) {
+    const int r = item % (a.B * ng);  // QK head fastest
+    it.cl = item / (a.B * ng);
+    it.bi = r / ng;
+    it.h = (r % ng) * G;
+    it.bh = it.bi * a.Hv + it.h;
+    it.hq = it.h / (a.Hv / a.Hqk);
+    it.t0 = (c_begin + it.cl) * C;
+    it.Lc = min(C, a.T - it.t0);
+    it.slot = slot_index(sm, it.bh, it.cl);
+    it.hstride = (size_t)sm.stride;
   } else {
     it.bh = item % (a.B * a.Hv);      // value head fastest: heads sharing q, k run together
     it.cl = item / (a.B * a.Hv);
@@ -271,6 +292,7 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int
     it.t0 = (c_begin + it.cl) * C;
     it.Lc = min(C, a.T - it.t0);
     it.slot = slot_index(sm, it.bh, it.cl);
+    it.hstride = (size_t)sm.stride;
   }
   return it;
 }
@@ -302,7 +324,9 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   uint32_t* s_wmax = reinterpret_cast<uint32_t*>(sflag + 2);   // max |U_w| of the item (float bits)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_items = VL ? a.cu_chk[a.nseq] * a.Hv : a.B * a.Hv * n_seg;
+  // QKG: one item per (chunk, sequence, QK head), for its G value heads
+  const int G = QKG ? a.Hv / a.Hqk : 1;
+  const int n_items = (VL ? a.cu_chk[a.nseq] * a.Hv : a.B * a.Hv * n_seg) / G;
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(bar_a, 1);
@@ -354,8 +378,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     const size_t r = (size_t)it.bi * a.T + it.t0 + i0 + u;
     return QKG ? r * a.Hqk + it.hq : r * a.Hv + it.h;
   };
-  auto w_row = [&](const Item& it, int u) -> size_t {
-    return full ? ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hv + it.h : gate_row(it, u);
+  auto w_row = [&](const Item& it, int hv, int u) -> size_t {   // w of value head hv
+    return full ? ((size_t)it.bi * a.T + it.t0 + i0 + u) * a.Hv + hv : gate_row(it, u);
   };
   auto qkv_tok = [&](const Item& it, int u) -> size_t {
     return (size_t)it.bi * a.T + it.t0 + i0 + u;
@@ -372,13 +396,13 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   // The per-channel α tile of an item comes by one TMA copy (rows of the
   // tensor map [B·T][H_v][128]), requested by thread 0 one item ahead.
   auto fetch_alpha = [&](int item_) {
-    const Item nx = decode_item<VL>(a, c_begin, item_, sm);
+    const Item nx = decode_item<VL, QKG>(a, c_begin, item_, sm);
     mbar_arrive_expect_tx(bar_a, C * D * (LG ? 2 : 4));
     tma_load_3d(smem + P_ALPHA, &amap, 0, QKG ? nx.hq : nx.h, nx.bi * a.T + nx.t0, bar_a);
   };
   uint32_t phase_a = 0;
   auto load_alpha_key0 = [&](int item_) {
-    const Item it = decode_item<VL>(a, c_begin, item_, sm);
+    const Item it = decode_item<VL, QKG>(a, c_begin, item_, sm);
 #pragma unroll
     for (int u = 0; u < 4; ++u) load_key1(it, u, u);
     if (use_amap) {
@@ -494,7 +518,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   if (use_amap && tid == 0 && (counter ? *s_item : (int)blockIdx.x) < n_items)
     fetch_alpha(counter ? *s_item : (int)blockIdx.x);
   for (int item = counter ? *s_item : (int)blockIdx.x; item < n_items;) {
-    const Item it = decode_item<VL>(a, c_begin, item, sm);
+    const Item it = decode_item<VL, QKG>(a, c_begin, item, sm);
     uint8_t* slot = static_cast<uint8_t*>(a.workspace) + WS_HEAD + it.slot * SLOT;
     if constexpr (CV) fused_qk(it);
     load_alpha_key0(item);
@@ -539,7 +563,8 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       exact = !(mall >= kStrongDecay);
     }
     if (exact) {
-      if (tid == 0) *reinterpret_cast<int*>(slot + SL_FLAG) = 1;
+      if (tid == 0)
+        for (int g = 0; g < G; ++g) *reinterpret_cast<int*>(slot + (size_t)g * it.hstride * SLOT + SL_FLAG) = 1;
       // every thread has read the quarter minima and α (pass 1); thread 0's
       // s_item is visible after this barrier
       __syncthreads();
@@ -661,23 +686,63 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #undef GDN2_PASS2
 #undef GDN2_GRAM_TILE
 #undef GDN2_TILE
-    // the write side, consumed after the Gram products
+    // the write side of value head hv, consumed after the Gram products
     float4 wv[8];
     constexpr int NV = CV ? 11 : 8;   // CV: raw v of the 8 tokens and the 3 before them (conv at the Z step)
     uint2 vv[NV];
-    const int choff_v = 2 * a.Hqk * D + it.h * D;
+    auto load_write = [&](int hv) {
+      const int choff_v = 2 * a.Hqk * D + hv * D;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const bool ok = it.Lc == C || i0 + u < it.Lc;
-      wv[u] = ok ? gate4<LG>(src.w, w_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
-      if constexpr (!CV)
-        vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
-                   : make_uint2(0, 0);
-    }
-    if constexpr (CV) {
+      for (int u = 0; u < 8; ++u) {
+        const bool ok = it.Lc == C || i0 + u < it.Lc;
+        wv[u] = ok ? gate4<LG>(src.w, w_row(it, hv, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if constexpr (!CV)
+          vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + hv) * D + c0))
+                     : make_uint2(0, 0);
+      }
+      if constexpr (CV) {
 #pragma unroll
-      for (int j = 0; j < NV; ++j)
-        vv[j] = (a.conv_w != nullptr || j >= 3) ? raw4(src.v, a.Hv, it.h, choff_v, it, i0 - 3 + j) : make_uint2(0, 0);
+        for (int j = 0; j < NV; ++j)
+          vv[j] = (a.conv_w != nullptr || j >= 3) ? raw4(src.v, a.Hv, hv, choff_v, it, i0 - 3 + j) : make_uint2(0, 0);
+      }
+    };
+    // Z = w ⊙ v of value head hv (no decay) to its tile, read by the U_w
+    // product (CV: v convolved here, from its raw rows)
+    auto write_z = [&](int hv) {
+      const int choff_v = 2 * a.Hqk * D + hv * D;
+      float4 Wv[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        Wv[c] = CV && a.conv_w ? __ldg(reinterpret_cast<const float4*>(a.conv_w + (size_t)(choff_v + c0 + c) * 4))
+                               : make_float4(0.f, 0.f, 0.f, 1.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float vx[4];
+        if constexpr (CV)
+          conv4(vv, u, Wv, vx);
+        else
+          unpack4_bf16(vv[u], vx);
+        st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
+            pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
+      }
+    };
+    if constexpr (QKG) {
+      load_write(it.h);
+    } else {
+      const int choff_v = 2 * a.Hqk * D + it.h * D;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool ok = it.Lc == C || i0 + u < it.Lc;
+        wv[u] = ok ? gate4<LG>(src.w, w_row(it, it.h, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if constexpr (!CV)
+          vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
+                     : make_uint2(0, 0);
+      }
+      if constexpr (CV) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j)
+          vv[j] = (a.conv_w != nullptr || j >= 3) ? raw4(src.v, a.Hv, it.h, choff_v, it, i0 - 3 + j) : make_uint2(0, 0);
+      }
     }
     sync_for_mma();
 
@@ -743,22 +808,25 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     }
 
 
-    // Z = w ⊙ v (no decay) to its tile, read by the Y/U_w products (CV: v
-    // convolved here, from its raw rows)
-    float4 Wv[4];
+    if constexpr (QKG) {
+      write_z(it.h);
+    } else {
+      const int choff_v = 2 * a.Hqk * D + it.h * D;
+      float4 Wv[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      Wv[c] = CV && a.conv_w ? __ldg(reinterpret_cast<const float4*>(a.conv_w + (size_t)(choff_v + c0 + c) * 4))
-                             : make_float4(0.f, 0.f, 0.f, 1.f);
+      for (int c = 0; c < 4; ++c)
+        Wv[c] = CV && a.conv_w ? __ldg(reinterpret_cast<const float4*>(a.conv_w + (size_t)(choff_v + c0 + c) * 4))
+                               : make_float4(0.f, 0.f, 0.f, 1.f);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float vx[4];
-      if constexpr (CV)
-        conv4(vv, u, Wv, vx);
-      else
-        unpack4_bf16(vv[u], vx);
-      st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
-          pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
+      for (int u = 0; u < 8; ++u) {
+        float vx[4];
+        if constexpr (CV)
+          conv4(vv, u, Wv, vx);
+        else
+          unpack4_bf16(vv[u], vx);
+        st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
+            pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
+      }
     }
 
     // -------- A = (I + T)⁻¹, blocked
@@ -884,64 +952,144 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
     sync_for_mma();
 
     // -------- −Yᵀ = −Ēᵀ Aᵀ, U_wᵀ = Zᵀ Aᵀ (Ē carries the sign, Z here is the write side w ⊙ v)
-    if (tid == 0) {
-      const uint64_t eb = desc_mn_sw(smem_u32(smem + P_EB), 0, BS_ROW64);
-      const uint64_t z = desc_mn_sw(smem_u32(smem + P_Z), 0, BS_ROW64);
-      const uint64_t ai = desc_k_sw(smem_u32(smem + P_AINV), 0, BS_ROW64);
+    if constexpr (!QKG) {
+      if (tid == 0) {
+        const uint64_t eb = desc_mn_sw(smem_u32(smem + P_EB), 0, BS_ROW64);
+        const uint64_t z = desc_mn_sw(smem_u32(smem + P_Z), 0, BS_ROW64);
+        const uint64_t ai = desc_k_sw(smem_u32(smem + P_AINV), 0, BS_ROW64);
 #pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks)
-        mma16(tmem + PT_YT, eb + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
-              ks > 0);
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma16(tmem + PT_YT, eb + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
+                ks > 0);
 #pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks)
-        mma16(tmem + PT_UW, z + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
-              ks > 0);
-      mma_commit(bar);
-    }
-    __syncwarp();
-    wait_mma(bar, phase, sflag);
-    // the products have read Ē and Z: their space takes the next item's α
-    if (use_amap && tid == 0) {
-      const int nx = counter ? *s_item : item + (int)gridDim.x;
-      if (nx < n_items) fetch_alpha(nx);
-    }
+        for (int ks = 0; ks < C / 16; ++ks)
+          mma16(tmem + PT_UW, z + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
+                ks > 0);
+        mma_commit(bar);
+      }
+      __syncwarp();
+      wait_mma(bar, phase, sflag);
+      // the products have read Ē and Z: their space takes the next item's α
+      if (use_amap && tid == 0) {
+        const int nx = counter ? *s_item : item + (int)gridDim.x;
+        if (nx < n_items) fetch_alpha(nx);
+      }
 
-    {
-      // warps 0..3: Yᵀ rows (key lanes); warps 4..7: U_wᵀ rows (dv lanes),
-      // staged in the (now free) Gram operand space and stored by two bulk
-      // copies, byte for byte the slot's layout
-      const uint32_t col = hc == 0 ? PT_YT : PT_UW;
-      const int stg = P_YS + hc * 16384;
-      uint32_t wm = 0;                   // max |U_w| (the scan scales its state by it)
+      {
+        // warps 0..3: Yᵀ rows (key lanes); warps 4..7: U_wᵀ rows (dv lanes),
+        // staged in the (now free) Gram operand space and stored by two bulk
+        // copies, byte for byte the slot's layout
+        const uint32_t col = hc == 0 ? PT_YT : PT_UW;
+        const int stg = P_YS + hc * 16384;
+        uint32_t wm = 0;                 // max |U_w| (the scan scales its state by it)
 #pragma unroll
-      for (int cb0 = 0; cb0 < 64; cb0 += 32) {
-        float v[32];
-        tmem_ld16(t_lane + col + cb0, v);
-        tmem_ld16(t_lane + col + cb0 + 16, v + 16);
-        tmem_wait_ld();
+        for (int cb0 = 0; cb0 < 64; cb0 += 32) {
+          float v[32];
+          tmem_ld16(t_lane + col + cb0, v);
+          tmem_ld16(t_lane + col + cb0 + 16, v + 16);
+          tmem_wait_ld();
 #pragma unroll
-        for (int cb = 0; cb < 32; cb += 8) st16(smem, stg + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
+          for (int cb = 0; cb < 32; cb += 8) st16(smem, stg + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
+          if (hc == 1) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) wm = max(wm, __float_as_uint(v[u]) & 0x7fffffffu);
+          }
+        }
         if (hc == 1) {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) wm = max(wm, __float_as_uint(v[u]) & 0x7fffffffu);
+          wm = __reduce_max_sync(0xffffffffu, wm);
+          if (lane == 0) atomicMax(s_wmax, wm);
         }
       }
-      if (hc == 1) {
-        wm = __reduce_max_sync(0xffffffffu, wm);
-        if (lane == 0) atomicMax(s_wmax, wm);
+      fence_async_smem();
+      fence_before_sync();
+      __syncthreads();
+      fence_after_sync();
+      if (tid == 0) {
+        bulk_s2g(slot + SL_YT, smem + P_YS, 16384);
+        bulk_s2g(slot + SL_UW, smem + P_YS + 16384, 16384);
+        bulk_commit();
+        *reinterpret_cast<int*>(slot + SL_FLAG) = 0;   // written here, not by the exact kernel
+        *reinterpret_cast<uint32_t*>(slot + SL_WM) = *s_wmax;
+        *s_wmax = 0;                     // (the next item's maxima come after two barriers)
       }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    if (tid == 0) {
-      bulk_s2g(slot + SL_YT, smem + P_YS, 16384);
-      bulk_s2g(slot + SL_UW, smem + P_YS + 16384, 16384);
-      bulk_commit();
-      *reinterpret_cast<int*>(slot + SL_FLAG) = 0;   // written here, not by the exact kernel
-      *reinterpret_cast<uint32_t*>(slot + SL_WM) = *s_wmax;
-      *s_wmax = 0;                       // (the next item's maxima come after two barriers)
+    } else {
+      // With α and b owned by the QK head (QKG) everything so far is shared by its
+      // G value heads: the item makes U_w for each in turn (the next head's w, v
+      // requested while the current product runs) and writes the shared tiles
+      // once, to the slot of the group's first head, where every head's scan
+      // reads them.
+      for (int g = 0; g < G; ++g) {
+        uint8_t* slot_g = slot + (size_t)g * it.hstride * SLOT;
+        if (g > 0) {
+          write_z(it.h + g);
+          sync_for_mma();
+        }
+        if (tid == 0) {
+          const uint64_t eb = desc_mn_sw(smem_u32(smem + P_EB), 0, BS_ROW64);
+          const uint64_t z = desc_mn_sw(smem_u32(smem + P_Z), 0, BS_ROW64);
+          const uint64_t ai = desc_k_sw(smem_u32(smem + P_AINV), 0, BS_ROW64);
+          if (g == 0) {
+  #pragma unroll
+            for (int ks = 0; ks < C / 16; ++ks)
+              mma16(tmem + PT_YT, eb + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
+                    ks > 0);
+          }
+  #pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks)
+            mma16(tmem + PT_UW, z + mn_step_sw(ks), ai + k_step_sw(ks, BS_ROW64), idesc_f16(128, 64, true, false),
+                  ks > 0);
+          mma_commit(bar);
+        }
+        if (QKG && g + 1 < G) load_write(it.h + g + 1);   // (this thread's Z of head g is written)
+        __syncwarp();
+        wait_mma(bar, phase, sflag);
+        // the products have read Ē and Z: their space takes the next item's α
+        if (g == G - 1 && use_amap && tid == 0) {
+          const int nx = counter ? *s_item : item + (int)gridDim.x;
+          if (nx < n_items) fetch_alpha(nx);
+        }
+        if (g > 0) {                       // the previous head's U_wᵀ staging has been read
+          if (tid == 0) bulk_wait_read_all();
+          __syncthreads();
+        }
+        if (g == 0 || hc == 1) {
+          // warps 0..3: Yᵀ rows (key lanes; first head only); warps 4..7: U_wᵀ
+          // rows (dv lanes), staged in the (now free) Gram operand space and
+          // stored by bulk copies, byte for byte the slot's layout
+          const uint32_t col = hc == 0 ? PT_YT : PT_UW;
+          const int stg = P_YS + hc * 16384;
+          uint32_t wm = 0;                 // max |U_w| (the scan scales its state by it)
+  #pragma unroll
+          for (int cb0 = 0; cb0 < 64; cb0 += 32) {
+            float v[32];
+            tmem_ld16(t_lane + col + cb0, v);
+            tmem_ld16(t_lane + col + cb0 + 16, v + 16);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int cb = 0; cb < 32; cb += 8) st16(smem, stg + sw_off(row, cb0 + cb, BS_ROW128), pack8_f16(v + cb));
+            if (hc == 1) {
+  #pragma unroll
+              for (int u = 0; u < 32; ++u) wm = max(wm, __float_as_uint(v[u]) & 0x7fffffffu);
+            }
+          }
+          if (hc == 1) {
+            wm = __reduce_max_sync(0xffffffffu, wm);
+            if (lane == 0) atomicMax(s_wmax, wm);
+          }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0) {
+          if (g == 0) bulk_s2g(slot + SL_YT, smem + P_YS, 16384);
+          bulk_s2g(slot_g + SL_UW, smem + P_YS + 16384, 16384);
+          bulk_commit();
+          *reinterpret_cast<int*>(slot_g + SL_FLAG) = 0;   // written here, not by the exact kernel
+          *reinterpret_cast<uint32_t*>(slot_g + SL_WM) = *s_wmax;
+          *s_wmax = 0;                     // (the next maxima come after two barriers)
+        }
+      }
     }
     item = counter ? *s_item : item + (int)gridDim.x;   // written before the barriers above
   }
@@ -1279,7 +1427,9 @@ template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat
 }
 template <> __device__ __forceinline__ void store_out<float>(float* dst, float x) { *dst = x; }
 
-template <typename TOut>
+// SHARED: α and b belong to the QK heads, and the tiles a QK head's value heads
+// share sit in the slots of each group's first head (see the prep).
+template <typename TOut, bool SHARED>
 __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs a, int c_begin, int n_seg_arg,
                                                                       SlotMap sm, const float* S_in, float* S_out) {
   using L = ScanLayout;
@@ -1313,6 +1463,10 @@ __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs
   const size_t tok0 = a.nseq ? (size_t)a.cu_tok[bi] : (size_t)bi * a.T + (size_t)c_begin * C;
   const int trem = a.nseq ? a.cu_tok[bi + 1] - a.cu_tok[bi] : a.T - c_begin * C;
   const uint8_t* slots = static_cast<const uint8_t*>(a.workspace) + WS_HEAD + slot0 * SLOT;
+  // SHARED: the tiles the value heads of a QK head share come from the slots
+  // of the group's first head (U_w and max |U_w| are every head's own)
+  const int hg = SHARED ? h % (a.Hv / a.Hqk) : 0;
+  const uint8_t* slots_sh = slots - (size_t)hg * (a.nseq ? (size_t)n_seg : (size_t)sm.stride) * SLOT;
   TOut* og = static_cast<TOut*>(a.o);
   if (n_seg == 0) {
     // an empty packed sequence: its final state is its initial one
@@ -1344,8 +1498,17 @@ __global__ void __launch_bounds__(ScanLayout::NS, 1) chunk_scan_kernel(ChunkArgs
     if (lane == 0) {
       auto load = [&](int c) {
         uint8_t* stg = smem + (c & 1) * L::STAGE;
+        const uint8_t* own = slots + (size_t)c * SLOT;
         mbar_arrive_expect_tx(&full[c & 1], SLOT_USED);
-        bulk_g2s(stg, slots + (size_t)c * SLOT, SLOT_USED, &full[c & 1]);
+        if (!SHARED || hg == 0) {
+          bulk_g2s(stg, own, SLOT_USED, &full[c & 1]);
+        } else {
+          const uint8_t* sh = slots_sh + (size_t)c * SLOT;
+          bulk_g2s(stg + SL_YT, sh + SL_YT, SL_UW - SL_YT, &full[c & 1]);
+          bulk_g2s(stg + SL_UW, own + SL_UW, SL_KE - SL_UW, &full[c & 1]);
+          bulk_g2s(stg + SL_KE, sh + SL_KE, SL_WM - SL_KE, &full[c & 1]);
+          bulk_g2s(stg + SL_WM, own + SL_WM, SLOT_USED - SL_WM, &full[c & 1]);
+        }
       };
       int issued = 0, landed = 0;       // chunks whose copies were issued / seen complete
       bool any_mma = false;
@@ -1809,7 +1972,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   // Scan: one CTA per (sequence, value head).
   const int scan_ctas = BH;
-  auto scan = o_bf16 ? chunk_scan_kernel<__nv_bfloat16> : chunk_scan_kernel<float>;
+  const bool qkg = a.Hg != a.Hv;
+  auto scan = o_bf16 ? (qkg ? chunk_scan_kernel<__nv_bfloat16, true> : chunk_scan_kernel<__nv_bfloat16, false>)
+                     : (qkg ? chunk_scan_kernel<float, true> : chunk_scan_kernel<float, false>);
   const int scan_threads = ScanLayout::NS;
   const int scan_smem = ScanLayout::SMEM;
   if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
@@ -1824,7 +1989,6 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   const int prep_ctas = sms * 2;
   CUtensorMap amap{};
   const int use_amap = a.gate_mode != GDN2_GATES_GDN && a.alpha != nullptr && encode_alpha_map(a, &amap) ? 1 : 0;
-  const bool qkg = a.Hg != a.Hv;
   const PrepFn prep = vl ? prep_variant<true>(cv, a.gate_logits != 0, qkg) : prep_variant<false>(cv, a.gate_logits != 0, qkg);
 
   // overlapped segments: whole sequence in the workspace, idle SMs beside the
@@ -1850,8 +2014,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     // overlapped: every chunk has its own slot; otherwise the segment's slots start at 0
     const SlotMap sm = nseg_ov > 0 ? SlotMap{nchunks, c0} : SlotMap{seg, 0};
     int* counter = nseg_ov > 0 ? reinterpret_cast<int*>(ws) + 1 + k : nullptr;
-    const int items = vl ? nchunks * a.Hv : BH * n;
-    const int grid = std::min(items, prep_ctas);
+    const int items = vl ? nchunks * a.Hv : BH * n;           // (chunk, sequence, value head)
+    const int prep_items = qkg ? items / (a.Hv / a.Hqk) : items;   // QK-owned gates: one per head group
+    const int grid = std::min(prep_items, prep_ctas);
     if (items == 0) {
       // nothing to prepare (packed sequences, all empty)
     } else if (nseg_ov > 0 && k > 0) {
