@@ -228,8 +228,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t b
 }
 
 // Bulk (non-tensor) asynchronous copy global → shared of `bytes` (multiple of
-// 16, both addresses 16-byte aligned), completing on `mbar` as transactions.
-// No multicast.
+// 16, both addresses 16-byte aligned), completing on `mbar` as transactions;
+// the destination is this CTA's own shared memory only.
 __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* mbar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
@@ -238,8 +238,8 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       : "memory");
 }
 
-// Tiled tensor copy global → shared of one box of a 3-D tensor map (no
-// multicast), completing on `mbar` as transactions. The innermost coordinate
+// Tiled tensor copy global → shared of one box of a 3-D tensor map into this
+// CTA's own shared memory, completing on `mbar` as transactions. The innermost coordinate
 // x times the element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* tmap, int x, int y, int z, uint64_t* mbar) {
   asm volatile(
