@@ -125,6 +125,9 @@ constexpr int P_PQ = 8192;            // quarter products [4][128] fp32
 constexpr int P_RED = P_PQ + 4 * D * 4;
 constexpr int P_SUMS = P_RED + 32;    // fused load: per-half sums of squares of k, q [2][64 tok][2] fp32
 static_assert(P_SUMS + 2 * C * 2 * 4 <= 12288, "quarter products and sums must stay in the unused Gram rows");
+constexpr int P_BETA = P_RED + 128;   // scalar β of the next item (TMA box: 64 tokens × 16 bytes of heads);
+                                      // not with the fused load, whose sums use these bytes
+static_assert(P_BETA % 128 == 0 && P_BETA + C * 16 <= 12288, "β box in the unused Gram rows");
 constexpr int P_GM = 32768;
 constexpr int P_KM = 65536;
 constexpr int P_EB = 81920;
@@ -305,10 +308,16 @@ __device__ __forceinline__ Item decode_item(const ChunkArgs& a, int c_begin, int
 // alpha and b belong to the QK heads; VL: sequences of different lengths
 // packed along T (one compiled copy each, so that no form pays for the
 // others' addressing at the register limit).
-template <bool CV, bool LG, bool QKG, bool VL>
+// Gates that come by TMA, one item ahead (bits of `tgates`): the per-channel α tile;
+// a box of scalar α (Gated DeltaNet layout); a box of scalar β (tied layouts,
+// b = w = β). Each box holds the item's 64 tokens × 16 bytes of heads.
+// The boxes exist in a compiled copy of their own (BOX), so that the
+// per-channel copies carry none of their code.
+constexpr int TG_ATILE = 1, TG_ABOX = 2, TG_BBOX = 4;
+template <bool CV, bool LG, bool QKG, bool VL, bool BOX>
 __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_begin, int n_seg, SlotMap sm,
                                                            int* counter, const __grid_constant__ CUtensorMap amap,
-                                                           int use_amap) {
+                                                           const __grid_constant__ CUtensorMap bmap, int tgates) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + P_BAR);
   uint64_t* bar_a = bar + 1;            // the α tile has landed
@@ -384,29 +393,63 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   auto qkv_tok = [&](const Item& it, int u) -> size_t {
     return (size_t)it.bi * a.T + it.t0 + i0 + u;
   };
+  constexpr int GE = LG ? 8 : 4;       // gate values per 16 bytes
+  // a scalar gate of token row u of the item from a box (σ of a logit)
+  auto box_gate = [&](const Item& it, int off, int u) -> float {
+    const int col = (QKG ? it.hq : it.h) % GE;
+    if (LG) return sigmoid_f32(__uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(smem + off + u * 16 + col * 2) << 16));
+    return *reinterpret_cast<const float*>(smem + off + u * 16 + col * 4);
+  };
   auto load_key1 = [&](const Item& it, int u, int s) {
     const bool ok = it.Lc == C || i0 + u < it.Lc;
     const size_t tq = qkv_tok(it, u) * a.Hqk + it.hq;
-    bq[s] = ok ? gate4<LG>(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (BOX && (tgates & TG_BBOX)) {
+      const float bt = ok ? box_gate(it, P_BETA, i0 + u) : 0.f;
+      bq[s] = make_float4(bt, bt, bt, bt);
+    } else {
+      bq[s] = ok ? gate4<LG>(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if constexpr (!CV) {   // (CV: k and q come from pass 0)
       kk[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
       qq[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.q + tq * D + c0)) : make_uint2(0, 0);
     }
   };
   // The per-channel α tile of an item comes by one TMA copy (rows of the
-  // tensor map [B·T][H_v][128]), requested by thread 0 one item ahead.
+  // tensor map [B·T][H_g][128]), requested by thread 0 one item ahead; so do
+  // the boxes of scalar gates (rows of [B·T][H_g], the 16-byte column block
+  // that holds the item's head).
   auto fetch_alpha = [&](int item_) {
     const Item nx = decode_item<VL, QKG>(a, c_begin, item_, sm);
-    mbar_arrive_expect_tx(bar_a, C * D * (LG ? 2 : 4));
-    tma_load_3d(smem + P_ALPHA, &amap, 0, QKG ? nx.hq : nx.h, nx.bi * a.T + nx.t0, bar_a);
+    const int hg = QKG ? nx.hq : nx.h;
+    const int row = nx.bi * a.T + nx.t0;
+    mbar_arrive_expect_tx(bar_a, ((tgates & TG_ATILE) ? C * D * (LG ? 2 : 4) : 0) + ((BOX && (tgates & TG_ABOX)) ? C * 16 : 0) +
+                                     ((BOX && (tgates & TG_BBOX)) ? C * 16 : 0));
+    if (tgates & TG_ATILE) tma_load_3d(smem + P_ALPHA, &amap, 0, hg, row, bar_a);
+    if constexpr (BOX) {
+      if (tgates & TG_ABOX) tma_load_2d(smem + P_ALPHA, &amap, hg / GE * GE, row, bar_a);
+      if (tgates & TG_BBOX) tma_load_2d(smem + P_BETA, &bmap, hg / GE * GE, row, bar_a);
+    }
   };
   uint32_t phase_a = 0;
   auto load_alpha_key0 = [&](int item_) {
     const Item it = decode_item<VL, QKG>(a, c_begin, item_, sm);
+    if (BOX && (tgates & TG_BBOX)) {
+      wait_mma(bar_a, phase_a, sflag);   // (β of the key side is in the box)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) load_key1(it, u, u);
-    if (use_amap) {
-      wait_mma(bar_a, phase_a, sflag);
+      for (int u = 0; u < 4; ++u) load_key1(it, u, u);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) load_key1(it, u, u);
+      if (tgates) wait_mma(bar_a, phase_a, sflag);
+    }
+    if (BOX && (tgates & TG_ABOX)) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool ok = it.Lc == C || i0 + u < it.Lc;    // rows past the sequence's end: α = 1
+        const float al = ok ? box_gate(it, P_ALPHA, i0 + u) : 1.f;
+        f[u][0] = al; f[u][1] = al; f[u][2] = al; f[u][3] = al;
+      }
+    } else if (tgates & TG_ATILE) {
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const bool ok = it.Lc == C || i0 + u < it.Lc;    // rows past the sequence's end: α = 1
@@ -515,7 +558,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
   };
 
   uint32_t phase = 0;
-  if (use_amap && tid == 0 && (counter ? *s_item : (int)blockIdx.x) < n_items)
+  if (tgates && tid == 0 && (counter ? *s_item : (int)blockIdx.x) < n_items)
     fetch_alpha(counter ? *s_item : (int)blockIdx.x);
   for (int item = counter ? *s_item : (int)blockIdx.x; item < n_items;) {
     const Item it = decode_item<VL, QKG>(a, c_begin, item, sm);
@@ -569,7 +612,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       // s_item is visible after this barrier
       __syncthreads();
       const int nx = counter ? *s_item : item + (int)gridDim.x;
-      if (use_amap && tid == 0 && nx < n_items) fetch_alpha(nx);
+      if (tgates && tid == 0 && nx < n_items) fetch_alpha(nx);
       item = nx;
       continue;
     }
@@ -695,7 +738,17 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const bool ok = it.Lc == C || i0 + u < it.Lc;
-        wv[u] = ok ? gate4<LG>(src.w, w_row(it, hv, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (BOX && (tgates & TG_BBOX)) {
+          // tied: w = β, the same for every head of the group (QKG); from the
+          // box for the first head, kept for the others (whose turn comes after
+          // the inverse has reused the box's bytes)
+          if (hv == it.h) {
+            const float bt = ok ? box_gate(it, P_BETA, i0 + u) : 0.f;
+            wv[u] = make_float4(bt, bt, bt, bt);
+          }
+        } else {
+          wv[u] = ok ? gate4<LG>(src.w, w_row(it, hv, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         if constexpr (!CV)
           vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + hv) * D + c0))
                      : make_uint2(0, 0);
@@ -733,7 +786,12 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const bool ok = it.Lc == C || i0 + u < it.Lc;
-        wv[u] = ok ? gate4<LG>(src.w, w_row(it, it.h, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (BOX && (tgates & TG_BBOX)) {              // tied: w = β, from the box
+          const float bt = ok ? box_gate(it, P_BETA, i0 + u) : 0.f;
+          wv[u] = make_float4(bt, bt, bt, bt);
+        } else {
+          wv[u] = ok ? gate4<LG>(src.w, w_row(it, it.h, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         if constexpr (!CV)
           vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
                      : make_uint2(0, 0);
@@ -970,7 +1028,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       __syncwarp();
       wait_mma(bar, phase, sflag);
       // the products have read Ē and Z: their space takes the next item's α
-      if (use_amap && tid == 0) {
+      if (tgates && tid == 0) {
         const int nx = counter ? *s_item : item + (int)gridDim.x;
         if (nx < n_items) fetch_alpha(nx);
       }
@@ -1044,7 +1102,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
         __syncwarp();
         wait_mma(bar, phase, sflag);
         // the products have read Ē and Z: their space takes the next item's α
-        if (g == G - 1 && use_amap && tid == 0) {
+        if (g == G - 1 && tgates && tid == 0) {
           const int nx = counter ? *s_item : item + (int)gridDim.x;
           if (nx < n_items) fetch_alpha(nx);
         }
@@ -1887,8 +1945,7 @@ namespace {
 // them: H_v, or H_qk when shared) for the prep's tile loads (box: 64 tokens × 1 head × 128
 // channels). false if the driver entry point is unavailable (the prep then reads α with
 // plain loads).
-bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
-  const cuuint64_t esz = a.gate_logits ? 2 : 4;
+PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled encode = [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -1897,6 +1954,31 @@ bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
       fn = nullptr;
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
   }();
+  return encode;
+}
+
+// Tensor map of a scalar gate [B·T][H_g] (fp32, or bf16 logits) for boxes of
+// 64 tokens × 16 bytes of heads. false where a row of heads is not a multiple
+// of 16 bytes (the map's stride rule; the prep then reads the gate with
+// plain loads) or the driver entry point is unavailable.
+bool encode_scalar_gate_map(const ChunkArgs& a, const float* g, CUtensorMap* m) {
+  const cuuint64_t esz = a.gate_logits ? 2 : 4;
+  PFN_cuTensorMapEncodeTiled encode = tensor_map_encoder();
+  if (encode == nullptr || ((cuuint64_t)a.Hg * esz) % 16 != 0) return false;
+  const cuuint64_t rows = a.nseq ? (cuuint64_t)a.T : (cuuint64_t)a.B * (cuuint64_t)a.T;
+  const cuuint64_t dims[2] = {(cuuint64_t)a.Hg, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)a.Hg * esz};
+  const cuuint32_t box[2] = {(cuuint32_t)(16 / esz), (cuuint32_t)C};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(m, a.gate_logits ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                const_cast<float*>(g), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
+  const cuuint64_t esz = a.gate_logits ? 2 : 4;
+  PFN_cuTensorMapEncodeTiled encode = tensor_map_encoder();
   if (encode == nullptr) return false;
   const cuuint64_t rows = a.nseq ? (cuuint64_t)a.T : (cuuint64_t)a.B * (cuuint64_t)a.T;   // token rows
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.Hg, rows};
@@ -1917,14 +1999,19 @@ bool encode_alpha_map(const ChunkArgs& a, CUtensorMap* m) {
 // needed). With the whole
 // sequence in the workspace and SMs left idle by the scan, the segments are
 // pipelined (see the note on overlapped segments above).
-using PrepFn = void (*)(ChunkArgs, int, int, SlotMap, int*, const CUtensorMap, int);
+using PrepFn = void (*)(ChunkArgs, int, int, SlotMap, int*, const CUtensorMap, const CUtensorMap, int);
 template <bool VL>
 PrepFn prep_variant(bool cv, bool lg, bool qkg) {
   if (cv)
-    return lg ? (qkg ? chunk_prep_kernel<true, true, true, VL> : chunk_prep_kernel<true, true, false, VL>)
-              : (qkg ? chunk_prep_kernel<true, false, true, VL> : chunk_prep_kernel<true, false, false, VL>);
-  return lg ? (qkg ? chunk_prep_kernel<false, true, true, VL> : chunk_prep_kernel<false, true, false, VL>)
-            : (qkg ? chunk_prep_kernel<false, false, true, VL> : chunk_prep_kernel<false, false, false, VL>);
+    return lg ? (qkg ? chunk_prep_kernel<true, true, true, VL, false> : chunk_prep_kernel<true, true, false, VL, false>)
+              : (qkg ? chunk_prep_kernel<true, false, true, VL, false> : chunk_prep_kernel<true, false, false, VL, false>);
+  return lg ? (qkg ? chunk_prep_kernel<false, true, true, VL, false> : chunk_prep_kernel<false, true, false, VL, false>)
+            : (qkg ? chunk_prep_kernel<false, false, true, VL, false> : chunk_prep_kernel<false, false, false, VL, false>);
+}
+// the copies with the scalar-gate boxes (tied gate layouts; fixed-length sequences, no fused load)
+PrepFn prep_box_variant(bool lg, bool qkg) {
+  return lg ? (qkg ? chunk_prep_kernel<false, true, true, false, true> : chunk_prep_kernel<false, true, false, false, true>)
+            : (qkg ? chunk_prep_kernel<false, false, true, false, true> : chunk_prep_kernel<false, false, false, false, true>);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
@@ -1956,10 +2043,12 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     if (seg < 1) return cudaErrorInvalidValue;
   }
 
-  for (bool f16 : {false, true})   // (the fused-load copy and the plain one)
+  for (int f16 : {0, 1, 2})   // (the fused-load copy, the plain one, the one with the gate boxes)
     for (bool lg : {false, true})
       for (bool qg : {false, true}) {
-        const PrepFn prep = vl ? prep_variant<true>(f16, lg, qg) : prep_variant<false>(f16, lg, qg);
+        const PrepFn prep = f16 == 2 ? prep_box_variant(lg, qg)
+                          : vl       ? prep_variant<true>(f16 == 1, lg, qg)
+                                     : prep_variant<false>(f16 == 1, lg, qg);
         if ((e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM)) != cudaSuccess)
           return e;
         // all of the unified L1/shared storage as shared memory, so that two prep CTAs fit an SM
@@ -1987,9 +2076,21 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
   // occupancy calculator reports one for any kernel that allocates tensor
   // memory, so the count is set here.
   const int prep_ctas = sms * 2;
-  CUtensorMap amap{};
-  const int use_amap = a.gate_mode != GDN2_GATES_GDN && a.alpha != nullptr && encode_alpha_map(a, &amap) ? 1 : 0;
-  const PrepFn prep = vl ? prep_variant<true>(cv, a.gate_logits != 0, qkg) : prep_variant<false>(cv, a.gate_logits != 0, qkg);
+  CUtensorMap amap{}, bmap{};
+  int tgates = 0;   // gates by TMA
+  if (a.gate_mode != GDN2_GATES_GDN) {
+    if (a.alpha != nullptr && encode_alpha_map(a, &amap)) tgates |= TG_ATILE;
+  } else if (a.alpha != nullptr && encode_scalar_gate_map(a, a.alpha, &amap)) {
+    tgates |= TG_ABOX;
+  }
+  // (the fused load keeps its sums where the β box would go)
+  if (a.gate_mode != GDN2_GATES_FULL && !cv && a.b != nullptr && encode_scalar_gate_map(a, a.b, &bmap)) tgates |= TG_BBOX;
+  // the boxes of scalar gates: in their own copy of the prep, for fixed-length sequences without the fused load
+  const bool box = !vl && !cv && (tgates & (TG_ABOX | TG_BBOX)) != 0;
+  if (!box) tgates &= TG_ATILE;
+  const PrepFn prep = box ? prep_box_variant(a.gate_logits != 0, qkg)
+                    : vl  ? prep_variant<true>(cv, a.gate_logits != 0, qkg)
+                          : prep_variant<false>(cv, a.gate_logits != 0, qkg);
 
   // overlapped segments: whole sequence in the workspace, idle SMs beside the
   // scan, S_T given (the state passes from segment to segment through it)
@@ -2020,10 +2121,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, int o_bf16, cudaStream_t s) {
     if (items == 0) {
       // nothing to prepare (packed sequences, all empty)
     } else if (nseg_ov > 0 && k > 0) {
-      if ((e = launch_dependent(prep, grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap, use_amap)) != cudaSuccess)
+      if ((e = launch_dependent(prep, grid, NP, P_SMEM, s, a, c0, n, sm, counter, amap, bmap, tgates)) != cudaSuccess)
         return e;
     } else {
-      prep<<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter, amap, use_amap);
+      prep<<<grid, NP, P_SMEM, s>>>(a, c0, n, sm, counter, amap, bmap, tgates);
     }
     // the items whose decay the prep's factors cannot take, exactly
     if (items > 0) fix<<<(items + FX_ITEMS - 1) / FX_ITEMS, FX_THREADS, FX_SMEM, s>>>(a, c0, n, sm);

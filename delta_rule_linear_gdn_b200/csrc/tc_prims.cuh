@@ -248,6 +248,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* tmap, in
       : "memory");
 }
 
+// The same for one box of a 2-D tensor map.
+__device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* tmap, int x, int y, uint64_t* mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
+      ::"r"(smem_u32(dst_smem)), "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(mbar))
+      : "memory");
+}
+
 // Bulk (non-tensor) asynchronous copy shared → global of `bytes` (multiple of
 // 16, both addresses 16-byte aligned), tracked by the issuing thread's bulk
 // groups: commit, then wait until the source may be overwritten (.read) or

@@ -125,3 +125,27 @@ def test_noalloc_with_qk_gates():
     torch.cuda.synchronize()
     torch.testing.assert_close(o2, o, rtol=0, atol=0)
     torch.testing.assert_close(S2, S, rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("gate_mode", ["kda", "gdn"])
+@pytest.mark.parametrize("gate_logits", [False, True])
+@pytest.mark.parametrize("qk", [False, True])
+def test_tied_gates_by_tma_box(gate_mode, gate_logits, qk):
+    """The layer's head counts (16 QK / 48 V heads): a row of gates is a
+    multiple of 16 bytes, so the tensor-core prep takes the tied layouts'
+    scalar gates (β, and α in the Gated DeltaNet layout) by TMA boxes one item
+    ahead. Two sequences with a ragged tail, values and logits, gates per value
+    head and per QK head (bit for bit the same call with the rows repeated),
+    every head against the oracle."""
+    w = replace(workload("prefill_t4096"), T=200, B=2, s0="normal")
+    inp = make_inputs(w, seed=62, gate_mode=gate_mode, gate_logits=gate_logits, gates_per_qk_head=qk)
+    c = to_cuda(inp)
+    kw = dict(chunk=64, gate_mode=gate_mode, gate_logits=gate_logits, o_dtype=torch.float32)
+    o, S = run(c, gates_per_qk_head=qk, **kw)
+    if qk:
+        o_rep, S_rep = run(repeated(c, w.H_v), **kw)
+        torch.testing.assert_close(o, o_rep, rtol=0, atol=0)
+        torch.testing.assert_close(S, S_rep, rtol=0, atol=0)
+    o_ref, S_ref = oracle_chunk(inp, gate_mode=gate_mode, gate_logits=gate_logits, gates_per_qk_head=qk)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(S, S_ref, TOL_BF16, "S_T")
