@@ -212,7 +212,18 @@ struct PrepSrc {
 
 // Gate of one token for 4 channels, or the token's scalar gate broadcast: the
 // fp32 values, or σ of the bf16 logits (LG).
-template <bool LG>
+// σ(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh approximation: one
+// special-function operation where the exponential and the reciprocal take
+// two. For the erase and write strengths b, w only, which enter fp16 operand
+// tiles whose rounding is of the same order as this form's error; the decay
+// α, whose products compound over a chunk, keeps the exponential form.
+__device__ __forceinline__ float sigmoid_tanh_f32(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
+
+template <bool LG, bool FAST = false>
 __device__ __forceinline__ float4 gate4(const float* g, size_t gt, int c0, bool per_channel) {
   if (!LG) {
     if (per_channel) return __ldg(reinterpret_cast<const float4*>(g + gt * D + c0));
@@ -223,6 +234,8 @@ __device__ __forceinline__ float4 gate4(const float* g, size_t gt, int c0, bool 
   if (per_channel) {
     float x[4];
     unpack4_bf16(__ldg(reinterpret_cast<const uint2*>(h + gt * D + c0)), x);
+    if (FAST)
+      return make_float4(sigmoid_tanh_f32(x[0]), sigmoid_tanh_f32(x[1]), sigmoid_tanh_f32(x[2]), sigmoid_tanh_f32(x[3]));
     return make_float4(sigmoid_f32(x[0]), sigmoid_f32(x[1]), sigmoid_f32(x[2]), sigmoid_f32(x[3]));
   }
   const float s = sigmoid_f32(__uint_as_float((uint32_t)__ldg(h + gt) << 16));
@@ -407,7 +420,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
       const float bt = ok ? box_gate(it, P_BETA, i0 + u) : 0.f;
       bq[s] = make_float4(bt, bt, bt, bt);
     } else {
-      bq[s] = ok ? gate4<LG>(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+      bq[s] = ok ? gate4<LG, true>(src.b, gate_row(it, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if constexpr (!CV) {   // (CV: k and q come from pass 0)
       kk[s] = ok ? __ldg(reinterpret_cast<const uint2*>(src.k + tq * D + c0)) : make_uint2(0, 0);
@@ -747,7 +760,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
             wv[u] = make_float4(bt, bt, bt, bt);
           }
         } else {
-          wv[u] = ok ? gate4<LG>(src.w, w_row(it, hv, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+          wv[u] = ok ? gate4<LG, true>(src.w, w_row(it, hv, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         if constexpr (!CV)
           vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + hv) * D + c0))
@@ -790,7 +803,7 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           const float bt = ok ? box_gate(it, P_BETA, i0 + u) : 0.f;
           wv[u] = make_float4(bt, bt, bt, bt);
         } else {
-          wv[u] = ok ? gate4<LG>(src.w, w_row(it, it.h, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
+          wv[u] = ok ? gate4<LG, true>(src.w, w_row(it, it.h, u), c0, full) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         if constexpr (!CV)
           vv[u] = ok ? __ldg(reinterpret_cast<const uint2*>(src.v + (qkv_tok(it, u) * a.Hv + it.h) * D + c0))
@@ -884,6 +897,32 @@ __global__ void __launch_bounds__(NP, 2) chunk_prep_kernel(ChunkArgs a, int c_be
           unpack4_bf16(vv[u], vx);
         st8(smem, P_Z + (uint32_t)(i0 + u) * 128 + piece(u, BS_ROW64),
             pack4_f16(wv[u].x * vx[0], wv[u].y * vx[1], wv[u].z * vx[2], wv[u].w * vx[3]));
+      }
+    }
+
+    // Gates as logits: the next item's rows of k, q, v (and of the bf16
+    // logits of b and w when they are per channel) toward L2 while this
+    // item's inverse and products run, so that its own loads of them, early in
+    // its operand passes, wait on L2 rather than on DRAM. Every such row is
+    // 256 bytes, two lines: thread t with t % 4 < 2 covers line t % 4 of
+    // token row t / 4 (only rows the item reads). (With fp32 gates, QK-owned
+    // gates or the conv in the load the same hint made the prep slower.)
+    if constexpr (LG && !QKG && !CV) {
+      const int nx = counter ? *s_item : item + (int)gridDim.x;
+      const int tok = tid >> 2, sub = tid & 3;
+      if (nx < n_items && sub < 2) {
+        const Item nt = decode_item<VL, QKG>(a, c_begin, nx, sm);
+        if (nt.Lc == C || tok < nt.Lc) {
+          const size_t r = (size_t)nt.bi * a.T + nt.t0 + tok;
+          const size_t qk_off = (r * a.Hqk + nt.hq) * D + sub * 64, v_off = (r * a.Hv + nt.h) * D + sub * 64;
+          prefetch_l2(src.k + qk_off);
+          prefetch_l2(src.q + qk_off);
+          prefetch_l2(src.v + v_off);
+          if (full) {
+            prefetch_l2(reinterpret_cast<const uint16_t*>(src.b) + v_off);
+            prefetch_l2(reinterpret_cast<const uint16_t*>(src.w) + v_off);
+          }
+        }
       }
     }
 

@@ -256,6 +256,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* tmap, in
       : "memory");
 }
 
+// Hint that the 128-byte line holding `p` (a valid global address) be brought
+// into L2; no register receives data and nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p));
+}
+
 // Bulk (non-tensor) asynchronous copy shared → global of `bytes` (multiple of
 // 16, both addresses 16-byte aligned), tracked by the issuing thread's bulk
 // groups: commit, then wait until the source may be overwritten (.read) or
