@@ -52,12 +52,12 @@ L2_BYTES = 126 * 2**20
 # launches of one T=32768 call, and the hash of the kernel sources they were
 # taken on (with other sources the figure is stale and the bench reports
 # null). Taken on the T=4096 case (its 2 segments' prep and scan launches,
-# 802.1 MB per call, 1.83x its algorithmic bytes) and scaled by the chunk
+# 802.4 MB per call, 1.83x its algorithmic bytes) and scaled by the chunk
 # count (x8): the slot round trip, which is most of the excess, grows with the
 # chunks; the full-size workload is too large for a multi-metric capture.
 TRAFFIC_KERNEL_SOURCES = ("delta_rule_linear_gdn_b200/csrc/chunk_tc.cu", "delta_rule_linear_gdn_b200/csrc/tc_prims.cuh")
-TRAFFIC = {"sha1": "60c7bdd77f6184b4746f4a725218c901df23b4e7",
-           "bytes_per_call": 6416926720}
+TRAFFIC = {"sha1": "34f4ca12cb460ea74255900992863d368e16e93a",
+           "bytes_per_call": 6419318784}
 
 
 def peaks():
