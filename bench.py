@@ -344,7 +344,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=PREFILL, choices=[PREFILL, "prefill_t4096"],
                     help="prefill workload to time (the small one is for profiler captures)")
@@ -847,40 +847,66 @@ def run_head_split(args, w, dev, stream, barrier, world):
 
 def run_e2e(args, w, inp, o, S_T, ws, dev, stream, barrier, tokens_per_step):
     """The same prefill through the public call with host buffers: pinned
-    host->device copies of the inputs, the call, device->host copies of o and
-    S_T, all on the timed stream."""
+    host->device copies of each step's inputs, the call, device->host copies
+    of its o and S_T, all inside the timed region. Steps are pipelined over
+    two buffer sets, as a serving loop would run them: step i+1's inputs
+    cross PCIe (on a copy stream) while step i computes and its results come
+    back (on a third stream), so the link's two directions overlap."""
     import torch
     from delta_rule_linear_gdn_b200 import gdn2
     host = {k: inp[k].cpu().pin_memory() for k in ("q", "k", "v", "alpha", "b", "w")}
-    dev_in = {k: torch.empty_like(inp[k]) for k in host}
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    S_host = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    NB = 2
+    dev_in = [{k: torch.empty_like(inp[k]) for k in host} for _ in range(NB)]
+    o_dev = [o, torch.empty_like(o)]
+    S_dev = [S_T, torch.empty_like(S_T)]
+    o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(NB)]
+    S_host = [torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory() for _ in range(NB)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
+    d2h = o_host[0].numel() * o_host[0].element_size() + S_host[0].numel() * S_host[0].element_size()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(NB)]     # inputs of buffer set j landed
+    ev_done = [torch.cuda.Event() for _ in range(NB)]   # the call on set j is done (its inputs are free)
+    ev_out = [torch.cuda.Event() for _ in range(NB)]    # o, S_T of set j are on the host (free again)
 
-    def e2e_call():
-        for k_ in host:
-            dev_in[k_].copy_(host[k_], non_blocking=True)
-        gdn2.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["b"], dev_in["w"], None,
-                       chunk=w.chunk, o=o, S_T=S_T, workspace=ws, stream=stream)
-        o_host.copy_(o, non_blocking=True)
-        S_host.copy_(S_T, non_blocking=True)
+    def e2e_step(i):
+        j = i % NB
+        with torch.cuda.stream(up):
+            if i >= NB:
+                up.wait_event(ev_done[j])
+            for k_ in host:
+                dev_in[j][k_].copy_(host[k_], non_blocking=True)
+            ev_in[j].record(up)
+        stream.wait_event(ev_in[j])
+        if i >= NB:
+            stream.wait_event(ev_out[j])
+        gdn2.chunk_fwd(dev_in[j]["q"], dev_in[j]["k"], dev_in[j]["v"], dev_in[j]["alpha"], dev_in[j]["b"],
+                       dev_in[j]["w"], None, chunk=w.chunk, o=o_dev[j], S_T=S_dev[j], workspace=ws, stream=stream)
+        ev_done[j].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[j])
+            o_host[j].copy_(o_dev[j], non_blocking=True)
+            S_host[j].copy_(S_dev[j], non_blocking=True)
+            ev_out[j].record(down)
 
-    with torch.cuda.stream(stream):
-        e2e_call()
+    def run(n):
+        for i in range(n):
+            e2e_step(i)
+        for j in range(min(n, NB)):
+            stream.wait_event(ev_out[j])
+
+    run(NB)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.e2e_steps):
-            e2e_call()
+    up.wait_event(e0)
+    run(args.e2e_steps)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ems = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
     return {"value": tokens_per_step / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ems, "pipelined": "2 buffer sets, copies on 2 side streams"}
 
 
 if __name__ == "__main__":
