@@ -54,3 +54,18 @@ def test_tied_gate_bytes_and_backward_flops():
     # backward: 18 d^2 per token and value head (B=8, T=8192)
     bw = workload("conv_prefill_b8_t8192")
     assert bench.bwd_flops(bw) == 8 * 8192 * HV * 18 * D * D
+
+
+def test_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
+    """`roofline.traffic` comes from an ncu capture of particular kernel
+    sources: it is reported while the sources hash to the captured ones and
+    is null once they change (or when no capture is recorded)."""
+    sha = bench.kernel_sources_sha1()
+    assert len(sha) == 40 and sha == bench.kernel_sources_sha1()   # stable over reads
+    monkeypatch.setitem(bench.TRAFFIC, "sha1", sha)
+    monkeypatch.setitem(bench.TRAFFIC, "bytes_per_call", 123456)
+    assert bench.measured_traffic() == 123456
+    monkeypatch.setitem(bench.TRAFFIC, "sha1", "0" * 40)
+    assert bench.measured_traffic() is None
+    monkeypatch.setitem(bench.TRAFFIC, "sha1", None)
+    assert bench.measured_traffic() is None
